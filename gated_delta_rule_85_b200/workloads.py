@@ -1,0 +1,233 @@
+"""Seeded synthetic inputs for the KDA operator.
+
+This module holds no KDA arithmetic: it only draws the operator's inputs with
+the distributions and shapes of the workloads the tests and the benchmark use,
+so the CUDA path and the fp64 oracle can be fed the exact same tensors.
+
+Distributions (per the workload definitions):
+  q, k      ~ N(0, 1), then L2-normalised over dk per (token, head) in fp32,
+              then cast to the input dtype (bf16 or fp32)
+  v         ~ N(0, 1), cast to the input dtype
+  log_alpha = -softplus(x), x ~ N(-2, 1), fp32, one value per channel
+  beta      = sigmoid(x), x ~ N(0, 1), fp32, one value per (token, head)
+  states    ~ N(0, 0.01^2) fp32 (std 0.01), or zeros
+Every tensor is drawn from its own generator seeded with (seed, stream id), so
+one tensor's draw does not depend on another's size.  Large tensors are drawn
+in token slices of fixed size so device memory for temporaries stays bounded.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+_STREAM = {"q": 1, "k": 2, "v": 3, "log_alpha": 4, "beta": 5, "init_state": 6}
+_SLICE_TOKENS = 1 << 15
+
+
+@dataclass(frozen=True)
+class PrefillShape:
+    B: int
+    T: int
+    H: int
+    dk: int
+    dv: int
+    dtype: torch.dtype = torch.bfloat16
+    init_state: str = "normal"          # "normal" (std 0.01) or "zeros"
+    cu_seqlens: tuple | None = None      # packed layout when set (B must be 1)
+
+    @property
+    def num_seqs(self) -> int:
+        return self.B if self.cu_seqlens is None else len(self.cu_seqlens) - 1
+
+
+@dataclass(frozen=True)
+class DecodeShape:
+    N: int
+    H: int
+    dk: int
+    dv: int
+    steps: int
+    dtype: torch.dtype = torch.bfloat16
+
+
+def _gen(device, seed: int, stream: int, sub: int = 0) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed((int(seed) * 1_000_003 + stream * 7919 + sub) & 0x7FFF_FFFF_FFFF_FFFF)
+    return g
+
+
+def _normal(shape, device, seed, stream, mean=0.0, std=1.0):
+    """fp32 normal draw, generated in token slices along dim 0*dim1 rows."""
+    out = torch.empty(shape, dtype=torch.float32, device=device)
+    flat = out.view(-1, shape[-1]) if len(shape) > 1 else out.view(-1, 1)
+    rows = flat.shape[0]
+    per = max(1, _SLICE_TOKENS * 32)
+    for i, r0 in enumerate(range(0, rows, per)):
+        r1 = min(rows, r0 + per)
+        flat[r0:r1].normal_(mean, std, generator=_gen(device, seed, stream, i))
+    return out
+
+
+def _unit_rows(x: torch.Tensor) -> torch.Tensor:
+    """L2-normalise the last axis in fp32 (input preparation, not KDA math)."""
+    n = torch.linalg.vector_norm(x, dim=-1, keepdim=True).clamp_min(1e-6)
+    return x / n
+
+
+def draw_qk(shape, device, seed, stream, dtype):
+    """[..., dk] keys/queries: normal, unit rows in fp32, then cast, sliced to bound memory."""
+    out = torch.empty(shape, dtype=dtype, device=device)
+    flat_out = out.view(-1, shape[-1])
+    rows = flat_out.shape[0]
+    per = _SLICE_TOKENS * 32
+    for i, r0 in enumerate(range(0, rows, per)):
+        r1 = min(rows, r0 + per)
+        x = torch.empty((r1 - r0, shape[-1]), dtype=torch.float32, device=device)
+        x.normal_(0.0, 1.0, generator=_gen(device, seed, stream, i))
+        flat_out[r0:r1] = _unit_rows(x).to(dtype)
+    return out
+
+
+def draw_v(shape, device, seed, stream, dtype):
+    out = torch.empty(shape, dtype=dtype, device=device)
+    flat_out = out.view(-1, shape[-1])
+    rows = flat_out.shape[0]
+    per = _SLICE_TOKENS * 32
+    for i, r0 in enumerate(range(0, rows, per)):
+        r1 = min(rows, r0 + per)
+        x = torch.empty((r1 - r0, shape[-1]), dtype=torch.float32, device=device)
+        x.normal_(0.0, 1.0, generator=_gen(device, seed, stream, i))
+        flat_out[r0:r1] = x.to(dtype)
+    return out
+
+
+def draw_log_alpha(shape, device, seed, stream):
+    """-softplus(N(-2, 1)) per channel, fp32."""
+    out = torch.empty(shape, dtype=torch.float32, device=device)
+    flat = out.view(-1, shape[-1])
+    rows = flat.shape[0]
+    per = _SLICE_TOKENS * 32
+    for i, r0 in enumerate(range(0, rows, per)):
+        r1 = min(rows, r0 + per)
+        x = flat[r0:r1]
+        x.normal_(-2.0, 1.0, generator=_gen(device, seed, stream, i))
+        torch.nn.functional.softplus(x, out=x)
+        x.neg_()
+    return out
+
+
+def draw_beta(shape, device, seed, stream):
+    """sigmoid(N(0, 1)) per (token, head), fp32."""
+    x = torch.empty(shape, dtype=torch.float32, device=device)
+    x.normal_(0.0, 1.0, generator=_gen(device, seed, stream))
+    return torch.sigmoid(x)
+
+
+def draw_state(shape, device, seed, stream, kind="normal"):
+    if kind == "zeros":
+        return torch.zeros(shape, dtype=torch.float32, device=device)
+    x = torch.empty(shape, dtype=torch.float32, device=device)
+    x.normal_(0.0, 0.01, generator=_gen(device, seed, stream))
+    return x
+
+
+def prefill_inputs(shape: PrefillShape, seed: int = 0, device="cpu") -> dict:
+    """All prefill inputs of one workload, drawn in the order q, k, v, log_alpha, beta, init_state."""
+    B, T, H, dk, dv = shape.B, shape.T, shape.H, shape.dk, shape.dv
+    d = {
+        "q": draw_qk((B, T, H, dk), device, seed, _STREAM["q"], shape.dtype),
+        "k": draw_qk((B, T, H, dk), device, seed, _STREAM["k"], shape.dtype),
+        "v": draw_v((B, T, H, dv), device, seed, _STREAM["v"], shape.dtype),
+        "log_alpha": draw_log_alpha((B, T, H, dk), device, seed, _STREAM["log_alpha"]),
+        "beta": draw_beta((B, T, H), device, seed, _STREAM["beta"]),
+    }
+    N = shape.num_seqs
+    d["init_state"] = (None if shape.init_state == "none"
+                       else draw_state((N, H, dk, dv), device, seed, _STREAM["init_state"], shape.init_state))
+    d["cu_seqlens"] = (None if shape.cu_seqlens is None
+                       else torch.tensor(shape.cu_seqlens, dtype=torch.int32, device=device))
+    return d
+
+
+def decode_step_inputs(shape: DecodeShape, step: int, seed: int = 0, device="cpu") -> dict:
+    """Per-step decode inputs (q, k, v [N, H, d], log_alpha [N, H, dk], beta [N, H])."""
+    N, H, dk, dv = shape.N, shape.H, shape.dk, shape.dv
+    base = seed * 65_537 + 100 + step
+    return {
+        "q": draw_qk((N, H, dk), device, base, _STREAM["q"], shape.dtype),
+        "k": draw_qk((N, H, dk), device, base, _STREAM["k"], shape.dtype),
+        "v": draw_v((N, H, dv), device, base, _STREAM["v"], shape.dtype),
+        "log_alpha": draw_log_alpha((N, H, dk), device, base, _STREAM["log_alpha"]),
+        "beta": draw_beta((N, H), device, base, _STREAM["beta"]),
+    }
+
+
+def decode_all_steps(shape: DecodeShape, seed: int = 0, device="cpu") -> dict:
+    """Every step's inputs stacked on a leading [steps] axis, plus the initial states."""
+    N, H, dk, dv, S = shape.N, shape.H, shape.dk, shape.dv, shape.steps
+    out = {
+        "q": torch.empty((S, N, H, dk), dtype=shape.dtype, device=device),
+        "k": torch.empty((S, N, H, dk), dtype=shape.dtype, device=device),
+        "v": torch.empty((S, N, H, dv), dtype=shape.dtype, device=device),
+        "log_alpha": torch.empty((S, N, H, dk), dtype=torch.float32, device=device),
+        "beta": torch.empty((S, N, H), dtype=torch.float32, device=device),
+    }
+    for s in range(S):
+        one = decode_step_inputs(shape, s, seed, device)
+        for key in out:
+            out[key][s].copy_(one[key])
+    out["state"] = draw_state((N, H, dk, dv), device, seed, _STREAM["init_state"])
+    return out
+
+
+def varlen_lengths(total: int = 1 << 20, lo: int = 1024, hi: int = 262_144, seed: int = 0) -> list[int]:
+    """Log-uniform sequence lengths in [lo, hi] that fill `total` tokens.
+
+    Draw floor(exp(U(ln lo, ln hi))) in order with numpy PCG64(seed); stop when
+    the next draw would overflow `total`; extend the last kept sequence by the
+    remainder so the lengths sum to `total` exactly.
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lens: list[int] = []
+    used = 0
+    while True:
+        L = int(math.floor(math.exp(rng.uniform(math.log(lo), math.log(hi)))))
+        if used + L > total:
+            break
+        lens.append(L)
+        used += L
+    if not lens:
+        return [total]
+    lens[-1] += total - used
+    return lens
+
+
+def cu_from_lengths(lengths) -> tuple:
+    cu = [0]
+    for L in lengths:
+        cu.append(cu[-1] + int(L))
+    return tuple(cu)
+
+
+# The five workloads the operator is measured and checked on.
+CONFIGS = {
+    "tiny_f32": PrefillShape(B=1, T=256, H=2, dk=64, dv=64, dtype=torch.float32, init_state="zeros"),
+    "prefill_8k": PrefillShape(B=1, T=8192, H=32, dk=128, dv=128, dtype=torch.bfloat16),
+    "prefill_128k": PrefillShape(B=1, T=131072, H=32, dk=128, dv=128, dtype=torch.bfloat16),
+    "decode_b256": DecodeShape(N=256, H=32, dk=128, dv=128, steps=1024, dtype=torch.bfloat16),
+}
+
+
+def varlen_1m_shape() -> PrefillShape:
+    cu = cu_from_lengths(varlen_lengths())
+    return PrefillShape(B=1, T=cu[-1], H=32, dk=128, dv=128, dtype=torch.bfloat16, cu_seqlens=cu)
+
+
+def to_f64(x: torch.Tensor | None):
+    """Exact values of a tensor as a float64 numpy array (bf16 widens exactly)."""
+    if x is None:
+        return None
+    return x.detach().to("cpu", torch.float64).numpy()
