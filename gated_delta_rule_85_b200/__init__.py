@@ -1,0 +1,216 @@
+"""B200-native Kimi Delta Attention (KDA) operator: Python binding of libkda.
+
+Thin ctypes marshalling over the C ABI in include/kda.h: every step of the
+operator runs in the CUDA kernels of libkda.so; PyTorch only provides device
+memory and the current stream.  There is no CPU fallback: calling an operator
+without the built library, or without a CUDA device, raises.
+
+    o, S = chunk_forward(q, k, v, log_alpha, beta, init_state, cu_seqlens=None)
+    o    = recurrent_step(q, k, v, log_alpha, beta, state)      # state in place
+
+The recurrence ("Kimi Delta Attention 徹底解説" (tech-tide.dev), § "Kimi Delta
+Attention の仕組み"), per (sequence, head), with a dk x dv fp32 state S:
+    S' = Diag(exp(log_alpha_t)) S;  S = S' + beta_t k_t (v_t - S'^T k_t)^T;  o_t = S^T q_t
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "chunk_forward", "chunk_forward_simt", "recurrent_step", "workspace_size", "device_status",
+    "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
+    "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE",
+]
+
+KDA_BF16 = 0
+KDA_F32 = 1
+CHUNK = 64
+DEV_WAIT_TIMEOUT = 0x1
+DEV_DECAY_RANGE = 0x2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+
+class KDAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"kda error {code}: {msg}")
+        self.code = code
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libkda.so")
+
+
+def load_library():
+    """Load libkda.so (built by gated_delta_rule_85_b200/build.py); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"libkda.so is not built ({path}); run gated_delta_rule_85_b200/build.py")
+    lib = ctypes.CDLL(path)
+    vp, fp, ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    ci, sz = ctypes.c_int, ctypes.c_size_t
+    lib.kda_chunk_forward.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, ip] + [ci] * 8 + [vp, sz, vp]
+    lib.kda_chunk_forward.restype = ci
+    lib.kda_chunk_forward_simt.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, ip] + [ci] * 8 + [vp]
+    lib.kda_chunk_forward_simt.restype = ci
+    lib.kda_chunk_forward_workspace_size.argtypes = [ci] * 8
+    lib.kda_chunk_forward_workspace_size.restype = sz
+    lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ci] * 5 + [vp]
+    lib.kda_recurrent_step.restype = ci
+    lib.kda_last_error.argtypes = []
+    lib.kda_last_error.restype = ctypes.c_char_p
+    lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci, vp]
+    lib.kda_get_device_status.restype = ci
+    lib.kda_api_version.argtypes = []
+    lib.kda_api_version.restype = ci
+    _lib = lib
+    return lib
+
+
+def last_error() -> str:
+    return load_library().kda_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise KDAError(rc, last_error())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; q/k/v must be bfloat16 or float32")
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be on the same CUDA device")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous in the documented layouts")
+
+
+def workspace_size(B, T, H, dk, dv, num_seqs, dtype=KDA_BF16) -> int:
+    return int(load_library().kda_chunk_forward_workspace_size(B, T, H, dk, dv, num_seqs, dtype, CHUNK))
+
+
+def _prefill_args(q, k, v, log_alpha, beta, init_state, cu_seqlens):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape[:3] != q.shape[:3] or beta.shape != q.shape[:3]:
+        raise ValueError("shape mismatch among q, k, v, log_alpha, beta")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k and v must share a dtype")
+    if log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise ValueError("log_alpha and beta must be float32")
+    N = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    if init_state is not None and (init_state.shape != (N, H, dk, dv) or init_state.dtype != torch.float32):
+        raise ValueError("init_state must be float32 [N, H, dk, dv]")
+    return B, T, H, dk, dv, N
+
+
+def _to_device(ts, device):
+    return [None if t is None else t.to(device, non_blocking=True) for t in ts]
+
+
+def chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, o=None,
+                  final_state=True, workspace=None, simt=False):
+    """Chunked KDA prefill (64-token chunks) through kda_chunk_forward.
+
+    Tensors are in the include/kda.h layouts.  `final_state` may be True
+    (allocate and return), False (skip) or a preallocated float32 tensor.
+    With `simt=True` the fp32 CUDA-core path (kda_chunk_forward_simt) runs
+    instead of the tensor-core path.  Host (CPU) inputs are copied to the
+    current CUDA device and the results copied back, all inside this call.
+    Returns (o, final_state or None).
+    """
+    if not q.is_cuda:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        args = _to_device([q, k, v, log_alpha, beta, init_state, cu_seqlens], dev)
+        fs_dev = final_state if isinstance(final_state, bool) else True
+        o_d, s_d = chunk_forward(*args, final_state=fs_dev, workspace=workspace, simt=simt)
+        o_h = o if o is not None else torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True)
+        o_h.copy_(o_d, non_blocking=True)
+        s_h = None
+        if s_d is not None:
+            s_h = final_state if isinstance(final_state, torch.Tensor) else \
+                torch.empty(s_d.shape, dtype=s_d.dtype, pin_memory=True)
+            s_h.copy_(s_d, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+        return o_h, s_h
+    B, T, H, dk, dv, N = _prefill_args(q, k, v, log_alpha, beta, init_state, cu_seqlens)
+    _need_cuda(q, k, v, log_alpha, beta, init_state, cu_seqlens)
+    lib = load_library()
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is True:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    elif final_state is False:
+        final_state = None
+    _need_cuda(o, final_state)
+    dt = _dtype_code(q)
+    st = _stream(q.device)
+    if simt:
+        rc = lib.kda_chunk_forward_simt(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(o),
+                                        _p(final_state), _p(cu_seqlens), B, T, H, dk, dv, N, dt, CHUNK, st)
+    else:
+        need = int(lib.kda_chunk_forward_workspace_size(B, T, H, dk, dv, N, dt, CHUNK))
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        rc = lib.kda_chunk_forward(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(o),
+                                   _p(final_state), _p(cu_seqlens), B, T, H, dk, dv, N, dt, CHUNK,
+                                   _p(workspace), ws_bytes, st)
+    _check(rc)
+    return o, final_state
+
+
+def chunk_forward_simt(*args, **kw):
+    """kda_chunk_forward_simt: the fp32 CUDA-core prefill path."""
+    return chunk_forward(*args, simt=True, **kw)
+
+
+def recurrent_step(q, k, v, log_alpha, beta, state, o=None):
+    """One KDA decode step (kda_recurrent_step); `state` [N, H, dk, dv] fp32 is updated in place."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape[:2] != q.shape[:2] or beta.shape != q.shape[:2]:
+        raise ValueError("shape mismatch among q, k, v, log_alpha, beta")
+    if state.shape != (N, H, dk, dv) or state.dtype != torch.float32:
+        raise ValueError("state must be float32 [N, H, dk, dv]")
+    _need_cuda(q, k, v, log_alpha, beta, state)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    rc = load_library().kda_recurrent_step(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(state), _p(o),
+                                           N, H, dk, dv, _dtype_code(q), _stream(q.device))
+    _check(rc)
+    return o
+
+
+def device_status(clear: bool = True) -> int:
+    """Device status word (KDA_DEV_* bits) of the current device; synchronises."""
+    bits = ctypes.c_uint(0)
+    rc = load_library().kda_get_device_status(ctypes.byref(bits), int(clear),
+                                              _stream(torch.cuda.current_device()))
+    if rc not in (0, -6):
+        _check(rc)
+    return int(bits.value)

@@ -1,0 +1,82 @@
+// Shared device helpers for the KDA kernels (one translation unit: kda_lib.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Per-device status word; kernels OR KDA_DEV_* flags into it.
+__device__ unsigned int g_status;
+
+__device__ __forceinline__ void flag_status(unsigned int bits) { atomicOr(&g_status, bits); }
+
+// ----------------------------------------------------------------- input access
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+    static __device__ __forceinline__ float load(const float *p) { return *p; }
+    static __device__ __forceinline__ void store(float *p, float x) { *p = x; }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+};
+
+// Load 4 consecutive elements (16-byte aligned for float, 8-byte for bf16) as floats.
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+__device__ __forceinline__ void store4(float *p, float4 x) { *reinterpret_cast<float4 *>(p) = x; }
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 x) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(x.z, x.w);
+    uint2 raw;
+    raw.x = *reinterpret_cast<uint32_t *>(&a);
+    raw.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = raw;
+}
+
+// Streaming (evict-first) 128-bit global access for data touched exactly once.
+__device__ __forceinline__ float4 ld_stream(const float *p) {
+    float4 r;
+    asm volatile("ld.global.cs.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "l"(p));
+    return r;
+}
+__device__ __forceinline__ void st_stream(float *p, float4 v) {
+    asm volatile("st.global.cs.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+
+// Token range of sequence n in the flattened [B*T] token axis.  Packed offsets
+// are clamped to [0, T] (B == 1 there) so a malformed cu_seqlens can never
+// address memory outside the caller's tensors.
+__device__ __forceinline__ void seq_span(const int32_t *cu_seqlens, int T, int n, long long &t0,
+                                         long long &t1) {
+    if (cu_seqlens) {
+        t0 = min(max(cu_seqlens[n], 0), T);
+        t1 = min(max(cu_seqlens[n + 1], (int)t0), T);
+    } else {
+        t0 = (long long)n * T;
+        t1 = t0 + T;
+    }
+}
+
+}  // namespace kda

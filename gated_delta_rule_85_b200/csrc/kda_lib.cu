@@ -1,0 +1,195 @@
+// libkda: the C ABI declared in include/kda.h.  One translation unit holds every
+// kernel so the device status word is a single symbol per device.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "kda_common.cuh"
+#include "kda_decode.cuh"
+#include "kda_chunk_simt.cuh"
+#include "kda_chunk_tc.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(KDA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+// Validation shared by both prefill entry points.
+int check_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *init_state, const void *o, const float *final_state,
+                  const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                  int dtype, int chunk) {
+    if (!q || !k || !v || !log_alpha || !beta || !o)
+        return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta and o are required");
+    if (B < 1 || T < 0 || H < 1 || num_seqs < 0)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d num_seqs=%d", B, T, H, num_seqs);
+    if (H > 65535) return fail(KDA_ERR_UNSUPPORTED, "H=%d above 65535", H);
+    if (cu_seqlens) {
+        if (B != 1) return fail(KDA_ERR_INVALID_ARG, "packed (cu_seqlens) input needs B == 1, got %d", B);
+        if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "packed input needs num_seqs >= 1");
+    } else if (num_seqs != B) {
+        return fail(KDA_ERR_INVALID_ARG, "num_seqs (%d) must equal B (%d) without cu_seqlens", num_seqs, B);
+    }
+    if (num_seqs > 65535) return fail(KDA_ERR_UNSUPPORTED, "num_seqs=%d above 65535", num_seqs);
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+        return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: each must be 64 or 128", dk, dv);
+    if (chunk != 64) return fail(KDA_ERR_UNSUPPORTED, "chunk=%d: only 64 is supported", chunk);
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "dtype=%d", dtype);
+    const void *p16[] = {q, k, v, log_alpha, o, init_state, final_state};
+    const char *n16[] = {"q", "k", "v", "log_alpha", "o", "init_state", "final_state"};
+    for (int i = 0; i < 7; ++i)
+        if (p16[i] && !aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
+    if (!aligned(beta, 4)) return fail(KDA_ERR_MISALIGNED, "beta is not 4-byte aligned");
+    if (cu_seqlens && !aligned(cu_seqlens, 4)) return fail(KDA_ERR_MISALIGNED, "cu_seqlens is not 4-byte aligned");
+    return KDA_OK;
+}
+
+template <int DK, typename Tin>
+int launch_simt(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int T,
+                int H, int dv, int num_seqs, cudaStream_t st) {
+    constexpr size_t smem = kda::simt::Smem<DK>::bytes;
+    auto kern = kda::chunk_simt_kernel<DK, Tin>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chunk_simt)");
+    dim3 grid(dv / kda::simt::DVT, H, num_seqs);
+    kern<<<grid, kda::simt::NT, smem, st>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta,
+                                             init_state, (Tin *)o, final_state, cu_seqlens, T, H, dv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_simt launch");
+    return KDA_OK;
+}
+
+template <int DK, int DV, typename Tin>
+int launch_decode(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                  float *state, void *o, long long pairs, cudaStream_t st) {
+    kda::decode_step_kernel<DK, DV, Tin><<<(unsigned)pairs, 256, 0, st>>>(
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta, state, (Tin *)o);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_api_version(void) { return KDA_API_VERSION; }
+
+const char *kda_last_error(void) { return g_err; }
+
+size_t kda_chunk_forward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype,
+                                        int chunk) {
+    (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)chunk;
+    if (dtype != KDA_BF16) return 0;
+    return kda::tc::workspace_bytes(num_seqs);
+}
+
+int kda_chunk_forward_simt(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *init_state, void *o, float *final_state,
+                           const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                           int dtype, int chunk, void *stream) {
+    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
+                           dv, num_seqs, dtype, chunk);
+    if (rc) return rc;
+    if (num_seqs == 0) return KDA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == KDA_BF16) {
+        if (dk == 64)
+            return launch_simt<64, __nv_bfloat16>(q, k, v, log_alpha, beta, init_state, o, final_state,
+                                                  cu_seqlens, T, H, dv, num_seqs, st);
+        return launch_simt<128, __nv_bfloat16>(q, k, v, log_alpha, beta, init_state, o, final_state,
+                                               cu_seqlens, T, H, dv, num_seqs, st);
+    }
+    if (dk == 64)
+        return launch_simt<64, float>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T,
+                                      H, dv, num_seqs, st);
+    return launch_simt<128, float>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H,
+                                   dv, num_seqs, st);
+}
+
+int kda_chunk_forward(const void *q, const void *k, const void *v, const float *log_alpha,
+                      const float *beta, const float *init_state, void *o, float *final_state,
+                      const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                      int dtype, int chunk, void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
+                           dv, num_seqs, dtype, chunk);
+    if (rc) return rc;
+    if (dtype == KDA_F32)
+        return kda_chunk_forward_simt(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B,
+                                      T, H, dk, dv, num_seqs, dtype, chunk, stream);
+    const size_t need = kda::tc::workspace_bytes(num_seqs);
+    if (need && (!workspace || ws_bytes < need))
+        return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", need, ws_bytes);
+    if (workspace && !aligned(workspace, 256)) return fail(KDA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (num_seqs == 0) return KDA_OK;
+    char msg[256] = "";
+    rc = kda::tc::launch(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk, dv,
+                         num_seqs, workspace, (cudaStream_t)stream, msg, sizeof(msg));
+    if (rc) return fail(rc, "%s", msg);
+    return KDA_OK;
+}
+
+int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, float *state, void *o, int N, int H, int dk, int dv, int dtype,
+                       void *stream) {
+    if (!q || !k || !v || !log_alpha || !beta || !state || !o)
+        return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta, state and o are required");
+    if (N < 0 || H < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d", N, H);
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+        return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: each must be 64 or 128", dk, dv);
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "dtype=%d", dtype);
+    const void *p16[] = {q, k, v, log_alpha, o, state};
+    const char *n16[] = {"q", "k", "v", "log_alpha", "o", "state"};
+    for (int i = 0; i < 6; ++i)
+        if (!aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
+    if (!aligned(beta, 4)) return fail(KDA_ERR_MISALIGNED, "beta is not 4-byte aligned");
+    const long long pairs = (long long)N * H;
+    if (pairs == 0) return KDA_OK;
+    if (pairs > 0x7fffffffLL) return fail(KDA_ERR_UNSUPPORTED, "N*H=%lld too large", pairs);
+    cudaStream_t st = (cudaStream_t)stream;
+#define KDA_DEC(DKv, DVv)                                                                              \
+    if (dk == DKv && dv == DVv)                                                                        \
+        return dtype == KDA_BF16                                                                       \
+                   ? launch_decode<DKv, DVv, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o, pairs, st) \
+                   : launch_decode<DKv, DVv, float>(q, k, v, log_alpha, beta, state, o, pairs, st);
+    KDA_DEC(64, 64)
+    KDA_DEC(64, 128)
+    KDA_DEC(128, 64)
+    KDA_DEC(128, 128)
+#undef KDA_DEC
+    return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d", dk, dv);
+}
+
+int kda_get_device_status(unsigned int *bits, int clear, void *stream) {
+    if (!bits) return fail(KDA_ERR_INVALID_ARG, "bits is required");
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned int host = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&host, kda::g_status, sizeof(host), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (clear && host) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbolAsync(kda::g_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    }
+    *bits = host;
+    if (host) return fail(KDA_ERR_DEVICE, "device status flags 0x%x", host);
+    return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,161 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) operator.
+ *
+ * What the operator computes ("Kimi Delta Attention 徹底解説" (tech-tide.dev),
+ * § "なぜ今「線形アテンション」なのか" and § "Kimi Delta Attention の仕組み";
+ * "Kimi Linear、独自の土俵でFull Attentionを上回る" (remio.ai),
+ * § "Kimi Linearがより賢いRecurrent Memoryを使う方法"): each (sequence, head)
+ * keeps a fixed-size state S (dk x dv, fp32).  For every token t, in order,
+ *
+ *     S'  = Diag(alpha_t) S          alpha_t = exp(log_alpha_t), one rate per key channel
+ *     S   = S' + beta_t k_t (v_t - S'^T k_t)^T
+ *     o_t = S^T q_t
+ *
+ * Decode runs this token by token; prefill regroups the same computation into
+ * 64-token chunks (same result up to rounding).  No normalisation of q or k and
+ * no 1/sqrt(d) scale is applied inside the operator.
+ *
+ * Layouts (row-major, last index contiguous; every tensor dense, no strides):
+ *   q, k        [B, T, H, dk]   dtype (bf16 or fp32)
+ *   v, o        [B, T, H, dv]   dtype
+ *   log_alpha   [B, T, H, dk]   fp32, must be <= 0 and finite
+ *   beta        [B, T, H]       fp32
+ *   states      [N, H, dk, dv]  fp32 (dv contiguous); the same layout for
+ *                               prefill's init/final state and decode's state,
+ *                               so a prefill's final_state is directly a valid
+ *                               decode state (a state-layout mismatch between
+ *                               chunked prefill and decode is the failure the
+ *                               remio.ai page reports in § "オープンコードにより
+ *                               主張は検証可能になる一方、ソフトウェアスタックは
+ *                               リスクを加える").
+ *   packed (varlen) prefill: B == 1, T = total tokens, cu_seqlens [N+1] int32 on
+ *   the device, non-decreasing, cu_seqlens[0] == 0, cu_seqlens[N] == T;
+ *   sequence n is tokens [cu_seqlens[n], cu_seqlens[n+1]) and the state never
+ *   crosses a sequence boundary.  Without cu_seqlens, N == B and each batch row
+ *   is one sequence of T tokens.
+ *
+ * Ownership and execution: the caller allocates and owns every buffer (device
+ * memory unless stated).  The library never allocates, frees or synchronises
+ * in these calls; work is enqueued on `stream` (a cudaStream_t passed as
+ * void*, NULL = the legacy default stream) and the call returns immediately.
+ * Pointers to tensors must be 16-byte aligned (beta and cu_seqlens: 4-byte).
+ * Inputs must not alias outputs, except decode's in-place state.
+ *
+ * Errors: every call returns KDA_OK (0) or a negative kda_status.  Argument
+ * errors are detected on the host before anything is enqueued (nothing runs).
+ * A failed launch returns KDA_ERR_CUDA.  Conditions found on the device are
+ * accumulated in a per-device status word read by kda_get_device_status().
+ * kda_last_error() gives a message for the calling thread's last failure.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_API_VERSION 1
+
+typedef enum kda_status {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = -1,   /* NULL required pointer, bad shape or count */
+    KDA_ERR_UNSUPPORTED = -2,   /* dk/dv not in {64, 128}, chunk != 64, bad dtype */
+    KDA_ERR_MISALIGNED = -3,    /* pointer alignment below the requirement */
+    KDA_ERR_CUDA = -4,          /* a CUDA runtime call or kernel launch failed */
+    KDA_ERR_WORKSPACE = -5,     /* workspace missing or smaller than required */
+    KDA_ERR_DEVICE = -6         /* kda_get_device_status() found a device-side flag */
+} kda_status;
+
+typedef enum kda_dtype {
+    KDA_BF16 = 0,
+    KDA_F32 = 1
+} kda_dtype;
+
+/* Device status word bits (kda_get_device_status). */
+#define KDA_DEV_WAIT_TIMEOUT 0x1u    /* a bounded on-chip wait gave up; that CTA's output is invalid */
+#define KDA_DEV_DECAY_RANGE 0x2u     /* tensor-core prefill: within one 64-token chunk a channel's
+                                        accumulated log-decay fell below -80; the factorised decay
+                                        operands lose range there (see kda_chunk_forward) */
+
+/*
+ * Chunked prefill, 64-token chunks.
+ *
+ * Source: the KDA recurrence above; the chunked regrouping is the prefill mode of
+ * "Kimi Delta Attention 徹底解説" § "Kimi Delta Attention の仕組み" and the
+ * chunkwise, diagonal-plus-low-rank form of "Kimi Linear、独自の土俵でFull Attention
+ * を上回る" § "Kimi Linearがより賢いRecurrent Memoryを使う方法".
+ *
+ *   q, k, v       inputs in `dtype`, layouts above (required)
+ *   log_alpha     fp32 [B,T,H,dk] (required); beta fp32 [B,T,H] (required)
+ *   init_state    fp32 [N,H,dk,dv] or NULL (zeros)
+ *   o             output [B,T,H,dv] in `dtype` (required); rounded to nearest-even
+ *   final_state   fp32 [N,H,dk,dv] or NULL (not written)
+ *   cu_seqlens    int32 [N+1] device array or NULL (dense batch)
+ *   B, T, H       batch, tokens per row, heads (T may be 0)
+ *   dk, dv        64 or 128 each
+ *   num_seqs      N; must equal B when cu_seqlens is NULL
+ *   dtype         KDA_BF16: tensor-core (tcgen05) path, bf16 operands with fp32
+ *                 accumulation; KDA_F32: fp32 CUDA-core path
+ *   chunk         must be 64
+ *   workspace     device scratch of at least kda_chunk_forward_workspace_size()
+ *                 bytes, 256-byte aligned (may be NULL when that size is 0)
+ *
+ * Precondition of the tensor-core path: for every chunk and channel the summed
+ * log-decay over the chunk is >= -80 (alpha products stay above e^-80); below it
+ * the chunk-start factorisation of the decay is out of fp32/bf16 range and the
+ * call flags KDA_DEV_DECAY_RANGE.  The fp32 path has no such limit.
+ */
+size_t kda_chunk_forward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                        int dtype, int chunk);
+
+int kda_chunk_forward(const void *q, const void *k, const void *v, const float *log_alpha,
+                      const float *beta, const float *init_state, void *o, float *final_state,
+                      const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                      int dtype, int chunk, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Same contract as kda_chunk_forward, computed entirely on CUDA cores in fp32
+ * (inputs in either dtype are widened exactly).  The accuracy reference for the
+ * tensor-core path and the path taken for KDA_F32.  Needs no workspace.
+ */
+int kda_chunk_forward_simt(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *init_state, void *o, float *final_state,
+                           const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv,
+                           int num_seqs, int dtype, int chunk, void *stream);
+
+/*
+ * One decode step for N sequences: the token recurrence with T = 1, state
+ * updated in place.  Source: the recurrence above ("Kimi Delta Attention 徹底解説"
+ * § "Kimi Delta Attention の仕組み": decode is the token-by-token recurrence).
+ *
+ *   q, k     [N, H, dk] in dtype;  v, o [N, H, dv] in dtype
+ *   log_alpha fp32 [N, H, dk];     beta fp32 [N, H]
+ *   state    fp32 [N, H, dk, dv], read once and written once (in place)
+ * Each state is streamed once from HBM and written back once.
+ */
+int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, float *state, void *o, int N, int H, int dk, int dv,
+                       int dtype, void *stream);
+
+/* Message for the calling thread's last non-OK return ("" if none). */
+const char *kda_last_error(void);
+
+/*
+ * Reads (and, if `clear` is non-zero, resets) the current device's status word
+ * after synchronising `stream`.  *bits receives KDA_DEV_* flags.  Returns KDA_OK
+ * when no flag is set, KDA_ERR_DEVICE when some flag is set, KDA_ERR_CUDA when
+ * the read failed.  This call synchronises; use it off the hot path.
+ */
+int kda_get_device_status(unsigned int *bits, int clear, void *stream);
+
+/* KDA_API_VERSION of the loaded library. */
+int kda_api_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

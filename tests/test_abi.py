@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+function include/kda.h declares, and rejects bad arguments before enqueuing work.
+Every call below breaks exactly one rule that is checked before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_85_b200 as kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, CUDA, WORKSPACE = 0, -1, -2, -3, -4, -5
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_85_b200.build import build
+    build()
+    return kda.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "kda_chunk_forward" in names and "kda_recurrent_step" in names
+    for name in names:
+        assert hasattr(lib, name), f"libkda.so does not export {name}"
+    assert lib.kda_api_version() == 1
+
+
+# fake but 256-byte aligned "device" addresses: never dereferenced, every call fails validation
+A = [0x10000 * (i + 1) for i in range(12)]
+
+
+def prefill(lib, **over):
+    a = dict(q=A[0], k=A[1], v=A[2], g=A[3], b=A[4], s0=A[5], o=A[6], fs=A[7], cu=None,
+             B=1, T=128, H=2, dk=128, dv=128, N=1, dtype=0, chunk=64, ws=A[8], wsb=1 << 20, st=None)
+    a.update(over)
+    return lib.kda_chunk_forward(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["o"], a["fs"], a["cu"],
+                                 a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dtype"], a["chunk"],
+                                 a["ws"], a["wsb"], a["st"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), INVALID),
+    (dict(o=None), INVALID),
+    (dict(beta_missing=True), INVALID),
+    (dict(T=-1), INVALID),
+    (dict(H=0), INVALID),
+    (dict(N=2), INVALID),                       # N != B without cu_seqlens
+    (dict(cu=A[9], B=2, N=2), INVALID),         # packed input needs B == 1
+    (dict(dk=96), UNSUPPORTED),
+    (dict(dv=256), UNSUPPORTED),
+    (dict(chunk=32), UNSUPPORTED),
+    (dict(dtype=7), UNSUPPORTED),
+    (dict(q=A[0] + 8), MISALIGNED),
+    (dict(fs=A[7] + 4), MISALIGNED),
+    (dict(b=A[4] + 2), MISALIGNED),
+])
+def test_prefill_rejects(lib, over, code):
+    if over.pop("beta_missing", False):
+        over["b"] = None
+    assert prefill(lib, **over) == code
+    assert lib.kda_last_error().decode() != ""
+
+
+def test_simt_rejects(lib):
+    rc = lib.kda_chunk_forward_simt(A[0], A[1], A[2], A[3], A[4], None, A[6], None, None,
+                                    1, 64, 1, 64, 48, 1, 1, 64, None)
+    assert rc == UNSUPPORTED
+
+
+def step(lib, **over):
+    a = dict(q=A[0], k=A[1], v=A[2], g=A[3], b=A[4], s=A[5], o=A[6], N=4, H=2, dk=128, dv=128, dtype=0, st=None)
+    a.update(over)
+    return lib.kda_recurrent_step(a["q"], a["k"], a["v"], a["g"], a["b"], a["s"], a["o"], a["N"], a["H"],
+                                  a["dk"], a["dv"], a["dtype"], a["st"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(s=None), INVALID),
+    (dict(N=-1), INVALID),
+    (dict(dk=32), UNSUPPORTED),
+    (dict(dtype=3), UNSUPPORTED),
+    (dict(s=A[5] + 4), MISALIGNED),
+    (dict(v=A[2] + 2), MISALIGNED),
+])
+def test_step_rejects(lib, over, code):
+    assert step(lib, **over) == code
+
+
+def test_empty_work_is_a_no_op(lib):
+    assert step(lib, N=0) == OK
+
+
+def test_status_requires_pointer(lib):
+    assert lib.kda_get_device_status(None, 0, None) == INVALID
