@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""KDA operator benchmark: chunked-prefill and decode tokens/s on B200.
+
+One step = one chunked prefill (kda_chunk_forward, tcgen05 kernel) of the
+"prefill_8k" workload: B=1, T=8192, H=32, dk=dv=128, bf16 q/k/v, fp32 gates,
+fp32 initial state, 64-token chunks.  The decode workload (N=256 sequences,
+H=32, one token per step through kda_recurrent_step, fresh inputs per step) is
+timed in the same run and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line.  For N > 1 it runs under torch.distributed (one process
+per GPU); every rank processes its own full workload (weak scaling, no
+collective on the data path) and the step time is the max over ranks.
+--impl reference times the fp64 CPU oracle (the reference arm) on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = dict(B=1, T=8192, H=32, dk=128, dv=128)
+DECODE = dict(N=256, H=32, dk=128, dv=128, steps=1024)
+CHUNK = 64
+# Algorithmic bytes per token-head: q, k, v (bf16) + log_alpha (fp32) + beta + o (bf16).
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 4 * 128 + 4 + 2 * 128          # 1540
+STATE_BYTES = 4 * 128 * 128                                                   # one fp32 state
+# Algorithmic flops per token-head of the chunked form (C x C products at full size
+# plus the three C x d^2 state products): 10 C d + 6 d^2.
+PREFILL_FLOPS_PER_TOKEN_HEAD = 10 * CHUNK * 128 + 6 * 128 * 128               # 180224
+DECODE_BYTES_PER_PAIR = 2 * STATE_BYTES + PREFILL_BYTES_PER_TOKEN_HEAD        # 132612
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._h = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def run_prefill(args, world, rank, dev):
+    import torch
+
+    import gated_delta_rule_85_b200 as kda
+    from gated_delta_rule_85_b200.workloads import PrefillShape, prefill_inputs
+
+    shape = PrefillShape(**PREFILL, dtype=torch.bfloat16)
+    d = prefill_inputs(shape, seed=rank, device=dev)
+    o = torch.empty((1, PREFILL["T"], PREFILL["H"], PREFILL["dv"]), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, PREFILL["H"], 128, 128), dtype=torch.float32, device=dev)
+    ws_n = kda.workspace_size(1, PREFILL["T"], PREFILL["H"], 128, 128, 1)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev) if ws_n else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], None,
+                          o=o, final_state=fs, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if kda.device_status() != 0:
+        raise RuntimeError("device status flags set after warm-up")
+    if not (torch.isfinite(o.float()).all() and torch.isfinite(fs).all()):
+        raise RuntimeError("non-finite prefill output")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        t_all0 = torch.cuda.Event(enable_timing=True)
+        t_all1 = torch.cuda.Event(enable_timing=True)
+        t_all0.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_all1.record(stream)
+        torch.cuda.synchronize(dev)
+    _barrier(world)
+    total_ms = t_all0.elapsed_time(t_all1)
+    per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = _max_over_ranks(total_ms, world, dev)
+
+    # End to end through the public API with host buffers: H2D of every input,
+    # the kernel, D2H of o and the final state, every step.
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in d.items()}
+    h2d = sum(v.numel() * v.element_size() for k, v in host.items() if v is not None)
+    d2h = o.numel() * o.element_size() + fs.numel() * fs.element_size()
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+    e2e_steps = max(2, min(args.steps, 10))
+    kda.chunk_forward(host["q"], host["k"], host["v"], host["log_alpha"], host["beta"], host["init_state"],
+                      None, o=o_h, final_state=fs_h)
+    _barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        kda.chunk_forward(host["q"], host["k"], host["v"], host["log_alpha"], host["beta"], host["init_state"],
+                          None, o=o_h, final_state=fs_h)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    del d
+    return dict(total_ms=total_ms, per_launch_ms=per_launch_ms, clocks=clk.summary(), e2e_ms=e2e_ms,
+                h2d=h2d, d2h=d2h, e2e_steps=e2e_steps)
+
+
+def run_decode(args, world, rank, dev):
+    """1024 consecutive decode steps of 256 sequences, captured in one CUDA graph."""
+    import torch
+
+    import gated_delta_rule_85_b200 as kda
+    from gated_delta_rule_85_b200.workloads import DecodeShape, decode_all_steps
+
+    shape = DecodeShape(**DECODE, dtype=torch.bfloat16)
+    d = decode_all_steps(shape, seed=rank, device=dev)
+    state = d["state"]
+    o = torch.empty((DECODE["N"], DECODE["H"], 128), dtype=torch.bfloat16, device=dev)
+    S = DECODE["steps"]
+
+    def run_all():
+        for s in range(S):
+            kda.recurrent_step(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["beta"][s], state, o=o)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        run_all()                       # warm-up (also loads the module)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_all()
+    torch.cuda.synchronize(dev)
+    for _ in range(max(1, args.warmup // 4)):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    reps = max(2, min(args.steps // 10, 10))
+    stream = torch.cuda.current_stream(dev)
+    _barrier(world)
+    with ClockSampler(dev.index) as clk:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if not torch.isfinite(state).all():
+        raise RuntimeError("non-finite decode state")
+    del g, d, state
+    return dict(ms=ms, launches=reps * S, clocks=clk.summary())
+
+
+def cpu_baseline(heads=32, threads=0):
+    """fp64 oracle on the prefill_8k workload (a bounded sample of heads), host cores."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from gated_delta_rule_85_b200.workloads import PrefillShape, prefill_inputs, to_f64
+
+    shape = PrefillShape(**PREFILL, dtype=torch.bfloat16)
+    d = prefill_inputs(shape, seed=0, device="cpu")
+    arrs = [np.ascontiguousarray(to_f64(d[x])[:, :, :heads]) for x in ("q", "k", "v", "log_alpha", "beta")]
+    s0 = np.ascontiguousarray(to_f64(d["init_state"])[:, :heads])
+    cores = threads or oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle.forward(*arrs, init_state=s0, nthreads=cores)
+    dt = time.perf_counter() - t0
+    token_heads = PREFILL["T"] * heads
+    return {"value": token_heads / dt / PREFILL["H"], "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "seconds": dt,
+            "sample": f"fp64 token recurrence on {heads} of {PREFILL['H']} heads x {PREFILL['T']} tokens of "
+                      f"prefill_8k (rate scaled to all {PREFILL['H']} heads)"}
+
+
+def config_block():
+    return {"workload": "prefill_8k", "B": PREFILL["B"], "T": PREFILL["T"], "H": PREFILL["H"],
+            "dk": PREFILL["dk"], "dv": PREFILL["dv"], "chunk": CHUNK, "global_batch": PREFILL["B"],
+            "seq_len": PREFILL["T"], "parallelism": "replicas",
+            "l2": "inputs larger than L2 (408 MB per step vs 126 MB)"}
+
+
+def main_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    samples = []
+    heads = 16
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(heads=heads)
+        if i >= args.warmup:
+            samples.append(r)
+    secs = [s["seconds"] for s in samples]
+    value = statistics.median([s["value"] for s in samples])
+    line = {
+        "impl": "reference", "metric": "KDA chunked prefill tokens/s (B=1, T=8192, H=32, d=128)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(secs) * PREFILL["H"] / heads, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_block(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": samples[0]["cores"], "kind": "oracle",
+                         "sample": samples[0]["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="kda", choices=["kda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return main_reference(args)
+
+    import torch
+
+    world, rank, local = _dist()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    import gated_delta_rule_85_b200 as kda
+
+    kda.load_library()
+
+    pre = run_prefill(args, world, rank, dev)
+    dec = None if args.no_decode else run_decode(args, world, rank, dev)
+
+    hbm_gbs, bf16_tflops, peak_src = _peaks()
+    ms_step = pre["total_ms"] / args.steps
+    tokens = PREFILL["B"] * PREFILL["T"]
+    value = world * tokens / (ms_step * 1e-3)
+    token_heads = tokens * PREFILL["H"]
+    alg_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * PREFILL["H"] * STATE_BYTES
+    alg_flops = token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD
+    launch_ms = statistics.mean(pre["per_launch_ms"])
+    gbs = alg_bytes / (launch_ms * 1e-3) / 1e9
+    tflops = alg_flops / (launch_ms * 1e-3) / 1e12
+    line = {
+        "metric": "KDA chunked prefill tokens/s (B=1, T=8192, H=32, d=128)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": config_block(),
+        "roofline": {"kernel": "chunk_tc_kernel", "bound": "hbm", "achieved": gbs, "peak": hbm_gbs,
+                     "unit": "GB/s", "frac": gbs / hbm_gbs, "traffic": None,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
+                     "algorithmic_bytes": alg_bytes, "launch_ms": launch_ms,
+                     "tensor": {"achieved_tflops": tflops, "peak_tflops": bf16_tflops,
+                                "frac": tflops / bf16_tflops, "algorithmic_flops": alg_flops}},
+        "e2e": {"value": world * tokens / (pre["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"],
+                "api": "gated_delta_rule_85_b200.chunk_forward with pinned host tensors"},
+        "gpu_launches": args.steps,
+        "clocks": pre["clocks"],
+    }
+    if dec is not None:
+        step_ms = dec["ms"] / dec["launches"]
+        dbytes = DECODE["N"] * DECODE["H"] * DECODE_BYTES_PER_PAIR
+        dgbs = dbytes / (step_ms * 1e-3) / 1e9
+        line["decode"] = {
+            "metric": "KDA decode tokens/s (N=256 sequences, H=32, d=128, 1 token per step)",
+            "value": world * DECODE["N"] / (step_ms * 1e-3), "unit": "tokens/s", "ms_per_step": step_ms,
+            "steps": dec["launches"], "graph": "1024 steps per CUDA graph replay",
+            "roofline": {"kernel": "decode_step_kernel", "bound": "hbm", "achieved": dgbs, "peak": hbm_gbs,
+                         "unit": "GB/s", "frac": dgbs / hbm_gbs, "traffic": None, "algorithmic_bytes": dbytes},
+            "clocks": dec["clocks"],
+        }
+        line["gpu_launches"] += dec["launches"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(heads=32)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

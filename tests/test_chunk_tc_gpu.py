@@ -1,0 +1,92 @@
+"""kda_chunk_forward (tcgen05 tensor-core prefill, bf16) vs the fp64 oracle (GPU).
+
+Bound for bf16 inputs: rel-L2 <= 1e-2 and max-abs <= 5e-2 on o and the final state."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_85_b200 as kda
+from gated_delta_rule_85_b200.workloads import PrefillShape, prefill_inputs, to_f64
+from kda_testutil import assert_close, oracle_prefill, rel_l2
+
+pytestmark = pytest.mark.gpu
+BF16 = torch.bfloat16
+
+
+def _run(shape, seed=0, final_state=True):
+    d = prefill_inputs(shape, seed, torch.device("cuda"))
+    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"],
+                             d["cu_seqlens"], final_state=final_state)
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    return d, o, S
+
+
+def _check(shape, seed=0):
+    d, o, S = _run(shape, seed)
+    o_ref, S_ref = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+    assert_close(to_f64(S), S_ref, BF16, "final state")
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 130, 517])
+def test_lengths_d128(T):
+    _check(PrefillShape(B=1, T=T, H=2, dk=128, dv=128, dtype=BF16), seed=T)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+def test_head_dims(dk, dv):
+    _check(PrefillShape(B=2, T=200, H=2, dk=dk, dv=dv, dtype=BF16), seed=dk * 3 + dv)
+
+
+def test_many_chunks_wide_tiles():
+    """Enough (sequence, head) pairs that the 64-column value tiles are used."""
+    _check(PrefillShape(B=4, T=300, H=40, dk=128, dv=128, dtype=BF16), seed=11)
+
+
+def test_zero_initial_state_and_no_final_state():
+    shape = PrefillShape(B=1, T=150, H=2, dk=128, dv=128, dtype=BF16, init_state="none")
+    d, o, S = _run(shape, seed=4, final_state=False)
+    assert S is None
+    o_ref, _ = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+
+
+def test_varlen_with_empty_and_short_sequences():
+    cu = (0, 0, 1, 64, 64, 200, 391)
+    _check(PrefillShape(B=1, T=391, H=3, dk=128, dv=128, dtype=BF16, cu_seqlens=cu), seed=9)
+
+
+def test_matches_fp32_path_closely():
+    """Tensor-core and fp32 CUDA-core paths on the same bf16 inputs."""
+    shape = PrefillShape(B=1, T=1024, H=4, dk=128, dv=128, dtype=BF16)
+    d, o, S = _run(shape, seed=21)
+    o2, S2 = kda.chunk_forward_simt(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"])
+    torch.cuda.synchronize()
+    assert rel_l2(to_f64(o), to_f64(o2)) < 1e-2
+    assert rel_l2(to_f64(S), to_f64(S2)) < 1e-2
+
+
+def test_full_replacement_regime():
+    """beta = 1: the delta rule overwrites the value stored under each key; the
+    chunked tensor-core form must still agree with the recurrence."""
+    shape = PrefillShape(B=1, T=256, H=2, dk=128, dv=128, dtype=BF16)
+    d = prefill_inputs(shape, 5, torch.device("cuda"))
+    d["beta"].fill_(1.0)
+    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"])
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+    assert_close(to_f64(S), S_ref, BF16, "final state")
+
+
+def test_scalar_gate_gated_deltanet_regime():
+    """log_alpha equal across channels (the Gated DeltaNet special case)."""
+    shape = PrefillShape(B=1, T=256, H=2, dk=128, dv=128, dtype=BF16)
+    d = prefill_inputs(shape, 6, torch.device("cuda"))
+    d["log_alpha"].copy_(d["log_alpha"][..., :1].expand_as(d["log_alpha"]))
+    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"])
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+    assert_close(to_f64(S), S_ref, BF16, "final state")
