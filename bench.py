@@ -175,6 +175,9 @@ def run_prefill(args, world, rank, dev):
     per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = _max_over_ranks(total_ms, world, dev)
 
+    if args.no_e2e:
+        return dict(total_ms=total_ms, per_launch_ms=per_launch_ms, clocks=clk.summary(), e2e_ms=float("nan"),
+                    h2d=0, d2h=0, e2e_steps=0)
     # End to end through the public API with host buffers: H2D of every input,
     # the kernel, D2H of o and the final state, every step.
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in d.items()}
@@ -311,6 +314,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="kda", choices=["kda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
