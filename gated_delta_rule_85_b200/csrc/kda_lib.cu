@@ -32,10 +32,11 @@ int check_prefill(const void *q, const void *k, const void *v, const float *log_
                   const float *beta, const float *init_state, const void *o, const float *final_state,
                   const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
                   int dtype, int chunk) {
-    if (!q || !k || !v || !log_alpha || !beta || !o)
-        return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta and o are required");
     if (B < 1 || T < 0 || H < 1 || num_seqs < 0)
         return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d num_seqs=%d", B, T, H, num_seqs);
+    // With no tokens the per-token tensors are empty and may be NULL.
+    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !o))
+        return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta and o are required");
     if (H > 65535) return fail(KDA_ERR_UNSUPPORTED, "H=%d above 65535", H);
     if (cu_seqlens) {
         if (B != 1) return fail(KDA_ERR_INVALID_ARG, "packed (cu_seqlens) input needs B == 1, got %d", B);
@@ -52,7 +53,7 @@ int check_prefill(const void *q, const void *k, const void *v, const float *log_
     const char *n16[] = {"q", "k", "v", "log_alpha", "o", "init_state", "final_state"};
     for (int i = 0; i < 7; ++i)
         if (p16[i] && !aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
-    if (!aligned(beta, 4)) return fail(KDA_ERR_MISALIGNED, "beta is not 4-byte aligned");
+    if (beta && !aligned(beta, 4)) return fail(KDA_ERR_MISALIGNED, "beta is not 4-byte aligned");
     if (cu_seqlens && !aligned(cu_seqlens, 4)) return fail(KDA_ERR_MISALIGNED, "cu_seqlens is not 4-byte aligned");
     return KDA_OK;
 }
@@ -146,9 +147,10 @@ int kda_chunk_forward(const void *q, const void *k, const void *v, const float *
 int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,
                        const float *beta, float *state, void *o, int N, int H, int dk, int dv, int dtype,
                        void *stream) {
+    if (N < 0 || H < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d", N, H);
+    if (N == 0) return KDA_OK;   // nothing to do; empty tensors may carry NULL pointers
     if (!q || !k || !v || !log_alpha || !beta || !state || !o)
         return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta, state and o are required");
-    if (N < 0 || H < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d", N, H);
     if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
         return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: each must be 64 or 128", dk, dv);
     if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "dtype=%d", dtype);

@@ -88,10 +88,10 @@ typedef enum kda_dtype {
  * chunkwise, diagonal-plus-low-rank form of "Kimi Linear、独自の土俵でFull Attention
  * を上回る" § "Kimi Linearがより賢いRecurrent Memoryを使う方法".
  *
- *   q, k, v       inputs in `dtype`, layouts above (required)
- *   log_alpha     fp32 [B,T,H,dk] (required); beta fp32 [B,T,H] (required)
+ *   q, k, v       inputs in `dtype`, layouts above (required when T > 0)
+ *   log_alpha     fp32 [B,T,H,dk]; beta fp32 [B,T,H] (required when T > 0)
  *   init_state    fp32 [N,H,dk,dv] or NULL (zeros)
- *   o             output [B,T,H,dv] in `dtype` (required); rounded to nearest-even
+ *   o             output [B,T,H,dv] in `dtype` (required when T > 0); rounded to nearest-even
  *   final_state   fp32 [N,H,dk,dv] or NULL (not written)
  *   cu_seqlens    int32 [N+1] device array or NULL (dense batch)
  *   B, T, H       batch, tokens per row, heads (T may be 0)
@@ -134,6 +134,7 @@ int kda_chunk_forward_simt(const void *q, const void *k, const void *v, const fl
  *   q, k     [N, H, dk] in dtype;  v, o [N, H, dv] in dtype
  *   log_alpha fp32 [N, H, dk];     beta fp32 [N, H]
  *   state    fp32 [N, H, dk, dv], read once and written once (in place)
+ * N == 0 is a no-op (pointers may then be NULL).
  * Each state is streamed once from HBM and written back once.
  */
 int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -36,12 +36,19 @@ def assert_close(got, want, dtype, what=""):
 
 
 def oracle_prefill(d, heads=None):
-    """Oracle on the inputs dict (optionally a subset of heads).  Returns (o, S) float64."""
+    """Oracle on the inputs dict (optionally a subset of heads, selected on the
+    device before widening to float64).  Returns (o, S) float64."""
     keys = ["q", "k", "v", "log_alpha", "beta"]
-    arrs = [to_f64(d[x]) for x in keys]
-    s0 = to_f64(d.get("init_state"))
-    if heads is not None:
-        arrs = [a[:, :, heads] for a in arrs]
-        s0 = None if s0 is None else s0[:, heads]
+
+    def pick(x, state=False):
+        if x is None:
+            return None
+        if heads is not None:
+            idx = torch.as_tensor(heads, device=x.device)
+            x = x.index_select(1 if state else 2, idx)
+        return to_f64(x)
+
+    arrs = [pick(d[x]) for x in keys]
+    s0 = pick(d.get("init_state"), state=True)
     cu = None if d.get("cu_seqlens") is None else d["cu_seqlens"].cpu().numpy()
     return oracle.forward(*arrs, init_state=s0, cu_seqlens=cu)

@@ -1,0 +1,107 @@
+"""Full-size parity on the five workloads, in the launch configuration the
+benchmark uses, against the fp64 oracle on sampled heads / (sequence, head)
+pairs (each sample covers every token of its sequence).
+
+  tiny_f32      B=1 H=2 T=256 d=64 fp32            all outputs       rel-L2 <= 1e-4
+  prefill_8k    B=1 H=32 T=8192 d=128 bf16         all 32 heads      rel-L2 <= 1e-2, max-abs <= 5e-2
+  prefill_128k  B=1 H=32 T=131072 d=128 bf16       8 heads
+  decode_b256   N=256 H=32 d=128, 1024 steps        64 (n, h) pairs, every step
+  varlen_1m     1,048,576 packed tokens (22 seqs)   2 heads, all sequences; then 256 decode steps
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_85_b200 as kda
+import oracle
+from gated_delta_rule_85_b200.workloads import (CONFIGS, DecodeShape, decode_step_inputs, draw_state,
+                                                prefill_inputs, to_f64, varlen_1m_shape)
+from kda_testutil import assert_close, oracle_prefill
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+BF16 = torch.bfloat16
+DEV = "cuda"
+
+
+def _prefill(d):
+    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], d["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    return o, S
+
+
+def test_tiny_f32_through_main_entry_point():
+    shape = CONFIGS["tiny_f32"]
+    d = prefill_inputs(shape, 0, torch.device(DEV))
+    o, S = _prefill(d)
+    o_ref, S_ref = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, torch.float32, "o")
+    assert_close(to_f64(S), S_ref, torch.float32, "final state")
+
+
+def test_prefill_8k_all_heads():
+    shape = CONFIGS["prefill_8k"]
+    d = prefill_inputs(shape, 0, torch.device(DEV))
+    o, S = _prefill(d)
+    o_ref, S_ref = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+    assert_close(to_f64(S), S_ref, BF16, "final state")
+
+
+def test_prefill_128k_sampled_heads():
+    shape = CONFIGS["prefill_128k"]
+    d = prefill_inputs(shape, 0, torch.device(DEV))
+    o, S = _prefill(d)
+    heads = [0, 4, 9, 13, 18, 22, 27, 31]
+    o_ref, S_ref = oracle_prefill(d, heads)
+    assert_close(to_f64(o[:, :, heads]), o_ref, BF16, "o")
+    assert_close(to_f64(S[:, heads]), S_ref, BF16, "final state")
+
+
+def test_decode_b256_1024_steps_sampled_pairs():
+    shape = CONFIGS["decode_b256"]
+    dev = torch.device(DEV)
+    state = draw_state((shape.N, shape.H, shape.dk, shape.dv), dev, 0, 6)
+    rng = np.random.default_rng(0)
+    flat = rng.choice(shape.N * shape.H, size=64, replace=False)
+    n_idx = torch.tensor(flat // shape.H, device=dev)
+    h_idx = torch.tensor(flat % shape.H, device=dev)
+    S_ref = to_f64(state[n_idx, h_idx])[:, None]          # [64, 1, dk, dv]: pairs as sequences
+    o_got, o_want = [], []
+    for t in range(shape.steps):
+        d = decode_step_inputs(shape, t, 0, dev)
+        o = kda.recurrent_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], state)
+        sel = [to_f64(d[x][n_idx, h_idx])[:, None] for x in ("q", "k", "v", "log_alpha", "beta")]
+        o_t, S_ref = oracle.step(*sel, S_ref)
+        o_want.append(o_t[:, 0])
+        o_got.append(to_f64(o[n_idx, h_idx]))
+    torch.cuda.synchronize()
+    assert_close(np.stack(o_got), np.stack(o_want), BF16, "o (all steps)")
+    assert_close(to_f64(state[n_idx, h_idx]), S_ref[:, 0], BF16, "final state")
+
+
+def test_varlen_1m_then_decode_sampled_heads():
+    shape = varlen_1m_shape()
+    assert shape.T == 1 << 20 and shape.num_seqs == 22
+    dev = torch.device(DEV)
+    d = prefill_inputs(shape, 0, dev)
+    o, S = _prefill(d)
+    heads = [5, 26]
+    o_ref, S_ref = oracle_prefill(d, heads)
+    assert_close(to_f64(o[:, :, heads]), o_ref, BF16, "o")
+    assert_close(to_f64(S[:, heads]), S_ref, BF16, "final state")
+    del d, o
+    # 256 decode steps per sequence, continuing from the prefill's final state in place
+    dshape = DecodeShape(N=shape.num_seqs, H=shape.H, dk=shape.dk, dv=shape.dv, steps=256, dtype=BF16)
+    o_got, o_want = [], []
+    S_ref = S_ref.copy()
+    for t in range(dshape.steps):
+        st = decode_step_inputs(dshape, t, 1, dev)
+        od = kda.recurrent_step(st["q"], st["k"], st["v"], st["log_alpha"], st["beta"], S)
+        sel = [to_f64(st[x][:, heads]) for x in ("q", "k", "v", "log_alpha", "beta")]
+        o_t, S_ref = oracle.step(*sel, S_ref)
+        o_want.append(o_t)
+        o_got.append(to_f64(od[:, heads]))
+    torch.cuda.synchronize()
+    assert_close(np.stack(o_got), np.stack(o_want), BF16, "decode o")
+    assert_close(to_f64(S[:, heads]), S_ref, BF16, "state after decode")
