@@ -42,25 +42,25 @@ namespace tc {
 constexpr int C = 64;
 constexpr int NT = 256;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;   // 1 s: far beyond any legitimate latency
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;
 // TMEM column map (fp32 accumulators, lane = row)
-constexpr uint32_t COL_GRAM = 0;    // [128 x 64]  rows 0-63 Khat Rk^T, rows 64-127 Qhat Rk^T
-constexpr uint32_t COL_XY = 64;     // [128 x DVT] rows 0-63 X, rows 64-127 Y (then O)
-constexpr uint32_t COL_KT = 128;    // [128 x 64]  Kt (and Pt rows 64-127 when dk = 64)
-constexpr uint32_t COL_PT = 192;    // [128 x 64]  rows 64-127 Pt (dk = 128)
-constexpr uint32_t COL_DS = 0;      // [128 x DVT] Kt Z (reuses the Gram columns)
+constexpr uint32_t COL_XY = 0;      // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O
+constexpr uint32_t COL_GRAM = 128;  // [128 x 64]  rows 0-63 Kp Kbar^T, rows 64-127 Qp Kbar^T
+constexpr uint32_t COL_KT = 192;    // [128 x 64]  Kt (lanes 0..dk-1)
+constexpr uint32_t COL_PT = 256;    // [128 x 64]  Pt (lanes 64-127)
+constexpr uint32_t COL_DS = 320;    // [128 x DVT] Kt Z (lanes 0..dk-1)
 constexpr int AS = 68;              // fp32 row stride of the 64 x 64 scratch matrices (16-byte rows)
 
 template <int DK, int DVT>
 struct Layout {
     static constexpr int KA = DK / 64;                       // 64-element K atoms along dk
     // bf16 MMA operands, 128-byte swizzled, 1024-byte aligned
-    static constexpr int KQ = 0;                             // [KA][128][128 B] Khat (0-63), Qhat (64-127)
-    static constexpr int RK = KQ + KA * 128 * 128;           // [KA][64][128 B]  Rk
-    static constexpr int SB = RK + KA * 64 * 128;            // [KA][DVT][128 B] S^T (bf16): B operand
-    static constexpr int KP = SB + KA * DVT * 128;           // [DK+64][128 B]   Kbar^T -> Kt ; Aqk -> Pt
+    static constexpr int KQ = 0;                             // [KA][128][128 B] Kp (0-63), Qp (64-127)
+    static constexpr int KB = KQ + KA * 128 * 128;           // [KA][64][128 B]  Kbar (rows = tokens)
+    static constexpr int KP = KB + KA * 64 * 128;            // [DK+64][128 B]   Kt (0..DK-1), Aqk -> Pt (DK..)
     static constexpr int TB = KP + (DK + 64) * 128;          // [64][128 B]      Tb^T
-    static constexpr int ZT = TB + 64 * 128;                 // [DVT][128 B]     Z^T
+    static constexpr int SB = TB + 64 * 128;                 // [KA][DVT][128 B] (e^{G_last} S)^T
+    static constexpr int ZT = SB + KA * DVT * 128;           // [DVT][128 B]     Z^T
     // dense TMA input tiles; the fp32 scratch of the UT transform aliases them
     static constexpr int QIN = ZT + DVT * 128;               // bf16 [64][DK]
     static constexpr int KIN = QIN + 64 * DK * 2;            // bf16 [64][DK]
@@ -71,22 +71,21 @@ struct Layout {
     static constexpr int FM = FT + 64 * AS * 4;              // fp32 [32][36]   block-product scratch
     static constexpr int SCR_BYTES = 2 * 64 * AS * 4 + 32 * 36 * 4;
     static constexpr int SPAN = IN_BYTES > SCR_BYTES ? IN_BYTES : SCR_BYTES;
-    static constexpr int VIN = QIN + SPAN;                   // bf16 [2][64][DVT]
-    static constexpr int FB = VIN + 2 * 64 * DVT * 2;        // fp32 [2][64]    beta
-    static constexpr int FD = FB + 2 * 64 * 4;               // fp32 [DK]       e^{G_last}
-    static constexpr int NSEG = NT / (DK / 2);               // token segments in the factor stage
-    static constexpr int FSEG = FD + DK * 4;                 // fp32 [NSEG][DK] segment sums of log_alpha
+    static constexpr int VIN = QIN + SPAN;                   // bf16 [64][DVT]
+    static constexpr int FB = VIN + 64 * DVT * 2;            // fp32 [2][64]    beta
+    static constexpr int NSEG = NT / (DK / 4);               // token segments in the factor stage
+    static constexpr int FSEG = FB + 2 * 64 * 4;             // fp32 [NSEG][DK] segment sums of log_alpha
     static constexpr int MISC = FSEG + NSEG * DK * 4;        // mbarriers, TMEM base, flags
     static constexpr int BYTES = MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024 B
-    static_assert(KQ % 1024 == 0 && RK % 1024 == 0 && SB % 1024 == 0 && KP % 1024 == 0 &&
-                      TB % 1024 == 0 && ZT % 1024 == 0 && QIN % 1024 == 0 && VIN % 128 == 0,
+    static_assert(KQ % 1024 == 0 && KB % 1024 == 0 && KP % 1024 == 0 && TB % 1024 == 0 && SB % 1024 == 0 &&
+                      ZT % 1024 == 0 && QIN % 1024 == 0 && VIN % 128 == 0,
                   "tile alignment");
     static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
-// Byte offset of bf16 element (row, k) in a K-major, 128-byte-swizzled tile whose
-// K atoms (64 elements each) hold `rows` rows.
+// Byte offset of bf16 element (row, k) in a 128-byte-swizzled tile whose 64-wide
+// K atoms hold `rows` rows each.
 __device__ __forceinline__ uint32_t sw128(int row, int k, int rows) {
     const int atom = k >> 6, kk = k & 63;
     return (uint32_t)(atom * rows * 128 + row * 128 + ((((kk >> 3) ^ (row & 7))) << 4) + ((kk & 7) << 1));
@@ -106,6 +105,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ void st_bf16x2(uint8_t *base, uint32_t off, float a, float b) {
     *reinterpret_cast<uint32_t *>(base + off) = pack_bf16(a, b);
 }
+// Four consecutive values of a row as one 8-byte store (8-byte aligned offsets).
+__device__ __forceinline__ void st_bf16x4(uint8_t *base, uint32_t off, float a, float b, float c, float d) {
+    *reinterpret_cast<uint2 *>(base + off) = make_uint2(pack_bf16(a, b), pack_bf16(c, d));
+}
+__device__ __forceinline__ float4 ld_bf16x4(const uint8_t *p) {
+    const uint2 r = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
 // Eight consecutive values of a row as one 16-byte swizzled store.
 __device__ __forceinline__ void st_bf16x8(uint8_t *base, uint32_t off, const float *x) {
     *reinterpret_cast<uint4 *>(base + off) =
@@ -118,76 +127,101 @@ __device__ __forceinline__ float exp2_fast(float x) {
     return y;
 }
 
-// Descriptor of the 16-wide K step `s` of a swizzled tile at `addr` with `rows`
-// rows per K atom, starting at row r0 (a multiple of 8).
+// Descriptor of the 16-wide K step `s` of a K-major swizzled tile at `addr` with
+// `rows` rows per K atom, starting at row r0 (a multiple of 8).
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr, int s, int rows, int r0 = 0) {
     return ptx::desc_kmajor_sw128(addr + (uint32_t)((s >> 2) * rows * 128 + r0 * 128 + (s & 3) * 32));
 }
 
-// T = (I + A)^{-1} for a 64 x 64 strictly lower A (fp32, row stride AS): the four
-// 16 x 16 diagonal blocks by forward substitution, then the block-triangular
-// inverse [L11 0; L21 L22]^{-1} = [L11^-1 0; -L22^-1 L21 L11^-1  L22^-1] at 32 and
-// 64, each block product register-tiled over 256 threads.  The lower triangle
-// of T and the zero upper triangles of its four 16 x 16 diagonal blocks are
-// written; nothing reads T above those blocks.
-__device__ __forceinline__ void invert_unit_lower64(const float *A, float *Tm, float *M, int tid) {
-    if (tid < 64) {
-        const int o = 16 * (tid >> 4), l = tid & 15;
-        float x[16];
+__device__ __forceinline__ uint32_t f2tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// d (16 x 8 fragment of one warp) += X (16 x 8K, row-major, stride sx) * Y (8K x 8,
+// row-major, stride sy) on the tensor cores with tf32 inputs and fp32
+// accumulation (m16n8k8 fragments: lane = 4 g + t).
+template <int KSTEPS>
+__device__ __forceinline__ void warp_mm16x8_tf32(float (&d)[4], const float *X, int sx, const float *Y, int sy,
+                                                 int lane) {
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float acc = 0.f;
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+        const int k0 = ks * 8;
+        const uint32_t a0 = f2tf32(X[g * sx + k0 + t]), a1 = f2tf32(X[(g + 8) * sx + k0 + t]);
+        const uint32_t a2 = f2tf32(X[g * sx + k0 + t + 4]), a3 = f2tf32(X[(g + 8) * sx + k0 + t + 4]);
+        const uint32_t b0 = f2tf32(Y[(k0 + t) * sy + g]), b1 = f2tf32(Y[(k0 + t + 4) * sy + g]);
+        asm volatile(
+            "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+}
+
+__device__ __forceinline__ void warp_store16x8(float *Z, int sz, const float (&d)[4], float sign, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2 *>(Z + g * sz + 2 * t) = make_float2(sign * d[0], sign * d[1]);
+    *reinterpret_cast<float2 *>(Z + (g + 8) * sz + 2 * t) = make_float2(sign * d[2], sign * d[3]);
+}
+
+// Diagonal 16 x 16 blocks of T = (I + A)^{-1} (A strictly lower, fp32, row stride
+// AS) by forward substitution: 64 threads, one block column each, zeros above the
+// diagonal included.
+__device__ __forceinline__ void invert_diag_blocks(const float *A, float *Tm, int t64) {
+    const int o = 16 * (t64 >> 4), l = t64 & 15;
+    float x[16];
 #pragma unroll
-            for (int j = 0; j < i; ++j) acc = fmaf(A[(o + i) * AS + o + j], x[j], acc);
-            x[i] = (i < l) ? 0.f : ((i == l) ? 1.f : -acc);
+    for (int i = 0; i < 16; ++i) {
+        float acc = 0.f;
+#pragma unroll
+        for (int j4 = 0; j4 < 16; j4 += 4) {
+            if (j4 < i) {
+                const float4 a = *reinterpret_cast<const float4 *>(A + (o + i) * AS + o + j4);
+                if (j4 + 0 < i) acc = fmaf(a.x, x[j4 + 0], acc);
+                if (j4 + 1 < i) acc = fmaf(a.y, x[j4 + 1], acc);
+                if (j4 + 2 < i) acc = fmaf(a.z, x[j4 + 2], acc);
+                if (j4 + 3 < i) acc = fmaf(a.w, x[j4 + 3], acc);
+            }
         }
-        // the whole block column, zeros above the diagonal included: the vectorised
-        // block products below read a few of those entries
+        x[i] = (i < l) ? 0.f : ((i == l) ? 1.f : -acc);
+    }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) Tm[(o + i) * AS + o + l] = x[i];
+    for (int i = 0; i < 16; ++i) Tm[(o + i) * AS + o + l] = x[i];
+}
+
+// The rest of T once its diagonal blocks are in place and blocks (0,1) and (2,3)
+// are zero: the block-triangular inverse [L11 0; L21 L22]^{-1} =
+// [L11^-1 0; -L22^-1 L21 L11^-1  L22^-1] at 32 (two pairs of 16-blocks) and at 64,
+// each block product one 16 x 8 tile per warp on the tensor cores (tf32 inputs,
+// fp32 accumulation).  All 256 threads take part.
+__device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, float *M, int warp, int lane) {
+    if (warp < 4) {   // M_p = A[2p+1][2p] T[2p][2p]
+        const int p = warp >> 1, nt = warp & 1, ro = 32 * p + 16, co = 32 * p;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        warp_mm16x8_tf32<2>(d, A + ro * AS + co, AS, Tm + co * AS + co + 8 * nt, AS, lane);
+        warp_store16x8(M + p * 16 * 36 + 8 * nt, 36, d, 1.f, lane);
     }
     __syncthreads();
-    {   // M_p = A[2p+1][2p] T[2p][2p]; then T[2p+1][2p] = -T[2p+1][2p+1] M_p   (p = 0, 1)
-        const int p = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
-        const int ro = 32 * p + 16, co = 32 * p;
-        float a0 = 0.f, a1 = 0.f;
-        for (int j = c; j < 16; ++j) {
-            const float a = A[(ro + r) * AS + co + j];
-            const float2 t = *reinterpret_cast<const float2 *>(Tm + (co + j) * AS + co + c);
-            a0 = fmaf(a, t.x, a0);
-            a1 = fmaf(a, t.y, a1);
-        }
-        *reinterpret_cast<float2 *>(M + p * 16 * 36 + r * 36 + c) = make_float2(a0, a1);
-        __syncthreads();
-        float b0 = 0.f, b1 = 0.f;
-        for (int j = 0; j <= r; ++j) {
-            const float t = Tm[(ro + r) * AS + ro + j];
-            const float2 m = *reinterpret_cast<const float2 *>(M + p * 16 * 36 + j * 36 + c);
-            b0 = fmaf(t, m.x, b0);
-            b1 = fmaf(t, m.y, b1);
-        }
-        *reinterpret_cast<float2 *>(Tm + (ro + r) * AS + co + c) = make_float2(-b0, -b1);
+    if (warp < 4) {   // T[2p+1][2p] = -T[2p+1][2p+1] M_p
+        const int p = warp >> 1, nt = warp & 1, ro = 32 * p + 16, co = 32 * p;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        warp_mm16x8_tf32<2>(d, Tm + ro * AS + ro, AS, M + p * 16 * 36 + 8 * nt, 36, lane);
+        warp_store16x8(Tm + ro * AS + co + 8 * nt, AS, d, -1.f, lane);
     }
     __syncthreads();
-    {   // M = A[hi][lo] T[lo][lo]; then T[hi][lo] = -T[hi][hi] M   (32 x 32 blocks)
-        const int r = tid >> 3, c = (tid & 7) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = c; j < 32; ++j) {
-            const float a = A[(32 + r) * AS + j];
-            const float4 t = *reinterpret_cast<const float4 *>(Tm + j * AS + c);
-            acc.x = fmaf(a, t.x, acc.x); acc.y = fmaf(a, t.y, acc.y);
-            acc.z = fmaf(a, t.z, acc.z); acc.w = fmaf(a, t.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(M + r * 36 + c) = acc;
-        __syncthreads();
-        float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j <= r; ++j) {
-            const float t = Tm[(32 + r) * AS + 32 + j];
-            const float4 m = *reinterpret_cast<const float4 *>(M + j * 36 + c);
-            b.x = fmaf(t, m.x, b.x); b.y = fmaf(t, m.y, b.y);
-            b.z = fmaf(t, m.z, b.z); b.w = fmaf(t, m.w, b.w);
-        }
-        *reinterpret_cast<float4 *>(Tm + (32 + r) * AS + c) = make_float4(-b.x, -b.y, -b.z, -b.w);
+    const int mt = warp >> 2, nt = warp & 3;
+    {   // M = A[hi][lo] T[lo][lo]
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        warp_mm16x8_tf32<4>(d, A + (32 + 16 * mt) * AS, AS, Tm + 8 * nt, AS, lane);
+        warp_store16x8(M + 16 * mt * 36 + 8 * nt, 36, d, 1.f, lane);
+    }
+    __syncthreads();
+    {   // T[hi][lo] = -T[hi][hi] M
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        warp_mm16x8_tf32<4>(d, Tm + (32 + 16 * mt) * AS + 32, AS, M + 8 * nt, 36, lane);
+        warp_store16x8(Tm + (32 + 16 * mt) * AS + 8 * nt, AS, d, -1.f, lane);
     }
     __syncthreads();
 }
@@ -216,6 +250,9 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 u, float *x) {
     }
 }
 
+// Threads are grouped by TMEM lane quadrant: warp w reads lanes 32 (w % 4) ..
+// 32 (w % 4) + 31.  State row r (= key channel = TMEM lane) is held by the two
+// warps with w % 4 == r / 32, one per half of the value tile's columns.
 template <int DK, int DVT>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -224,8 +261,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 __nv_bfloat16 *__restrict__ o, float *__restrict__ final_state,
                 const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
     using L = Layout<DK, DVT>;
-    static_assert(DVT % 16 == 0 && DVT >= 16 && DVT <= 64, "value tile");
-    constexpr int NPAIR = DK / 2, NSEG = L::NSEG, SEGLEN = C / NSEG;
+    static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
+    constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG;   // factor stage: 4 channels x SEGLEN tokens
+    constexpr int CPT = DVT / 2;                              // state / output columns per thread
     constexpr float LOG2E = 1.4426950408889634f;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -234,14 +272,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *fT = reinterpret_cast<float *>(sm + L::FT);
     float *fM = reinterpret_cast<float *>(sm + L::FM);
     float *fB = reinterpret_cast<float *>(sm + L::FB);
-    float *fD = reinterpret_cast<float *>(sm + L::FD);
     float *fSeg = reinterpret_cast<float *>(sm + L::FSEG);
-    const uint32_t bar_mma = sb + L::MISC, bar_in = sb + L::MISC + 8;
-    const uint32_t bar_v0 = sb + L::MISC + 16;          // + 8 * buffer
+    const uint32_t bar_mma = sb + L::MISC, bar_in = sb + L::MISC + 8, bar_v = sb + L::MISC + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 32);
     int *fail_flag = reinterpret_cast<int *>(sm + L::MISC + 36);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
     const int col_base = blockIdx.x * DVT, h = blockIdx.y, n = blockIdx.z;
 
     long long t0, t1;
@@ -255,8 +292,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
         ptx::mbar_init(bar_mma, 1);
         ptx::mbar_init(bar_in, 1);
-        ptx::mbar_init(bar_v0, 1);
-        ptx::mbar_init(bar_v0 + 8, 1);
+        ptx::mbar_init(bar_v, 1);
         *fail_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_q);
@@ -268,8 +304,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);   // this warp's TMEM lane quadrant
-    uint32_t ph_mma = 0, ph_in = 0, ph_v[2] = {0u, 0u};
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);   // this warp's TMEM lane quadrant
+    uint32_t ph_mma = 0, ph_in = 0, ph_v = 0;
 
     auto issue_inputs = [&](int ci) {   // thread 0 only
         const int z = (int)(t0 + (long long)ci * C);
@@ -280,18 +316,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
     auto issue_v = [&](int ci) {        // thread 0 only
         const int z = (int)(t0 + (long long)ci * C);
-        const uint32_t bar = bar_v0 + 8u * (uint32_t)(ci & 1);
-        ptx::mbar_arrive_expect_tx(bar, (uint32_t)(C * DVT * 2));
-        ptx::tma_load_3d(sb + L::VIN + (uint32_t)((ci & 1) * C * DVT * 2), &tm_v, bar, col_base, h, z);
+        ptx::mbar_arrive_expect_tx(bar_v, (uint32_t)(C * DVT * 2));
+        ptx::tma_load_3d(sb + L::VIN, &tm_v, bar_v, col_base, h, z);
     };
 
-    const bool has_row = tid < DK;
-    const long long st_off = ((long long)n * H + h) * DK * DV + col_base;
-    float S[DVT];
+    // state rows held by this thread: row = key channel = TMEM lane
+    const int srow = quad * 32 + lane;
+    const bool has_row = srow < DK;
+    const int scol = half * CPT;
+    const long long st_off = ((long long)n * H + h) * DK * DV + col_base + scol;
+    float S[CPT];
 #pragma unroll
-    for (int j = 0; j < DVT; j += 4) {
+    for (int j = 0; j < CPT; j += 4) {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (has_row && init_state) x = load4(init_state + st_off + (long long)tid * DV + j);
+        if (has_row && init_state) x = load4(init_state + st_off + (long long)srow * DV + j);
         S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
     }
     if (nck > 0) {
@@ -303,10 +341,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int L0 = (int)min((long long)C, t1 - t0);
             fB[tid] = tid < L0 ? beta[(t0 + tid) * H + h] : 0.f;
         }
-        if (has_row) {
-#pragma unroll
-            for (int j = 0; j < DVT; ++j) st_bf16(sm, L::SB + sw128(j, tid, DVT), S[j]);
-        }
     }
 
     bool ok = true;
@@ -315,86 +349,100 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int Lc = (int)min((long long)C, t1 - cs);
         const int buf = ci & 1;
         float beta_next = 0.f;
-        if (ci + 1 < nck) {
-            if (tid == 0) issue_v(ci + 1);
-            if (tid < C) {
-                const int Ln = (int)min((long long)C, t1 - cs - C);
-                beta_next = tid < Ln ? beta[(cs + C + tid) * H + h] : 0.f;
-            }
+        if (ci + 1 < nck && tid < C) {
+            const int Ln = (int)min((long long)C, t1 - cs - C);
+            beta_next = tid < Ln ? beta[(cs + C + tid) * H + h] : 0.f;
         }
 
-        // ---- 1. decay factors -> bf16 operand tiles (two channels x one token segment per thread)
+        // ---- 1. decay factors (one exp per element) -> Kp, Qp, Kbar; e^{G_last} S -> bf16 operand
         if (!(ok = wait_all(bar_in, ph_in))) break;
+        float dch = 0.f;   // e^{G_last} of this thread's state row
         {
-            const int pr = tid % NPAIR, seg = tid / NPAIR, c0 = 2 * pr;
+            const int cg = tid % NCG, seg = tid / NCG, c0 = 4 * cg, i0 = seg * SEGLEN;
             const float *gin = reinterpret_cast<const float *>(sm + L::GIN);
-            float s0 = 0.f, s1 = 0.f;
+            const uint8_t *qin = sm + L::QIN, *kin = sm + L::KIN;
+            float al[SEGLEN][4];
+            float4 sg = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int u = 0; u < SEGLEN; ++u) {
-                const int i = seg * SEGLEN + u;
-                if (i < Lc) {
-                    const float2 g2 = *reinterpret_cast<const float2 *>(gin + i * DK + c0);
-                    s0 += g2.x;
-                    s1 += g2.y;
-                }
+                float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i0 + u < Lc) g4 = *reinterpret_cast<const float4 *>(gin + (i0 + u) * DK + c0);
+                sg.x += g4.x; sg.y += g4.y; sg.z += g4.z; sg.w += g4.w;
+                al[u][0] = g4.x; al[u][1] = g4.y; al[u][2] = g4.z; al[u][3] = g4.w;
             }
-            fSeg[seg * DK + c0] = s0;
-            fSeg[seg * DK + c0 + 1] = s1;
+            *reinterpret_cast<float4 *>(fSeg + seg * DK + c0) = sg;
             __syncthreads();
-            float G0 = 0.f, G1 = 0.f, tot0 = 0.f, tot1 = 0.f;
+            float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int s = 0; s < NSEG; ++s) {
-                const float a = fSeg[s * DK + c0], b = fSeg[s * DK + c0 + 1];
-                if (s < seg) { G0 += a; G1 += b; }
-                tot0 += a;
-                tot1 += b;
-            }
-            const float d0 = expf(tot0), d1 = expf(tot1);
-            if (seg == 0) {
-                fD[c0] = d0;
-                fD[c0 + 1] = d1;
-                if (tot0 < -80.f || tot1 < -80.f) flag_status(KDA_DEV_DECAY_RANGE);
-            }
-            const __nv_bfloat162 *qin = reinterpret_cast<const __nv_bfloat162 *>(sm + L::QIN);
-            const __nv_bfloat162 *kin = reinterpret_cast<const __nv_bfloat162 *>(sm + L::KIN);
+            for (int s2 = 0; s2 < NSEG; ++s2) {
+                const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
+                const float xv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-            for (int u = 0; u < SEGLEN; u += 2) {
-                float kb0[2], kb1[2];
-#pragma unroll
-                for (int w = 0; w < 2; ++w) {
-                    const int i = seg * SEGLEN + u + w;
-                    float2 q2 = make_float2(0.f, 0.f), k2 = make_float2(0.f, 0.f), g2 = make_float2(0.f, 0.f);
-                    if (i < Lc) {
-                        q2 = __bfloat1622float2(qin[(i * DK + c0) >> 1]);
-                        k2 = __bfloat1622float2(kin[(i * DK + c0) >> 1]);
-                        g2 = *reinterpret_cast<const float2 *>(gin + i * DK + c0);
-                    }
-                    G0 += g2.x;
-                    G1 += g2.y;
-                    const float e0 = exp2_fast(G0 * LOG2E), e1 = exp2_fast(G1 * LOG2E);
-                    const float r0 = exp2_fast(-G0 * LOG2E), r1 = exp2_fast(-G1 * LOG2E);
-                    st_bf16x2(sm, L::KQ + sw128(i, c0, 128), k2.x * e0, k2.y * e1);
-                    st_bf16x2(sm, L::KQ + sw128(64 + i, c0, 128), q2.x * e0, q2.y * e1);
-                    st_bf16x2(sm, L::RK + sw128(i, c0, 64), k2.x * r0, k2.y * r1);
-                    kb0[w] = k2.x * (d0 * r0);
-                    kb1[w] = k2.y * (d1 * r1);
+                for (int e = 0; e < 4; ++e) {
+                    if (s2 < seg) pre[e] += xv[e];
+                    tot[e] += xv[e];
                 }
-                const int i0 = seg * SEGLEN + u;
-                st_bf16x2(sm, L::KP + sw128(c0, i0, DK + 64), kb0[0], kb0[1]);
-                st_bf16x2(sm, L::KP + sw128(c0 + 1, i0, DK + 64), kb1[0], kb1[1]);
             }
+            if (seg == 0 && (tot[0] < -80.f || tot[1] < -80.f || tot[2] < -80.f || tot[3] < -80.f))
+                flag_status(KDA_DEV_DECAY_RANGE);
+            if (has_row) {
+                float tr = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < NSEG; ++s2) tr += fSeg[s2 * DK + srow];
+                dch = expf(tr);
+            }
+#pragma unroll
+            for (int u = 0; u < SEGLEN; ++u)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) al[u][e] = exp2_fast(al[u][e] * LOG2E);
+            const float sgv[4] = {sg.x, sg.y, sg.z, sg.w};
+            // forward: ef = e^{G_i - G_last} (>= 1; bounded by e^80 under the range precondition)
+            float ef[4], eb[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ef[e] = expf(pre[e] - tot[e]);
+                eb[e] = expf(tot[e] - pre[e] - sgv[e]);
+            }
+#pragma unroll
+            for (int u = 0; u < SEGLEN; ++u) {
+                const int i = i0 + u;
+                float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < Lc) {
+                    q4 = ld_bf16x4(qin + (i * DK + c0) * 2);
+                    k4 = ld_bf16x4(kin + (i * DK + c0) * 2);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ef[e] *= al[u][e];
+                st_bf16x4(sm, L::KQ + sw128(i, c0, 128), k4.x * ef[0], k4.y * ef[1], k4.z * ef[2], k4.w * ef[3]);
+                st_bf16x4(sm, L::KQ + sw128(64 + i, c0, 128), q4.x * ef[0], q4.y * ef[1], q4.z * ef[2],
+                          q4.w * ef[3]);
+            }
+            // backward: eb = e^{G_last - G_i} (<= 1)
+#pragma unroll
+            for (int u = SEGLEN - 1; u >= 0; --u) {
+                const int i = i0 + u;
+                float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < Lc) k4 = ld_bf16x4(kin + (i * DK + c0) * 2);
+                st_bf16x4(sm, L::KB + sw128(i, c0, 64), k4.x * eb[0], k4.y * eb[1], k4.z * eb[2], k4.w * eb[3]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) eb[e] *= al[u][e];
+            }
+        }
+        if (has_row) {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::SB + sw128(scol + j, srow, DVT), dch * S[j]);
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 2. Gram [Khat; Qhat] Rk^T and [X; Y] = [Khat; Qhat] S
+        // ---- 2. Gram [Kp; Qp] Kbar^T and [X; Y] = [Kp; Qp] (e^{G_last} S)
         if (tid == 0) {
             ptx::tc_fence_after();
             constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64), ix = ptx::idesc_bf16_f32(128, DVT);
 #pragma unroll
             for (int s = 0; s < DK / 16; ++s)
-                ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::RK, s, 64), ig, s > 0);
+                ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KB, s, 64), ig, s > 0);
 #pragma unroll
             for (int s = 0; s < DK / 16; ++s)
                 ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::SB, s, DVT), ix, s > 0);
@@ -402,43 +450,47 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
 
-        // ---- 3. Gram -> Diag(beta) Akk (fp32) and masked Aqk (bf16); Z = V - X; UT transform
-        if (warp < 4) {
+        // ---- 3. Gram -> Diag(beta) Akk (fp32) -> diagonal blocks of T (warps 0-1);
+        //        masked Aqk -> bf16 (warps 2-3); Z = V - X (warps 4-5); zero blocks of T (6-7)
+        if (warp < 2) {
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 float g32[32];
                 ptx::tmem_ld32(tl + COL_GRAM + hh * 32, g32);
                 ptx::tmem_wait_ld();
-                if (tid < 64) {
-                    const int i = tid;
-                    const float bi = fB[buf * C + i];
+                const int i = tid;
+                const float bi = fB[buf * C + i];
 #pragma unroll
-                    for (int u = 0; u < 32; u += 4) {
-                        const int j = hh * 32 + u;
-                        float4 a;
-                        a.x = (j + 0 < i) ? bi * g32[u + 0] : 0.f;
-                        a.y = (j + 1 < i) ? bi * g32[u + 1] : 0.f;
-                        a.z = (j + 2 < i) ? bi * g32[u + 2] : 0.f;
-                        a.w = (j + 3 < i) ? bi * g32[u + 3] : 0.f;
-                        *reinterpret_cast<float4 *>(fA + i * AS + j) = a;
-                    }
-                } else {
-                    const int i = tid - 64;
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) g32[u] = (hh * 32 + u <= i) ? g32[u] : 0.f;
-#pragma unroll
-                    for (int gq = 0; gq < 4; ++gq)
-                        st_bf16x8(sm, L::KP + (uint32_t)(DK + i) * 128 + ((((hh * 4 + gq) ^ ((DK + i) & 7))) << 4),
-                                  g32 + gq * 8);
+                for (int u = 0; u < 32; u += 4) {
+                    const int j = hh * 32 + u;
+                    float4 a;
+                    a.x = (j + 0 < i) ? bi * g32[u + 0] : 0.f;
+                    a.y = (j + 1 < i) ? bi * g32[u + 1] : 0.f;
+                    a.z = (j + 2 < i) ? bi * g32[u + 2] : 0.f;
+                    a.w = (j + 3 < i) ? bi * g32[u + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(fA + i * AS + j) = a;
                 }
+            }
+            asm volatile("bar.sync 1, 64;" ::: "memory");   // rows of A from both warps
+            invert_diag_blocks(fA, fT, tid);
+        } else if (warp < 4) {
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                float g32[32];
+                ptx::tmem_ld32(tl + COL_GRAM + hh * 32, g32);
+                ptx::tmem_wait_ld();
+                const int i = tid - 64;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) g32[u] = (hh * 32 + u <= i) ? g32[u] : 0.f;
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq)
+                    st_bf16x8(sm, L::KP + sw128_chunk(DK + i, hh * 4 + gq), g32 + gq * 8);
             }
         } else if (warp < 6) {
             // X rows (TMEM lanes 0-63) -> Z = V - X -> Z^T
-            int lf = 0;
-            if (!ptx::mbar_wait_bounded(bar_v0 + 8u * (uint32_t)buf, ph_v[buf], WAIT_LIMIT_NS)) lf = 1;
-            if (lf) *fail_flag = 1;
-            const int j = (warp - 4) * 32 + lane;
-            const uint8_t *vin = sm + L::VIN + buf * C * DVT * 2;
+            if (!ptx::mbar_wait_bounded(bar_v, ph_v, WAIT_LIMIT_NS)) *fail_flag = 1;
+            const int j = quad * 32 + lane;
+            const uint8_t *vin = sm + L::VIN;
 #pragma unroll 1
             for (int cc = 0; cc < DVT / 16; ++cc) {
                 float x16[16], v16[16];
@@ -454,10 +506,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int u = 0; u < 16; ++u) st_bf16(sm, L::ZT + sw128(cc * 16 + u, j, DVT), v16[u] - x16[u]);
             }
+        } else {
+            // blocks (0,1) and (2,3) of T are read by the merge products as zeros
+            const int t = tid - 192;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int e = t + 64 * m, blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                fT[(32 * blk + r) * AS + 32 * blk + 16 + c] = 0.f;
+            }
         }
-        ph_v[buf] ^= 1u;
+        ph_v ^= 1u;
         __syncthreads();
-        invert_unit_lower64(fA, fT, fM, tid);
+        if (tid == 0 && ci + 1 < nck) issue_v(ci + 1);   // V tile consumed
+        invert_merge_blocks(fA, fT, fM, warp, lane);
         {   // Tb^T[j][l] = T[l][j] beta_j   (l >= j)
             const int j = tid & 63, lq = tid >> 6;
             const float bj = fB[buf * C + j];
@@ -474,102 +535,83 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 4. Kt = Kbar^T Tb, Pt = Aqk Tb ; next chunk's inputs (scratch is free now)
+        // ---- 4. Kt = Kbar^T Tb (Kbar read MN-major), Pt = Aqk Tb ; next chunk's inputs
         if (tid == 0) {
             if (ci + 1 < nck) issue_inputs(ci + 1);
             ptx::tc_fence_after();
-            constexpr uint32_t ik = ptx::idesc_bf16_f32(128, 64);
+            constexpr uint32_t ikt = ptx::idesc_bf16_f32(128, 64, true, false);
+            constexpr uint32_t ipt = ptx::idesc_bf16_f32(128, 64);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + COL_KT, kdesc(sb + L::KP, s, DK + 64), kdesc(sb + L::TB, s, 64), ik, s > 0);
-            if (DK == 128) {
+                ptx::mma_bf16(tmem + COL_KT, ptx::desc_mnmajor_sw128(sb + L::KB + s * 2048, 64 * 128, 1024),
+                              kdesc(sb + L::TB, s, 64), ikt, s > 0);
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    ptx::mma_bf16(tmem + COL_PT, kdesc(sb + L::KP, s, DK + 64, 64), kdesc(sb + L::TB, s, 64), ik,
-                                  s > 0);
-            }
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + COL_PT, kdesc(sb + L::KP, s, DK + 64, DK - 64), kdesc(sb + L::TB, s, 64), ipt,
+                              s > 0);
             ptx::mma_commit(bar_mma);
         }
         if (!(ok = wait_all(bar_mma, ph_mma, *fail_flag))) break;
 
         // ---- 5. Kt, Pt -> bf16 A operands
-        if (warp < 4) {
+        if (warp < DK / 32) {
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 float k32[32];
                 ptx::tmem_ld32(tl + COL_KT + hh * 32, k32);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int gq = 0; gq < 4; ++gq)
-                    st_bf16x8(sm, L::KP + (uint32_t)tid * 128 + ((((hh * 4 + gq) ^ (tid & 7))) << 4), k32 + gq * 8);
+                for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::KP + sw128_chunk(srow, hh * 4 + gq), k32 + gq * 8);
             }
-        } else if (DK == 128 && warp >= 6) {
-            const int i = (warp - 6) * 32 + lane;
+        } else if (warp >= 6) {
+            const int i = (quad - 2) * 32 + lane;
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 float p32[32];
                 ptx::tmem_ld32(tl + COL_PT + hh * 32, p32);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int gq = 0; gq < 4; ++gq)
-                    st_bf16x8(sm, L::KP + (uint32_t)(DK + i) * 128 + ((((hh * 4 + gq) ^ ((DK + i) & 7))) << 4),
-                              p32 + gq * 8);
+                for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::KP + sw128_chunk(DK + i, hh * 4 + gq), p32 + gq * 8);
             }
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 6. dS = Kt Z ; O = Y + Pt Z
+        // ---- 6. dS = Kt Z ; O = Y + Pt Z (accumulated onto the Y rows of [X; Y])
         if (tid == 0) {
             ptx::tc_fence_after();
             constexpr uint32_t iz = ptx::idesc_bf16_f32(128, DVT);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
                 ptx::mma_bf16(tmem + COL_DS, kdesc(sb + L::KP, s, DK + 64), kdesc(sb + L::ZT, s, DVT), iz, s > 0);
-            if (DK == 128) {
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KP, s, DK + 64, 64), kdesc(sb + L::ZT, s, DVT), iz, 1);
-            }
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KP, s, DK + 64, DK - 64), kdesc(sb + L::ZT, s, DVT), iz, 1);
             ptx::mma_commit(bar_mma);
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
 
-        // ---- 7. S <- Diag(e^{G_last}) S + dS (and its bf16 copy for the next chunk); store O rows
-        if (warp < 4) {
-            const float dch = has_row ? fD[tid] : 0.f;
+        // ---- 7. S <- Diag(e^{G_last}) S + dS ; store O rows (TMEM lanes 64-127)
+        if (has_row) {
 #pragma unroll
-            for (int cc = 0; cc < DVT / 16; ++cc) {
+            for (int cc = 0; cc < CPT / 16; ++cc) {
                 float d16[16];
-                ptx::tmem_ld16(tl + COL_DS + cc * 16, d16);
+                ptx::tmem_ld16(tl + COL_DS + scol + cc * 16, d16);
                 ptx::tmem_wait_ld();
-                if (has_row) {
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
-                }
+                for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
             }
-            if (has_row && ci + 1 < nck) {
-#pragma unroll
-                for (int j = 0; j < DVT; ++j) st_bf16(sm, L::SB + sw128(j, tid, DVT), S[j]);
-            }
-        } else if (warp >= 6) {
-            const int i = (warp - 6) * 32 + lane;
+        }
+        if (quad >= 2) {
+            const int i = (quad - 2) * 32 + lane;
 #pragma unroll 1
-            for (int cc = 0; cc < DVT / 16; ++cc) {
+            for (int cc = 0; cc < CPT / 16; ++cc) {
                 float o16[16];
-                ptx::tmem_ld16(tl + COL_XY + cc * 16, o16);
-                if (DK == 64) {
-                    float p16[16];
-                    ptx::tmem_ld16(tl + COL_DS + cc * 16, p16);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) o16[u] += p16[u];
-                } else {
-                    ptx::tmem_wait_ld();
-                }
+                ptx::tmem_ld16(tl + COL_XY + scol + cc * 16, o16);
+                ptx::tmem_wait_ld();
                 if (i < Lc) {
-                    __nv_bfloat16 *dst = o + ((cs + i) * H + h) * DV + col_base + cc * 16;
+                    __nv_bfloat16 *dst = o + ((cs + i) * H + h) * DV + col_base + scol + cc * 16;
                     reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pack_bf16(o16[0], o16[1]), pack_bf16(o16[2], o16[3]),
                                                                    pack_bf16(o16[4], o16[5]), pack_bf16(o16[6], o16[7]));
                     reinterpret_cast<uint4 *>(dst)[1] =
@@ -585,8 +627,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     if (ok && final_state && has_row) {
 #pragma unroll
-        for (int j = 0; j < DVT; j += 4)
-            store4(final_state + st_off + (long long)tid * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
+        for (int j = 0; j < CPT; j += 4)
+            store4(final_state + st_off + (long long)srow * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -663,8 +705,6 @@ int launch_t(const void *q, const void *k, const void *v, const float *log_alpha
     return KDA_OK;
 }
 
-// Value-tile width: 64 columns when there are enough (sequence, head, tile) work
-// items to fill the GPU twice over, else 32 for more CTAs.
 inline int launch(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                   const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int B, int T,
                   int H, int dk, int dv, int num_seqs, void *workspace, cudaStream_t st, char *msg,
@@ -688,16 +728,22 @@ inline int launch(const void *q, const void *k, const void *v, const float *log_
         snprintf(msg, msg_len, "B*T=%lld exceeds the 2^31 token limit of the TMA coordinates", tokens);
         return KDA_ERR_UNSUPPORTED;
     }
-    const long long items64 = (long long)num_seqs * H * (dv / 64);
-    const bool wide = items64 >= 2 * 148;
+    // Value-tile width: the widest tile (fewest duplicated per-chunk operand
+    // builds) that still gives at least two CTAs per SM; else 32 columns.
+    const long long chains = (long long)num_seqs * H;
+    int dvt = 32;
+    for (int cand = dv; cand >= 32; cand /= 2)
+        if (chains * (dv / cand) >= 2 * 148) { dvt = cand; break; }
 #define KDA_TC(DKv, DVTv)                                                                                   \
     return launch_t<DKv, DVTv>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T, \
                                H, dv, num_seqs, st, msg, msg_len)
     if (dk == 128) {
-        if (wide) KDA_TC(128, 64);
+        if (dvt == 128) KDA_TC(128, 128);
+        if (dvt == 64) KDA_TC(128, 64);
         KDA_TC(128, 32);
     }
-    if (wide) KDA_TC(64, 64);
+    if (dvt == 128) KDA_TC(64, 128);
+    if (dvt == 64) KDA_TC(64, 64);
     KDA_TC(64, 32);
 #undef KDA_TC
 }

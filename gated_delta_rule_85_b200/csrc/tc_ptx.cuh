@@ -145,11 +145,28 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t smem_addr) {
     return d;
 }
 
-// Instruction descriptor: kind::f16 with bf16 A and B (both K-major), fp32 D.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+// Descriptor of an MN-major bf16 operand in the 128-byte swizzle layout: each
+// 128-byte row holds 64 consecutive M (or N) elements of one K index, 8 K rows
+// form a 1024-byte swizzle atom, K atoms are `sbo` bytes apart and 64-element MN
+// blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor: kind::f16 with bf16 A and B, fp32 D; A and B K-major
+// unless a_mn / b_mn select MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false, bool b_mn = false) {
     return (1u << 4)                  // D format: f32
            | (1u << 7)                // A format: bf16
            | (1u << 10)               // B format: bf16
+           | ((a_mn ? 1u : 0u) << 15)
+           | ((b_mn ? 1u : 0u) << 16)
            | ((uint32_t)(N >> 3) << 17)
            | ((uint32_t)(M >> 4) << 24);
 }

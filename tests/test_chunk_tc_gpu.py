@@ -39,9 +39,15 @@ def test_head_dims(dk, dv):
     _check(PrefillShape(B=2, T=200, H=2, dk=dk, dv=dv, dtype=BF16), seed=dk * 3 + dv)
 
 
-def test_many_chunks_wide_tiles():
-    """Enough (sequence, head) pairs that the 64-column value tiles are used."""
-    _check(PrefillShape(B=4, T=300, H=40, dk=128, dv=128, dtype=BF16), seed=11)
+@pytest.mark.parametrize("B,H,dk,dv", [
+    (4, 40, 128, 128),    # 160 (sequence, head) chains -> 64-column value tiles
+    (4, 80, 128, 128),    # 320 chains -> 128-column value tiles
+    (4, 80, 64, 128),
+    (4, 80, 64, 64),      # dv = 64 -> one 64-column tile
+])
+def test_value_tile_widths(B, H, dk, dv):
+    """The launcher picks the value-tile width from the number of chains; cover each."""
+    _check(PrefillShape(B=B, T=150, H=H, dk=dk, dv=dv, dtype=BF16), seed=11 + H + dk)
 
 
 def test_zero_initial_state_and_no_final_state():
