@@ -203,6 +203,43 @@ def run_prefill(args, world, rank, dev):
                 h2d=h2d, d2h=d2h, e2e_steps=e2e_steps)
 
 
+def run_prefill_varlen(args, world, rank, dev):
+    """The 1,048,576-token packed (varlen) prefill: 22 sequences x 32 heads."""
+    import torch
+
+    import gated_delta_rule_85_b200 as kda
+    from gated_delta_rule_85_b200.workloads import prefill_inputs, varlen_1m_shape
+
+    shape = varlen_1m_shape()
+    d = prefill_inputs(shape, seed=rank, device=dev)
+    o = torch.empty((1, shape.T, shape.H, shape.dv), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((shape.num_seqs, shape.H, shape.dk, shape.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], d["cu_seqlens"],
+                          o=o, final_state=fs)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    reps = 3
+    _barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    token_heads = shape.T * shape.H
+    alg_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * shape.num_seqs * shape.H * STATE_BYTES
+    del d, o, fs
+    return dict(ms=ms, tokens=shape.T, alg_bytes=alg_bytes, alg_flops=token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD,
+                seqs=shape.num_seqs, launches=reps)
+
+
 def run_decode(args, world, rank, dev):
     """1024 consecutive decode steps of 256 sequences, captured in one CUDA graph."""
     import torch
@@ -315,6 +352,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the 1M-token packed prefill line")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -339,6 +377,7 @@ def main(argv=None):
 
     pre = run_prefill(args, world, rank, dev)
     dec = None if args.no_decode else run_decode(args, world, rank, dev)
+    vl = None if args.no_varlen else run_prefill_varlen(args, world, rank, dev)
 
     hbm_gbs, bf16_tflops, peak_src = _peaks()
     ms_step = pre["total_ms"] / args.steps
@@ -380,6 +419,18 @@ def main(argv=None):
             "clocks": dec["clocks"],
         }
         line["gpu_launches"] += dec["launches"]
+    if vl is not None:
+        vgbs = vl["alg_bytes"] / (vl["ms"] * 1e-3) / 1e9
+        vtf = vl["alg_flops"] / (vl["ms"] * 1e-3) / 1e12
+        line["prefill_varlen_1m"] = {
+            "metric": "KDA packed (varlen) prefill tokens/s (1,048,576 tokens in 22 sequences, H=32, d=128)",
+            "value": world * vl["tokens"] / (vl["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": vl["ms"],
+            "roofline": {"kernel": "chunk_tc_kernel", "bound": "hbm", "achieved": vgbs, "peak": hbm_gbs,
+                         "unit": "GB/s", "frac": vgbs / hbm_gbs, "traffic": None,
+                         "algorithmic_bytes": vl["alg_bytes"],
+                         "tensor": {"achieved_tflops": vtf, "peak_tflops": bf16_tflops, "frac": vtf / bf16_tflops}},
+        }
+        line["gpu_launches"] += vl["launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(heads=32)
     if rank == 0:

@@ -166,10 +166,24 @@ __device__ __forceinline__ void warp_store16x8(float *Z, int sz, const float (&d
     *reinterpret_cast<float2 *>(Z + (g + 8) * sz + 2 * t) = make_float2(sign * d[2], sign * d[3]);
 }
 
+// The same 16 x 8 tile of T (rows r0.., columns c0..) as Tb^T entries:
+// Tb^T[c][r] = sign * T[r][c] * beta_c, bf16, into the swizzled operand tile.
+__device__ __forceinline__ void warp_store16x8_tbt(uint8_t *tb, int r0, int c0, const float (&d)[4], float sign,
+                                                  const float *beta, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const int ca = c0 + 2 * t, cb = ca + 1;
+    const float ba = sign * beta[ca], bb = sign * beta[cb];
+    st_bf16(tb, sw128(ca, r0 + g, 64), d[0] * ba);
+    st_bf16(tb, sw128(cb, r0 + g, 64), d[1] * bb);
+    st_bf16(tb, sw128(ca, r0 + g + 8, 64), d[2] * ba);
+    st_bf16(tb, sw128(cb, r0 + g + 8, 64), d[3] * bb);
+}
+
 // Diagonal 16 x 16 blocks of T = (I + A)^{-1} (A strictly lower, fp32, row stride
 // AS) by forward substitution: 64 threads, one block column each, zeros above the
 // diagonal included.
-__device__ __forceinline__ void invert_diag_blocks(const float *A, float *Tm, int t64) {
+__device__ __forceinline__ void invert_diag_blocks(const float *A, float *Tm, uint8_t *tb, const float *beta,
+                                                   int t64) {
     const int o = 16 * (t64 >> 4), l = t64 & 15;
     float x[16];
 #pragma unroll
@@ -189,6 +203,13 @@ __device__ __forceinline__ void invert_diag_blocks(const float *A, float *Tm, in
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) Tm[(o + i) * AS + o + l] = x[i];
+    // Tb^T[o+l][o+i] = T[o+i][o+l] beta_{o+l}: one 32-byte row segment of the bf16 operand
+    const float bl = beta[o + l];
+    float t16[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t16[i] = x[i] * bl;
+    st_bf16x8(tb, sw128_chunk(o + l, o / 8), t16);
+    st_bf16x8(tb, sw128_chunk(o + l, o / 8 + 1), t16 + 8);
 }
 
 // The rest of T once its diagonal blocks are in place and blocks (0,1) and (2,3)
@@ -196,7 +217,8 @@ __device__ __forceinline__ void invert_diag_blocks(const float *A, float *Tm, in
 // [L11^-1 0; -L22^-1 L21 L11^-1  L22^-1] at 32 (two pairs of 16-blocks) and at 64,
 // each block product one 16 x 8 tile per warp on the tensor cores (tf32 inputs,
 // fp32 accumulation).  All 256 threads take part.
-__device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, float *M, int warp, int lane) {
+__device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, float *M, uint8_t *tb,
+                                                    const float *beta, int warp, int lane) {
     if (warp < 4) {   // M_p = A[2p+1][2p] T[2p][2p]
         const int p = warp >> 1, nt = warp & 1, ro = 32 * p + 16, co = 32 * p;
         float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -209,6 +231,7 @@ __device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, f
         float d[4] = {0.f, 0.f, 0.f, 0.f};
         warp_mm16x8_tf32<2>(d, Tm + ro * AS + ro, AS, M + p * 16 * 36 + 8 * nt, 36, lane);
         warp_store16x8(Tm + ro * AS + co + 8 * nt, AS, d, -1.f, lane);
+        warp_store16x8_tbt(tb, ro, co + 8 * nt, d, -1.f, beta, lane);
     }
     __syncthreads();
     const int mt = warp >> 2, nt = warp & 3;
@@ -221,9 +244,8 @@ __device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, f
     {   // T[hi][lo] = -T[hi][hi] M
         float d[4] = {0.f, 0.f, 0.f, 0.f};
         warp_mm16x8_tf32<4>(d, Tm + (32 + 16 * mt) * AS + 32, AS, M + 8 * nt, 36, lane);
-        warp_store16x8(Tm + (32 + 16 * mt) * AS + 8 * nt, AS, d, -1.f, lane);
+        warp_store16x8_tbt(tb, 32 + 16 * mt, 8 * nt, d, -1.f, beta, lane);
     }
-    __syncthreads();
 }
 
 // Every thread waits for the next completion of an mbarrier; all agree on the
@@ -400,8 +422,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             float ef[4], eb[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                ef[e] = expf(pre[e] - tot[e]);
-                eb[e] = expf(tot[e] - pre[e] - sgv[e]);
+                ef[e] = exp2_fast((pre[e] - tot[e]) * LOG2E);
+                eb[e] = exp2_fast((tot[e] - pre[e] - sgv[e]) * LOG2E);
             }
 #pragma unroll
             for (int u = 0; u < SEGLEN; ++u) {
@@ -472,7 +494,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             asm volatile("bar.sync 1, 64;" ::: "memory");   // rows of A from both warps
-            invert_diag_blocks(fA, fT, tid);
+            invert_diag_blocks(fA, fT, sm + L::TB, fB + buf * C, tid);
         } else if (warp < 4) {
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
@@ -507,30 +529,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int u = 0; u < 16; ++u) st_bf16(sm, L::ZT + sw128(cc * 16 + u, j, DVT), v16[u] - x16[u]);
             }
         } else {
-            // blocks (0,1) and (2,3) of T are read by the merge products as zeros
+            // blocks (0,1) and (2,3) of T are read by the merge products as zeros;
+            // Tb^T is zero below its block diagonal (six 16 x 16 blocks, 16-byte stores)
             const int t = tid - 192;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int e = t + 64 * m, blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
                 fT[(32 * blk + r) * AS + 32 * blk + 16 + c] = 0.f;
             }
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int m = 0; m < 3; ++m) {
+                const int e = t + 64 * m;                  // 0..191: 6 blocks x 16 rows x 2 groups
+                const int blk = e >> 5, r = (e >> 1) & 15, gh = e & 1;
+                const int bi = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);   // row block of Tb^T
+                const int bj = blk < 3 ? 0 : (blk < 5 ? 1 : 2);               // column block (< bi)
+                *reinterpret_cast<uint4 *>(sm + L::TB + sw128_chunk(16 * bi + r, 2 * bj + gh)) = z;
+            }
         }
         ph_v ^= 1u;
         __syncthreads();
         if (tid == 0 && ci + 1 < nck) issue_v(ci + 1);   // V tile consumed
-        invert_merge_blocks(fA, fT, fM, warp, lane);
-        {   // Tb^T[j][l] = T[l][j] beta_j   (l >= j)
-            const int j = tid & 63, lq = tid >> 6;
-            const float bj = fB[buf * C + j];
-            float t16[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int l = lq * 16 + u;
-                t16[u] = (l >= j) ? fT[l * AS + j] * bj : 0.f;
-            }
-            st_bf16x8(sm, L::TB + sw128_chunk(j, 2 * lq), t16);
-            st_bf16x8(sm, L::TB + sw128_chunk(j, 2 * lq + 1), t16 + 8);
-        }
+        invert_merge_blocks(fA, fT, fM, sm + L::TB, fB + buf * C, warp, lane);
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
