@@ -44,8 +44,8 @@ constexpr int NT = 256;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;   // 1 s: far beyond any legitimate latency
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM column map (fp32 accumulators, lane = row)
-constexpr uint32_t COL_XY = 0;      // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O
-constexpr uint32_t COL_GRAM = 128;  // [128 x 64]  rows 0-63 Kp Kbar^T, rows 64-127 Qp Kbar^T
+constexpr uint32_t COL_GRAM = 0;    // [128 x 64]  rows 0-63 Kp Kbar^T, rows 64-127 Qp Kbar^T
+constexpr uint32_t COL_XY = 64;     // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O (same MMA as the Gram)
 constexpr uint32_t COL_KT = 192;    // [128 x 64]  Kt (lanes 0..dk-1)
 constexpr uint32_t COL_PT = 256;    // [128 x 64]  Pt (lanes 64-127)
 constexpr uint32_t COL_DS = 320;    // [128 x DVT] Kt Z (lanes 0..dk-1)
@@ -56,11 +56,12 @@ struct Layout {
     static constexpr int KA = DK / 64;                       // 64-element K atoms along dk
     // bf16 MMA operands, 128-byte swizzled, 1024-byte aligned
     static constexpr int KQ = 0;                             // [KA][128][128 B] Kp (0-63), Qp (64-127)
-    static constexpr int KB = KQ + KA * 128 * 128;           // [KA][64][128 B]  Kbar (rows = tokens)
-    static constexpr int KP = KB + KA * 64 * 128;            // [DK+64][128 B]   Kt (0..DK-1), Aqk -> Pt (DK..)
+    static constexpr int KSR = 64 + DVT;                     // rows of the combined B operand
+    static constexpr int KS = KQ + KA * 128 * 128;           // [KA][64+DVT][128 B] rows 0-63 Kbar (tokens),
+                                                             //   rows 64.. (e^{G_last} S)^T (value columns)
+    static constexpr int KP = KS + KA * KSR * 128;           // [DK+64][128 B]   Kt (0..DK-1), Aqk -> Pt (DK..)
     static constexpr int TB = KP + (DK + 64) * 128;          // [64][128 B]      Tb^T
-    static constexpr int SB = TB + 64 * 128;                 // [KA][DVT][128 B] (e^{G_last} S)^T
-    static constexpr int ZT = SB + KA * DVT * 128;           // [DVT][128 B]     Z^T
+    static constexpr int ZT = TB + 64 * 128;                 // [DVT][128 B]     Z^T
     // dense TMA input tiles; the fp32 scratch of the UT transform aliases them
     static constexpr int QIN = ZT + DVT * 128;               // bf16 [64][DK]
     static constexpr int KIN = QIN + 64 * DK * 2;            // bf16 [64][DK]
@@ -78,8 +79,8 @@ struct Layout {
     static constexpr int MISC = FSEG + NSEG * DK * 4;        // mbarriers, TMEM base, flags
     static constexpr int BYTES = MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024 B
-    static_assert(KQ % 1024 == 0 && KB % 1024 == 0 && KP % 1024 == 0 && TB % 1024 == 0 && SB % 1024 == 0 &&
-                      ZT % 1024 == 0 && QIN % 1024 == 0 && VIN % 128 == 0,
+    static_assert(KQ % 1024 == 0 && KS % 1024 == 0 && KP % 1024 == 0 && TB % 1024 == 0 && ZT % 1024 == 0 &&
+                      QIN % 1024 == 0 && VIN % 128 == 0,
                   "tile alignment");
     static_assert(ALLOC <= 232448, "shared memory budget");
 };
@@ -445,29 +446,26 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int i = i0 + u;
                 float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (i < Lc) k4 = ld_bf16x4(kin + (i * DK + c0) * 2);
-                st_bf16x4(sm, L::KB + sw128(i, c0, 64), k4.x * eb[0], k4.y * eb[1], k4.z * eb[2], k4.w * eb[3]);
+                st_bf16x4(sm, L::KS + sw128(i, c0, L::KSR), k4.x * eb[0], k4.y * eb[1], k4.z * eb[2], k4.w * eb[3]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) eb[e] *= al[u][e];
             }
         }
         if (has_row) {
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::SB + sw128(scol + j, srow, DVT), dch * S[j]);
+            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::KS + sw128(64 + scol + j, srow, L::KSR), dch * S[j]);
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 2. Gram [Kp; Qp] Kbar^T and [X; Y] = [Kp; Qp] (e^{G_last} S)
+        // ---- 2. [Gram | X; Y] = [Kp; Qp] [Kbar; e^{G_last} S^T]^T in one N = 64 + DVT MMA chain
         if (tid == 0) {
             ptx::tc_fence_after();
-            constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64), ix = ptx::idesc_bf16_f32(128, DVT);
+            constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64 + DVT);
 #pragma unroll
             for (int s = 0; s < DK / 16; ++s)
-                ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KB, s, 64), ig, s > 0);
-#pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::SB, s, DVT), ix, s > 0);
+                ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KS, s, L::KSR), ig, s > 0);
             ptx::mma_commit(bar_mma);
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
@@ -563,7 +561,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t ipt = ptx::idesc_bf16_f32(128, 64);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + COL_KT, ptx::desc_mnmajor_sw128(sb + L::KB + s * 2048, 64 * 128, 1024),
+                ptx::mma_bf16(tmem + COL_KT, ptx::desc_mnmajor_sw128(sb + L::KS + s * 2048, L::KSR * 128, 1024),
                               kdesc(sb + L::TB, s, 64), ikt, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
