@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "chunk_forward", "chunk_forward_simt", "recurrent_step", "workspace_size", "device_status",
     "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
-    "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE",
+    "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "ALGOS",
 ]
 
 KDA_BF16 = 0
@@ -30,6 +30,8 @@ KDA_F32 = 1
 CHUNK = 64
 DEV_WAIT_TIMEOUT = 0x1
 DEV_DECAY_RANGE = 0x2
+# tensor-core prefill schedules (KDA_ALGO_* in include/kda.h)
+ALGOS = {"auto": 0, "fused": 1, "two_pass": 2}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
@@ -62,6 +64,10 @@ def load_library():
     lib.kda_chunk_forward_simt.restype = ci
     lib.kda_chunk_forward_workspace_size.argtypes = [ci] * 8
     lib.kda_chunk_forward_workspace_size.restype = sz
+    lib.kda_chunk_forward_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, ip] + [ci] * 9 + [vp, sz, vp]
+    lib.kda_chunk_forward_ex.restype = ci
+    lib.kda_chunk_forward_workspace_size_ex.argtypes = [ci] * 9
+    lib.kda_chunk_forward_workspace_size_ex.restype = sz
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ci] * 5 + [vp]
     lib.kda_recurrent_step.restype = ci
     lib.kda_last_error.argtypes = []
@@ -107,8 +113,15 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous in the documented layouts")
 
 
-def workspace_size(B, T, H, dk, dv, num_seqs, dtype=KDA_BF16) -> int:
-    return int(load_library().kda_chunk_forward_workspace_size(B, T, H, dk, dv, num_seqs, dtype, CHUNK))
+def _algo_code(algo: str) -> int:
+    if algo not in ALGOS:
+        raise ValueError(f"algo must be one of {sorted(ALGOS)}, got {algo!r}")
+    return ALGOS[algo]
+
+
+def workspace_size(B, T, H, dk, dv, num_seqs, dtype=KDA_BF16, algo="auto") -> int:
+    return int(load_library().kda_chunk_forward_workspace_size_ex(B, T, H, dk, dv, num_seqs, dtype, CHUNK,
+                                                                  _algo_code(algo)))
 
 
 def _prefill_args(q, k, v, log_alpha, beta, init_state, cu_seqlens):
@@ -133,21 +146,23 @@ def _to_device(ts, device):
 
 
 def chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, o=None,
-                  final_state=True, workspace=None, simt=False):
-    """Chunked KDA prefill (64-token chunks) through kda_chunk_forward.
+                  final_state=True, workspace=None, simt=False, algo="auto"):
+    """Chunked KDA prefill (64-token chunks) through kda_chunk_forward_ex.
 
     Tensors are in the include/kda.h layouts.  `final_state` may be True
     (allocate and return), False (skip) or a preallocated float32 tensor.
-    With `simt=True` the fp32 CUDA-core path (kda_chunk_forward_simt) runs
-    instead of the tensor-core path.  Host (CPU) inputs are copied to the
-    current CUDA device and the results copied back, all inside this call.
+    `algo` picks the tensor-core schedule ("auto", "fused", "two_pass"); the
+    workspace it needs is allocated here unless `workspace` (uint8, CUDA) is
+    given.  With `simt=True` the fp32 CUDA-core path (kda_chunk_forward_simt)
+    runs instead.  Host (CPU) inputs are copied to the current CUDA device and
+    the results copied back, all inside this call.
     Returns (o, final_state or None).
     """
     if not q.is_cuda:
         dev = torch.device("cuda", torch.cuda.current_device())
         args = _to_device([q, k, v, log_alpha, beta, init_state, cu_seqlens], dev)
         fs_dev = final_state if isinstance(final_state, bool) else True
-        o_d, s_d = chunk_forward(*args, final_state=fs_dev, workspace=workspace, simt=simt)
+        o_d, s_d = chunk_forward(*args, final_state=fs_dev, workspace=workspace, simt=simt, algo=algo)
         o_h = o if o is not None else torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True)
         o_h.copy_(o_d, non_blocking=True)
         s_h = None
@@ -168,18 +183,19 @@ def chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *,
         final_state = None
     _need_cuda(o, final_state)
     dt = _dtype_code(q)
+    ac = _algo_code(algo)
     st = _stream(q.device)
     if simt:
         rc = lib.kda_chunk_forward_simt(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(o),
                                         _p(final_state), _p(cu_seqlens), B, T, H, dk, dv, N, dt, CHUNK, st)
     else:
-        need = int(lib.kda_chunk_forward_workspace_size(B, T, H, dk, dv, N, dt, CHUNK))
+        need = int(lib.kda_chunk_forward_workspace_size_ex(B, T, H, dk, dv, N, dt, CHUNK, ac))
         if need and workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-        rc = lib.kda_chunk_forward(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(o),
-                                   _p(final_state), _p(cu_seqlens), B, T, H, dk, dv, N, dt, CHUNK,
-                                   _p(workspace), ws_bytes, st)
+        rc = lib.kda_chunk_forward_ex(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(o),
+                                      _p(final_state), _p(cu_seqlens), B, T, H, dk, dv, N, dt, CHUNK, ac,
+                                      _p(workspace), ws_bytes, st)
     _check(rc)
     return o, final_state
 

@@ -1,0 +1,615 @@
+// KDA chunked prefill in two passes, for inputs with few (sequence, head) chains.
+//
+// Same chunk algebra as chunk_tc_kernel (kda_chunk_tc.cuh; "Kimi Linear、独自の土俵で
+// Full Attentionを上回る" (remio.ai), § "Kimi Linearがより賢いRecurrent Memoryを使う方法":
+// chunkwise algorithm on a diagonal-plus-low-rank transition).  Everything of a
+// chunk that does not involve the state -- the decay factors, the Gram matrix, the
+// UT transform T = (I + Diag(beta) Akk)^{-1} and the products Kt = Kbar^T Tb,
+// Pt = Aqk Tb -- depends on that chunk's inputs alone.  The fused kernel builds
+// it inside the serial walk over chunks, once per value-column tile.  Here
+//
+//   pass 1, chunk_intra_kernel: one CTA per (chunk, head), all chunks at once,
+//       writes the bf16 operands [Kp; Qp], [Kt; Pt] and e^{G_last} of the chunk to
+//       a workspace record laid out byte for byte like the shared-memory tiles the
+//       second pass feeds to the tensor cores;
+//   pass 2, chunk_inter_kernel: one CTA per (value tile, head, sequence) walks
+//       the chunks in order with only the state-dependent work left on the
+//       serial path: X; Y = [Kp; Qp] (e^{G_last} S), Z = V - X,
+//       S <- Diag(e^{G_last}) S + Kt Z, O = Y + Pt Z.
+//
+// Chunk slots: chunk c of sequence n (tokens [t0, t1)) is record
+// n + floor(t0 / 64) + c, unique and below ceil(total tokens / 64) + N for any
+// token ranges; a dense batch uses t0 = n T.
+#pragma once
+
+#include "kda_chunk_tc.cuh"
+
+namespace kda {
+namespace tc {
+
+// Workspace record of one (chunk slot, head).
+template <int DK>
+struct Rec {
+    static constexpr int KA = DK / 64;
+    static constexpr int KQ = 0;                          // [KA][128][128 B]  Kp (rows 0-63), Qp (rows 64-127)
+    static constexpr int KP = KA * 128 * 128;             // [DK+64][128 B]    Kt (rows 0..DK-1), Pt (DK..DK+63)
+    static constexpr int DCH = KP + (DK + 64) * 128;      // fp32 [DK]         e^{G_last}
+    static constexpr int BYTES = (DCH + DK * 4 + 1023) / 1024 * 1024;
+};
+
+inline long long chunk_slots(long long tokens, int num_seqs) { return (tokens + C - 1) / C + num_seqs; }
+
+inline size_t two_pass_workspace_bytes(long long tokens, int H, int dk, int num_seqs) {
+    if (tokens <= 0) return 0;
+    const size_t rec = dk == 64 ? (size_t)Rec<64>::BYTES : (size_t)Rec<128>::BYTES;
+    return (size_t)chunk_slots(tokens, num_seqs) * (size_t)H * rec;
+}
+
+// First token of sequence n (clamped like seq_span).
+__device__ __forceinline__ long long seq_begin(const int32_t *cu_seqlens, int T, int n) {
+    return cu_seqlens ? (long long)min(max(cu_seqlens[n], 0), T) : (long long)n * T;
+}
+
+// ------------------------------------------------------------------ pass 1
+
+template <int DK>
+struct IntraLayout {
+    static constexpr int KA = DK / 64;
+    static constexpr int KQ_BYTES = KA * 128 * 128;
+    static constexpr int SCR_BYTES = 2 * 64 * AS * 4 + 32 * 36 * 4;
+    static constexpr int R1 = ((KQ_BYTES > SCR_BYTES ? KQ_BYTES : SCR_BYTES) + 1023) / 1024 * 1024;
+    static constexpr int KQ = 0;                          // [KA][128][128 B] Kp, Qp; then the fp32 scratch:
+    static constexpr int FA = 0;                          //   fp32 [64][AS] Diag(beta) Akk
+    static constexpr int FT = FA + 64 * AS * 4;           //   fp32 [64][AS] T
+    static constexpr int FM = FT + 64 * AS * 4;           //   fp32 [32][36] block products
+    static constexpr int KB = R1;                         // [KA][64][128 B]  Kbar
+    static constexpr int TB = KB + KA * 64 * 128;         // [64][128 B]      Tb^T
+    static constexpr int AQ = TB + 64 * 128;              // [64][128 B]      masked Aqk (rows 64-127 of [Tb^T; Aqk])
+    static constexpr int FB = AQ + 64 * 128;              // fp32 [64]        beta
+    static constexpr int NSEG = NT / (DK / 4);
+    static constexpr int FSEG = FB + 64 * 4;              // fp32 [NSEG][DK]  segment sums of log_alpha
+    static constexpr int MISC = FSEG + NSEG * DK * 4;     // mbarrier, TMEM base
+    static constexpr int BYTES = MISC + 64;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(KB % 1024 == 0 && TB % 1024 == 0 && AQ % 1024 == 0, "tile alignment");
+    static_assert(2 * (ALLOC + 1024) <= 233472, "two CTAs per SM");
+};
+
+constexpr uint32_t INTRA_TMEM_COLS = 256;
+constexpr uint32_t ICOL_GRAM = 0;     // [128 x 64] rows 0-63 Kp Kbar^T, rows 64-127 Qp Kbar^T
+constexpr uint32_t ICOL_KT = 64;      // [128 x 64] Kt (lanes 0..dk-1)
+constexpr uint32_t ICOL_PT = 128;     // [128 x 64] Pt (lanes 64-127)
+
+__device__ __forceinline__ float4 bf16x4_to_float4(uint2 r) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ void st_global_bf16x8(uint8_t *p, const float *x) {
+    *reinterpret_cast<uint4 *>(p) =
+        make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+}
+
+template <int DK>
+__global__ void __launch_bounds__(NT, 2)
+chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                   const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, uint8_t *__restrict__ ws) {
+    using L = IntraLayout<DK>;
+    using R = Rec<DK>;
+    constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG;
+    constexpr float LOG2E = 1.4426950408889634f;
+    const int slot = blockIdx.x, h = blockIdx.y;
+
+    // the sequence owning this slot: the last n whose first slot n + floor(t0_n / 64) is <= slot
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (mid + seq_begin(cu_seqlens, T, mid) / C <= slot) lo = mid;
+        else hi = mid - 1;
+    }
+    long long t0, t1;
+    seq_span(cu_seqlens, T, lo, t0, t1);
+    const long long cs = t0 + (long long)(slot - (lo + t0 / C)) * C;
+    if (cs < t0 || cs >= t1) return;   // slot without a chunk (the whole CTA leaves)
+    const int Lc = (int)min((long long)C, t1 - cs);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = ptx::smem_u32(sm);
+    float *fA = reinterpret_cast<float *>(sm + L::FA);
+    float *fT = reinterpret_cast<float *>(sm + L::FT);
+    float *fM = reinterpret_cast<float *>(sm + L::FM);
+    float *fB = reinterpret_cast<float *>(sm + L::FB);
+    float *fSeg = reinterpret_cast<float *>(sm + L::FSEG);
+    const uint32_t bar_mma = sb + L::MISC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 8);
+    uint8_t *rec = ws + ((size_t)slot * H + h) * R::BYTES;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTRA_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (tid == 0) {
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+    }
+    if (tid < C) fB[tid] = tid < Lc ? beta[(cs + tid) * H + h] : 0.f;
+
+    // ---- 1. decay factors -> Kp, Qp (written to the record too), Kbar, e^{G_last}
+    {
+        const int cg = tid % NCG, seg = tid / NCG, c0 = 4 * cg, i0 = seg * SEGLEN;
+        float al[SEGLEN][4];
+        uint2 qv[SEGLEN], kv[SEGLEN];
+        float4 sg = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < SEGLEN; ++u) {
+            float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            qv[u] = make_uint2(0u, 0u);
+            kv[u] = make_uint2(0u, 0u);
+            if (i0 + u < Lc) {
+                const long long off = ((cs + i0 + u) * H + h) * DK + c0;
+                g4 = __ldcs(reinterpret_cast<const float4 *>(log_alpha + off));
+                qv[u] = __ldcs(reinterpret_cast<const uint2 *>(q + off));
+                kv[u] = __ldcs(reinterpret_cast<const uint2 *>(k + off));
+            }
+            sg.x += g4.x; sg.y += g4.y; sg.z += g4.z; sg.w += g4.w;
+            al[u][0] = g4.x; al[u][1] = g4.y; al[u][2] = g4.z; al[u][3] = g4.w;
+        }
+        *reinterpret_cast<float4 *>(fSeg + seg * DK + c0) = sg;
+        __syncthreads();
+        float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int s2 = 0; s2 < NSEG; ++s2) {
+            const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
+            const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (s2 < seg) pre[e] += xv[e];
+                tot[e] += xv[e];
+            }
+        }
+        if (seg == 0) {
+            if (tot[0] < -80.f || tot[1] < -80.f || tot[2] < -80.f || tot[3] < -80.f) flag_status(KDA_DEV_DECAY_RANGE);
+            *reinterpret_cast<float4 *>(rec + R::DCH + c0 * 4) =
+                make_float4(expf(tot[0]), expf(tot[1]), expf(tot[2]), expf(tot[3]));
+        }
+#pragma unroll
+        for (int u = 0; u < SEGLEN; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) al[u][e] = exp2_fast(al[u][e] * LOG2E);
+        const float sgv[4] = {sg.x, sg.y, sg.z, sg.w};
+        float ef[4], eb[4];   // e^{G_i - G_last} (>= 1), e^{G_last - G_i} (<= 1)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            ef[e] = exp2_fast((pre[e] - tot[e]) * LOG2E);
+            eb[e] = exp2_fast((tot[e] - pre[e] - sgv[e]) * LOG2E);
+        }
+#pragma unroll
+        for (int u = 0; u < SEGLEN; ++u) {
+            const int i = i0 + u;
+            const float4 q4 = bf16x4_to_float4(qv[u]);
+            const float4 k4 = bf16x4_to_float4(kv[u]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ef[e] *= al[u][e];
+            st_bf16x4(sm, L::KQ + sw128(i, c0, 128), k4.x * ef[0], k4.y * ef[1], k4.z * ef[2], k4.w * ef[3]);
+            st_bf16x4(sm, L::KQ + sw128(64 + i, c0, 128), q4.x * ef[0], q4.y * ef[1], q4.z * ef[2], q4.w * ef[3]);
+        }
+#pragma unroll
+        for (int u = SEGLEN - 1; u >= 0; --u) {
+            const int i = i0 + u;
+            const float4 k4 = bf16x4_to_float4(kv[u]);
+            st_bf16x4(sm, L::KB + sw128(i, c0, 64), k4.x * eb[0], k4.y * eb[1], k4.z * eb[2], k4.w * eb[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) eb[e] *= al[u][e];
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t ph_mma = 0;
+
+    // ---- 2. Gram = [Kp; Qp] Kbar^T; the Kp/Qp image goes to the record meanwhile
+    if (tid == 0) {
+        ptx::bulk_store(rec + R::KQ, sb + L::KQ, (uint32_t)L::KQ_BYTES);
+        ptx::bulk_commit();
+        constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64);
+#pragma unroll
+        for (int s = 0; s < DK / 16; ++s)
+            ptx::mma_bf16(tmem + ICOL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KB, s, 64), ig, s > 0);
+        ptx::mma_commit(bar_mma);
+        ptx::bulk_wait_read_all();   // the fp32 scratch below overwrites the Kp/Qp tile
+    }
+    bool ok = wait_all(bar_mma, ph_mma);
+
+    if (ok) {
+        // ---- 3. Diag(beta) Akk -> diagonal blocks of T (warps 0-1); masked Aqk (warps 2-3);
+        //         zero blocks of T and Tb^T (warps 6-7)
+        if (warp < 2) {
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                float g32[32];
+                ptx::tmem_ld32(tl + ICOL_GRAM + hh * 32, g32);
+                ptx::tmem_wait_ld();
+                const int i = tid;
+                const float bi = fB[i];
+#pragma unroll
+                for (int u = 0; u < 32; u += 4) {
+                    const int j = hh * 32 + u;
+                    float4 a;
+                    a.x = (j + 0 < i) ? bi * g32[u + 0] : 0.f;
+                    a.y = (j + 1 < i) ? bi * g32[u + 1] : 0.f;
+                    a.z = (j + 2 < i) ? bi * g32[u + 2] : 0.f;
+                    a.w = (j + 3 < i) ? bi * g32[u + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(fA + i * AS + j) = a;
+                }
+            }
+            asm volatile("bar.sync 1, 64;" ::: "memory");
+            invert_diag_blocks(fA, fT, sm + L::TB, fB, tid);
+        } else if (warp < 4) {
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                float g32[32];
+                ptx::tmem_ld32(tl + ICOL_GRAM + hh * 32, g32);
+                ptx::tmem_wait_ld();
+                const int i = tid - 64;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) g32[u] = (hh * 32 + u <= i) ? g32[u] : 0.f;
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::AQ + sw128_chunk(i, hh * 4 + gq), g32 + gq * 8);
+            }
+        } else if (warp >= 6) {
+            const int t = tid - 192;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int e = t + 64 * m, blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                fT[(32 * blk + r) * AS + 32 * blk + 16 + c] = 0.f;
+            }
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int m = 0; m < 3; ++m) {
+                const int e = t + 64 * m;
+                const int blk = e >> 5, r = (e >> 1) & 15, gh = e & 1;
+                const int bi = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                const int bj = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                *reinterpret_cast<uint4 *>(sm + L::TB + sw128_chunk(16 * bi + r, 2 * bj + gh)) = z;
+            }
+        }
+        __syncthreads();
+        invert_merge_blocks(fA, fT, fM, sm + L::TB, fB, warp, lane);
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- 4. Kt = Kbar^T Tb (Kbar read MN-major); Pt = Aqk Tb from the M = 128 operand [Tb^T; Aqk]
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t ikt = ptx::idesc_bf16_f32(128, 64, true, false);
+            constexpr uint32_t ipt = ptx::idesc_bf16_f32(128, 64);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + ICOL_KT, ptx::desc_mnmajor_sw128(sb + L::KB + s * 2048, 64 * 128, 1024),
+                              kdesc(sb + L::TB, s, 64), ikt, s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + ICOL_PT, kdesc(sb + L::TB, s, 128), kdesc(sb + L::TB, s, 64), ipt, s > 0);
+            ptx::mma_commit(bar_mma);
+        }
+        ok = wait_all(bar_mma, ph_mma);
+    }
+
+    if (ok) {
+        // ---- 5. Kt, Pt -> bf16 images in the record (each thread one 64-byte half row)
+        uint8_t *kp = rec + R::KP;
+        if (quad < DK / 32) {
+            float x[32];
+            ptx::tmem_ld32(tl + ICOL_KT + half * 32, x);
+            ptx::tmem_wait_ld();
+            const int row = quad * 32 + lane;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) st_global_bf16x8(kp + sw128_chunk(row, half * 4 + gq), x + gq * 8);
+        }
+        if (quad >= 2) {
+            float x[32];
+            ptx::tmem_ld32(tl + ICOL_PT + half * 32, x);
+            ptx::tmem_wait_ld();
+            const int row = DK + (quad - 2) * 32 + lane;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) st_global_bf16x8(kp + sw128_chunk(row, half * 4 + gq), x + gq * 8);
+        }
+    }
+    if (tid == 0) ptx::bulk_wait_all();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, INTRA_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ pass 2
+
+template <int DK, int DVT, int NBUF>
+struct InterLayout {
+    static constexpr int KA = DK / 64;
+    static constexpr int REC = Rec<DK>::BYTES;
+    static constexpr int SP = NBUF * REC;                 // [KA][DVT][128 B] (e^{G_last} S)^T
+    static constexpr int ZT = SP + KA * DVT * 128;        // [DVT][128 B]     Z^T
+    static constexpr int VIN = ZT + DVT * 128;            // bf16 [NBUF][64][DVT]
+    static constexpr int MISC = VIN + NBUF * C * DVT * 2; // mbarriers, TMEM base, flags
+    static constexpr int BYTES = MISC + 64;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(REC % 1024 == 0 && SP % 1024 == 0 && ZT % 1024 == 0 && VIN % 128 == 0, "tile alignment");
+};
+
+template <int DK, int DVT>
+constexpr int inter_nbuf() {
+    return InterLayout<DK, DVT, 3>::ALLOC <= 232448 ? 3 : 2;
+}
+
+constexpr uint32_t INTER_TMEM_COLS = 256;
+constexpr uint32_t XCOL_XY = 0;       // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O
+constexpr uint32_t XCOL_DS = 128;     // [128 x DVT] Kt Z (lanes 0..dk-1)
+
+template <int DK, int DVT, int NBUF>
+__global__ void __launch_bounds__(NT, 1)
+chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__restrict__ ws,
+                   const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
+                   float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
+    using L = InterLayout<DK, DVT, NBUF>;
+    using R = Rec<DK>;
+    static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
+    constexpr int CPT = DVT / 2;
+    constexpr uint32_t TX = (uint32_t)(R::BYTES + C * DVT * 2);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = ptx::smem_u32(sm);
+    const uint32_t bar_rec = sb + L::MISC, bar_mma = sb + L::MISC + 32;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 40);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int col_base = blockIdx.x * DVT, h = blockIdx.y, n = blockIdx.z;
+
+    long long t0, t1;
+    seq_span(cu_seqlens, T, n, t0, t1);
+    const int nck = (int)((t1 - t0 + C - 1) / C);
+    const long long first = n + t0 / C;   // slot of chunk 0
+
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTER_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int b = 0; b < NBUF; ++b) ptx::mbar_init(bar_rec + 8 * b, 1);
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tm_v);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t ph_mma = 0, ph_rec = 0;   // ph_rec: one parity bit per buffer
+
+    auto issue = [&](int ci) {   // thread 0: record and V tile of chunk ci into buffer ci % NBUF
+        const int b = ci % NBUF;
+        const uint32_t bar = bar_rec + 8 * b;
+        ptx::mbar_arrive_expect_tx(bar, TX);
+        ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * R::BYTES, (uint32_t)R::BYTES, bar);
+        ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, &tm_v, bar, col_base, h, (int)(t0 + (long long)ci * C));
+    };
+
+    const int srow = quad * 32 + lane;
+    const bool has_row = srow < DK;
+    const int scol = half * CPT;
+    const long long st_off = ((long long)n * H + h) * DK * DV + col_base + scol;
+    float S[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; j += 4) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (has_row && init_state) x = load4(init_state + st_off + (long long)srow * DV + j);
+        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+    }
+    if (tid == 0)
+        for (int ci = 0; ci < NBUF && ci < nck; ++ci) issue(ci);
+
+    bool ok = true;
+    for (int ci = 0; ci < nck; ++ci) {
+        const long long cs = t0 + (long long)ci * C;
+        const int Lc = (int)min((long long)C, t1 - cs);
+        const int b = ci % NBUF;
+        const uint32_t rb = sb + b * R::BYTES;
+        uint32_t ph = (ph_rec >> b) & 1u;
+        ok = wait_all(bar_rec + 8 * b, ph);
+        ph_rec ^= 1u << b;
+        if (!ok) break;
+
+        // ---- 1. (e^{G_last} S)^T -> bf16 B operand
+        const float dch = has_row ? reinterpret_cast<const float *>(sm + b * R::BYTES + R::DCH)[srow] : 0.f;
+        if (has_row) {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::SP + sw128(scol + j, srow, DVT), dch * S[j]);
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- 2. [X; Y] = [Kp; Qp] (e^{G_last} S)
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t ix = ptx::idesc_bf16_f32(128, DVT);
+#pragma unroll
+            for (int s = 0; s < DK / 16; ++s)
+                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KQ, s, 128), kdesc(sb + L::SP, s, DVT), ix, s > 0);
+            ptx::mma_commit(bar_mma);
+        }
+        if (!(ok = wait_all(bar_mma, ph_mma))) break;
+
+        // ---- 3. Z = V - X (X in TMEM lanes 0-63) -> Z^T
+        if (quad < 2) {
+            const int j = quad * 32 + lane;
+            const uint8_t *vin = sm + L::VIN + b * C * DVT * 2;
+#pragma unroll 1
+            for (int cc = 0; cc < CPT / 16; ++cc) {
+                float x16[16], v16[16];
+                ptx::tmem_ld16(tl + XCOL_XY + scol + cc * 16, x16);
+                if (j < Lc) {
+                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(vin + (j * DVT + scol + cc * 16) * 2), v16);
+                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(vin + (j * DVT + scol + cc * 16 + 8) * 2), v16 + 8);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) v16[u] = 0.f;
+                }
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) st_bf16(sm, L::ZT + sw128(scol + cc * 16 + u, j, DVT), v16[u] - x16[u]);
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- 4. dS = Kt Z ; O = Y + Pt Z (onto the Y rows of [X; Y])
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t iz = ptx::idesc_bf16_f32(128, DVT);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + XCOL_DS, kdesc(rb + R::KP, s, DK + 64), kdesc(sb + L::ZT, s, DVT), iz, s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KP, s, DK + 64, DK - 64), kdesc(sb + L::ZT, s, DVT), iz, 1);
+            ptx::mma_commit(bar_mma);
+        }
+        if (!(ok = wait_all(bar_mma, ph_mma))) break;
+        if (tid == 0 && ci + NBUF < nck) issue(ci + NBUF);   // buffer b fully consumed
+
+        // ---- 5. S <- Diag(e^{G_last}) S + dS ; O rows (TMEM lanes 64-127) -> o
+        if (has_row) {
+#pragma unroll
+            for (int cc = 0; cc < CPT / 16; ++cc) {
+                float d16[16];
+                ptx::tmem_ld16(tl + XCOL_DS + scol + cc * 16, d16);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
+            }
+        }
+        if (quad >= 2) {
+            const int i = (quad - 2) * 32 + lane;
+#pragma unroll 1
+            for (int cc = 0; cc < CPT / 16; ++cc) {
+                float o16[16];
+                ptx::tmem_ld16(tl + XCOL_XY + scol + cc * 16, o16);
+                ptx::tmem_wait_ld();
+                if (i < Lc) {
+                    __nv_bfloat16 *dst = o + ((cs + i) * H + h) * DV + col_base + scol + cc * 16;
+                    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pack_bf16(o16[0], o16[1]), pack_bf16(o16[2], o16[3]),
+                                                                   pack_bf16(o16[4], o16[5]), pack_bf16(o16[6], o16[7]));
+                    reinterpret_cast<uint4 *>(dst)[1] =
+                        make_uint4(pack_bf16(o16[8], o16[9]), pack_bf16(o16[10], o16[11]),
+                                   pack_bf16(o16[12], o16[13]), pack_bf16(o16[14], o16[15]));
+                }
+            }
+        }
+        ptx::tc_fence_before();
+    }
+
+    __syncthreads();
+    if (ok && final_state && has_row) {
+#pragma unroll
+        for (int j = 0; j < CPT; j += 4)
+            store4(final_state + st_off + (long long)srow * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, INTER_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+template <int DK, int DVT>
+int launch_two_pass_t(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                      const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
+                      long long tokens, int T, int H, int dv, int num_seqs, void *workspace, cudaStream_t st,
+                      char *msg, size_t msg_len) {
+    CUtensorMap tv;
+    if (!make_tmap(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, dv, DVT)) {
+        snprintf(msg, msg_len, "building TMA descriptors failed (driver entry point cuTensorMapEncodeTiled)");
+        return KDA_ERR_CUDA;
+    }
+    const long long slots = chunk_slots(tokens, num_seqs);
+    if (slots > 0x7fffffffLL) {
+        snprintf(msg, msg_len, "%lld chunk slots exceed the grid limit", slots);
+        return KDA_ERR_UNSUPPORTED;
+    }
+    constexpr int smem1 = IntraLayout<DK>::ALLOC;
+    auto k1 = chunk_intra_kernel<DK>;
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
+    if (e != cudaSuccess) {
+        snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_intra): %s", cudaGetErrorString(e));
+        return KDA_ERR_CUDA;
+    }
+    k1<<<dim3((unsigned)slots, H), NT, smem1, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
+                                                     beta, cu_seqlens, T, H, num_seqs, (uint8_t *)workspace);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        snprintf(msg, msg_len, "chunk_intra launch: %s", cudaGetErrorString(e));
+        return KDA_ERR_CUDA;
+    }
+    constexpr int NBUF = inter_nbuf<DK, DVT>();
+    constexpr int smem2 = InterLayout<DK, DVT, NBUF>::ALLOC;
+    static_assert(smem2 <= 232448, "shared memory budget");
+    auto k2 = chunk_inter_kernel<DK, DVT, NBUF>;
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+    if (e != cudaSuccess) {
+        snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_inter): %s", cudaGetErrorString(e));
+        return KDA_ERR_CUDA;
+    }
+    k2<<<dim3(dv / DVT, H, num_seqs), NT, smem2, st>>>(tv, (const uint8_t *)workspace, init_state,
+                                                        (__nv_bfloat16 *)o, final_state, cu_seqlens, T, H, dv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        snprintf(msg, msg_len, "chunk_inter launch: %s", cudaGetErrorString(e));
+        return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
+inline int launch_two_pass(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                           const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
+                           long long tokens, int T, int H, int dk, int dv, int num_seqs, void *workspace,
+                           cudaStream_t st, char *msg, size_t msg_len) {
+    // value-tile width of the recurrence pass: the widest that still gives one CTA per SM
+    const long long chains = (long long)num_seqs * H;
+    int dvt = 32;
+    for (int cand = dv; cand >= 32; cand /= 2)
+        if (chains * (dv / cand) >= 148) { dvt = cand; break; }
+#define KDA_2P(DKv, DVTv)                                                                                        \
+    return launch_two_pass_t<DKv, DVTv>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, \
+                                        T, H, dv, num_seqs, workspace, st, msg, msg_len)
+    if (dk == 128) {
+        if (dvt == 128) KDA_2P(128, 128);
+        if (dvt == 64) KDA_2P(128, 64);
+        KDA_2P(128, 32);
+    }
+    if (dvt == 128) KDA_2P(64, 128);
+    if (dvt == 64) KDA_2P(64, 64);
+    KDA_2P(64, 32);
+#undef KDA_2P
+}
+
+}  // namespace tc
+}  // namespace kda

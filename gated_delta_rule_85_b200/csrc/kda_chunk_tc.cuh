@@ -656,11 +656,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
-inline size_t workspace_bytes(int num_seqs) {
-    (void)num_seqs;
-    return 0;
-}
-
 // ------------------------------------------------------------------ host side
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -723,29 +718,24 @@ int launch_t(const void *q, const void *k, const void *v, const float *log_alpha
     return KDA_OK;
 }
 
-inline int launch(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
-                  const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int B, int T,
-                  int H, int dk, int dv, int num_seqs, void *workspace, cudaStream_t st, char *msg,
-                  size_t msg_len) {
-    (void)workspace;
-    const long long tokens = (long long)B * T;
-    if (tokens == 0) {
-        // no tokens: the final state is the initial state (or zeros)
-        if (final_state) {
-            const size_t bytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
-            cudaError_t e = init_state ? cudaMemcpyAsync(final_state, init_state, bytes, cudaMemcpyDeviceToDevice, st)
-                                       : cudaMemsetAsync(final_state, 0, bytes, st);
-            if (e != cudaSuccess) {
-                snprintf(msg, msg_len, "state copy: %s", cudaGetErrorString(e));
-                return KDA_ERR_CUDA;
-            }
-        }
-        return KDA_OK;
+// No tokens: the final state is the initial state (or zeros).
+inline int state_passthrough(const float *init_state, float *final_state, int num_seqs, int H, int dk, int dv,
+                             cudaStream_t st, char *msg, size_t msg_len) {
+    if (!final_state) return KDA_OK;
+    const size_t bytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
+    cudaError_t e = init_state ? cudaMemcpyAsync(final_state, init_state, bytes, cudaMemcpyDeviceToDevice, st)
+                               : cudaMemsetAsync(final_state, 0, bytes, st);
+    if (e != cudaSuccess) {
+        snprintf(msg, msg_len, "state copy: %s", cudaGetErrorString(e));
+        return KDA_ERR_CUDA;
     }
-    if (tokens > 0x7fffffffLL) {
-        snprintf(msg, msg_len, "B*T=%lld exceeds the 2^31 token limit of the TMA coordinates", tokens);
-        return KDA_ERR_UNSUPPORTED;
-    }
+    return KDA_OK;
+}
+
+inline int launch_fused(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                        const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
+                        long long tokens, int T, int H, int dk, int dv, int num_seqs, cudaStream_t st, char *msg,
+                        size_t msg_len) {
     // Value-tile width: the widest tile (fewest duplicated per-chunk operand
     // builds) that still gives at least two CTAs per SM; else 32 columns.
     const long long chains = (long long)num_seqs * H;

@@ -8,6 +8,7 @@
 #include "kda_decode.cuh"
 #include "kda_chunk_simt.cuh"
 #include "kda_chunk_tc.cuh"
+#include "kda_chunk_2pass.cuh"
 
 namespace {
 
@@ -58,6 +59,23 @@ int check_prefill(const void *q, const void *k, const void *v, const float *log_
     return KDA_OK;
 }
 
+// Which tensor-core schedule runs, and the workspace it needs.
+struct Plan {
+    int algo;
+    size_t ws;
+};
+
+constexpr size_t kAutoTwoPassLimit = (size_t)4 << 30;   // AUTO takes TWO_PASS only up to this workspace
+constexpr long long kAutoChainLimit = 2 * 148;          // ... and below this many (sequence, head) chains
+
+Plan plan_prefill(long long tokens, int H, int dk, int num_seqs, int algo) {
+    const size_t ws2 = kda::tc::two_pass_workspace_bytes(tokens, H, dk, num_seqs);
+    if (algo == KDA_ALGO_AUTO)
+        algo = ((long long)num_seqs * H < kAutoChainLimit && ws2 <= kAutoTwoPassLimit) ? KDA_ALGO_TWO_PASS
+                                                                                       : KDA_ALGO_FUSED;
+    return Plan{algo, algo == KDA_ALGO_TWO_PASS ? ws2 : 0};
+}
+
 template <int DK, typename Tin>
 int launch_simt(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                 const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int T,
@@ -92,11 +110,16 @@ int kda_api_version(void) { return KDA_API_VERSION; }
 
 const char *kda_last_error(void) { return g_err; }
 
+size_t kda_chunk_forward_workspace_size_ex(int B, int T, int H, int dk, int dv, int num_seqs, int dtype,
+                                           int chunk, int algo) {
+    (void)dv; (void)chunk;
+    if (dtype != KDA_BF16 || B < 1 || T < 0 || H < 1 || num_seqs < 0 || (dk != 64 && dk != 128)) return 0;
+    return plan_prefill((long long)B * T, H, dk, num_seqs, algo).ws;
+}
+
 size_t kda_chunk_forward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype,
                                         int chunk) {
-    (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)chunk;
-    if (dtype != KDA_BF16) return 0;
-    return kda::tc::workspace_bytes(num_seqs);
+    return kda_chunk_forward_workspace_size_ex(B, T, H, dk, dv, num_seqs, dtype, chunk, KDA_ALGO_AUTO);
 }
 
 int kda_chunk_forward_simt(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -122,26 +145,46 @@ int kda_chunk_forward_simt(const void *q, const void *k, const void *v, const fl
                                    dv, num_seqs, st);
 }
 
+int kda_chunk_forward_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                         const float *beta, const float *init_state, void *o, float *final_state,
+                         const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                         int dtype, int chunk, int algo, void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
+                           dv, num_seqs, dtype, chunk);
+    if (rc) return rc;
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_FUSED && algo != KDA_ALGO_TWO_PASS)
+        return fail(KDA_ERR_INVALID_ARG, "algo=%d is not a KDA_ALGO_* value", algo);
+    if (dtype == KDA_F32)
+        return kda_chunk_forward_simt(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B,
+                                      T, H, dk, dv, num_seqs, dtype, chunk, stream);
+    const long long tokens = (long long)B * T;
+    const Plan plan = plan_prefill(tokens, H, dk, num_seqs, algo);
+    if (plan.ws && (!workspace || ws_bytes < plan.ws))
+        return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", plan.ws, ws_bytes);
+    if (workspace && !aligned(workspace, 256)) return fail(KDA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (num_seqs == 0) return KDA_OK;
+    if (tokens > 0x7fffffffLL)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T=%lld exceeds the 2^31 token limit of the TMA coordinates", tokens);
+    char msg[256] = "";
+    cudaStream_t st = (cudaStream_t)stream;
+    if (tokens == 0)
+        rc = kda::tc::state_passthrough(init_state, final_state, num_seqs, H, dk, dv, st, msg, sizeof(msg));
+    else if (plan.algo == KDA_ALGO_TWO_PASS)
+        rc = kda::tc::launch_two_pass(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T,
+                                      H, dk, dv, num_seqs, workspace, st, msg, sizeof(msg));
+    else
+        rc = kda::tc::launch_fused(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T, H,
+                                   dk, dv, num_seqs, st, msg, sizeof(msg));
+    if (rc) return fail(rc, "%s", msg);
+    return KDA_OK;
+}
+
 int kda_chunk_forward(const void *q, const void *k, const void *v, const float *log_alpha,
                       const float *beta, const float *init_state, void *o, float *final_state,
                       const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
                       int dtype, int chunk, void *workspace, size_t ws_bytes, void *stream) {
-    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
-                           dv, num_seqs, dtype, chunk);
-    if (rc) return rc;
-    if (dtype == KDA_F32)
-        return kda_chunk_forward_simt(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B,
-                                      T, H, dk, dv, num_seqs, dtype, chunk, stream);
-    const size_t need = kda::tc::workspace_bytes(num_seqs);
-    if (need && (!workspace || ws_bytes < need))
-        return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", need, ws_bytes);
-    if (workspace && !aligned(workspace, 256)) return fail(KDA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
-    if (num_seqs == 0) return KDA_OK;
-    char msg[256] = "";
-    rc = kda::tc::launch(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk, dv,
-                         num_seqs, workspace, (cudaStream_t)stream, msg, sizeof(msg));
-    if (rc) return fail(rc, "%s", msg);
-    return KDA_OK;
+    return kda_chunk_forward_ex(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
+                                dv, num_seqs, dtype, chunk, KDA_ALGO_AUTO, workspace, ws_bytes, stream);
 }
 
 int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -117,6 +117,39 @@ int kda_chunk_forward(const void *q, const void *k, const void *v, const float *
                       int dtype, int chunk, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Schedules of the tensor-core prefill.  Both compute the same chunk algebra in
+ * the same precision; they differ in where the state-independent part of each
+ * chunk (decay factors, Gram matrix, UT transform, Kt = Kbar^T T Diag(beta),
+ * Pt = Aqk T Diag(beta)) is built.
+ *
+ *   KDA_ALGO_FUSED     one kernel; each CTA (value-column tile, head, sequence)
+ *                      builds it inside its serial walk over the chunks.  No
+ *                      workspace.  Best when there are many (sequence, head)
+ *                      chains.
+ *   KDA_ALGO_TWO_PASS  a first kernel builds it for every (chunk, head) at once
+ *                      into the workspace (about 57 KB per chunk and head at
+ *                      dk = 128, 33 KB at dk = 64); a second kernel walks the
+ *                      chunks with only the state-dependent products left.
+ *                      Best when there are few chains.
+ *   KDA_ALGO_AUTO      TWO_PASS when num_seqs * H < 296 and its workspace is at
+ *                      most 4 GiB, else FUSED.  kda_chunk_forward uses AUTO.
+ */
+#define KDA_ALGO_AUTO 0
+#define KDA_ALGO_FUSED 1
+#define KDA_ALGO_TWO_PASS 2
+
+/* Workspace bytes kda_chunk_forward_ex needs for these sizes and `algo` (0 when none). */
+size_t kda_chunk_forward_workspace_size_ex(int B, int T, int H, int dk, int dv, int num_seqs,
+                                           int dtype, int chunk, int algo);
+
+/* kda_chunk_forward with an explicit schedule (KDA_ALGO_*; ignored for KDA_F32, which
+ * always takes the fp32 CUDA-core path).  An unknown `algo` is KDA_ERR_INVALID_ARG. */
+int kda_chunk_forward_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                         const float *beta, const float *init_state, void *o, float *final_state,
+                         const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                         int dtype, int chunk, int algo, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Same contract as kda_chunk_forward, computed entirely on CUDA cores in fp32
  * (inputs in either dtype are widened exactly).  The accuracy reference for the
  * tensor-core path and the path taken for KDA_F32.  Needs no workspace.

@@ -22,21 +22,26 @@ pytestmark = pytest.mark.gpu
 BF16 = torch.bfloat16
 
 
-def _fwd(d, sl=slice(None), s0="init", simt=False):
+def _fwd(d, sl=slice(None), s0="init", simt=False, algo="auto"):
     init = d["init_state"] if isinstance(s0, str) else s0
     return kda.chunk_forward(d["q"][:, sl].contiguous(), d["k"][:, sl].contiguous(), d["v"][:, sl].contiguous(),
-                             d["log_alpha"][:, sl].contiguous(), d["beta"][:, sl].contiguous(), init, simt=simt)
+                             d["log_alpha"][:, sl].contiguous(), d["beta"][:, sl].contiguous(), init, simt=simt,
+                             algo=algo)
+
+
+# the tensor-core path under each schedule, and the fp32 CUDA-core path
+PATHS = [("fused", False), ("two_pass", False), ("auto", True)]
 
 
 @pytest.mark.parametrize("split", [64, 100, 320])
-@pytest.mark.parametrize("simt", [False, True])
-def test_split_prefill_resumes_exactly(split, simt):
+@pytest.mark.parametrize("algo,simt", PATHS)
+def test_split_prefill_resumes_exactly(split, algo, simt):
     dtype = torch.float32 if simt else BF16
     shape = PrefillShape(B=1, T=500, H=3, dk=128, dv=128, dtype=dtype)
     d = prefill_inputs(shape, 31, torch.device("cuda"))
-    o1, S1 = _fwd(d, slice(0, split), simt=simt)
-    o2, S2 = _fwd(d, slice(split, None), s0=S1, simt=simt)
-    o, S = _fwd(d, simt=simt)
+    o1, S1 = _fwd(d, slice(0, split), simt=simt, algo=algo)
+    o2, S2 = _fwd(d, slice(split, None), s0=S1, simt=simt, algo=algo)
+    o, S = _fwd(d, simt=simt, algo=algo)
     torch.cuda.synchronize()
     o_ref, S_ref = oracle_prefill(d)
     o_cat = np.concatenate([to_f64(o1), to_f64(o2)], axis=1)
@@ -47,14 +52,15 @@ def test_split_prefill_resumes_exactly(split, simt):
         assert torch.equal(torch.cat([o1, o2], dim=1), o) and torch.equal(S2, S)
 
 
+@pytest.mark.parametrize("algo", ["fused", "two_pass"])
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128)])
-def test_prefill_then_decode_matches_one_recurrence(dk, dv):
+def test_prefill_then_decode_matches_one_recurrence(dk, dv, algo):
     """The prefill's final_state is directly the decode state (one layout for both)."""
     T0, steps = 333, 24
     shape = PrefillShape(B=2, T=T0, H=4, dk=dk, dv=dv, dtype=BF16)
     dev = torch.device("cuda")
     d = prefill_inputs(shape, 40, dev)
-    o, S = _fwd(d)
+    o, S = _fwd(d, algo=algo)
     dshape = DecodeShape(N=2, H=4, dk=dk, dv=dv, steps=steps, dtype=BF16)
     dec = [decode_step_inputs(dshape, t, 41, dev) for t in range(steps)]
     o_dec = [kda.recurrent_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S) for x in dec]
@@ -69,18 +75,18 @@ def test_prefill_then_decode_matches_one_recurrence(dk, dv):
     assert_close(to_f64(S), S_ref, BF16, "final state")
 
 
-@pytest.mark.parametrize("simt", [False, True])
-def test_packed_equals_separate_runs(simt):
+@pytest.mark.parametrize("algo,simt", PATHS)
+def test_packed_equals_separate_runs(algo, simt):
     dtype = torch.float32 if simt else BF16
     lens = [70, 0, 129, 1, 256, 33]
     cu = tuple(np.cumsum([0] + lens).tolist())
     shape = PrefillShape(B=1, T=cu[-1], H=2, dk=128, dv=128, dtype=dtype, cu_seqlens=cu)
     d = prefill_inputs(shape, 50, torch.device("cuda"))
     o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], d["cu_seqlens"],
-                             simt=simt)
+                             simt=simt, algo=algo)
     for n, L in enumerate(lens):
         sl = slice(cu[n], cu[n + 1])
-        on, Sn = _fwd(d, sl, s0=d["init_state"][n:n + 1].contiguous(), simt=simt)
+        on, Sn = _fwd(d, sl, s0=d["init_state"][n:n + 1].contiguous(), simt=simt, algo=algo)
         torch.cuda.synchronize()
         if L:
             assert rel_l2(to_f64(o[:, sl]), to_f64(on)) < (1e-6 if simt else 5e-3)
@@ -92,33 +98,36 @@ def test_packed_equals_separate_runs(simt):
     assert torch.equal(S[1], d["init_state"][1])   # empty sequence keeps its state
 
 
-def test_value_column_permutation_is_equivariant():
+@pytest.mark.parametrize("algo", ["fused", "two_pass"])
+def test_value_column_permutation_is_equivariant(algo):
     shape = PrefillShape(B=1, T=200, H=2, dk=128, dv=128, dtype=BF16)
     d = prefill_inputs(shape, 60, torch.device("cuda"))
     perm = torch.randperm(128, generator=torch.Generator().manual_seed(0)).cuda()
-    o, S = _fwd(d)
+    o, S = _fwd(d, algo=algo)
     d2 = dict(d)
     d2["v"] = d["v"][..., perm].contiguous()
     d2["init_state"] = d["init_state"][..., perm].contiguous()
-    o2, S2 = _fwd(d2)
+    o2, S2 = _fwd(d2, algo=algo)
     torch.cuda.synchronize()
     assert rel_l2(to_f64(o2), to_f64(o[..., perm])) < 5e-3
     assert rel_l2(to_f64(S2), to_f64(S[..., perm])) < 5e-3
 
 
-def test_empty_and_zero_length_inputs():
+@pytest.mark.parametrize("algo", ["fused", "two_pass"])
+def test_empty_and_zero_length_inputs(algo):
     dev = torch.device("cuda")
     shape = PrefillShape(B=2, T=0, H=2, dk=128, dv=128, dtype=BF16)
     d = prefill_inputs(shape, 70, dev)
-    o, S = _fwd(d)
+    o, S = _fwd(d, algo=algo)
     torch.cuda.synchronize()
     assert o.numel() == 0 and torch.equal(S, d["init_state"])
-    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None)
+    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, algo=algo)
     torch.cuda.synchronize()
     assert torch.count_nonzero(S) == 0
 
 
-def test_decay_range_flag():
+@pytest.mark.parametrize("algo", ["fused", "two_pass"])
+def test_decay_range_flag(algo):
     """A chunk whose summed log-decay falls below -80 is outside the tensor-core
     path's factorisation range: the call raises KDA_DEV_DECAY_RANGE; the fp32
     path handles it and matches the oracle."""
@@ -126,7 +135,7 @@ def test_decay_range_flag():
     d = prefill_inputs(shape, 80, torch.device("cuda"))
     d["log_alpha"][:, :64, 0, :8] = -2.0           # 64 tokens x -2 = -128 in channels 0..7 of head 0
     kda.device_status(clear=True)
-    kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"])
+    kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], algo=algo)
     torch.cuda.synchronize()
     assert kda.device_status(clear=True) & kda.DEV_DECAY_RANGE
     o, S = kda.chunk_forward_simt(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"])

@@ -23,8 +23,9 @@ BF16 = torch.bfloat16
 DEV = "cuda"
 
 
-def _prefill(d):
-    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], d["cu_seqlens"])
+def _prefill(d, algo="auto"):
+    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], d["cu_seqlens"],
+                             algo=algo)
     torch.cuda.synchronize()
     assert kda.device_status() == 0
     return o, S
@@ -40,12 +41,14 @@ def test_tiny_f32_through_main_entry_point():
 
 
 def test_prefill_8k_all_heads():
+    """The benchmark's launch (AUTO: two-pass for 32 chains) and the fused schedule."""
     shape = CONFIGS["prefill_8k"]
     d = prefill_inputs(shape, 0, torch.device(DEV))
-    o, S = _prefill(d)
     o_ref, S_ref = oracle_prefill(d)
-    assert_close(to_f64(o), o_ref, BF16, "o")
-    assert_close(to_f64(S), S_ref, BF16, "final state")
+    for algo in ("auto", "fused"):
+        o, S = _prefill(d, algo)
+        assert_close(to_f64(o), o_ref, BF16, f"o ({algo})")
+        assert_close(to_f64(S), S_ref, BF16, f"final state ({algo})")
 
 
 def test_prefill_128k_sampled_heads():
@@ -90,7 +93,12 @@ def test_varlen_1m_then_decode_sampled_heads():
     o_ref, S_ref = oracle_prefill(d, heads)
     assert_close(to_f64(o[:, :, heads]), o_ref, BF16, "o")
     assert_close(to_f64(S[:, heads]), S_ref, BF16, "final state")
-    del d, o
+    # the same packed input under the two-pass schedule (AUTO takes the fused one here)
+    o2, S2 = _prefill(d, "two_pass")
+    assert_close(to_f64(o2[:, :, heads]), o_ref, BF16, "o (two-pass)")
+    assert_close(to_f64(S2[:, heads]), S_ref, BF16, "final state (two-pass)")
+    del d, o, o2, S2
+    torch.cuda.empty_cache()
     # 256 decode steps per sequence, continuing from the prefill's final state in place
     dshape = DecodeShape(N=shape.num_seqs, H=shape.H, dk=shape.dk, dv=shape.dv, steps=256, dtype=BF16)
     o_got, o_want = [], []
