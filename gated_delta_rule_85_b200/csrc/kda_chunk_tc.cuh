@@ -41,7 +41,7 @@ namespace tc {
 
 constexpr int C = 64;
 constexpr int NT = 256;
-constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;   // 1 s: far beyond any legitimate latency
+constexpr long long WAIT_LIMIT_CYCLES = 2000000000ll;   // >= 1 s at any SM clock up to 2 GHz: far beyond any legitimate latency
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM column map (fp32 accumulators, lane = row)
 constexpr uint32_t COL_GRAM = 0;    // [128 x 64]  rows 0-63 Kp Kbar^T, rows 64-127 Qp Kbar^T
@@ -253,7 +253,7 @@ __device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, f
 // outcome (a shared "failed" flag from warp-local waits is folded in).  Returns
 // false, and flags the device status, on timeout.
 __device__ __forceinline__ bool wait_all(uint32_t mbar, uint32_t &phase, int local_fail = 0) {
-    const bool ok = ptx::mbar_wait_bounded(mbar, phase, WAIT_LIMIT_NS);
+    const bool ok = ptx::mbar_wait_bounded(mbar, phase, WAIT_LIMIT_CYCLES);
     phase ^= 1u;
     if (__syncthreads_or((!ok) || local_fail)) {
         if (threadIdx.x == 0) flag_status(KDA_DEV_WAIT_TIMEOUT);
@@ -508,7 +508,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         } else if (warp < 6) {
             // X rows (TMEM lanes 0-63) -> Z = V - X -> Z^T
-            if (!ptx::mbar_wait_bounded(bar_v, ph_v, WAIT_LIMIT_NS)) *fail_flag = 1;
+            if (!ptx::mbar_wait_bounded(bar_v, ph_v, WAIT_LIMIT_CYCLES)) *fail_flag = 1;
             const int j = quad * 32 + lane;
             const uint8_t *vin = sm + L::VIN;
 #pragma unroll 1
