@@ -20,7 +20,7 @@ import os
 import torch
 
 __all__ = [
-    "chunk_forward", "chunk_forward_simt", "recurrent_step", "workspace_size", "device_status",
+    "chunk_forward", "chunk_forward_simt", "chunk_forward_static_ws", "recurrent_step", "workspace_size", "device_status",
     "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
     "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "ALGOS",
 ]
@@ -32,6 +32,8 @@ DEV_WAIT_TIMEOUT = 0x1
 DEV_DECAY_RANGE = 0x2
 # tensor-core prefill schedules (KDA_ALGO_* in include/kda.h)
 ALGOS = {"auto": 0, "fused": 1, "two_pass": 2}
+# size of the built-in scratch of kda_chunk_forward_static_ws (KDA_STATIC_WS_BYTES)
+STATIC_WS_BYTES = 64 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
@@ -68,6 +70,8 @@ def load_library():
     lib.kda_chunk_forward_ex.restype = ci
     lib.kda_chunk_forward_workspace_size_ex.argtypes = [ci] * 9
     lib.kda_chunk_forward_workspace_size_ex.restype = sz
+    lib.kda_chunk_forward_static_ws.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, ip] + [ci] * 8 + [vp]
+    lib.kda_chunk_forward_static_ws.restype = ci
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ci] * 5 + [vp]
     lib.kda_recurrent_step.restype = ci
     lib.kda_last_error.argtypes = []
@@ -196,6 +200,27 @@ def chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *,
         rc = lib.kda_chunk_forward_ex(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(o),
                                       _p(final_state), _p(cu_seqlens), B, T, H, dk, dv, N, dt, CHUNK, ac,
                                       _p(workspace), ws_bytes, st)
+    _check(rc)
+    return o, final_state
+
+
+def chunk_forward_static_ws(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, o=None,
+                            final_state=True):
+    """kda_chunk_forward_static_ws: the two-pass prefill on the library's built-in
+    scratch (no workspace argument, nothing allocated by the library).  Device
+    tensors only; the caller's outputs are allocated here unless given."""
+    B, T, H, dk, dv, N = _prefill_args(q, k, v, log_alpha, beta, init_state, cu_seqlens)
+    _need_cuda(q, k, v, log_alpha, beta, init_state, cu_seqlens)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is True:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    elif final_state is False:
+        final_state = None
+    _need_cuda(o, final_state)
+    rc = load_library().kda_chunk_forward_static_ws(
+        _p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(o), _p(final_state), _p(cu_seqlens),
+        B, T, H, dk, dv, N, _dtype_code(q), CHUNK, _stream(q.device))
     _check(rc)
     return o, final_state
 

@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
@@ -74,6 +75,34 @@ Plan plan_prefill(long long tokens, int H, int dk, int num_seqs, int algo) {
         algo = ((long long)num_seqs * H < kAutoChainLimit && ws2 <= kAutoTwoPassLimit) ? KDA_ALGO_TWO_PASS
                                                                                        : KDA_ALGO_FUSED;
     return Plan{algo, algo == KDA_ALGO_TWO_PASS ? ws2 : 0};
+}
+
+// Scratch of kda_chunk_forward_static_ws: file scope, reserved on each device
+// with the module; its address is looked up once per device.
+static __device__ __align__(256) uint8_t g_static_ws[KDA_STATIC_WS_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_static_ws on the current device (nullptr on failure, with
+// the CUDA error in *err).
+void *static_ws_address(cudaError_t *err) {
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= kMaxDevices) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_static_ws);
+        if (*err != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
 }
 
 template <int DK, typename Tin>
@@ -185,6 +214,33 @@ int kda_chunk_forward(const void *q, const void *k, const void *v, const float *
                       int dtype, int chunk, void *workspace, size_t ws_bytes, void *stream) {
     return kda_chunk_forward_ex(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
                                 dv, num_seqs, dtype, chunk, KDA_ALGO_AUTO, workspace, ws_bytes, stream);
+}
+
+int kda_chunk_forward_static_ws(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, const float *init_state, void *o, float *final_state,
+                                const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                                int dtype, int chunk, void *stream) {
+    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
+                           dv, num_seqs, dtype, chunk);
+    if (rc) return rc;
+    if (dtype == KDA_F32)
+        return kda_chunk_forward_simt(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B,
+                                      T, H, dk, dv, num_seqs, dtype, chunk, stream);
+    const size_t need = plan_prefill((long long)B * T, H, dk, num_seqs, KDA_ALGO_TWO_PASS).ws;
+    if (need > KDA_STATIC_WS_BYTES)
+        return fail(KDA_ERR_WORKSPACE,
+                    "these sizes need %zu bytes of two-pass scratch; the built-in scratch holds %zu "
+                    "(KDA_STATIC_WS_BYTES); use kda_chunk_forward_ex with a caller workspace",
+                    need, (size_t)KDA_STATIC_WS_BYTES);
+    if (num_seqs == 0) return KDA_OK;
+    void *ws = nullptr;
+    if (need) {
+        cudaError_t e = cudaSuccess;
+        ws = static_ws_address(&e);
+        if (!ws) return cuda_fail(e, "looking up the built-in scratch (cudaGetSymbolAddress)");
+    }
+    return kda_chunk_forward_ex(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
+                                dv, num_seqs, dtype, chunk, KDA_ALGO_TWO_PASS, ws, need, stream);
 }
 
 int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -150,6 +150,40 @@ int kda_chunk_forward_ex(const void *q, const void *k, const void *v, const floa
                          int dtype, int chunk, int algo, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * kda_chunk_forward_static_ws: the two-pass prefill (KDA_ALGO_TWO_PASS) without a
+ * caller workspace.  It allocates nothing: its scratch is one file-scope device
+ * array of KDA_STATIC_WS_BYTES inside libkda, reserved on each device when the
+ * library's device code is loaded there.  The pages have no counterpart of this
+ * call; it exists for callers that cannot allocate device memory at call time:
+ * code inside a region that forbids allocation (a latency-critical serving loop
+ * that must not enter an allocator, or a stream-ordered section whose allocator
+ * would synchronise), plain-C hosts with no device allocator of their own, and
+ * callers already at their memory limit.
+ *
+ *   arguments     as kda_chunk_forward, without workspace / ws_bytes
+ *   capacity      the two-pass workspace for these sizes
+ *                 (kda_chunk_forward_workspace_size_ex(..., KDA_ALGO_TWO_PASS))
+ *                 must fit in KDA_STATIC_WS_BYTES, else KDA_ERR_WORKSPACE is
+ *                 returned before anything is touched or enqueued
+ *   KDA_F32       takes the fp32 CUDA-core path, which needs no scratch
+ *   zeroing       nothing in the scratch has to start at zero: the first pass
+ *                 writes every record the second pass reads
+ *   first call    on each device, the scratch address is looked up once
+ *                 (cudaGetSymbolAddress); make that first call outside stream
+ *                 capture
+ *   concurrency   all calls on one device share the one scratch array: calls
+ *                 that can overlap in time (different streams, or host threads
+ *                 without ordering) race and corrupt each other's results;
+ *                 order them on one stream
+ */
+#define KDA_STATIC_WS_BYTES ((size_t)64 << 20)
+
+int kda_chunk_forward_static_ws(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, const float *init_state, void *o, float *final_state,
+                                const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv,
+                                int num_seqs, int dtype, int chunk, void *stream);
+
+/*
  * Same contract as kda_chunk_forward, computed entirely on CUDA cores in fp32
  * (inputs in either dtype are widened exactly).  The accuracy reference for the
  * tensor-core path and the path taken for KDA_F32.  Needs no workspace.
