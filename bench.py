@@ -39,6 +39,14 @@ STATE_BYTES = 4 * 128 * 128                                                   # 
 # plus the three C x d^2 state products): 10 C d + 6 d^2.
 PREFILL_FLOPS_PER_TOKEN_HEAD = 10 * CHUNK * 128 + 6 * 128 * 128               # 180224
 DECODE_BYTES_PER_PAIR = 2 * STATE_BYTES + PREFILL_BYTES_PER_TOKEN_HEAD        # 132612
+# DRAM bytes (read + write) per launch from ncu captures of the current kernels on
+# these workloads (profiles/*.md); keyed by the kernels one step runs.  A kernel set
+# without a capture on its workload reports null.
+NCU_TRAFFIC = {
+    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.7e6 + 182.0e6 + 308.3e6 + 54.0e6,
+    ("prefill_8k", "chunk_tc_kernel"): 338.8e6 + 56.0e6,
+    ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.7e6,
+}
 
 
 def _peaks():
@@ -130,6 +138,12 @@ def _barrier(world):
         dist.barrier()
 
 
+def _job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput under weak scaling: every rank processes its own full
+    workload in the step time (already the max over ranks)."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def run_prefill(args, world, rank, dev):
     import torch
 
@@ -140,15 +154,15 @@ def run_prefill(args, world, rank, dev):
     d = prefill_inputs(shape, seed=rank, device=dev)
     o = torch.empty((1, PREFILL["T"], PREFILL["H"], PREFILL["dv"]), dtype=torch.bfloat16, device=dev)
     fs = torch.empty((1, PREFILL["H"], 128, 128), dtype=torch.float32, device=dev)
-    ws_n = kda.workspace_size(1, PREFILL["T"], PREFILL["H"], 128, 128, 1)
+    ws_n = kda.workspace_size(1, PREFILL["T"], PREFILL["H"], 128, 128, 1, algo=args.algo)
     ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev) if ws_n else None
-    # AUTO takes the two-pass schedule (two kernels per call) exactly when it needs a workspace
+    # the two-pass schedule (two kernels per call) is exactly the one that needs a workspace
     kernels = ["chunk_intra_kernel", "chunk_inter_kernel"] if ws_n else ["chunk_tc_kernel"]
     stream = torch.cuda.current_stream(dev)
 
     def step():
         kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], None,
-                          o=o, final_state=fs, workspace=ws)
+                          o=o, final_state=fs, workspace=ws, algo=args.algo)
 
     for _ in range(args.warmup):
         step()
@@ -189,14 +203,14 @@ def run_prefill(args, world, rank, dev):
     fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
     e2e_steps = max(2, min(args.steps, 10))
     kda.chunk_forward(host["q"], host["k"], host["v"], host["log_alpha"], host["beta"], host["init_state"],
-                      None, o=o_h, final_state=fs_h)
+                      None, o=o_h, final_state=fs_h, algo=args.algo)
     _barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
         kda.chunk_forward(host["q"], host["k"], host["v"], host["log_alpha"], host["beta"], host["init_state"],
-                          None, o=o_h, final_state=fs_h)
+                          None, o=o_h, final_state=fs_h, algo=args.algo)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
@@ -316,10 +330,10 @@ def cpu_baseline(heads=32, threads=0):
                       f"prefill_8k (rate scaled to all {PREFILL['H']} heads)"}
 
 
-def config_block():
+def config_block(algo="auto"):
     return {"workload": "prefill_8k", "B": PREFILL["B"], "T": PREFILL["T"], "H": PREFILL["H"],
             "dk": PREFILL["dk"], "dv": PREFILL["dv"], "chunk": CHUNK, "global_batch": PREFILL["B"],
-            "seq_len": PREFILL["T"], "parallelism": "replicas",
+            "seq_len": PREFILL["T"], "parallelism": "replicas", "schedule": algo,
             "l2": "inputs larger than L2 (408 MB per step vs 126 MB)"}
 
 
@@ -358,6 +372,8 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--no-varlen", action="store_true", help="skip the 1M-token packed prefill line")
+    ap.add_argument("--algo", default="auto", choices=["auto", "fused", "two_pass"],
+                    help="tensor-core prefill schedule of the headline line (kda_chunk_forward_ex)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -387,7 +403,7 @@ def main(argv=None):
     hbm_gbs, bf16_tflops, peak_src = _peaks()
     ms_step = pre["total_ms"] / args.steps
     tokens = PREFILL["B"] * PREFILL["T"]
-    value = world * tokens / (ms_step * 1e-3)
+    value = _job_tokens_per_s(world, tokens, ms_step)
     token_heads = tokens * PREFILL["H"]
     alg_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * PREFILL["H"] * STATE_BYTES
     alg_flops = token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD
@@ -398,9 +414,10 @@ def main(argv=None):
         "metric": "KDA chunked prefill tokens/s (B=1, T=8192, H=32, d=128)",
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic", "config": config_block(),
+        "dtype": "bf16", "data": "synthetic", "config": config_block(args.algo),
         "roofline": {"kernel": " + ".join(pre["kernels"]), "bound": "hbm", "achieved": gbs, "peak": hbm_gbs,
-                     "unit": "GB/s", "frac": gbs / hbm_gbs, "traffic": None,
+                     "unit": "GB/s", "frac": gbs / hbm_gbs,
+                     "traffic": NCU_TRAFFIC.get(("prefill_8k", " + ".join(pre["kernels"]))),
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
                      "algorithmic_bytes": alg_bytes, "launch_ms": launch_ms,
                      "tensor": {"achieved_tflops": tflops, "peak_tflops": bf16_tflops,
@@ -420,7 +437,9 @@ def main(argv=None):
             "value": world * DECODE["N"] / (step_ms * 1e-3), "unit": "tokens/s", "ms_per_step": step_ms,
             "steps": dec["launches"], "graph": "1024 steps per CUDA graph replay",
             "roofline": {"kernel": "decode_step_kernel", "bound": "hbm", "achieved": dgbs, "peak": hbm_gbs,
-                         "unit": "GB/s", "frac": dgbs / hbm_gbs, "traffic": None, "algorithmic_bytes": dbytes},
+                         "unit": "GB/s", "frac": dgbs / hbm_gbs,
+                         "traffic": NCU_TRAFFIC.get(("decode_b256", "decode_step_kernel")),
+                         "algorithmic_bytes": dbytes},
             "clocks": dec["clocks"],
         }
         line["gpu_launches"] += dec["launches"]
