@@ -62,7 +62,8 @@ chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
     float *sU = sm + L::u, *sB = sm + L::b, *sD = sm + L::d;
 
     const int tid = threadIdx.x;
-    const int col_base = blockIdx.x * DVT, h = blockIdx.y, n = blockIdx.z;
+    const int col_base = blockIdx.x * DVT, h = blockIdx.y;
+    const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
     long long t0, t1;
     seq_span(cu_seqlens, T, n, t0, t1);
     const long long state_off = ((long long)n * H + h) * DK * DV + col_base;

@@ -302,7 +302,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
-    const int col_base = blockIdx.x * DVT, h = blockIdx.y, n = blockIdx.z;
+    const int col_base = blockIdx.x * DVT, h = blockIdx.y;
+    const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
 
     long long t0, t1;
     seq_span(cu_seqlens, T, n, t0, t1);

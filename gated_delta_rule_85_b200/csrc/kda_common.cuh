@@ -79,4 +79,36 @@ __device__ __forceinline__ void seq_span(const int32_t *cu_seqlens, int T, int n
     }
 }
 
+// Sequence handled by this CTA (grid index z).  Packed inputs of up to 256
+// sequences are taken longest first (z-th longest, ties by index): the hardware
+// starts CTAs roughly in grid order, and starting the longest chains first keeps
+// one long sequence from finishing alone at the end (longest-processing-time-first
+// list scheduling).  Dense batches (equal lengths) and larger counts keep z.
+// Clamped lengths make the ranks a permutation for any cu_seqlens contents.
+// Every thread of the CTA must call it (it synchronises).
+__device__ __forceinline__ int seq_for_cta(const int32_t *cu_seqlens, int T, int num_seqs) {
+    const int z = blockIdx.z;
+    if (!cu_seqlens || num_seqs <= 1 || num_seqs > 256) return z;
+    __shared__ int s_len[256];
+    __shared__ int s_pick;
+    for (int i = threadIdx.x; i < num_seqs; i += blockDim.x) {
+        long long a, b;
+        seq_span(cu_seqlens, T, i, a, b);
+        s_len[i] = (int)(b - a);
+    }
+    if (threadIdx.x == 0) s_pick = z;
+    __syncthreads();
+    for (int n = threadIdx.x; n < num_seqs; n += blockDim.x) {
+        const int ln = s_len[n];
+        int rank = 0;
+        for (int m = 0; m < num_seqs; ++m) {
+            const int lm = s_len[m];
+            rank += (lm > ln) || (lm == ln && m < n);
+        }
+        if (rank == z) s_pick = n;
+    }
+    __syncthreads();
+    return s_pick;
+}
+
 }  // namespace kda
