@@ -259,8 +259,10 @@ def run_prefill_varlen(args, world, rank, dev):
                 seqs=shape.num_seqs, launches=reps * len(kernels), kernels=kernels)
 
 
-def run_decode(args, world, rank, dev):
-    """1024 consecutive decode steps of 256 sequences, captured in one CUDA graph."""
+def run_decode(args, world, rank, dev, pool_slots=0):
+    """1024 consecutive decode steps of 256 sequences, captured in one CUDA graph.
+    With pool_slots > 0 the states live in a pool of that many slots and the
+    sequences use a seeded random choice of them (kda_recurrent_step_slots)."""
     import torch
 
     import gated_delta_rule_85_b200 as kda
@@ -271,10 +273,21 @@ def run_decode(args, world, rank, dev):
     state = d["state"]
     o = torch.empty((DECODE["N"], DECODE["H"], 128), dtype=torch.bfloat16, device=dev)
     S = DECODE["steps"]
+    if pool_slots:
+        g = torch.Generator().manual_seed(1000 + rank)
+        slots = torch.randperm(pool_slots, generator=g)[:DECODE["N"]].to(torch.int32).to(dev)
+        pool = torch.zeros((pool_slots, DECODE["H"], 128, 128), dtype=torch.float32, device=dev)
+        pool[slots.long()] = state
+        del state
+        state = pool
 
     def run_all():
         for s in range(S):
-            kda.recurrent_step(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["beta"][s], state, o=o)
+            if pool_slots:
+                kda.recurrent_step_slots(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["beta"][s], state,
+                                         slots, o=o)
+            else:
+                kda.recurrent_step(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["beta"][s], state, o=o)
 
     side = torch.cuda.Stream(dev)
     side.wait_stream(torch.cuda.current_stream(dev))
@@ -372,6 +385,7 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--no-varlen", action="store_true", help="skip the 1M-token packed prefill line")
+    ap.add_argument("--no-slots", action="store_true", help="skip the state-pool decode line")
     ap.add_argument("--algo", default="auto", choices=["auto", "fused", "two_pass"],
                     help="tensor-core prefill schedule of the headline line (kda_chunk_forward_ex)")
     args = ap.parse_args(argv)
@@ -398,6 +412,7 @@ def main(argv=None):
 
     pre = run_prefill(args, world, rank, dev)
     dec = None if args.no_decode else run_decode(args, world, rank, dev)
+    dsl = None if (args.no_decode or args.no_slots) else run_decode(args, world, rank, dev, pool_slots=512)
     vl = None if args.no_varlen else run_prefill_varlen(args, world, rank, dev)
 
     hbm_gbs, bf16_tflops, peak_src = _peaks()
@@ -443,6 +458,20 @@ def main(argv=None):
             "clocks": dec["clocks"],
         }
         line["gpu_launches"] += dec["launches"]
+    if dsl is not None:
+        step_ms = dsl["ms"] / dsl["launches"]
+        dbytes = DECODE["N"] * DECODE["H"] * DECODE_BYTES_PER_PAIR + DECODE["N"] * 4   # + the slot table
+        dgbs = dbytes / (step_ms * 1e-3) / 1e9
+        line["decode_slots"] = {
+            "metric": "KDA decode tokens/s on a state pool (N=256 sequences in 512 slots, H=32, d=128)",
+            "value": world * DECODE["N"] / (step_ms * 1e-3), "unit": "tokens/s", "ms_per_step": step_ms,
+            "steps": dsl["launches"], "graph": "1024 steps per CUDA graph replay",
+            "roofline": {"kernel": "decode_step_kernel (slot table)", "bound": "hbm", "achieved": dgbs,
+                         "peak": hbm_gbs, "unit": "GB/s", "frac": dgbs / hbm_gbs, "traffic": None,
+                         "algorithmic_bytes": dbytes},
+            "clocks": dsl["clocks"],
+        }
+        line["gpu_launches"] += dsl["launches"]
     if vl is not None:
         vgbs = vl["alg_bytes"] / (vl["ms"] * 1e-3) / 1e9
         vtf = vl["alg_flops"] / (vl["ms"] * 1e-3) / 1e12

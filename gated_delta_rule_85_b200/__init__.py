@@ -20,9 +20,10 @@ import os
 import torch
 
 __all__ = [
-    "chunk_forward", "chunk_forward_simt", "chunk_forward_static_ws", "recurrent_step", "workspace_size", "device_status",
+    "chunk_forward", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
+    "recurrent_step_slots", "workspace_size", "device_status",
     "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
-    "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "ALGOS",
+    "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "DEV_BAD_SLOT", "ALGOS",
 ]
 
 KDA_BF16 = 0
@@ -30,6 +31,7 @@ KDA_F32 = 1
 CHUNK = 64
 DEV_WAIT_TIMEOUT = 0x1
 DEV_DECAY_RANGE = 0x2
+DEV_BAD_SLOT = 0x4
 # tensor-core prefill schedules (KDA_ALGO_* in include/kda.h)
 ALGOS = {"auto": 0, "fused": 1, "two_pass": 2}
 # size of the built-in scratch of kda_chunk_forward_static_ws (KDA_STATIC_WS_BYTES)
@@ -72,6 +74,10 @@ def load_library():
     lib.kda_chunk_forward_workspace_size_ex.restype = sz
     lib.kda_chunk_forward_static_ws.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, ip] + [ci] * 8 + [vp]
     lib.kda_chunk_forward_static_ws.restype = ci
+    lib.kda_chunk_forward_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, ip] + [ci] * 10 + [vp, sz, vp]
+    lib.kda_chunk_forward_slots.restype = ci
+    lib.kda_recurrent_step_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp] + [ci] * 6 + [vp]
+    lib.kda_recurrent_step_slots.restype = ci
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ci] * 5 + [vp]
     lib.kda_recurrent_step.restype = ci
     lib.kda_last_error.argtypes = []
@@ -243,6 +249,57 @@ def recurrent_step(q, k, v, log_alpha, beta, state, o=None):
         o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
     rc = load_library().kda_recurrent_step(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(state), _p(o),
                                            N, H, dk, dv, _dtype_code(q), _stream(q.device))
+    _check(rc)
+    return o
+
+
+def _check_slots(slots, n):
+    if slots.dtype != torch.int32 or slots.shape != (n,) or not slots.is_cuda:
+        raise ValueError(f"slots must be a CUDA int32 tensor of shape ({n},)")
+
+
+def chunk_forward_slots(q, k, v, log_alpha, beta, state_pool, slots, cu_seqlens=None, *, o=None, workspace=None,
+                        algo="auto"):
+    """Prefill from and into a state pool (kda_chunk_forward_slots): sequence n
+    starts from state_pool[slots[n]] and its final state is written back there
+    (slot -1: start from zeros, write nothing).  Device tensors; returns o."""
+    B, T, H, dk, dv, N = _prefill_args(q, k, v, log_alpha, beta, None, cu_seqlens)
+    if state_pool.dim() != 4 or state_pool.shape[1:] != (H, dk, dv) or state_pool.dtype != torch.float32:
+        raise ValueError("state_pool must be float32 [num_slots, H, dk, dv]")
+    _check_slots(slots, N)
+    _need_cuda(q, k, v, log_alpha, beta, state_pool, slots, cu_seqlens)
+    lib = load_library()
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    dt = _dtype_code(q)
+    ac = _algo_code(algo)
+    need = int(lib.kda_chunk_forward_workspace_size_ex(B, T, H, dk, dv, N, dt, CHUNK, ac))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.kda_chunk_forward_slots(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(state_pool), _p(slots),
+                                     _p(o), _p(cu_seqlens), B, T, H, dk, dv, N, state_pool.shape[0], dt, CHUNK,
+                                     ac, _p(workspace), ws_bytes, _stream(q.device))
+    _check(rc)
+    return o
+
+
+def recurrent_step_slots(q, k, v, log_alpha, beta, state_pool, slots, o=None):
+    """One decode step on a state pool (kda_recurrent_step_slots): sequence n uses
+    and updates state_pool[slots[n]] in place (slot -1: padding, o row zero)."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape[:2] != q.shape[:2] or beta.shape != q.shape[:2]:
+        raise ValueError("shape mismatch among q, k, v, log_alpha, beta")
+    if state_pool.dim() != 4 or state_pool.shape[1:] != (H, dk, dv) or state_pool.dtype != torch.float32:
+        raise ValueError("state_pool must be float32 [num_slots, H, dk, dv]")
+    _check_slots(slots, N)
+    _need_cuda(q, k, v, log_alpha, beta, state_pool, slots)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    rc = load_library().kda_recurrent_step_slots(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(state_pool),
+                                                 _p(slots), _p(o), N, H, dk, dv, state_pool.shape[0],
+                                                 _dtype_code(q), _stream(q.device))
     _check(rc)
     return o
 

@@ -364,7 +364,8 @@ template <int DK, int DVT, int NBUF>
 __global__ void __launch_bounds__(NT, 1)
 chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__restrict__ ws,
                    const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
-                   float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
+                   float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV,
+                   const int32_t *__restrict__ slots, int num_slots) {
     using L = InterLayout<DK, DVT, NBUF>;
     using R = Rec<DK>;
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
@@ -414,12 +415,13 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
     const int srow = quad * 32 + lane;
     const bool has_row = srow < DK;
     const int scol = half * CPT;
-    const long long st_off = ((long long)n * H + h) * DK * DV + col_base + scol;
+    const int row = state_row(slots, num_slots, n);
+    const long long st_off = ((long long)(row < 0 ? 0 : row) * H + h) * DK * DV + col_base + scol;
     float S[CPT];
 #pragma unroll
     for (int j = 0; j < CPT; j += 4) {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (has_row && init_state) x = load4(init_state + st_off + (long long)srow * DV + j);
+        if (has_row && init_state && row >= 0) x = load4(init_state + st_off + (long long)srow * DV + j);
         S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
     }
     if (tid == 0)
@@ -528,7 +530,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
     }
 
     __syncthreads();
-    if (ok && final_state && has_row) {
+    if (ok && final_state && has_row && row >= 0) {
 #pragma unroll
         for (int j = 0; j < CPT; j += 4)
             store4(final_state + st_off + (long long)srow * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
@@ -546,16 +548,16 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
 template <int DK, int DVT>
 int launch_two_pass_t(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                       const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
-                      long long tokens, int T, int H, int dv, int num_seqs, void *workspace, cudaStream_t st,
-                      char *msg, size_t msg_len) {
+                      long long tokens, int T, int H, int dv, int num_seqs, const int32_t *slots, int num_slots,
+                      void *workspace, cudaStream_t st, char *msg, size_t msg_len) {
     CUtensorMap tv;
     if (!make_tmap(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, dv, DVT)) {
         snprintf(msg, msg_len, "building TMA descriptors failed (driver entry point cuTensorMapEncodeTiled)");
         return KDA_ERR_CUDA;
     }
-    const long long slots = chunk_slots(tokens, num_seqs);
-    if (slots > 0x7fffffffLL) {
-        snprintf(msg, msg_len, "%lld chunk slots exceed the grid limit", slots);
+    const long long rec_slots = chunk_slots(tokens, num_seqs);   // workspace records per head
+    if (rec_slots > 0x7fffffffLL) {
+        snprintf(msg, msg_len, "%lld chunk slots exceed the grid limit", rec_slots);
         return KDA_ERR_UNSUPPORTED;
     }
     constexpr int smem1 = IntraLayout<DK>::ALLOC;
@@ -565,7 +567,7 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_intra): %s", cudaGetErrorString(e));
         return KDA_ERR_CUDA;
     }
-    k1<<<dim3((unsigned)slots, H), NT, smem1, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
+    k1<<<dim3((unsigned)rec_slots, H), NT, smem1, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
                                                      beta, cu_seqlens, T, H, num_seqs, (uint8_t *)workspace);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
@@ -582,7 +584,8 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         return KDA_ERR_CUDA;
     }
     k2<<<dim3(dv / DVT, H, num_seqs), NT, smem2, st>>>(tv, (const uint8_t *)workspace, init_state,
-                                                        (__nv_bfloat16 *)o, final_state, cu_seqlens, T, H, dv);
+                                                        (__nv_bfloat16 *)o, final_state, cu_seqlens, T, H, dv,
+                                                        slots, num_slots);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "chunk_inter launch: %s", cudaGetErrorString(e));
@@ -593,8 +596,8 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
 
 inline int launch_two_pass(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                            const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
-                           long long tokens, int T, int H, int dk, int dv, int num_seqs, void *workspace,
-                           cudaStream_t st, char *msg, size_t msg_len) {
+                           long long tokens, int T, int H, int dk, int dv, int num_seqs, const int32_t *slots,
+                           int num_slots, void *workspace, cudaStream_t st, char *msg, size_t msg_len) {
     // value-tile width of the recurrence pass: the widest that still gives one CTA per SM
     const long long chains = (long long)num_seqs * H;
     int dvt = 32;
@@ -602,7 +605,7 @@ inline int launch_two_pass(const void *q, const void *k, const void *v, const fl
         if (chains * (dv / cand) >= 148) { dvt = cand; break; }
 #define KDA_2P(DKv, DVTv)                                                                                        \
     return launch_two_pass_t<DKv, DVTv>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, \
-                                        T, H, dv, num_seqs, workspace, st, msg, msg_len)
+                                        T, H, dv, num_seqs, slots, num_slots, workspace, st, msg, msg_len)
     if (dk == 128) {
         if (dvt == 128) KDA_2P(128, 128);
         if (dvt == 64) KDA_2P(128, 64);

@@ -52,7 +52,7 @@ chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
                   const float *__restrict__ init_state, Tin *__restrict__ o,
                   float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens, int T, int H,
-                  int DV) {
+                  int DV, const int32_t *__restrict__ slots, int num_slots) {
     using namespace simt;
     using L = Smem<DK>;
     constexpr int DKP = L::DKP, CP = L::CP;
@@ -66,11 +66,12 @@ chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
     const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
     long long t0, t1;
     seq_span(cu_seqlens, T, n, t0, t1);
-    const long long state_off = ((long long)n * H + h) * DK * DV + col_base;
+    const int row = state_row(slots, num_slots, n);
+    const long long state_off = ((long long)(row < 0 ? 0 : row) * H + h) * DK * DV + col_base;
 
     for (int idx = tid; idx < DK * DVT; idx += NT) {
         const int c = idx / DVT, j = idx % DVT;
-        sS[idx] = init_state ? init_state[state_off + (long long)c * DV + j] : 0.f;
+        sS[idx] = (init_state && row >= 0) ? init_state[state_off + (long long)c * DV + j] : 0.f;
     }
 
     for (long long cs = t0; cs < t1; cs += C) {
@@ -187,7 +188,7 @@ chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
         }
     }
     __syncthreads();
-    if (final_state) {
+    if (final_state && row >= 0) {
         for (int idx = tid; idx < DK * DVT; idx += NT) {
             const int c = idx / DVT, j = idx % DVT;
             final_state[state_off + (long long)c * DV + j] = sS[idx];

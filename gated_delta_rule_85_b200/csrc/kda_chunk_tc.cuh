@@ -282,7 +282,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                 const float *__restrict__ beta, const float *__restrict__ init_state,
                 __nv_bfloat16 *__restrict__ o, float *__restrict__ final_state,
-                const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
+                const int32_t *__restrict__ cu_seqlens, int T, int H, int DV, const int32_t *__restrict__ slots,
+                int num_slots) {
     using L = Layout<DK, DVT>;
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
     constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG;   // factor stage: 4 channels x SEGLEN tokens
@@ -348,12 +349,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int srow = quad * 32 + lane;
     const bool has_row = srow < DK;
     const int scol = half * CPT;
-    const long long st_off = ((long long)n * H + h) * DK * DV + col_base + scol;
+    const int row = state_row(slots, num_slots, n);
+    const long long st_off = ((long long)(row < 0 ? 0 : row) * H + h) * DK * DV + col_base + scol;
     float S[CPT];
 #pragma unroll
     for (int j = 0; j < CPT; j += 4) {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (has_row && init_state) x = load4(init_state + st_off + (long long)srow * DV + j);
+        if (has_row && init_state && row >= 0) x = load4(init_state + st_off + (long long)srow * DV + j);
         S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
     }
     if (nck > 0) {
@@ -644,7 +646,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 
     __syncthreads();
-    if (ok && final_state && has_row) {
+    if (ok && final_state && has_row && row >= 0) {
 #pragma unroll
         for (int j = 0; j < CPT; j += 4)
             store4(final_state + st_off + (long long)srow * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
@@ -692,7 +694,8 @@ inline bool make_tmap(CUtensorMap *m, const void *base, CUtensorMapDataType dt, 
 template <int DK, int DVT>
 int launch_t(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
              const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, long long tokens,
-             int T, int H, int dv, int num_seqs, cudaStream_t st, char *msg, size_t msg_len) {
+             int T, int H, int dv, int num_seqs, const int32_t *slots, int num_slots, cudaStream_t st, char *msg,
+             size_t msg_len) {
     CUtensorMap tq, tk, tg, tv;
     if (!make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DK, DK) ||
         !make_tmap(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DK, DK) ||
@@ -710,7 +713,7 @@ int launch_t(const void *q, const void *k, const void *v, const float *log_alpha
     }
     dim3 grid(dv / DVT, H, num_seqs);
     kern<<<grid, NT, smem, st>>>(tq, tk, tg, tv, beta, init_state, (__nv_bfloat16 *)o, final_state, cu_seqlens,
-                                  T, H, dv);
+                                  T, H, dv, slots, num_slots);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "chunk_tc launch: %s", cudaGetErrorString(e));
@@ -735,8 +738,8 @@ inline int state_passthrough(const float *init_state, float *final_state, int nu
 
 inline int launch_fused(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                         const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
-                        long long tokens, int T, int H, int dk, int dv, int num_seqs, cudaStream_t st, char *msg,
-                        size_t msg_len) {
+                        long long tokens, int T, int H, int dk, int dv, int num_seqs, const int32_t *slots,
+                        int num_slots, cudaStream_t st, char *msg, size_t msg_len) {
     // Value-tile width: the widest tile (fewest duplicated per-chunk operand
     // builds) that still gives at least two CTAs per SM; else 32 columns.
     const long long chains = (long long)num_seqs * H;
@@ -745,7 +748,7 @@ inline int launch_fused(const void *q, const void *k, const void *v, const float
         if (chains * (dv / cand) >= 2 * 148) { dvt = cand; break; }
 #define KDA_TC(DKv, DVTv)                                                                                   \
     return launch_t<DKv, DVTv>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T, \
-                               H, dv, num_seqs, st, msg, msg_len)
+                               H, dv, num_seqs, slots, num_slots, st, msg, msg_len)
     if (dk == 128) {
         if (dvt == 128) KDA_TC(128, 128);
         if (dvt == 64) KDA_TC(128, 64);

@@ -79,6 +79,19 @@ __device__ __forceinline__ void seq_span(const int32_t *cu_seqlens, int T, int n
     }
 }
 
+// State row of sequence n: slots[n] when a slot table is given, n otherwise.
+// -1 means "no state": start from zeros and write nothing back.  Entries outside
+// [-1, num_slots) flag KDA_DEV_BAD_SLOT and count as -1.  Uniform over the CTA.
+__device__ __forceinline__ int state_row(const int32_t *slots, int num_slots, int n) {
+    if (!slots) return n;
+    const int s = slots[n];
+    if (s < -1 || s >= num_slots) {
+        if (threadIdx.x == 0) flag_status(KDA_DEV_BAD_SLOT);
+        return -1;
+    }
+    return s;
+}
+
 // Sequence handled by this CTA (grid index z).  Packed inputs of up to 256
 // sequences are taken longest first (z-th longest, ties by index): the hardware
 // starts CTAs roughly in grid order, and starting the longest chains first keeps

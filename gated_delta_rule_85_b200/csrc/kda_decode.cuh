@@ -21,7 +21,8 @@ template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                    const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                   float *__restrict__ state, Tin *__restrict__ o) {
+                   float *__restrict__ state, Tin *__restrict__ o, const int32_t *__restrict__ slots,
+                   int num_slots, int H) {
     constexpr int NSTRIPE = DV / 32;          // 32-column stripes
     constexpr int RG = 8 / NSTRIPE;           // row groups (warps per stripe)
     constexpr int ROWS_PER_GROUP = DK / RG;
@@ -39,7 +40,13 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
     __shared__ float s_red[RG][2][DV];
     __shared__ float s_qk[8];
 
-    float *S = state + pair * (long long)(DK * DV);
+    // state of this (sequence, head): row n, or its slot in a state pool
+    const int row = state_row(slots, num_slots, (int)(pair / H));
+    if (row < 0) {   // no state: a padding entry; its output row is zero
+        if (rg == 0 && rl == 0) store4(o + pair * DV + col0, make_float4(0.f, 0.f, 0.f, 0.f));
+        return;
+    }
+    float *S = state + ((long long)row * H + pair % H) * (long long)(DK * DV);
 
     // The state dominates the traffic: put all of this thread's loads in flight first.
     float4 s[RPT];

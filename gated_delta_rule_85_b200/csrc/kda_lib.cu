@@ -108,14 +108,15 @@ void *static_ws_address(cudaError_t *err) {
 template <int DK, typename Tin>
 int launch_simt(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                 const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int T,
-                int H, int dv, int num_seqs, cudaStream_t st) {
+                int H, int dv, int num_seqs, const int32_t *slots, int num_slots, cudaStream_t st) {
     constexpr size_t smem = kda::simt::Smem<DK>::bytes;
     auto kern = kda::chunk_simt_kernel<DK, Tin>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chunk_simt)");
     dim3 grid(dv / kda::simt::DVT, H, num_seqs);
     kern<<<grid, kda::simt::NT, smem, st>>>((const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta,
-                                             init_state, (Tin *)o, final_state, cu_seqlens, T, H, dv);
+                                             init_state, (Tin *)o, final_state, cu_seqlens, T, H, dv, slots,
+                                             num_slots);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "chunk_simt launch");
     return KDA_OK;
@@ -123,12 +124,99 @@ int launch_simt(const void *q, const void *k, const void *v, const float *log_al
 
 template <int DK, int DV, typename Tin>
 int launch_decode(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
-                  float *state, void *o, long long pairs, cudaStream_t st) {
+                  float *state, void *o, long long pairs, const int32_t *slots, int num_slots, int H,
+                  cudaStream_t st) {
     kda::decode_step_kernel<DK, DV, Tin><<<(unsigned)pairs, 256, 0, st>>>(
-        (const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta, state, (Tin *)o);
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta, state, (Tin *)o, slots, num_slots, H);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
     return KDA_OK;
+}
+
+// The fp32 CUDA-core prefill after argument checks; `slots` (or NULL) maps
+// sequences to state rows.
+int simt_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+              const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int T, int H,
+              int dk, int dv, int num_seqs, int dtype, const int32_t *slots, int num_slots, cudaStream_t st) {
+    if (num_seqs == 0) return KDA_OK;
+    if (dtype == KDA_BF16) {
+        if (dk == 64)
+            return launch_simt<64, __nv_bfloat16>(q, k, v, log_alpha, beta, init_state, o, final_state,
+                                                  cu_seqlens, T, H, dv, num_seqs, slots, num_slots, st);
+        return launch_simt<128, __nv_bfloat16>(q, k, v, log_alpha, beta, init_state, o, final_state,
+                                               cu_seqlens, T, H, dv, num_seqs, slots, num_slots, st);
+    }
+    if (dk == 64)
+        return launch_simt<64, float>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T,
+                                      H, dv, num_seqs, slots, num_slots, st);
+    return launch_simt<128, float>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H,
+                                   dv, num_seqs, slots, num_slots, st);
+}
+
+// The tensor-core prefill after argument checks (dtype KDA_BF16, algo valid).
+int prefill_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                 const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int B, int T,
+                 int H, int dk, int dv, int num_seqs, int algo, const int32_t *slots, int num_slots,
+                 void *workspace, size_t ws_bytes, cudaStream_t st) {
+    const long long tokens = (long long)B * T;
+    const Plan plan = plan_prefill(tokens, H, dk, num_seqs, algo);
+    if (plan.ws && (!workspace || ws_bytes < plan.ws))
+        return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", plan.ws, ws_bytes);
+    if (workspace && !aligned(workspace, 256)) return fail(KDA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (num_seqs == 0) return KDA_OK;
+    if (tokens > 0x7fffffffLL)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T=%lld exceeds the 2^31 token limit of the TMA coordinates", tokens);
+    char msg[256] = "";
+    int rc;
+    if (tokens == 0)
+        rc = slots ? KDA_OK   // states stay in their slots
+                   : kda::tc::state_passthrough(init_state, final_state, num_seqs, H, dk, dv, st, msg, sizeof(msg));
+    else if (plan.algo == KDA_ALGO_TWO_PASS)
+        rc = kda::tc::launch_two_pass(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T,
+                                      H, dk, dv, num_seqs, slots, num_slots, workspace, st, msg, sizeof(msg));
+    else
+        rc = kda::tc::launch_fused(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T, H,
+                                   dk, dv, num_seqs, slots, num_slots, st, msg, sizeof(msg));
+    if (rc) return fail(rc, "%s", msg);
+    return KDA_OK;
+}
+
+// Decode argument checks shared by both decode entry points.
+int check_decode(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                 const float *state, const void *o, int N, int H, int dk, int dv, int dtype) {
+    if (N < 0 || H < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d", N, H);
+    if (N == 0) return KDA_OK;   // nothing to do; empty tensors may carry NULL pointers
+    if (!q || !k || !v || !log_alpha || !beta || !state || !o)
+        return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta, state and o are required");
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+        return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: each must be 64 or 128", dk, dv);
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "dtype=%d", dtype);
+    const void *p16[] = {q, k, v, log_alpha, o, state};
+    const char *n16[] = {"q", "k", "v", "log_alpha", "o", "state"};
+    for (int i = 0; i < 6; ++i)
+        if (!aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
+    if (!aligned(beta, 4)) return fail(KDA_ERR_MISALIGNED, "beta is not 4-byte aligned");
+    if ((long long)N * H > 0x7fffffffLL) return fail(KDA_ERR_UNSUPPORTED, "N*H=%lld too large", (long long)N * H);
+    return KDA_OK;
+}
+
+int decode_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                float *state, void *o, int N, int H, int dk, int dv, int dtype, const int32_t *slots,
+                int num_slots, cudaStream_t st) {
+    const long long pairs = (long long)N * H;
+    if (pairs == 0) return KDA_OK;
+#define KDA_DEC(DKv, DVv)                                                                                     \
+    if (dk == DKv && dv == DVv)                                                                               \
+        return dtype == KDA_BF16 ? launch_decode<DKv, DVv, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o, \
+                                                                          pairs, slots, num_slots, H, st)     \
+                                 : launch_decode<DKv, DVv, float>(q, k, v, log_alpha, beta, state, o, pairs,  \
+                                                                  slots, num_slots, H, st);
+    KDA_DEC(64, 64)
+    KDA_DEC(64, 128)
+    KDA_DEC(128, 64)
+    KDA_DEC(128, 128)
+#undef KDA_DEC
+    return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d", dk, dv);
 }
 
 }  // namespace
@@ -158,20 +246,8 @@ int kda_chunk_forward_simt(const void *q, const void *k, const void *v, const fl
     int rc = check_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
                            dv, num_seqs, dtype, chunk);
     if (rc) return rc;
-    if (num_seqs == 0) return KDA_OK;
-    cudaStream_t st = (cudaStream_t)stream;
-    if (dtype == KDA_BF16) {
-        if (dk == 64)
-            return launch_simt<64, __nv_bfloat16>(q, k, v, log_alpha, beta, init_state, o, final_state,
-                                                  cu_seqlens, T, H, dv, num_seqs, st);
-        return launch_simt<128, __nv_bfloat16>(q, k, v, log_alpha, beta, init_state, o, final_state,
-                                               cu_seqlens, T, H, dv, num_seqs, st);
-    }
-    if (dk == 64)
-        return launch_simt<64, float>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T,
-                                      H, dv, num_seqs, st);
-    return launch_simt<128, float>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H,
-                                   dv, num_seqs, st);
+    return simt_impl(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H, dk, dv, num_seqs,
+                     dtype, nullptr, 0, (cudaStream_t)stream);
 }
 
 int kda_chunk_forward_ex(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -184,28 +260,31 @@ int kda_chunk_forward_ex(const void *q, const void *k, const void *v, const floa
     if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_FUSED && algo != KDA_ALGO_TWO_PASS)
         return fail(KDA_ERR_INVALID_ARG, "algo=%d is not a KDA_ALGO_* value", algo);
     if (dtype == KDA_F32)
-        return kda_chunk_forward_simt(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B,
-                                      T, H, dk, dv, num_seqs, dtype, chunk, stream);
-    const long long tokens = (long long)B * T;
-    const Plan plan = plan_prefill(tokens, H, dk, num_seqs, algo);
-    if (plan.ws && (!workspace || ws_bytes < plan.ws))
-        return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", plan.ws, ws_bytes);
-    if (workspace && !aligned(workspace, 256)) return fail(KDA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
-    if (num_seqs == 0) return KDA_OK;
-    if (tokens > 0x7fffffffLL)
-        return fail(KDA_ERR_UNSUPPORTED, "B*T=%lld exceeds the 2^31 token limit of the TMA coordinates", tokens);
-    char msg[256] = "";
-    cudaStream_t st = (cudaStream_t)stream;
-    if (tokens == 0)
-        rc = kda::tc::state_passthrough(init_state, final_state, num_seqs, H, dk, dv, st, msg, sizeof(msg));
-    else if (plan.algo == KDA_ALGO_TWO_PASS)
-        rc = kda::tc::launch_two_pass(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T,
-                                      H, dk, dv, num_seqs, workspace, st, msg, sizeof(msg));
-    else
-        rc = kda::tc::launch_fused(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T, H,
-                                   dk, dv, num_seqs, st, msg, sizeof(msg));
-    if (rc) return fail(rc, "%s", msg);
-    return KDA_OK;
+        return simt_impl(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H, dk, dv,
+                         num_seqs, dtype, nullptr, 0, (cudaStream_t)stream);
+    return prefill_impl(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk, dv,
+                        num_seqs, algo, nullptr, 0, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+int kda_chunk_forward_slots(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, float *state_pool, const int32_t *slots, void *o,
+                            const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                            int num_slots, int dtype, int chunk, int algo, void *workspace, size_t ws_bytes,
+                            void *stream) {
+    int rc = check_prefill(q, k, v, log_alpha, beta, state_pool, o, state_pool, cu_seqlens, B, T, H, dk, dv,
+                           num_seqs, dtype, chunk);
+    if (rc) return rc;
+    if (num_seqs > 0 && (!state_pool || !slots))
+        return fail(KDA_ERR_INVALID_ARG, "state_pool and slots are required");
+    if (num_slots < 1) return fail(KDA_ERR_INVALID_ARG, "num_slots=%d must be at least 1", num_slots);
+    if (slots && !aligned(slots, 4)) return fail(KDA_ERR_MISALIGNED, "slots is not 4-byte aligned");
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_FUSED && algo != KDA_ALGO_TWO_PASS)
+        return fail(KDA_ERR_INVALID_ARG, "algo=%d is not a KDA_ALGO_* value", algo);
+    if (dtype == KDA_F32)
+        return simt_impl(q, k, v, log_alpha, beta, state_pool, o, state_pool, cu_seqlens, T, H, dk, dv,
+                         num_seqs, dtype, slots, num_slots, (cudaStream_t)stream);
+    return prefill_impl(q, k, v, log_alpha, beta, state_pool, o, state_pool, cu_seqlens, B, T, H, dk, dv,
+                        num_seqs, algo, slots, num_slots, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
 int kda_chunk_forward(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -246,33 +325,21 @@ int kda_chunk_forward_static_ws(const void *q, const void *k, const void *v, con
 int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,
                        const float *beta, float *state, void *o, int N, int H, int dk, int dv, int dtype,
                        void *stream) {
-    if (N < 0 || H < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d", N, H);
-    if (N == 0) return KDA_OK;   // nothing to do; empty tensors may carry NULL pointers
-    if (!q || !k || !v || !log_alpha || !beta || !state || !o)
-        return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta, state and o are required");
-    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
-        return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: each must be 64 or 128", dk, dv);
-    if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "dtype=%d", dtype);
-    const void *p16[] = {q, k, v, log_alpha, o, state};
-    const char *n16[] = {"q", "k", "v", "log_alpha", "o", "state"};
-    for (int i = 0; i < 6; ++i)
-        if (!aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
-    if (!aligned(beta, 4)) return fail(KDA_ERR_MISALIGNED, "beta is not 4-byte aligned");
-    const long long pairs = (long long)N * H;
-    if (pairs == 0) return KDA_OK;
-    if (pairs > 0x7fffffffLL) return fail(KDA_ERR_UNSUPPORTED, "N*H=%lld too large", pairs);
-    cudaStream_t st = (cudaStream_t)stream;
-#define KDA_DEC(DKv, DVv)                                                                              \
-    if (dk == DKv && dv == DVv)                                                                        \
-        return dtype == KDA_BF16                                                                       \
-                   ? launch_decode<DKv, DVv, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o, pairs, st) \
-                   : launch_decode<DKv, DVv, float>(q, k, v, log_alpha, beta, state, o, pairs, st);
-    KDA_DEC(64, 64)
-    KDA_DEC(64, 128)
-    KDA_DEC(128, 64)
-    KDA_DEC(128, 128)
-#undef KDA_DEC
-    return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d", dk, dv);
+    int rc = check_decode(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype);
+    if (rc || N == 0) return rc;
+    return decode_impl(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype, nullptr, 0, (cudaStream_t)stream);
+}
+
+int kda_recurrent_step_slots(const void *q, const void *k, const void *v, const float *log_alpha,
+                             const float *beta, float *state_pool, const int32_t *slots, void *o, int N, int H,
+                             int dk, int dv, int num_slots, int dtype, void *stream) {
+    int rc = check_decode(q, k, v, log_alpha, beta, state_pool, o, N, H, dk, dv, dtype);
+    if (rc || N == 0) return rc;
+    if (!slots) return fail(KDA_ERR_INVALID_ARG, "slots is required");
+    if (!aligned(slots, 4)) return fail(KDA_ERR_MISALIGNED, "slots is not 4-byte aligned");
+    if (num_slots < 1) return fail(KDA_ERR_INVALID_ARG, "num_slots=%d must be at least 1", num_slots);
+    return decode_impl(q, k, v, log_alpha, beta, state_pool, o, N, H, dk, dv, dtype, slots, num_slots,
+                       (cudaStream_t)stream);
 }
 
 int kda_get_device_status(unsigned int *bits, int clear, void *stream) {

@@ -79,6 +79,8 @@ typedef enum kda_dtype {
 #define KDA_DEV_DECAY_RANGE 0x2u     /* tensor-core prefill: within one 64-token chunk a channel's
                                         accumulated log-decay fell below -80; the factorised decay
                                         operands lose range there (see kda_chunk_forward) */
+#define KDA_DEV_BAD_SLOT 0x4u        /* a state-slot table entry was outside [-1, num_slots); that
+                                        sequence was treated as having no slot (see *_slots) */
 
 /*
  * Chunked prefill, 64-token chunks.
@@ -207,6 +209,37 @@ int kda_chunk_forward_simt(const void *q, const void *k, const void *v, const fl
 int kda_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,
                        const float *beta, float *state, void *o, int N, int H, int dk, int dv,
                        int dtype, void *stream);
+
+/*
+ * State slots: the states live in a pool and each sequence names its slot, the
+ * layout serving stacks use for batched decode with continuous batching and for
+ * prefix caching (a prefill that resumes from a cached prefix state).  Sources:
+ * "Kimi Linear、独自の土俵でFull Attentionを上回る" (remio.ai), § "オープンコードに
+ * より主張は検証可能になる一方、ソフトウェアスタックはリスクを加える" (batched
+ * decode, prefix caching and state across chunk boundaries as the behaviour to
+ * test) and § "Kimi Linearリリース後に注目すべき点" (prefix reuse, continuous
+ * batching); "Kimi Linearは広がりつつある…" (orcarouter.ai), § "既に起こった採用は
+ * サービングスタックの中にあります" (KDA prefix caching in serving stacks).
+ *
+ *   state_pool   fp32 [num_slots, H, dk, dv] (dv contiguous), updated in place
+ *   slots        int32 [N] device array: slot of sequence n, or -1 for "no state"
+ *                (prefill: start from zeros and write nothing back; decode: a
+ *                padding row whose output is zero).  Entries outside
+ *                [-1, num_slots) set KDA_DEV_BAD_SLOT and count as -1.  Two
+ *                sequences must not name the same slot in one call (their
+ *                updates would race).
+ * Everything else is as in kda_chunk_forward_ex / kda_recurrent_step; the
+ * workspace is kda_chunk_forward_workspace_size_ex's for the same sizes and algo.
+ */
+int kda_chunk_forward_slots(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, float *state_pool, const int32_t *slots, void *o,
+                            const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                            int num_slots, int dtype, int chunk, int algo, void *workspace, size_t ws_bytes,
+                            void *stream);
+
+int kda_recurrent_step_slots(const void *q, const void *k, const void *v, const float *log_alpha,
+                             const float *beta, float *state_pool, const int32_t *slots, void *o, int N, int H,
+                             int dk, int dv, int num_slots, int dtype, void *stream);
 
 /* Message for the calling thread's last non-OK return ("" if none). */
 const char *kda_last_error(void);

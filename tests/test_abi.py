@@ -146,3 +146,19 @@ def test_static_ws_rejects_oversize_before_touching_the_device(lib):
     msg = lib.kda_last_error().decode()
     assert "KDA_STATIC_WS_BYTES" in msg and "kda_chunk_forward_ex" in msg
     assert lib.kda_chunk_forward_workspace_size_ex(1, T, 32, 128, 128, 1, 0, 64, 2) > kda.STATIC_WS_BYTES
+
+
+def test_slot_entry_points_reject(lib):
+    pre = lambda slots, num_slots, align=0: lib.kda_chunk_forward_slots(
+        A[0], A[1], A[2], A[3], A[4], A[5], slots, A[6], None, 1, 128, 2, 128, 128, 1, num_slots, 0, 64, 0,
+        A[8], 1 << 24, None)
+    assert pre(None, 4) == INVALID                 # slot table missing
+    assert pre(A[9], 0) == INVALID                 # empty pool
+    assert pre(A[9] + 2, 4) == MISALIGNED          # slot table below 4-byte alignment
+    dec = lambda slots, num_slots: lib.kda_recurrent_step_slots(
+        A[0], A[1], A[2], A[3], A[4], A[5], slots, A[6], 4, 2, 128, 128, num_slots, 0, None)
+    assert dec(None, 8) == INVALID
+    assert dec(A[9], 0) == INVALID
+    assert dec(A[9] + 1, 8) == MISALIGNED
+    assert lib.kda_recurrent_step_slots(A[0], A[1], A[2], A[3], A[4], A[5], A[9], A[6], 0, 2, 128, 128, 8, 0,
+                                        None) == OK   # no sequences: nothing to do
