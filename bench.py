@@ -219,6 +219,42 @@ def run_prefill(args, world, rank, dev):
                 h2d=h2d, d2h=d2h, e2e_steps=e2e_steps, kernels=kernels)
 
 
+def run_prefill_gdn(args, world, rank, dev):
+    """prefill_8k with a Gated DeltaNet scalar gate (kda_gdn_chunk_forward), CUDA events per call."""
+    import torch
+
+    import gated_delta_rule_85_b200 as kda
+    from gated_delta_rule_85_b200.workloads import PrefillShape, prefill_inputs
+
+    shape = PrefillShape(**PREFILL, dtype=torch.bfloat16, gate="scalar")
+    d = prefill_inputs(shape, seed=rank, device=dev)
+    o = torch.empty((1, PREFILL["T"], PREFILL["H"], PREFILL["dv"]), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, PREFILL["H"], 128, 128), dtype=torch.float32, device=dev)
+    ws_n = kda.workspace_size(1, PREFILL["T"], PREFILL["H"], 128, 128, 1)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev) if ws_n else None
+
+    def step():
+        kda.gdn_chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], o=o,
+                              final_state=fs, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    reps = max(5, min(args.steps, 50))
+    _barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    del d
+    return dict(ms=ms, launches=reps * (2 if ws_n else 1))
+
+
 def run_prefill_varlen(args, world, rank, dev):
     """The 1,048,576-token packed (varlen) prefill: 22 sequences x 32 heads."""
     import torch
@@ -386,6 +422,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--no-varlen", action="store_true", help="skip the 1M-token packed prefill line")
     ap.add_argument("--no-slots", action="store_true", help="skip the state-pool decode line")
+    ap.add_argument("--no-gdn", action="store_true", help="skip the Gated DeltaNet (scalar gate) prefill line")
     ap.add_argument("--algo", default="auto", choices=["auto", "fused", "two_pass"],
                     help="tensor-core prefill schedule of the headline line (kda_chunk_forward_ex)")
     args = ap.parse_args(argv)
@@ -414,6 +451,7 @@ def main(argv=None):
     dec = None if args.no_decode else run_decode(args, world, rank, dev)
     dsl = None if (args.no_decode or args.no_slots) else run_decode(args, world, rank, dev, pool_slots=512)
     vl = None if args.no_varlen else run_prefill_varlen(args, world, rank, dev)
+    gd = None if args.no_gdn else run_prefill_gdn(args, world, rank, dev)
 
     hbm_gbs, bf16_tflops, peak_src = _peaks()
     ms_step = pre["total_ms"] / args.steps
@@ -458,6 +496,19 @@ def main(argv=None):
             "clocks": dec["clocks"],
         }
         line["gpu_launches"] += dec["launches"]
+    if gd is not None:
+        gbytes = token_heads * (PREFILL_BYTES_PER_TOKEN_HEAD - 4 * 128 + 4) + 2 * PREFILL["H"] * STATE_BYTES
+        ggbs = gbytes / (gd["ms"] * 1e-3) / 1e9
+        gtf = alg_flops / (gd["ms"] * 1e-3) / 1e12
+        line["prefill_gdn_8k"] = {
+            "metric": "Gated DeltaNet (scalar gate) chunked prefill tokens/s (B=1, T=8192, H=32, d=128)",
+            "value": world * tokens / (gd["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": gd["ms"],
+            "roofline": {"kernel": "chunk_intra_kernel + chunk_inter_kernel (scalar gate)", "bound": "hbm",
+                         "achieved": ggbs, "peak": hbm_gbs, "unit": "GB/s", "frac": ggbs / hbm_gbs, "traffic": None,
+                         "algorithmic_bytes": gbytes,
+                         "tensor": {"achieved_tflops": gtf, "peak_tflops": bf16_tflops, "frac": gtf / bf16_tflops}},
+        }
+        line["gpu_launches"] += gd["launches"]
     if dsl is not None:
         step_ms = dsl["ms"] / dsl["launches"]
         dbytes = DECODE["N"] * DECODE["H"] * DECODE_BYTES_PER_PAIR + DECODE["N"] * 4   # + the slot table

@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "chunk_forward", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
-    "recurrent_step_slots", "workspace_size", "device_status",
+    "recurrent_step_slots", "gdn_chunk_forward", "gdn_recurrent_step", "workspace_size", "device_status",
     "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
     "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "DEV_BAD_SLOT", "ALGOS",
 ]
@@ -78,6 +78,10 @@ def load_library():
     lib.kda_chunk_forward_slots.restype = ci
     lib.kda_recurrent_step_slots.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp] + [ci] * 6 + [vp]
     lib.kda_recurrent_step_slots.restype = ci
+    lib.kda_gdn_chunk_forward.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, ip] + [ci] * 9 + [vp, sz, vp]
+    lib.kda_gdn_chunk_forward.restype = ci
+    lib.kda_gdn_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ci] * 5 + [vp]
+    lib.kda_gdn_recurrent_step.restype = ci
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ci] * 5 + [vp]
     lib.kda_recurrent_step.restype = ci
     lib.kda_last_error.argtypes = []
@@ -300,6 +304,52 @@ def recurrent_step_slots(q, k, v, log_alpha, beta, state_pool, slots, o=None):
     rc = load_library().kda_recurrent_step_slots(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(state_pool),
                                                  _p(slots), _p(o), N, H, dk, dv, state_pool.shape[0],
                                                  _dtype_code(q), _stream(q.device))
+    _check(rc)
+    return o
+
+
+def gdn_chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, o=None, final_state=True,
+                      workspace=None, algo="auto"):
+    """Gated DeltaNet prefill (kda_gdn_chunk_forward): log_alpha is one scalar per
+    (token, head), shape [B, T, H].  Device tensors; returns (o, final_state or None)."""
+    B, T, H, dk = q.shape
+    if log_alpha.shape != q.shape[:3] or log_alpha.dtype != torch.float32:
+        raise ValueError("log_alpha must be float32 [B, T, H] for the scalar gate")
+    _, _, _, _, dv, N = _prefill_args(q, k, v, log_alpha.unsqueeze(-1).expand(q.shape), beta, init_state, cu_seqlens)
+    _need_cuda(q, k, v, log_alpha, beta, init_state, cu_seqlens)
+    lib = load_library()
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is True:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    elif final_state is False:
+        final_state = None
+    dt = _dtype_code(q)
+    ac = _algo_code(algo)
+    need = int(lib.kda_chunk_forward_workspace_size_ex(B, T, H, dk, dv, N, dt, CHUNK, ac))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.kda_gdn_chunk_forward(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(o),
+                                   _p(final_state), _p(cu_seqlens), B, T, H, dk, dv, N, dt, CHUNK, ac,
+                                   _p(workspace), ws_bytes, _stream(q.device))
+    _check(rc)
+    return o, final_state
+
+
+def gdn_recurrent_step(q, k, v, log_alpha, beta, state, o=None):
+    """One Gated DeltaNet decode step (kda_gdn_recurrent_step); log_alpha [N, H]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if log_alpha.shape != q.shape[:2] or log_alpha.dtype != torch.float32:
+        raise ValueError("log_alpha must be float32 [N, H] for the scalar gate")
+    if state.shape != (N, H, dk, dv) or state.dtype != torch.float32:
+        raise ValueError("state must be float32 [N, H, dk, dv]")
+    _need_cuda(q, k, v, log_alpha, beta, state)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    rc = load_library().kda_gdn_recurrent_step(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(state), _p(o),
+                                               N, H, dk, dv, _dtype_code(q), _stream(q.device))
     _check(rc)
     return o
 

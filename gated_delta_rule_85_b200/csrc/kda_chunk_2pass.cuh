@@ -91,7 +91,8 @@ __device__ __forceinline__ void st_global_bf16x8(uint8_t *p, const float *x) {
         make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
 }
 
-template <int DK>
+// GS: scalar gate, log_alpha [tokens, H] (Gated DeltaNet), else [tokens, H, DK].
+template <int DK, bool GS>
 __global__ void __launch_bounds__(NT, 2)
 chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -153,7 +154,12 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             kv[u] = make_uint2(0u, 0u);
             if (i0 + u < Lc) {
                 const long long off = ((cs + i0 + u) * H + h) * DK + c0;
-                g4 = __ldcs(reinterpret_cast<const float4 *>(log_alpha + off));
+                if constexpr (GS) {
+                    const float gs = __ldg(log_alpha + (cs + i0 + u) * H + h);
+                    g4 = make_float4(gs, gs, gs, gs);
+                } else {
+                    g4 = __ldcs(reinterpret_cast<const float4 *>(log_alpha + off));
+                }
                 qv[u] = __ldcs(reinterpret_cast<const uint2 *>(q + off));
                 kv[u] = __ldcs(reinterpret_cast<const uint2 *>(k + off));
             }
@@ -545,7 +551,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
 
 // ------------------------------------------------------------------ host side
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool GS>
 int launch_two_pass_t(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                       const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
                       long long tokens, int T, int H, int dv, int num_seqs, const int32_t *slots, int num_slots,
@@ -561,7 +567,7 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         return KDA_ERR_UNSUPPORTED;
     }
     constexpr int smem1 = IntraLayout<DK>::ALLOC;
-    auto k1 = chunk_intra_kernel<DK>;
+    auto k1 = chunk_intra_kernel<DK, GS>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_intra): %s", cudaGetErrorString(e));
@@ -597,15 +603,21 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
 inline int launch_two_pass(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                            const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
                            long long tokens, int T, int H, int dk, int dv, int num_seqs, const int32_t *slots,
-                           int num_slots, void *workspace, cudaStream_t st, char *msg, size_t msg_len) {
+                           int num_slots, bool gate_scalar, void *workspace, cudaStream_t st, char *msg,
+                           size_t msg_len) {
     // value-tile width of the recurrence pass: the widest that still gives one CTA per SM
     const long long chains = (long long)num_seqs * H;
     int dvt = 32;
     for (int cand = dv; cand >= 32; cand /= 2)
         if (chains * (dv / cand) >= 148) { dvt = cand; break; }
-#define KDA_2P(DKv, DVTv)                                                                                        \
-    return launch_two_pass_t<DKv, DVTv>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, \
-                                        T, H, dv, num_seqs, slots, num_slots, workspace, st, msg, msg_len)
+#define KDA_2P(DKv, DVTv)                                                                                         \
+    return gate_scalar                                                                                             \
+               ? launch_two_pass_t<DKv, DVTv, true>(q, k, v, log_alpha, beta, init_state, o, final_state,         \
+                                                    cu_seqlens, tokens, T, H, dv, num_seqs, slots, num_slots,     \
+                                                    workspace, st, msg, msg_len)                                   \
+               : launch_two_pass_t<DKv, DVTv, false>(q, k, v, log_alpha, beta, init_state, o, final_state,        \
+                                                     cu_seqlens, tokens, T, H, dv, num_seqs, slots, num_slots,    \
+                                                     workspace, st, msg, msg_len)
     if (dk == 128) {
         if (dvt == 128) KDA_2P(128, 128);
         if (dvt == 64) KDA_2P(128, 64);

@@ -46,7 +46,8 @@ struct Smem {
 };
 }  // namespace simt
 
-template <int DK, typename Tin>
+// GS: scalar gate, log_alpha [tokens, H] (Gated DeltaNet), else [tokens, H, DK].
+template <int DK, typename Tin, bool GS>
 __global__ void __launch_bounds__(simt::NT, 1)
 chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -84,7 +85,7 @@ chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
                 const long long off = ((cs + i) * H + h) * DK + c;
                 qv = Elem<Tin>::load(q + off);
                 kv = Elem<Tin>::load(k + off);
-                gv = log_alpha[off];
+                gv = GS ? log_alpha[(cs + i) * H + h] : log_alpha[off];
             }
             sQ[i * DKP + c] = qv;
             sK[i * DKP + c] = kv;

@@ -276,14 +276,16 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 u, float *x) {
 // Threads are grouped by TMEM lane quadrant: warp w reads lanes 32 (w % 4) ..
 // 32 (w % 4) + 31.  State row r (= key channel = TMEM lane) is held by the two
 // warps with w % 4 == r / 32, one per half of the value tile's columns.
-template <int DK, int DVT>
+// GS: scalar gate (Gated DeltaNet), read from g_scalar [tokens, H] instead of the
+// per-channel log_alpha tile that tm_g describes.
+template <int DK, int DVT, bool GS>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                 const float *__restrict__ beta, const float *__restrict__ init_state,
                 __nv_bfloat16 *__restrict__ o, float *__restrict__ final_state,
                 const int32_t *__restrict__ cu_seqlens, int T, int H, int DV, const int32_t *__restrict__ slots,
-                int num_slots) {
+                int num_slots, const float *__restrict__ g_scalar) {
     using L = Layout<DK, DVT>;
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
     constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG;   // factor stage: 4 channels x SEGLEN tokens
@@ -322,7 +324,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
-        ptx::prefetch_tmap(&tm_g);
+        if constexpr (!GS) ptx::prefetch_tmap(&tm_g);
         ptx::prefetch_tmap(&tm_v);
     }
     ptx::tc_fence_before();
@@ -334,10 +336,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     auto issue_inputs = [&](int ci) {   // thread 0 only
         const int z = (int)(t0 + (long long)ci * C);
-        ptx::mbar_arrive_expect_tx(bar_in, (uint32_t)L::IN_BYTES);
+        ptx::mbar_arrive_expect_tx(bar_in, (uint32_t)(GS ? L::IN_BYTES / 2 : L::IN_BYTES));
         ptx::tma_load_3d(sb + L::QIN, &tm_q, bar_in, 0, h, z);
         ptx::tma_load_3d(sb + L::KIN, &tm_k, bar_in, 0, h, z);
-        ptx::tma_load_3d(sb + L::GIN, &tm_g, bar_in, 0, h, z);
+        if constexpr (!GS) ptx::tma_load_3d(sb + L::GIN, &tm_g, bar_in, 0, h, z);
     };
     auto issue_v = [&](int ci) {        // thread 0 only
         const int z = (int)(t0 + (long long)ci * C);
@@ -392,7 +394,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int u = 0; u < SEGLEN; ++u) {
                 float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i0 + u < Lc) g4 = *reinterpret_cast<const float4 *>(gin + (i0 + u) * DK + c0);
+                if (i0 + u < Lc) {
+                    if constexpr (GS) {
+                        const float gs = __ldg(g_scalar + (cs + i0 + u) * H + h);
+                        g4 = make_float4(gs, gs, gs, gs);
+                    } else {
+                        g4 = *reinterpret_cast<const float4 *>(gin + (i0 + u) * DK + c0);
+                    }
+                }
                 sg.x += g4.x; sg.y += g4.y; sg.z += g4.z; sg.w += g4.w;
                 al[u][0] = g4.x; al[u][1] = g4.y; al[u][2] = g4.z; al[u][3] = g4.w;
             }
@@ -691,7 +700,7 @@ inline bool make_tmap(CUtensorMap *m, const void *base, CUtensorMapDataType dt, 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool GS>
 int launch_t(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
              const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, long long tokens,
              int T, int H, int dv, int num_seqs, const int32_t *slots, int num_slots, cudaStream_t st, char *msg,
@@ -699,13 +708,14 @@ int launch_t(const void *q, const void *k, const void *v, const float *log_alpha
     CUtensorMap tq, tk, tg, tv;
     if (!make_tmap(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DK, DK) ||
         !make_tmap(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DK, DK) ||
-        !make_tmap(&tg, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, DK, DK) ||
+        (!GS && !make_tmap(&tg, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, DK, DK)) ||
         !make_tmap(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, dv, DVT)) {
         snprintf(msg, msg_len, "building TMA descriptors failed (driver entry point cuTensorMapEncodeTiled)");
         return KDA_ERR_CUDA;
     }
+    if (GS) tg = tq;   // unused: the scalar gate is read directly
     constexpr int smem = Layout<DK, DVT>::ALLOC;
-    auto kern = chunk_tc_kernel<DK, DVT>;
+    auto kern = chunk_tc_kernel<DK, DVT, GS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_tc): %s", cudaGetErrorString(e));
@@ -713,7 +723,7 @@ int launch_t(const void *q, const void *k, const void *v, const float *log_alpha
     }
     dim3 grid(dv / DVT, H, num_seqs);
     kern<<<grid, NT, smem, st>>>(tq, tk, tg, tv, beta, init_state, (__nv_bfloat16 *)o, final_state, cu_seqlens,
-                                  T, H, dv, slots, num_slots);
+                                  T, H, dv, slots, num_slots, GS ? log_alpha : nullptr);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "chunk_tc launch: %s", cudaGetErrorString(e));
@@ -739,16 +749,20 @@ inline int state_passthrough(const float *init_state, float *final_state, int nu
 inline int launch_fused(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                         const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
                         long long tokens, int T, int H, int dk, int dv, int num_seqs, const int32_t *slots,
-                        int num_slots, cudaStream_t st, char *msg, size_t msg_len) {
+                        int num_slots, bool gate_scalar, cudaStream_t st, char *msg, size_t msg_len) {
     // Value-tile width: the widest tile (fewest duplicated per-chunk operand
     // builds) that still gives at least two CTAs per SM; else 32 columns.
     const long long chains = (long long)num_seqs * H;
     int dvt = 32;
     for (int cand = dv; cand >= 32; cand /= 2)
         if (chains * (dv / cand) >= 2 * 148) { dvt = cand; break; }
-#define KDA_TC(DKv, DVTv)                                                                                   \
-    return launch_t<DKv, DVTv>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T, \
-                               H, dv, num_seqs, slots, num_slots, st, msg, msg_len)
+#define KDA_TC(DKv, DVTv)                                                                                      \
+    return gate_scalar ? launch_t<DKv, DVTv, true>(q, k, v, log_alpha, beta, init_state, o, final_state,      \
+                                                   cu_seqlens, tokens, T, H, dv, num_seqs, slots, num_slots,  \
+                                                   st, msg, msg_len)                                          \
+                       : launch_t<DKv, DVTv, false>(q, k, v, log_alpha, beta, init_state, o, final_state,     \
+                                                    cu_seqlens, tokens, T, H, dv, num_seqs, slots, num_slots, \
+                                                    st, msg, msg_len)
     if (dk == 128) {
         if (dvt == 128) KDA_TC(128, 128);
         if (dvt == 64) KDA_TC(128, 64);

@@ -17,7 +17,8 @@
 
 namespace kda {
 
-template <int DK, int DV, typename Tin>
+// GS: scalar gate, one log_alpha per (sequence, head) (Gated DeltaNet), else one per key channel.
+template <int DK, int DV, typename Tin, bool GS>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                    const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -56,7 +57,7 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
     const long long kb = pair * DK;
     float qk = 0.f;
     for (int c = tid; c < DK; c += 256) {
-        const float a = expf(log_alpha[kb + c]);
+        const float a = expf(GS ? log_alpha[pair] : log_alpha[kb + c]);
         const float kc = Elem<Tin>::load(k + kb + c);
         const float qc = Elem<Tin>::load(q + kb + c);
         s_a[c] = a;

@@ -33,7 +33,7 @@ int cuda_fail(cudaError_t e, const char *what) {
 int check_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
                   const float *beta, const float *init_state, const void *o, const float *final_state,
                   const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
-                  int dtype, int chunk) {
+                  int dtype, int chunk, bool gate_scalar = false) {
     if (B < 1 || T < 0 || H < 1 || num_seqs < 0)
         return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d num_seqs=%d", B, T, H, num_seqs);
     // With no tokens the per-token tensors are empty and may be NULL.
@@ -51,10 +51,12 @@ int check_prefill(const void *q, const void *k, const void *v, const float *log_
         return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d: each must be 64 or 128", dk, dv);
     if (chunk != 64) return fail(KDA_ERR_UNSUPPORTED, "chunk=%d: only 64 is supported", chunk);
     if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "dtype=%d", dtype);
-    const void *p16[] = {q, k, v, log_alpha, o, init_state, final_state};
+    const void *p16[] = {q, k, v, gate_scalar ? nullptr : log_alpha, o, init_state, final_state};
     const char *n16[] = {"q", "k", "v", "log_alpha", "o", "init_state", "final_state"};
     for (int i = 0; i < 7; ++i)
         if (p16[i] && !aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
+    if (gate_scalar && log_alpha && !aligned(log_alpha, 4))
+        return fail(KDA_ERR_MISALIGNED, "log_alpha is not 4-byte aligned");
     if (beta && !aligned(beta, 4)) return fail(KDA_ERR_MISALIGNED, "beta is not 4-byte aligned");
     if (cu_seqlens && !aligned(cu_seqlens, 4)) return fail(KDA_ERR_MISALIGNED, "cu_seqlens is not 4-byte aligned");
     return KDA_OK;
@@ -105,12 +107,12 @@ void *static_ws_address(cudaError_t *err) {
     return addr[dev];
 }
 
-template <int DK, typename Tin>
+template <int DK, typename Tin, bool GS>
 int launch_simt(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                 const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int T,
                 int H, int dv, int num_seqs, const int32_t *slots, int num_slots, cudaStream_t st) {
     constexpr size_t smem = kda::simt::Smem<DK>::bytes;
-    auto kern = kda::chunk_simt_kernel<DK, Tin>;
+    auto kern = kda::chunk_simt_kernel<DK, Tin, GS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chunk_simt)");
     dim3 grid(dv / kda::simt::DVT, H, num_seqs);
@@ -122,11 +124,11 @@ int launch_simt(const void *q, const void *k, const void *v, const float *log_al
     return KDA_OK;
 }
 
-template <int DK, int DV, typename Tin>
+template <int DK, int DV, typename Tin, bool GS>
 int launch_decode(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                   float *state, void *o, long long pairs, const int32_t *slots, int num_slots, int H,
                   cudaStream_t st) {
-    kda::decode_step_kernel<DK, DV, Tin><<<(unsigned)pairs, 256, 0, st>>>(
+    kda::decode_step_kernel<DK, DV, Tin, GS><<<(unsigned)pairs, 256, 0, st>>>(
         (const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta, state, (Tin *)o, slots, num_slots, H);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
@@ -137,27 +139,34 @@ int launch_decode(const void *q, const void *k, const void *v, const float *log_
 // sequences to state rows.
 int simt_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
               const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int T, int H,
-              int dk, int dv, int num_seqs, int dtype, const int32_t *slots, int num_slots, cudaStream_t st) {
+              int dk, int dv, int num_seqs, int dtype, const int32_t *slots, int num_slots, bool gate_scalar,
+              cudaStream_t st) {
     if (num_seqs == 0) return KDA_OK;
+#define KDA_SIMT(DKv, TT, GSv)                                                                                  \
+    return launch_simt<DKv, TT, GSv>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H, dv, \
+                                     num_seqs, slots, num_slots, st)
     if (dtype == KDA_BF16) {
-        if (dk == 64)
-            return launch_simt<64, __nv_bfloat16>(q, k, v, log_alpha, beta, init_state, o, final_state,
-                                                  cu_seqlens, T, H, dv, num_seqs, slots, num_slots, st);
-        return launch_simt<128, __nv_bfloat16>(q, k, v, log_alpha, beta, init_state, o, final_state,
-                                               cu_seqlens, T, H, dv, num_seqs, slots, num_slots, st);
+        if (dk == 64) {
+            if (gate_scalar) KDA_SIMT(64, __nv_bfloat16, true);
+            KDA_SIMT(64, __nv_bfloat16, false);
+        }
+        if (gate_scalar) KDA_SIMT(128, __nv_bfloat16, true);
+        KDA_SIMT(128, __nv_bfloat16, false);
     }
-    if (dk == 64)
-        return launch_simt<64, float>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T,
-                                      H, dv, num_seqs, slots, num_slots, st);
-    return launch_simt<128, float>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H,
-                                   dv, num_seqs, slots, num_slots, st);
+    if (dk == 64) {
+        if (gate_scalar) KDA_SIMT(64, float, true);
+        KDA_SIMT(64, float, false);
+    }
+    if (gate_scalar) KDA_SIMT(128, float, true);
+    KDA_SIMT(128, float, false);
+#undef KDA_SIMT
 }
 
 // The tensor-core prefill after argument checks (dtype KDA_BF16, algo valid).
 int prefill_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                  const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int B, int T,
                  int H, int dk, int dv, int num_seqs, int algo, const int32_t *slots, int num_slots,
-                 void *workspace, size_t ws_bytes, cudaStream_t st) {
+                 bool gate_scalar, void *workspace, size_t ws_bytes, cudaStream_t st) {
     const long long tokens = (long long)B * T;
     const Plan plan = plan_prefill(tokens, H, dk, num_seqs, algo);
     if (plan.ws && (!workspace || ws_bytes < plan.ws))
@@ -173,17 +182,19 @@ int prefill_impl(const void *q, const void *k, const void *v, const float *log_a
                    : kda::tc::state_passthrough(init_state, final_state, num_seqs, H, dk, dv, st, msg, sizeof(msg));
     else if (plan.algo == KDA_ALGO_TWO_PASS)
         rc = kda::tc::launch_two_pass(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T,
-                                      H, dk, dv, num_seqs, slots, num_slots, workspace, st, msg, sizeof(msg));
+                                      H, dk, dv, num_seqs, slots, num_slots, gate_scalar, workspace, st, msg,
+                                      sizeof(msg));
     else
         rc = kda::tc::launch_fused(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T, H,
-                                   dk, dv, num_seqs, slots, num_slots, st, msg, sizeof(msg));
+                                   dk, dv, num_seqs, slots, num_slots, gate_scalar, st, msg, sizeof(msg));
     if (rc) return fail(rc, "%s", msg);
     return KDA_OK;
 }
 
 // Decode argument checks shared by both decode entry points.
 int check_decode(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
-                 const float *state, const void *o, int N, int H, int dk, int dv, int dtype) {
+                 const float *state, const void *o, int N, int H, int dk, int dv, int dtype,
+                 bool gate_scalar = false) {
     if (N < 0 || H < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d", N, H);
     if (N == 0) return KDA_OK;   // nothing to do; empty tensors may carry NULL pointers
     if (!q || !k || !v || !log_alpha || !beta || !state || !o)
@@ -194,7 +205,8 @@ int check_decode(const void *q, const void *k, const void *v, const float *log_a
     const void *p16[] = {q, k, v, log_alpha, o, state};
     const char *n16[] = {"q", "k", "v", "log_alpha", "o", "state"};
     for (int i = 0; i < 6; ++i)
-        if (!aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
+        if (!aligned(p16[i], (i == 3 && gate_scalar) ? 4 : 16))
+            return fail(KDA_ERR_MISALIGNED, "%s is not %d-byte aligned", n16[i], (i == 3 && gate_scalar) ? 4 : 16);
     if (!aligned(beta, 4)) return fail(KDA_ERR_MISALIGNED, "beta is not 4-byte aligned");
     if ((long long)N * H > 0x7fffffffLL) return fail(KDA_ERR_UNSUPPORTED, "N*H=%lld too large", (long long)N * H);
     return KDA_OK;
@@ -202,20 +214,25 @@ int check_decode(const void *q, const void *k, const void *v, const float *log_a
 
 int decode_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                 float *state, void *o, int N, int H, int dk, int dv, int dtype, const int32_t *slots,
-                int num_slots, cudaStream_t st) {
+                int num_slots, bool gate_scalar, cudaStream_t st) {
     const long long pairs = (long long)N * H;
     if (pairs == 0) return KDA_OK;
-#define KDA_DEC(DKv, DVv)                                                                                     \
-    if (dk == DKv && dv == DVv)                                                                               \
-        return dtype == KDA_BF16 ? launch_decode<DKv, DVv, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o, \
-                                                                          pairs, slots, num_slots, H, st)     \
-                                 : launch_decode<DKv, DVv, float>(q, k, v, log_alpha, beta, state, o, pairs,  \
-                                                                  slots, num_slots, H, st);
+#define KDA_DEC1(DKv, DVv, TT)                                                                                 \
+    return gate_scalar ? launch_decode<DKv, DVv, TT, true>(q, k, v, log_alpha, beta, state, o, pairs, slots,  \
+                                                           num_slots, H, st)                                  \
+                       : launch_decode<DKv, DVv, TT, false>(q, k, v, log_alpha, beta, state, o, pairs, slots, \
+                                                            num_slots, H, st);
+#define KDA_DEC(DKv, DVv)                             \
+    if (dk == DKv && dv == DVv) {                     \
+        if (dtype == KDA_BF16) KDA_DEC1(DKv, DVv, __nv_bfloat16) \
+        KDA_DEC1(DKv, DVv, float)                     \
+    }
     KDA_DEC(64, 64)
     KDA_DEC(64, 128)
     KDA_DEC(128, 64)
     KDA_DEC(128, 128)
 #undef KDA_DEC
+#undef KDA_DEC1
     return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d", dk, dv);
 }
 
@@ -247,7 +264,7 @@ int kda_chunk_forward_simt(const void *q, const void *k, const void *v, const fl
                            dv, num_seqs, dtype, chunk);
     if (rc) return rc;
     return simt_impl(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H, dk, dv, num_seqs,
-                     dtype, nullptr, 0, (cudaStream_t)stream);
+                     dtype, nullptr, 0, false, (cudaStream_t)stream);
 }
 
 int kda_chunk_forward_ex(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -261,9 +278,9 @@ int kda_chunk_forward_ex(const void *q, const void *k, const void *v, const floa
         return fail(KDA_ERR_INVALID_ARG, "algo=%d is not a KDA_ALGO_* value", algo);
     if (dtype == KDA_F32)
         return simt_impl(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H, dk, dv,
-                         num_seqs, dtype, nullptr, 0, (cudaStream_t)stream);
+                         num_seqs, dtype, nullptr, 0, false, (cudaStream_t)stream);
     return prefill_impl(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk, dv,
-                        num_seqs, algo, nullptr, 0, workspace, ws_bytes, (cudaStream_t)stream);
+                        num_seqs, algo, nullptr, 0, false, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
 int kda_chunk_forward_slots(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -282,9 +299,9 @@ int kda_chunk_forward_slots(const void *q, const void *k, const void *v, const f
         return fail(KDA_ERR_INVALID_ARG, "algo=%d is not a KDA_ALGO_* value", algo);
     if (dtype == KDA_F32)
         return simt_impl(q, k, v, log_alpha, beta, state_pool, o, state_pool, cu_seqlens, T, H, dk, dv,
-                         num_seqs, dtype, slots, num_slots, (cudaStream_t)stream);
+                         num_seqs, dtype, slots, num_slots, false, (cudaStream_t)stream);
     return prefill_impl(q, k, v, log_alpha, beta, state_pool, o, state_pool, cu_seqlens, B, T, H, dk, dv,
-                        num_seqs, algo, slots, num_slots, workspace, ws_bytes, (cudaStream_t)stream);
+                        num_seqs, algo, slots, num_slots, false, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
 int kda_chunk_forward(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -327,7 +344,8 @@ int kda_recurrent_step(const void *q, const void *k, const void *v, const float 
                        void *stream) {
     int rc = check_decode(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype);
     if (rc || N == 0) return rc;
-    return decode_impl(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype, nullptr, 0, (cudaStream_t)stream);
+    return decode_impl(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype, nullptr, 0, false,
+                       (cudaStream_t)stream);
 }
 
 int kda_recurrent_step_slots(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -338,7 +356,32 @@ int kda_recurrent_step_slots(const void *q, const void *k, const void *v, const 
     if (!slots) return fail(KDA_ERR_INVALID_ARG, "slots is required");
     if (!aligned(slots, 4)) return fail(KDA_ERR_MISALIGNED, "slots is not 4-byte aligned");
     if (num_slots < 1) return fail(KDA_ERR_INVALID_ARG, "num_slots=%d must be at least 1", num_slots);
-    return decode_impl(q, k, v, log_alpha, beta, state_pool, o, N, H, dk, dv, dtype, slots, num_slots,
+    return decode_impl(q, k, v, log_alpha, beta, state_pool, o, N, H, dk, dv, dtype, slots, num_slots, false,
+                       (cudaStream_t)stream);
+}
+
+int kda_gdn_chunk_forward(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *init_state, void *o, float *final_state,
+                          const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs, int dtype,
+                          int chunk, int algo, void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
+                           dv, num_seqs, dtype, chunk, true);
+    if (rc) return rc;
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_FUSED && algo != KDA_ALGO_TWO_PASS)
+        return fail(KDA_ERR_INVALID_ARG, "algo=%d is not a KDA_ALGO_* value", algo);
+    if (dtype == KDA_F32)
+        return simt_impl(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H, dk, dv,
+                         num_seqs, dtype, nullptr, 0, true, (cudaStream_t)stream);
+    return prefill_impl(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk, dv,
+                        num_seqs, algo, nullptr, 0, true, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+int kda_gdn_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, float *state, void *o, int N, int H, int dk, int dv, int dtype,
+                           void *stream) {
+    int rc = check_decode(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype, true);
+    if (rc || N == 0) return rc;
+    return decode_impl(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype, nullptr, 0, true,
                        (cudaStream_t)stream);
 }
 

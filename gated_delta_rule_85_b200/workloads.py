@@ -8,7 +8,8 @@ Distributions (per the workload definitions):
   q, k      ~ N(0, 1), then L2-normalised over dk per (token, head) in fp32,
               then cast to the input dtype (bf16 or fp32)
   v         ~ N(0, 1), cast to the input dtype
-  log_alpha = -softplus(x), x ~ N(-2, 1), fp32, one value per channel
+  log_alpha = -softplus(x), x ~ N(-2, 1), fp32, one value per channel (KDA), or
+              one per (token, head) for the scalar gate of Gated DeltaNet
   beta      = sigmoid(x), x ~ N(0, 1), fp32, one value per (token, head)
   states    ~ N(0, 0.01^2) fp32 (std 0.01), or zeros
 Every tensor is drawn from its own generator seeded with (seed, stream id), so
@@ -37,6 +38,7 @@ class PrefillShape:
     dtype: torch.dtype = torch.bfloat16
     init_state: str = "normal"          # "normal" (std 0.01) or "zeros"
     cu_seqlens: tuple | None = None      # packed layout when set (B must be 1)
+    gate: str = "channel"                # "channel": log_alpha [B, T, H, dk]; "scalar": [B, T, H]
 
     @property
     def num_seqs(self) -> int:
@@ -51,6 +53,7 @@ class DecodeShape:
     dv: int
     steps: int
     dtype: torch.dtype = torch.bfloat16
+    gate: str = "channel"                # "channel": log_alpha [N, H, dk]; "scalar": [N, H]
 
 
 def _gen(device, seed: int, stream: int, sub: int = 0) -> torch.Generator:
@@ -141,7 +144,8 @@ def prefill_inputs(shape: PrefillShape, seed: int = 0, device="cpu") -> dict:
         "q": draw_qk((B, T, H, dk), device, seed, _STREAM["q"], shape.dtype),
         "k": draw_qk((B, T, H, dk), device, seed, _STREAM["k"], shape.dtype),
         "v": draw_v((B, T, H, dv), device, seed, _STREAM["v"], shape.dtype),
-        "log_alpha": draw_log_alpha((B, T, H, dk), device, seed, _STREAM["log_alpha"]),
+        "log_alpha": draw_log_alpha((B, T, H, dk) if shape.gate == "channel" else (B, T, H), device, seed,
+                                    _STREAM["log_alpha"]),
         "beta": draw_beta((B, T, H), device, seed, _STREAM["beta"]),
     }
     N = shape.num_seqs
@@ -160,7 +164,8 @@ def decode_step_inputs(shape: DecodeShape, step: int, seed: int = 0, device="cpu
         "q": draw_qk((N, H, dk), device, base, _STREAM["q"], shape.dtype),
         "k": draw_qk((N, H, dk), device, base, _STREAM["k"], shape.dtype),
         "v": draw_v((N, H, dv), device, base, _STREAM["v"], shape.dtype),
-        "log_alpha": draw_log_alpha((N, H, dk), device, base, _STREAM["log_alpha"]),
+        "log_alpha": draw_log_alpha((N, H, dk) if shape.gate == "channel" else (N, H), device, base,
+                                    _STREAM["log_alpha"]),
         "beta": draw_beta((N, H), device, base, _STREAM["beta"]),
     }
 
@@ -172,7 +177,8 @@ def decode_all_steps(shape: DecodeShape, seed: int = 0, device="cpu") -> dict:
         "q": torch.empty((S, N, H, dk), dtype=shape.dtype, device=device),
         "k": torch.empty((S, N, H, dk), dtype=shape.dtype, device=device),
         "v": torch.empty((S, N, H, dv), dtype=shape.dtype, device=device),
-        "log_alpha": torch.empty((S, N, H, dk), dtype=torch.float32, device=device),
+        "log_alpha": torch.empty((S, N, H, dk) if shape.gate == "channel" else (S, N, H), dtype=torch.float32,
+                                 device=device),
         "beta": torch.empty((S, N, H), dtype=torch.float32, device=device),
     }
     for s in range(S):

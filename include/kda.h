@@ -241,6 +241,29 @@ int kda_recurrent_step_slots(const void *q, const void *k, const void *v, const 
                              const float *beta, float *state_pool, const int32_t *slots, void *o, int N, int H,
                              int dk, int dv, int num_slots, int dtype, void *stream);
 
+/*
+ * Gated DeltaNet: the same recurrence with one decay rate per (token, head)
+ * instead of one per key channel, S' = alpha_t S with a scalar alpha_t
+ * ("Kimi Delta Attention 徹底解説" (tech-tide.dev), § "Kimi Delta Attention の仕組み":
+ * Gated DeltaNet decays the whole state by one scalar, KDA makes it a diagonal
+ * matrix; "Kimi Linearは広がりつつある…" (orcarouter.ai): serving stacks ship fused
+ * KDA and Gated DeltaNet kernels).  The same kernels run with the gate read as a
+ * scalar, so the gate stream is 4 instead of 4 dk bytes per token-head.
+ *
+ *   log_alpha   fp32 [B, T, H] (prefill) or [N, H] (decode), 4-byte aligned;
+ *               every other argument, the workspace (kda_chunk_forward_workspace_size_ex
+ *               with the same sizes and algo) and the error behaviour are as in
+ *               kda_chunk_forward_ex / kda_recurrent_step.
+ */
+int kda_gdn_chunk_forward(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *init_state, void *o, float *final_state,
+                          const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs, int dtype,
+                          int chunk, int algo, void *workspace, size_t ws_bytes, void *stream);
+
+int kda_gdn_recurrent_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, float *state, void *o, int N, int H, int dk, int dv, int dtype,
+                           void *stream);
+
 /* Message for the calling thread's last non-OK return ("" if none). */
 const char *kda_last_error(void);
 
