@@ -27,7 +27,7 @@ import numpy as np
 
 from .build import build_oracle, library_path
 
-__all__ = ["forward", "unrolled", "step", "max_threads", "library_path", "build_oracle"]
+__all__ = ["forward", "backward", "unrolled", "step", "max_threads", "library_path", "build_oracle"]
 
 _lib = None
 
@@ -47,6 +47,8 @@ def _load():
         c_int = ctypes.c_int
         lib.kda_oracle_forward.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ip] + [c_int] * 7
         lib.kda_oracle_forward.restype = c_int
+        lib.kda_oracle_backward.argtypes = [dp] * 14 + [ip] + [c_int] * 7
+        lib.kda_oracle_backward.restype = c_int
         lib.kda_oracle_unrolled.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp] + [c_int] * 5
         lib.kda_oracle_unrolled.restype = c_int
         lib.kda_oracle_step.argtypes = [dp, dp, dp, dp, dp, dp, dp] + [c_int] * 5
@@ -102,6 +104,44 @@ def forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, nthreads
     if rc != 0:
         raise ValueError(f"oracle.forward failed with code {rc}")
     return o, fs
+
+
+def backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal=None, cu_seqlens=None, nthreads=0):
+    """Gradients of L = sum <d_o, o> + <dfinal, final_state> by reverse-mode
+    differentiation of the token recurrence (fp64).
+
+    Shapes as in :func:`forward`; d_o is [B, T, H, dv], dfinal is
+    [N, H, dk, dv] or None (zero).  Returns a dict with dq, dk, dv,
+    dlog_alpha, dbeta and dinit_state (dL/dS_0, also when init_state is None).
+    """
+    q, k, v, g, b, do = (_f64(x) for x in (q, k, v, log_alpha, beta, d_o))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if (k.shape != q.shape or g.shape != q.shape or v.shape[:3] != q.shape[:3]
+            or b.shape != q.shape[:3] or do.shape != v.shape):
+        raise ValueError("oracle.backward: inconsistent shapes")
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        N = cu.shape[0] - 1
+    else:
+        N = B
+    s0 = None if init_state is None else _f64(init_state)
+    dS = None if dfinal is None else _f64(dfinal)
+    for name, x in (("init_state", s0), ("dfinal", dS)):
+        if x is not None and x.shape != (N, H, dk, dv):
+            raise ValueError(f"oracle.backward: {name} shape")
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v),
+               dlog_alpha=np.zeros_like(g), dbeta=np.zeros_like(b),
+               dinit_state=np.zeros((N, H, dk, dv), dtype=np.float64))
+    cu_p = None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    rc = _load().kda_oracle_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(s0), _ptr(do), _ptr(dS),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dlog_alpha"]),
+        _ptr(out["dbeta"]), _ptr(out["dinit_state"]), cu_p, B, T, H, dk, dv, N, int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle.backward failed with code {rc}")
+    return out
 
 
 def unrolled(q, k, v, log_alpha, beta, init_state=None):

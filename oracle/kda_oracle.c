@@ -255,6 +255,197 @@ int kda_oracle_unrolled(const double *q, const double *k, const double *v,
 }
 
 /*
+ * Reverse-mode derivative of kda_oracle_forward (the "chunkwise training
+ * algorithm" of "Kimi Linear、独自の土俵でFull Attentionを上回る" (remio.ai),
+ * § "Kimi Linearがより賢いRecurrent Memoryを使う方法", needs these gradients;
+ * here they are taken of the plain token recurrence, not of any chunk form).
+ *
+ * For the scalar loss  L = sum_t <do_t, o_t> + <dfinal, S_T>  (do and dfinal
+ * are given; dfinal may be NULL = 0) it returns dL/dq, dL/dk, dL/dv,
+ * dL/dlog_alpha, dL/dbeta and dL/dinit_state (every output is required;
+ * dinit_state is dL/dS_0 whether or not init_state is NULL).
+ *
+ * One token, written with its intermediates:
+ *     a  = exp(g_t)               Sp = Diag(a) S          r = Sp^T k_t
+ *     u  = beta_t (v_t - r)       Sn = Sp + k_t u^T       o_t = Sn^T q_t
+ * and its adjoint, with dS the adjoint of Sn on entry:
+ *     dq_t  = Sn do_t                           dS  += q_t do_t^T
+ *     dk_t  = dS u                              du   = dS^T k_t
+ *     dbeta = <du, v_t - r>                     dv_t = beta_t du
+ *     dr    = -beta_t du                        dSp  = dS + k_t dr^T
+ *     dk_t += Sp dr                             dg_t[c] = sum_j dSp[c][j] Sp[c][j]
+ *     dS    = Diag(a) dSp                       (adjoint of S before the token)
+ * (dg_t uses d exp(g)/dg = exp(g): dL/dg_c = a_c sum_j dSp[c][j] S[c][j].)
+ *
+ * The reverse sweep needs the state before every token.  They are recomputed,
+ * with the forward's own arithmetic, from states kept every KDA_ORACLE_CKPT
+ * tokens, so memory is (T / KDA_ORACLE_CKPT + KDA_ORACLE_CKPT) dk dv doubles
+ * per (sequence, head) in flight instead of T dk dv; the values are the same.
+ */
+#define KDA_ORACLE_CKPT 64
+
+/* One forward token on S in place; keeps Sp (the decayed state) and r if asked. */
+static void token_forward(double *S, double *Sp, double *r, double *alpha,
+                          const double *qt, const double *kt, const double *vt,
+                          const double *gt, double bt, int dk, int dv) {
+    (void)qt;
+    for (int c = 0; c < dk; ++c) alpha[c] = exp(gt[c]);
+    for (int c = 0; c < dk; ++c)
+        for (int j = 0; j < dv; ++j) S[(size_t)c * dv + j] *= alpha[c];
+    if (Sp) memcpy(Sp, S, sizeof(double) * (size_t)dk * dv);
+    for (int j = 0; j < dv; ++j) r[j] = 0.0;
+    for (int c = 0; c < dk; ++c)
+        for (int j = 0; j < dv; ++j) r[j] += S[(size_t)c * dv + j] * kt[c];
+    for (int c = 0; c < dk; ++c)
+        for (int j = 0; j < dv; ++j) S[(size_t)c * dv + j] += kt[c] * bt * (vt[j] - r[j]);
+}
+
+int kda_oracle_backward(const double *q, const double *k, const double *v,
+                        const double *log_alpha, const double *beta,
+                        const double *init_state, const double *d_o, const double *dfinal,
+                        double *dq, double *dk_out, double *dv_out, double *dlog_alpha,
+                        double *dbeta, double *dinit_state,
+                        const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv,
+                        int num_seqs, int nthreads) {
+    int rc = check_args(cu_seqlens, B, T, H, dk, dv, num_seqs);
+    if (rc) return rc;
+    if (!q || !k || !v || !log_alpha || !beta || !d_o) return KDA_ORACLE_EINVAL;
+    if (!dq || !dk_out || !dv_out || !dlog_alpha || !dbeta || !dinit_state) return KDA_ORACLE_EINVAL;
+    const long pairs = (long)num_seqs * H;
+    const size_t kv = (size_t)dk * dv;
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel
+#endif
+    {
+        double *S = (double *)malloc(sizeof(double) * kv);
+        double *Sp = (double *)malloc(sizeof(double) * kv);
+        double *dS = (double *)malloc(sizeof(double) * kv);
+        double *seg = (double *)malloc(sizeof(double) * kv * KDA_ORACLE_CKPT);
+        double *r = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *du = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *alpha = (double *)malloc(sizeof(double) * (size_t)dk);
+        double *ckpt = NULL;
+        size_t ckpt_cap = 0;
+        int ok = S && Sp && dS && seg && r && u && du && alpha;
+        if (!ok) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            failed = 1;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (long p = 0; p < pairs; ++p) {
+            if (!ok) continue;
+            const int n = (int)(p / H), h = (int)(p % H);
+            long t0, t1;
+            seq_range(cu_seqlens, B, T, n, &t0, &t1);
+            const long L = t1 - t0;
+            const long nck = (L + KDA_ORACLE_CKPT - 1) / KDA_ORACLE_CKPT;
+            if ((size_t)(nck > 0 ? nck : 1) > ckpt_cap) {
+                free(ckpt);
+                ckpt_cap = (size_t)(nck > 0 ? nck : 1);
+                ckpt = (double *)malloc(sizeof(double) * kv * ckpt_cap);
+                if (!ckpt) {
+                    ckpt_cap = 0;
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+                    failed = 1;
+                    continue;
+                }
+            }
+            /* forward: keep the state before tokens t0, t0 + CKPT, t0 + 2 CKPT, ... */
+            if (init_state)
+                memcpy(S, init_state + (size_t)p * kv, sizeof(double) * kv);
+            else
+                memset(S, 0, sizeof(double) * kv);
+            for (long t = t0; t < t1; ++t) {
+                if ((t - t0) % KDA_ORACLE_CKPT == 0)
+                    memcpy(ckpt + (size_t)((t - t0) / KDA_ORACLE_CKPT) * kv, S, sizeof(double) * kv);
+                const size_t tk = ((size_t)t * H + h) * dk, tv = ((size_t)t * H + h) * dv;
+                token_forward(S, NULL, r, alpha, q + tk, k + tk, v + tv, log_alpha + tk,
+                              beta[(size_t)t * H + h], dk, dv);
+            }
+            /* reverse sweep */
+            if (dfinal)
+                memcpy(dS, dfinal + (size_t)p * kv, sizeof(double) * kv);
+            else
+                memset(dS, 0, sizeof(double) * kv);
+            for (long sgi = nck - 1; sgi >= 0; --sgi) {
+                const long s0 = t0 + sgi * KDA_ORACLE_CKPT;
+                const long s1 = (s0 + KDA_ORACLE_CKPT < t1) ? s0 + KDA_ORACLE_CKPT : t1;
+                /* states before each token of the segment */
+                memcpy(S, ckpt + (size_t)sgi * kv, sizeof(double) * kv);
+                for (long t = s0; t < s1; ++t) {
+                    memcpy(seg + (size_t)(t - s0) * kv, S, sizeof(double) * kv);
+                    const size_t tk = ((size_t)t * H + h) * dk, tv = ((size_t)t * H + h) * dv;
+                    token_forward(S, NULL, r, alpha, q + tk, k + tk, v + tv, log_alpha + tk,
+                                  beta[(size_t)t * H + h], dk, dv);
+                }
+                for (long t = s1 - 1; t >= s0; --t) {
+                    const size_t tk = ((size_t)t * H + h) * dk, tv = ((size_t)t * H + h) * dv;
+                    const double bt = beta[(size_t)t * H + h];
+                    const double *qt = q + tk, *kt = k + tk, *vt = v + tv, *dot = d_o + tv;
+                    /* recompute this token: S <- state after it, Sp, r, u */
+                    memcpy(S, seg + (size_t)(t - s0) * kv, sizeof(double) * kv);
+                    token_forward(S, Sp, r, alpha, qt, kt, vt, log_alpha + tk, bt, dk, dv);
+                    for (int j = 0; j < dv; ++j) u[j] = bt * (vt[j] - r[j]);
+                    /* o_t = Sn^T q_t */
+                    for (int c = 0; c < dk; ++c) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dv; ++j) acc += S[(size_t)c * dv + j] * dot[j];
+                        dq[tk + c] = acc;
+                    }
+                    for (int c = 0; c < dk; ++c)
+                        for (int j = 0; j < dv; ++j) dS[(size_t)c * dv + j] += qt[c] * dot[j];
+                    /* Sn = Sp + k u^T */
+                    for (int c = 0; c < dk; ++c) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dv; ++j) acc += dS[(size_t)c * dv + j] * u[j];
+                        dk_out[tk + c] = acc;
+                    }
+                    for (int j = 0; j < dv; ++j) {
+                        double acc = 0.0;
+                        for (int c = 0; c < dk; ++c) acc += dS[(size_t)c * dv + j] * kt[c];
+                        du[j] = acc;
+                    }
+                    /* u = beta (v - r) */
+                    double db = 0.0;
+                    for (int j = 0; j < dv; ++j) db += du[j] * (vt[j] - r[j]);
+                    dbeta[(size_t)t * H + h] = db;
+                    for (int j = 0; j < dv; ++j) dv_out[tv + j] = bt * du[j];
+                    /* r = Sp^T k: dr = -beta du; dSp = dS + k dr^T; dk += Sp dr */
+                    for (int j = 0; j < dv; ++j) du[j] = -bt * du[j];
+                    for (int c = 0; c < dk; ++c) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dv; ++j) {
+                            dS[(size_t)c * dv + j] += kt[c] * du[j];
+                            acc += Sp[(size_t)c * dv + j] * du[j];
+                        }
+                        dk_out[tk + c] += acc;
+                    }
+                    /* Sp = Diag(exp(g)) S_prev */
+                    for (int c = 0; c < dk; ++c) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dv; ++j) acc += dS[(size_t)c * dv + j] * Sp[(size_t)c * dv + j];
+                        dlog_alpha[tk + c] = acc;
+                        for (int j = 0; j < dv; ++j) dS[(size_t)c * dv + j] *= alpha[c];
+                    }
+                }
+            }
+            memcpy(dinit_state + (size_t)p * kv, dS, sizeof(double) * kv);
+        }
+        free(S); free(Sp); free(dS); free(seg); free(r); free(u); free(du); free(alpha); free(ckpt);
+    }
+    return failed ? KDA_ORACLE_ENOMEM : KDA_ORACLE_OK;
+}
+
+/*
  * One decode step for N independent (sequence, head) states, in place:
  * the same recurrence as kda_oracle_forward with T = 1.  q, k, log_alpha
  * are [N, H, dk], v and o are [N, H, dv], beta is [N, H], state [N, H, dk, dv].

@@ -2,7 +2,7 @@
 
 Each case below plants one mistake in a private copy of oracle/kda_oracle.c
 (on the CPU, in a temporary directory), builds it, and runs the pin suite
-against that copy; the suite has to fail.  The shipped oracle is untouched.
+against that copy (forward and gradient pins); the suite has to fail.  The shipped oracle is untouched.
 """
 import os
 import subprocess
@@ -48,6 +48,25 @@ MUTANTS = {
     "read_before_write": lambda s: _move(s, READ_BLOCK, R_MARK),
     "alpha_not_exponentiated": lambda s: s.replace("alpha[c] = exp(log_alpha[tk + c]);",
                                                    "alpha[c] = 1.0 + log_alpha[tk + c];", 1),
+    # reverse sweep (oracle.backward)
+    "bwd_prediction_adjoint_dropped": lambda s: s.replace(
+        "dS[(size_t)c * dv + j] += kt[c] * du[j];", "(void)0;", 1),
+    "bwd_key_term_of_prediction_dropped": lambda s: s.replace(
+        "dk_out[tk + c] += acc;", "dk_out[tk + c] += 0.0 * acc;", 1),
+    "bwd_adjoint_not_decayed": lambda s: s.replace(
+        "for (int j = 0; j < dv; ++j) dS[(size_t)c * dv + j] *= alpha[c];", "", 1),
+    "bwd_value_grad_without_beta": lambda s: s.replace(
+        "dv_out[tv + j] = bt * du[j];", "dv_out[tv + j] = du[j];", 1),
+    "bwd_beta_grad_sign": lambda s: s.replace(
+        "db += du[j] * (vt[j] - r[j]);", "db += du[j] * (vt[j] + r[j]);", 1),
+    "bwd_query_grad_from_decayed_state": lambda s: s.replace(
+        "acc += S[(size_t)c * dv + j] * dot[j];", "acc += Sp[(size_t)c * dv + j] * dot[j];", 1),
+    "bwd_gate_grad_from_new_state": lambda s: s.replace(
+        "acc += dS[(size_t)c * dv + j] * Sp[(size_t)c * dv + j];",
+        "acc += dS[(size_t)c * dv + j] * S[(size_t)c * dv + j];", 1),
+    "bwd_segment_restarts_from_first_checkpoint": lambda s: s.replace(
+        "memcpy(S, ckpt + (size_t)sgi * kv, sizeof(double) * kv);",
+        "memcpy(S, ckpt, sizeof(double) * kv);", 1),
 }
 
 
@@ -63,6 +82,7 @@ def test_pins_reject_mutant(name, tmp_path):
                    check=True)
     env = dict(os.environ, KDA_ORACLE_LIB=str(so))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(HERE, "test_oracle_pins.py")],
+                        os.path.join(HERE, "test_oracle_pins.py"),
+                        os.path.join(HERE, "test_oracle_backward_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0, f"pins accepted mutant {name}:\n{r.stdout[-2000:]}"
