@@ -7,6 +7,7 @@ without the built library, or without a CUDA device, raises.
 
     o, S = chunk_forward(q, k, v, log_alpha, beta, init_state, cu_seqlens=None)
     o    = recurrent_step(q, k, v, log_alpha, beta, state)      # state in place
+    g    = chunk_backward(q, k, v, log_alpha, beta, d_o, init_state)   # dict of gradients
 
 The recurrence ("Kimi Delta Attention 徹底解説" (tech-tide.dev), § "Kimi Delta
 Attention の仕組み"), per (sequence, head), with a dk x dv fp32 state S:
@@ -20,7 +21,7 @@ import os
 import torch
 
 __all__ = [
-    "chunk_forward", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
+    "chunk_forward", "chunk_backward", "backward_workspace_size", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
     "recurrent_step_slots", "gdn_chunk_forward", "gdn_recurrent_step", "workspace_size", "device_status",
     "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
     "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "DEV_BAD_SLOT", "ALGOS",
@@ -84,6 +85,11 @@ def load_library():
     lib.kda_gdn_recurrent_step.restype = ci
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ci] * 5 + [vp]
     lib.kda_recurrent_step.restype = ci
+    lib.kda_chunk_backward.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, ip] + \
+        [ci] * 8 + [vp, sz, vp]
+    lib.kda_chunk_backward.restype = ci
+    lib.kda_chunk_backward_workspace_size.argtypes = [ci] * 6
+    lib.kda_chunk_backward_workspace_size.restype = sz
     lib.kda_last_error.argtypes = []
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci, vp]
@@ -212,6 +218,52 @@ def chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *,
                                       _p(workspace), ws_bytes, st)
     _check(rc)
     return o, final_state
+
+
+def backward_workspace_size(B, T, H, dk, dv, num_seqs) -> int:
+    return int(load_library().kda_chunk_backward_workspace_size(B, T, H, dk, dv, num_seqs))
+
+
+def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=None, cu_seqlens=None, *,
+                   dinit_state=True, workspace=None, out=None):
+    """Gradients of sum <d_o, o> + <dfinal_state, final_state> through the chunked
+    prefill (kda_chunk_backward): a dict with dq, dk, dv (in q's dtype),
+    dlog_alpha, dbeta and dinit_state (float32; None when dinit_state=False).
+
+    Inputs are the forward call's, in the include/kda.h layouts; d_o has o's
+    shape and dtype, dfinal_state is float32 [N, H, dk, dv] or None (zero).
+    The workspace (uint8, CUDA) and the outputs (`out`, a dict with any of the
+    keys above) are allocated here unless given.  Device tensors only.
+    """
+    B, T, H, dk, dv, N = _prefill_args(q, k, v, log_alpha, beta, init_state, cu_seqlens)
+    if d_o.shape != v.shape or d_o.dtype != q.dtype:
+        raise ValueError("d_o must have o's shape and dtype")
+    if dfinal_state is not None and (dfinal_state.shape != (N, H, dk, dv) or dfinal_state.dtype != torch.float32):
+        raise ValueError("dfinal_state must be float32 [N, H, dk, dv]")
+    _need_cuda(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, cu_seqlens)
+    lib = load_library()
+    g = dict(out or {})
+    dev = q.device
+    g.setdefault("dq", torch.empty_like(q))
+    g.setdefault("dk", torch.empty_like(k))
+    g.setdefault("dv", torch.empty_like(v))
+    g.setdefault("dlog_alpha", torch.empty_like(log_alpha))
+    g.setdefault("dbeta", torch.empty_like(beta))
+    if dinit_state:
+        g.setdefault("dinit_state", torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev))
+    else:
+        g["dinit_state"] = None
+    _need_cuda(*g.values())
+    need = int(lib.kda_chunk_backward_workspace_size(B, T, H, dk, dv, N))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.kda_chunk_backward(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(d_o),
+                                _p(dfinal_state), _p(g["dq"]), _p(g["dk"]), _p(g["dv"]), _p(g["dlog_alpha"]),
+                                _p(g["dbeta"]), _p(g["dinit_state"]), _p(cu_seqlens), B, T, H, dk, dv, N,
+                                _dtype_code(q), CHUNK, _p(workspace), ws_bytes, _stream(dev))
+    _check(rc)
+    return g
 
 
 def chunk_forward_static_ws(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, o=None,

@@ -10,6 +10,7 @@
 #include "kda_chunk_simt.cuh"
 #include "kda_chunk_tc.cuh"
 #include "kda_chunk_2pass.cuh"
+#include "kda_bwd_simt.cuh"
 
 namespace {
 
@@ -236,6 +237,37 @@ int decode_impl(const void *q, const void *k, const void *v, const float *log_al
     return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d", dk, dv);
 }
 
+template <int DK, typename Tin>
+int launch_backward(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                    const float *init_state, const void *d_o, const float *dfinal, void *dq, void *dk_out,
+                    void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state, const int32_t *cu_seqlens,
+                    long long tokens, int T, int H, int dv, int num_seqs, void *workspace, cudaStream_t st) {
+    namespace b = kda::bwd;
+    constexpr size_t sm1 = b::SweepSmem<DK>::bytes, sm2 = b::ChunkSmem<DK>::bytes;
+    auto k1 = b::bwd_sweep_kernel<DK, Tin>;
+    auto k2 = b::bwd_chunk_kernel<DK, Tin>;
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(bwd_sweep)");
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(bwd_chunk)");
+    const long long slots = b::chunk_slots(tokens, num_seqs);
+    float *hs = (float *)workspace;
+    float *part = tokens > 0 ? hs + (size_t)slots * H * DK * dv : nullptr;
+    k1<<<dim3(dv / b::DVT, H, num_seqs), b::NT, sm1, st>>>(
+        (const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta, init_state, (const Tin *)d_o, dfinal,
+        (Tin *)dv_out, dinit_state, cu_seqlens, T, H, dv, hs, part);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "bwd_sweep launch");
+    if (tokens > 0) {
+        k2<<<dim3((unsigned)slots, H), b::NT, sm2, st>>>((const Tin *)q, (const Tin *)k, log_alpha, beta,
+                                                         cu_seqlens, T, H, dv, num_seqs, part, (Tin *)dq,
+                                                         (Tin *)dk_out, dlog_alpha, dbeta);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "bwd_chunk launch");
+    }
+    return KDA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -383,6 +415,51 @@ int kda_gdn_recurrent_step(const void *q, const void *k, const void *v, const fl
     if (rc || N == 0) return rc;
     return decode_impl(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype, nullptr, 0, true,
                        (cudaStream_t)stream);
+}
+
+size_t kda_chunk_backward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs) {
+    if (B < 1 || T < 0 || H < 1 || num_seqs < 0 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
+    return kda::bwd::backward_workspace_bytes((long long)B * T, H, dk, dv, num_seqs);
+}
+
+int kda_chunk_backward(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, const float *init_state, const void *d_o,
+                       const float *dfinal_state, void *dq, void *dk_out, void *dv_out, float *dlog_alpha,
+                       float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
+                       int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
+                       void *stream) {
+    // The forward checks cover the inputs (o stands in for d_o).
+    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, cu_seqlens, B, T, H, dk, dv,
+                           num_seqs, dtype, chunk);
+    if (rc) return rc;
+    if (T > 0 && (!dq || !dk_out || !dv_out || !dlog_alpha || !dbeta))
+        return fail(KDA_ERR_INVALID_ARG, "dq, dk, dv, dlog_alpha and dbeta are required");
+    const void *p16[] = {dq, dk_out, dv_out, dlog_alpha, dinit_state};
+    const char *n16[] = {"dq", "dk", "dv", "dlog_alpha", "dinit_state"};
+    for (int i = 0; i < 5; ++i)
+        if (p16[i] && !aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
+    if (dbeta && !aligned(dbeta, 4)) return fail(KDA_ERR_MISALIGNED, "dbeta is not 4-byte aligned");
+    const long long tokens = (long long)B * T;
+    const size_t need = kda::bwd::backward_workspace_bytes(tokens, H, dk, dv, num_seqs);
+    if (need > 0 && (!workspace || ws_bytes < need))
+        return fail(KDA_ERR_WORKSPACE, "backward workspace of %zu bytes needed, %zu given%s", need, ws_bytes,
+                    workspace ? "" : " (NULL)");
+    if (workspace && !aligned(workspace, 16)) return fail(KDA_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+    if (kda::bwd::chunk_slots(tokens, num_seqs) > 0x7fffffffLL)
+        return fail(KDA_ERR_UNSUPPORTED, "too many chunk slots for one grid");
+    if (num_seqs == 0) return KDA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+#define KDA_BWD(DKv, TT)                                                                                      \
+    return launch_backward<DKv, TT>(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, \
+                                    dlog_alpha, dbeta, dinit_state, cu_seqlens, tokens, T, H, dv, num_seqs,     \
+                                    workspace, st)
+    if (dtype == KDA_BF16) {
+        if (dk == 64) KDA_BWD(64, __nv_bfloat16);
+        KDA_BWD(128, __nv_bfloat16);
+    }
+    if (dk == 64) KDA_BWD(64, float);
+    KDA_BWD(128, float);
+#undef KDA_BWD
 }
 
 int kda_get_device_status(unsigned int *bits, int clear, void *stream) {

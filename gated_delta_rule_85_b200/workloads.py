@@ -12,6 +12,7 @@ Distributions (per the workload definitions):
               one per (token, head) for the scalar gate of Gated DeltaNet
   beta      = sigmoid(x), x ~ N(0, 1), fp32, one value per (token, head)
   states    ~ N(0, 0.01^2) fp32 (std 0.01), or zeros
+  backward cotangents: d_o ~ N(0, 1) in the input dtype, dfinal_state ~ N(0, 1) fp32
 Every tensor is drawn from its own generator seeded with (seed, stream id), so
 one tensor's draw does not depend on another's size.  Large tensors are drawn
 in token slices of fixed size so device memory for temporaries stays bounded.
@@ -24,7 +25,7 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-_STREAM = {"q": 1, "k": 2, "v": 3, "log_alpha": 4, "beta": 5, "init_state": 6}
+_STREAM = {"q": 1, "k": 2, "v": 3, "log_alpha": 4, "beta": 5, "init_state": 6, "d_o": 7, "dfinal_state": 8}
 _SLICE_TOKENS = 1 << 15
 
 
@@ -154,6 +155,17 @@ def prefill_inputs(shape: PrefillShape, seed: int = 0, device="cpu") -> dict:
     d["cu_seqlens"] = (None if shape.cu_seqlens is None
                        else torch.tensor(shape.cu_seqlens, dtype=torch.int32, device=device))
     return d
+
+
+def backward_cotangents(shape: PrefillShape, seed: int = 0, device="cpu", dfinal: bool = True) -> dict:
+    """dL/do [B, T, H, dv] (input dtype) and dL/dfinal_state [N, H, dk, dv] fp32 (or None)."""
+    B, T, H, dk, dv = shape.B, shape.T, shape.H, shape.dk, shape.dv
+    d_o = draw_v((B, T, H, dv), device, seed, _STREAM["d_o"], shape.dtype)
+    dS = None
+    if dfinal:
+        dS = torch.empty((shape.num_seqs, H, dk, dv), dtype=torch.float32, device=device)
+        dS.normal_(0.0, 1.0, generator=_gen(device, seed, _STREAM["dfinal_state"]))
+    return {"d_o": d_o, "dfinal_state": dS}
 
 
 def decode_step_inputs(shape: DecodeShape, step: int, seed: int = 0, device="cpu") -> dict:

@@ -264,6 +264,49 @@ int kda_gdn_recurrent_step(const void *q, const void *k, const void *v, const fl
                            const float *beta, float *state, void *o, int N, int H, int dk, int dv, int dtype,
                            void *stream);
 
+/*
+ * Backward of the chunked prefill: the gradients of
+ *     L = sum_t <d_o_t, o_t> + <dfinal_state, final_state>
+ * with respect to every input of kda_chunk_forward -- what the chunkwise
+ * training algorithm needs ("Kimi Linear、独自の土俵でFull Attentionを上回る"
+ * (remio.ai), § "Kimi Linearがより賢いRecurrent Memoryを使う方法"), for the
+ * recurrence of "Kimi Delta Attention 徹底解説" (tech-tide.dev),
+ * § "Kimi Delta Attention の仕組み".  fp32 arithmetic on CUDA cores with the
+ * exact pairwise decay (no range precondition), for dtype KDA_BF16 and KDA_F32.
+ *
+ *   q, k, v, log_alpha, beta, init_state, cu_seqlens, B, T, H, dk, dv,
+ *   num_seqs, dtype, chunk
+ *                 the forward call's inputs, layouts and rules as in
+ *                 kda_chunk_forward (init_state NULL = zeros).
+ *   d_o           [B, T, H, dv] in dtype: dL/do.
+ *   dfinal_state  fp32 [N, H, dk, dv] or NULL (zero): dL/dfinal_state.
+ *   dq, dk_out    [B, T, H, dk] in dtype;  dv_out [B, T, H, dv] in dtype.
+ *   dlog_alpha    fp32 [B, T, H, dk];  dbeta fp32 [B, T, H].
+ *   dinit_state   fp32 [N, H, dk, dv], or NULL (not computed): dL/dinit_state,
+ *                 the gradient at the given initial state (at zero when
+ *                 init_state is NULL).
+ *   workspace     device memory of at least kda_chunk_backward_workspace_size()
+ *                 bytes for the same sizes, 16-byte aligned; no contents are
+ *                 required.  Per (64-token chunk slot, head) it holds the fp32
+ *                 state at the chunk's start (4 dk dv bytes) and the partial
+ *                 sums of every 32-column value tile (about 132 KB per tile at
+ *                 dk = 128).  Calls that can overlap in time need separate
+ *                 workspaces.
+ * The caller owns every buffer; all pointers except cu_seqlens and beta are
+ * 16-byte aligned.  Every gradient is overwritten, not accumulated; tokens
+ * outside every sequence (packed input with cu_seqlens[N] < T) are not written.
+ * Errors: as kda_chunk_forward, plus KDA_ERR_WORKSPACE for a missing or small
+ * workspace; nothing is launched on an error.
+ */
+size_t kda_chunk_backward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs);
+
+int kda_chunk_backward(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, const float *init_state, const void *d_o,
+                       const float *dfinal_state, void *dq, void *dk_out, void *dv_out, float *dlog_alpha,
+                       float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
+                       int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
+                       void *stream);
+
 /* Message for the calling thread's last non-OK return ("" if none). */
 const char *kda_last_error(void);
 

@@ -162,3 +162,49 @@ def test_slot_entry_points_reject(lib):
     assert dec(A[9] + 1, 8) == MISALIGNED
     assert lib.kda_recurrent_step_slots(A[0], A[1], A[2], A[3], A[4], A[5], A[9], A[6], 0, 2, 128, 128, 8, 0,
                                         None) == OK   # no sequences: nothing to do
+
+
+# backward workspace per (chunk slot, head): the fp32 chunk-start state (4 dk dv
+# bytes) and, per 32-column value tile, 3 [64][dk] + 2 [64][64] + 64 + dk floats
+def bwd_ws(slots, H, dk, dv):
+    part = 3 * 64 * dk + 2 * 64 * 64 + 64 + dk
+    return slots * H * (dk * dv + (dv // 32) * part) * 4
+
+
+def test_backward_workspace_sizes(lib):
+    f = lib.kda_chunk_backward_workspace_size
+    assert f(1, 8192, 32, 128, 128, 1) == bwd_ws(129, 32, 128, 128)
+    assert f(3, 100, 2, 64, 64, 3) == bwd_ws(5 + 3, 2, 64, 64)
+    assert f(1, 100, 2, 128, 64, 1) == bwd_ws(2 + 1, 2, 128, 64)
+    assert f(2, 0, 2, 128, 128, 2) == 0          # no tokens
+    assert f(1, 100, 2, 96, 128, 1) == 0         # unsupported dk
+
+
+def backward(lib, **over):
+    a = dict(q=A[0], k=A[1], v=A[2], g=A[3], b=A[4], s0=A[5], do=A[6], dF=A[7], dq=A[8], dk_=A[9], dv_=A[10],
+             dg=A[11], db=A[11] + 0x8000, ds0=A[11] + 0x4000, cu=None, B=1, T=128, H=2, dk=128, dv=128, N=1,
+             dtype=0, chunk=64, ws=A[0] + 0x8000, wsb=1 << 30, st=None)
+    a.update(over)
+    return lib.kda_chunk_backward(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["do"], a["dF"], a["dq"],
+                                  a["dk_"], a["dv_"], a["dg"], a["db"], a["ds0"], a["cu"], a["B"], a["T"], a["H"],
+                                  a["dk"], a["dv"], a["N"], a["dtype"], a["chunk"], a["ws"], a["wsb"], a["st"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(do=None), INVALID),
+    (dict(dq=None), INVALID),
+    (dict(db=None), INVALID),
+    (dict(N=2), INVALID),
+    (dict(dk=96), UNSUPPORTED),
+    (dict(chunk=32), UNSUPPORTED),
+    (dict(dtype=5), UNSUPPORTED),
+    (dict(do=A[6] + 8), MISALIGNED),
+    (dict(dg=A[11] + 4), MISALIGNED),
+    (dict(ds0=A[11] + 0x4000 + 8), MISALIGNED),
+    (dict(db=A[11] + 0x8000 + 2), MISALIGNED),
+    (dict(ws=None, wsb=0), WORKSPACE),
+    (dict(wsb=1000), WORKSPACE),
+])
+def test_backward_rejects(lib, over, code):
+    assert backward(lib, **over) == code
+    assert lib.kda_last_error().decode() != ""

@@ -1,0 +1,159 @@
+"""Backward of the chunked prefill (kda_chunk_backward) against the fp64 oracle's
+reverse-mode gradients of the token recurrence, on the same inputs.
+
+The loss is L = sum <d_o, o> + <dfinal_state, final_state> with seeded
+cotangents; every gradient (dq, dk, dv, dlog_alpha, dbeta, dinit_state) is
+compared element by element.  The backward computes in fp32 from the exact
+input values, so the operator's bounds apply: rel-L2 <= 1e-4 for fp32 inputs;
+for bf16 inputs rel-L2 <= 1e-2 and max-abs <= 5e-2 relative to the largest
+reference magnitude (gradients are not O(1) quantities like o and S).
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_85_b200 as kda
+import oracle
+from gated_delta_rule_85_b200.workloads import PrefillShape, backward_cotangents, prefill_inputs, to_f64
+from kda_testutil import max_abs, rel_l2
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+BF16 = torch.bfloat16
+GRADS = ["dq", "dk", "dv", "dlog_alpha", "dbeta", "dinit_state"]
+
+
+def _pick(x, heads, axis):
+    if x is None:
+        return None
+    if heads is not None:
+        x = x.index_select(axis, torch.as_tensor(heads, device=x.device))
+    return to_f64(x)
+
+
+def oracle_grads(d, c, heads=None):
+    cu = None if d.get("cu_seqlens") is None else d["cu_seqlens"].cpu().numpy()
+    return oracle.backward(*(_pick(d[n], heads, 2) for n in ("q", "k", "v", "log_alpha", "beta")),
+                           _pick(c["d_o"], heads, 2), init_state=_pick(d.get("init_state"), heads, 1),
+                           dfinal=_pick(c.get("dfinal_state"), heads, 1), cu_seqlens=cu)
+
+
+def check(got, want, dtype, heads=None, what=""):
+    for name in GRADS:
+        if got.get(name) is None:
+            continue
+        axis = 1 if name == "dinit_state" else 2
+        g = _pick(got[name], heads, axis)
+        w = want[name]
+        assert np.all(np.isfinite(g)), f"{what} {name}: non-finite"
+        r = rel_l2(g, w)
+        if dtype == torch.float32:
+            assert r <= 1e-4, f"{what} {name}: rel-L2 {r:.2e}"
+        else:
+            assert r <= 1e-2, f"{what} {name}: rel-L2 {r:.2e}"
+            scale = max(1.0, float(np.max(np.abs(w)))) if w.size else 1.0
+            m = max_abs(g, w)
+            assert m <= 5e-2 * scale, f"{what} {name}: max-abs {m:.2e} (scale {scale:.2e})"
+
+
+def run(d, c, **kw):
+    return kda.chunk_backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], c["d_o"], d.get("init_state"),
+                              c.get("dfinal_state"), d.get("cu_seqlens"), **kw)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, BF16])
+@pytest.mark.parametrize("B,T,H,dk,dv", [(2, 200, 2, 128, 128), (2, 130, 3, 64, 64), (1, 64, 2, 128, 64),
+                                         (3, 1, 2, 64, 128), (1, 333, 1, 128, 128)])
+def test_backward_matches_oracle(dtype, B, T, H, dk, dv):
+    shape = PrefillShape(B=B, T=T, H=H, dk=dk, dv=dv, dtype=dtype)
+    d = prefill_inputs(shape, 100 + T + dk, DEV)
+    c = backward_cotangents(shape, 200 + T, DEV)
+    got = run(d, c)
+    torch.cuda.synchronize()
+    check(got, oracle_grads(d, c), dtype, what=f"B{B} T{T} dk{dk} dv{dv}")
+    assert kda.device_status() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, BF16])
+def test_backward_packed_sequences(dtype):
+    """Packed input with empty, single-token, exact-chunk and ragged sequences;
+    equal bit for bit to running each sequence alone."""
+    lens = [0, 1, 63, 64, 65, 130, 7, 0]
+    cu = tuple(np.cumsum([0] + lens).tolist())
+    shape = PrefillShape(B=1, T=sum(lens), H=3, dk=128, dv=128, dtype=dtype, cu_seqlens=cu)
+    d = prefill_inputs(shape, 7, DEV)
+    c = backward_cotangents(shape, 8, DEV)
+    got = run(d, c)
+    torch.cuda.synchronize()
+    check(got, oracle_grads(d, c), dtype, what="packed")
+    for n, L in enumerate(lens):
+        a = cu[n]
+        one = {x: d[x][:, a:a + L] for x in ("q", "k", "v", "log_alpha", "beta")}
+        one["init_state"] = d["init_state"][n:n + 1]
+        co = {"d_o": c["d_o"][:, a:a + L], "dfinal_state": c["dfinal_state"][n:n + 1]}
+        g1 = run(one, co)
+        for name in GRADS:
+            whole = got[name][n:n + 1] if name == "dinit_state" else got[name][:, a:a + L]
+            assert torch.equal(whole, g1[name]), (n, name)
+
+
+def test_backward_without_states():
+    """init_state NULL (zeros) and dfinal_state NULL (zero cotangent): dinit_state is
+    the gradient at the zero state."""
+    shape = PrefillShape(B=2, T=150, H=2, dk=64, dv=128, dtype=torch.float32, init_state="none")
+    d = prefill_inputs(shape, 31, DEV)
+    assert d["init_state"] is None
+    c = backward_cotangents(shape, 32, DEV, dfinal=False)
+    got = run(d, c)
+    torch.cuda.synchronize()
+    check(got, oracle_grads(d, c), torch.float32, what="no states")
+    assert got["dinit_state"].abs().max().item() > 0
+
+
+def test_backward_no_tokens():
+    """T = 0: nothing to differentiate through; dinit_state = dfinal_state exactly."""
+    shape = PrefillShape(B=3, T=0, H=2, dk=128, dv=64, dtype=BF16)
+    d = prefill_inputs(shape, 5, DEV)
+    c = backward_cotangents(shape, 6, DEV)
+    got = run(d, c)
+    torch.cuda.synchronize()
+    assert torch.equal(got["dinit_state"], c["dfinal_state"])
+    c["dfinal_state"] = None
+    got = run(d, c)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(got["dinit_state"]).item() == 0
+
+
+def test_backward_is_deterministic():
+    shape = PrefillShape(B=1, T=300, H=4, dk=128, dv=128, dtype=BF16)
+    d = prefill_inputs(shape, 9, DEV)
+    c = backward_cotangents(shape, 10, DEV)
+    a = run(d, c)
+    b = run(d, c)
+    for name in GRADS:
+        assert torch.equal(a[name], b[name]), name
+
+
+def test_backward_skips_dinit_state():
+    shape = PrefillShape(B=1, T=100, H=2, dk=64, dv=64, dtype=BF16)
+    d = prefill_inputs(shape, 11, DEV)
+    c = backward_cotangents(shape, 12, DEV)
+    full = run(d, c)
+    part = run(d, c, dinit_state=False)
+    assert part["dinit_state"] is None
+    for name in GRADS[:-1]:
+        assert torch.equal(full[name], part[name]), name
+
+
+@pytest.mark.slow
+def test_backward_prefill_8k_sampled_heads():
+    """Full-size prefill_8k (B=1, T=8192, H=32, d=128, bf16) in one call; the oracle
+    runs on three of the 32 heads (heads are independent)."""
+    shape = PrefillShape(B=1, T=8192, H=32, dk=128, dv=128, dtype=BF16)
+    d = prefill_inputs(shape, 0, DEV)
+    c = backward_cotangents(shape, 0, DEV)
+    got = run(d, c)
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    heads = [0, 17, 31]
+    check(got, oracle_grads(d, c, heads), BF16, heads=heads, what="prefill_8k")
