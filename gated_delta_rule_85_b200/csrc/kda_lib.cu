@@ -237,33 +237,52 @@ int decode_impl(const void *q, const void *k, const void *v, const float *log_al
     return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d", dk, dv);
 }
 
+template <typename K>
+int set_smem(K kern, size_t bytes, const char *what) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, what);
+}
+
 template <int DK, typename Tin>
 int launch_backward(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                     const float *init_state, const void *d_o, const float *dfinal, void *dq, void *dk_out,
                     void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state, const int32_t *cu_seqlens,
                     long long tokens, int T, int H, int dv, int num_seqs, void *workspace, cudaStream_t st) {
     namespace b = kda::bwd;
-    constexpr size_t sm1 = b::SweepSmem<DK>::bytes, sm2 = b::ChunkSmem<DK>::bytes;
-    auto k1 = b::bwd_sweep_kernel<DK, Tin>;
-    auto k2 = b::bwd_chunk_kernel<DK, Tin>;
-    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(bwd_sweep)");
-    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(bwd_chunk)");
-    const long long slots = b::chunk_slots(tokens, num_seqs);
-    float *hs = (float *)workspace;
-    float *part = tokens > 0 ? hs + (size_t)slots * H * DK * dv : nullptr;
-    k1<<<dim3(dv / b::DVT, H, num_seqs), b::NT, sm1, st>>>(
-        (const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta, init_state, (const Tin *)d_o, dfinal,
-        (Tin *)dv_out, dinit_state, cu_seqlens, T, H, dv, hs, part);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "bwd_sweep launch");
+    auto k_prep = b::bwd_prep_kernel<DK, Tin>;
+    auto k_state = b::bwd_state_kernel<DK, Tin>;
+    auto k_part = b::bwd_part_kernel<DK, Tin>;
+    auto k_chunk = b::bwd_chunk_kernel<DK, Tin>;
+    int rc;
+    if ((rc = set_smem(k_prep, b::PrepSmem<DK>::bytes, "cudaFuncSetAttribute(bwd_prep)"))) return rc;
+    if ((rc = set_smem(k_state, b::StateSmem<DK>::bytes, "cudaFuncSetAttribute(bwd_state)"))) return rc;
+    if ((rc = set_smem(k_part, b::PartSmem<DK>::bytes, "cudaFuncSetAttribute(bwd_part)"))) return rc;
+    if ((rc = set_smem(k_chunk, b::ChunkSmem<DK>::bytes, "cudaFuncSetAttribute(bwd_chunk)"))) return rc;
+    const long long slots = tokens > 0 ? b::chunk_slots(tokens, num_seqs) : 0;
+    const size_t sh = (size_t)slots * H;
+    float *rec = (float *)workspace;
+    float *ckpt = tokens > 0 ? rec + sh * b::Rec<DK>::FLOATS : nullptr;
+    float *dckpt = tokens > 0 ? ckpt + sh * DK * dv : nullptr;
+    float *part = tokens > 0 ? dckpt + sh * DK * dv : nullptr;
+    const dim3 per_chunk((unsigned)slots, H);
+    cudaError_t e;
     if (tokens > 0) {
-        k2<<<dim3((unsigned)slots, H), b::NT, sm2, st>>>((const Tin *)q, (const Tin *)k, log_alpha, beta,
-                                                         cu_seqlens, T, H, dv, num_seqs, part, (Tin *)dq,
-                                                         (Tin *)dk_out, dlog_alpha, dbeta);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "bwd_chunk launch");
+        k_prep<<<per_chunk, b::NT, b::PrepSmem<DK>::bytes, st>>>((const Tin *)q, (const Tin *)k, log_alpha, beta,
+                                                                  cu_seqlens, T, H, num_seqs, rec);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_prep launch");
+    }
+    k_state<<<dim3(2 * (dv / b::DVT), H, num_seqs), b::NT, b::StateSmem<DK>::bytes, st>>>(
+        (const Tin *)v, init_state, (const Tin *)d_o, dfinal, dinit_state, cu_seqlens, T, H, dv, rec, ckpt, dckpt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_state launch");
+    if (tokens > 0) {
+        k_part<<<per_chunk, b::NT, b::PartSmem<DK>::bytes, st>>>((const Tin *)v, beta, (const Tin *)d_o,
+                                                                  (Tin *)dv_out, cu_seqlens, T, H, dv, num_seqs,
+                                                                  rec, ckpt, dckpt, part);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_part launch");
+        k_chunk<<<per_chunk, b::NT, b::ChunkSmem<DK>::bytes, st>>>((const Tin *)q, (const Tin *)k, log_alpha,
+                                                                    beta, cu_seqlens, T, H, num_seqs, part,
+                                                                    (Tin *)dq, (Tin *)dk_out, dlog_alpha, dbeta);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_chunk launch");
     }
     return KDA_OK;
 }

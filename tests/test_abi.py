@@ -164,11 +164,13 @@ def test_slot_entry_points_reject(lib):
                                         None) == OK   # no sequences: nothing to do
 
 
-# backward workspace per (chunk slot, head): the fp32 chunk-start state (4 dk dv
-# bytes) and, per 32-column value tile, 3 [64][dk] + 2 [64][64] + 64 + dk floats
+# backward workspace per (chunk slot, head), fp32: the chunk record (3 [64][dk]
+# + 5 [64][64] + [dk][64] + dk), the state at the chunk's start and the adjoint at
+# its end ([dk][dv] each), and the column sums (3 [64][dk] + 2 [64][64] + 64 + dk)
 def bwd_ws(slots, H, dk, dv):
+    rec = 3 * 64 * dk + 5 * 64 * 64 + dk * 64 + dk
     part = 3 * 64 * dk + 2 * 64 * 64 + 64 + dk
-    return slots * H * (dk * dv + (dv // 32) * part) * 4
+    return slots * H * (rec + 2 * dk * dv + part) * 4
 
 
 def test_backward_workspace_sizes(lib):
