@@ -152,14 +152,16 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1
 }
 
 // d[16 x 8] += A[16 x K] B[K x 8] for one warp.  Element (r, k) of A is
-// A[r * ar + k * ak], element (k, n) of B is B[k * bk + n * bn]; K is a multiple
-// of 8.  Lane (g = lane / 4, t = lane % 4) holds d rows g and g + 8, columns
+// A[r * ar + k * ak], element (k, n) of B is B[k * bk + n * bn]; K (a multiple
+// of 8) is a compile-time constant so the k-steps unroll.  Lane (g = lane / 4, t = lane % 4) holds d rows g and g + 8, columns
 // 2t and 2t + 1.  SPLIT sums hi.hi + hi.lo + lo.hi of the tf32 split operands.
-template <bool SPLIT>
+template <bool SPLIT, int K>
 __device__ __forceinline__ void warp_mma(float (&d)[4], const float *A, int ar, int ak, const float *B, int bk,
-                                         int bn, int K) {
+                                         int bn) {
+    static_assert(K % 8 == 0, "K must be a multiple of 8");
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const float *a_lo = A + g * ar + t * ak, *b_lo = B + t * bk + g * bn;
+#pragma unroll
     for (int k0 = 0; k0 < K; k0 += 8) {
         const float *a = a_lo + k0 * ak, *b = b_lo + k0 * bk;
         const float fa0 = a[0], fa1 = a[8 * ar], fa2 = a[4 * ak], fa3 = a[8 * ar + 4 * ak];
@@ -187,47 +189,100 @@ __device__ __forceinline__ void warp_tile_out(const float (&d)[4], int r0, int c
     epi(r0 + g + 8, c0 + 2 * t + 1, d[3]);
 }
 
-// Block product out[M x N] = A1 B1 (+ A2 B2), 16 x 8 output tiles dealt to the
-// warps round-robin; every output element goes once through epi(row, col, v).
-template <int M, int N, bool SPLIT, typename Epi>
+// d[TW][16 x 8] += A[16 x K] B[K x 8 TW] for one warp: a strip of TW adjacent
+// output tiles sharing the A fragment, so TW independent MMAs are in flight per
+// k-step instead of one dependent chain.
+template <bool SPLIT, int K, int TW>
+__device__ __forceinline__ void warp_mma_strip(float (&d)[TW][4], const float *A, int ar, int ak, const float *B,
+                                               int bk, int bn) {
+    static_assert(K % 8 == 0, "K must be a multiple of 8");
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const float *a_lo = A + g * ar + t * ak, *b_lo = B + t * bk + g * bn;
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const float *a = a_lo + k0 * ak;
+        const float fa0 = a[0], fa1 = a[8 * ar], fa2 = a[4 * ak], fa3 = a[8 * ar + 4 * ak];
+        const uint32_t a0 = to_tf32(fa0), a1 = to_tf32(fa1), a2 = to_tf32(fa2), a3 = to_tf32(fa3);
+        uint32_t l0 = 0, l1 = 0, l2 = 0, l3 = 0;
+        if (SPLIT) {
+            l0 = to_tf32(fa0 - __uint_as_float(a0));
+            l1 = to_tf32(fa1 - __uint_as_float(a1));
+            l2 = to_tf32(fa2 - __uint_as_float(a2));
+            l3 = to_tf32(fa3 - __uint_as_float(a3));
+        }
+#pragma unroll
+        for (int w = 0; w < TW; ++w) {
+            const float *b = b_lo + k0 * bk + w * 8 * bn;
+            const float fb0 = b[0], fb1 = b[4 * bk];
+            const uint32_t b0 = to_tf32(fb0), b1 = to_tf32(fb1);
+            if (SPLIT) {
+                const uint32_t m0 = to_tf32(fb0 - __uint_as_float(b0)), m1 = to_tf32(fb1 - __uint_as_float(b1));
+                mma_tf32(d[w], l0, l1, l2, l3, b0, b1);
+                mma_tf32(d[w], a0, a1, a2, a3, m0, m1);
+            }
+            mma_tf32(d[w], a0, a1, a2, a3, b0, b1);
+        }
+    }
+}
+
+// Block product out[M x N] = A1 B1 (+ A2 B2): each warp takes a strip of one
+// 16-row block by TW 8-column tiles; every output element goes once through
+// epi(row, col, v).
+template <int M, int N, bool SPLIT, int K1, int K2 = 0, typename Epi>
 __device__ __forceinline__ void block_mma(const float *A1, int ar1, int ak1, const float *B1, int bk1, int bn1,
-                                          int K1, const float *A2, int ar2, int ak2, const float *B2, int bk2,
-                                          int bn2, int K2, Epi &&epi) {
-    constexpr int NTN = N / 8, TILES = (M / 16) * NTN;
-    for (int tile = threadIdx.x >> 5; tile < TILES; tile += NT / 32) {
-        const int r0 = (tile / NTN) * 16, c0 = (tile % NTN) * 8;
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-        warp_mma<SPLIT>(d, A1 + r0 * ar1, ar1, ak1, B1 + c0 * bn1, bk1, bn1, K1);
-        if (K2) warp_mma<SPLIT>(d, A2 + r0 * ar2, ar2, ak2, B2 + c0 * bn2, bk2, bn2, K2);
-        warp_tile_out(d, r0, c0, epi);
+                                          const float *A2, int ar2, int ak2, const float *B2, int bk2, int bn2,
+                                          Epi &&epi) {
+    constexpr int NW = NT / 32, NTN = N / 8, TILES = (M / 16) * NTN;
+    constexpr int TW = TILES >= NW ? TILES / NW : 1;
+    static_assert(TILES % NW == 0 || TILES < NW, "tiles must spread evenly over the warps");
+    static_assert(NTN % TW == 0, "a strip stays inside one 16-row block");
+    constexpr int STRIPS = TILES / TW;
+    for (int strip = threadIdx.x >> 5; strip < STRIPS; strip += NW) {
+        const int r0 = (strip / (NTN / TW)) * 16, c0 = (strip % (NTN / TW)) * TW * 8;
+        float d[TW][4];
+#pragma unroll
+        for (int w = 0; w < TW; ++w) d[w][0] = d[w][1] = d[w][2] = d[w][3] = 0.f;
+        warp_mma_strip<SPLIT, K1, TW>(d, A1 + r0 * ar1, ar1, ak1, B1 + c0 * bn1, bk1, bn1);
+        if constexpr (K2 > 0) warp_mma_strip<SPLIT, K2, TW>(d, A2 + r0 * ar2, ar2, ak2, B2 + c0 * bn2, bk2, bn2);
+#pragma unroll
+        for (int w = 0; w < TW; ++w) warp_tile_out(d[w], r0, c0 + 8 * w, epi);
     }
 }
 
 // ------------------------------------------------------------------ chunk helpers
 
-// Loads one chunk's q (optional), k and log_alpha rows (zero past Lc) and
-// beta, then turns log_alpha into the running sum G (per channel).
+// Loads one chunk's q, k and log_alpha rows (zero past Lc) and beta (if sB),
+// then turns log_alpha into the running sum G (per channel).  Every thread
+// issues all of its 4-element vector loads before the first shared store.
 template <int DK, typename Tin>
 __device__ __forceinline__ void load_chunk_qkg(const Tin *__restrict__ q, const Tin *__restrict__ k,
                                                const float *__restrict__ log_alpha, const float *__restrict__ beta,
                                                long long cs, int Lc, int H, int h, float *sQ, float *sK, float *sG,
                                                float *sB) {
     constexpr int DKP = Pad<DK>::K;
+    constexpr int NV = C * DK / 4 / NT;   // 4-element vectors per thread and tensor
     const int tid = threadIdx.x;
-    for (int idx = tid; idx < C * DK; idx += NT) {
-        const int i = idx / DK, c = idx % DK;
-        float qv = 0.f, kv = 0.f, gv = 0.f;
+    float4 rq[NV], rk[NV], rg[NV];
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int e = (tid + u * NT) * 4, i = e / DK, c = e % DK;
+        rq[u] = rk[u] = rg[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (i < Lc) {
             const long long off = ((cs + i) * H + h) * DK + c;
-            if (sQ) qv = Elem<Tin>::load(q + off);
-            kv = Elem<Tin>::load(k + off);
-            gv = log_alpha[off];
+            rq[u] = load4(q + off);
+            rk[u] = load4(k + off);
+            rg[u] = *reinterpret_cast<const float4 *>(log_alpha + off);
         }
-        if (sQ) sQ[i * DKP + c] = qv;
-        sK[i * DKP + c] = kv;
-        sG[i * DKP + c] = gv;
     }
-    for (int i = tid; i < C; i += NT) sB[i] = i < Lc ? beta[(cs + i) * H + h] : 0.f;
+    const float bv = (sB && tid < C && tid < Lc) ? beta[(cs + tid) * H + h] : 0.f;
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int e = (tid + u * NT) * 4, i = e / DK, c = e % DK;
+        *reinterpret_cast<float4 *>(sQ + i * DKP + c) = rq[u];
+        *reinterpret_cast<float4 *>(sK + i * DKP + c) = rk[u];
+        *reinterpret_cast<float4 *>(sG + i * DKP + c) = rg[u];
+    }
+    if (sB && tid < C) sB[tid] = bv;
     __syncthreads();
     for (int c = tid; c < DK; c += NT) {
         float acc = 0.f;
@@ -239,27 +294,103 @@ __device__ __forceinline__ void load_chunk_qkg(const Tin *__restrict__ q, const 
     __syncthreads();
 }
 
-// Akk (strictly lower) and Aqk (lower with the diagonal), zero elsewhere, with
-// the exact pairwise decay.  Row i is paired with row 63 - i for balance.
-template <int DK>
+__device__ __forceinline__ void cp_async16(float *dst, const float *src) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most one committed group (the most recent) is still in flight.
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// rows x cols fp32 (cols a multiple of 4; source rows src_ld apart, default
+// cols) into shared rows of stride ld, as 16-byte asynchronous copies.
+__device__ __forceinline__ void async_rows(float *dst, int ld, const float *src, int rows, int cols,
+                                           long long src_ld = -1) {
+    const int q4 = cols / 4;
+    const long long sld = src_ld < 0 ? cols : src_ld;
+    for (int idx = threadIdx.x; idx < rows * q4; idx += NT) {
+        const int r = idx / q4, c4 = (idx % q4) * 4;
+        cp_async16(dst + r * ld + c4, src + r * sld + c4);
+    }
+}
+
+// 16-row sub-blocks of a chunk.  For i in a later block than j, with r the
+// first row of i's block (j < r <= i) or s the last row of j's block
+// (j <= s < i), the decay factors split into two factors that are both <= 1:
+//   e^{G_i - G_j} = e^{G_i - G_r} e^{G_r - G_j} = e^{G_i - G_s} e^{G_s - G_j}
+// so the off-diagonal blocks become products of decay-scaled operands on the
+// tensor cores; only the 16 x 16 diagonal blocks take the exact pairwise exponent.
+constexpr int SB = 16;             // sub-block rows
+constexpr int NSB = C / SB;        // sub-blocks per chunk
+constexpr int SCR_ROWS = C - SB;   // largest off-diagonal operand (48 rows)
+
+// Akk (strictly lower) and Aqk (lower with the diagonal), zero elsewhere.
+// scr holds 2 * SB + SCR_ROWS rows of stride DKP.
+template <int DK, bool SPLIT>
 __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, const float *sG, float *sAkk,
-                                            float *sAqk) {
+                                            float *sAqk, float *scr) {
     constexpr int DKP = Pad<DK>::K;
-    const int tid = threadIdx.x, l8 = tid & 7, ip = tid >> 3;
-    for (int half = 0; half < 2; ++half) {
-        const int i = half ? (C - 1 - ip) : ip;
-        for (int j = l8; j < C; j += 8) {
+    const int tid = threadIdx.x;
+    for (int idx = tid; idx < C * CP; idx += NT) {
+        sAkk[idx] = 0.f;
+        sAqk[idx] = 0.f;
+    }
+    __syncthreads();
+    // diagonal blocks, exact: 8 lanes per (i, j) pair, each lane DK / 8 channels
+    {
+        constexpr int PAIRS = NSB * SB * (SB + 1) / 2;
+        const int l8 = tid & 7;
+        for (int p = tid >> 3; p < PAIRS; p += NT / 8) {
+            const int b = p / (SB * (SB + 1) / 2);
+            int rem = p % (SB * (SB + 1) / 2), ii = 0;
+            while (rem > ii) rem -= ++ii;
+            const int i = b * SB + ii, j = b * SB + rem;   // rem <= ii
             float akk = 0.f, aqk = 0.f;
-            if (j <= i) {
-                for (int c = 0; c < DK; ++c) {
-                    const float kj = sK[j * DKP + c] * expf(sG[i * DKP + c] - sG[j * DKP + c]);
-                    akk = fmaf(sK[i * DKP + c], kj, akk);
-                    aqk = fmaf(sQ[i * DKP + c], kj, aqk);
-                }
+            for (int c = l8; c < DK; c += 8) {
+                const float kj = sK[j * DKP + c] * __expf(sG[i * DKP + c] - sG[j * DKP + c]);
+                akk = fmaf(sK[i * DKP + c], kj, akk);
+                aqk = fmaf(sQ[i * DKP + c], kj, aqk);
             }
-            sAkk[i * CP + j] = (j < i) ? akk : 0.f;
-            sAqk[i * CP + j] = aqk;
+            for (int o = 1; o < 8; o <<= 1) {
+                akk += __shfl_xor_sync(0xffffffffu, akk, o);
+                aqk += __shfl_xor_sync(0xffffffffu, aqk, o);
+            }
+            if (l8 == 0) {
+                if (j < i) sAkk[i * CP + j] = akk;
+                sAqk[i * CP + j] = aqk;
+            }
         }
+    }
+    // blocks below the diagonal: rows of block bi against rows j < r = 16 bi
+    float *sL = scr, *sR = scr + 2 * SB * DKP;   // [k; q] rows of block bi, then k_j e^{G_r - G_j}
+    for (int bi = 1; bi < NSB; ++bi) {
+        const int r = bi * SB;
+        __syncthreads();
+        for (int idx = tid; idx < SB * DK; idx += NT) {
+            const int ii = idx / DK, c = idx % DK, i = r + ii;
+            const float e = __expf(sG[i * DKP + c] - sG[r * DKP + c]);
+            sL[ii * DKP + c] = sK[i * DKP + c] * e;
+            sL[(SB + ii) * DKP + c] = sQ[i * DKP + c] * e;
+        }
+        for (int idx = tid; idx < r * DK; idx += NT) {
+            const int j = idx / DK, c = idx % DK;
+            sR[j * DKP + c] = sK[j * DKP + c] * __expf(sG[r * DKP + c] - sG[j * DKP + c]);
+        }
+        __syncthreads();
+        // [Akk; Aqk] rows of block bi = [k; q]-scaled rows times the scaled earlier keys
+        constexpr int NTN_MAX = SCR_ROWS / 8;
+        const int ntn = r / 8;
+        for (int t = tid >> 5; t < 2 * ntn; t += NT / 32) {
+            const int r0 = (t / ntn) * SB, c0 = (t % ntn) * 8;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_mma<SPLIT, DK>(d, sL + r0 * DKP, DKP, 1, sR + c0 * DKP, 1, DKP);
+            warp_tile_out(d, r0, c0, [&](int row, int j, float x) {
+                if (row < SB) sAkk[(r + row) * CP + j] = x;
+                else sAqk[(r + row - SB) * CP + j] = x;
+            });
+        }
+        (void)NTN_MAX;
     }
     __syncthreads();
 }
@@ -270,17 +401,32 @@ __device__ __forceinline__ void chunk_factors(float *sQ, float *sK, float *sG, f
     constexpr int DKP = Pad<DK>::K;
     for (int c = threadIdx.x; c < DK; c += NT) {
         const float gl = sG[(C - 1) * DKP + c];
-        sD[c] = expf(gl);
+        sD[c] = __expf(gl);
         for (int i = 0; i < C; ++i) {
             const float gi = sG[i * DKP + c];
-            const float e = expf(gi);
+            const float e = __expf(gi);
             const float kc = sK[i * DKP + c];
             sQ[i * DKP + c] *= e;
             sK[i * DKP + c] = kc * e;
-            sG[i * DKP + c] = kc * expf(gl - gi);
+            sG[i * DKP + c] = kc * __expf(gl - gi);
         }
     }
     __syncthreads();
+}
+
+// Block row BI (rows r..r+15, r = 16 BI) of T = (I + Diag(beta) Akk)^{-1} below
+// the diagonal, from its diagonal block and the block rows above:
+//   Y = Diag(beta) Akk[r..r+16)[0..r) T[0..r)[0..r)   (in scr)
+//   T[r..r+16)[0..r) = -T[r..r+16)[r..r+16) Y
+template <bool SPLIT, int BI>
+__device__ __forceinline__ void t_block_row(const float *sAkk, const float *sB, float *sT, float *scr) {
+    constexpr int r = BI * SB;
+    __syncthreads();
+    block_mma<SB, r, SPLIT, r>(sAkk + r * CP, CP, 1, sT, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
+                               [&](int ii, int j, float x) { scr[ii * CP + j] = sB[r + ii] * x; });
+    __syncthreads();
+    block_mma<SB, r, SPLIT, SB>(sT + r * CP + r, CP, 1, scr, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
+                                [&](int ii, int j, float x) { sT[(r + ii) * CP + j] = -x; });
 }
 
 // ------------------------------------------------------------------ prep
@@ -295,7 +441,8 @@ struct PrepSmem {
     static constexpr int aqk = akk + C * CP;     // [C][CP]
     static constexpr int ti = aqk + C * CP;      // [C][CP]  T
     static constexpr int tb = ti + C * CP;       // [C][CP]  Tb
-    static constexpr int b = tb + C * CP;        // [C]
+    static constexpr int scr = tb + C * CP;      // [2 SB + SCR_ROWS][DKP] Gram operands
+    static constexpr int b = scr + (2 * SB + SCR_ROWS) * DKP;   // [C]
     static constexpr int d = b + C;              // [DK]
     static constexpr int total = d + DK;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
@@ -319,24 +466,28 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
     if (!chunk_of_slot(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
 
     load_chunk_qkg<DK, Tin>(q, k, log_alpha, beta, cs, Lc, H, h, sQ, sK, sG, sB);
-    chunk_grams<DK>(sQ, sK, sG, sAkk, sAqk);
+    chunk_grams<DK, SPLIT>(sQ, sK, sG, sAkk, sAqk, sm + L::scr);
     chunk_factors<DK>(sQ, sK, sG, sD);
-    // T = (I + Diag(beta) Akk)^{-1}, a column of the identity at a time:
-    // X_i = [i == col] - beta_i sum_{m<i} Akk[i][m] X_m; 8 lanes per column.
+    // T = (I + Diag(beta) Akk)^{-1}: the 16 x 16 diagonal blocks by forward
+    // substitution (4 lanes per column, all 64 columns at once), then each block
+    // row below the diagonal from the rows above it (t_block_row).
+    for (int idx = tid; idx < C * CP; idx += NT) sT[idx] = 0.f;
+    __syncthreads();
     {
-        const int l8 = tid & 7;
-        for (int col = tid >> 3; col < C; col += NT / 8) {
-            for (int i = 0; i < C; ++i) {
-                float part = 0.f;
-                for (int m = l8; m < i; m += 8) part = fmaf(sAkk[i * CP + m], sT[m * CP + col], part);
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                part += __shfl_xor_sync(0xffffffffu, part, 4);
-                if (l8 == 0) sT[i * CP + col] = (i == col ? 1.f : 0.f) - sB[i] * part;
-                __syncwarp();
-            }
+        const int prob = tid >> 2, l4 = tid & 3, b0 = (prob / SB) * SB, col = prob % SB;
+        for (int ii = 0; ii < SB; ++ii) {
+            const int i = b0 + ii;
+            float part = 0.f;
+            for (int m = l4; m < ii; m += 4) part = fmaf(sAkk[i * CP + b0 + m], sT[(b0 + m) * CP + b0 + col], part);
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            if (l4 == 0) sT[i * CP + b0 + col] = (ii == col ? 1.f : 0.f) - sB[i] * part;
+            __syncwarp();
         }
     }
+    t_block_row<SPLIT, 1>(sAkk, sB, sT, sm + L::scr);
+    t_block_row<SPLIT, 2>(sAkk, sB, sT, sm + L::scr);
+    t_block_row<SPLIT, 3>(sAkk, sB, sT, sm + L::scr);
     __syncthreads();
     for (int idx = tid; idx < C * C; idx += NT) {
         const int i = idx / C, j = idx % C;
@@ -359,13 +510,16 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
         r[R::TB + idx] = sTb[i * CP + j];
     }
     // Pt = Aqk Tb;  Kt = Kb^T Tb
-    block_mma<C, C, SPLIT>(sAqk, CP, 1, sTb, CP, 1, C, nullptr, 0, 0, nullptr, 0, 0, 0,
+    block_mma<C, C, SPLIT, C>(sAqk, CP, 1, sTb, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
                            [&](int i, int j, float x) { r[R::PT + i * C + j] = x; });
-    block_mma<DK, C, SPLIT>(sG, 1, DKP, sTb, CP, 1, C, nullptr, 0, 0, nullptr, 0, 0, 0,
+    block_mma<DK, C, SPLIT, C>(sG, 1, DKP, sTb, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
                             [&](int c, int j, float x) { r[R::KT + c * C + j] = x; });
 }
 
 // ------------------------------------------------------------------ state sweeps
+
+constexpr int SV = 64;        // value columns per state-sweep CTA
+constexpr int SVP = SV + 4;   // padded row stride of [*][SV] tiles
 
 template <int DK>
 struct StateSmem {
@@ -374,14 +528,20 @@ struct StateSmem {
     static constexpr int qh = kh + C * DKP;      // [C][DKP]  Qh (backward)
     static constexpr int kt = qh + C * DKP;      // [DK][CP]  Kt
     static constexpr int pt = kt + DK * CP;      // [C][CP]   Pt (backward)
-    static constexpr int s = pt + C * CP;        // [DK][TP]  S or dS
-    static constexpr int x = s + DK * TP;        // [C][TP]   V or dO
-    static constexpr int y = x + C * TP;         // [C][TP]   W or -mu
-    static constexpr int d = y + C * TP;         // [DK]
+    static constexpr int s = pt + C * CP;        // [DK][SVP] S or dS
+    static constexpr int x = s + DK * SVP;       // [C][SVP]  V or dO
+    static constexpr int y = x + C * SVP;        // [C][SVP]  W or -mu
+    static constexpr int d = y + C * SVP;        // [DK]      e^{G_C}
     static constexpr int total = d + DK;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
 
+// Each chunk is two products, and each product's record matrices are one group
+// of asynchronous copies issued while the other product runs:
+//   forward   A: W = V - Kh S            {Kh}          B: S <- Diag(D) S + Kt W     {Kt, D}
+//   backward  A: -mu = -(Pt^T dO + Kt^T dS) {Pt, Kt}   B: dS <- Diag(D) dS + Qh^T dO + Kh^T (-mu)  {Qh, Kh, D}
+// Groups are committed in the order A(0), B(0), A(1), B(1), ... (empty past the
+// last chunk), so "all but the most recent group done" is always the one needed.
 template <int DK, typename Tin>
 __global__ void __launch_bounds__(NT, 1)
 bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state, const Tin *__restrict__ d_o,
@@ -392,13 +552,13 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
     using R = Rec<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     float *sKh = sm + L::kh, *sQh = sm + L::qh, *sKt = sm + L::kt, *sPt = sm + L::pt;
     float *sS = sm + L::s, *sX = sm + L::x, *sY = sm + L::y, *sD = sm + L::d;
     const int tid = threadIdx.x;
-    const int ntile = DV / DVT;
+    const int ntile = DV / SV;
     const bool backward = blockIdx.x >= ntile;
-    const int tile = blockIdx.x % ntile, col_base = tile * DVT, h = blockIdx.y;
+    const int tile = blockIdx.x % ntile, col_base = tile * SV, h = blockIdx.y;
     const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
     long long t0, t1;
     seq_span(cu_seqlens, T, n, t0, t1);
@@ -406,61 +566,101 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
     const int nch = (int)((t1 - t0 + C - 1) / C);
     const long long st_off = ((long long)n * H + h) * DK * DV + col_base;
     const float *src = backward ? dfinal : init_state;
-    for (int idx = tid; idx < DK * DVT; idx += NT) {
-        const int c = idx / DVT, j = idx % DVT;
-        sS[c * TP + j] = src ? src[st_off + (long long)c * DV + j] : 0.f;
+    for (int idx = tid; idx < DK * SV; idx += NT) {
+        const int c = idx / SV, j = idx % SV;
+        sS[c * SVP + j] = src ? src[st_off + (long long)c * DV + j] : 0.f;
     }
+    auto rec_of = [&](int step) {
+        const int ci = backward ? nch - 1 - step : step;
+        return rec + ((first + ci) * H + h) * (long long)R::FLOATS;
+    };
+    auto issue_a = [&](int step) {
+        if (step < nch) {
+            const float *rp = rec_of(step);
+            if (backward) {
+                async_rows(sPt, CP, rp + R::PT, C, C);
+                async_rows(sKt, CP, rp + R::KT, DK, C);
+            } else {
+                async_rows(sKh, DKP, rp + R::KH, C, DK);
+            }
+        }
+        cp_async_commit();
+    };
+    auto issue_b = [&](int step) {
+        if (step < nch) {
+            const float *rp = rec_of(step);
+            if (backward) {
+                async_rows(sQh, DKP, rp + R::QH, C, DK);
+                async_rows(sKh, DKP, rp + R::KH, C, DK);
+            } else {
+                async_rows(sKt, CP, rp + R::KT, DK, C);
+            }
+            async_rows(sD, DK, rp + R::D, 1, DK);
+        }
+        cp_async_commit();
+    };
+    // V (forward) or dO (backward) rows of a chunk, this thread's share, in registers
+    constexpr int XPT = C * SV / NT;
+    float xr[XPT];
+    const Tin *xin = backward ? d_o : v;
+    auto load_x = [&](int step, float (&out)[XPT]) {
+        const int ci = backward ? nch - 1 - step : step;
+        const long long cs = t0 + (long long)ci * C;
+        const int Lc = (int)min((long long)C, t1 - cs);
+#pragma unroll
+        for (int u = 0; u < XPT; ++u) {
+            const int idx = tid + u * NT, i = idx / SV, j = idx % SV;
+            out[u] = i < Lc ? Elem<Tin>::load(xin + ((cs + i) * H + h) * DV + col_base + j) : 0.f;
+        }
+    };
+    issue_a(0);
+    issue_b(0);
     for (int step = 0; step < nch; ++step) {
         const int ci = backward ? nch - 1 - step : step;
         const long long cs = t0 + (long long)ci * C;
         const int Lc = (int)min((long long)C, t1 - cs);
         const long long slot = first + ci;
-        const float *rp = rec + (slot * H + h) * R::FLOATS;
-        __syncthreads();
+        __syncthreads();   // S (or dS) final for this chunk; X free
         // checkpoint: the state at the chunk's start (forward) or the adjoint at its end
         float *cp = (backward ? dckpt : ckpt) + (slot * H + h) * (long long)DK * DV + col_base;
-        for (int idx = tid; idx < DK * DVT; idx += NT) {
-            const int c = idx / DVT, j = idx % DVT;
-            cp[(long long)c * DV + j] = sS[c * TP + j];
+        for (int idx = tid; idx < DK * SV; idx += NT) {
+            const int c = idx / SV, j = idx % SV;
+            cp[(long long)c * DV + j] = sS[c * SVP + j];
         }
-        const Tin *xin = backward ? d_o : v;
-        for (int idx = tid; idx < C * DVT; idx += NT) {
-            const int i = idx / DVT, j = idx % DVT;
-            sX[i * TP + j] = i < Lc ? Elem<Tin>::load(xin + ((cs + i) * H + h) * DV + col_base + j) : 0.f;
+        if (step == 0) load_x(step, xr);
+#pragma unroll
+        for (int u = 0; u < XPT; ++u) {
+            const int idx = tid + u * NT, i = idx / SV, j = idx % SV;
+            sX[i * SVP + j] = xr[u];
         }
-        for (int idx = tid; idx < C * DK; idx += NT) {
-            const int i = idx / DK, c = idx % DK;
-            sKh[i * DKP + c] = rp[R::KH + idx];
-            if (backward) sQh[i * DKP + c] = rp[R::QH + idx];
-        }
-        for (int idx = tid; idx < DK * C; idx += NT) sKt[(idx / C) * CP + idx % C] = rp[R::KT + idx];
-        if (backward)
-            for (int idx = tid; idx < C * C; idx += NT) sPt[(idx / C) * CP + idx % C] = rp[R::PT + idx];
-        for (int c = tid; c < DK; c += NT) sD[c] = rp[R::D + c];
+        cp_async_wait_prev();   // group A of this chunk
         __syncthreads();
-        if (!backward) {
-            // W = V - Kh S
-            block_mma<C, DVT, SPLIT>(sKh, DKP, 1, sS, TP, 1, DK, nullptr, 0, 0, nullptr, 0, 0, 0,
-                                     [&](int i, int j, float x) { sY[i * TP + j] = sX[i * TP + j] - x; });
-            __syncthreads();
-            // S <- Diag(D) S + Kt W
-            block_mma<DK, DVT, SPLIT>(sKt, CP, 1, sY, TP, 1, C, nullptr, 0, 0, nullptr, 0, 0, 0,
-                                      [&](int c, int j, float x) { sS[c * TP + j] = sD[c] * sS[c * TP + j] + x; });
-        } else {
-            // -mu = -(Pt^T dO + Kt^T dS)
-            block_mma<C, DVT, SPLIT>(sPt, 1, CP, sX, TP, 1, C, sKt, 1, CP, sS, TP, 1, DK,
-                                     [&](int i, int j, float x) { sY[i * TP + j] = -x; });
-            __syncthreads();
-            // dS <- Diag(D) dS + Qh^T dO + Kh^T (-mu)
-            block_mma<DK, DVT, SPLIT>(sQh, 1, DKP, sX, TP, 1, C, sKh, 1, DKP, sY, TP, 1, C,
-                                      [&](int c, int j, float x) { sS[c * TP + j] = sD[c] * sS[c * TP + j] + x; });
-        }
+        if (!backward)
+            block_mma<C, SV, SPLIT, DK>(sKh, DKP, 1, sS, SVP, 1, nullptr, 0, 0, nullptr, 0, 0,
+                                    [&](int i, int j, float x) { sY[i * SVP + j] = sX[i * SVP + j] - x; });
+        else
+            block_mma<C, SV, SPLIT, C, DK>(sPt, 1, CP, sX, SVP, 1, sKt, 1, CP, sS, SVP, 1,
+                                    [&](int i, int j, float x) { sY[i * SVP + j] = -x; });
+        __syncthreads();   // group A's buffers are free
+        issue_a(step + 1);
+        if (step + 1 < nch) load_x(step + 1, xr);   // next chunk's V or dO, in flight during product B
+        cp_async_wait_prev();   // group B of this chunk
+        __syncthreads();
+        if (!backward)
+            block_mma<DK, SV, SPLIT, C>(sKt, CP, 1, sY, SVP, 1, nullptr, 0, 0, nullptr, 0, 0,
+                                     [&](int c, int j, float x) { sS[c * SVP + j] = sD[c] * sS[c * SVP + j] + x; });
+        else
+            block_mma<DK, SV, SPLIT, C, C>(sQh, 1, DKP, sX, SVP, 1, sKh, 1, DKP, sY, SVP, 1,
+                                     [&](int c, int j, float x) { sS[c * SVP + j] = sD[c] * sS[c * SVP + j] + x; });
+        __syncthreads();   // group B's buffers are free
+        issue_b(step + 1);
     }
+    cp_async_wait_all();
     __syncthreads();
     if (backward && dinit_state) {
-        for (int idx = tid; idx < DK * DVT; idx += NT) {
-            const int c = idx / DVT, j = idx % DVT;
-            dinit_state[st_off + (long long)c * DV + j] = sS[c * TP + j];
+        for (int idx = tid; idx < DK * SV; idx += NT) {
+            const int c = idx / SV, j = idx % SV;
+            dinit_state[st_off + (long long)c * DV + j] = sS[c * SVP + j];
         }
     }
 }
@@ -512,18 +712,13 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
     int Lc;
     if (!chunk_of_slot(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
     const float *rp = rec + ((long long)slot * H + h) * R::FLOATS;
-    for (int idx = tid; idx < C * DK; idx += NT) {
-        const int i = idx / DK, c = idx % DK;
-        sKh[i * DKP + c] = rp[R::KH + idx];
-        sKb[i * DKP + c] = rp[R::KB + idx];
-    }
-    for (int idx = tid; idx < C * C; idx += NT) {
-        const int i = idx / C, j = idx % C;
-        sAkk[i * CP + j] = rp[R::AKK + idx];
-        sAqk[i * CP + j] = rp[R::AQK + idx];
-        sT[i * CP + j] = rp[R::TI + idx];
-        sTb[i * CP + j] = rp[R::TB + idx];
-    }
+    async_rows(sKh, DKP, rp + R::KH, C, DK);
+    async_rows(sKb, DKP, rp + R::KB, C, DK);
+    async_rows(sAkk, CP, rp + R::AKK, C, C);
+    async_rows(sAqk, CP, rp + R::AQK, C, C);
+    async_rows(sT, CP, rp + R::TI, C, C);
+    async_rows(sTb, CP, rp + R::TB, C, C);
+    cp_async_commit();
     for (int i = tid; i < C; i += NT) {
         sB[i] = i < Lc ? beta[(cs + i) * H + h] : 0.f;
         sDB[i] = 0.f;
@@ -542,32 +737,45 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
     for (int tile = 0; tile < DV / DVT; ++tile) {
         const int col_base = tile * DVT;
         __syncthreads();   // the previous tile is done with every buffer
-        for (int idx = tid; idx < DK * DVT; idx += NT) {
-            const int c = idx / DVT, j = idx % DVT;
-            sS[c * TP + j] = ckpt[st_base + (long long)c * DV + col_base + j];
-            sdS[c * TP + j] = dckpt[st_base + (long long)c * DV + col_base + j];
+        async_rows(sS, TP, ckpt + st_base + col_base, DK, DVT, DV);
+        async_rows(sdS, TP, dckpt + st_base + col_base, DK, DVT, DV);
+        cp_async_commit();
+        {
+            constexpr int NV = C * DVT / 4 / NT;   // 4-element vectors of V and dO per thread
+            float4 rv[NV], rd[NV];
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const int e = (tid + u * NT) * 4, i = e / DVT, j = e % DVT;
+                rv[u] = rd[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < Lc) {
+                    const long long off = ((cs + i) * H + h) * DV + col_base + j;
+                    rv[u] = load4(v + off);
+                    rd[u] = load4(d_o + off);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const int e = (tid + u * NT) * 4, i = e / DVT, j = e % DVT;
+                *reinterpret_cast<float4 *>(sW + i * TP + j) = rv[u];
+                *reinterpret_cast<float4 *>(sDO + i * TP + j) = rd[u];
+            }
         }
-        for (int idx = tid; idx < C * DVT; idx += NT) {
-            const int i = idx / DVT, j = idx % DVT;
-            const long long off = ((cs + i) * H + h) * DV + col_base + j;
-            sW[i * TP + j] = i < Lc ? Elem<Tin>::load(v + off) : 0.f;
-            sDO[i * TP + j] = i < Lc ? Elem<Tin>::load(d_o + off) : 0.f;
-        }
+        cp_async_wait_all();
         __syncthreads();
         // W = V - Kh S (in place: each element is read and written by its owner only)
-        block_mma<C, DVT, SPLIT>(sKh, DKP, 1, sS, TP, 1, DK, nullptr, 0, 0, nullptr, 0, 0, 0,
+        block_mma<C, DVT, SPLIT, DK>(sKh, DKP, 1, sS, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sW[i * TP + j] -= x; });
         __syncthreads();
         // U = Tb W;  dU = Aqk^T dO + Kb dS
-        block_mma<C, DVT, SPLIT>(sTb, CP, 1, sW, TP, 1, C, nullptr, 0, 0, nullptr, 0, 0, 0,
+        block_mma<C, DVT, SPLIT, C>(sTb, CP, 1, sW, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sU[i * TP + j] = x; });
-        block_mma<C, DVT, SPLIT>(sAqk, 1, CP, sDO, TP, 1, C, sKb, DKP, 1, sdS, TP, 1, DK,
+        block_mma<C, DVT, SPLIT, C, DK>(sAqk, 1, CP, sDO, TP, 1, sKb, DKP, 1, sdS, TP, 1,
                                  [&](int i, int j, float x) { sdU[i * TP + j] = x; });
         __syncthreads();
         // R = W - Akk U (in place of W);  lam = T^T dU
-        block_mma<C, DVT, SPLIT>(sAkk, CP, 1, sU, TP, 1, C, nullptr, 0, 0, nullptr, 0, 0, 0,
+        block_mma<C, DVT, SPLIT, C>(sAkk, CP, 1, sU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sW[i * TP + j] -= x; });
-        block_mma<C, DVT, SPLIT>(sT, 1, CP, sdU, TP, 1, C, nullptr, 0, 0, nullptr, 0, 0, 0,
+        block_mma<C, DVT, SPLIT, C>(sT, 1, CP, sdU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sL[i * TP + j] = x; });
         __syncthreads();
         // dbeta: <lam_i, R_i> (one warp per 8 rows; the same lane adds every tile)
@@ -593,32 +801,47 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
 #pragma unroll
         for (int r = 0; r < TQ; ++r) {
             const int t2 = warp + r * NW, r0 = (t2 / (DK / 8)) * 16, c0 = (t2 % (DK / 8)) * 8;
-            warp_mma<SPLIT>(a_dq[r], sDO + r0 * TP, TP, 1, sS + c0 * TP, 1, TP, DVT);
-            warp_mma<SPLIT>(a_dkh[r], sL + r0 * TP, TP, 1, sS + c0 * TP, 1, TP, DVT);
-            warp_mma<SPLIT>(a_dkb[r], sU + r0 * TP, TP, 1, sdS + c0 * TP, 1, TP, DVT);
+            warp_mma<SPLIT, DVT>(a_dq[r], sDO + r0 * TP, TP, 1, sS + c0 * TP, 1, TP);
+            warp_mma<SPLIT, DVT>(a_dkh[r], sL + r0 * TP, TP, 1, sS + c0 * TP, 1, TP);
+            warp_mma<SPLIT, DVT>(a_dkb[r], sU + r0 * TP, TP, 1, sdS + c0 * TP, 1, TP);
         }
 #pragma unroll
         for (int r = 0; r < TA; ++r) {
             const int t2 = warp + r * NW, r0 = (t2 / (C / 8)) * 16, c0 = (t2 % (C / 8)) * 8;
-            warp_mma<SPLIT>(a_aq[r], sDO + r0 * TP, TP, 1, sU + c0 * TP, 1, TP, DVT);
-            warp_mma<SPLIT>(a_ak[r], sL + r0 * TP, TP, 1, sU + c0 * TP, 1, TP, DVT);
+            warp_mma<SPLIT, DVT>(a_aq[r], sDO + r0 * TP, TP, 1, sU + c0 * TP, 1, TP);
+            warp_mma<SPLIT, DVT>(a_ak[r], sL + r0 * TP, TP, 1, sU + c0 * TP, 1, TP);
         }
         if (tid < DK)
             for (int j = 0; j < DVT; ++j) a_gc = fmaf(sS[tid * TP + j], sdS[tid * TP + j], a_gc);
     }
     float *pp = part + ((long long)slot * H + h) * P::FLOATS;
+    {
+        const int lane = tid & 31, g = lane >> 2, t = lane & 3;
+        auto put = [&](float *base, int ld, const float (&d)[4], int r0, int c0, float sgn) {
+            *reinterpret_cast<float2 *>(base + (r0 + g) * ld + c0 + 2 * t) = make_float2(sgn * d[0], sgn * d[1]);
+            *reinterpret_cast<float2 *>(base + (r0 + g + 8) * ld + c0 + 2 * t) = make_float2(sgn * d[2], sgn * d[3]);
+        };
 #pragma unroll
-    for (int r = 0; r < TQ; ++r) {
-        const int t2 = warp + r * NW, r0 = (t2 / (DK / 8)) * 16, c0 = (t2 % (DK / 8)) * 8;
-        warp_tile_out(a_dq[r], r0, c0, [&](int i, int c, float x) { pp[P::DQ + i * DK + c] = x; });
-        warp_tile_out(a_dkh[r], r0, c0, [&](int i, int c, float x) { pp[P::DKH + i * DK + c] = -x; });
-        warp_tile_out(a_dkb[r], r0, c0, [&](int i, int c, float x) { pp[P::DKB + i * DK + c] = x; });
-    }
+        for (int r = 0; r < TQ; ++r) {
+            const int t2 = warp + r * NW, r0 = (t2 / (DK / 8)) * 16, c0 = (t2 % (DK / 8)) * 8;
+            put(pp + P::DQ, DK, a_dq[r], r0, c0, 1.f);
+            put(pp + P::DKH, DK, a_dkh[r], r0, c0, -1.f);
+            put(pp + P::DKB, DK, a_dkb[r], r0, c0, 1.f);
+        }
 #pragma unroll
-    for (int r = 0; r < TA; ++r) {
-        const int t2 = warp + r * NW, r0 = (t2 / (C / 8)) * 16, c0 = (t2 % (C / 8)) * 8;
-        warp_tile_out(a_aq[r], r0, c0, [&](int i, int j, float x) { pp[P::AQK + i * C + j] = j <= i ? x : 0.f; });
-        warp_tile_out(a_ak[r], r0, c0, [&](int i, int j, float x) { pp[P::AKK + i * C + j] = j < i ? -x : 0.f; });
+        for (int r = 0; r < TA; ++r) {
+            const int t2 = warp + r * NW, r0 = (t2 / (C / 8)) * 16, c0 = (t2 % (C / 8)) * 8;
+            // keep j <= i of dAqk and j < i of dAkk; zero the rest
+            float aq[4], ak[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = r0 + g + (e >> 1) * 8, j = c0 + 2 * t + (e & 1);
+                aq[e] = j <= i ? a_aq[r][e] : 0.f;
+                ak[e] = j < i ? -a_ak[r][e] : 0.f;
+            }
+            put(pp + P::AQK, C, aq, r0, c0, 1.f);
+            put(pp + P::AKK, C, ak, r0, c0, 1.f);
+        }
     }
     __syncthreads();
     for (int i = tid; i < C; i += NT) pp[P::DB + i] = sDB[i];
@@ -629,17 +852,134 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
 
 template <int DK>
 struct ChunkSmem {
-    static constexpr int q = 0;                  // [C][DK]
-    static constexpr int k = q + C * DK;         // [C][DK]
-    static constexpr int g = k + C * DK;         // [C][DK] G
-    static constexpr int dk = g + C * DK;        // [C][DK] row terms of dk
-    static constexpr int dg = dk + C * DK;       // [C][DK] row terms of dG
-    static constexpr int ck = dg + C * DK;       // [C][DK] column terms
-    static constexpr int da = ck + C * DK;       // [C][CP] dAqk (j <= i) and dAkk (stored at [j][i], j < i)
-    static constexpr int gc = da + C * CP;       // [NT / 2] per row group: sum_i k_i b_i (a dG_C term)
-    static constexpr int total = gc + NT / 2;
+    static constexpr int DKP = Pad<DK>::K;
+    static constexpr int q = 0;                  // [C][DKP]
+    static constexpr int k = q + C * DKP;        // [C][DKP]
+    static constexpr int g = k + C * DKP;        // [C][DKP] G
+    static constexpr int acc = g + C * DKP;      // [C][DKP] dq, then dk
+    static constexpr int dg = acc + C * DKP;     // [C][DKP] dG
+    static constexpr int aq = dg + C * DKP;      // [C][CP]  dAqk (lower with the diagonal)
+    static constexpr int ak = aq + C * CP;       // [C][CP]  dAkk (strictly lower)
+    static constexpr int scr = ak + C * CP;      // [SCR_ROWS][DKP] decay-scaled operand
+    static constexpr int total = scr + SCR_ROWS * DKP;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
+
+// Pair terms of the diagonal 16 x 16 blocks, exact, one thread per (channel,
+// block): rows  acc_i += sum_{j<=i} A1[i][j] k_j E_ij (+ k_i times that into dG
+// when rows_to_dg), and with A2 (dk phase) the column terms
+// acc_j += sum_{i>=j} (A1[i][j] q_i + [i>j] A2[i][j] k_i) E_ij, dG_j -= k_j (that),
+// plus the row terms of A2.  Q phase: A1 = dAqk, no A2.  K phase: A1 = dAqk
+// (columns only), A2 = dAkk (rows and columns).
+template <int DK, bool KPHASE>
+__device__ __forceinline__ void diag_pair_terms(const float *sQ, const float *sK, const float *sG, const float *sAq,
+                                                const float *sAk, float *sAcc, float *sDg) {
+    constexpr int DKP = Pad<DK>::K;
+    constexpr int NG = NT / DK;   // thread groups per channel
+    const int c = threadIdx.x % DK, grp = threadIdx.x / DK;
+    for (int b = grp; b < NSB; b += NG) {
+        const int r = b * SB;
+        float colacc[SB];
+#pragma unroll
+        for (int jj = 0; jj < SB; ++jj) colacc[jj] = 0.f;
+#pragma unroll
+        for (int ii = 0; ii < SB; ++ii) {
+            const int i = r + ii;
+            const float gi = sG[i * DKP + c], qi = sQ[i * DKP + c], ki = sK[i * DKP + c];
+            float row = 0.f;
+#pragma unroll
+            for (int jj = 0; jj <= ii; ++jj) {
+                const int j = r + jj;
+                const float e = __expf(gi - sG[j * DKP + c]);
+                if (!KPHASE) {
+                    row = fmaf(sAq[i * CP + j], sK[j * DKP + c] * e, row);
+                } else {
+                    const float akk = jj < ii ? sAk[i * CP + j] : 0.f;
+                    row = fmaf(akk, sK[j * DKP + c] * e, row);
+                    colacc[jj] = fmaf(fmaf(sAq[i * CP + j], qi, akk * ki), e, colacc[jj]);
+                }
+            }
+            sAcc[i * DKP + c] += row;
+            if (KPHASE) sDg[i * DKP + c] += ki * row;
+        }
+        if (KPHASE) {
+#pragma unroll
+            for (int jj = 0; jj < SB; ++jj) {
+                const int j = r + jj;
+                sAcc[j * DKP + c] += colacc[jj];
+                sDg[j * DKP + c] -= sK[j * DKP + c] * colacc[jj];
+            }
+        }
+    }
+}
+
+// Row terms of the blocks below the diagonal: for block bi (rows r..r+15),
+// acc_i += e^{G_i - G_r} sum_{j<r} A[i][j] (k_j e^{G_r - G_j}); dG_i += k_i (that)
+// when to_dg.
+template <int DK, bool SPLIT, int BI>
+__device__ __forceinline__ void offdiag_row_block(const float *sK, const float *sG, const float *sA, float *scr,
+                                                  float *sAcc, float *sDg, bool to_dg) {
+    constexpr int DKP = Pad<DK>::K, r = BI * SB;
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < r * DK; idx += NT) {
+        const int j = idx / DK, c = idx % DK;
+        scr[j * DKP + c] = sK[j * DKP + c] * __expf(sG[r * DKP + c] - sG[j * DKP + c]);
+    }
+    __syncthreads();
+    block_mma<SB, DK, SPLIT, r>(sA + r * CP, CP, 1, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
+                                [&](int ii, int c, float x) {
+                                    const int i = r + ii;
+                                    x *= __expf(sG[i * DKP + c] - sG[r * DKP + c]);
+                                    sAcc[i * DKP + c] += x;
+                                    if (to_dg) sDg[i * DKP + c] += sK[i * DKP + c] * x;
+                                });
+}
+
+template <int DK, bool SPLIT>
+__device__ __forceinline__ void offdiag_rows(const float *sK, const float *sG, const float *sA, float *scr,
+                                             float *sAcc, float *sDg, bool to_dg) {
+    static_assert(NSB == 4, "three blocks below the diagonal");
+    offdiag_row_block<DK, SPLIT, 1>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+    offdiag_row_block<DK, SPLIT, 2>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+    offdiag_row_block<DK, SPLIT, 3>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+    __syncthreads();
+}
+
+// Column terms of the blocks below the diagonal: for block bj (columns
+// 16 bj..16 bj+15, last row s), acc_j += e^{G_s - G_j} sum_{i>s} A[i][j] (X_i e^{G_i - G_s})
+// and dG_j -= k_j (that), for (A, X) = (dAqk, q) and (dAkk, k).
+template <int DK, bool SPLIT, int BJ>
+__device__ __forceinline__ void offdiag_col_block(const float *sQ, const float *sK, const float *sG,
+                                                  const float *sAq, const float *sAk, float *scr, float *sAcc,
+                                                  float *sDg) {
+    constexpr int DKP = Pad<DK>::K, s = BJ * SB + SB - 1, n = C - 1 - s;   // rows s+1 .. C-1
+    for (int pass = 0; pass < 2; ++pass) {
+        const float *X = pass ? sK : sQ;
+        const float *A = pass ? sAk : sAq;
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < n * DK; idx += NT) {
+            const int ii = idx / DK, c = idx % DK, i = s + 1 + ii;
+            scr[ii * DKP + c] = X[i * DKP + c] * __expf(sG[i * DKP + c] - sG[s * DKP + c]);
+        }
+        __syncthreads();
+        block_mma<SB, DK, SPLIT, n>(A + (s + 1) * CP + BJ * SB, 1, CP, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
+                                    [&](int jj, int c, float x) {
+                                        const int j = BJ * SB + jj;
+                                        x *= __expf(sG[s * DKP + c] - sG[j * DKP + c]);
+                                        sAcc[j * DKP + c] += x;
+                                        sDg[j * DKP + c] -= sK[j * DKP + c] * x;
+                                    });
+    }
+}
+
+template <int DK, bool SPLIT>
+__device__ __forceinline__ void offdiag_cols(const float *sQ, const float *sK, const float *sG, const float *sAq,
+                                             const float *sAk, float *scr, float *sAcc, float *sDg) {
+    offdiag_col_block<DK, SPLIT, 0>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    offdiag_col_block<DK, SPLIT, 1>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    offdiag_col_block<DK, SPLIT, 2>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    __syncthreads();
+}
 
 template <int DK, typename Tin>
 __global__ void __launch_bounds__(NT, 1)
@@ -649,99 +989,92 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
                  float *__restrict__ dlog_alpha, float *__restrict__ dbeta) {
     using L = ChunkSmem<DK>;
     using P = Part<DK>;
+    constexpr int DKP = L::DKP;
+    constexpr bool SPLIT = sizeof(Tin) == 4;
     extern __shared__ float sm[];
-    float *sQ = sm + L::q, *sK = sm + L::k, *sG = sm + L::g, *sDk = sm + L::dk, *sDg = sm + L::dg;
-    float *sCk = sm + L::ck, *sDA = sm + L::da, *sGC = sm + L::gc;
+    float *sQ = sm + L::q, *sK = sm + L::k, *sG = sm + L::g, *sAcc = sm + L::acc, *sDg = sm + L::dg;
+    float *sAq = sm + L::aq, *sAk = sm + L::ak, *scr = sm + L::scr;
     const int tid = threadIdx.x, slot = blockIdx.x, h = blockIdx.y;
     long long cs;
     int Lc;
     if (!chunk_of_slot(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
     const float *pp = part + ((long long)slot * H + h) * P::FLOATS;
+    constexpr int NV = C * DK / 4 / NT;   // 4-element vectors per thread
+    // dAqk (zero above the diagonal) and dAkk (zero on and above it) by async copy
+    async_rows(sAq, CP, pp + P::AQK, C, C);
+    async_rows(sAk, CP, pp + P::AKK, C, C);
+    cp_async_commit();
+    for (int i = tid; i < Lc; i += NT) dbeta[(cs + i) * H + h] = pp[P::DB + i];
+    load_chunk_qkg<DK, Tin>(q, k, log_alpha, nullptr, cs, Lc, H, h, sQ, sK, sG, nullptr);
 
+    // ---- dq = e^G dQh + pair terms of dAqk;  dG = q dq
+    {
+        float4 r[NV];
+#pragma unroll
+        for (int u = 0; u < NV; ++u) r[u] = *reinterpret_cast<const float4 *>(pp + P::DQ + (tid + u * NT) * 4);
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int e = (tid + u * NT) * 4, i = e / DK, c = e % DK;
+            const float *g = sG + i * DKP + c;
+            *reinterpret_cast<float4 *>(sAcc + i * DKP + c) =
+                make_float4(__expf(g[0]) * r[u].x, __expf(g[1]) * r[u].y, __expf(g[2]) * r[u].z, __expf(g[3]) * r[u].w);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    diag_pair_terms<DK, false>(sQ, sK, sG, sAq, nullptr, sAcc, nullptr);
+    offdiag_rows<DK, SPLIT>(sK, sG, sAq, scr, sAcc, nullptr, false);
+    // dq out; dk starts at a + b and dG at q dq + k (a - b); sum_i k_i b_i per
+    // channel (a dG_C term) goes to scr, one row per group of rows
+    {
+        float4 ra[NV], rb[NV];
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            ra[u] = *reinterpret_cast<const float4 *>(pp + P::DKH + (tid + u * NT) * 4);
+            rb[u] = *reinterpret_cast<const float4 *>(pp + P::DKB + (tid + u * NT) * 4);
+        }
+        float kb[4] = {0.f, 0.f, 0.f, 0.f};
+        const int c = (tid * 4) % DK;   // the same 4 channels for every u (NT * 4 is a multiple of DK)
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int e = (tid + u * NT) * 4, i = e / DK;
+            const float ha[4] = {ra[u].x, ra[u].y, ra[u].z, ra[u].w}, hb[4] = {rb[u].x, rb[u].y, rb[u].z, rb[u].w};
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int o = i * DKP + c + v;
+                const float x = sAcc[o];
+                if (i < Lc) Elem<Tin>::store(dq + ((cs + i) * H + h) * DK + c + v, x);
+                const float gi = sG[o], gC = sG[(C - 1) * DKP + c + v];
+                const float a = __expf(gi) * ha[v], b = __expf(gC - gi) * hb[v];
+                const float kk = sK[o];
+                sDg[o] = sQ[o] * x + kk * (a - b);
+                sAcc[o] = a + b;
+                kb[v] = fmaf(kk, b, kb[v]);
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < 4; ++v) scr[((tid * 4) / DK) * DKP + c + v] = kb[v];
+    }
+    __syncthreads();
+    float kb_sum = 0.f;   // this thread's channel (tid < DK) of sum_i k_i b_i
+    if (tid < DK)
+        for (int gq = 0; gq < NT * 4 / DK; ++gq) kb_sum += scr[gq * DKP + tid];
+    __syncthreads();
+    // ---- dk = a + b + pair terms of dAkk (rows) and of dAqk, dAkk (columns)
+    diag_pair_terms<DK, true>(sQ, sK, sG, sAq, sAk, sAcc, sDg);
+    offdiag_rows<DK, SPLIT>(sK, sG, sAk, scr, sAcc, sDg, true);
+    offdiag_cols<DK, SPLIT>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
     for (int idx = tid; idx < C * DK; idx += NT) {
         const int i = idx / DK, c = idx % DK;
-        float qv = 0.f, kv = 0.f, gv = 0.f;
-        if (i < Lc) {
-            const long long off = ((cs + i) * H + h) * DK + c;
-            qv = Elem<Tin>::load(q + off);
-            kv = Elem<Tin>::load(k + off);
-            gv = log_alpha[off];
-        }
-        sQ[idx] = qv;
-        sK[idx] = kv;
-        sG[idx] = gv;
+        if (i < Lc) Elem<Tin>::store(dk_out + ((cs + i) * H + h) * DK + c, sAcc[i * DKP + c]);
     }
-    // dAqk on and below the diagonal, dAkk transposed above it
-    for (int idx = tid; idx < C * C; idx += NT) {
-        const int i = idx / C, j = idx % C;
-        if (j > i) continue;
-        sDA[i * CP + j] = pp[P::AQK + idx];
-        if (j < i) sDA[j * CP + i] = pp[P::AKK + idx];
-    }
-    for (int i = tid; i < Lc; i += NT) dbeta[(cs + i) * H + h] = pp[P::DB + i];
-    __syncthreads();
+    // ---- dG_C terms, then dlog_alpha_s = sum_{i>=s} dG_i
     for (int c = tid; c < DK; c += NT) {
-        float acc = 0.f;
-        for (int i = 0; i < C; ++i) {
-            acc += sG[i * DK + c];
-            sG[i * DK + c] = acc;
-        }
-    }
-    __syncthreads();
-
-    // Threads split into DK-wide groups: even groups take row terms (row i),
-    // odd groups column terms (column j); with 4 groups (DK = 64) each role
-    // alternates rows between its two groups.
-    constexpr int NG = NT / DK, NPART = NG / 2;
-    const int c = tid % DK, grp = tid / DK, role = grp & 1, prt = grp >> 1;
-    const float gC = sG[(C - 1) * DK + c];
-    if (role == 0) {
-        float kb_sum = 0.f;   // sum_i k_i b_i, a dG_C term
-        for (int i = prt; i < C; i += NPART) {
-            const float gi = sG[i * DK + c], qi = sQ[i * DK + c], ki = sK[i * DK + c];
-            const float eg = expf(gi);
-            const float dqh = eg * pp[P::DQ + i * DK + c], a = eg * pp[P::DKH + i * DK + c];
-            const float b = expf(gC - gi) * pp[P::DKB + i * DK + c];
-            float pq = 0.f, pk = 0.f;
-            for (int j = 0; j <= i; ++j) {
-                const float kj = sK[j * DK + c] * expf(gi - sG[j * DK + c]);
-                pq = fmaf(sDA[i * CP + j], kj, pq);
-                if (j < i) pk = fmaf(sDA[j * CP + i], kj, pk);
-            }
-            if (i < Lc) Elem<Tin>::store(dq + ((cs + i) * H + h) * DK + c, dqh + pq);
-            sDk[i * DK + c] = a + b + pk;
-            sDg[i * DK + c] = qi * (dqh + pq) + ki * (a - b + pk);
-            kb_sum = fmaf(ki, b, kb_sum);
-        }
-        sGC[prt * DK + c] = kb_sum;
-    } else {
-        for (int j = prt; j < C; j += NPART) {
-            const float gj = sG[j * DK + c];
-            float acc = 0.f;
-            for (int i = j; i < C; ++i) {
-                const float e = expf(sG[i * DK + c] - gj);
-                float x = sDA[i * CP + j] * sQ[i * DK + c];
-                if (i > j) x = fmaf(sDA[j * CP + i], sK[i * DK + c], x);
-                acc = fmaf(x, e, acc);
-            }
-            sCk[j * DK + c] = acc;
-        }
-    }
-    __syncthreads();
-    // dk = row + column terms; dG = row dG - k (column terms); dG_C; dlog_alpha = reverse cumsum
-    for (int idx = tid; idx < C * DK; idx += NT) {
-        const int i = idx / DK, cc = idx % DK;
-        const float ck = sCk[idx];
-        if (i < Lc) Elem<Tin>::store(dk_out + ((cs + i) * H + h) * DK + cc, sDk[idx] + ck);
-        sDg[idx] -= sK[idx] * ck;
-    }
-    __syncthreads();
-    for (int cc = tid; cc < DK; cc += NT) {
-        float acc = expf(sG[(C - 1) * DK + cc]) * pp[P::DGC + cc];
-        for (int p2 = 0; p2 < NPART; ++p2) acc += sGC[p2 * DK + cc];
+        const float gC = sG[(C - 1) * DKP + c];
+        float acc = __expf(gC) * pp[P::DGC + c] + kb_sum;
         for (int i = C - 1; i >= 0; --i) {
-            acc += sDg[i * DK + cc];
-            if (i < Lc) dlog_alpha[((cs + i) * H + h) * DK + cc] = acc;
+            acc += sDg[i * DKP + c];
+            if (i < Lc) dlog_alpha[((cs + i) * H + h) * DK + c] = acc;
         }
     }
 }

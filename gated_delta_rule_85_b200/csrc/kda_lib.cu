@@ -271,7 +271,7 @@ int launch_backward(const void *q, const void *k, const void *v, const float *lo
                                                                   cu_seqlens, T, H, num_seqs, rec);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_prep launch");
     }
-    k_state<<<dim3(2 * (dv / b::DVT), H, num_seqs), b::NT, b::StateSmem<DK>::bytes, st>>>(
+    k_state<<<dim3(2 * (dv / b::SV), H, num_seqs), b::NT, b::StateSmem<DK>::bytes, st>>>(
         (const Tin *)v, init_state, (const Tin *)d_o, dfinal, dinit_state, cu_seqlens, T, H, dv, rec, ckpt, dckpt);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_state launch");
     if (tokens > 0) {
