@@ -5,7 +5,8 @@ One step = one chunked prefill (kda_chunk_forward, tcgen05 kernel) of the
 "prefill_8k" workload: B=1, T=8192, H=32, dk=dv=128, bf16 q/k/v, fp32 gates,
 fp32 initial state, 64-token chunks.  The decode workload (N=256 sequences,
 H=32, one token per step through kda_recurrent_step, fresh inputs per step) is
-timed in the same run and reported under "decode".
+timed in the same run and reported under "decode"; the backward of the
+prefill_8k workload (kda_chunk_backward) under "backward_8k".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -39,6 +40,12 @@ STATE_BYTES = 4 * 128 * 128                                                   # 
 # plus the three C x d^2 state products): 10 C d + 6 d^2.
 PREFILL_FLOPS_PER_TOKEN_HEAD = 10 * CHUNK * 128 + 6 * 128 * 128               # 180224
 DECODE_BYTES_PER_PAIR = 2 * STATE_BYTES + PREFILL_BYTES_PER_TOKEN_HEAD        # 132612
+# Backward, per token-head: q, k, v, d_o (bf16) + log_alpha + beta read, dq, dk, dv
+# (bf16) + dlog_alpha + dbeta written; per (sequence, head) init_state and
+# dfinal_state read, dinit_state written.  Flops: the gradient of every forward
+# product is two products of the same size (recomputation is not credited).
+BACKWARD_BYTES_PER_TOKEN_HEAD = 4 * 2 * 128 + 4 * 128 + 4 + 3 * 2 * 128 + 4 * 128 + 4   # 2824
+BACKWARD_FLOPS_PER_TOKEN_HEAD = 2 * PREFILL_FLOPS_PER_TOKEN_HEAD                      # 360448
 # DRAM bytes (read + write) per launch from ncu captures of the current kernels on
 # these workloads (profiles/*.md); keyed by the kernels one step runs.  A kernel set
 # without a capture on its workload reports null.
@@ -46,6 +53,9 @@ NCU_TRAFFIC = {
     ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.7e6 + 182.0e6 + 308.3e6 + 54.0e6,
     ("prefill_8k", "chunk_tc_kernel"): 338.8e6 + 56.0e6,
     ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.7e6,
+    # backward: all four kernels of one call; T=2048 captured, T=8192 scaled by the chunk slots (129 / 33)
+    ("backward_T2048", "bwd"): 775.6e6 + 419.9e6,
+    ("backward_T8192", "bwd"): (775.6e6 + 419.9e6) * 129 / 33,
 }
 
 
@@ -255,6 +265,43 @@ def run_prefill_gdn(args, world, rank, dev):
     return dict(ms=ms, launches=reps * (2 if ws_n else 1))
 
 
+def run_backward(args, world, rank, dev):
+    """Backward of the prefill_8k workload (kda_chunk_backward), CUDA events per call."""
+    import torch
+
+    import gated_delta_rule_85_b200 as kda
+    from gated_delta_rule_85_b200.workloads import PrefillShape, backward_cotangents, prefill_inputs
+
+    cfg = dict(PREFILL, T=args.backward_T)
+    shape = PrefillShape(**cfg, dtype=torch.bfloat16)
+    d = prefill_inputs(shape, seed=rank, device=dev)
+    c = backward_cotangents(shape, seed=rank, device=dev)
+    ws = torch.empty(kda.backward_workspace_size(1, cfg["T"], cfg["H"], 128, 128, 1), dtype=torch.uint8,
+                     device=dev)
+    out = {}
+
+    def step():
+        out.update(kda.chunk_backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], c["d_o"],
+                                      d["init_state"], c["dfinal_state"], workspace=ws, out=out))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    reps = max(5, min(args.steps, 30))
+    _barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    del d, c, ws, out
+    return dict(ms=ms, launches=reps * 4)
+
+
 def run_prefill_varlen(args, world, rank, dev):
     """The 1,048,576-token packed (varlen) prefill: 22 sequences x 32 heads."""
     import torch
@@ -411,6 +458,36 @@ def main_reference(args):
     return 0
 
 
+def backward_block(args, world, bw, hbm_gbs, bf16_tflops):
+    T, H = args.backward_T, PREFILL["H"]
+    bbytes = T * H * BACKWARD_BYTES_PER_TOKEN_HEAD + 3 * H * STATE_BYTES
+    bflops = T * H * BACKWARD_FLOPS_PER_TOKEN_HEAD
+    bgbs = bbytes / (bw["ms"] * 1e-3) / 1e9
+    btf = bflops / (bw["ms"] * 1e-3) / 1e12
+    return {
+        "metric": f"KDA chunked backward tokens/s (gradients of the prefill: B=1, T={T}, H={H}, d=128)",
+        "value": world * T / (bw["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": bw["ms"],
+        "roofline": {"kernel": "bwd_prep_kernel + bwd_state_kernel + bwd_part_kernel + bwd_chunk_kernel",
+                     "bound": "hbm", "achieved": bgbs, "peak": hbm_gbs, "unit": "GB/s", "frac": bgbs / hbm_gbs,
+                     "traffic": NCU_TRAFFIC.get((f"backward_T{T}", "bwd")), "algorithmic_bytes": bbytes,
+                     "tensor": {"achieved_tflops": btf, "peak_tflops": bf16_tflops, "frac": btf / bf16_tflops,
+                                "algorithmic_flops": bflops}},
+    }
+
+
+def main_backward_only(args, world, rank, dev):
+    bw = run_backward(args, world, rank, dev)
+    hbm_gbs, bf16_tflops, _ = _peaks()
+    line = backward_block(args, world, bw, hbm_gbs, bf16_tflops)
+    line.update({"n_gpus": world, "steps": max(5, min(args.steps, 30)), "warmup": args.warmup,
+                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                 "data": "synthetic", "config": {"workload": f"backward T={args.backward_T} H=32 d=128 bf16"},
+                 "gpu_launches": bw["launches"]})
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -423,6 +500,10 @@ def main(argv=None):
     ap.add_argument("--no-varlen", action="store_true", help="skip the 1M-token packed prefill line")
     ap.add_argument("--no-slots", action="store_true", help="skip the state-pool decode line")
     ap.add_argument("--no-gdn", action="store_true", help="skip the Gated DeltaNet (scalar gate) prefill line")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward (gradients) line")
+    ap.add_argument("--only-backward", action="store_true",
+                    help="time only the backward and print its line (profiling a smaller --backward-T)")
+    ap.add_argument("--backward-T", type=int, default=PREFILL["T"], help="tokens of the backward workload")
     ap.add_argument("--algo", default="auto", choices=["auto", "fused", "two_pass"],
                     help="tensor-core prefill schedule of the headline line (kda_chunk_forward_ex)")
     args = ap.parse_args(argv)
@@ -447,11 +528,20 @@ def main(argv=None):
 
     kda.load_library()
 
+    if args.only_backward:
+        rc = main_backward_only(args, world, rank, dev)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+            dist.destroy_process_group()
+        return rc
     pre = run_prefill(args, world, rank, dev)
     dec = None if args.no_decode else run_decode(args, world, rank, dev)
     dsl = None if (args.no_decode or args.no_slots) else run_decode(args, world, rank, dev, pool_slots=512)
     vl = None if args.no_varlen else run_prefill_varlen(args, world, rank, dev)
     gd = None if args.no_gdn else run_prefill_gdn(args, world, rank, dev)
+    bw = None if args.no_backward else run_backward(args, world, rank, dev)
 
     hbm_gbs, bf16_tflops, peak_src = _peaks()
     ms_step = pre["total_ms"] / args.steps
@@ -509,6 +599,9 @@ def main(argv=None):
                          "tensor": {"achieved_tflops": gtf, "peak_tflops": bf16_tflops, "frac": gtf / bf16_tflops}},
         }
         line["gpu_launches"] += gd["launches"]
+    if bw is not None:
+        line["backward_8k"] = backward_block(args, world, bw, hbm_gbs, bf16_tflops)
+        line["gpu_launches"] += bw["launches"]
     if dsl is not None:
         step_ms = dsl["ms"] / dsl["launches"]
         dbytes = DECODE["N"] * DECODE["H"] * DECODE_BYTES_PER_PAIR + DECODE["N"] * 4   # + the slot table
