@@ -53,6 +53,7 @@
 #pragma once
 
 #include "kda_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace kda {
 namespace bwd {
@@ -71,21 +72,39 @@ struct Pad {
 
 inline long long chunk_slots(long long tokens, int num_seqs) { return (tokens + C - 1) / C + num_seqs; }
 
-// Per (chunk slot, head) record of bwd_prep_kernel, in floats.
+// Per (chunk slot, head) record of bwd_prep_kernel, in floats.  Rows carry the
+// shared-memory padding (stride DK + 4 or C + 4, pad entries unused), so each
+// matrix moves between global and shared memory as one bulk copy.
 template <int DK>
 struct Rec {
-    static constexpr int KH = 0;                 // [C][DK]  e^G k
-    static constexpr int QH = KH + C * DK;       // [C][DK]  e^G q
-    static constexpr int KB = QH + C * DK;       // [C][DK]  e^{G_C - G} k
-    static constexpr int AKK = KB + C * DK;      // [C][C]   strictly lower (zero elsewhere)
-    static constexpr int AQK = AKK + C * C;      // [C][C]   lower with the diagonal (zero above)
-    static constexpr int TI = AQK + C * C;       // [C][C]   T = (I + Diag(beta) Akk)^{-1}, unit lower
-    static constexpr int TB = TI + C * C;        // [C][C]   Tb = T Diag(beta)
-    static constexpr int PT = TB + C * C;        // [C][C]   Aqk Tb
-    static constexpr int KT = PT + C * C;        // [DK][C]  Kb^T Tb
-    static constexpr int D = KT + DK * C;        // [DK]     e^{G_C}
+    static constexpr int DKP = DK + 4, CPR = C + 4;
+    static constexpr int KH = 0;                 // [C][DKP]   e^G k
+    static constexpr int QH = KH + C * DKP;      // [C][DKP]   e^G q
+    static constexpr int KB = QH + C * DKP;      // [C][DKP]   e^{G_C - G} k
+    static constexpr int AKK = KB + C * DKP;     // [C][CPR]   strictly lower (zero elsewhere)
+    static constexpr int AQK = AKK + C * CPR;    // [C][CPR]   lower with the diagonal (zero above)
+    static constexpr int TI = AQK + C * CPR;     // [C][CPR]   T = (I + Diag(beta) Akk)^{-1}, unit lower
+    static constexpr int TB = TI + C * CPR;      // [C][CPR]   Tb = T Diag(beta)
+    static constexpr int PT = TB + C * CPR;      // [C][CPR]   Aqk Tb
+    static constexpr int KT = PT + C * CPR;      // [DK][CPR]  Kb^T Tb
+    static constexpr int D = KT + DK * CPR;      // [DK]       e^{G_C}
     static constexpr int FLOATS = D + DK;
+    static constexpr uint32_t ROWS_K = C * DKP * 4, ROWS_C = C * CPR * 4, KT_BYTES = DK * CPR * 4;
 };
+
+constexpr long long kWaitLimit = 2000000000ll;   // bounded waits: >= 1 s at any SM clock up to 2 GHz
+
+// Every thread waits for the next phase of a copy barrier; all agree on the
+// outcome.  False (and KDA_DEV_WAIT_TIMEOUT flagged) if it did not complete.
+__device__ __forceinline__ bool wait_copies(uint32_t mbar, uint32_t &phase) {
+    const bool ok = ptx::mbar_wait_bounded(mbar, phase, kWaitLimit);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+        if (threadIdx.x == 0) flag_status(KDA_DEV_WAIT_TIMEOUT);
+        return false;
+    }
+    return true;
+}
 
 // Per (chunk slot, head) sums over the value columns, in floats.
 template <int DK>
@@ -457,7 +476,7 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
     using R = Rec<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
-    extern __shared__ float sm[];
+    extern __shared__ __align__(128) float sm[];
     float *sQ = sm + L::q, *sK = sm + L::k, *sG = sm + L::g, *sAkk = sm + L::akk, *sAqk = sm + L::aqk;
     float *sT = sm + L::ti, *sTb = sm + L::tb, *sB = sm + L::b, *sD = sm + L::d;
     const int tid = threadIdx.x, slot = blockIdx.x, h = blockIdx.y;
@@ -495,25 +514,25 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
     }
     __syncthreads();
     float *r = rec + ((long long)slot * H + h) * R::FLOATS;
-    for (int idx = tid; idx < C * DK; idx += NT) {
-        const int i = idx / DK, c = idx % DK;
-        r[R::KH + idx] = sK[i * DKP + c];
-        r[R::QH + idx] = sQ[i * DKP + c];
-        r[R::KB + idx] = sG[i * DKP + c];
-    }
-    for (int c = tid; c < DK; c += NT) r[R::D + c] = sD[c];
-    for (int idx = tid; idx < C * C; idx += NT) {
-        const int i = idx / C, j = idx % C;
-        r[R::AKK + idx] = sAkk[i * CP + j];
-        r[R::AQK + idx] = sAqk[i * CP + j];
-        r[R::TI + idx] = sT[i * CP + j];
-        r[R::TB + idx] = sTb[i * CP + j];
+    // the shared-memory matrices already have the record's row layout: one bulk store each
+    if (tid == 0) {
+        ptx::fence_proxy_async_smem();
+        ptx::bulk_store(r + R::KH, ptx::smem_u32(sK), R::ROWS_K);
+        ptx::bulk_store(r + R::QH, ptx::smem_u32(sQ), R::ROWS_K);
+        ptx::bulk_store(r + R::KB, ptx::smem_u32(sG), R::ROWS_K);
+        ptx::bulk_store(r + R::AKK, ptx::smem_u32(sAkk), R::ROWS_C);
+        ptx::bulk_store(r + R::AQK, ptx::smem_u32(sAqk), R::ROWS_C);
+        ptx::bulk_store(r + R::TI, ptx::smem_u32(sT), R::ROWS_C);
+        ptx::bulk_store(r + R::TB, ptx::smem_u32(sTb), R::ROWS_C);
+        ptx::bulk_store(r + R::D, ptx::smem_u32(sD), DK * 4);
+        ptx::bulk_commit();
     }
     // Pt = Aqk Tb;  Kt = Kb^T Tb
     block_mma<C, C, SPLIT, C>(sAqk, CP, 1, sTb, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
-                           [&](int i, int j, float x) { r[R::PT + i * C + j] = x; });
+                              [&](int i, int j, float x) { r[R::PT + i * CP + j] = x; });
     block_mma<DK, C, SPLIT, C>(sG, 1, DKP, sTb, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
-                            [&](int c, int j, float x) { r[R::KT + c * C + j] = x; });
+                               [&](int c, int j, float x) { r[R::KT + c * CP + j] = x; });
+    if (tid == 0) ptx::bulk_wait_read_all();   // shared memory stays valid until the stores have read it
 }
 
 // ------------------------------------------------------------------ state sweeps
@@ -552,7 +571,7 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
     using R = Rec<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
-    extern __shared__ __align__(16) float sm[];
+    extern __shared__ __align__(128) float sm[];
     float *sKh = sm + L::kh, *sQh = sm + L::qh, *sKt = sm + L::kt, *sPt = sm + L::pt;
     float *sS = sm + L::s, *sX = sm + L::x, *sY = sm + L::y, *sD = sm + L::d;
     const int tid = threadIdx.x;
@@ -574,43 +593,62 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
         const int ci = backward ? nch - 1 - step : step;
         return rec + ((first + ci) * H + h) * (long long)R::FLOATS;
     };
+    // one thread issues each group as bulk copies completing on its barrier
+    __shared__ __align__(8) uint64_t bars[2];
+    const uint32_t bar_a = ptx::smem_u32(&bars[0]), bar_b = ptx::smem_u32(&bars[1]);
+    uint32_t ph_a = 0, ph_b = 0;
+    bool pend_a = false, pend_b = false;
+    if (tid == 0) {
+        ptx::mbar_init(bar_a, 1);
+        ptx::mbar_init(bar_b, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
     auto issue_a = [&](int step) {
-        if (step < nch) {
-            const float *rp = rec_of(step);
-            if (backward) {
-                async_rows(sPt, CP, rp + R::PT, C, C);
-                async_rows(sKt, CP, rp + R::KT, DK, C);
-            } else {
-                async_rows(sKh, DKP, rp + R::KH, C, DK);
-            }
+        if (step >= nch) return;
+        pend_a = true;
+        if (tid != 0) return;
+        const float *rp = rec_of(step);
+        if (backward) {
+            ptx::mbar_arrive_expect_tx(bar_a, R::ROWS_C + R::KT_BYTES);
+            ptx::bulk_load(ptx::smem_u32(sPt), rp + R::PT, R::ROWS_C, bar_a);
+            ptx::bulk_load(ptx::smem_u32(sKt), rp + R::KT, R::KT_BYTES, bar_a);
+        } else {
+            ptx::mbar_arrive_expect_tx(bar_a, R::ROWS_K);
+            ptx::bulk_load(ptx::smem_u32(sKh), rp + R::KH, R::ROWS_K, bar_a);
         }
-        cp_async_commit();
     };
     auto issue_b = [&](int step) {
-        if (step < nch) {
-            const float *rp = rec_of(step);
-            if (backward) {
-                async_rows(sQh, DKP, rp + R::QH, C, DK);
-                async_rows(sKh, DKP, rp + R::KH, C, DK);
-            } else {
-                async_rows(sKt, CP, rp + R::KT, DK, C);
-            }
-            async_rows(sD, DK, rp + R::D, 1, DK);
+        if (step >= nch) return;
+        pend_b = true;
+        if (tid != 0) return;
+        const float *rp = rec_of(step);
+        if (backward) {
+            ptx::mbar_arrive_expect_tx(bar_b, 2 * R::ROWS_K + DK * 4);
+            ptx::bulk_load(ptx::smem_u32(sQh), rp + R::QH, R::ROWS_K, bar_b);
+            ptx::bulk_load(ptx::smem_u32(sKh), rp + R::KH, R::ROWS_K, bar_b);
+        } else {
+            ptx::mbar_arrive_expect_tx(bar_b, R::KT_BYTES + DK * 4);
+            ptx::bulk_load(ptx::smem_u32(sKt), rp + R::KT, R::KT_BYTES, bar_b);
         }
-        cp_async_commit();
+        ptx::bulk_load(ptx::smem_u32(sD), rp + R::D, DK * 4, bar_b);
     };
-    // V (forward) or dO (backward) rows of a chunk, this thread's share, in registers
-    constexpr int XPT = C * SV / NT;
-    float xr[XPT];
+    bool ok = true;
+    // V (forward) or dO (backward) rows of a chunk, this thread's share, as raw
+    // 16-byte vectors in registers (converted only when stored to shared memory)
+    constexpr int XV = 16 / (int)sizeof(Tin);       // elements per vector
+    constexpr int XPT = C * SV / XV / NT;           // vectors per thread
+    uint4 xr[XPT];
     const Tin *xin = backward ? d_o : v;
-    auto load_x = [&](int step, float (&out)[XPT]) {
+    auto load_x = [&](int step) {
         const int ci = backward ? nch - 1 - step : step;
         const long long cs = t0 + (long long)ci * C;
         const int Lc = (int)min((long long)C, t1 - cs);
 #pragma unroll
         for (int u = 0; u < XPT; ++u) {
-            const int idx = tid + u * NT, i = idx / SV, j = idx % SV;
-            out[u] = i < Lc ? Elem<Tin>::load(xin + ((cs + i) * H + h) * DV + col_base + j) : 0.f;
+            const int e = (tid + u * NT) * XV, i = e / SV, j = e % SV;
+            xr[u] = i < Lc ? *reinterpret_cast<const uint4 *>(xin + ((cs + i) * H + h) * DV + col_base + j)
+                           : make_uint4(0u, 0u, 0u, 0u);
         }
     };
     issue_a(0);
@@ -623,18 +661,29 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
         __syncthreads();   // S (or dS) final for this chunk; X free
         // checkpoint: the state at the chunk's start (forward) or the adjoint at its end
         float *cp = (backward ? dckpt : ckpt) + (slot * H + h) * (long long)DK * DV + col_base;
-        for (int idx = tid; idx < DK * SV; idx += NT) {
-            const int c = idx / SV, j = idx % SV;
-            cp[(long long)c * DV + j] = sS[c * SVP + j];
+        for (int idx = tid; idx < DK * SV / 4; idx += NT) {
+            const int c = idx / (SV / 4), j = (idx % (SV / 4)) * 4;
+            *reinterpret_cast<float4 *>(cp + (long long)c * DV + j) = *reinterpret_cast<const float4 *>(sS + c * SVP + j);
         }
-        if (step == 0) load_x(step, xr);
+        if (step == 0) load_x(step);
 #pragma unroll
         for (int u = 0; u < XPT; ++u) {
-            const int idx = tid + u * NT, i = idx / SV, j = idx % SV;
-            sX[i * SVP + j] = xr[u];
+            const int e = (tid + u * NT) * XV, i = e / SV, j = e % SV;
+            float *dst = sX + i * SVP + j;
+            if constexpr (sizeof(Tin) == 2) {
+                const uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[q2]));
+                    dst[2 * q2] = f.x;
+                    dst[2 * q2 + 1] = f.y;
+                }
+            } else {
+                *reinterpret_cast<uint4 *>(dst) = xr[u];
+            }
         }
-        cp_async_wait_prev();   // group A of this chunk
-        __syncthreads();
+        pend_a = false;
+        if (!(ok = wait_copies(bar_a, ph_a))) break;   // group A of this chunk
         if (!backward)
             block_mma<C, SV, SPLIT, DK>(sKh, DKP, 1, sS, SVP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                     [&](int i, int j, float x) { sY[i * SVP + j] = sX[i * SVP + j] - x; });
@@ -643,9 +692,9 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
                                     [&](int i, int j, float x) { sY[i * SVP + j] = -x; });
         __syncthreads();   // group A's buffers are free
         issue_a(step + 1);
-        if (step + 1 < nch) load_x(step + 1, xr);   // next chunk's V or dO, in flight during product B
-        cp_async_wait_prev();   // group B of this chunk
-        __syncthreads();
+        if (step + 1 < nch) load_x(step + 1);   // next chunk's V or dO, in flight during product B
+        pend_b = false;
+        if (!(ok = wait_copies(bar_b, ph_b))) break;   // group B of this chunk
         if (!backward)
             block_mma<DK, SV, SPLIT, C>(sKt, CP, 1, sY, SVP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                      [&](int c, int j, float x) { sS[c * SVP + j] = sD[c] * sS[c * SVP + j] + x; });
@@ -655,7 +704,11 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
         __syncthreads();   // group B's buffers are free
         issue_b(step + 1);
     }
-    cp_async_wait_all();
+    if (!ok) {   // a copy did not arrive: wait (bounded) for any still in flight, then leave
+        if (pend_a) ptx::mbar_wait_bounded(bar_a, ph_a, kWaitLimit);
+        if (pend_b) ptx::mbar_wait_bounded(bar_b, ph_b, kWaitLimit);
+        return;
+    }
     __syncthreads();
     if (backward && dinit_state) {
         for (int idx = tid; idx < DK * SV; idx += NT) {
@@ -703,7 +756,7 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
     constexpr int NW = NT / 32;
     constexpr int TQ = (C / 16) * (DK / 8) / NW;   // [C][DK] output tiles per warp
     constexpr int TA = (C / 16) * (C / 8) / NW;    // [C][C] output tiles per warp
-    extern __shared__ float sm[];
+    extern __shared__ __align__(128) float sm[];
     float *sKh = sm + L::kh, *sKb = sm + L::kb, *sAkk = sm + L::akk, *sAqk = sm + L::aqk, *sT = sm + L::ti;
     float *sTb = sm + L::tb, *sS = sm + L::S, *sdS = sm + L::dS, *sW = sm + L::w, *sU = sm + L::u;
     float *sDO = sm + L::dout, *sdU = sm + L::du, *sL = sm + L::lam, *sB = sm + L::b, *sDB = sm + L::db;
@@ -712,13 +765,20 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
     int Lc;
     if (!chunk_of_slot(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
     const float *rp = rec + ((long long)slot * H + h) * R::FLOATS;
-    async_rows(sKh, DKP, rp + R::KH, C, DK);
-    async_rows(sKb, DKP, rp + R::KB, C, DK);
-    async_rows(sAkk, CP, rp + R::AKK, C, C);
-    async_rows(sAqk, CP, rp + R::AQK, C, C);
-    async_rows(sT, CP, rp + R::TI, C, C);
-    async_rows(sTb, CP, rp + R::TB, C, C);
-    cp_async_commit();
+    __shared__ __align__(8) uint64_t bar_rec;
+    const uint32_t bar = ptx::smem_u32(&bar_rec);
+    uint32_t ph = 0;
+    if (tid == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+        ptx::mbar_arrive_expect_tx(bar, 2 * R::ROWS_K + 4 * R::ROWS_C);
+        ptx::bulk_load(ptx::smem_u32(sKh), rp + R::KH, R::ROWS_K, bar);
+        ptx::bulk_load(ptx::smem_u32(sKb), rp + R::KB, R::ROWS_K, bar);
+        ptx::bulk_load(ptx::smem_u32(sAkk), rp + R::AKK, R::ROWS_C, bar);
+        ptx::bulk_load(ptx::smem_u32(sAqk), rp + R::AQK, R::ROWS_C, bar);
+        ptx::bulk_load(ptx::smem_u32(sT), rp + R::TI, R::ROWS_C, bar);
+        ptx::bulk_load(ptx::smem_u32(sTb), rp + R::TB, R::ROWS_C, bar);
+    }
     for (int i = tid; i < C; i += NT) {
         sB[i] = i < Lc ? beta[(cs + i) * H + h] : 0.f;
         sDB[i] = 0.f;
@@ -761,6 +821,10 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
             }
         }
         cp_async_wait_all();
+        if (tile == 0 && !wait_copies(bar, ph)) {   // the record did not arrive: wait (bounded) once more, leave
+            ptx::mbar_wait_bounded(bar, ph ^ 1u, kWaitLimit);
+            return;
+        }
         __syncthreads();
         // W = V - Kh S (in place: each element is read and written by its owner only)
         block_mma<C, DVT, SPLIT, DK>(sKh, DKP, 1, sS, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
@@ -991,7 +1055,7 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
     using P = Part<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
-    extern __shared__ float sm[];
+    extern __shared__ __align__(128) float sm[];
     float *sQ = sm + L::q, *sK = sm + L::k, *sG = sm + L::g, *sAcc = sm + L::acc, *sDg = sm + L::dg;
     float *sAq = sm + L::aq, *sAk = sm + L::ak, *scr = sm + L::scr;
     const int tid = threadIdx.x, slot = blockIdx.x, h = blockIdx.y;

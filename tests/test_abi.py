@@ -165,10 +165,11 @@ def test_slot_entry_points_reject(lib):
 
 
 # backward workspace per (chunk slot, head), fp32: the chunk record (3 [64][dk]
-# + 5 [64][64] + [dk][64] + dk), the state at the chunk's start and the adjoint at
-# its end ([dk][dv] each), and the column sums (3 [64][dk] + 2 [64][64] + 64 + dk)
+# + 5 [64][64] + [dk][64] + dk, rows padded by 4 floats), the state at the chunk's
+# start and the adjoint at its end ([dk][dv] each), and the column sums
+# (3 [64][dk] + 2 [64][64] + 64 + dk)
 def bwd_ws(slots, H, dk, dv):
-    rec = 3 * 64 * dk + 5 * 64 * 64 + dk * 64 + dk
+    rec = 3 * 64 * (dk + 4) + 5 * 64 * 68 + dk * 68 + dk
     part = 3 * 64 * dk + 2 * 64 * 64 + 64 + dk
     return slots * H * (rec + 2 * dk * dv + part) * 4
 
