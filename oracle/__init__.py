@@ -27,7 +27,7 @@ import numpy as np
 
 from .build import build_oracle, library_path
 
-__all__ = ["forward", "backward", "unrolled", "step", "max_threads", "library_path", "build_oracle"]
+__all__ = ["forward", "backward", "prologue", "unrolled", "step", "max_threads", "library_path", "build_oracle"]
 
 _lib = None
 
@@ -142,6 +142,29 @@ def backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal=None, cu_seq
     if rc != 0:
         raise ValueError(f"oracle.backward failed with code {rc}")
     return out
+
+
+def prologue(q_raw, k_raw, gate_x, eps=1e-6):
+    """Input prologue of the operator, fp64 (numpy), for the fused-prologue entry
+    points: q and k scaled to unit L2 norm over the key axis, and the per-channel
+    log-decay from the gate pre-activation x,
+
+        q = q_raw / max(|q_raw|_2, eps),   k likewise,   log_alpha = -softplus(x)
+
+    ("Kimi Linear、独自の土俵でFull Attentionを上回る" (remio.ai), § "Kimi Linearが
+    より賢いRecurrent Memoryを使う方法": the decay gate is computed per channel from
+    the current token; the pages leave its parametrisation open, so this module
+    takes the plainest form with alpha in (0, 1): alpha = exp(-softplus(x)) =
+    1 / (1 + e^x)).  softplus is evaluated as max(x, 0) + log1p(exp(-|x|)).
+    Shapes: q_raw, k_raw, gate_x [..., dk]; returns (q, k, log_alpha) float64.
+    """
+    q = _f64(q_raw)
+    k = _f64(k_raw)
+    x = _f64(gate_x)
+    qn = np.maximum(np.sqrt((q * q).sum(axis=-1, keepdims=True)), eps)
+    kn = np.maximum(np.sqrt((k * k).sum(axis=-1, keepdims=True)), eps)
+    log_alpha = -(np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x))))
+    return q / qn, k / kn, log_alpha
 
 
 def unrolled(q, k, v, log_alpha, beta, init_state=None):
