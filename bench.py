@@ -6,7 +6,8 @@ One step = one chunked prefill (kda_chunk_forward, tcgen05 kernel) of the
 fp32 initial state, 64-token chunks.  The decode workload (N=256 sequences,
 H=32, one token per step through kda_recurrent_step, fresh inputs per step) is
 timed in the same run and reported under "decode"; the backward of the
-prefill_8k workload (kda_chunk_backward) under "backward_8k".
+prefill_8k workload (kda_chunk_backward) under "backward_8k"; the same prefill on raw
+inputs through the fused prologue under "prefill_prologue_8k".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -46,6 +47,8 @@ DECODE_BYTES_PER_PAIR = 2 * STATE_BYTES + PREFILL_BYTES_PER_TOKEN_HEAD        # 
 # product is two products of the same size (recomputation is not credited).
 BACKWARD_BYTES_PER_TOKEN_HEAD = 4 * 2 * 128 + 4 * 128 + 4 + 3 * 2 * 128 + 4 * 128 + 4   # 2824
 BACKWARD_FLOPS_PER_TOKEN_HEAD = 2 * PREFILL_FLOPS_PER_TOKEN_HEAD                      # 360448
+# Fused prologue, per token-head: raw q, k, v and the gate pre-activation (bf16), beta, o.
+PROLOGUE_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 2 * 128 + 4 + 2 * 128                    # 1284
 # DRAM bytes (read + write) per launch from ncu captures of the current kernels on
 # these workloads (profiles/*.md); keyed by the kernels one step runs.  A kernel set
 # without a capture on its workload reports null.
@@ -263,6 +266,42 @@ def run_prefill_gdn(args, world, rank, dev):
     ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
     del d
     return dict(ms=ms, launches=reps * (2 if ws_n else 1))
+
+
+def run_prefill_prologue(args, world, rank, dev):
+    """prefill_8k on raw inputs through the fused prologue (kda_chunk_forward_prologue), CUDA events per call."""
+    import torch
+
+    import gated_delta_rule_85_b200 as kda
+    from gated_delta_rule_85_b200.workloads import PrefillShape, prefill_inputs
+
+    shape = PrefillShape(**PREFILL, dtype=torch.bfloat16, inputs="raw")
+    d = prefill_inputs(shape, seed=rank, device=dev)
+    o = torch.empty((1, PREFILL["T"], PREFILL["H"], PREFILL["dv"]), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, PREFILL["H"], 128, 128), dtype=torch.float32, device=dev)
+    ws = torch.empty(kda.workspace_size(1, PREFILL["T"], PREFILL["H"], 128, 128, 1, algo="two_pass"),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.chunk_forward_prologue(d["q"], d["k"], d["v"], d["gate_x"], d["beta"], d["init_state"], o=o,
+                                   final_state=fs, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    reps = max(5, min(args.steps, 50))
+    _barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    del d
+    return dict(ms=ms, launches=reps * 2)
 
 
 def run_backward(args, world, rank, dev):
@@ -501,6 +540,7 @@ def main(argv=None):
     ap.add_argument("--no-slots", action="store_true", help="skip the state-pool decode line")
     ap.add_argument("--no-gdn", action="store_true", help="skip the Gated DeltaNet (scalar gate) prefill line")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward (gradients) line")
+    ap.add_argument("--no-prologue", action="store_true", help="skip the fused-prologue (raw inputs) prefill line")
     ap.add_argument("--only-backward", action="store_true",
                     help="time only the backward and print its line (profiling a smaller --backward-T)")
     ap.add_argument("--backward-T", type=int, default=PREFILL["T"], help="tokens of the backward workload")
@@ -542,6 +582,7 @@ def main(argv=None):
     vl = None if args.no_varlen else run_prefill_varlen(args, world, rank, dev)
     gd = None if args.no_gdn else run_prefill_gdn(args, world, rank, dev)
     bw = None if args.no_backward else run_backward(args, world, rank, dev)
+    pr = None if args.no_prologue else run_prefill_prologue(args, world, rank, dev)
 
     hbm_gbs, bf16_tflops, peak_src = _peaks()
     ms_step = pre["total_ms"] / args.steps
@@ -599,6 +640,20 @@ def main(argv=None):
                          "tensor": {"achieved_tflops": gtf, "peak_tflops": bf16_tflops, "frac": gtf / bf16_tflops}},
         }
         line["gpu_launches"] += gd["launches"]
+    if pr is not None:
+        pbytes = token_heads * PROLOGUE_BYTES_PER_TOKEN_HEAD + 2 * PREFILL["H"] * STATE_BYTES
+        pgbs = pbytes / (pr["ms"] * 1e-3) / 1e9
+        ptf = alg_flops / (pr["ms"] * 1e-3) / 1e12
+        line["prefill_prologue_8k"] = {
+            "metric": "KDA chunked prefill tokens/s on raw inputs, q/k normalisation and gate in the kernel "
+                      "(B=1, T=8192, H=32, d=128)",
+            "value": world * tokens / (pr["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": pr["ms"],
+            "roofline": {"kernel": "chunk_intra_kernel (prologue) + chunk_inter_kernel", "bound": "hbm",
+                         "achieved": pgbs, "peak": hbm_gbs, "unit": "GB/s", "frac": pgbs / hbm_gbs, "traffic": None,
+                         "algorithmic_bytes": pbytes,
+                         "tensor": {"achieved_tflops": ptf, "peak_tflops": bf16_tflops, "frac": ptf / bf16_tflops}},
+        }
+        line["gpu_launches"] += pr["launches"]
     if bw is not None:
         line["backward_8k"] = backward_block(args, world, bw, hbm_gbs, bf16_tflops)
         line["gpu_launches"] += bw["launches"]

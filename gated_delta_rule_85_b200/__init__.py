@@ -17,11 +17,13 @@ from __future__ import annotations
 
 import ctypes
 import os
+from types import SimpleNamespace
 
 import torch
 
 __all__ = [
-    "chunk_forward", "chunk_backward", "backward_workspace_size", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
+    "chunk_forward", "chunk_backward", "backward_workspace_size", "chunk_forward_prologue",
+    "recurrent_step_prologue", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
     "recurrent_step_slots", "gdn_chunk_forward", "gdn_recurrent_step", "workspace_size", "device_status",
     "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
     "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "DEV_BAD_SLOT", "ALGOS",
@@ -85,6 +87,10 @@ def load_library():
     lib.kda_gdn_recurrent_step.restype = ci
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ci] * 5 + [vp]
     lib.kda_recurrent_step.restype = ci
+    lib.kda_chunk_forward_prologue.argtypes = [vp, vp, vp, vp, fp, fp, vp, fp, ip] + [ci] * 9 + [vp, sz, vp]
+    lib.kda_chunk_forward_prologue.restype = ci
+    lib.kda_recurrent_step_prologue.argtypes = [vp, vp, vp, vp, fp, fp, vp] + [ci] * 5 + [vp]
+    lib.kda_recurrent_step_prologue.restype = ci
     lib.kda_chunk_backward.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, ip] + \
         [ci] * 8 + [vp, sz, vp]
     lib.kda_chunk_backward.restype = ci
@@ -218,6 +224,54 @@ def chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *,
                                       _p(workspace), ws_bytes, st)
     _check(rc)
     return o, final_state
+
+
+def chunk_forward_prologue(q_raw, k_raw, v, gate_x, beta, init_state=None, cu_seqlens=None, *, o=None,
+                           final_state=True, workspace=None, algo="auto"):
+    """Chunked prefill on raw inputs (kda_chunk_forward_prologue): q and k are
+    scaled to unit norm over dk and log_alpha = -softplus(gate_x) inside the
+    kernels.  gate_x has q's shape and dtype.  Returns (o, final_state or None)."""
+    # the shared shape checks, with a metadata-only stand-in for an fp32 log_alpha
+    B, T, H, dk, dv, N = _prefill_args(q_raw, k_raw, v, SimpleNamespace(shape=gate_x.shape, dtype=torch.float32),
+                                       beta, init_state, cu_seqlens)
+    if gate_x.shape != q_raw.shape or gate_x.dtype != q_raw.dtype:
+        raise ValueError("gate_x must have q's shape and dtype")
+    _need_cuda(q_raw, k_raw, v, gate_x, beta, init_state, cu_seqlens)
+    lib = load_library()
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q_raw.dtype, device=q_raw.device)
+    if final_state is True:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q_raw.device)
+    elif final_state is False:
+        final_state = None
+    dt = _dtype_code(q_raw)
+    need = 0 if dt == KDA_F32 else int(lib.kda_chunk_forward_workspace_size_ex(B, T, H, dk, dv, N, dt, CHUNK,
+                                                                                ALGOS["two_pass"]))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_raw.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.kda_chunk_forward_prologue(_p(q_raw), _p(k_raw), _p(v), _p(gate_x), _p(beta), _p(init_state), _p(o),
+                                        _p(final_state), _p(cu_seqlens), B, T, H, dk, dv, N, dt, CHUNK,
+                                        _algo_code(algo), _p(workspace), ws_bytes, _stream(q_raw.device))
+    _check(rc)
+    return o, final_state
+
+
+def recurrent_step_prologue(q_raw, k_raw, v, gate_x, beta, state, o=None):
+    """One decode step on raw inputs (kda_recurrent_step_prologue); state updated in place."""
+    N, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    if k_raw.shape != q_raw.shape or gate_x.shape != q_raw.shape or gate_x.dtype != q_raw.dtype:
+        raise ValueError("q_raw, k_raw and gate_x must share shape and dtype")
+    if state.shape != (N, H, dk, dv) or state.dtype != torch.float32:
+        raise ValueError("state must be float32 [N, H, dk, dv]")
+    _need_cuda(q_raw, k_raw, v, gate_x, beta, state)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q_raw.dtype, device=q_raw.device)
+    rc = load_library().kda_recurrent_step_prologue(_p(q_raw), _p(k_raw), _p(v), _p(gate_x), _p(beta), _p(state),
+                                                    _p(o), N, H, dk, dv, _dtype_code(q_raw), _stream(q_raw.device))
+    _check(rc)
+    return o
 
 
 def backward_workspace_size(B, T, H, dk, dv, num_seqs) -> int:

@@ -80,6 +80,13 @@ constexpr uint32_t ICOL_GRAM = 0;     // [128 x 64] rows 0-63 Kp Kbar^T, rows 64
 constexpr uint32_t ICOL_KT = 64;      // [128 x 64] Kt (lanes 0..dk-1)
 constexpr uint32_t ICOL_PT = 128;     // [128 x 64] Pt (lanes 64-127)
 
+__device__ __forceinline__ float4 scale4(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
+
+__device__ __forceinline__ uint2 float4_to_bf16x4(float4 a) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+    return make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+}
+
 __device__ __forceinline__ float4 bf16x4_to_float4(uint2 r) {
     const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
     const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
@@ -92,7 +99,10 @@ __device__ __forceinline__ void st_global_bf16x8(uint8_t *p, const float *x) {
 }
 
 // GS: scalar gate, log_alpha [tokens, H] (Gated DeltaNet), else [tokens, H, DK].
-template <int DK, bool GS>
+// GS: scalar gate (Gated DeltaNet).  PRO: fused input prologue -- q and k are
+// raw (scaled here to unit norm over the key axis) and log_alpha points to the
+// bf16 gate pre-activation x [tokens, H, DK], log_alpha = -softplus(x).
+template <int DK, bool GS, bool PRO>
 __global__ void __launch_bounds__(NT, 2)
 chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -157,6 +167,10 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 if constexpr (GS) {
                     const float gs = __ldg(log_alpha + (cs + i0 + u) * H + h);
                     g4 = make_float4(gs, gs, gs, gs);
+                } else if constexpr (PRO) {
+                    const float4 x4 = bf16x4_to_float4(
+                        __ldcs(reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(log_alpha) + off)));
+                    g4 = make_float4(neg_softplus(x4.x), neg_softplus(x4.y), neg_softplus(x4.z), neg_softplus(x4.w));
                 } else {
                     g4 = __ldcs(reinterpret_cast<const float4 *>(log_alpha + off));
                 }
@@ -165,6 +179,24 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
             sg.x += g4.x; sg.y += g4.y; sg.z += g4.z; sg.w += g4.w;
             al[u][0] = g4.x; al[u][1] = g4.y; al[u][2] = g4.z; al[u][3] = g4.w;
+        }
+        // prologue: q and k rows to unit norm (a row's DK channels live in NCG
+        // consecutive lanes of one warp), rounded back to bf16 -- the same values
+        // as normalising in fp32 and then casting, as prepared inputs are made
+        if constexpr (PRO) {
+#pragma unroll
+            for (int u = 0; u < SEGLEN; ++u) {
+                const float4 a = bf16x4_to_float4(qv[u]), b = bf16x4_to_float4(kv[u]);
+                float sq = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+                float sk = b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
+#pragma unroll
+                for (int o = NCG / 2; o > 0; o >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                }
+                qv[u] = float4_to_bf16x4(scale4(a, inv_row_norm(sq)));
+                kv[u] = float4_to_bf16x4(scale4(b, inv_row_norm(sk)));
+            }
         }
         *reinterpret_cast<float4 *>(fSeg + seg * DK + c0) = sg;
         __syncthreads();
@@ -551,7 +583,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
 
 // ------------------------------------------------------------------ host side
 
-template <int DK, int DVT, bool GS>
+template <int DK, int DVT, bool GS, bool PRO>
 int launch_two_pass_t(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                       const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
                       long long tokens, int T, int H, int dv, int num_seqs, const int32_t *slots, int num_slots,
@@ -567,7 +599,7 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         return KDA_ERR_UNSUPPORTED;
     }
     constexpr int smem1 = IntraLayout<DK>::ALLOC;
-    auto k1 = chunk_intra_kernel<DK, GS>;
+    auto k1 = chunk_intra_kernel<DK, GS, PRO>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_intra): %s", cudaGetErrorString(e));
@@ -604,20 +636,19 @@ inline int launch_two_pass(const void *q, const void *k, const void *v, const fl
                            const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
                            long long tokens, int T, int H, int dk, int dv, int num_seqs, const int32_t *slots,
                            int num_slots, bool gate_scalar, void *workspace, cudaStream_t st, char *msg,
-                           size_t msg_len) {
+                           size_t msg_len, bool prologue = false) {
     // value-tile width of the recurrence pass: the widest that still gives one CTA per SM
     const long long chains = (long long)num_seqs * H;
     int dvt = 32;
     for (int cand = dv; cand >= 32; cand /= 2)
         if (chains * (dv / cand) >= 148) { dvt = cand; break; }
-#define KDA_2P(DKv, DVTv)                                                                                         \
-    return gate_scalar                                                                                             \
-               ? launch_two_pass_t<DKv, DVTv, true>(q, k, v, log_alpha, beta, init_state, o, final_state,         \
-                                                    cu_seqlens, tokens, T, H, dv, num_seqs, slots, num_slots,     \
-                                                    workspace, st, msg, msg_len)                                   \
-               : launch_two_pass_t<DKv, DVTv, false>(q, k, v, log_alpha, beta, init_state, o, final_state,        \
-                                                     cu_seqlens, tokens, T, H, dv, num_seqs, slots, num_slots,    \
-                                                     workspace, st, msg, msg_len)
+#define KDA_2P_ARGS                                                                                                \
+    (q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T, H, dv, num_seqs, slots, num_slots, \
+     workspace, st, msg, msg_len)
+#define KDA_2P(DKv, DVTv)                                                              \
+    return gate_scalar ? launch_two_pass_t<DKv, DVTv, true, false> KDA_2P_ARGS          \
+           : prologue  ? launch_two_pass_t<DKv, DVTv, false, true> KDA_2P_ARGS          \
+                       : launch_two_pass_t<DKv, DVTv, false, false> KDA_2P_ARGS
     if (dk == 128) {
         if (dvt == 128) KDA_2P(128, 128);
         if (dvt == 64) KDA_2P(128, 64);
@@ -627,6 +658,7 @@ inline int launch_two_pass(const void *q, const void *k, const void *v, const fl
     if (dvt == 64) KDA_2P(64, 64);
     KDA_2P(64, 32);
 #undef KDA_2P
+#undef KDA_2P_ARGS
 }
 
 }  // namespace tc

@@ -47,7 +47,10 @@ struct Smem {
 }  // namespace simt
 
 // GS: scalar gate, log_alpha [tokens, H] (Gated DeltaNet), else [tokens, H, DK].
-template <int DK, typename Tin, bool GS>
+// PRO: fused input prologue -- q and k raw (scaled here to unit norm over the key
+// axis), log_alpha points to the gate pre-activation x [tokens, H, DK] in Tin,
+// log_alpha = -softplus(x).
+template <int DK, typename Tin, bool GS, bool PRO>
 __global__ void __launch_bounds__(simt::NT, 1)
 chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -85,7 +88,8 @@ chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
                 const long long off = ((cs + i) * H + h) * DK + c;
                 qv = Elem<Tin>::load(q + off);
                 kv = Elem<Tin>::load(k + off);
-                gv = GS ? log_alpha[(cs + i) * H + h] : log_alpha[off];
+                if constexpr (PRO) gv = neg_softplus(Elem<Tin>::load(reinterpret_cast<const Tin *>(log_alpha) + off));
+                else gv = GS ? log_alpha[(cs + i) * H + h] : log_alpha[off];
             }
             sQ[i * DKP + c] = qv;
             sK[i * DKP + c] = kv;
@@ -97,6 +101,25 @@ chunk_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
         }
         for (int i = tid; i < C; i += NT) sB[i] = i < Lc ? beta[(cs + i) * H + h] : 0.f;
         __syncthreads();
+        if constexpr (PRO) {   // q, k rows to unit norm: 4 lanes per row
+            static_assert(NT == 4 * C, "4 threads per chunk row");
+            const int i = tid >> 2, l4 = tid & 3;
+            float sq = 0.f, sk = 0.f;
+            for (int c = l4; c < DK; c += 4) {
+                sq = fmaf(sQ[i * DKP + c], sQ[i * DKP + c], sq);
+                sk = fmaf(sK[i * DKP + c], sK[i * DKP + c], sk);
+            }
+            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+            sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+            sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+            sk += __shfl_xor_sync(0xffffffffu, sk, 2);
+            const float iq = inv_row_norm(sq), ik = inv_row_norm(sk);
+            for (int c = l4; c < DK; c += 4) {
+                sQ[i * DKP + c] *= iq;
+                sK[i * DKP + c] *= ik;
+            }
+            __syncthreads();
+        }
 
         // G: running sum of log-decay over the chunk, one channel per thread.
         for (int c = tid; c < DK; c += NT) {

@@ -65,6 +65,13 @@ __device__ __forceinline__ void st_stream(float *p, float4 v) {
                  : "memory");
 }
 
+// Input prologue: log_alpha = -softplus(x) from the gate pre-activation x,
+// evaluated as -(max(x, 0) + log(1 + exp(-|x|))) so no term overflows; the
+// fast exponential and logarithm keep the absolute error near 1e-7.
+__device__ __forceinline__ float neg_softplus(float x) { return -(fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x)))); }
+// 1 / max(|x|_2, 1e-6): the prologue's scale of a q or k row from its squared norm.
+__device__ __forceinline__ float inv_row_norm(float sumsq) { return 1.f / fmaxf(sqrtf(sumsq), 1e-6f); }
+
 // Token range of sequence n in the flattened [B*T] token axis.  Packed offsets
 // are clamped to [0, T] (B == 1 there) so a malformed cu_seqlens can never
 // address memory outside the caller's tensors.

@@ -18,7 +18,9 @@
 namespace kda {
 
 // GS: scalar gate, one log_alpha per (sequence, head) (Gated DeltaNet), else one per key channel.
-template <int DK, int DV, typename Tin, bool GS>
+// PRO: fused input prologue -- q and k raw (scaled here to unit norm), log_alpha
+// points to the gate pre-activation x [N, H, DK] in Tin, alpha = exp(-softplus(x)).
+template <int DK, int DV, typename Tin, bool GS, bool PRO>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                    const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -56,15 +58,54 @@ decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
 
     const long long kb = pair * DK;
     float qk = 0.f;
-    for (int c = tid; c < DK; c += 256) {
-        const float a = expf(GS ? log_alpha[pair] : log_alpha[kb + c]);
-        const float kc = Elem<Tin>::load(k + kb + c);
-        const float qc = Elem<Tin>::load(q + kb + c);
-        s_a[c] = a;
-        s_k[c] = kc;
-        s_ak[c] = a * kc;
-        s_aq[c] = a * qc;
-        qk = fmaf(qc, kc, qk);
+    if constexpr (!PRO) {
+        for (int c = tid; c < DK; c += 256) {
+            const float a = expf(GS ? log_alpha[pair] : log_alpha[kb + c]);
+            const float kc = Elem<Tin>::load(k + kb + c);
+            const float qc = Elem<Tin>::load(q + kb + c);
+            s_a[c] = a;
+            s_k[c] = kc;
+            s_ak[c] = a * kc;
+            s_aq[c] = a * qc;
+            qk = fmaf(qc, kc, qk);
+        }
+    } else {
+        // raw rows: one channel per thread (DK <= 256); the norms are block sums
+        static_assert(DK <= 256, "one key channel per thread");
+        __shared__ float s_nrm[8][2];
+        const int c = tid;
+        float qc = 0.f, kc = 0.f, a = 0.f;
+        if (c < DK) {
+            qc = Elem<Tin>::load(q + kb + c);
+            kc = Elem<Tin>::load(k + kb + c);
+            a = expf(neg_softplus(Elem<Tin>::load(reinterpret_cast<const Tin *>(log_alpha) + kb + c)));
+        }
+        float sq = qc * qc, sk = kc * kc;
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        }
+        if (lane == 0) {
+            s_nrm[warp][0] = sq;
+            s_nrm[warp][1] = sk;
+        }
+        __syncthreads();
+        float tq = 0.f, tk = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            tq += s_nrm[w][0];
+            tk += s_nrm[w][1];
+        }
+        qc *= inv_row_norm(tq);
+        kc *= inv_row_norm(tk);
+        if (c < DK) {
+            s_a[c] = a;
+            s_k[c] = kc;
+            s_ak[c] = a * kc;
+            s_aq[c] = a * qc;
+        }
+        qk = qc * kc;
     }
 #pragma unroll
     for (int off = 16; off; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);

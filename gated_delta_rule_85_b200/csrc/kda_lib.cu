@@ -108,12 +108,12 @@ void *static_ws_address(cudaError_t *err) {
     return addr[dev];
 }
 
-template <int DK, typename Tin, bool GS>
+template <int DK, typename Tin, bool GS, bool PRO = false>
 int launch_simt(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                 const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int T,
                 int H, int dv, int num_seqs, const int32_t *slots, int num_slots, cudaStream_t st) {
     constexpr size_t smem = kda::simt::Smem<DK>::bytes;
-    auto kern = kda::chunk_simt_kernel<DK, Tin, GS>;
+    auto kern = kda::chunk_simt_kernel<DK, Tin, GS, PRO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chunk_simt)");
     dim3 grid(dv / kda::simt::DVT, H, num_seqs);
@@ -125,11 +125,11 @@ int launch_simt(const void *q, const void *k, const void *v, const float *log_al
     return KDA_OK;
 }
 
-template <int DK, int DV, typename Tin, bool GS>
+template <int DK, int DV, typename Tin, bool GS, bool PRO = false>
 int launch_decode(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                   float *state, void *o, long long pairs, const int32_t *slots, int num_slots, int H,
                   cudaStream_t st) {
-    kda::decode_step_kernel<DK, DV, Tin, GS><<<(unsigned)pairs, 256, 0, st>>>(
+    kda::decode_step_kernel<DK, DV, Tin, GS, PRO><<<(unsigned)pairs, 256, 0, st>>>(
         (const Tin *)q, (const Tin *)k, (const Tin *)v, log_alpha, beta, state, (Tin *)o, slots, num_slots, H);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
@@ -141,11 +141,23 @@ int launch_decode(const void *q, const void *k, const void *v, const float *log_
 int simt_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
               const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens, int T, int H,
               int dk, int dv, int num_seqs, int dtype, const int32_t *slots, int num_slots, bool gate_scalar,
-              cudaStream_t st) {
+              cudaStream_t st, bool prologue = false) {
     if (num_seqs == 0) return KDA_OK;
 #define KDA_SIMT(DKv, TT, GSv)                                                                                  \
     return launch_simt<DKv, TT, GSv>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H, dv, \
                                      num_seqs, slots, num_slots, st)
+#define KDA_SIMT_PRO(DKv, TT)                                                                                         \
+    return launch_simt<DKv, TT, false, true>(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, T, H, \
+                                             dv, num_seqs, slots, num_slots, st)
+    if (prologue) {
+        if (dtype == KDA_BF16) {
+            if (dk == 64) KDA_SIMT_PRO(64, __nv_bfloat16);
+            KDA_SIMT_PRO(128, __nv_bfloat16);
+        }
+        if (dk == 64) KDA_SIMT_PRO(64, float);
+        KDA_SIMT_PRO(128, float);
+    }
+#undef KDA_SIMT_PRO
     if (dtype == KDA_BF16) {
         if (dk == 64) {
             if (gate_scalar) KDA_SIMT(64, __nv_bfloat16, true);
@@ -215,14 +227,14 @@ int check_decode(const void *q, const void *k, const void *v, const float *log_a
 
 int decode_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                 float *state, void *o, int N, int H, int dk, int dv, int dtype, const int32_t *slots,
-                int num_slots, bool gate_scalar, cudaStream_t st) {
+                int num_slots, bool gate_scalar, cudaStream_t st, bool prologue = false) {
     const long long pairs = (long long)N * H;
     if (pairs == 0) return KDA_OK;
-#define KDA_DEC1(DKv, DVv, TT)                                                                                 \
-    return gate_scalar ? launch_decode<DKv, DVv, TT, true>(q, k, v, log_alpha, beta, state, o, pairs, slots,  \
-                                                           num_slots, H, st)                                  \
-                       : launch_decode<DKv, DVv, TT, false>(q, k, v, log_alpha, beta, state, o, pairs, slots, \
-                                                            num_slots, H, st);
+#define KDA_DEC_ARGS (q, k, v, log_alpha, beta, state, o, pairs, slots, num_slots, H, st)
+#define KDA_DEC1(DKv, DVv, TT)                                                      \
+    return gate_scalar ? launch_decode<DKv, DVv, TT, true, false> KDA_DEC_ARGS       \
+           : prologue  ? launch_decode<DKv, DVv, TT, false, true> KDA_DEC_ARGS       \
+                       : launch_decode<DKv, DVv, TT, false, false> KDA_DEC_ARGS;
 #define KDA_DEC(DKv, DVv)                             \
     if (dk == DKv && dv == DVv) {                     \
         if (dtype == KDA_BF16) KDA_DEC1(DKv, DVv, __nv_bfloat16) \
@@ -234,6 +246,7 @@ int decode_impl(const void *q, const void *k, const void *v, const float *log_al
     KDA_DEC(128, 128)
 #undef KDA_DEC
 #undef KDA_DEC1
+#undef KDA_DEC_ARGS
     return fail(KDA_ERR_UNSUPPORTED, "dk=%d dv=%d", dk, dv);
 }
 
@@ -434,6 +447,49 @@ int kda_gdn_recurrent_step(const void *q, const void *k, const void *v, const fl
     if (rc || N == 0) return rc;
     return decode_impl(q, k, v, log_alpha, beta, state, o, N, H, dk, dv, dtype, nullptr, 0, true,
                        (cudaStream_t)stream);
+}
+
+int kda_chunk_forward_prologue(const void *q_raw, const void *k_raw, const void *v, const void *gate_x,
+                               const float *beta, const float *init_state, void *o, float *final_state,
+                               const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                               int dtype, int chunk, int algo, void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_prefill(q_raw, k_raw, v, (const float *)gate_x, beta, init_state, o, final_state, cu_seqlens, B,
+                           T, H, dk, dv, num_seqs, dtype, chunk);
+    if (rc) return rc;
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_FUSED && algo != KDA_ALGO_TWO_PASS)
+        return fail(KDA_ERR_INVALID_ARG, "algo=%d is not a KDA_ALGO_* value", algo);
+    if (dtype == KDA_F32)
+        return simt_impl(q_raw, k_raw, v, (const float *)gate_x, beta, init_state, o, final_state, cu_seqlens, T, H,
+                         dk, dv, num_seqs, dtype, nullptr, 0, false, (cudaStream_t)stream, true);
+    if (algo == KDA_ALGO_FUSED)
+        return fail(KDA_ERR_UNSUPPORTED, "the fused schedule reads prepared inputs; use KDA_ALGO_TWO_PASS or AUTO");
+    const long long tokens = (long long)B * T;
+    const size_t need = kda::tc::two_pass_workspace_bytes(tokens, H, dk, num_seqs);
+    if (need && (!workspace || ws_bytes < need))
+        return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", need, ws_bytes);
+    if (workspace && !aligned(workspace, 256)) return fail(KDA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (num_seqs == 0) return KDA_OK;
+    if (tokens > 0x7fffffffLL)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T=%lld exceeds the 2^31 token limit of the TMA coordinates", tokens);
+    char msg[256] = "";
+    cudaStream_t st = (cudaStream_t)stream;
+    if (tokens == 0)
+        rc = kda::tc::state_passthrough(init_state, final_state, num_seqs, H, dk, dv, st, msg, sizeof(msg));
+    else
+        rc = kda::tc::launch_two_pass(q_raw, k_raw, v, (const float *)gate_x, beta, init_state, o, final_state,
+                                      cu_seqlens, tokens, T, H, dk, dv, num_seqs, nullptr, 0, false, workspace, st,
+                                      msg, sizeof(msg), true);
+    if (rc) return fail(rc, "%s", msg);
+    return KDA_OK;
+}
+
+int kda_recurrent_step_prologue(const void *q_raw, const void *k_raw, const void *v, const void *gate_x,
+                                const float *beta, float *state, void *o, int N, int H, int dk, int dv, int dtype,
+                                void *stream) {
+    int rc = check_decode(q_raw, k_raw, v, (const float *)gate_x, beta, state, o, N, H, dk, dv, dtype);
+    if (rc) return rc;
+    return decode_impl(q_raw, k_raw, v, (const float *)gate_x, beta, state, o, N, H, dk, dv, dtype, nullptr, 0, false,
+                       (cudaStream_t)stream, true);
 }
 
 size_t kda_chunk_backward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs) {

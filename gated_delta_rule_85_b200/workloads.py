@@ -13,6 +13,8 @@ Distributions (per the workload definitions):
   beta      = sigmoid(x), x ~ N(0, 1), fp32, one value per (token, head)
   states    ~ N(0, 0.01^2) fp32 (std 0.01), or zeros
   backward cotangents: d_o ~ N(0, 1) in the input dtype, dfinal_state ~ N(0, 1) fp32
+  raw inputs (fused-prologue entry points): q, k ~ N(0, 1) not normalised, and the
+              gate pre-activation gate_x ~ N(-2, 1), all in the input dtype
 Every tensor is drawn from its own generator seeded with (seed, stream id), so
 one tensor's draw does not depend on another's size.  Large tensors are drawn
 in token slices of fixed size so device memory for temporaries stays bounded.
@@ -25,7 +27,8 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-_STREAM = {"q": 1, "k": 2, "v": 3, "log_alpha": 4, "beta": 5, "init_state": 6, "d_o": 7, "dfinal_state": 8}
+_STREAM = {"q": 1, "k": 2, "v": 3, "log_alpha": 4, "beta": 5, "init_state": 6, "d_o": 7, "dfinal_state": 8,
+           "gate_x": 9}
 _SLICE_TOKENS = 1 << 15
 
 
@@ -40,6 +43,7 @@ class PrefillShape:
     init_state: str = "normal"          # "normal" (std 0.01) or "zeros"
     cu_seqlens: tuple | None = None      # packed layout when set (B must be 1)
     gate: str = "channel"                # "channel": log_alpha [B, T, H, dk]; "scalar": [B, T, H]
+    inputs: str = "prepared"             # "raw": q, k unnormalised and gate_x instead of log_alpha
 
     @property
     def num_seqs(self) -> int:
@@ -55,6 +59,7 @@ class DecodeShape:
     steps: int
     dtype: torch.dtype = torch.bfloat16
     gate: str = "channel"                # "channel": log_alpha [N, H, dk]; "scalar": [N, H]
+    inputs: str = "prepared"             # "raw": q, k unnormalised and gate_x instead of log_alpha
 
 
 def _gen(device, seed: int, stream: int, sub: int = 0) -> torch.Generator:
@@ -108,6 +113,20 @@ def draw_v(shape, device, seed, stream, dtype):
     return out
 
 
+def draw_raw(shape, device, seed, stream, dtype, mean=0.0):
+    """N(mean, 1) drawn in fp32, then cast (raw q, k or gate pre-activation)."""
+    out = torch.empty(shape, dtype=dtype, device=device)
+    flat_out = out.view(-1, shape[-1])
+    rows = flat_out.shape[0]
+    per = _SLICE_TOKENS * 32
+    for i, r0 in enumerate(range(0, rows, per)):
+        r1 = min(rows, r0 + per)
+        x = torch.empty((r1 - r0, shape[-1]), dtype=torch.float32, device=device)
+        x.normal_(mean, 1.0, generator=_gen(device, seed, stream, i))
+        flat_out[r0:r1] = x.to(dtype)
+    return out
+
+
 def draw_log_alpha(shape, device, seed, stream):
     """-softplus(N(-2, 1)) per channel, fp32."""
     out = torch.empty(shape, dtype=torch.float32, device=device)
@@ -141,6 +160,20 @@ def draw_state(shape, device, seed, stream, kind="normal"):
 def prefill_inputs(shape: PrefillShape, seed: int = 0, device="cpu") -> dict:
     """All prefill inputs of one workload, drawn in the order q, k, v, log_alpha, beta, init_state."""
     B, T, H, dk, dv = shape.B, shape.T, shape.H, shape.dk, shape.dv
+    if shape.inputs == "raw":
+        d = {
+            "q": draw_raw((B, T, H, dk), device, seed, _STREAM["q"], shape.dtype),
+            "k": draw_raw((B, T, H, dk), device, seed, _STREAM["k"], shape.dtype),
+            "v": draw_v((B, T, H, dv), device, seed, _STREAM["v"], shape.dtype),
+            "gate_x": draw_raw((B, T, H, dk), device, seed, _STREAM["gate_x"], shape.dtype, mean=-2.0),
+            "beta": draw_beta((B, T, H), device, seed, _STREAM["beta"]),
+        }
+        N = shape.num_seqs
+        d["init_state"] = (None if shape.init_state == "none"
+                           else draw_state((N, H, dk, dv), device, seed, _STREAM["init_state"], shape.init_state))
+        d["cu_seqlens"] = (None if shape.cu_seqlens is None
+                           else torch.tensor(shape.cu_seqlens, dtype=torch.int32, device=device))
+        return d
     d = {
         "q": draw_qk((B, T, H, dk), device, seed, _STREAM["q"], shape.dtype),
         "k": draw_qk((B, T, H, dk), device, seed, _STREAM["k"], shape.dtype),
@@ -172,6 +205,14 @@ def decode_step_inputs(shape: DecodeShape, step: int, seed: int = 0, device="cpu
     """Per-step decode inputs (q, k, v [N, H, d], log_alpha [N, H, dk], beta [N, H])."""
     N, H, dk, dv = shape.N, shape.H, shape.dk, shape.dv
     base = seed * 65_537 + 100 + step
+    if shape.inputs == "raw":
+        return {
+            "q": draw_raw((N, H, dk), device, base, _STREAM["q"], shape.dtype),
+            "k": draw_raw((N, H, dk), device, base, _STREAM["k"], shape.dtype),
+            "v": draw_v((N, H, dv), device, base, _STREAM["v"], shape.dtype),
+            "gate_x": draw_raw((N, H, dk), device, base, _STREAM["gate_x"], shape.dtype, mean=-2.0),
+            "beta": draw_beta((N, H), device, base, _STREAM["beta"]),
+        }
     return {
         "q": draw_qk((N, H, dk), device, base, _STREAM["q"], shape.dtype),
         "k": draw_qk((N, H, dk), device, base, _STREAM["k"], shape.dtype),

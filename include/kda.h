@@ -265,6 +265,36 @@ int kda_gdn_recurrent_step(const void *q, const void *k, const void *v, const fl
                            void *stream);
 
 /*
+ * Fused input prologue: the operator on raw inputs, with the two input steps
+ * that precede it done inside the kernels instead of as separate passes over
+ * memory -- q and k scaled to unit L2 norm over the key axis (row / max(|row|_2,
+ * 1e-6)), and the per-channel decay from the gate pre-activation x,
+ * log_alpha = -softplus(x), i.e. alpha = 1 / (1 + e^x).  "Kimi Linear、独自の土俵で
+ * Full Attentionを上回る" (remio.ai), § "Kimi Linearがより賢いRecurrent Memoryを使う
+ * 方法" computes the decay per channel from the current token; the pages leave
+ * the parametrisation open, and this is its plainest form with alpha in (0, 1).
+ * The gate stream is x in the input dtype (2 dk bytes per token-head for bf16
+ * instead of 4 dk for fp32 log_alpha).
+ *
+ *   q_raw, k_raw  [B, T, H, dk] in dtype, any scale (zero rows stay zero).
+ *   gate_x        [B, T, H, dk] (prefill) or [N, H, dk] (decode) in dtype,
+ *                 16-byte aligned.
+ * Every other argument and the error behaviour are as in kda_chunk_forward_ex /
+ * kda_recurrent_step.  dtype KDA_BF16 runs the two-pass tensor-core schedule
+ * (AUTO means TWO_PASS here; its workspace is
+ * kda_chunk_forward_workspace_size_ex(..., KDA_ALGO_TWO_PASS); KDA_ALGO_FUSED is
+ * KDA_ERR_UNSUPPORTED), KDA_F32 the fp32 CUDA-core path.
+ */
+int kda_chunk_forward_prologue(const void *q_raw, const void *k_raw, const void *v, const void *gate_x,
+                               const float *beta, const float *init_state, void *o, float *final_state,
+                               const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs,
+                               int dtype, int chunk, int algo, void *workspace, size_t ws_bytes, void *stream);
+
+int kda_recurrent_step_prologue(const void *q_raw, const void *k_raw, const void *v, const void *gate_x,
+                                const float *beta, float *state, void *o, int N, int H, int dk, int dv, int dtype,
+                                void *stream);
+
+/*
  * Backward of the chunked prefill: the gradients of
  *     L = sum_t <d_o_t, o_t> + <dfinal_state, final_state>
  * with respect to every input of kda_chunk_forward -- what the chunkwise

@@ -211,3 +211,19 @@ def backward(lib, **over):
 def test_backward_rejects(lib, over, code):
     assert backward(lib, **over) == code
     assert lib.kda_last_error().decode() != ""
+
+
+def test_prologue_entry_points_reject(lib):
+    pro = lambda **o: lib.kda_chunk_forward_prologue(
+        o.get("q", A[0]), A[1], A[2], o.get("x", A[3]), A[4], A[5], A[6], A[7], None, 1, 128, 2, 128, 128, 1,
+        o.get("dtype", 0), 64, o.get("algo", 0), o.get("ws", A[8]), o.get("wsb", 1 << 24), None)
+    assert pro(x=None) == INVALID                  # gate pre-activation missing
+    assert pro(x=A[3] + 8) == MISALIGNED           # gate below 16-byte alignment
+    assert pro(algo=1) == UNSUPPORTED              # the fused schedule takes prepared inputs only
+    assert pro(algo=9) == INVALID
+    assert pro(ws=None, wsb=0) == WORKSPACE        # two-pass workspace missing
+    assert pro(dtype=4) == UNSUPPORTED
+    step = lambda **o: lib.kda_recurrent_step_prologue(A[0], A[1], A[2], o.get("x", A[3]), A[4], A[5], A[6], 4, 2,
+                                                       128, 128, 0, None)
+    assert step(x=None) == INVALID
+    assert step(x=A[3] + 4) == MISALIGNED
