@@ -343,12 +343,28 @@ __device__ __forceinline__ void async_rows(float *dst, int ld, const float *src,
 constexpr int SB = 16;             // sub-block rows
 constexpr int NSB = C / SB;        // sub-blocks per chunk
 constexpr int SCR_ROWS = C - SB;   // largest off-diagonal operand (48 rows)
+constexpr float DIAG_RANGE = 40.f;   // largest in-block log-decay taken through a block boundary
+
+// True when every channel decays by at most DIAG_RANGE (in log) across each
+// 16-row block, so the diagonal blocks can go through the block boundary with a
+// factor of at most e^DIAG_RANGE.  Uniform over the CTA (it synchronises).
+template <int DK>
+__device__ __forceinline__ bool diag_blocks_in_range(const float *sG) {
+    constexpr int DKP = Pad<DK>::K;
+    bool bad = false;
+    for (int c = threadIdx.x; c < DK; c += NT)
+#pragma unroll
+        for (int b = 0; b < NSB; ++b) bad |= sG[(b * SB) * DKP + c] - sG[(b * SB + SB - 1) * DKP + c] > DIAG_RANGE;
+    return !__syncthreads_or(bad);
+}
 
 // Akk (strictly lower) and Aqk (lower with the diagonal), zero elsewhere.
-// scr holds 2 * SB + SCR_ROWS rows of stride DKP.
+// scr holds 2 SB + C rows of stride DKP.  The diagonal blocks take the exact
+// pairwise exponent unless `diag` (every block's decay range within DIAG_RANGE),
+// in which case they join the tensor-core products through the block boundary.
 template <int DK, bool SPLIT>
 __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, const float *sG, float *sAkk,
-                                            float *sAqk, float *scr) {
+                                            float *sAqk, float *scr, bool diag) {
     constexpr int DKP = Pad<DK>::K;
     const int tid = threadIdx.x;
     for (int idx = tid; idx < C * CP; idx += NT) {
@@ -356,8 +372,7 @@ __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, co
         sAqk[idx] = 0.f;
     }
     __syncthreads();
-    // diagonal blocks, exact: 8 lanes per (i, j) pair, each lane DK / 8 channels
-    {
+    if (!diag) {   // diagonal blocks, exact: 8 lanes per (i, j) pair, each lane DK / 8 channels
         constexpr int PAIRS = NSB * SB * (SB + 1) / 2;
         const int l8 = tid & 7;
         for (int p = tid >> 3; p < PAIRS; p += NT / 8) {
@@ -381,10 +396,11 @@ __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, co
             }
         }
     }
-    // blocks below the diagonal: rows of block bi against rows j < r = 16 bi
+    // rows of block bi against the scaled keys of rows j < r (and, with `diag`,
+    // of the block itself, j < r + 16, masked to j < i / j <= i)
     float *sL = scr, *sR = scr + 2 * SB * DKP;   // [k; q] rows of block bi, then k_j e^{G_r - G_j}
-    for (int bi = 1; bi < NSB; ++bi) {
-        const int r = bi * SB;
+    for (int bi = diag ? 0 : 1; bi < NSB; ++bi) {
+        const int r = bi * SB, ncol = diag ? r + SB : r;
         __syncthreads();
         for (int idx = tid; idx < SB * DK; idx += NT) {
             const int ii = idx / DK, c = idx % DK, i = r + ii;
@@ -392,24 +408,26 @@ __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, co
             sL[ii * DKP + c] = sK[i * DKP + c] * e;
             sL[(SB + ii) * DKP + c] = sQ[i * DKP + c] * e;
         }
-        for (int idx = tid; idx < r * DK; idx += NT) {
+        for (int idx = tid; idx < ncol * DK; idx += NT) {
             const int j = idx / DK, c = idx % DK;
             sR[j * DKP + c] = sK[j * DKP + c] * __expf(sG[r * DKP + c] - sG[j * DKP + c]);
         }
         __syncthreads();
-        // [Akk; Aqk] rows of block bi = [k; q]-scaled rows times the scaled earlier keys
-        constexpr int NTN_MAX = SCR_ROWS / 8;
-        const int ntn = r / 8;
+        const int ntn = ncol / 8;
         for (int t = tid >> 5; t < 2 * ntn; t += NT / 32) {
             const int r0 = (t / ntn) * SB, c0 = (t % ntn) * 8;
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             warp_mma<SPLIT, DK>(d, sL + r0 * DKP, DKP, 1, sR + c0 * DKP, 1, DKP);
             warp_tile_out(d, r0, c0, [&](int row, int j, float x) {
-                if (row < SB) sAkk[(r + row) * CP + j] = x;
-                else sAqk[(r + row - SB) * CP + j] = x;
+                if (row < SB) {
+                    const int i = r + row;
+                    if (j < i) sAkk[i * CP + j] = x;
+                } else {
+                    const int i = r + row - SB;
+                    if (j <= i) sAqk[i * CP + j] = x;
+                }
             });
         }
-        (void)NTN_MAX;
     }
     __syncthreads();
 }
@@ -460,8 +478,8 @@ struct PrepSmem {
     static constexpr int aqk = akk + C * CP;     // [C][CP]
     static constexpr int ti = aqk + C * CP;      // [C][CP]  T
     static constexpr int tb = ti + C * CP;       // [C][CP]  Tb
-    static constexpr int scr = tb + C * CP;      // [2 SB + SCR_ROWS][DKP] Gram operands
-    static constexpr int b = scr + (2 * SB + SCR_ROWS) * DKP;   // [C]
+    static constexpr int scr = tb + C * CP;      // [2 SB + C][DKP] Gram operands
+    static constexpr int b = scr + (2 * SB + C) * DKP;   // [C]
     static constexpr int d = b + C;              // [DK]
     static constexpr int total = d + DK;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
@@ -485,7 +503,7 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
     if (!chunk_of_slot(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
 
     load_chunk_qkg<DK, Tin>(q, k, log_alpha, beta, cs, Lc, H, h, sQ, sK, sG, sB);
-    chunk_grams<DK, SPLIT>(sQ, sK, sG, sAkk, sAqk, sm + L::scr);
+    chunk_grams<DK, SPLIT>(sQ, sK, sG, sAkk, sAqk, sm + L::scr, diag_blocks_in_range<DK>(sG));
     chunk_factors<DK>(sQ, sK, sG, sD);
     // T = (I + Diag(beta) Akk)^{-1}: the 16 x 16 diagonal blocks by forward
     // substitution (4 lanes per column, all 64 columns at once), then each block
@@ -754,8 +772,15 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
     constexpr int NW = NT / 32;
+    // Column sums accumulate in registers across the value tiles: each warp owns a
+    // strip of one 16-row block by TQ (TA) adjacent 8-column tiles of the [C][DK]
+    // ([C][C]) sums.
     constexpr int TQ = (C / 16) * (DK / 8) / NW;   // [C][DK] output tiles per warp
     constexpr int TA = (C / 16) * (C / 8) / NW;    // [C][C] output tiles per warp
+    static_assert((DK / 8) % TQ == 0 && (C / 8) % TA == 0, "strips stay inside one row block");
+    const int wq = (int)(threadIdx.x >> 5);
+    const int q_r0 = (wq / ((DK / 8) / TQ)) * 16, q_c0 = (wq % ((DK / 8) / TQ)) * TQ * 8;
+    const int a_r0 = (wq / ((C / 8) / TA)) * 16, a_c0 = (wq % ((C / 8) / TA)) * TA * 8;
     extern __shared__ __align__(128) float sm[];
     float *sKh = sm + L::kh, *sKb = sm + L::kb, *sAkk = sm + L::akk, *sAqk = sm + L::aqk, *sT = sm + L::ti;
     float *sTb = sm + L::tb, *sS = sm + L::S, *sdS = sm + L::dS, *sW = sm + L::w, *sU = sm + L::u;
@@ -862,19 +887,11 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         __syncthreads();
         // sums over this tile's columns, kept in registers across tiles:
         // dO S^T, mu S^T, U dS^T ([C][DK]) and dO U^T, mu U^T ([C][C])
-#pragma unroll
-        for (int r = 0; r < TQ; ++r) {
-            const int t2 = warp + r * NW, r0 = (t2 / (DK / 8)) * 16, c0 = (t2 % (DK / 8)) * 8;
-            warp_mma<SPLIT, DVT>(a_dq[r], sDO + r0 * TP, TP, 1, sS + c0 * TP, 1, TP);
-            warp_mma<SPLIT, DVT>(a_dkh[r], sL + r0 * TP, TP, 1, sS + c0 * TP, 1, TP);
-            warp_mma<SPLIT, DVT>(a_dkb[r], sU + r0 * TP, TP, 1, sdS + c0 * TP, 1, TP);
-        }
-#pragma unroll
-        for (int r = 0; r < TA; ++r) {
-            const int t2 = warp + r * NW, r0 = (t2 / (C / 8)) * 16, c0 = (t2 % (C / 8)) * 8;
-            warp_mma<SPLIT, DVT>(a_aq[r], sDO + r0 * TP, TP, 1, sU + c0 * TP, 1, TP);
-            warp_mma<SPLIT, DVT>(a_ak[r], sL + r0 * TP, TP, 1, sU + c0 * TP, 1, TP);
-        }
+        warp_mma_strip<SPLIT, DVT, TQ>(a_dq, sDO + q_r0 * TP, TP, 1, sS + q_c0 * TP, 1, TP);
+        warp_mma_strip<SPLIT, DVT, TQ>(a_dkh, sL + q_r0 * TP, TP, 1, sS + q_c0 * TP, 1, TP);
+        warp_mma_strip<SPLIT, DVT, TQ>(a_dkb, sU + q_r0 * TP, TP, 1, sdS + q_c0 * TP, 1, TP);
+        warp_mma_strip<SPLIT, DVT, TA>(a_aq, sDO + a_r0 * TP, TP, 1, sU + a_c0 * TP, 1, TP);
+        warp_mma_strip<SPLIT, DVT, TA>(a_ak, sL + a_r0 * TP, TP, 1, sU + a_c0 * TP, 1, TP);
         if (tid < DK)
             for (int j = 0; j < DVT; ++j) a_gc = fmaf(sS[tid * TP + j], sdS[tid * TP + j], a_gc);
     }
@@ -887,14 +904,14 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         };
 #pragma unroll
         for (int r = 0; r < TQ; ++r) {
-            const int t2 = warp + r * NW, r0 = (t2 / (DK / 8)) * 16, c0 = (t2 % (DK / 8)) * 8;
+            const int r0 = q_r0, c0 = q_c0 + 8 * r;
             put(pp + P::DQ, DK, a_dq[r], r0, c0, 1.f);
             put(pp + P::DKH, DK, a_dkh[r], r0, c0, -1.f);
             put(pp + P::DKB, DK, a_dkb[r], r0, c0, 1.f);
         }
 #pragma unroll
         for (int r = 0; r < TA; ++r) {
-            const int t2 = warp + r * NW, r0 = (t2 / (C / 8)) * 16, c0 = (t2 % (C / 8)) * 8;
+            const int r0 = a_r0, c0 = a_c0 + 8 * r;
             // keep j <= i of dAqk and j < i of dAkk; zero the rest
             float aq[4], ak[4];
 #pragma unroll
@@ -977,20 +994,21 @@ __device__ __forceinline__ void diag_pair_terms(const float *sQ, const float *sK
     }
 }
 
-// Row terms of the blocks below the diagonal: for block bi (rows r..r+15),
-// acc_i += e^{G_i - G_r} sum_{j<r} A[i][j] (k_j e^{G_r - G_j}); dG_i += k_i (that)
-// when to_dg.
-template <int DK, bool SPLIT, int BI>
-__device__ __forceinline__ void offdiag_row_block(const float *sK, const float *sG, const float *sA, float *scr,
-                                                  float *sAcc, float *sDg, bool to_dg) {
-    constexpr int DKP = Pad<DK>::K, r = BI * SB;
+// Row terms of block bi (rows r..r+15, r = 16 bi) over columns j in [J0, J1), J1 <= r:
+// acc_i += e^{G_i - G_r} sum_j A[i][j] (k_j e^{G_r - G_j}); dG_i += k_i (that) when
+// to_dg.  Both factors are <= 1.
+template <int DK, bool SPLIT, int BI, int J0, int J1>
+__device__ __forceinline__ void row_terms(const float *sK, const float *sG, const float *sA, float *scr,
+                                          float *sAcc, float *sDg, bool to_dg) {
+    constexpr int DKP = Pad<DK>::K, r = BI * SB, n = J1 - J0;
+    static_assert(n > 0 && n <= SCR_ROWS, "operand fits the scratch");
     __syncthreads();
-    for (int idx = threadIdx.x; idx < r * DK; idx += NT) {
-        const int j = idx / DK, c = idx % DK;
-        scr[j * DKP + c] = sK[j * DKP + c] * __expf(sG[r * DKP + c] - sG[j * DKP + c]);
+    for (int idx = threadIdx.x; idx < n * DK; idx += NT) {
+        const int jj = idx / DK, c = idx % DK, j = J0 + jj;
+        scr[jj * DKP + c] = sK[j * DKP + c] * __expf(sG[r * DKP + c] - sG[j * DKP + c]);
     }
     __syncthreads();
-    block_mma<SB, DK, SPLIT, r>(sA + r * CP, CP, 1, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
+    block_mma<SB, DK, SPLIT, n>(sA + r * CP + J0, CP, 1, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                 [&](int ii, int c, float x) {
                                     const int i = r + ii;
                                     x *= __expf(sG[i * DKP + c] - sG[r * DKP + c]);
@@ -999,34 +1017,35 @@ __device__ __forceinline__ void offdiag_row_block(const float *sK, const float *
                                 });
 }
 
+// Row terms of the blocks below the diagonal.
 template <int DK, bool SPLIT>
-__device__ __forceinline__ void offdiag_rows(const float *sK, const float *sG, const float *sA, float *scr,
-                                             float *sAcc, float *sDg, bool to_dg) {
-    static_assert(NSB == 4, "three blocks below the diagonal");
-    offdiag_row_block<DK, SPLIT, 1>(sK, sG, sA, scr, sAcc, sDg, to_dg);
-    offdiag_row_block<DK, SPLIT, 2>(sK, sG, sA, scr, sAcc, sDg, to_dg);
-    offdiag_row_block<DK, SPLIT, 3>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+__device__ __forceinline__ void pair_rows(const float *sK, const float *sG, const float *sA, float *scr, float *sAcc,
+                                          float *sDg, bool to_dg) {
+    static_assert(NSB == 4 && SCR_ROWS == 48, "four 16-row blocks");
+    row_terms<DK, SPLIT, 1, 0, 16>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+    row_terms<DK, SPLIT, 2, 0, 32>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+    row_terms<DK, SPLIT, 3, 0, 48>(sK, sG, sA, scr, sAcc, sDg, to_dg);
     __syncthreads();
 }
 
-// Column terms of the blocks below the diagonal: for block bj (columns
-// 16 bj..16 bj+15, last row s), acc_j += e^{G_s - G_j} sum_{i>s} A[i][j] (X_i e^{G_i - G_s})
-// and dG_j -= k_j (that), for (A, X) = (dAqk, q) and (dAkk, k).
-template <int DK, bool SPLIT, int BJ>
-__device__ __forceinline__ void offdiag_col_block(const float *sQ, const float *sK, const float *sG,
-                                                  const float *sAq, const float *sAk, float *scr, float *sAcc,
-                                                  float *sDg) {
-    constexpr int DKP = Pad<DK>::K, s = BJ * SB + SB - 1, n = C - 1 - s;   // rows s+1 .. C-1
+// Column terms of block bj (columns 16 bj..16 bj+15, last row s) over rows i in
+// [I0, I1), I0 > s: acc_j += e^{G_s - G_j} sum_i A[i][j] (X_i e^{G_i - G_s}),
+// dG_j -= k_j (that), for (A, X) = (dAqk, q) and (dAkk, k).  Both factors are <= 1.
+template <int DK, bool SPLIT, int BJ, int I0, int I1>
+__device__ __forceinline__ void col_terms(const float *sQ, const float *sK, const float *sG, const float *sAq,
+                                          const float *sAk, float *scr, float *sAcc, float *sDg) {
+    constexpr int DKP = Pad<DK>::K, s = BJ * SB + SB - 1, n = I1 - I0;
+    static_assert(n > 0 && n <= SCR_ROWS, "operand fits the scratch");
     for (int pass = 0; pass < 2; ++pass) {
         const float *X = pass ? sK : sQ;
         const float *A = pass ? sAk : sAq;
         __syncthreads();
         for (int idx = threadIdx.x; idx < n * DK; idx += NT) {
-            const int ii = idx / DK, c = idx % DK, i = s + 1 + ii;
+            const int ii = idx / DK, c = idx % DK, i = I0 + ii;
             scr[ii * DKP + c] = X[i * DKP + c] * __expf(sG[i * DKP + c] - sG[s * DKP + c]);
         }
         __syncthreads();
-        block_mma<SB, DK, SPLIT, n>(A + (s + 1) * CP + BJ * SB, 1, CP, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<SB, DK, SPLIT, n>(A + I0 * CP + BJ * SB, 1, CP, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                     [&](int jj, int c, float x) {
                                         const int j = BJ * SB + jj;
                                         x *= __expf(sG[s * DKP + c] - sG[j * DKP + c]);
@@ -1036,12 +1055,13 @@ __device__ __forceinline__ void offdiag_col_block(const float *sQ, const float *
     }
 }
 
+// Column terms of the blocks below the diagonal.
 template <int DK, bool SPLIT>
-__device__ __forceinline__ void offdiag_cols(const float *sQ, const float *sK, const float *sG, const float *sAq,
-                                             const float *sAk, float *scr, float *sAcc, float *sDg) {
-    offdiag_col_block<DK, SPLIT, 0>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
-    offdiag_col_block<DK, SPLIT, 1>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
-    offdiag_col_block<DK, SPLIT, 2>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+__device__ __forceinline__ void pair_cols(const float *sQ, const float *sK, const float *sG, const float *sAq,
+                                          const float *sAk, float *scr, float *sAcc, float *sDg) {
+    col_terms<DK, SPLIT, 0, 16, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    col_terms<DK, SPLIT, 1, 32, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    col_terms<DK, SPLIT, 2, 48, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
     __syncthreads();
 }
 
@@ -1086,8 +1106,10 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
     }
     cp_async_wait_all();
     __syncthreads();
+    // The diagonal blocks stay exact on CUDA cores here: taking them through the
+    // block boundary costs two more scaled operands per phase, which measured slower.
     diag_pair_terms<DK, false>(sQ, sK, sG, sAq, nullptr, sAcc, nullptr);
-    offdiag_rows<DK, SPLIT>(sK, sG, sAq, scr, sAcc, nullptr, false);
+    pair_rows<DK, SPLIT>(sK, sG, sAq, scr, sAcc, nullptr, false);
     // dq out; dk starts at a + b and dG at q dq + k (a - b); sum_i k_i b_i per
     // channel (a dG_C term) goes to scr, one row per group of rows
     {
@@ -1126,8 +1148,8 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
     __syncthreads();
     // ---- dk = a + b + pair terms of dAkk (rows) and of dAqk, dAkk (columns)
     diag_pair_terms<DK, true>(sQ, sK, sG, sAq, sAk, sAcc, sDg);
-    offdiag_rows<DK, SPLIT>(sK, sG, sAk, scr, sAcc, sDg, true);
-    offdiag_cols<DK, SPLIT>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    pair_rows<DK, SPLIT>(sK, sG, sAk, scr, sAcc, sDg, true);
+    pair_cols<DK, SPLIT>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
     for (int idx = tid; idx < C * DK; idx += NT) {
         const int i = idx / DK, c = idx % DK;
         if (i < Lc) Elem<Tin>::store(dk_out + ((cs + i) * H + h) * DK + c, sAcc[i * DKP + c]);

@@ -97,6 +97,21 @@ def test_backward_packed_sequences(dtype):
             assert torch.equal(whole, g1[name]), (n, name)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, BF16])
+def test_backward_strong_decay_blocks(dtype):
+    """Sequence 0 decays by ~3.5 per token (more than the in-block range the
+    diagonal blocks may take through a block boundary), sequence 1 as usual: both
+    the exact diagonal path and the tensor-core one run, and both match."""
+    shape = PrefillShape(B=2, T=160, H=2, dk=128, dv=128, dtype=dtype)
+    d = prefill_inputs(shape, 77, DEV)
+    gen = torch.Generator(device=DEV).manual_seed(79)
+    d["log_alpha"][0] = -3.5 + 0.2 * torch.rand(d["log_alpha"][0].shape, generator=gen, device=DEV)
+    c = backward_cotangents(shape, 78, DEV)
+    got = run(d, c)
+    torch.cuda.synchronize()
+    check(got, oracle_grads(d, c), dtype, what="strong decay")
+
+
 def test_backward_without_states():
     """init_state NULL (zeros) and dfinal_state NULL (zero cotangent): dinit_state is
     the gradient at the zero state."""
