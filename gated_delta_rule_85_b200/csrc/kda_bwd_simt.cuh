@@ -61,6 +61,8 @@ namespace bwd {
 constexpr int C = 64;      // chunk length
 constexpr int DVT = 32;    // value columns per tile
 constexpr int NT = 256;    // threads per CTA
+constexpr int CHUNK_NT = 512;   // threads per CTA of bwd_chunk_kernel (latency-bound SIMT phases)
+constexpr int PREP_NT = 512;    // threads per CTA of bwd_prep_kernel
 // Padded row strides of shared-memory tiles: 4 mod 32 floats, so the tensor-core
 // fragment loads (8 rows x 4 columns per warp) hit 32 distinct banks.
 constexpr int TP = DVT + 4;   // [*][DVT]
@@ -247,11 +249,11 @@ __device__ __forceinline__ void warp_mma_strip(float (&d)[TW][4], const float *A
 // Block product out[M x N] = A1 B1 (+ A2 B2): each warp takes a strip of one
 // 16-row block by TW 8-column tiles; every output element goes once through
 // epi(row, col, v).
-template <int M, int N, bool SPLIT, int K1, int K2 = 0, typename Epi>
+template <int M, int N, bool SPLIT, int K1, int K2 = 0, int NTH = NT, typename Epi>
 __device__ __forceinline__ void block_mma(const float *A1, int ar1, int ak1, const float *B1, int bk1, int bn1,
                                           const float *A2, int ar2, int ak2, const float *B2, int bk2, int bn2,
                                           Epi &&epi) {
-    constexpr int NW = NT / 32, NTN = N / 8, TILES = (M / 16) * NTN;
+    constexpr int NW = NTH / 32, NTN = N / 8, TILES = (M / 16) * NTN;
     constexpr int TW = TILES >= NW ? TILES / NW : 1;
     static_assert(TILES % NW == 0 || TILES < NW, "tiles must spread evenly over the warps");
     static_assert(NTN % TW == 0, "a strip stays inside one 16-row block");
@@ -273,18 +275,18 @@ __device__ __forceinline__ void block_mma(const float *A1, int ar1, int ak1, con
 // Loads one chunk's q, k and log_alpha rows (zero past Lc) and beta (if sB),
 // then turns log_alpha into the running sum G (per channel).  Every thread
 // issues all of its 4-element vector loads before the first shared store.
-template <int DK, typename Tin>
+template <int DK, typename Tin, int NTH = NT>
 __device__ __forceinline__ void load_chunk_qkg(const Tin *__restrict__ q, const Tin *__restrict__ k,
                                                const float *__restrict__ log_alpha, const float *__restrict__ beta,
                                                long long cs, int Lc, int H, int h, float *sQ, float *sK, float *sG,
                                                float *sB) {
     constexpr int DKP = Pad<DK>::K;
-    constexpr int NV = C * DK / 4 / NT;   // 4-element vectors per thread and tensor
+    constexpr int NV = C * DK / 4 / NTH;   // 4-element vectors per thread and tensor
     const int tid = threadIdx.x;
     float4 rq[NV], rk[NV], rg[NV];
 #pragma unroll
     for (int u = 0; u < NV; ++u) {
-        const int e = (tid + u * NT) * 4, i = e / DK, c = e % DK;
+        const int e = (tid + u * NTH) * 4, i = e / DK, c = e % DK;
         rq[u] = rk[u] = rg[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (i < Lc) {
             const long long off = ((cs + i) * H + h) * DK + c;
@@ -296,14 +298,14 @@ __device__ __forceinline__ void load_chunk_qkg(const Tin *__restrict__ q, const 
     const float bv = (sB && tid < C && tid < Lc) ? beta[(cs + tid) * H + h] : 0.f;
 #pragma unroll
     for (int u = 0; u < NV; ++u) {
-        const int e = (tid + u * NT) * 4, i = e / DK, c = e % DK;
+        const int e = (tid + u * NTH) * 4, i = e / DK, c = e % DK;
         *reinterpret_cast<float4 *>(sQ + i * DKP + c) = rq[u];
         *reinterpret_cast<float4 *>(sK + i * DKP + c) = rk[u];
         *reinterpret_cast<float4 *>(sG + i * DKP + c) = rg[u];
     }
     if (sB && tid < C) sB[tid] = bv;
     __syncthreads();
-    for (int c = tid; c < DK; c += NT) {
+    for (int c = tid; c < DK; c += NTH) {
         float acc = 0.f;
         for (int i = 0; i < C; ++i) {
             acc += sG[i * DKP + c];
@@ -328,7 +330,7 @@ __device__ __forceinline__ void async_rows(float *dst, int ld, const float *src,
                                            long long src_ld = -1) {
     const int q4 = cols / 4;
     const long long sld = src_ld < 0 ? cols : src_ld;
-    for (int idx = threadIdx.x; idx < rows * q4; idx += NT) {
+    for (int idx = threadIdx.x; idx < rows * q4; idx += blockDim.x) {
         const int r = idx / q4, c4 = (idx % q4) * 4;
         cp_async16(dst + r * ld + c4, src + r * sld + c4);
     }
@@ -348,11 +350,11 @@ constexpr float DIAG_RANGE = 40.f;   // largest in-block log-decay taken through
 // True when every channel decays by at most DIAG_RANGE (in log) across each
 // 16-row block, so the diagonal blocks can go through the block boundary with a
 // factor of at most e^DIAG_RANGE.  Uniform over the CTA (it synchronises).
-template <int DK>
+template <int DK, int NTH>
 __device__ __forceinline__ bool diag_blocks_in_range(const float *sG) {
     constexpr int DKP = Pad<DK>::K;
     bool bad = false;
-    for (int c = threadIdx.x; c < DK; c += NT)
+    for (int c = threadIdx.x; c < DK; c += NTH)
 #pragma unroll
         for (int b = 0; b < NSB; ++b) bad |= sG[(b * SB) * DKP + c] - sG[(b * SB + SB - 1) * DKP + c] > DIAG_RANGE;
     return !__syncthreads_or(bad);
@@ -362,12 +364,12 @@ __device__ __forceinline__ bool diag_blocks_in_range(const float *sG) {
 // scr holds 2 SB + C rows of stride DKP.  The diagonal blocks take the exact
 // pairwise exponent unless `diag` (every block's decay range within DIAG_RANGE),
 // in which case they join the tensor-core products through the block boundary.
-template <int DK, bool SPLIT>
+template <int DK, bool SPLIT, int NTH>
 __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, const float *sG, float *sAkk,
                                             float *sAqk, float *scr, bool diag) {
     constexpr int DKP = Pad<DK>::K;
     const int tid = threadIdx.x;
-    for (int idx = tid; idx < C * CP; idx += NT) {
+    for (int idx = tid; idx < C * CP; idx += NTH) {
         sAkk[idx] = 0.f;
         sAqk[idx] = 0.f;
     }
@@ -375,7 +377,8 @@ __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, co
     if (!diag) {   // diagonal blocks, exact: 8 lanes per (i, j) pair, each lane DK / 8 channels
         constexpr int PAIRS = NSB * SB * (SB + 1) / 2;
         const int l8 = tid & 7;
-        for (int p = tid >> 3; p < PAIRS; p += NT / 8) {
+        static_assert((PAIRS % (NTH / 8)) % 4 == 0, "uniform trip counts within each warp");
+        for (int p = tid >> 3; p < PAIRS; p += NTH / 8) {
             const int b = p / (SB * (SB + 1) / 2);
             int rem = p % (SB * (SB + 1) / 2), ii = 0;
             while (rem > ii) rem -= ++ii;
@@ -402,19 +405,19 @@ __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, co
     for (int bi = diag ? 0 : 1; bi < NSB; ++bi) {
         const int r = bi * SB, ncol = diag ? r + SB : r;
         __syncthreads();
-        for (int idx = tid; idx < SB * DK; idx += NT) {
+        for (int idx = tid; idx < SB * DK; idx += NTH) {
             const int ii = idx / DK, c = idx % DK, i = r + ii;
             const float e = __expf(sG[i * DKP + c] - sG[r * DKP + c]);
             sL[ii * DKP + c] = sK[i * DKP + c] * e;
             sL[(SB + ii) * DKP + c] = sQ[i * DKP + c] * e;
         }
-        for (int idx = tid; idx < ncol * DK; idx += NT) {
+        for (int idx = tid; idx < ncol * DK; idx += NTH) {
             const int j = idx / DK, c = idx % DK;
             sR[j * DKP + c] = sK[j * DKP + c] * __expf(sG[r * DKP + c] - sG[j * DKP + c]);
         }
         __syncthreads();
         const int ntn = ncol / 8;
-        for (int t = tid >> 5; t < 2 * ntn; t += NT / 32) {
+        for (int t = tid >> 5; t < 2 * ntn; t += NTH / 32) {
             const int r0 = (t / ntn) * SB, c0 = (t % ntn) * 8;
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             warp_mma<SPLIT, DK>(d, sL + r0 * DKP, DKP, 1, sR + c0 * DKP, 1, DKP);
@@ -432,21 +435,24 @@ __device__ __forceinline__ void chunk_grams(const float *sQ, const float *sK, co
     __syncthreads();
 }
 
-// q -> e^G q, k -> e^G k and G -> e^{G_C - G} k; d = e^{G_C}.
-template <int DK>
+// q -> e^G q, k -> e^G k and G -> e^{G_C - G} k; d = e^{G_C}.  Every thread keeps
+// one channel (NTH is a multiple of DK) and takes every (NTH / DK)-th row; G_C is
+// read by all before any row is overwritten.
+template <int DK, int NTH>
 __device__ __forceinline__ void chunk_factors(float *sQ, float *sK, float *sG, float *sD) {
-    constexpr int DKP = Pad<DK>::K;
-    for (int c = threadIdx.x; c < DK; c += NT) {
-        const float gl = sG[(C - 1) * DKP + c];
-        sD[c] = __expf(gl);
-        for (int i = 0; i < C; ++i) {
-            const float gi = sG[i * DKP + c];
-            const float e = __expf(gi);
-            const float kc = sK[i * DKP + c];
-            sQ[i * DKP + c] *= e;
-            sK[i * DKP + c] = kc * e;
-            sG[i * DKP + c] = kc * __expf(gl - gi);
-        }
+    constexpr int DKP = Pad<DK>::K, RSTEP = NTH / DK;
+    static_assert(NTH % DK == 0, "one channel per thread");
+    const int c = threadIdx.x % DK, i0 = threadIdx.x / DK;
+    const float gl = sG[(C - 1) * DKP + c];
+    if (i0 == 0) sD[c] = __expf(gl);
+    __syncthreads();
+    for (int i = i0; i < C; i += RSTEP) {
+        const float gi = sG[i * DKP + c];
+        const float e = __expf(gi);
+        const float kc = sK[i * DKP + c];
+        sQ[i * DKP + c] *= e;
+        sK[i * DKP + c] = kc * e;
+        sG[i * DKP + c] = kc * __expf(gl - gi);
     }
     __syncthreads();
 }
@@ -455,14 +461,14 @@ __device__ __forceinline__ void chunk_factors(float *sQ, float *sK, float *sG, f
 // the diagonal, from its diagonal block and the block rows above:
 //   Y = Diag(beta) Akk[r..r+16)[0..r) T[0..r)[0..r)   (in scr)
 //   T[r..r+16)[0..r) = -T[r..r+16)[r..r+16) Y
-template <bool SPLIT, int BI>
+template <bool SPLIT, int BI, int NTH>
 __device__ __forceinline__ void t_block_row(const float *sAkk, const float *sB, float *sT, float *scr) {
     constexpr int r = BI * SB;
     __syncthreads();
-    block_mma<SB, r, SPLIT, r>(sAkk + r * CP, CP, 1, sT, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
+    block_mma<SB, r, SPLIT, r, 0, NTH>(sAkk + r * CP, CP, 1, sT, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                [&](int ii, int j, float x) { scr[ii * CP + j] = sB[r + ii] * x; });
     __syncthreads();
-    block_mma<SB, r, SPLIT, SB>(sT + r * CP + r, CP, 1, scr, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
+    block_mma<SB, r, SPLIT, SB, 0, NTH>(sT + r * CP + r, CP, 1, scr, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                 [&](int ii, int j, float x) { sT[(r + ii) * CP + j] = -x; });
 }
 
@@ -486,7 +492,7 @@ struct PrepSmem {
 };
 
 template <int DK, typename Tin>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(PREP_NT, 1)
 bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const float *__restrict__ log_alpha,
                 const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
                 float *__restrict__ rec) {
@@ -494,6 +500,7 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
     using R = Rec<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
+    constexpr int NTH = PREP_NT;
     extern __shared__ __align__(128) float sm[];
     float *sQ = sm + L::q, *sK = sm + L::k, *sG = sm + L::g, *sAkk = sm + L::akk, *sAqk = sm + L::aqk;
     float *sT = sm + L::ti, *sTb = sm + L::tb, *sB = sm + L::b, *sD = sm + L::d;
@@ -502,15 +509,15 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
     int Lc;
     if (!chunk_of_slot(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
 
-    load_chunk_qkg<DK, Tin>(q, k, log_alpha, beta, cs, Lc, H, h, sQ, sK, sG, sB);
-    chunk_grams<DK, SPLIT>(sQ, sK, sG, sAkk, sAqk, sm + L::scr, diag_blocks_in_range<DK>(sG));
-    chunk_factors<DK>(sQ, sK, sG, sD);
+    load_chunk_qkg<DK, Tin, NTH>(q, k, log_alpha, beta, cs, Lc, H, h, sQ, sK, sG, sB);
+    chunk_grams<DK, SPLIT, NTH>(sQ, sK, sG, sAkk, sAqk, sm + L::scr, diag_blocks_in_range<DK, NTH>(sG));
+    chunk_factors<DK, NTH>(sQ, sK, sG, sD);
     // T = (I + Diag(beta) Akk)^{-1}: the 16 x 16 diagonal blocks by forward
     // substitution (4 lanes per column, all 64 columns at once), then each block
     // row below the diagonal from the rows above it (t_block_row).
-    for (int idx = tid; idx < C * CP; idx += NT) sT[idx] = 0.f;
+    for (int idx = tid; idx < C * CP; idx += NTH) sT[idx] = 0.f;
     __syncthreads();
-    {
+    if (tid < NSB * SB * 4) {   // 64 columns x 4 lanes: whole warps, so the shuffles stay full
         const int prob = tid >> 2, l4 = tid & 3, b0 = (prob / SB) * SB, col = prob % SB;
         for (int ii = 0; ii < SB; ++ii) {
             const int i = b0 + ii;
@@ -522,11 +529,11 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
             __syncwarp();
         }
     }
-    t_block_row<SPLIT, 1>(sAkk, sB, sT, sm + L::scr);
-    t_block_row<SPLIT, 2>(sAkk, sB, sT, sm + L::scr);
-    t_block_row<SPLIT, 3>(sAkk, sB, sT, sm + L::scr);
+    t_block_row<SPLIT, 1, NTH>(sAkk, sB, sT, sm + L::scr);
+    t_block_row<SPLIT, 2, NTH>(sAkk, sB, sT, sm + L::scr);
+    t_block_row<SPLIT, 3, NTH>(sAkk, sB, sT, sm + L::scr);
     __syncthreads();
-    for (int idx = tid; idx < C * C; idx += NT) {
+    for (int idx = tid; idx < C * C; idx += NTH) {
         const int i = idx / C, j = idx % C;
         sTb[i * CP + j] = sT[i * CP + j] * sB[j];
     }
@@ -546,9 +553,9 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
         ptx::bulk_commit();
     }
     // Pt = Aqk Tb;  Kt = Kb^T Tb
-    block_mma<C, C, SPLIT, C>(sAqk, CP, 1, sTb, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
+    block_mma<C, C, SPLIT, C, 0, NTH>(sAqk, CP, 1, sTb, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
                               [&](int i, int j, float x) { r[R::PT + i * CP + j] = x; });
-    block_mma<DK, C, SPLIT, C>(sG, 1, DKP, sTb, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
+    block_mma<DK, C, SPLIT, C, 0, NTH>(sG, 1, DKP, sTb, CP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                [&](int c, int j, float x) { r[R::KT + c * CP + j] = x; });
     if (tid == 0) ptx::bulk_wait_read_all();   // shared memory stays valid until the stores have read it
 }
@@ -952,11 +959,11 @@ struct ChunkSmem {
 // acc_j += sum_{i>=j} (A1[i][j] q_i + [i>j] A2[i][j] k_i) E_ij, dG_j -= k_j (that),
 // plus the row terms of A2.  Q phase: A1 = dAqk, no A2.  K phase: A1 = dAqk
 // (columns only), A2 = dAkk (rows and columns).
-template <int DK, bool KPHASE>
+template <int DK, bool KPHASE, int NTH>
 __device__ __forceinline__ void diag_pair_terms(const float *sQ, const float *sK, const float *sG, const float *sAq,
                                                 const float *sAk, float *sAcc, float *sDg) {
     constexpr int DKP = Pad<DK>::K;
-    constexpr int NG = NT / DK;   // thread groups per channel
+    constexpr int NG = NTH / DK;   // thread groups per channel
     const int c = threadIdx.x % DK, grp = threadIdx.x / DK;
     for (int b = grp; b < NSB; b += NG) {
         const int r = b * SB;
@@ -997,18 +1004,18 @@ __device__ __forceinline__ void diag_pair_terms(const float *sQ, const float *sK
 // Row terms of block bi (rows r..r+15, r = 16 bi) over columns j in [J0, J1), J1 <= r:
 // acc_i += e^{G_i - G_r} sum_j A[i][j] (k_j e^{G_r - G_j}); dG_i += k_i (that) when
 // to_dg.  Both factors are <= 1.
-template <int DK, bool SPLIT, int BI, int J0, int J1>
+template <int DK, bool SPLIT, int NTH, int BI, int J0, int J1>
 __device__ __forceinline__ void row_terms(const float *sK, const float *sG, const float *sA, float *scr,
                                           float *sAcc, float *sDg, bool to_dg) {
     constexpr int DKP = Pad<DK>::K, r = BI * SB, n = J1 - J0;
     static_assert(n > 0 && n <= SCR_ROWS, "operand fits the scratch");
     __syncthreads();
-    for (int idx = threadIdx.x; idx < n * DK; idx += NT) {
+    for (int idx = threadIdx.x; idx < n * DK; idx += NTH) {
         const int jj = idx / DK, c = idx % DK, j = J0 + jj;
         scr[jj * DKP + c] = sK[j * DKP + c] * __expf(sG[r * DKP + c] - sG[j * DKP + c]);
     }
     __syncthreads();
-    block_mma<SB, DK, SPLIT, n>(sA + r * CP + J0, CP, 1, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
+    block_mma<SB, DK, SPLIT, n, 0, NTH>(sA + r * CP + J0, CP, 1, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                 [&](int ii, int c, float x) {
                                     const int i = r + ii;
                                     x *= __expf(sG[i * DKP + c] - sG[r * DKP + c]);
@@ -1018,20 +1025,20 @@ __device__ __forceinline__ void row_terms(const float *sK, const float *sG, cons
 }
 
 // Row terms of the blocks below the diagonal.
-template <int DK, bool SPLIT>
+template <int DK, bool SPLIT, int NTH>
 __device__ __forceinline__ void pair_rows(const float *sK, const float *sG, const float *sA, float *scr, float *sAcc,
                                           float *sDg, bool to_dg) {
     static_assert(NSB == 4 && SCR_ROWS == 48, "four 16-row blocks");
-    row_terms<DK, SPLIT, 1, 0, 16>(sK, sG, sA, scr, sAcc, sDg, to_dg);
-    row_terms<DK, SPLIT, 2, 0, 32>(sK, sG, sA, scr, sAcc, sDg, to_dg);
-    row_terms<DK, SPLIT, 3, 0, 48>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+    row_terms<DK, SPLIT, NTH, 1, 0, 16>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+    row_terms<DK, SPLIT, NTH, 2, 0, 32>(sK, sG, sA, scr, sAcc, sDg, to_dg);
+    row_terms<DK, SPLIT, NTH, 3, 0, 48>(sK, sG, sA, scr, sAcc, sDg, to_dg);
     __syncthreads();
 }
 
 // Column terms of block bj (columns 16 bj..16 bj+15, last row s) over rows i in
 // [I0, I1), I0 > s: acc_j += e^{G_s - G_j} sum_i A[i][j] (X_i e^{G_i - G_s}),
 // dG_j -= k_j (that), for (A, X) = (dAqk, q) and (dAkk, k).  Both factors are <= 1.
-template <int DK, bool SPLIT, int BJ, int I0, int I1>
+template <int DK, bool SPLIT, int NTH, int BJ, int I0, int I1>
 __device__ __forceinline__ void col_terms(const float *sQ, const float *sK, const float *sG, const float *sAq,
                                           const float *sAk, float *scr, float *sAcc, float *sDg) {
     constexpr int DKP = Pad<DK>::K, s = BJ * SB + SB - 1, n = I1 - I0;
@@ -1040,12 +1047,12 @@ __device__ __forceinline__ void col_terms(const float *sQ, const float *sK, cons
         const float *X = pass ? sK : sQ;
         const float *A = pass ? sAk : sAq;
         __syncthreads();
-        for (int idx = threadIdx.x; idx < n * DK; idx += NT) {
+        for (int idx = threadIdx.x; idx < n * DK; idx += NTH) {
             const int ii = idx / DK, c = idx % DK, i = I0 + ii;
             scr[ii * DKP + c] = X[i * DKP + c] * __expf(sG[i * DKP + c] - sG[s * DKP + c]);
         }
         __syncthreads();
-        block_mma<SB, DK, SPLIT, n>(A + I0 * CP + BJ * SB, 1, CP, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<SB, DK, SPLIT, n, 0, NTH>(A + I0 * CP + BJ * SB, 1, CP, scr, DKP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                     [&](int jj, int c, float x) {
                                         const int j = BJ * SB + jj;
                                         x *= __expf(sG[s * DKP + c] - sG[j * DKP + c]);
@@ -1056,17 +1063,17 @@ __device__ __forceinline__ void col_terms(const float *sQ, const float *sK, cons
 }
 
 // Column terms of the blocks below the diagonal.
-template <int DK, bool SPLIT>
+template <int DK, bool SPLIT, int NTH>
 __device__ __forceinline__ void pair_cols(const float *sQ, const float *sK, const float *sG, const float *sAq,
                                           const float *sAk, float *scr, float *sAcc, float *sDg) {
-    col_terms<DK, SPLIT, 0, 16, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
-    col_terms<DK, SPLIT, 1, 32, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
-    col_terms<DK, SPLIT, 2, 48, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    col_terms<DK, SPLIT, NTH, 0, 16, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    col_terms<DK, SPLIT, NTH, 1, 32, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    col_terms<DK, SPLIT, NTH, 2, 48, 64>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
     __syncthreads();
 }
 
 template <int DK, typename Tin>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(CHUNK_NT, 1)
 bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const float *__restrict__ log_alpha,
                  const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
                  const float *__restrict__ part, Tin *__restrict__ dq, Tin *__restrict__ dk_out,
@@ -1075,6 +1082,7 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
     using P = Part<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
+    constexpr int NTH = CHUNK_NT;
     extern __shared__ __align__(128) float sm[];
     float *sQ = sm + L::q, *sK = sm + L::k, *sG = sm + L::g, *sAcc = sm + L::acc, *sDg = sm + L::dg;
     float *sAq = sm + L::aq, *sAk = sm + L::ak, *scr = sm + L::scr;
@@ -1083,22 +1091,22 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
     int Lc;
     if (!chunk_of_slot(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
     const float *pp = part + ((long long)slot * H + h) * P::FLOATS;
-    constexpr int NV = C * DK / 4 / NT;   // 4-element vectors per thread
+    constexpr int NV = C * DK / 4 / NTH;   // 4-element vectors per thread
     // dAqk (zero above the diagonal) and dAkk (zero on and above it) by async copy
     async_rows(sAq, CP, pp + P::AQK, C, C);
     async_rows(sAk, CP, pp + P::AKK, C, C);
     cp_async_commit();
-    for (int i = tid; i < Lc; i += NT) dbeta[(cs + i) * H + h] = pp[P::DB + i];
-    load_chunk_qkg<DK, Tin>(q, k, log_alpha, nullptr, cs, Lc, H, h, sQ, sK, sG, nullptr);
+    for (int i = tid; i < Lc; i += NTH) dbeta[(cs + i) * H + h] = pp[P::DB + i];
+    load_chunk_qkg<DK, Tin, NTH>(q, k, log_alpha, nullptr, cs, Lc, H, h, sQ, sK, sG, nullptr);
 
     // ---- dq = e^G dQh + pair terms of dAqk;  dG = q dq
     {
         float4 r[NV];
 #pragma unroll
-        for (int u = 0; u < NV; ++u) r[u] = *reinterpret_cast<const float4 *>(pp + P::DQ + (tid + u * NT) * 4);
+        for (int u = 0; u < NV; ++u) r[u] = *reinterpret_cast<const float4 *>(pp + P::DQ + (tid + u * NTH) * 4);
 #pragma unroll
         for (int u = 0; u < NV; ++u) {
-            const int e = (tid + u * NT) * 4, i = e / DK, c = e % DK;
+            const int e = (tid + u * NTH) * 4, i = e / DK, c = e % DK;
             const float *g = sG + i * DKP + c;
             *reinterpret_cast<float4 *>(sAcc + i * DKP + c) =
                 make_float4(__expf(g[0]) * r[u].x, __expf(g[1]) * r[u].y, __expf(g[2]) * r[u].z, __expf(g[3]) * r[u].w);
@@ -1108,22 +1116,22 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
     __syncthreads();
     // The diagonal blocks stay exact on CUDA cores here: taking them through the
     // block boundary costs two more scaled operands per phase, which measured slower.
-    diag_pair_terms<DK, false>(sQ, sK, sG, sAq, nullptr, sAcc, nullptr);
-    pair_rows<DK, SPLIT>(sK, sG, sAq, scr, sAcc, nullptr, false);
+    diag_pair_terms<DK, false, NTH>(sQ, sK, sG, sAq, nullptr, sAcc, nullptr);
+    pair_rows<DK, SPLIT, NTH>(sK, sG, sAq, scr, sAcc, nullptr, false);
     // dq out; dk starts at a + b and dG at q dq + k (a - b); sum_i k_i b_i per
     // channel (a dG_C term) goes to scr, one row per group of rows
     {
         float4 ra[NV], rb[NV];
 #pragma unroll
         for (int u = 0; u < NV; ++u) {
-            ra[u] = *reinterpret_cast<const float4 *>(pp + P::DKH + (tid + u * NT) * 4);
-            rb[u] = *reinterpret_cast<const float4 *>(pp + P::DKB + (tid + u * NT) * 4);
+            ra[u] = *reinterpret_cast<const float4 *>(pp + P::DKH + (tid + u * NTH) * 4);
+            rb[u] = *reinterpret_cast<const float4 *>(pp + P::DKB + (tid + u * NTH) * 4);
         }
         float kb[4] = {0.f, 0.f, 0.f, 0.f};
-        const int c = (tid * 4) % DK;   // the same 4 channels for every u (NT * 4 is a multiple of DK)
+        const int c = (tid * 4) % DK;   // the same 4 channels for every u (NTH * 4 is a multiple of DK)
 #pragma unroll
         for (int u = 0; u < NV; ++u) {
-            const int e = (tid + u * NT) * 4, i = e / DK;
+            const int e = (tid + u * NTH) * 4, i = e / DK;
             const float ha[4] = {ra[u].x, ra[u].y, ra[u].z, ra[u].w}, hb[4] = {rb[u].x, rb[u].y, rb[u].z, rb[u].w};
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -1144,18 +1152,18 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
     __syncthreads();
     float kb_sum = 0.f;   // this thread's channel (tid < DK) of sum_i k_i b_i
     if (tid < DK)
-        for (int gq = 0; gq < NT * 4 / DK; ++gq) kb_sum += scr[gq * DKP + tid];
+        for (int gq = 0; gq < NTH * 4 / DK; ++gq) kb_sum += scr[gq * DKP + tid];
     __syncthreads();
     // ---- dk = a + b + pair terms of dAkk (rows) and of dAqk, dAkk (columns)
-    diag_pair_terms<DK, true>(sQ, sK, sG, sAq, sAk, sAcc, sDg);
-    pair_rows<DK, SPLIT>(sK, sG, sAk, scr, sAcc, sDg, true);
-    pair_cols<DK, SPLIT>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
-    for (int idx = tid; idx < C * DK; idx += NT) {
+    diag_pair_terms<DK, true, NTH>(sQ, sK, sG, sAq, sAk, sAcc, sDg);
+    pair_rows<DK, SPLIT, NTH>(sK, sG, sAk, scr, sAcc, sDg, true);
+    pair_cols<DK, SPLIT, NTH>(sQ, sK, sG, sAq, sAk, scr, sAcc, sDg);
+    for (int idx = tid; idx < C * DK; idx += NTH) {
         const int i = idx / DK, c = idx % DK;
         if (i < Lc) Elem<Tin>::store(dk_out + ((cs + i) * H + h) * DK + c, sAcc[i * DKP + c]);
     }
     // ---- dG_C terms, then dlog_alpha_s = sum_{i>=s} dG_i
-    for (int c = tid; c < DK; c += NT) {
+    for (int c = tid; c < DK; c += NTH) {
         const float gC = sG[(C - 1) * DKP + c];
         float acc = __expf(gC) * pp[P::DGC + c] + kb_sum;
         for (int i = C - 1; i >= 0; --i) {

@@ -280,7 +280,7 @@ int launch_backward(const void *q, const void *k, const void *v, const float *lo
     const dim3 per_chunk((unsigned)slots, H);
     cudaError_t e;
     if (tokens > 0) {
-        k_prep<<<per_chunk, b::NT, b::PrepSmem<DK>::bytes, st>>>((const Tin *)q, (const Tin *)k, log_alpha, beta,
+        k_prep<<<per_chunk, b::PREP_NT, b::PrepSmem<DK>::bytes, st>>>((const Tin *)q, (const Tin *)k, log_alpha, beta,
                                                                   cu_seqlens, T, H, num_seqs, rec);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_prep launch");
     }
@@ -292,7 +292,7 @@ int launch_backward(const void *q, const void *k, const void *v, const float *lo
                                                                   (Tin *)dv_out, cu_seqlens, T, H, dv, num_seqs,
                                                                   rec, ckpt, dckpt, part);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_part launch");
-        k_chunk<<<per_chunk, b::NT, b::ChunkSmem<DK>::bytes, st>>>((const Tin *)q, (const Tin *)k, log_alpha,
+        k_chunk<<<per_chunk, b::CHUNK_NT, b::ChunkSmem<DK>::bytes, st>>>((const Tin *)q, (const Tin *)k, log_alpha,
                                                                     beta, cu_seqlens, T, H, num_seqs, part,
                                                                     (Tin *)dq, (Tin *)dk_out, dlog_alpha, dbeta);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_chunk launch");
