@@ -63,6 +63,12 @@ constexpr int DVT = 32;    // value columns per tile
 constexpr int NT = 256;    // threads per CTA
 constexpr int CHUNK_NT = 512;   // threads per CTA of bwd_chunk_kernel (latency-bound SIMT phases)
 constexpr int PREP_NT = 512;    // threads per CTA of bwd_prep_kernel
+// threads per CTA of bwd_part_kernel (512 measured no faster, and fp32 inputs'
+// split products need more registers than 512 threads leave)
+template <typename Tin>
+struct PartThreads {
+    static constexpr int value = 256;
+};
 // Padded row strides of shared-memory tiles: 4 mod 32 floats, so the tensor-core
 // fragment loads (8 rows x 4 columns per warp) hit 32 distinct banks.
 constexpr int TP = DVT + 4;   // [*][DVT]
@@ -768,7 +774,7 @@ struct PartSmem {
 };
 
 template <int DK, typename Tin>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(PartThreads<Tin>::value, 1)
 bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const Tin *__restrict__ d_o,
                 Tin *__restrict__ dv_out, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV,
                 int num_seqs, const float *__restrict__ rec, const float *__restrict__ ckpt,
@@ -778,7 +784,7 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
     using P = Part<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
-    constexpr int NW = NT / 32;
+    constexpr int NTH = PartThreads<Tin>::value, NW = NTH / 32;
     // Column sums accumulate in registers across the value tiles: each warp owns a
     // strip of one 16-row block by TQ (TA) adjacent 8-column tiles of the [C][DK]
     // ([C][C]) sums.
@@ -811,7 +817,7 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         ptx::bulk_load(ptx::smem_u32(sT), rp + R::TI, R::ROWS_C, bar);
         ptx::bulk_load(ptx::smem_u32(sTb), rp + R::TB, R::ROWS_C, bar);
     }
-    for (int i = tid; i < C; i += NT) {
+    for (int i = tid; i < C; i += NTH) {
         sB[i] = i < Lc ? beta[(cs + i) * H + h] : 0.f;
         sDB[i] = 0.f;
     }
@@ -833,11 +839,11 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         async_rows(sdS, TP, dckpt + st_base + col_base, DK, DVT, DV);
         cp_async_commit();
         {
-            constexpr int NV = C * DVT / 4 / NT;   // 4-element vectors of V and dO per thread
+            constexpr int NV = C * DVT / 4 / NTH;   // 4-element vectors of V and dO per thread
             float4 rv[NV], rd[NV];
 #pragma unroll
             for (int u = 0; u < NV; ++u) {
-                const int e = (tid + u * NT) * 4, i = e / DVT, j = e % DVT;
+                const int e = (tid + u * NTH) * 4, i = e / DVT, j = e % DVT;
                 rv[u] = rd[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (i < Lc) {
                     const long long off = ((cs + i) * H + h) * DV + col_base + j;
@@ -847,7 +853,7 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
             }
 #pragma unroll
             for (int u = 0; u < NV; ++u) {
-                const int e = (tid + u * NT) * 4, i = e / DVT, j = e % DVT;
+                const int e = (tid + u * NTH) * 4, i = e / DVT, j = e % DVT;
                 *reinterpret_cast<float4 *>(sW + i * TP + j) = rv[u];
                 *reinterpret_cast<float4 *>(sDO + i * TP + j) = rd[u];
             }
@@ -859,19 +865,19 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         }
         __syncthreads();
         // W = V - Kh S (in place: each element is read and written by its owner only)
-        block_mma<C, DVT, SPLIT, DK>(sKh, DKP, 1, sS, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<C, DVT, SPLIT, DK, 0, NTH>(sKh, DKP, 1, sS, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sW[i * TP + j] -= x; });
         __syncthreads();
         // U = Tb W;  dU = Aqk^T dO + Kb dS
-        block_mma<C, DVT, SPLIT, C>(sTb, CP, 1, sW, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<C, DVT, SPLIT, C, 0, NTH>(sTb, CP, 1, sW, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sU[i * TP + j] = x; });
-        block_mma<C, DVT, SPLIT, C, DK>(sAqk, 1, CP, sDO, TP, 1, sKb, DKP, 1, sdS, TP, 1,
+        block_mma<C, DVT, SPLIT, C, DK, NTH>(sAqk, 1, CP, sDO, TP, 1, sKb, DKP, 1, sdS, TP, 1,
                                  [&](int i, int j, float x) { sdU[i * TP + j] = x; });
         __syncthreads();
         // R = W - Akk U (in place of W);  lam = T^T dU
-        block_mma<C, DVT, SPLIT, C>(sAkk, CP, 1, sU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<C, DVT, SPLIT, C, 0, NTH>(sAkk, CP, 1, sU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sW[i * TP + j] -= x; });
-        block_mma<C, DVT, SPLIT, C>(sT, 1, CP, sdU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<C, DVT, SPLIT, C, 0, NTH>(sT, 1, CP, sdU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sL[i * TP + j] = x; });
         __syncthreads();
         // dbeta: <lam_i, R_i> (one warp per 8 rows; the same lane adds every tile)
@@ -885,7 +891,7 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         }
         __syncthreads();
         // mu = beta lam; dV = mu
-        for (int idx = tid; idx < C * DVT; idx += NT) {
+        for (int idx = tid; idx < C * DVT; idx += NTH) {
             const int i = idx / DVT, j = idx % DVT;
             const float mu = sB[i] * sL[i * TP + j];
             sL[i * TP + j] = mu;
@@ -932,7 +938,7 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         }
     }
     __syncthreads();
-    for (int i = tid; i < C; i += NT) pp[P::DB + i] = sDB[i];
+    for (int i = tid; i < C; i += NTH) pp[P::DB + i] = sDB[i];
     if (tid < DK) pp[P::DGC + tid] = a_gc;
 }
 

@@ -288,7 +288,7 @@ int launch_backward(const void *q, const void *k, const void *v, const float *lo
         (const Tin *)v, init_state, (const Tin *)d_o, dfinal, dinit_state, cu_seqlens, T, H, dv, rec, ckpt, dckpt);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_state launch");
     if (tokens > 0) {
-        k_part<<<per_chunk, b::NT, b::PartSmem<DK>::bytes, st>>>((const Tin *)v, beta, (const Tin *)d_o,
+        k_part<<<per_chunk, b::PartThreads<Tin>::value, b::PartSmem<DK>::bytes, st>>>((const Tin *)v, beta, (const Tin *)d_o,
                                                                   (Tin *)dv_out, cu_seqlens, T, H, dv, num_seqs,
                                                                   rec, ckpt, dckpt, part);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_part launch");
