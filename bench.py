@@ -57,8 +57,8 @@ NCU_TRAFFIC = {
     ("prefill_8k", "chunk_tc_kernel"): 338.8e6 + 56.0e6,
     ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.7e6,
     # backward: all four kernels of one call; T=2048 captured, T=8192 scaled by the chunk slots (129 / 33)
-    ("backward_T2048", "bwd"): 775.6e6 + 419.9e6,
-    ("backward_T8192", "bwd"): (775.6e6 + 419.9e6) * 129 / 33,
+    ("backward_T2048", "bwd"): 795.3e6 + 431.1e6,
+    ("backward_T8192", "bwd"): (795.3e6 + 431.1e6) * 129 / 33,
 }
 
 
