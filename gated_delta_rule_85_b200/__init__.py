@@ -22,7 +22,7 @@ from types import SimpleNamespace
 import torch
 
 __all__ = [
-    "chunk_forward", "chunk_backward", "backward_workspace_size", "chunk_forward_prologue",
+    "chunk_forward", "chunk_backward", "gdn_chunk_backward", "backward_workspace_size", "chunk_forward_prologue",
     "recurrent_step_prologue", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
     "recurrent_step_slots", "gdn_chunk_forward", "gdn_recurrent_step", "workspace_size", "device_status",
     "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
@@ -94,6 +94,8 @@ def load_library():
     lib.kda_chunk_backward.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, vp, vp, fp, fp, fp, ip] + \
         [ci] * 8 + [vp, sz, vp]
     lib.kda_chunk_backward.restype = ci
+    lib.kda_gdn_chunk_backward.argtypes = lib.kda_chunk_backward.argtypes
+    lib.kda_gdn_chunk_backward.restype = ci
     lib.kda_chunk_backward_workspace_size.argtypes = [ci] * 6
     lib.kda_chunk_backward_workspace_size.restype = sz
     lib.kda_last_error.argtypes = []
@@ -278,8 +280,18 @@ def backward_workspace_size(B, T, H, dk, dv, num_seqs) -> int:
     return int(load_library().kda_chunk_backward_workspace_size(B, T, H, dk, dv, num_seqs))
 
 
+def gdn_chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=None, cu_seqlens=None, *,
+                       dinit_state=True, workspace=None, out=None):
+    """Gradients through the Gated DeltaNet prefill (kda_gdn_chunk_backward):
+    log_alpha and the returned dlog_alpha are [B, T, H]; otherwise as chunk_backward."""
+    if log_alpha.shape != q.shape[:3]:
+        raise ValueError("log_alpha must be [B, T, H] (one rate per token-head)")
+    return chunk_backward(q, k, v, log_alpha, beta, d_o, init_state, dfinal_state, cu_seqlens,
+                          dinit_state=dinit_state, workspace=workspace, out=out, _gate_scalar=True)
+
+
 def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=None, cu_seqlens=None, *,
-                   dinit_state=True, workspace=None, out=None):
+                   dinit_state=True, workspace=None, out=None, _gate_scalar=False):
     """Gradients of sum <d_o, o> + <dfinal_state, final_state> through the chunked
     prefill (kda_chunk_backward): a dict with dq, dk, dv (in q's dtype),
     dlog_alpha, dbeta and dinit_state (float32; None when dinit_state=False).
@@ -289,7 +301,8 @@ def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=
     The workspace (uint8, CUDA) and the outputs (`out`, a dict with any of the
     keys above) are allocated here unless given.  Device tensors only.
     """
-    B, T, H, dk, dv, N = _prefill_args(q, k, v, log_alpha, beta, init_state, cu_seqlens)
+    gate = SimpleNamespace(shape=q.shape, dtype=log_alpha.dtype) if _gate_scalar else log_alpha
+    B, T, H, dk, dv, N = _prefill_args(q, k, v, gate, beta, init_state, cu_seqlens)
     if d_o.shape != v.shape or d_o.dtype != q.dtype:
         raise ValueError("d_o must have o's shape and dtype")
     if dfinal_state is not None and (dfinal_state.shape != (N, H, dk, dv) or dfinal_state.dtype != torch.float32):
@@ -312,10 +325,10 @@ def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib.kda_chunk_backward(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(d_o),
-                                _p(dfinal_state), _p(g["dq"]), _p(g["dk"]), _p(g["dv"]), _p(g["dlog_alpha"]),
-                                _p(g["dbeta"]), _p(g["dinit_state"]), _p(cu_seqlens), B, T, H, dk, dv, N,
-                                _dtype_code(q), CHUNK, _p(workspace), ws_bytes, _stream(dev))
+    entry = lib.kda_gdn_chunk_backward if _gate_scalar else lib.kda_chunk_backward
+    rc = entry(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(d_o), _p(dfinal_state), _p(g["dq"]),
+               _p(g["dk"]), _p(g["dv"]), _p(g["dlog_alpha"]), _p(g["dbeta"]), _p(g["dinit_state"]), _p(cu_seqlens),
+               B, T, H, dk, dv, N, _dtype_code(q), CHUNK, _p(workspace), ws_bytes, _stream(dev))
     _check(rc)
     return g
 

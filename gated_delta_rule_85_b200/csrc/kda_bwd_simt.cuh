@@ -279,9 +279,10 @@ __device__ __forceinline__ void block_mma(const float *A1, int ar1, int ak1, con
 // ------------------------------------------------------------------ chunk helpers
 
 // Loads one chunk's q, k and log_alpha rows (zero past Lc) and beta (if sB),
-// then turns log_alpha into the running sum G (per channel).  Every thread
+// then turns log_alpha into the running sum G (per channel).  GS: log_alpha is
+// one value per (token, head) (Gated DeltaNet), broadcast over the channels.  Every thread
 // issues all of its 4-element vector loads before the first shared store.
-template <int DK, typename Tin, int NTH = NT>
+template <int DK, typename Tin, int NTH = NT, bool GS = false>
 __device__ __forceinline__ void load_chunk_qkg(const Tin *__restrict__ q, const Tin *__restrict__ k,
                                                const float *__restrict__ log_alpha, const float *__restrict__ beta,
                                                long long cs, int Lc, int H, int h, float *sQ, float *sK, float *sG,
@@ -298,7 +299,12 @@ __device__ __forceinline__ void load_chunk_qkg(const Tin *__restrict__ q, const 
             const long long off = ((cs + i) * H + h) * DK + c;
             rq[u] = load4(q + off);
             rk[u] = load4(k + off);
-            rg[u] = *reinterpret_cast<const float4 *>(log_alpha + off);
+            if constexpr (GS) {   // one decay rate per (token, head), broadcast over the key channels
+                const float gs = log_alpha[(cs + i) * H + h];
+                rg[u] = make_float4(gs, gs, gs, gs);
+            } else {
+                rg[u] = *reinterpret_cast<const float4 *>(log_alpha + off);
+            }
         }
     }
     const float bv = (sB && tid < C && tid < Lc) ? beta[(cs + tid) * H + h] : 0.f;
@@ -497,7 +503,7 @@ struct PrepSmem {
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
 
-template <int DK, typename Tin>
+template <int DK, typename Tin, bool GS>
 __global__ void __launch_bounds__(PREP_NT, 1)
 bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const float *__restrict__ log_alpha,
                 const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
@@ -515,7 +521,7 @@ bwd_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const floa
     int Lc;
     if (!chunk_of_slot(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
 
-    load_chunk_qkg<DK, Tin, NTH>(q, k, log_alpha, beta, cs, Lc, H, h, sQ, sK, sG, sB);
+    load_chunk_qkg<DK, Tin, NTH, GS>(q, k, log_alpha, beta, cs, Lc, H, h, sQ, sK, sG, sB);
     chunk_grams<DK, SPLIT, NTH>(sQ, sK, sG, sAkk, sAqk, sm + L::scr, diag_blocks_in_range<DK, NTH>(sG));
     chunk_factors<DK, NTH>(sQ, sK, sG, sD);
     // T = (I + Diag(beta) Akk)^{-1}: the 16 x 16 diagonal blocks by forward
@@ -1078,7 +1084,9 @@ __device__ __forceinline__ void pair_cols(const float *sQ, const float *sK, cons
     __syncthreads();
 }
 
-template <int DK, typename Tin>
+// GS: scalar gate (Gated DeltaNet) -- log_alpha and dlog_alpha are [tokens, H];
+// the gradient of a rate broadcast over the channels is the sum over them.
+template <int DK, typename Tin, bool GS>
 __global__ void __launch_bounds__(CHUNK_NT, 1)
 bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const float *__restrict__ log_alpha,
                  const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
@@ -1103,7 +1111,7 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
     async_rows(sAk, CP, pp + P::AKK, C, C);
     cp_async_commit();
     for (int i = tid; i < Lc; i += NTH) dbeta[(cs + i) * H + h] = pp[P::DB + i];
-    load_chunk_qkg<DK, Tin, NTH>(q, k, log_alpha, nullptr, cs, Lc, H, h, sQ, sK, sG, nullptr);
+    load_chunk_qkg<DK, Tin, NTH, GS>(q, k, log_alpha, nullptr, cs, Lc, H, h, sQ, sK, sG, nullptr);
 
     // ---- dq = e^G dQh + pair terms of dAqk;  dG = q dq
     {
@@ -1174,7 +1182,18 @@ bwd_chunk_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const flo
         float acc = __expf(gC) * pp[P::DGC + c] + kb_sum;
         for (int i = C - 1; i >= 0; --i) {
             acc += sDg[i * DKP + c];
-            if (i < Lc) dlog_alpha[((cs + i) * H + h) * DK + c] = acc;
+            if constexpr (GS) sDg[i * DKP + c] = acc;
+            else if (i < Lc) dlog_alpha[((cs + i) * H + h) * DK + c] = acc;
+        }
+    }
+    if constexpr (GS) {   // dlog_alpha of the shared rate: the sum over the channels, one warp per row
+        __syncthreads();
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int i = warp; i < Lc; i += NTH / 32) {
+            float x = 0.f;
+            for (int c = lane; c < DK; c += 32) x += sDg[i * DKP + c];
+            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+            if (lane == 0) dlog_alpha[(cs + i) * H + h] = x;
         }
     }
 }

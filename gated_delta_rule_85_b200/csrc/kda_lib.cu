@@ -256,16 +256,16 @@ int set_smem(K kern, size_t bytes, const char *what) {
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, what);
 }
 
-template <int DK, typename Tin>
+template <int DK, typename Tin, bool GS>
 int launch_backward(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                     const float *init_state, const void *d_o, const float *dfinal, void *dq, void *dk_out,
                     void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state, const int32_t *cu_seqlens,
                     long long tokens, int T, int H, int dv, int num_seqs, void *workspace, cudaStream_t st) {
     namespace b = kda::bwd;
-    auto k_prep = b::bwd_prep_kernel<DK, Tin>;
+    auto k_prep = b::bwd_prep_kernel<DK, Tin, GS>;
     auto k_state = b::bwd_state_kernel<DK, Tin>;
     auto k_part = b::bwd_part_kernel<DK, Tin>;
-    auto k_chunk = b::bwd_chunk_kernel<DK, Tin>;
+    auto k_chunk = b::bwd_chunk_kernel<DK, Tin, GS>;
     int rc;
     if ((rc = set_smem(k_prep, b::PrepSmem<DK>::bytes, "cudaFuncSetAttribute(bwd_prep)"))) return rc;
     if ((rc = set_smem(k_state, b::StateSmem<DK>::bytes, "cudaFuncSetAttribute(bwd_state)"))) return rc;
@@ -298,6 +298,50 @@ int launch_backward(const void *q, const void *k, const void *v, const float *lo
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd_chunk launch");
     }
     return KDA_OK;
+}
+
+// Both backward entry points after the shared checks; gate_scalar: Gated DeltaNet.
+int backward_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                  const float *init_state, const void *d_o, const float *dfinal_state, void *dq, void *dk_out,
+                  void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state, const int32_t *cu_seqlens,
+                  int B, int T, int H, int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace,
+                  size_t ws_bytes, void *stream, bool gate_scalar) {
+    // The forward checks cover the inputs (o stands in for d_o).
+    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, cu_seqlens, B, T, H, dk, dv,
+                           num_seqs, dtype, chunk, gate_scalar);
+    if (rc) return rc;
+    if (T > 0 && (!dq || !dk_out || !dv_out || !dlog_alpha || !dbeta))
+        return fail(KDA_ERR_INVALID_ARG, "dq, dk, dv, dlog_alpha and dbeta are required");
+    const void *p16[] = {dq, dk_out, dv_out, gate_scalar ? nullptr : dlog_alpha, dinit_state};
+    const char *n16[] = {"dq", "dk", "dv", "dlog_alpha", "dinit_state"};
+    for (int i = 0; i < 5; ++i)
+        if (p16[i] && !aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
+    if (dbeta && !aligned(dbeta, 4)) return fail(KDA_ERR_MISALIGNED, "dbeta is not 4-byte aligned");
+    if (gate_scalar && dlog_alpha && !aligned(dlog_alpha, 4))
+        return fail(KDA_ERR_MISALIGNED, "dlog_alpha is not 4-byte aligned");
+    const long long tokens = (long long)B * T;
+    const size_t need = kda::bwd::backward_workspace_bytes(tokens, H, dk, dv, num_seqs);
+    if (need > 0 && (!workspace || ws_bytes < need))
+        return fail(KDA_ERR_WORKSPACE, "backward workspace of %zu bytes needed, %zu given%s", need, ws_bytes,
+                    workspace ? "" : " (NULL)");
+    if (workspace && !aligned(workspace, 16)) return fail(KDA_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+    if (kda::bwd::chunk_slots(tokens, num_seqs) > 0x7fffffffLL)
+        return fail(KDA_ERR_UNSUPPORTED, "too many chunk slots for one grid");
+    if (num_seqs == 0) return KDA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+#define KDA_BWD_ARGS                                                                                      \
+    (q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, dlog_alpha, dbeta, dinit_state, \
+     cu_seqlens, tokens, T, H, dv, num_seqs, workspace, st)
+#define KDA_BWD(DKv, TT) \
+    return gate_scalar ? launch_backward<DKv, TT, true> KDA_BWD_ARGS : launch_backward<DKv, TT, false> KDA_BWD_ARGS
+    if (dtype == KDA_BF16) {
+        if (dk == 64) KDA_BWD(64, __nv_bfloat16);
+        KDA_BWD(128, __nv_bfloat16);
+    }
+    if (dk == 64) KDA_BWD(64, float);
+    KDA_BWD(128, float);
+#undef KDA_BWD
+#undef KDA_BWD_ARGS
 }
 
 }  // namespace
@@ -503,38 +547,20 @@ int kda_chunk_backward(const void *q, const void *k, const void *v, const float 
                        float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
                        int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
                        void *stream) {
-    // The forward checks cover the inputs (o stands in for d_o).
-    int rc = check_prefill(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, cu_seqlens, B, T, H, dk, dv,
-                           num_seqs, dtype, chunk);
-    if (rc) return rc;
-    if (T > 0 && (!dq || !dk_out || !dv_out || !dlog_alpha || !dbeta))
-        return fail(KDA_ERR_INVALID_ARG, "dq, dk, dv, dlog_alpha and dbeta are required");
-    const void *p16[] = {dq, dk_out, dv_out, dlog_alpha, dinit_state};
-    const char *n16[] = {"dq", "dk", "dv", "dlog_alpha", "dinit_state"};
-    for (int i = 0; i < 5; ++i)
-        if (p16[i] && !aligned(p16[i], 16)) return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", n16[i]);
-    if (dbeta && !aligned(dbeta, 4)) return fail(KDA_ERR_MISALIGNED, "dbeta is not 4-byte aligned");
-    const long long tokens = (long long)B * T;
-    const size_t need = kda::bwd::backward_workspace_bytes(tokens, H, dk, dv, num_seqs);
-    if (need > 0 && (!workspace || ws_bytes < need))
-        return fail(KDA_ERR_WORKSPACE, "backward workspace of %zu bytes needed, %zu given%s", need, ws_bytes,
-                    workspace ? "" : " (NULL)");
-    if (workspace && !aligned(workspace, 16)) return fail(KDA_ERR_MISALIGNED, "workspace is not 16-byte aligned");
-    if (kda::bwd::chunk_slots(tokens, num_seqs) > 0x7fffffffLL)
-        return fail(KDA_ERR_UNSUPPORTED, "too many chunk slots for one grid");
-    if (num_seqs == 0) return KDA_OK;
-    cudaStream_t st = (cudaStream_t)stream;
-#define KDA_BWD(DKv, TT)                                                                                      \
-    return launch_backward<DKv, TT>(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, \
-                                    dlog_alpha, dbeta, dinit_state, cu_seqlens, tokens, T, H, dv, num_seqs,     \
-                                    workspace, st)
-    if (dtype == KDA_BF16) {
-        if (dk == 64) KDA_BWD(64, __nv_bfloat16);
-        KDA_BWD(128, __nv_bfloat16);
-    }
-    if (dk == 64) KDA_BWD(64, float);
-    KDA_BWD(128, float);
-#undef KDA_BWD
+    return backward_impl(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, dlog_alpha,
+                         dbeta, dinit_state, cu_seqlens, B, T, H, dk, dv, num_seqs, dtype, chunk, workspace, ws_bytes,
+                         stream, false);
+}
+
+int kda_gdn_chunk_backward(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *init_state, const void *d_o,
+                           const float *dfinal_state, void *dq, void *dk_out, void *dv_out, float *dlog_alpha,
+                           float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
+                           int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
+                           void *stream) {
+    return backward_impl(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, dlog_alpha,
+                         dbeta, dinit_state, cu_seqlens, B, T, H, dk, dv, num_seqs, dtype, chunk, workspace, ws_bytes,
+                         stream, true);
 }
 
 int kda_get_device_status(unsigned int *bits, int clear, void *stream) {

@@ -337,6 +337,22 @@ int kda_chunk_backward(const void *q, const void *k, const void *v, const float 
                        int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
                        void *stream);
 
+/*
+ * Backward of the Gated DeltaNet prefill (kda_gdn_chunk_forward): the same
+ * gradients as kda_chunk_backward with the decay rate shared by the key
+ * channels -- log_alpha and dlog_alpha are fp32 [B, T, H] (4-byte aligned), and
+ * dlog_alpha is the sum over the channels of the per-channel gradient (the
+ * gradient of a value broadcast over them).  Everything else, the workspace
+ * (kda_chunk_backward_workspace_size) and the error behaviour are as in
+ * kda_chunk_backward.
+ */
+int kda_gdn_chunk_backward(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *init_state, const void *d_o,
+                           const float *dfinal_state, void *dq, void *dk_out, void *dv_out, float *dlog_alpha,
+                           float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
+                           int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
+                           void *stream);
+
 /* Message for the calling thread's last non-OK return ("" if none). */
 const char *kda_last_error(void);
 
