@@ -252,10 +252,57 @@ __device__ __forceinline__ void warp_mma_strip(float (&d)[TW][4], const float *A
     }
 }
 
+// bf16 operands (m16n8k16, fp32 accumulate): the precision of the forward's
+// tensor-core path, for bf16 inputs on the serial state sweeps.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two fp32 values (p[0], p[stride]) packed as bf16 (first in the low half).
+__device__ __forceinline__ uint32_t pack_bf16x2(const float *p, int stride) {
+    float x0, x1;
+    if (stride == 1) {
+        const float2 v = *reinterpret_cast<const float2 *>(p);
+        x0 = v.x;
+        x1 = v.y;
+    } else {
+        x0 = p[0];
+        x1 = p[stride];
+    }
+    __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// warp_mma_strip with bf16 operands; K a multiple of 16, pairs along k 8-byte
+// aligned when contiguous (even strides and offsets).
+template <int K, int TW>
+__device__ __forceinline__ void warp_mma_strip_bf16(float (&d)[TW][4], const float *A, int ar, int ak, const float *B,
+                                                    int bk, int bn) {
+    static_assert(K % 16 == 0, "K must be a multiple of 16");
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const float *a_lo = A + g * ar + 2 * t * ak, *b_lo = B + 2 * t * bk + g * bn;
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        const float *a = a_lo + k0 * ak;
+        const uint32_t a0 = pack_bf16x2(a, ak), a1 = pack_bf16x2(a + 8 * ar, ak);
+        const uint32_t a2 = pack_bf16x2(a + 8 * ak, ak), a3 = pack_bf16x2(a + 8 * ar + 8 * ak, ak);
+#pragma unroll
+        for (int w = 0; w < TW; ++w) {
+            const float *b = b_lo + k0 * bk + w * 8 * bn;
+            mma_bf16_16816(d[w], a0, a1, a2, a3, pack_bf16x2(b, bk), pack_bf16x2(b + 8 * bk, bk));
+        }
+    }
+}
+
 // Block product out[M x N] = A1 B1 (+ A2 B2): each warp takes a strip of one
 // 16-row block by TW 8-column tiles; every output element goes once through
 // epi(row, col, v).
-template <int M, int N, bool SPLIT, int K1, int K2 = 0, int NTH = NT, typename Epi>
+template <int M, int N, bool SPLIT, int K1, int K2 = 0, int NTH = NT, bool BF = false, typename Epi>
 __device__ __forceinline__ void block_mma(const float *A1, int ar1, int ak1, const float *B1, int bk1, int bn1,
                                           const float *A2, int ar2, int ak2, const float *B2, int bk2, int bn2,
                                           Epi &&epi) {
@@ -269,8 +316,13 @@ __device__ __forceinline__ void block_mma(const float *A1, int ar1, int ak1, con
         float d[TW][4];
 #pragma unroll
         for (int w = 0; w < TW; ++w) d[w][0] = d[w][1] = d[w][2] = d[w][3] = 0.f;
-        warp_mma_strip<SPLIT, K1, TW>(d, A1 + r0 * ar1, ar1, ak1, B1 + c0 * bn1, bk1, bn1);
-        if constexpr (K2 > 0) warp_mma_strip<SPLIT, K2, TW>(d, A2 + r0 * ar2, ar2, ak2, B2 + c0 * bn2, bk2, bn2);
+        if constexpr (BF) {
+            warp_mma_strip_bf16<K1, TW>(d, A1 + r0 * ar1, ar1, ak1, B1 + c0 * bn1, bk1, bn1);
+            if constexpr (K2 > 0) warp_mma_strip_bf16<K2, TW>(d, A2 + r0 * ar2, ar2, ak2, B2 + c0 * bn2, bk2, bn2);
+        } else {
+            warp_mma_strip<SPLIT, K1, TW>(d, A1 + r0 * ar1, ar1, ak1, B1 + c0 * bn1, bk1, bn1);
+            if constexpr (K2 > 0) warp_mma_strip<SPLIT, K2, TW>(d, A2 + r0 * ar2, ar2, ak2, B2 + c0 * bn2, bk2, bn2);
+        }
 #pragma unroll
         for (int w = 0; w < TW; ++w) warp_tile_out(d[w], r0, c0 + 8 * w, epi);
     }
@@ -608,6 +660,7 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
     using R = Rec<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
+    constexpr bool BF = sizeof(Tin) == 2;   // bf16 inputs: bf16 operands, as the forward's tensor-core path
     extern __shared__ __align__(128) float sm[];
     float *sKh = sm + L::kh, *sQh = sm + L::qh, *sKt = sm + L::kt, *sPt = sm + L::pt;
     float *sS = sm + L::s, *sX = sm + L::x, *sY = sm + L::y, *sD = sm + L::d;
@@ -722,10 +775,10 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
         pend_a = false;
         if (!(ok = wait_copies(bar_a, ph_a))) break;   // group A of this chunk
         if (!backward)
-            block_mma<C, SV, SPLIT, DK>(sKh, DKP, 1, sS, SVP, 1, nullptr, 0, 0, nullptr, 0, 0,
+            block_mma<C, SV, SPLIT, DK, 0, NT, BF>(sKh, DKP, 1, sS, SVP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                     [&](int i, int j, float x) { sY[i * SVP + j] = sX[i * SVP + j] - x; });
         else
-            block_mma<C, SV, SPLIT, C, DK>(sPt, 1, CP, sX, SVP, 1, sKt, 1, CP, sS, SVP, 1,
+            block_mma<C, SV, SPLIT, C, DK, NT, BF>(sPt, 1, CP, sX, SVP, 1, sKt, 1, CP, sS, SVP, 1,
                                     [&](int i, int j, float x) { sY[i * SVP + j] = -x; });
         __syncthreads();   // group A's buffers are free
         issue_a(step + 1);
@@ -733,10 +786,10 @@ bwd_state_kernel(const Tin *__restrict__ v, const float *__restrict__ init_state
         pend_b = false;
         if (!(ok = wait_copies(bar_b, ph_b))) break;   // group B of this chunk
         if (!backward)
-            block_mma<DK, SV, SPLIT, C>(sKt, CP, 1, sY, SVP, 1, nullptr, 0, 0, nullptr, 0, 0,
+            block_mma<DK, SV, SPLIT, C, 0, NT, BF>(sKt, CP, 1, sY, SVP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                      [&](int c, int j, float x) { sS[c * SVP + j] = sD[c] * sS[c * SVP + j] + x; });
         else
-            block_mma<DK, SV, SPLIT, C, C>(sQh, 1, DKP, sX, SVP, 1, sKh, 1, DKP, sY, SVP, 1,
+            block_mma<DK, SV, SPLIT, C, C, NT, BF>(sQh, 1, DKP, sX, SVP, 1, sKh, 1, DKP, sY, SVP, 1,
                                      [&](int c, int j, float x) { sS[c * SVP + j] = sD[c] * sS[c * SVP + j] + x; });
         __syncthreads();   // group B's buffers are free
         issue_b(step + 1);
@@ -790,6 +843,7 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
     using P = Part<DK>;
     constexpr int DKP = L::DKP;
     constexpr bool SPLIT = sizeof(Tin) == 4;
+    constexpr bool BF = sizeof(Tin) == 2;   // bf16 inputs: bf16 operands
     constexpr int NTH = PartThreads<Tin>::value, NW = NTH / 32;
     // Column sums accumulate in registers across the value tiles: each warp owns a
     // strip of one 16-row block by TQ (TA) adjacent 8-column tiles of the [C][DK]
@@ -871,19 +925,19 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         }
         __syncthreads();
         // W = V - Kh S (in place: each element is read and written by its owner only)
-        block_mma<C, DVT, SPLIT, DK, 0, NTH>(sKh, DKP, 1, sS, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<C, DVT, SPLIT, DK, 0, NTH, BF>(sKh, DKP, 1, sS, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sW[i * TP + j] -= x; });
         __syncthreads();
         // U = Tb W;  dU = Aqk^T dO + Kb dS
-        block_mma<C, DVT, SPLIT, C, 0, NTH>(sTb, CP, 1, sW, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<C, DVT, SPLIT, C, 0, NTH, BF>(sTb, CP, 1, sW, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sU[i * TP + j] = x; });
-        block_mma<C, DVT, SPLIT, C, DK, NTH>(sAqk, 1, CP, sDO, TP, 1, sKb, DKP, 1, sdS, TP, 1,
+        block_mma<C, DVT, SPLIT, C, DK, NTH, BF>(sAqk, 1, CP, sDO, TP, 1, sKb, DKP, 1, sdS, TP, 1,
                                  [&](int i, int j, float x) { sdU[i * TP + j] = x; });
         __syncthreads();
         // R = W - Akk U (in place of W);  lam = T^T dU
-        block_mma<C, DVT, SPLIT, C, 0, NTH>(sAkk, CP, 1, sU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<C, DVT, SPLIT, C, 0, NTH, BF>(sAkk, CP, 1, sU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sW[i * TP + j] -= x; });
-        block_mma<C, DVT, SPLIT, C, 0, NTH>(sT, 1, CP, sdU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
+        block_mma<C, DVT, SPLIT, C, 0, NTH, BF>(sT, 1, CP, sdU, TP, 1, nullptr, 0, 0, nullptr, 0, 0,
                                  [&](int i, int j, float x) { sL[i * TP + j] = x; });
         __syncthreads();
         // dbeta: <lam_i, R_i> (one warp per 8 rows; the same lane adds every tile)
@@ -906,11 +960,19 @@ bwd_part_kernel(const Tin *__restrict__ v, const float *__restrict__ beta, const
         __syncthreads();
         // sums over this tile's columns, kept in registers across tiles:
         // dO S^T, mu S^T, U dS^T ([C][DK]) and dO U^T, mu U^T ([C][C])
-        warp_mma_strip<SPLIT, DVT, TQ>(a_dq, sDO + q_r0 * TP, TP, 1, sS + q_c0 * TP, 1, TP);
-        warp_mma_strip<SPLIT, DVT, TQ>(a_dkh, sL + q_r0 * TP, TP, 1, sS + q_c0 * TP, 1, TP);
-        warp_mma_strip<SPLIT, DVT, TQ>(a_dkb, sU + q_r0 * TP, TP, 1, sdS + q_c0 * TP, 1, TP);
-        warp_mma_strip<SPLIT, DVT, TA>(a_aq, sDO + a_r0 * TP, TP, 1, sU + a_c0 * TP, 1, TP);
-        warp_mma_strip<SPLIT, DVT, TA>(a_ak, sL + a_r0 * TP, TP, 1, sU + a_c0 * TP, 1, TP);
+        if constexpr (BF) {
+            warp_mma_strip_bf16<DVT, TQ>(a_dq, sDO + q_r0 * TP, TP, 1, sS + q_c0 * TP, 1, TP);
+            warp_mma_strip_bf16<DVT, TQ>(a_dkh, sL + q_r0 * TP, TP, 1, sS + q_c0 * TP, 1, TP);
+            warp_mma_strip_bf16<DVT, TQ>(a_dkb, sU + q_r0 * TP, TP, 1, sdS + q_c0 * TP, 1, TP);
+            warp_mma_strip_bf16<DVT, TA>(a_aq, sDO + a_r0 * TP, TP, 1, sU + a_c0 * TP, 1, TP);
+            warp_mma_strip_bf16<DVT, TA>(a_ak, sL + a_r0 * TP, TP, 1, sU + a_c0 * TP, 1, TP);
+        } else {
+            warp_mma_strip<SPLIT, DVT, TQ>(a_dq, sDO + q_r0 * TP, TP, 1, sS + q_c0 * TP, 1, TP);
+            warp_mma_strip<SPLIT, DVT, TQ>(a_dkh, sL + q_r0 * TP, TP, 1, sS + q_c0 * TP, 1, TP);
+            warp_mma_strip<SPLIT, DVT, TQ>(a_dkb, sU + q_r0 * TP, TP, 1, sdS + q_c0 * TP, 1, TP);
+            warp_mma_strip<SPLIT, DVT, TA>(a_aq, sDO + a_r0 * TP, TP, 1, sU + a_c0 * TP, 1, TP);
+            warp_mma_strip<SPLIT, DVT, TA>(a_ak, sL + a_r0 * TP, TP, 1, sU + a_c0 * TP, 1, TP);
+        }
         if (tid < DK)
             for (int j = 0; j < DVT; ++j) a_gc = fmaf(sS[tid * TP + j], sdS[tid * TP + j], a_gc);
     }

@@ -202,3 +202,29 @@ def test_gdn_backward_matches_oracle(dtype, packed):
     torch.testing.assert_close(got["dlog_alpha"], full["dlog_alpha"].sum(-1), rtol=1e-4, atol=1e-4)
     for name in ("dq", "dk", "dv", "dbeta", "dinit_state"):
         assert torch.equal(got[name], full[name]), name
+
+
+@pytest.mark.parametrize("split", [128, 100])
+def test_backward_split_resume_chain_rule(split):
+    """Split a sequence at token `split`: the second part starts from the state the
+    forward reaches there, and its dL/dinit_state is the first part's dfinal.  The
+    gradients of the two parts together equal one call (the state hand-off of the
+    chain rule), fp32."""
+    shape = PrefillShape(B=1, T=300, H=2, dk=64, dv=64, dtype=torch.float32)
+    d = prefill_inputs(shape, 55, DEV)
+    c = backward_cotangents(shape, 56, DEV)
+    whole = run(d, c)
+    cut = lambda x, a, b: x[:, a:b].contiguous()
+    first = {x: cut(d[x], 0, split) for x in ("q", "k", "v", "log_alpha", "beta")}
+    first["init_state"] = d["init_state"]
+    second = {x: cut(d[x], split, 300) for x in ("q", "k", "v", "log_alpha", "beta")}
+    _, S_mid = kda.chunk_forward(*(first[x] for x in ("q", "k", "v", "log_alpha", "beta")), first["init_state"],
+                                 simt=True)
+    second["init_state"] = S_mid
+    g2 = run(second, {"d_o": cut(c["d_o"], split, 300), "dfinal_state": c["dfinal_state"]})
+    g1 = run(first, {"d_o": cut(c["d_o"], 0, split), "dfinal_state": g2["dinit_state"]})
+    torch.cuda.synchronize()
+    for name in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+        both = torch.cat([g1[name], g2[name]], dim=1)
+        torch.testing.assert_close(both, whole[name], rtol=1e-4, atol=1e-5, msg=name)
+    torch.testing.assert_close(g1["dinit_state"], whole["dinit_state"], rtol=1e-4, atol=1e-5)
