@@ -157,25 +157,36 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         float al[SEGLEN][4];
         uint2 qv[SEGLEN], kv[SEGLEN];
         float4 sg = make_float4(0.f, 0.f, 0.f, 0.f);
+        // all loads first, unconditionally (rows past Lc read the last valid row
+        // and are zeroed afterwards), so every one is in flight before any is used
+        float4 gv[SEGLEN];
 #pragma unroll
         for (int u = 0; u < SEGLEN; ++u) {
-            float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            qv[u] = make_uint2(0u, 0u);
-            kv[u] = make_uint2(0u, 0u);
-            if (i0 + u < Lc) {
-                const long long off = ((cs + i0 + u) * H + h) * DK + c0;
-                if constexpr (GS) {
-                    const float gs = __ldg(log_alpha + (cs + i0 + u) * H + h);
-                    g4 = make_float4(gs, gs, gs, gs);
-                } else if constexpr (PRO) {
-                    const float4 x4 = bf16x4_to_float4(
-                        __ldcs(reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(log_alpha) + off)));
-                    g4 = make_float4(neg_softplus(x4.x), neg_softplus(x4.y), neg_softplus(x4.z), neg_softplus(x4.w));
-                } else {
-                    g4 = __ldcs(reinterpret_cast<const float4 *>(log_alpha + off));
-                }
-                qv[u] = __ldcs(reinterpret_cast<const uint2 *>(q + off));
-                kv[u] = __ldcs(reinterpret_cast<const uint2 *>(k + off));
+            const long long row = cs + min(i0 + u, Lc - 1);
+            const long long off = (row * H + h) * DK + c0;
+            if constexpr (GS) {
+                const float gs = __ldg(log_alpha + row * H + h);
+                gv[u] = make_float4(gs, gs, gs, gs);
+            } else if constexpr (PRO) {
+                const uint2 xr = __ldcs(reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(log_alpha) + off));
+                gv[u] = make_float4(__uint_as_float(xr.x), __uint_as_float(xr.y), 0.f, 0.f);   // raw bf16 pairs
+            } else {
+                gv[u] = __ldcs(reinterpret_cast<const float4 *>(log_alpha + off));
+            }
+            qv[u] = __ldcs(reinterpret_cast<const uint2 *>(q + off));
+            kv[u] = __ldcs(reinterpret_cast<const uint2 *>(k + off));
+        }
+#pragma unroll
+        for (int u = 0; u < SEGLEN; ++u) {
+            float4 g4 = gv[u];
+            if constexpr (PRO) {
+                const float4 x4 = bf16x4_to_float4(make_uint2(__float_as_uint(g4.x), __float_as_uint(g4.y)));
+                g4 = make_float4(neg_softplus(x4.x), neg_softplus(x4.y), neg_softplus(x4.z), neg_softplus(x4.w));
+            }
+            if (i0 + u >= Lc) {
+                g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                qv[u] = make_uint2(0u, 0u);
+                kv[u] = make_uint2(0u, 0u);
             }
             sg.x += g4.x; sg.y += g4.y; sg.z += g4.z; sg.w += g4.w;
             al[u][0] = g4.x; al[u][1] = g4.y; al[u][2] = g4.z; al[u][3] = g4.w;
