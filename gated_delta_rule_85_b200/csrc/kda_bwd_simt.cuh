@@ -1,4 +1,5 @@
-// KDA chunked backward on CUDA cores, fp32 throughout.
+// KDA chunked backward: tensor-core products (warp-level mma.sync) with fp32
+// accumulation, the rest fp32 on CUDA cores.
 //
 // Gradients of L = sum_t <do_t, o_t> + <dS_T, S_T> for the recurrence of
 // "Kimi Delta Attention 徹底解説" (tech-tide.dev), § "Kimi Delta Attention の仕組み",
@@ -12,11 +13,11 @@
 //   Aqk[i][j] = sum_c q_ic k_jc e^{G_ic - G_jc}  (j <= i)
 //   Qh = e^G q, Kh = e^G k, Kb = e^{G_C - G} k, D = e^{G_C}
 //   W = V - Kh S;  U_i = beta_i R_i,  R_i = W_i - sum_{j<i} Akk[i][j] U_j
-//     (so U = Tb W with Tb = (I + Diag(beta) Akk)^{-1} Diag(beta))
+//     (so U = Tb W with T = (I + Diag(beta) Akk)^{-1}, Tb = T Diag(beta))
 //   O = Qh S + Aqk U;  S_next = Diag(D) S + Kb^T U = Diag(D) S + Kt W,  Kt = Kb^T Tb
 // Backward of the chunk, given dO and dS (the adjoint of S_next):
 //   dU = Aqk^T dO + Kb dS
-//   lam: (I + Diag(beta) Akk)^T lam = dU   (back substitution)
+//   lam = T^T dU   (the adjoint of the forward substitution)
 //   mu = beta lam = Pt^T dO + Kt^T dS,  Pt = Aqk Tb
 //   dV = mu;  dbeta_i = <lam_i, R_i>
 //   dAkk[i][j] = -<mu_i, U_j> (j < i);  dAqk[i][j] = <dO_i, U_j> (j <= i)
@@ -27,13 +28,13 @@
 //   dq_i = e^{G_i} dQh_i + sum_{j<=i} dAqk[i][j] k_j E_ij
 //   dk_i = a_i + b_i + sum_{j<i} dAkk[i][j] k_j E_ij
 //          + sum_{m>=i} (dAqk[m][i] q_m + [m>i] dAkk[m][i] k_m) E_mi
-//   dG_i = q_i (dq_i) + k_i (a_i - b_i + row Akk terms) - k_i (column terms of dk_i)
+//   dG_i = q_i dq_i + k_i (a_i - b_i + the Akk row terms) - k_i (the column terms of dk_i)
 //   dG_C += D sum_j S[:, j] dS[:, j] + sum_i k_i b_i;   dlog_alpha_s = sum_{i>=s} dG_i
 //
 // Kernels, in launch order:
 //   bwd_prep_kernel   one CTA per (chunk slot, head): G, Akk, Aqk, the decay
 //                     factors, T, Tb, Kt and Pt, written as a record.
-//   bwd_state_kernel  one CTA per (direction, 32-column value tile, head,
+//   bwd_state_kernel  one CTA per (direction, 64-column value tile, head,
 //                     sequence): the only serial work.  Forward it stores the
 //                     state at every chunk start (S <- Diag(D) S + Kt (V - Kh S));
 //                     backward the adjoint at every chunk end
@@ -41,13 +42,14 @@
 //   bwd_part_kernel   one CTA per (chunk slot, head): everything column-separable
 //                     (U = Tb W, R = W - Akk U, lam = T^T dU, mu, dV, and the sums
 //                     over the value columns of dQh, dKh, dKb, dAqk, dAkk, dbeta,
-//                     S.dS), value tile by tile.
-// The dense products run on the tensor cores as warp-level m16n8k8 tf32 MMAs
-// with fp32 accumulation; for fp32 inputs each operand is split into a tf32
-// high part and a tf32 remainder and three products are summed (hi.hi + hi.lo
-// + lo.hi), which keeps fp32 accuracy.  Everything else is fp32 on CUDA cores.
+//                     S.dS), 32-column value tile by tile.
 //   bwd_chunk_kernel  one CTA per (chunk slot, head): the chain rule through the
 //                     decay factors; writes dq, dk, dlog_alpha, dbeta.
+// Operand precision: fp32 inputs use m16n8k8 tf32 MMAs with each operand split
+// into a tf32 high part and remainder, three products summed (hi.hi + hi.lo +
+// lo.hi), which keeps fp32 accuracy; bf16 inputs use bf16 m16n8k16 MMAs on the
+// state sweeps and column sums (the precision of the forward's tensor-core path)
+// and tf32 for the record.  Accumulation is fp32 everywhere.
 // Chunk slots as in the two-pass forward: chunk c of sequence n (tokens
 // [t0, t1)) is slot n + floor(t0 / 64) + c.
 #pragma once
@@ -384,8 +386,6 @@ __device__ __forceinline__ void cp_async16(float *dst, const float *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Waits until at most one committed group (the most recent) is still in flight.
-__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // rows x cols fp32 (cols a multiple of 4; source rows src_ld apart, default

@@ -301,8 +301,12 @@ int kda_recurrent_step_prologue(const void *q_raw, const void *k_raw, const void
  * training algorithm needs ("Kimi Linear、独自の土俵でFull Attentionを上回る"
  * (remio.ai), § "Kimi Linearがより賢いRecurrent Memoryを使う方法"), for the
  * recurrence of "Kimi Delta Attention 徹底解説" (tech-tide.dev),
- * § "Kimi Delta Attention の仕組み".  fp32 arithmetic on CUDA cores with the
- * exact pairwise decay (no range precondition), for dtype KDA_BF16 and KDA_F32.
+ * § "Kimi Delta Attention の仕組み".  Tensor-core products with fp32
+ * accumulation (split tf32 for KDA_F32, keeping fp32 accuracy; bf16 and tf32
+ * operands for KDA_BF16), and no decay-range precondition: decay factors pass
+ * through 16-token block boundaries with both factors <= 1, and within a block
+ * take the exact pairwise exponent unless every channel's in-block decay is
+ * small enough to factor too.  For dtype KDA_BF16 and KDA_F32.
  *
  *   q, k, v, log_alpha, beta, init_state, cu_seqlens, B, T, H, dk, dv,
  *   num_seqs, dtype, chunk

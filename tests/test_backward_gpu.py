@@ -3,8 +3,9 @@ reverse-mode gradients of the token recurrence, on the same inputs.
 
 The loss is L = sum <d_o, o> + <dfinal_state, final_state> with seeded
 cotangents; every gradient (dq, dk, dv, dlog_alpha, dbeta, dinit_state) is
-compared element by element.  The backward computes in fp32 from the exact
-input values, so the operator's bounds apply: rel-L2 <= 1e-4 for fp32 inputs;
+compared element by element.  The backward accumulates in fp32 with the
+forward's operand precision (split tf32 for fp32 inputs, bf16/tf32 operands for
+bf16 inputs), so the operator's bounds apply: rel-L2 <= 1e-4 for fp32 inputs;
 for bf16 inputs rel-L2 <= 1e-2 and max-abs <= 5e-2 relative to the largest
 reference magnitude (gradients are not O(1) quantities like o and S).
 """
