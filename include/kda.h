@@ -325,7 +325,11 @@ int kda_recurrent_step_prologue(const void *q_raw, const void *k_raw, const void
  *                 state at the chunk's start (4 dk dv bytes) and the partial
  *                 sums of every 32-column value tile (about 132 KB per tile at
  *                 dk = 128).  Calls that can overlap in time need separate
- *                 workspaces.
+ *                 workspaces.  About 570 KB per (chunk, head) at dk = dv = 128
+ *                 (2 GB for 8192 tokens x 32 heads): a long input is taken in
+ *                 pieces from its end, each piece's dinit_state passed as the
+ *                 previous piece's dfinal_state and its init_state the forward
+ *                 state at the piece's start -- exact by the chain rule.
  * The caller owns every buffer; all pointers except cu_seqlens and beta are
  * 16-byte aligned.  Every gradient is overwritten, not accumulated; tokens
  * outside every sequence (packed input with cu_seqlens[N] < T) are not written.
