@@ -22,7 +22,7 @@ in token slices of fixed size so device memory for temporaries stays bounded.
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 
 import numpy as np
 import torch

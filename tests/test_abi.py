@@ -1,7 +1,6 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads, exports every
 function include/kda.h declares, and rejects bad arguments before enqueuing work.
 Every call below breaks exactly one rule that is checked before any launch."""
-import ctypes
 import os
 import re
 

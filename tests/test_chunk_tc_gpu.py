@@ -2,7 +2,6 @@
 under both schedules (fused; two-pass with workspace).
 
 Bound for bf16 inputs: rel-L2 <= 1e-2 and max-abs <= 5e-2 on o and the final state."""
-import numpy as np
 import pytest
 import torch
 
