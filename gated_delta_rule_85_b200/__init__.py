@@ -25,7 +25,7 @@ __all__ = [
     "chunk_forward", "chunk_backward", "gdn_chunk_backward", "backward_workspace_size", "chunk_forward_prologue",
     "recurrent_step_prologue", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
     "recurrent_step_slots", "gdn_chunk_forward", "gdn_recurrent_step", "workspace_size", "device_status",
-    "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
+    "debug_wait_timeout", "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
     "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "DEV_BAD_SLOT", "ALGOS",
 ]
 
@@ -102,6 +102,8 @@ def load_library():
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci, vp]
     lib.kda_get_device_status.restype = ci
+    lib.kda_debug_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+    lib.kda_debug_wait_timeout.restype = ci
     lib.kda_api_version.argtypes = []
     lib.kda_api_version.restype = ci
     _lib = lib
@@ -471,6 +473,13 @@ def gdn_recurrent_step(q, k, v, log_alpha, beta, state, o=None):
                                                N, H, dk, dv, _dtype_code(q), _stream(q.device))
     _check(rc)
     return o
+
+
+def debug_wait_timeout(limit_cycles: int = 2_000_000) -> None:
+    """Test hook: one CTA waits (bounded by `limit_cycles` SM cycles) on an mbarrier
+    nothing completes, so the device status word gets DEV_WAIT_TIMEOUT; asynchronous
+    on the current stream of the current device."""
+    _check(load_library().kda_debug_wait_timeout(int(limit_cycles), _stream(torch.cuda.current_device())))
 
 
 def device_status(clear: bool = True) -> int:

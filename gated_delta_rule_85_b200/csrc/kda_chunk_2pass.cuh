@@ -374,7 +374,10 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             for (int gq = 0; gq < 4; ++gq) st_global_bf16x8(kp + sw128_chunk(row, half * 4 + gq), x + gq * 8);
         }
     }
-    if (tid == 0) ptx::bulk_wait_all();
+    if (tid == 0) {
+        if (!ok) ptx::mbar_wait_bounded(bar_mma, ph_mma ^ 1u, WAIT_LIMIT_CYCLES);   // MMAs still in flight
+        ptx::bulk_wait_all();
+    }
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -452,9 +455,11 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     uint32_t ph_mma = 0, ph_rec = 0;   // ph_rec: one parity bit per buffer
+    int n_issued = 0, n_commit = 0;    // thread 0: chunks whose copies were issued, MMA commits
 
     auto issue = [&](int ci) {   // thread 0: record and V tile of chunk ci into buffer ci % NBUF
         const int b = ci % NBUF;
+        n_issued = ci + 1;
         const uint32_t bar = bar_rec + 8 * b;
         ptx::mbar_arrive_expect_tx(bar, TX);
         ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * R::BYTES, (uint32_t)R::BYTES, bar);
@@ -505,6 +510,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
             for (int s = 0; s < DK / 16; ++s)
                 ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KQ, s, 128), kdesc(sb + L::SP, s, DVT), ix, s > 0);
             ptx::mma_commit(bar_mma);
+            ++n_commit;
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
 
@@ -543,6 +549,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
             for (int s = 0; s < 4; ++s)
                 ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KP, s, DK + 64, DK - 64), kdesc(sb + L::ZT, s, DVT), iz, 1);
             ptx::mma_commit(bar_mma);
+            ++n_commit;
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
         if (tid == 0 && ci + NBUF < nck) issue(ci + NBUF);   // buffer b fully consumed
@@ -578,6 +585,13 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
         ptx::tc_fence_before();
     }
 
+    if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded), then leave
+        for (int b = 0; b < NBUF; ++b) {
+            const int arms = n_issued > b ? (n_issued - 1 - b) / NBUF + 1 : 0;   // loads into buffer b
+            if (arms > 0) ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((arms - 1) & 1), WAIT_LIMIT_CYCLES);
+        }
+        if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
+    }
     __syncthreads();
     if (ok && final_state && has_row && row >= 0) {
 #pragma unroll

@@ -333,9 +333,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);   // this warp's TMEM lane quadrant
     uint32_t ph_mma = 0, ph_in = 0, ph_v = 0;
+    int n_in = 0, n_v = 0, n_commit = 0;   // thread 0: arms of bar_in, bar_v and MMA commits
 
     auto issue_inputs = [&](int ci) {   // thread 0 only
         const int z = (int)(t0 + (long long)ci * C);
+        ++n_in;
         ptx::mbar_arrive_expect_tx(bar_in, (uint32_t)(GS ? L::IN_BYTES / 2 : L::IN_BYTES));
         ptx::tma_load_3d(sb + L::QIN, &tm_q, bar_in, 0, h, z);
         ptx::tma_load_3d(sb + L::KIN, &tm_k, bar_in, 0, h, z);
@@ -343,6 +345,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
     auto issue_v = [&](int ci) {        // thread 0 only
         const int z = (int)(t0 + (long long)ci * C);
+        ++n_v;
         ptx::mbar_arrive_expect_tx(bar_v, (uint32_t)(C * DVT * 2));
         ptx::tma_load_3d(sb + L::VIN, &tm_v, bar_v, col_base, h, z);
     };
@@ -479,6 +482,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int s = 0; s < DK / 16; ++s)
                 ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KS, s, L::KSR), ig, s > 0);
             ptx::mma_commit(bar_mma);
+            ++n_commit;
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
 
@@ -559,7 +563,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         ph_v ^= 1u;
         __syncthreads();
-        if (tid == 0 && ci + 1 < nck) issue_v(ci + 1);   // V tile consumed
+        if (tid == 0 && ci + 1 < nck && !*fail_flag) issue_v(ci + 1);   // V tile consumed
         invert_merge_blocks(fA, fT, fM, sm + L::TB, fB + buf * C, warp, lane);
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
@@ -580,6 +584,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ptx::mma_bf16(tmem + COL_PT, kdesc(sb + L::KP, s, DK + 64, DK - 64), kdesc(sb + L::TB, s, 64), ipt,
                               s > 0);
             ptx::mma_commit(bar_mma);
+            ++n_commit;
         }
         if (!(ok = wait_all(bar_mma, ph_mma, *fail_flag))) break;
 
@@ -619,6 +624,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int s = 0; s < 4; ++s)
                 ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KP, s, DK + 64, DK - 64), kdesc(sb + L::ZT, s, DVT), iz, 1);
             ptx::mma_commit(bar_mma);
+            ++n_commit;
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
 
@@ -654,6 +660,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_before();
     }
 
+    if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded), then leave
+        if (n_in > 0) ptx::mbar_wait_bounded(bar_in, (uint32_t)((n_in - 1) & 1), WAIT_LIMIT_CYCLES);
+        if (n_v > 0) ptx::mbar_wait_bounded(bar_v, (uint32_t)((n_v - 1) & 1), WAIT_LIMIT_CYCLES);
+        if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
+    }
     __syncthreads();
     if (ok && final_state && has_row && row >= 0) {
 #pragma unroll

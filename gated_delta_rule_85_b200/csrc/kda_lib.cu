@@ -346,6 +346,22 @@ int backward_impl(const void *q, const void *k, const void *v, const float *log_
 
 }  // namespace
 
+namespace kda {
+// An mbarrier that expects one arrival nobody makes: every thread's bounded wait
+// runs out after limit_cycles and the CTA flags the timeout like a real kernel.
+__global__ void wait_timeout_kernel(long long limit_cycles) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t addr = ptx::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(addr, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    const bool ok = ptx::mbar_wait_bounded(addr, 0u, limit_cycles);
+    if (__syncthreads_or(!ok) && threadIdx.x == 0) flag_status(KDA_DEV_WAIT_TIMEOUT);
+}
+}  // namespace kda
+
 extern "C" {
 
 int kda_api_version(void) { return KDA_API_VERSION; }
@@ -561,6 +577,15 @@ int kda_gdn_chunk_backward(const void *q, const void *k, const void *v, const fl
     return backward_impl(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, dlog_alpha,
                          dbeta, dinit_state, cu_seqlens, B, T, H, dk, dv, num_seqs, dtype, chunk, workspace, ws_bytes,
                          stream, true);
+}
+
+int kda_debug_wait_timeout(long long limit_cycles, void *stream) {
+    if (limit_cycles < 1 || limit_cycles > 2000000000ll)
+        return fail(KDA_ERR_INVALID_ARG, "limit_cycles must lie in [1, 2e9], got %lld", limit_cycles);
+    kda::wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_cycles);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "wait_timeout_kernel launch");
+    return KDA_OK;
 }
 
 int kda_get_device_status(unsigned int *bits, int clear, void *stream) {

@@ -372,6 +372,18 @@ const char *kda_last_error(void);
  */
 int kda_get_device_status(unsigned int *bits, int clear, void *stream);
 
+/*
+ * Test hook for the bounded waits every tensor-core kernel uses.  Launches one
+ * 32-thread CTA on `stream` that waits on a shared-memory mbarrier which no copy
+ * or arrival will ever complete, giving up after `limit_cycles` SM clock cycles
+ * (1 .. 2e9; 2e6 is about a millisecond); the wait runs out, the CTA flags
+ * KDA_DEV_WAIT_TIMEOUT in the status word and returns, and the context stays
+ * usable.  Returns KDA_OK once launched (read the flag with
+ * kda_get_device_status), KDA_ERR_INVALID_ARG for a limit outside the range,
+ * KDA_ERR_CUDA for a launch failure.
+ */
+int kda_debug_wait_timeout(long long limit_cycles, void *stream);
+
 /* KDA_API_VERSION of the loaded library. */
 int kda_api_version(void);
 

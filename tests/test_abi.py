@@ -226,3 +226,8 @@ def test_prologue_entry_points_reject(lib):
                                                        128, 128, 0, None)
     assert step(x=None) == INVALID
     assert step(x=A[3] + 4) == MISALIGNED
+
+
+def test_wait_timeout_hook_rejects_limits(lib):
+    assert lib.kda_debug_wait_timeout(0, None) == INVALID
+    assert lib.kda_debug_wait_timeout(3_000_000_000, None) == INVALID
