@@ -53,7 +53,7 @@ PROLOGUE_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 2 * 128 + 4 + 2 * 128             
 # without a capture on its workload reports null.
 NCU_TRAFFIC = {
     ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.8e6 + 181.5e6 + 308.3e6 + 50.5e6,
-    ("prefill_8k", "chunk_tc_kernel"): 339.1e6 + 56.5e6,
+    # chunk_tc_kernel (--algo fused): captured before its timeout-path change, so reported null
     ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.2e6,
     # backward: all four kernels of one call; T=2048 captured, T=8192 scaled by the chunk slots (129 / 33)
     ("backward_T2048", "bwd"): 795.0e6 + 428.8e6,
