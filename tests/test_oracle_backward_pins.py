@@ -209,3 +209,27 @@ def test_no_init_state_means_zero_state():
         assert np.array_equal(a[gname], b[gname])
     with pytest.raises(ValueError):
         oracle.backward(*args[:5], do[:, :3])
+
+
+def test_scalar_gate_gradient_is_the_channel_sum():
+    """Gated DeltaNet reading: one decay rate per token-head, applied to every key
+    channel.  The gradient of such a rate is the sum over the channels of the
+    per-channel gradients; checked against central differences that move all
+    channels of one (token, head) together."""
+    rng = np.random.default_rng(17)
+    x, do, dF = _case(rng, B=1, T=9, H=2, dk=4, dv=3)
+    g = -np.log1p(np.exp(rng.normal(-2.0, 1.0, size=(1, 9, 2))))
+    x["log_alpha"] = np.repeat(g[..., None], 4, axis=-1)
+    gr = oracle.backward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], do,
+                         init_state=x["init_state"], dfinal=dF)
+    d_scalar = gr["dlog_alpha"].sum(axis=-1)
+    eps = 1e-6
+    for t in range(9):
+        for h in range(2):
+            xp, xm = dict(x), dict(x)
+            xp["log_alpha"] = x["log_alpha"].copy()
+            xm["log_alpha"] = x["log_alpha"].copy()
+            xp["log_alpha"][0, t, h, :] += eps
+            xm["log_alpha"][0, t, h, :] -= eps
+            want = (_loss(oracle.forward, xp, do, dF) - _loss(oracle.forward, xm, do, dF)) / (2 * eps)
+            assert abs(d_scalar[0, t, h] - want) <= 1e-7 * (1.0 + abs(want)), (t, h, d_scalar[0, t, h], want)
