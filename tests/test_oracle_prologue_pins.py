@@ -53,3 +53,14 @@ def test_prologue_then_forward_equals_forward_on_prepared_inputs():
                             k / np.linalg.norm(k, axis=-1, keepdims=True), v, -np.log1p(np.exp(x)), b)
     np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(s1, s2, rtol=1e-12, atol=1e-13)
+
+
+def test_rows_shorter_than_eps_are_divided_by_eps():
+    """The floor of the divisor: a row of norm 1e-8 is divided by eps = 1e-6, so it
+    keeps its direction with norm 1e-2 instead of being blown up to a unit vector."""
+    q = np.zeros((1, 1, 1, 4))
+    q[0, 0, 0] = [6e-9, 0.0, -8e-9, 0.0]
+    qn, _, _ = oracle.prologue(q, q, np.zeros_like(q))
+    np.testing.assert_allclose(qn[0, 0, 0], [6e-3, 0.0, -8e-3, 0.0], rtol=1e-12, atol=0)
+    qn2, _, _ = oracle.prologue(q, q, np.zeros_like(q), eps=1e-9)
+    np.testing.assert_allclose(qn2[0, 0, 0], [0.6, 0.0, -0.8, 0.0], rtol=1e-12, atol=0)
