@@ -48,9 +48,9 @@ BACKWARD_BYTES_PER_TOKEN_HEAD = 4 * 2 * 128 + 4 * 128 + 4 + 3 * 2 * 128 + 4 * 12
 BACKWARD_FLOPS_PER_TOKEN_HEAD = 2 * PREFILL_FLOPS_PER_TOKEN_HEAD                      # 360448
 # Fused prologue, per token-head: raw q, k, v and the gate pre-activation (bf16), beta, o.
 PROLOGUE_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 2 * 128 + 4 + 2 * 128                    # 1284
-# DRAM bytes (read + write) per launch from ncu captures of the current kernels on
-# these workloads (profiles/*.md); keyed by the kernels one step runs.  A kernel set
-# without a capture on its workload reports null.
+# DRAM bytes (read + write) per launch, taken from ncu captures (dram__bytes_read.sum +
+# dram__bytes_write.sum) of the current kernels on these workloads; keyed by the kernels
+# one step runs.  A kernel set without a capture on its workload reports null.
 NCU_TRAFFIC = {
     ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.8e6 + 181.5e6 + 308.3e6 + 50.5e6,
     # chunk_tc_kernel (--algo fused): captured before its timeout-path change, so reported null

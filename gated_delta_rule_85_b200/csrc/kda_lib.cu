@@ -81,16 +81,48 @@ Plan plan_prefill(long long tokens, int H, int dk, int num_seqs, int algo) {
 }
 
 // Scratch of kda_chunk_forward_static_ws: file scope, reserved on each device
-// with the module; its address is looked up once per device.
+// with the module.  Its device address is looked up per device and kept with the
+// identity of the context it was taken in: after cudaDeviceReset (or any other
+// teardown of the primary context) the module is loaded again and the array may
+// move, so a changed context identity triggers a new lookup.
 static __device__ __align__(256) uint8_t g_static_ws[KDA_STATIC_WS_BYTES];
 
 constexpr int kMaxDevices = 64;
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique identity of the calling thread's current context (0 when there is none
+// or the driver cannot tell; 0 is never cached as valid).
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
 // Device address of g_static_ws on the current device (nullptr on failure, with
-// the CUDA error in *err).
+// the CUDA error in *err).  The symbol is looked up again whenever the current
+// context is not the one of the cached address.
 void *static_ws_address(cudaError_t *err) {
     static std::mutex mu;
     static void *addr[kMaxDevices] = {};
+    static unsigned long long ctx_of[kMaxDevices] = {};
     int dev = 0;
     *err = cudaGetDevice(&dev);
     if (*err != cudaSuccess) return nullptr;
@@ -99,11 +131,13 @@ void *static_ws_address(cudaError_t *err) {
         return nullptr;
     }
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!addr[dev] || ctx == 0 || ctx != ctx_of[dev]) {
         void *p = nullptr;
         *err = cudaGetSymbolAddress(&p, g_static_ws);
         if (*err != cudaSuccess) return nullptr;
         addr[dev] = p;
+        ctx_of[dev] = current_context_id();   // the lookup may have created the context
     }
     return addr[dev];
 }
@@ -447,11 +481,10 @@ int kda_chunk_forward_static_ws(const void *q, const void *k, const void *v, con
         return kda_chunk_forward_simt(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B,
                                       T, H, dk, dv, num_seqs, dtype, chunk, stream);
     const size_t need = plan_prefill((long long)B * T, H, dk, num_seqs, KDA_ALGO_TWO_PASS).ws;
+    // Too large for the built-in scratch: the fused schedule, which needs no scratch at all.
     if (need > KDA_STATIC_WS_BYTES)
-        return fail(KDA_ERR_WORKSPACE,
-                    "these sizes need %zu bytes of two-pass scratch; the built-in scratch holds %zu "
-                    "(KDA_STATIC_WS_BYTES); use kda_chunk_forward_ex with a caller workspace",
-                    need, (size_t)KDA_STATIC_WS_BYTES);
+        return kda_chunk_forward_ex(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,
+                                    dv, num_seqs, dtype, chunk, KDA_ALGO_FUSED, nullptr, 0, stream);
     if (num_seqs == 0) return KDA_OK;
     void *ws = nullptr;
     if (need) {

@@ -163,16 +163,20 @@ int kda_chunk_forward_ex(const void *q, const void *k, const void *v, const floa
  * callers already at their memory limit.
  *
  *   arguments     as kda_chunk_forward, without workspace / ws_bytes
- *   capacity      the two-pass workspace for these sizes
+ *   capacity      when the two-pass workspace for these sizes
  *                 (kda_chunk_forward_workspace_size_ex(..., KDA_ALGO_TWO_PASS))
- *                 must fit in KDA_STATIC_WS_BYTES, else KDA_ERR_WORKSPACE is
- *                 returned before anything is touched or enqueued
+ *                 fits in KDA_STATIC_WS_BYTES the two-pass schedule runs on the
+ *                 built-in scratch; larger sizes run the fused schedule
+ *                 (KDA_ALGO_FUSED), which needs no scratch at all, so no size is
+ *                 refused for lack of room
  *   KDA_F32       takes the fp32 CUDA-core path, which needs no scratch
  *   zeroing       nothing in the scratch has to start at zero: the first pass
  *                 writes every record the second pass reads
- *   first call    on each device, the scratch address is looked up once
- *                 (cudaGetSymbolAddress); make that first call outside stream
- *                 capture
+ *   first call    on each device the scratch address is looked up with
+ *                 cudaGetSymbolAddress and kept with the identity of the current
+ *                 context; after cudaDeviceReset (or any new primary context) the
+ *                 next call looks it up again.  Make the first call on a device,
+ *                 and the first after a reset, outside stream capture
  *   concurrency   all calls on one device share the one scratch array: calls
  *                 that can overlap in time (different streams, or host threads
  *                 without ordering) race and corrupt each other's results;

@@ -46,9 +46,19 @@ def test_static_scratch_matches_caller_workspace_on_consecutive_calls(shape):
         assert np.isfinite(o1.float().cpu().numpy()).all()
 
 
-def test_static_scratch_oversize_is_refused():
+def test_static_scratch_oversize_takes_the_fused_schedule():
+    """Sizes whose two-pass scratch would not fit the built-in array run the fused
+    schedule, which needs no scratch: bit-identical to kda_chunk_forward_ex with
+    algo=fused, on two consecutive calls."""
     shape = PrefillShape(B=1, T=8192, H=32, dk=128, dv=128, dtype=BF16)
-    d = prefill_inputs(shape, 7, torch.device("cuda"))
-    with pytest.raises(kda.KDAError) as e:
-        kda.chunk_forward_static_ws(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"])
-    assert e.value.code == -5
+    need = kda.workspace_size(1, 8192, 32, 128, 128, 1, algo="two_pass")
+    assert need > kda.STATIC_WS_BYTES
+    dev = torch.device("cuda")
+    for seed in (7, 8):
+        d = prefill_inputs(shape, seed, dev)
+        o1, S1 = kda.chunk_forward_static_ws(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"])
+        o2, S2 = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"],
+                                   algo="fused")
+        torch.cuda.synchronize()
+        assert kda.device_status() == 0
+        assert torch.equal(o1, o2) and torch.equal(S1, S2), f"differs from the fused schedule (seed {seed})"
