@@ -5,16 +5,17 @@
 // chunkwise algorithm on a diagonal-plus-low-rank transition).  Everything of a
 // chunk that does not involve the state -- the decay factors, the Gram matrix, the
 // UT transform T = (I + Diag(beta) Akk)^{-1} and the products Kt = Kbar^T Tb,
-// Pt = Aqk Tb -- depends on that chunk's inputs alone.  The fused kernel builds
-// it inside the serial walk over chunks, once per value-column tile.  Here
+// Pt = Aqk Tb -- depends on that chunk's inputs alone; its decay factors are exact
+// for any log_alpha <= 0 (the two tiers described in kda_chunk_tc.cuh).  The fused
+// kernel builds it inside the serial walk over chunks, once per value-column tile.  Here
 //
 //   pass 1, chunk_intra_kernel: one CTA per (chunk, head), all chunks at once,
-//       writes the bf16 operands [Kp; Qp], [Kt; Pt] and e^{G_last} of the chunk to
+//       writes the bf16 operands [e^G K; e^G Q], [Kt; Pt] and e^{G_last} of the chunk to
 //       a workspace record laid out byte for byte like the shared-memory tiles the
 //       second pass feeds to the tensor cores;
 //   pass 2, chunk_inter_kernel: one CTA per (value tile, head, sequence) walks
 //       the chunks in order with only the state-dependent work left on the
-//       serial path: X; Y = [Kp; Qp] (e^{G_last} S), Z = V - X,
+//       serial path: X; Y = [e^G K; e^G Q] S, Z = V - X,
 //       S <- Diag(e^{G_last}) S + Kt Z, O = Y + Pt Z.
 //
 // Chunk slots: chunk c of sequence n (tokens [t0, t1)) is record
@@ -31,7 +32,7 @@ namespace tc {
 template <int DK>
 struct Rec {
     static constexpr int KA = DK / 64;
-    static constexpr int KQ = 0;                          // [KA][128][128 B]  Kp (rows 0-63), Qp (rows 64-127)
+    static constexpr int KQ = 0;                          // [KA][128][128 B]  e^G K (rows 0-63), e^G Q (rows 64-127)
     static constexpr int KP = KA * 128 * 128;             // [DK+64][128 B]    Kt (rows 0..DK-1), Pt (DK..DK+63)
     static constexpr int DCH = KP + (DK + 64) * 128;      // fp32 [DK]         e^{G_last}
     static constexpr int BYTES = (DCH + DK * 4 + 1023) / 1024 * 1024;
@@ -39,10 +40,17 @@ struct Rec {
 
 inline long long chunk_slots(long long tokens, int num_seqs) { return (tokens + C - 1) / C + num_seqs; }
 
-inline size_t two_pass_workspace_bytes(long long tokens, int H, int dk, int num_seqs) {
+// Workspace: the records [slot][H] of the first pass, then one byte per (slot, head)
+// marking the chunks left to the tier-B kernel.
+inline size_t two_pass_records_bytes(long long tokens, int H, int dk, int num_seqs) {
     if (tokens <= 0) return 0;
     const size_t rec = dk == 64 ? (size_t)Rec<64>::BYTES : (size_t)Rec<128>::BYTES;
     return (size_t)chunk_slots(tokens, num_seqs) * (size_t)H * rec;
+}
+inline size_t two_pass_workspace_bytes(long long tokens, int H, int dk, int num_seqs) {
+    if (tokens <= 0) return 0;
+    const size_t marks = ((size_t)chunk_slots(tokens, num_seqs) * (size_t)H + 255) / 256 * 256;
+    return two_pass_records_bytes(tokens, H, dk, num_seqs) + marks;
 }
 
 // First token of sequence n (clamped like seq_span).
@@ -56,28 +64,35 @@ template <int DK>
 struct IntraLayout {
     static constexpr int KA = DK / 64;
     static constexpr int KQ_BYTES = KA * 128 * 128;
+    static constexpr int BT_BYTES = KA * BT_ROWS * 128;
     static constexpr int SCR_BYTES = 2 * 64 * AS * 4 + 32 * 36 * 4;
-    static constexpr int R1 = ((KQ_BYTES > SCR_BYTES ? KQ_BYTES : SCR_BYTES) + 1023) / 1024 * 1024;
-    static constexpr int KQ = 0;                          // [KA][128][128 B] Kp, Qp; then the fp32 scratch:
-    static constexpr int FA = 0;                          //   fp32 [64][AS] Diag(beta) Akk
+    static constexpr int RG_BYTES = ((BT_BYTES > SCR_BYTES ? BT_BYTES : SCR_BYTES) + 1023) / 1024 * 1024;
+    static constexpr int KQ = 0;                          // [KA][128][128 B] e^G K (rows 0-63), e^G Q (64-127);
+                                                          //   tier B: the block-relative rows first
+    static constexpr int RG = KQ + KQ_BYTES;              // tier B: block operands B_0..B_3; after the Gram:
+    static constexpr int FA = RG;                         //   fp32 [64][AS] Diag(beta) Akk
     static constexpr int FT = FA + 64 * AS * 4;           //   fp32 [64][AS] T
     static constexpr int FM = FT + 64 * AS * 4;           //   fp32 [32][36] block products
-    static constexpr int KB = R1;                         // [KA][64][128 B]  Kbar
+    static constexpr int KB = RG + RG_BYTES;              // [KA][64][128 B] tier A: e^{-G} K; tier B: Kbar
     static constexpr int TB = KB + KA * 64 * 128;         // [64][128 B]      Tb^T
     static constexpr int AQ = TB + 64 * 128;              // [64][128 B]      masked Aqk (rows 64-127 of [Tb^T; Aqk])
     static constexpr int FB = AQ + 64 * 128;              // fp32 [64]        beta
+    static constexpr int FD = FB + 64 * 4;                // fp32 [DK]        e^{G_last}
+    static constexpr int FN = FD + DK * 4;                // fp32 [2][64]     prologue: 1/|q_i|, 1/|k_i|
     static constexpr int NSEG = NT / (DK / 4);
-    static constexpr int FSEG = FB + 64 * 4;              // fp32 [NSEG][DK]  segment sums of log_alpha
-    static constexpr int MISC = FSEG + NSEG * DK * 4;     // mbarrier, TMEM base
+    static constexpr int FSEG = FN + 2 * 64 * 4;          // fp32 [NSEG][DK]  segment sums of log_alpha
+    static constexpr int BAD = FSEG + NSEG * DK * 4;      // u32 [4][DK/32]   (block, channel) pairs left to diag_fixup
+    static constexpr int MISC = BAD + 4 * (DK / 32) * 4;  // mbarrier, TMEM base
     static constexpr int BYTES = MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;
-    static_assert(KB % 1024 == 0 && TB % 1024 == 0 && AQ % 1024 == 0, "tile alignment");
+    static_assert(RG % 1024 == 0 && KB % 1024 == 0 && TB % 1024 == 0 && AQ % 1024 == 0, "tile alignment");
     static_assert(2 * (ALLOC + 1024) <= 233472, "two CTAs per SM");
 };
 
 constexpr uint32_t INTRA_TMEM_COLS = 256;
-constexpr uint32_t ICOL_GRAM = 0;     // [128 x 64] rows 0-63 Kp Kbar^T, rows 64-127 Qp Kbar^T
-constexpr uint32_t ICOL_KT = 64;      // [128 x 64] Kt (lanes 0..dk-1)
+constexpr uint32_t ICOL_GRAM = 0;     // tier A: [128 x 64] rows 0-63 (e^G K)(e^{-G} K)^T, rows 64-127 with Q
+constexpr uint32_t ICOL_BT = 64;      // tier B: block b's [128 x 16 (b+1)] at ICOL_BT + bt_row0(b)
+constexpr uint32_t ICOL_KT = 64;      // [128 x 64] Kt (lanes 0..dk-1), after the Gram is read
 constexpr uint32_t ICOL_PT = 128;     // [128 x 64] Pt (lanes 64-127)
 
 __device__ __forceinline__ float4 scale4(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
@@ -98,20 +113,78 @@ __device__ __forceinline__ void st_global_bf16x8(uint8_t *p, const float *x) {
         make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
 }
 
-// GS: scalar gate, log_alpha [tokens, H] (Gated DeltaNet), else [tokens, H, DK].
-// GS: scalar gate (Gated DeltaNet).  PRO: fused input prologue -- q and k are
-// raw (scaled here to unit norm over the key axis) and log_alpha points to the
-// bf16 gate pre-activation x [tokens, H, DK], log_alpha = -softplus(x).
+// Tier B of the first pass, lanes of warps 0-3 (row r of the k rows, warps 0-1, or of
+// the q rows, warps 2-3): the exact diagonal terms of the bad (block, channel) pairs
+// of the row's block, read from the inputs in global memory and added into the
+// Gram accumulator.  Kept out of line: it runs only for chunks that decay by more
+// than e^DECAY_LIM within 16 tokens.
 template <int DK, bool GS, bool PRO>
-__global__ void __launch_bounds__(NT, 2)
-chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                   const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, uint8_t *__restrict__ ws) {
+__device__ __noinline__ void intra_fixup(uint32_t tl, int quad, int warp, int r, int Lc, long long cs, int H, int h,
+                                         const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                                         const float *__restrict__ log_alpha, const uint32_t *bad, const float *fN) {
+    constexpr int NW = DK / 32;
+    constexpr float LOG2E = 1.4426950408889634f;
+    const int rb = r >> 4;
+    const uint32_t *mk = bad + rb * NW;
+    bool fix = false;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) fix |= mk[w] != 0u;
+    if (!__any_sync(0xffffffffu, fix)) return;
+    float fx[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) fx[jj] = 0.f;
+    if (fix) {
+        // chunk token t, channel c of a [tokens, H, DK] input: base + t * tstride + c
+        const long long tstride = (long long)H * DK, base = (cs * H + h) * DK;
+        auto kval = [&](int t, int c) -> float {
+            if (t >= Lc) return 0.f;
+            const float x = __bfloat162float(k[base + t * tstride + c]);
+            if constexpr (PRO) return __bfloat162float(__float2bfloat16_rn(x * fN[64 + t]));
+            return x;
+        };
+        auto alpha = [&](int t, int c) -> float {
+            if (t >= Lc) return 1.f;
+            float g;
+            if constexpr (GS) g = log_alpha[(cs + t) * H + h];
+            else if constexpr (PRO)
+                g = neg_softplus(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(log_alpha)[base + t * tstride + c]));
+            else g = log_alpha[base + t * tstride + c];
+            return exp2_fast(g * LOG2E);
+        };
+        auto xval = [&](int c) -> float {
+            if (r >= Lc) return 0.f;
+            if (warp < 2) return kval(r, c);
+            const float x = __bfloat162float(q[base + r * tstride + c]);
+            if constexpr (PRO) return __bfloat162float(__float2bfloat16_rn(x * fN[r]));
+            return x;
+        };
+        diag_fixup<NW>(fx, mk, rb, r, alpha, kval, xval);
+    }
+    diag_add(tl, ICOL_BT, quad, rb, fx);
+}
+
+// GS: scalar gate, log_alpha [tokens, H] (Gated DeltaNet).  PRO: fused input
+// prologue -- q and k are raw (scaled here to unit norm over the key axis) and
+// log_alpha points to the bf16 gate pre-activation x [tokens, H, DK],
+// log_alpha = -softplus(x).
+// One (chunk slot, head) of the first pass.  TB = false: tier A only -- a chunk
+// that needs tier B is only marked in `flags` (1; 0 for every other slot) and left
+// to chunk_intra_strong_kernel.  TB = true: tier B.  All threads of the CTA call
+// it; ph_mma carries the MMA mbarrier phase across calls.  Returns false when a
+// bounded wait ran out.
+template <int DK, bool GS, bool PRO, bool TB>
+__device__ __forceinline__ bool intra_chunk(int slot, int h, const __nv_bfloat16 *__restrict__ q,
+                                            const __nv_bfloat16 *__restrict__ k,
+                                            const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                                            const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
+                                            uint8_t *__restrict__ ws, uint8_t *__restrict__ flags, uint8_t *sm,
+                                            uint32_t tmem, uint32_t &ph_mma) {
     using L = IntraLayout<DK>;
     using R = Rec<DK>;
-    constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG;
+    constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG, SPB = 16 / SEGLEN, NW = DK / 32;
     constexpr float LOG2E = 1.4426950408889634f;
-    const int slot = blockIdx.x, h = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
 
     // the sequence owning this slot: the last n whose first slot n + floor(t0_n / 64) is <= slot
     int lo = 0, hi = num_seqs - 1;
@@ -123,40 +196,32 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     long long t0, t1;
     seq_span(cu_seqlens, T, lo, t0, t1);
     const long long cs = t0 + (long long)(slot - (lo + t0 / C)) * C;
-    if (cs < t0 || cs >= t1) return;   // slot without a chunk (the whole CTA leaves)
+    if (cs < t0 || cs >= t1) {   // slot without a chunk
+        if (!TB && tid == 0) flags[(size_t)slot * H + h] = 0;
+        return true;
+    }
     const int Lc = (int)min((long long)C, t1 - cs);
-
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = ptx::smem_u32(sm);
     float *fA = reinterpret_cast<float *>(sm + L::FA);
     float *fT = reinterpret_cast<float *>(sm + L::FT);
     float *fM = reinterpret_cast<float *>(sm + L::FM);
     float *fB = reinterpret_cast<float *>(sm + L::FB);
+    float *fD = reinterpret_cast<float *>(sm + L::FD);
+    float *fN = reinterpret_cast<float *>(sm + L::FN);
     float *fSeg = reinterpret_cast<float *>(sm + L::FSEG);
+    uint32_t *bad = reinterpret_cast<uint32_t *>(sm + L::BAD);
     const uint32_t bar_mma = sb + L::MISC;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 8);
     uint8_t *rec = ws + ((size_t)slot * H + h) * R::BYTES;
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
-
-    if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTRA_TMEM_COLS);
-        ptx::tmem_relinquish();
-    }
-    if (tid == 0) {
-        ptx::mbar_init(bar_mma, 1);
-        ptx::fence_mbar_init();
-    }
     if (tid < C) fB[tid] = tid < Lc ? beta[(cs + tid) * H + h] : 0.f;
+    if (tid < 4 * NW) bad[tid] = 0u;
 
-    // ---- 1. decay factors -> Kp, Qp (written to the record too), Kbar, e^{G_last}
+    // ---- 1. decay factors -> the Gram operands (tier A or B), Kbar, e^{G_last}
+    const int cg = tid % NCG, seg = tid / NCG, c0 = 4 * cg, i0 = seg * SEGLEN, blk = seg / SPB;
+    float al[SEGLEN][4];
+    uint2 qv[SEGLEN], kv[SEGLEN];
+    float4 sg = make_float4(0.f, 0.f, 0.f, 0.f);
     {
-        const int cg = tid % NCG, seg = tid / NCG, c0 = 4 * cg, i0 = seg * SEGLEN;
-        float al[SEGLEN][4];
-        uint2 qv[SEGLEN], kv[SEGLEN];
-        float4 sg = make_float4(0.f, 0.f, 0.f, 0.f);
         // all loads first, unconditionally (rows past Lc read the last valid row
         // and are zeroed afterwards), so every one is in flight before any is used
         float4 gv[SEGLEN];
@@ -191,53 +256,101 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             sg.x += g4.x; sg.y += g4.y; sg.z += g4.z; sg.w += g4.w;
             al[u][0] = g4.x; al[u][1] = g4.y; al[u][2] = g4.z; al[u][3] = g4.w;
         }
-        // prologue: q and k rows to unit norm (a row's DK channels live in NCG
-        // consecutive lanes of one warp), rounded back to bf16 -- the same values
-        // as normalising in fp32 and then casting, as prepared inputs are made
-        if constexpr (PRO) {
+    }
+    // prologue: q and k rows to unit norm (a row's DK channels live in NCG
+    // consecutive lanes of one warp), rounded back to bf16 -- the same values as
+    // normalising in fp32 and then casting, as prepared inputs are made
+    if constexpr (PRO) {
 #pragma unroll
-            for (int u = 0; u < SEGLEN; ++u) {
-                const float4 a = bf16x4_to_float4(qv[u]), b = bf16x4_to_float4(kv[u]);
-                float sq = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
-                float sk = b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
+        for (int u = 0; u < SEGLEN; ++u) {
+            const float4 a = bf16x4_to_float4(qv[u]), b = bf16x4_to_float4(kv[u]);
+            float sq = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+            float sk = b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
 #pragma unroll
-                for (int o = NCG / 2; o > 0; o >>= 1) {
-                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
-                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
-                }
-                qv[u] = float4_to_bf16x4(scale4(a, inv_row_norm(sq)));
-                kv[u] = float4_to_bf16x4(scale4(b, inv_row_norm(sk)));
+            for (int o = NCG / 2; o > 0; o >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                sk += __shfl_xor_sync(0xffffffffu, sk, o);
             }
-        }
-        *reinterpret_cast<float4 *>(fSeg + seg * DK + c0) = sg;
-        __syncthreads();
-        float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int s2 = 0; s2 < NSEG; ++s2) {
-            const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
-            const float xv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                if (s2 < seg) pre[e] += xv[e];
-                tot[e] += xv[e];
+            const float iq = inv_row_norm(sq), ik = inv_row_norm(sk);
+            if (cg == 0) {
+                fN[i0 + u] = iq;
+                fN[64 + i0 + u] = ik;
             }
+            qv[u] = float4_to_bf16x4(scale4(a, iq));
+            kv[u] = float4_to_bf16x4(scale4(b, ik));
         }
-        if (seg == 0) {
-            if (tot[0] < -80.f || tot[1] < -80.f || tot[2] < -80.f || tot[3] < -80.f) flag_status(KDA_DEV_DECAY_RANGE);
-            *reinterpret_cast<float4 *>(rec + R::DCH + c0 * 4) =
-                make_float4(expf(tot[0]), expf(tot[1]), expf(tot[2]), expf(tot[3]));
-        }
+    }
+    *reinterpret_cast<float4 *>(fSeg + seg * DK + c0) = sg;
+    // every segment sum >= -DECAY_LIM / NSEG proves every chunk sum >= -DECAY_LIM (tier A)
+    constexpr float SEG_LIM = -DECAY_LIM / NSEG;
+    const bool maybe_strong = __syncthreads_or(sg.x < SEG_LIM || sg.y < SEG_LIM || sg.z < SEG_LIM || sg.w < SEG_LIM) != 0;
+    // prefix sums over the segments: pre = G before this segment, tot = G_last,
+    // gsb = G before this thread's own 16-token block
+    float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f}, gsb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < SEGLEN; ++u)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) al[u][e] = exp2_fast(al[u][e] * LOG2E);
-        const float sgv[4] = {sg.x, sg.y, sg.z, sg.w};
-        float ef[4], eb[4];   // e^{G_i - G_last} (>= 1), e^{G_last - G_i} (<= 1)
+    for (int s2 = 0; s2 < NSEG; ++s2) {
+        const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
+        const float xv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            ef[e] = exp2_fast((pre[e] - tot[e]) * LOG2E);
-            eb[e] = exp2_fast((tot[e] - pre[e] - sgv[e]) * LOG2E);
+            if (s2 < seg) pre[e] += xv[e];
+            if (s2 < blk * SPB) gsb[e] += xv[e];
+            tot[e] += xv[e];
         }
+    }
+    // G before block b (b = 0..4; G_last at 4) for this thread's channels, from the segment sums
+    auto g_before = [&](int b, float (&gb)[4]) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) gb[e] = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < NSEG; ++s2) {
+            if (s2 >= b * SPB) break;
+            const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
+            gb[0] += x.x; gb[1] += x.y; gb[2] += x.z; gb[3] += x.w;
+        }
+    };
+    constexpr bool tier_b = TB;
+    if constexpr (!TB) {
+        if (maybe_strong) {
+            const bool strong =
+                tot[0] < -DECAY_LIM || tot[1] < -DECAY_LIM || tot[2] < -DECAY_LIM || tot[3] < -DECAY_LIM;
+            if (__syncthreads_or(strong)) {   // uniform over the CTA: leave this chunk to tier B
+                if (tid == 0) flags[(size_t)slot * H + h] = 1;
+                return true;
+            }
+        }
+        if (tid == 0) flags[(size_t)slot * H + h] = 0;
+    }
+    const float sgv[4] = {sg.x, sg.y, sg.z, sg.w};
+    if (seg == 0) {
+        const float4 d4 = make_float4(expf(tot[0]), expf(tot[1]), expf(tot[2]), expf(tot[3]));
+        *reinterpret_cast<float4 *>(rec + R::DCH + c0 * 4) = d4;
+        *reinterpret_cast<float4 *>(fD + c0) = d4;
+        if (tier_b) {
+#pragma unroll 1
+            for (int b = 0; b < 4; ++b) {
+                float ga[4], gz[4];
+                g_before(b, ga);
+                g_before(b + 1, gz);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (gz[e] - ga[e] < -DECAY_LIM) atomicOr(&bad[b * NW + (c0 + e) / 32], 1u << ((c0 + e) & 31));
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < SEGLEN; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) al[u][e] = exp2_fast(al[u][e] * LOG2E);
+
+    // rows e^{G_i - ref} x_i (<= 1) of the A operand; ref = 0 (tier A / the record) or the block start (tier B)
+    // rows e^{G_i - ref} x_i: ref = 0 into the A tile (tier A, the record's image) or
+    // the block start (tier B); to_rec: ref = 0 straight into the workspace record
+    // (tier B, whose A tile holds the block-relative rows)
+    auto store_rows = [&](bool rel_block, bool to_rec) {
+        float ef[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ef[e] = exp2_fast((pre[e] - (rel_block ? gsb[e] : 0.f)) * LOG2E);
 #pragma unroll
         for (int u = 0; u < SEGLEN; ++u) {
             const int i = i0 + u;
@@ -245,89 +358,135 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             const float4 k4 = bf16x4_to_float4(kv[u]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) ef[e] *= al[u][e];
-            st_bf16x4(sm, L::KQ + sw128(i, c0, 128), k4.x * ef[0], k4.y * ef[1], k4.z * ef[2], k4.w * ef[3]);
-            st_bf16x4(sm, L::KQ + sw128(64 + i, c0, 128), q4.x * ef[0], q4.y * ef[1], q4.z * ef[2], q4.w * ef[3]);
+            const uint2 kr = make_uint2(pack_bf16(k4.x * ef[0], k4.y * ef[1]), pack_bf16(k4.z * ef[2], k4.w * ef[3]));
+            const uint2 qr = make_uint2(pack_bf16(q4.x * ef[0], q4.y * ef[1]), pack_bf16(q4.z * ef[2], q4.w * ef[3]));
+            uint8_t *dst = to_rec ? rec + R::KQ : sm + L::KQ;
+            *reinterpret_cast<uint2 *>(dst + sw128(i, c0, 128)) = kr;
+            *reinterpret_cast<uint2 *>(dst + sw128(64 + i, c0, 128)) = qr;
         }
+    };
+    // rows e^{ref - G_j} k_j, j in this segment, into a 64-column-atom tile of `rows` rows;
+    // e0 = e^{ref - G at the segment end} per channel, multiplied by alpha going back
+    auto store_cols = [&](uint32_t tile, int rows, float (&e0)[4]) {
 #pragma unroll
         for (int u = SEGLEN - 1; u >= 0; --u) {
             const int i = i0 + u;
             const float4 k4 = bf16x4_to_float4(kv[u]);
-            st_bf16x4(sm, L::KB + sw128(i, c0, 64), k4.x * eb[0], k4.y * eb[1], k4.z * eb[2], k4.w * eb[3]);
+            st_bf16x4(sm, tile + sw128(i, c0, rows), k4.x * e0[0], k4.y * e0[1], k4.z * e0[2], k4.w * e0[3]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) eb[e] *= al[u][e];
+            for (int e = 0; e < 4; ++e) e0[e] *= al[u][e];
+        }
+    };
+    if constexpr (!TB) {
+        store_rows(false, false);
+        float er[4];   // e^{-G_j}: at most e^{DECAY_LIM} in a tier-A chunk
+#pragma unroll
+        for (int e = 0; e < 4; ++e) er[e] = exp2_fast(-(pre[e] + sgv[e]) * LOG2E);
+        store_cols(L::KB, 64, er);
+    } else {
+        store_rows(true, false);
+        store_rows(false, true);
+        float eb[4];   // Kbar: e^{G_last - G_j} <= 1
+#pragma unroll
+        for (int e = 0; e < 4; ++e) eb[e] = exp2_fast((tot[e] - pre[e] - sgv[e]) * LOG2E);
+        store_cols(L::KB, 64, eb);
+#pragma unroll 1
+        for (int b = blk; b < 4; ++b) {   // block b's operand holds tokens j < 16 (b + 1)
+            float ga[4], gz[4], eB[4];    // e^{G_s(b) - G_j}: <= 1 before block b, <= e^{DECAY_LIM} inside it
+            g_before(b, ga);
+            g_before(b + 1, gz);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const bool out = b == blk && gz[e] - ga[e] < -DECAY_LIM;   // bad pair: left to diag_fixup
+                eB[e] = out ? 0.f : exp2_fast(fminf(ga[e] - pre[e] - sgv[e], DECAY_LIM) * LOG2E);
+            }
+            store_cols(L::RG + bt_off(b, DK / 64), 16 * (b + 1), eB);
         }
     }
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t ph_mma = 0;
 
-    // ---- 2. Gram = [Kp; Qp] Kbar^T; the Kp/Qp image goes to the record meanwhile
+    // ---- 2. Gram; in tier A the tile is the record's e^G K / e^G Q image, stored meanwhile
     if (tid == 0) {
-        ptx::bulk_store(rec + R::KQ, sb + L::KQ, (uint32_t)L::KQ_BYTES);
-        ptx::bulk_commit();
-        constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64);
+        if constexpr (!TB) {
+            ptx::bulk_store(rec + R::KQ, sb + L::KQ, (uint32_t)L::KQ_BYTES);
+            ptx::bulk_commit();
+            constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64);
 #pragma unroll
-        for (int s = 0; s < DK / 16; ++s)
-            ptx::mma_bf16(tmem + ICOL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KB, s, 64), ig, s > 0);
+            for (int s = 0; s < DK / 16; ++s)
+                ptx::mma_bf16(tmem + ICOL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KB, s, 64), ig, s > 0);
+        } else {
+#pragma unroll 1
+            for (int b = 0; b < 4; ++b) {
+                const int rows = 16 * (b + 1);
+                const uint32_t ib = ptx::idesc_bf16_f32(128, rows);
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)
+                    ptx::mma_bf16(tmem + ICOL_BT + bt_row0(b), kdesc(sb + L::KQ, s, 128),
+                                  kdesc(sb + L::RG + bt_off(b, DK / 64), s, rows), ib, s > 0);
+            }
+        }
         ptx::mma_commit(bar_mma);
-        ptx::bulk_wait_read_all();   // the fp32 scratch below overwrites the Kp/Qp tile
     }
     bool ok = wait_all(bar_mma, ph_mma);
 
     if (ok) {
         // ---- 3. Diag(beta) Akk -> diagonal blocks of T (warps 0-1); masked Aqk (warps 2-3);
         //         zero blocks of T and Tb^T (warps 6-7)
-        if (warp < 2) {
+        if (warp < 4) {
+            const int r = tid & 63, rb = r >> 4;   // token row of this lane, its 16-row block
+            if constexpr (TB) intra_fixup<DK, GS, PRO>(tl, quad, warp, r, Lc, cs, H, h, q, k, log_alpha, bad, fN);
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 float g32[32];
-                ptx::tmem_ld32(tl + ICOL_GRAM + hh * 32, g32);
-                ptx::tmem_wait_ld();
-                const int i = tid;
-                const float bi = fB[i];
+                if constexpr (!TB) {
+                    ptx::tmem_ld32(tl + ICOL_GRAM + hh * 32, g32);
+                    ptx::tmem_wait_ld();
+                } else {
+                    gram_tier_b_ld32(tl, ICOL_BT, quad, hh, r, g32);
+                }
+                if (warp < 2) {
+                    const int i = r;
+                    const float bi = fB[i];
 #pragma unroll
-                for (int u = 0; u < 32; u += 4) {
-                    const int j = hh * 32 + u;
-                    float4 a;
-                    a.x = (j + 0 < i) ? bi * g32[u + 0] : 0.f;
-                    a.y = (j + 1 < i) ? bi * g32[u + 1] : 0.f;
-                    a.z = (j + 2 < i) ? bi * g32[u + 2] : 0.f;
-                    a.w = (j + 3 < i) ? bi * g32[u + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(fA + i * AS + j) = a;
+                    for (int u = 0; u < 32; u += 4) {
+                        const int j = hh * 32 + u;
+                        float4 a;
+                        a.x = (j + 0 < i) ? bi * g32[u + 0] : 0.f;
+                        a.y = (j + 1 < i) ? bi * g32[u + 1] : 0.f;
+                        a.z = (j + 2 < i) ? bi * g32[u + 2] : 0.f;
+                        a.w = (j + 3 < i) ? bi * g32[u + 3] : 0.f;
+                        *reinterpret_cast<float4 *>(fA + i * AS + j) = a;
+                    }
+                } else {
+                    const int i = r;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) g32[u] = (hh * 32 + u <= i) ? g32[u] : 0.f;
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::AQ + sw128_chunk(i, hh * 4 + gq), g32 + gq * 8);
                 }
             }
-            asm volatile("bar.sync 1, 64;" ::: "memory");
-            invert_diag_blocks(fA, fT, sm + L::TB, fB, tid);
-        } else if (warp < 4) {
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                float g32[32];
-                ptx::tmem_ld32(tl + ICOL_GRAM + hh * 32, g32);
-                ptx::tmem_wait_ld();
-                const int i = tid - 64;
-#pragma unroll
-                for (int u = 0; u < 32; ++u) g32[u] = (hh * 32 + u <= i) ? g32[u] : 0.f;
-#pragma unroll
-                for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::AQ + sw128_chunk(i, hh * 4 + gq), g32 + gq * 8);
+            if (warp < 2) {
+                asm volatile("bar.sync 1, 64;" ::: "memory");
+                invert_diag_blocks(fA, fT, sm + L::TB, fB, tid);
             }
         } else if (warp >= 6) {
             const int t = tid - 192;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
-                const int e = t + 64 * m, blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                fT[(32 * blk + r) * AS + 32 * blk + 16 + c] = 0.f;
+                const int e = t + 64 * m, blk2 = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                fT[(32 * blk2 + r) * AS + 32 * blk2 + 16 + c] = 0.f;
             }
             const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int m = 0; m < 3; ++m) {
                 const int e = t + 64 * m;
-                const int blk = e >> 5, r = (e >> 1) & 15, gh = e & 1;
-                const int bi = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                const int bj = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int blk2 = e >> 5, r = (e >> 1) & 15, gh = e & 1;
+                const int bi = blk2 < 3 ? blk2 + 1 : (blk2 < 5 ? blk2 - 1 : 3);
+                const int bj = blk2 < 3 ? 0 : (blk2 < 5 ? 1 : 2);
                 *reinterpret_cast<uint4 *>(sm + L::TB + sw128_chunk(16 * bi + r, 2 * bj + gh)) = z;
             }
         }
@@ -337,7 +496,7 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 4. Kt = Kbar^T Tb (Kbar read MN-major); Pt = Aqk Tb from the M = 128 operand [Tb^T; Aqk]
+        // ---- 4. Kt = (KB tile)^T Tb (read MN-major); Pt = Aqk Tb from the M = 128 operand [Tb^T; Aqk]
         if (tid == 0) {
             ptx::tc_fence_after();
             constexpr uint32_t ikt = ptx::idesc_bf16_f32(128, 64, true, false);
@@ -355,13 +514,19 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
 
     if (ok) {
-        // ---- 5. Kt, Pt -> bf16 images in the record (each thread one 64-byte half row)
+        // ---- 5. Kt, Pt -> bf16 images in the record (each thread one 64-byte half row);
+        //         tier A's KB tile is e^{-G} K, so its Kt rows take the factor e^{G_last}
         uint8_t *kp = rec + R::KP;
         if (quad < DK / 32) {
             float x[32];
             ptx::tmem_ld32(tl + ICOL_KT + half * 32, x);
             ptx::tmem_wait_ld();
             const int row = quad * 32 + lane;
+            if constexpr (!TB) {
+                const float dr = fD[row];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) x[u] *= dr;
+            }
 #pragma unroll
             for (int gq = 0; gq < 4; ++gq) st_global_bf16x8(kp + sw128_chunk(row, half * 4 + gq), x + gq * 8);
         }
@@ -378,9 +543,85 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         if (!ok) ptx::mbar_wait_bounded(bar_mma, ph_mma ^ 1u, WAIT_LIMIT_CYCLES);   // MMAs still in flight
         ptx::bulk_wait_all();
     }
+    return ok;
+}
+
+// First pass, tier A: one CTA per (chunk slot, head).
+template <int DK, bool GS, bool PRO>
+__global__ void __launch_bounds__(NT, 2)
+chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                   const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, uint8_t *__restrict__ ws,
+                   uint8_t *__restrict__ flags) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t bar_mma = ptx::smem_u32(sm) + IntraLayout<DK>::MISC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + IntraLayout<DK>::MISC + 8);
+    if ((threadIdx.x >> 5) == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTRA_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+    }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t ph_mma = 0;
+    intra_chunk<DK, GS, PRO, false>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta, cu_seqlens, T, H,
+                                    num_seqs, ws, flags, sm, tmem, ph_mma);
+    ptx::tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, INTRA_TMEM_COLS);
+    }
+}
+
+// First pass, tier B: the chunks chunk_intra_kernel marked, one CTA per SM walking
+// the (slot, head) marks; nothing to do (and quick) when no chunk decays that fast.
+template <int DK, bool GS, bool PRO>
+__global__ void __launch_bounds__(NT, 1)
+chunk_intra_strong_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                          const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                          const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
+                          uint8_t *__restrict__ ws, uint8_t *__restrict__ flags, long long items) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t bar_mma = ptx::smem_u32(sm) + IntraLayout<DK>::MISC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + IntraLayout<DK>::MISC + 8);
+    __shared__ int s_any;
+    if (threadIdx.x == 0) s_any = 0;
+    __syncthreads();
+    for (long long it = blockIdx.x + (long long)threadIdx.x * gridDim.x; it < items; it += (long long)blockDim.x * gridDim.x)
+        if (flags[it]) s_any = 1;
+    __syncthreads();
+    if (!s_any) return;   // no marked chunk for this CTA
+    if ((threadIdx.x >> 5) == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTRA_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t ph_mma = 0;
+    for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+        if (!flags[it]) continue;   // uniform: every thread reads the same mark
+        __syncthreads();            // the previous chunk's last shared-memory reads are done
+        if (!intra_chunk<DK, GS, PRO, true>((int)(it / H), (int)(it % H), q, k, log_alpha, beta, cu_seqlens, T, H,
+                                            num_seqs, ws, flags, sm, tmem, ph_mma))
+            break;
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, INTRA_TMEM_COLS);
     }
@@ -392,7 +633,7 @@ template <int DK, int DVT, int NBUF>
 struct InterLayout {
     static constexpr int KA = DK / 64;
     static constexpr int REC = Rec<DK>::BYTES;
-    static constexpr int SP = NBUF * REC;                 // [KA][DVT][128 B] (e^{G_last} S)^T
+    static constexpr int SP = NBUF * REC;                 // [KA][DVT][128 B] S^T (bf16)
     static constexpr int ZT = SP + KA * DVT * 128;        // [DVT][128 B]     Z^T
     static constexpr int VIN = ZT + DVT * 128;            // bf16 [NBUF][64][DVT]
     static constexpr int MISC = VIN + NBUF * C * DVT * 2; // mbarriers, TMEM base, flags
@@ -492,17 +733,17 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
         ph_rec ^= 1u << b;
         if (!ok) break;
 
-        // ---- 1. (e^{G_last} S)^T -> bf16 B operand
+        // ---- 1. S^T -> bf16 B operand
         const float dch = has_row ? reinterpret_cast<const float *>(sm + b * R::BYTES + R::DCH)[srow] : 0.f;
         if (has_row) {
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::SP + sw128(scol + j, srow, DVT), dch * S[j]);
+            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::SP + sw128(scol + j, srow, DVT), S[j]);
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 2. [X; Y] = [Kp; Qp] (e^{G_last} S)
+        // ---- 2. [X; Y] = [e^G K; e^G Q] S
         if (tid == 0) {
             ptx::tc_fence_after();
             constexpr uint32_t ix = ptx::idesc_bf16_f32(128, DVT);
@@ -608,6 +849,18 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
 
 // ------------------------------------------------------------------ host side
 
+// Multiprocessor count of the current device (148 on B200), looked up once per device.
+inline int sm_count() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        cached[dev] = (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) ? n : 148;
+    }
+    return cached[dev];
+}
+
 template <int DK, int DVT, bool GS, bool PRO>
 int launch_two_pass_t(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                       const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
@@ -624,6 +877,7 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         return KDA_ERR_UNSUPPORTED;
     }
     constexpr int smem1 = IntraLayout<DK>::ALLOC;
+    uint8_t *marks = (uint8_t *)workspace + two_pass_records_bytes(tokens, H, DK, num_seqs);
     auto k1 = chunk_intra_kernel<DK, GS, PRO>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
     if (e != cudaSuccess) {
@@ -631,10 +885,25 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         return KDA_ERR_CUDA;
     }
     k1<<<dim3((unsigned)rec_slots, H), NT, smem1, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
-                                                     beta, cu_seqlens, T, H, num_seqs, (uint8_t *)workspace);
+                                                     beta, cu_seqlens, T, H, num_seqs, (uint8_t *)workspace, marks);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "chunk_intra launch: %s", cudaGetErrorString(e));
+        return KDA_ERR_CUDA;
+    }
+    auto k1b = chunk_intra_strong_kernel<DK, GS, PRO>;
+    e = cudaFuncSetAttribute(k1b, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
+    if (e != cudaSuccess) {
+        snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_intra_strong): %s", cudaGetErrorString(e));
+        return KDA_ERR_CUDA;
+    }
+    const long long items = rec_slots * H;
+    const int ctas = (int)std::min<long long>(items, (long long)sm_count());
+    k1b<<<ctas, NT, smem1, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha, beta, cu_seqlens, T, H,
+                                 num_seqs, (uint8_t *)workspace, marks, items);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        snprintf(msg, msg_len, "chunk_intra_strong launch: %s", cudaGetErrorString(e));
         return KDA_ERR_CUDA;
     }
     constexpr int NBUF = inter_nbuf<DK, DVT>();

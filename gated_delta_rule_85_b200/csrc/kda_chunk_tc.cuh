@@ -8,20 +8,20 @@
 // chunkwise algorithm on a diagonal-plus-low-rank transition).
 //
 // For a chunk starting from state S (dk x dv), G_i = sum_{s<=i} log_alpha_s per channel:
-//   Khat = e^G * K, Qhat = e^G * Q, Rk = e^{-G} * K, Kbar = e^{G_last - G} * K
-//   Akk = strict_lower(Khat Rk^T), Aqk = lower(Qhat Rk^T)          (Gram, one MMA)
-//   X = Khat S, Y = Qhat S                                          (one MMA, state-dependent)
+//   Khat = e^G * K, Qhat = e^G * Q, Kbar = e^{G_last - G} * K        (every factor <= 1)
+//   Akk = strict_lower(Khat-Gram), Aqk = lower(Qhat-Gram)            (entries sum_c x_ic k_jc e^{G_ic - G_jc})
+//   X = Khat S, Y = Qhat S                                          (state-dependent)
 //   T = (I + Diag(beta) Akk)^{-1},  Tb = T Diag(beta)               (fp32, shared memory)
 //   Kt = Kbar^T Tb,  Pt = Aqk Tb                                    (one MMA pair)
 //   Z = V - X
 //   S <- Diag(e^{G_last}) S + Kt Z,   O = Y + Pt Z                   (one MMA pair)
-// The e^{-G} factor bounds the usable range: a channel's log-decay summed over one
-// chunk must stay >= -80 (checked; KDA_DEV_DECAY_RANGE otherwise).
+// The Gram's pairwise factors e^{G_ic - G_jc} are split into bf16 operands in two
+// tiers (see DECAY_LIM below), exact for any log_alpha <= 0.
 //
 // Mapping: one 256-thread CTA per (value-column tile of DVT, head, sequence) walks
 // the sequence's chunks in order.  TMA brings each chunk's q, k, log_alpha and v
 // tiles into shared memory, the next chunk's while the current one computes.
-// All threads build the decayed bf16 operands (two key channels x one token
+// All threads build the decayed bf16 operands (four key channels x one token
 // segment each); threads 0..dk-1 keep row c of the fp32 state in registers, which
 // is also TMEM lane c of every 128-row accumulator.  Thread 0 issues the MMAs;
 // completion is signalled through mbarriers with bounded waits.  bf16 operands
@@ -31,6 +31,7 @@
 
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstdio>
 
 #include "kda_common.cuh"
@@ -44,26 +45,39 @@ constexpr int NT = 256;
 constexpr long long WAIT_LIMIT_CYCLES = 2000000000ll;   // >= 1 s at any SM clock up to 2 GHz: far beyond any legitimate latency
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM column map (fp32 accumulators, lane = row)
-constexpr uint32_t COL_GRAM = 0;    // [128 x 64]  rows 0-63 Kp Kbar^T, rows 64-127 Qp Kbar^T
+constexpr uint32_t COL_GRAM = 0;    // [128 x 64]  tier A: rows 0-63 (e^G K)(e^{-G} K)^T, rows 64-127 with Q
 constexpr uint32_t COL_XY = 64;     // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O (same MMA as the Gram)
 constexpr uint32_t COL_KT = 192;    // [128 x 64]  Kt (lanes 0..dk-1)
 constexpr uint32_t COL_PT = 256;    // [128 x 64]  Pt (lanes 64-127)
 constexpr uint32_t COL_DS = 320;    // [128 x DVT] Kt Z (lanes 0..dk-1)
+constexpr uint32_t COL_BT = 192;    // tier B: block b's Gram [128 x 16 (b+1)] at COL_BT + bt_row0(b) (in KT..DS, free then)
 constexpr int AS = 68;              // fp32 row stride of the 64 x 64 scratch matrices (16-byte rows)
+constexpr float DECAY_LIM = 80.f;
+
+// First row of block b's operand in the tier-B operand region (tiles of 16 (b + 1)
+// rows: 0, 16, 48, 96) -- also its TMEM column offset.
+__host__ __device__ constexpr int bt_row0(int b) { return 8 * b * (b + 1); }
+constexpr int BT_ROWS = 160;   // bt_row0(4)
+
 
 template <int DK, int DVT>
 struct Layout {
     static constexpr int KA = DK / 64;                       // 64-element K atoms along dk
     // bf16 MMA operands, 128-byte swizzled, 1024-byte aligned
-    static constexpr int KQ = 0;                             // [KA][128][128 B] Kp (0-63), Qp (64-127)
+    static constexpr int KQ = 0;                             // [KA][128][128 B] e^G K (0-63), e^G Q (64-127);
+                                                             //   tier B: the block-relative rows first
     static constexpr int KSR = 64 + DVT;                     // rows of the combined B operand
-    static constexpr int KS = KQ + KA * 128 * 128;           // [KA][64+DVT][128 B] rows 0-63 Kbar (tokens),
-                                                             //   rows 64.. (e^{G_last} S)^T (value columns)
-    static constexpr int KP = KS + KA * KSR * 128;           // [DK+64][128 B]   Kt (0..DK-1), Aqk -> Pt (DK..)
-    static constexpr int TB = KP + (DK + 64) * 128;          // [64][128 B]      Tb^T
-    static constexpr int ZT = TB + 64 * 128;                 // [DVT][128 B]     Z^T
+    static constexpr int KS = KQ + KA * 128 * 128;           // [KA][64+DVT][128 B] rows 0-63: tier A e^{-G} K,
+                                                             //   tier B Kbar (tokens); rows 64..: S^T (value columns)
+    static constexpr int RX = KS + KA * KSR * 128;           // Kt/Pt, Tb^T, Z^T; tier B: block operands B_0..B_3
+    static constexpr int KP = RX;                            //   [DK+64][128 B] Kt (0..DK-1), Aqk -> Pt (DK..)
+    static constexpr int TB = KP + (DK + 64) * 128;          //   [64][128 B]    Tb^T
+    static constexpr int ZT = TB + 64 * 128;                 //   [DVT][128 B]   Z^T
+    static constexpr int RX_USE = ZT + DVT * 128 - RX;
+    static constexpr int BT_BYTES = KA * BT_ROWS * 128;
+    static constexpr int RX_BYTES = ((RX_USE > BT_BYTES ? RX_USE : BT_BYTES) + 1023) / 1024 * 1024;
     // dense TMA input tiles; the fp32 scratch of the UT transform aliases them
-    static constexpr int QIN = ZT + DVT * 128;               // bf16 [64][DK]
+    static constexpr int QIN = RX + RX_BYTES;                // bf16 [64][DK]
     static constexpr int KIN = QIN + 64 * DK * 2;            // bf16 [64][DK]
     static constexpr int GIN = KIN + 64 * DK * 2;            // fp32 [64][DK]
     static constexpr int IN_BYTES = 64 * DK * 8;
@@ -76,7 +90,8 @@ struct Layout {
     static constexpr int FB = VIN + 64 * DVT * 2;            // fp32 [2][64]    beta
     static constexpr int NSEG = NT / (DK / 4);               // token segments in the factor stage
     static constexpr int FSEG = FB + 2 * 64 * 4;             // fp32 [NSEG][DK] segment sums of log_alpha
-    static constexpr int MISC = FSEG + NSEG * DK * 4;        // mbarriers, TMEM base, flags
+    static constexpr int BAD = FSEG + NSEG * DK * 4;         // u32 [4][DK/32]  (block, channel) pairs left to diag_fixup
+    static constexpr int MISC = BAD + 4 * (DK / 32) * 4;     // mbarriers, TMEM base, flags
     static constexpr int BYTES = MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024 B
     static_assert(KQ % 1024 == 0 && KS % 1024 == 0 && KP % 1024 == 0 && TB % 1024 == 0 && ZT % 1024 == 0 &&
@@ -249,6 +264,113 @@ __device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, f
     }
 }
 
+// ------------------------------------------------------------------ exact decay factors
+//
+// The Gram matrices need e^{G_i - G_j} (i >= j, G the per-channel cumulative log
+// decay of the chunk), which is at most 1 but may be as small as the data makes it
+// (a channel can forget everything in one token).  It is split into two bf16 MMA
+// operands, one factor per side, in one of two tiers chosen per chunk:
+//   tier A (every channel's chunk decay >= -DECAY_LIM): rows e^{G_i} x_i (<= 1)
+//       against e^{-G_j} k_j (<= e^DECAY_LIM), one product of N = 64;
+//   tier B (otherwise): 16-token blocks.  Row i of block b is scaled relative to
+//       the block's start, e^{G_i - G_s(b)} x_i (<= 1), against the block's own
+//       operand B_b = e^{G_s(b) - G_j} k_j for j < 16 (b + 1): <= 1 for earlier
+//       blocks; inside block b the factor is e^{in-block decay}, used when that
+//       decay is >= -DECAY_LIM, and otherwise (a (block, channel) "bad" pair)
+//       the channel is left out of B_b and its 16 x 16 diagonal terms are added
+//       exactly in fp32 from running products of alpha (diag_fixup).
+// Every operand factor stays within e^{+-DECAY_LIM} (bf16 and fp32 reach e^88).
+// Byte offset of block b's operand tile ([KA][16 (b + 1)][128 B]) in the region.
+__device__ __forceinline__ uint32_t bt_off(int b, int KA) { return (uint32_t)(KA * 128 * bt_row0(b)); }
+
+// Tier-B Gram readout: 32 columns [32 hh, 32 hh + 32) of this lane's row r (0..63
+// within the k or the q rows), taken from the accumulator of the row's own 16-row
+// block.  The accumulator of block b sits at TMEM column col0 + bt_row0(b) and is
+// 16 (b + 1) wide; columns beyond it read a neighbour, but lie above the diagonal
+// and are masked by the caller.  quad: the warp's TMEM lane quadrant.
+__device__ __forceinline__ void gram_tier_b_ld32(uint32_t tl, uint32_t col0, int quad, int hh, int r,
+                                                 float (&v)[32]) {
+    const int bl = (quad & 1) * 2;   // the warp's rows cover blocks bl and bl + 1
+    if (hh == 1 && bl == 0) {        // rows 0..31: columns 32.. are above the diagonal
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = 0.f;
+        return;
+    }
+    const bool lo = (r >> 4) == bl;
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        float a[16], c[16];
+        ptx::tmem_ld16(tl + col0 + bt_row0(bl) + 32 * hh + 16 * p, a);
+        ptx::tmem_ld16(tl + col0 + bt_row0(bl + 1) + 32 * hh + 16 * p, c);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[16 * p + u] = lo ? a[u] : c[u];
+    }
+}
+
+// Adds fx (this lane's exact terms for columns 16 rb .. 16 rb + 15) into the
+// diagonal columns of its block's tier-B accumulator.  Warp-collective: the warp's
+// lanes cover blocks bl and bl + 1, so both column ranges are read and written back.
+__device__ __forceinline__ void diag_add(uint32_t tl, uint32_t col0, int quad, int rb, const float (&fx)[16]) {
+    const int bl = (quad & 1) * 2;
+    const uint32_t ca = tl + col0 + bt_row0(bl) + 16 * bl, cb = tl + col0 + bt_row0(bl + 1) + 16 * (bl + 1);
+    float va[16], vb[16];
+    ptx::tmem_ld16(ca, va);
+    ptx::tmem_ld16(cb, vb);
+    ptx::tmem_wait_ld();
+    uint32_t ua[16], ub[16];
+    const bool lo = rb == bl;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        ua[u] = __float_as_uint(lo ? va[u] + fx[u] : va[u]);
+        ub[u] = __float_as_uint(lo ? vb[u] : vb[u] + fx[u]);
+    }
+    ptx::tmem_st16(ca, ua);
+    ptx::tmem_st16(cb, ub);
+    ptx::tmem_wait_st();
+}
+
+// Exact diagonal-block terms of the channels left out of a tier-B operand: for
+// row i of block b and each channel c set in mask (NW words), for j = 16 b .. i,
+//   fx[j - 16 b] += x_ic k_jc prod_{t = j+1..i} alpha_tc
+// accumulated in fp32 from running products.  alpha(t, c), kv(t, c) and xv(c)
+// read the chunk's inputs (k and x zero, alpha anything, past the chunk end).
+template <int NW, class FA, class FK, class FX>
+__device__ __forceinline__ void diag_fixup(float (&fx)[16], const uint32_t *mask, int b, int i, FA alpha, FK kv,
+                                           FX xv) {
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) fx[jj] = 0.f;
+    const int j0 = 16 * b, il = i - j0;
+#pragma unroll 1
+    for (int w = 0; w < NW; ++w) {
+        uint32_t m = mask[w];
+#pragma unroll 1
+        while (m) {
+            const int c = 32 * w + __ffs(m) - 1;
+            m &= m - 1;
+            const float x = xv(c);
+            float P = 1.f;
+#pragma unroll
+            for (int hb = 1; hb >= 0; --hb) {   // j from i down to 16 b, eight at a time
+                float a[8], kk[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const bool on = 8 * hb + jj <= il;
+                    a[jj] = on ? alpha(j0 + 8 * hb + jj, c) : 0.f;
+                    kk[jj] = on ? kv(j0 + 8 * hb + jj, c) : 0.f;
+                }
+#pragma unroll
+                for (int jj = 7; jj >= 0; --jj) {
+                    if (8 * hb + jj <= il) {
+                        fx[8 * hb + jj] = fmaf(x * kk[jj], P, fx[8 * hb + jj]);
+                        P *= a[jj];
+                    }
+                }
+            }
+        }
+    }
+}
+
 // Every thread waits for the next completion of an mbarrier; all agree on the
 // outcome (a shared "failed" flag from warp-local waits is folded in).  Returns
 // false, and flags the device status, on timeout.
@@ -289,6 +411,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     using L = Layout<DK, DVT>;
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
     constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG;   // factor stage: 4 channels x SEGLEN tokens
+    constexpr int SPB = 16 / SEGLEN, NW = DK / 32;
     constexpr int CPT = DVT / 2;                              // state / output columns per thread
     constexpr float LOG2E = 1.4426950408889634f;
     extern __shared__ uint8_t smem_raw[];
@@ -299,6 +422,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *fM = reinterpret_cast<float *>(sm + L::FM);
     float *fB = reinterpret_cast<float *>(sm + L::FB);
     float *fSeg = reinterpret_cast<float *>(sm + L::FSEG);
+    uint32_t *bad = reinterpret_cast<uint32_t *>(sm + L::BAD);
     const uint32_t bar_mma = sb + L::MISC, bar_in = sb + L::MISC + 8, bar_v = sb + L::MISC + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 32);
     int *fail_flag = reinterpret_cast<int *>(sm + L::MISC + 36);
@@ -385,15 +509,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             beta_next = tid < Ln ? beta[(cs + C + tid) * H + h] : 0.f;
         }
 
-        // ---- 1. decay factors (one exp per element) -> Kp, Qp, Kbar; e^{G_last} S -> bf16 operand
+        // ---- 1. decay factors (one exp per element) -> the Gram operands (tier A or B), Kbar; S -> bf16 operand
         if (!(ok = wait_all(bar_in, ph_in))) break;
         float dch = 0.f;   // e^{G_last} of this thread's state row
+        bool tier_b;
         {
-            const int cg = tid % NCG, seg = tid / NCG, c0 = 4 * cg, i0 = seg * SEGLEN;
+            const int cg = tid % NCG, seg = tid / NCG, c0 = 4 * cg, i0 = seg * SEGLEN, blk = seg / SPB;
             const float *gin = reinterpret_cast<const float *>(sm + L::GIN);
             const uint8_t *qin = sm + L::QIN, *kin = sm + L::KIN;
             float al[SEGLEN][4];
             float4 sg = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (tid < 4 * NW) bad[tid] = 0u;
 #pragma unroll
             for (int u = 0; u < SEGLEN; ++u) {
                 float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -409,8 +535,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 al[u][0] = g4.x; al[u][1] = g4.y; al[u][2] = g4.z; al[u][3] = g4.w;
             }
             *reinterpret_cast<float4 *>(fSeg + seg * DK + c0) = sg;
-            __syncthreads();
-            float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+            // every segment sum >= -DECAY_LIM / NSEG proves every chunk sum >= -DECAY_LIM (tier A)
+            constexpr float SEG_LIM = -DECAY_LIM / NSEG;
+            const bool maybe_strong =
+                __syncthreads_or(sg.x < SEG_LIM || sg.y < SEG_LIM || sg.z < SEG_LIM || sg.w < SEG_LIM) != 0;
+            // pre = G before this segment, tot = G_last, gsb = G before this thread's 16-token block
+            float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f}, gsb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int s2 = 0; s2 < NSEG; ++s2) {
                 const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
@@ -418,11 +548,34 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     if (s2 < seg) pre[e] += xv[e];
+                    if (s2 < blk * SPB) gsb[e] += xv[e];
                     tot[e] += xv[e];
                 }
             }
-            if (seg == 0 && (tot[0] < -80.f || tot[1] < -80.f || tot[2] < -80.f || tot[3] < -80.f))
-                flag_status(KDA_DEV_DECAY_RANGE);
+            auto g_before = [&](int b, float (&gb)[4]) {   // G before block b (b = 4: G_last)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) gb[e] = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < NSEG; ++s2) {
+                    if (s2 >= b * SPB) break;
+                    const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
+                    gb[0] += x.x; gb[1] += x.y; gb[2] += x.z; gb[3] += x.w;
+                }
+            };
+            const bool strong =
+                tot[0] < -DECAY_LIM || tot[1] < -DECAY_LIM || tot[2] < -DECAY_LIM || tot[3] < -DECAY_LIM;
+            tier_b = maybe_strong && __syncthreads_or(strong) != 0;   // uniform over the CTA
+            if (tier_b && seg == 0) {
+#pragma unroll 1
+                for (int b = 0; b < 4; ++b) {
+                    float ga[4], gz[4];
+                    g_before(b, ga);
+                    g_before(b + 1, gz);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (gz[e] - ga[e] < -DECAY_LIM) atomicOr(&bad[b * NW + (c0 + e) / 32], 1u << ((c0 + e) & 31));
+                }
+            }
             if (has_row) {
                 float tr = 0.f;
 #pragma unroll
@@ -434,57 +587,180 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 4; ++e) al[u][e] = exp2_fast(al[u][e] * LOG2E);
             const float sgv[4] = {sg.x, sg.y, sg.z, sg.w};
-            // forward: ef = e^{G_i - G_last} (>= 1; bounded by e^80 under the range precondition)
-            float ef[4], eb[4];
+            // forward: rows e^{G_i - ref} [k_i; q_i] (<= 1), ref = 0 (tier A) or the block start (tier B)
+            {
+                float ef[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                ef[e] = exp2_fast((pre[e] - tot[e]) * LOG2E);
-                eb[e] = exp2_fast((tot[e] - pre[e] - sgv[e]) * LOG2E);
-            }
+                for (int e = 0; e < 4; ++e) ef[e] = exp2_fast((pre[e] - (tier_b ? gsb[e] : 0.f)) * LOG2E);
 #pragma unroll
-            for (int u = 0; u < SEGLEN; ++u) {
-                const int i = i0 + u;
-                float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < Lc) {
-                    q4 = ld_bf16x4(qin + (i * DK + c0) * 2);
-                    k4 = ld_bf16x4(kin + (i * DK + c0) * 2);
+                for (int u = 0; u < SEGLEN; ++u) {
+                    const int i = i0 + u;
+                    float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (i < Lc) {
+                        q4 = ld_bf16x4(qin + (i * DK + c0) * 2);
+                        k4 = ld_bf16x4(kin + (i * DK + c0) * 2);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) ef[e] *= al[u][e];
+                    st_bf16x4(sm, L::KQ + sw128(i, c0, 128), k4.x * ef[0], k4.y * ef[1], k4.z * ef[2], k4.w * ef[3]);
+                    st_bf16x4(sm, L::KQ + sw128(64 + i, c0, 128), q4.x * ef[0], q4.y * ef[1], q4.z * ef[2],
+                              q4.w * ef[3]);
                 }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) ef[e] *= al[u][e];
-                st_bf16x4(sm, L::KQ + sw128(i, c0, 128), k4.x * ef[0], k4.y * ef[1], k4.z * ef[2], k4.w * ef[3]);
-                st_bf16x4(sm, L::KQ + sw128(64 + i, c0, 128), q4.x * ef[0], q4.y * ef[1], q4.z * ef[2],
-                          q4.w * ef[3]);
             }
-            // backward: eb = e^{G_last - G_i} (<= 1)
+            // backward: rows e^{ref - G_j} k_j of a tile of `rows` rows (e0 at this segment's end)
+            auto store_cols = [&](uint32_t tile, int rows, float (&e0)[4]) {
 #pragma unroll
-            for (int u = SEGLEN - 1; u >= 0; --u) {
-                const int i = i0 + u;
-                float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < Lc) k4 = ld_bf16x4(kin + (i * DK + c0) * 2);
-                st_bf16x4(sm, L::KS + sw128(i, c0, L::KSR), k4.x * eb[0], k4.y * eb[1], k4.z * eb[2], k4.w * eb[3]);
+                for (int u = SEGLEN - 1; u >= 0; --u) {
+                    const int i = i0 + u;
+                    float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (i < Lc) k4 = ld_bf16x4(kin + (i * DK + c0) * 2);
+                    st_bf16x4(sm, tile + sw128(i, c0, rows), k4.x * e0[0], k4.y * e0[1], k4.z * e0[2], k4.w * e0[3]);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) eb[e] *= al[u][e];
+                    for (int e = 0; e < 4; ++e) e0[e] *= al[u][e];
+                }
+            };
+            {
+                float eb[4];   // tier A: e^{-G_j} (<= e^{DECAY_LIM}); tier B: Kbar, e^{G_last - G_j} (<= 1)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) eb[e] = exp2_fast(((tier_b ? tot[e] : 0.f) - pre[e] - sgv[e]) * LOG2E);
+                store_cols(L::KS, L::KSR, eb);
+            }
+            if (tier_b) {
+#pragma unroll 1
+                for (int b = blk; b < 4; ++b) {   // block b's operand holds tokens j < 16 (b + 1)
+                    float ga[4], gz[4], eB[4];
+                    g_before(b, ga);
+                    g_before(b + 1, gz);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const bool out = b == blk && gz[e] - ga[e] < -DECAY_LIM;   // bad pair: diag_fixup
+                        eB[e] = out ? 0.f : exp2_fast(fminf(ga[e] - pre[e] - sgv[e], DECAY_LIM) * LOG2E);
+                    }
+                    store_cols(L::RX + bt_off(b, DK / 64), 16 * (b + 1), eB);
+                }
             }
         }
         if (has_row) {
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::KS + sw128(64 + scol + j, srow, L::KSR), dch * S[j]);
+            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::KS + sw128(64 + scol + j, srow, L::KSR), S[j]);
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 2. [Gram | X; Y] = [Kp; Qp] [Kbar; e^{G_last} S^T]^T in one N = 64 + DVT MMA chain
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64 + DVT);
+        if (!tier_b) {
+            // ---- 2. [Gram | X; Y] = [e^G K; e^G Q] [e^{-G} K; S^T]^T in one N = 64 + DVT MMA chain
+            if (tid == 0) {
+                ptx::tc_fence_after();
+                constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64 + DVT);
 #pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KS, s, L::KSR), ig, s > 0);
-            ptx::mma_commit(bar_mma);
-            ++n_commit;
+                for (int s = 0; s < DK / 16; ++s)
+                    ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KS, s, L::KSR), ig, s > 0);
+                ptx::mma_commit(bar_mma);
+                ++n_commit;
+            }
+            if (!(ok = wait_all(bar_mma, ph_mma))) break;
+        } else {
+            // ---- 2B. Gram from the block-relative rows and the four block operands, then the
+            //          chunk-start rows e^G [K; Q] for [X; Y] = [e^G K; e^G Q] S
+            if (tid == 0) {
+                ptx::tc_fence_after();
+#pragma unroll 1
+                for (int b = 0; b < 4; ++b) {
+                    const int rows = 16 * (b + 1);
+                    const uint32_t ib = ptx::idesc_bf16_f32(128, rows);
+#pragma unroll
+                    for (int s = 0; s < DK / 16; ++s)
+                        ptx::mma_bf16(tmem + COL_BT + bt_row0(b), kdesc(sb + L::KQ, s, 128),
+                                      kdesc(sb + L::RX + bt_off(b, DK / 64), s, rows), ib, s > 0);
+                }
+                ptx::mma_commit(bar_mma);
+                ++n_commit;
+            }
+            if (!(ok = wait_all(bar_mma, ph_mma))) break;
+            {
+                const int cg = tid % NCG, seg = tid / NCG, c0 = 4 * cg, i0 = seg * SEGLEN;
+                const float *gin = reinterpret_cast<const float *>(sm + L::GIN);
+                const uint8_t *qin = sm + L::QIN, *kin = sm + L::KIN;
+                float ef[4] = {0.f, 0.f, 0.f, 0.f};   // G before this segment, then e^{G_i}
+#pragma unroll
+                for (int s2 = 0; s2 < NSEG; ++s2) {
+                    if (s2 >= seg) break;
+                    const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
+                    ef[0] += x.x; ef[1] += x.y; ef[2] += x.z; ef[3] += x.w;
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ef[e] = exp2_fast(ef[e] * LOG2E);
+#pragma unroll
+                for (int u = 0; u < SEGLEN; ++u) {
+                    const int i = i0 + u;
+                    float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (i < Lc) {
+                        q4 = ld_bf16x4(qin + (i * DK + c0) * 2);
+                        k4 = ld_bf16x4(kin + (i * DK + c0) * 2);
+                        if constexpr (GS) {
+                            const float gs = __ldg(g_scalar + (cs + i) * H + h);
+                            g4 = make_float4(gs, gs, gs, gs);
+                        } else {
+                            g4 = *reinterpret_cast<const float4 *>(gin + i * DK + c0);
+                        }
+                    }
+                    ef[0] *= exp2_fast(g4.x * LOG2E); ef[1] *= exp2_fast(g4.y * LOG2E);
+                    ef[2] *= exp2_fast(g4.z * LOG2E); ef[3] *= exp2_fast(g4.w * LOG2E);
+                    st_bf16x4(sm, L::KQ + sw128(i, c0, 128), k4.x * ef[0], k4.y * ef[1], k4.z * ef[2], k4.w * ef[3]);
+                    st_bf16x4(sm, L::KQ + sw128(64 + i, c0, 128), q4.x * ef[0], q4.y * ef[1], q4.z * ef[2],
+                              q4.w * ef[3]);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                ptx::tc_fence_after();
+                constexpr uint32_t ixy = ptx::idesc_bf16_f32(128, DVT);
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)
+                    ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KS, s, L::KSR, 64), ixy,
+                                  s > 0);
+                ptx::mma_commit(bar_mma);
+                ++n_commit;
+            }
+            // bad (block, channel) pairs: exact diagonal terms into the Gram accumulator,
+            // from the input tiles (still intact: the scratch overwrites them only in step 3)
+            if (warp < 4) {
+                const int r = tid & 63, rb = r >> 4;
+                const uint32_t *mk = bad + rb * NW;
+                bool fix = false;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) fix |= mk[w] != 0u;
+                if (__any_sync(0xffffffffu, fix)) {
+                    float fx[16];
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) fx[jj] = 0.f;
+                    if (fix) {
+                        const float *gin = reinterpret_cast<const float *>(sm + L::GIN);
+                        const __nv_bfloat16 *qin = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QIN);
+                        const __nv_bfloat16 *kin = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KIN);
+                        auto kval = [&](int t, int c) -> float { return t < Lc ? __bfloat162float(kin[t * DK + c]) : 0.f; };
+                        auto alpha = [&](int t, int c) -> float {
+                            if (t >= Lc) return 1.f;
+                            float g;
+                            if constexpr (GS) g = __ldg(g_scalar + (cs + t) * H + h);
+                            else g = gin[t * DK + c];
+                            return exp2_fast(g * LOG2E);
+                        };
+                        auto xval = [&](int c) -> float {
+                            if (r >= Lc) return 0.f;
+                            return __bfloat162float((warp < 2 ? kin : qin)[r * DK + c]);
+                        };
+                        diag_fixup<NW>(fx, mk, rb, r, alpha, kval, xval);
+                    }
+                    diag_add(tl, COL_BT, quad, rb, fx);
+                }
+            }
+            if (!(ok = wait_all(bar_mma, ph_mma))) break;   // [X; Y]; also orders the fixups before step 3
         }
-        if (!(ok = wait_all(bar_mma, ph_mma))) break;
 
         // ---- 3. Gram -> Diag(beta) Akk (fp32) -> diagonal blocks of T (warps 0-1);
         //        masked Aqk -> bf16 (warps 2-3); Z = V - X (warps 4-5); zero blocks of T (6-7)
@@ -492,8 +768,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 float g32[32];
-                ptx::tmem_ld32(tl + COL_GRAM + hh * 32, g32);
-                ptx::tmem_wait_ld();
+                if (!tier_b) {
+                    ptx::tmem_ld32(tl + COL_GRAM + hh * 32, g32);
+                    ptx::tmem_wait_ld();
+                } else {
+                    gram_tier_b_ld32(tl, COL_BT, quad, hh, tid, g32);
+                }
                 const int i = tid;
                 const float bi = fB[buf * C + i];
 #pragma unroll
@@ -513,8 +793,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 float g32[32];
-                ptx::tmem_ld32(tl + COL_GRAM + hh * 32, g32);
-                ptx::tmem_wait_ld();
+                if (!tier_b) {
+                    ptx::tmem_ld32(tl + COL_GRAM + hh * 32, g32);
+                    ptx::tmem_wait_ld();
+                } else {
+                    gram_tier_b_ld32(tl, COL_BT, quad, hh, tid - 64, g32);
+                }
                 const int i = tid - 64;
 #pragma unroll
                 for (int u = 0; u < 32; ++u) g32[u] = (hh * 32 + u <= i) ? g32[u] : 0.f;
@@ -588,13 +872,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!(ok = wait_all(bar_mma, ph_mma, *fail_flag))) break;
 
-        // ---- 5. Kt, Pt -> bf16 A operands
+        // ---- 5. Kt, Pt -> bf16 A operands (tier A: Kt rows take the factor e^{G_last})
         if (warp < DK / 32) {
+            const float dr = tier_b ? 1.f : dch;
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 float k32[32];
                 ptx::tmem_ld32(tl + COL_KT + hh * 32, k32);
                 ptx::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) k32[u] *= dr;
 #pragma unroll
                 for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::KP + sw128_chunk(srow, hh * 4 + gq), k32 + gq * 8);
             }

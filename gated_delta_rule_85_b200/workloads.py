@@ -15,6 +15,10 @@ Distributions (per the workload definitions):
   backward cotangents: d_o ~ N(0, 1) in the input dtype, dfinal_state ~ N(0, 1) fp32
   raw inputs (fused-prologue entry points): q, k ~ N(0, 1) not normalised, and the
               gate pre-activation gate_x ~ N(-2, 1), all in the input dtype
+  strong decay (strong_decay): parts of a gate tensor overwritten with fast
+              forgetting -- single-token hard resets (log_alpha = -100), whole
+              64-token chunks at log_alpha = -2, channels at -10 -- or, for a
+              gate pre-activation, the values x whose -softplus(x) is about those
 Every tensor is drawn from its own generator seeded with (seed, stream id), so
 one tensor's draw does not depend on another's size.  Large tensors are drawn
 in token slices of fixed size so device memory for temporaries stays bounded.
@@ -188,6 +192,46 @@ def prefill_inputs(shape: PrefillShape, seed: int = 0, device="cpu") -> dict:
     d["cu_seqlens"] = (None if shape.cu_seqlens is None
                        else torch.tensor(shape.cu_seqlens, dtype=torch.int32, device=device))
     return d
+
+
+STRONG_KINDS = ("reset", "minus2", "mixed")
+_STREAM_STRONG = 10
+
+
+def strong_decay(g: torch.Tensor, kind: str, seed: int, raw: bool = False) -> torch.Tensor:
+    """Overwrite parts of a gate tensor (in place; returned) with fast forgetting.
+
+    g is log_alpha [B, T, H, dk] (per channel) or [B, T, H] (one rate per
+    token-head), or with raw=True the gate pre-activation x [B, T, H, dk] of the
+    fused prologue, where x = 100, 10, 2 give -softplus(x) ~ -100, -10, -2.13.
+      reset   each entry independently with probability 1/32 becomes a hard reset (-100)
+      minus2  tokens [64, 192) of every row become -2 (whole chunks, summed -128 per chunk)
+      mixed   per channel gate: the first half of the channels -2 on every token, the next
+              eight -10, and resets with probability 1/64 in the rest; one rate per
+              token-head: tokens [0, 64) at -2 and resets with probability 1/16
+    """
+    if kind not in STRONG_KINDS:
+        raise ValueError(kind)
+    reset, m2, m10 = (100.0, 2.0, 10.0) if raw else (-100.0, -2.0, -10.0)
+    gen = _gen(g.device, seed, _STREAM_STRONG)
+    u = torch.empty(g.shape, dtype=torch.float32, device=g.device).uniform_(0.0, 1.0, generator=gen)
+    per_channel = g.dim() == 4
+    if kind == "reset":
+        g[u < 1 / 32] = reset
+    elif kind == "minus2":
+        g[:, 64:192] = m2
+    else:
+        if per_channel:
+            dk = g.shape[-1]
+            rest = torch.zeros(g.shape, dtype=torch.bool, device=g.device)
+            rest[..., dk // 2 + 8:] = True
+            g[rest & (u < 1 / 64)] = reset
+            g[..., : dk // 2] = m2
+            g[..., dk // 2: dk // 2 + 8] = m10
+        else:
+            g[u < 1 / 16] = reset
+            g[:, :64] = m2
+    return g
 
 
 def backward_cotangents(shape: PrefillShape, seed: int = 0, device="cpu", dfinal: bool = True) -> dict:

@@ -76,9 +76,8 @@ typedef enum kda_dtype {
 
 /* Device status word bits (kda_get_device_status). */
 #define KDA_DEV_WAIT_TIMEOUT 0x1u    /* a bounded on-chip wait gave up; that CTA's output is invalid */
-#define KDA_DEV_DECAY_RANGE 0x2u     /* tensor-core prefill: within one 64-token chunk a channel's
-                                        accumulated log-decay fell below -80; the factorised decay
-                                        operands lose range there (see kda_chunk_forward) */
+#define KDA_DEV_DECAY_RANGE 0x2u     /* reserved: no longer raised (the tensor-core prefill is exact
+                                        for any log_alpha <= 0; see kda_chunk_forward) */
 #define KDA_DEV_BAD_SLOT 0x4u        /* a state-slot table entry was outside [-1, num_slots); that
                                         sequence was treated as having no slot (see *_slots) */
 
@@ -105,10 +104,13 @@ typedef enum kda_dtype {
  *   workspace     device scratch of at least kda_chunk_forward_workspace_size()
  *                 bytes, 256-byte aligned (may be NULL when that size is 0)
  *
- * Precondition of the tensor-core path: for every chunk and channel the summed
- * log-decay over the chunk is >= -80 (alpha products stay above e^-80); below it
- * the chunk-start factorisation of the decay is out of fp32/bf16 range and the
- * call flags KDA_DEV_DECAY_RANGE.  The fp32 path has no such limit.
+ * Decay range: both paths are exact for every finite log_alpha <= 0, however
+ * strong (a channel may forget everything in one token).  The tensor-core path
+ * splits the pairwise decay e^{G_i - G_j} of a chunk into two bf16 operands whose
+ * factors stay within e^{+-80}: against the chunk start when every channel's
+ * decay summed over the chunk is >= -80, else against 16-token block starts, with
+ * the diagonal 16 x 16 terms of any block that decays by more than e^80 added in
+ * fp32.  Chunks of strong decay cost more (about four times the Gram products).
  */
 size_t kda_chunk_forward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
                                         int dtype, int chunk);

@@ -107,19 +107,24 @@ def test_status_requires_pointer(lib):
 REC128, REC64 = 58368, 33792   # two-pass workspace bytes per (chunk slot, head) at dk = 128 / 64
 
 
+def two_pass_ws(slots, H, rec):
+    """Records of every (chunk slot, head), then one mark byte each (rounded up to 256 bytes)."""
+    return slots * H * rec + (slots * H + 255) // 256 * 256
+
+
 def test_workspace_sizes(lib):
     f = lib.kda_chunk_forward_workspace_size_ex
     FUSED, TWO_PASS, AUTO = 1, 2, 0
     # slots = ceil(B*T / 64) + num_seqs
-    assert f(1, 8192, 32, 128, 128, 1, 0, 64, TWO_PASS) == (128 + 1) * 32 * REC128
+    assert f(1, 8192, 32, 128, 128, 1, 0, 64, TWO_PASS) == two_pass_ws(128 + 1, 32, REC128)
     assert f(1, 8192, 32, 128, 128, 1, 0, 64, FUSED) == 0
-    assert f(1, 8192, 32, 128, 128, 1, 0, 64, AUTO) == (128 + 1) * 32 * REC128     # 32 chains: two-pass
+    assert f(1, 8192, 32, 128, 128, 1, 0, 64, AUTO) == two_pass_ws(128 + 1, 32, REC128)     # 32 chains: two-pass
     assert f(1, 1 << 20, 32, 128, 128, 22, 0, 64, AUTO) == 0                         # 704 chains: fused
     assert f(1, 1 << 20, 8, 128, 128, 1, 0, 64, AUTO) == 0                           # > 4 GiB: fused
-    assert f(3, 100, 2, 64, 64, 3, 0, 64, TWO_PASS) == (5 + 3) * 2 * REC64
+    assert f(3, 100, 2, 64, 64, 3, 0, 64, TWO_PASS) == two_pass_ws(5 + 3, 2, REC64)
     assert f(1, 100, 2, 64, 64, 1, 1, 64, TWO_PASS) == 0                             # fp32 path
     assert f(2, 0, 2, 128, 128, 2, 0, 64, TWO_PASS) == 0                             # no tokens
-    assert lib.kda_chunk_forward_workspace_size(1, 8192, 32, 128, 128, 1, 0, 64) == (128 + 1) * 32 * REC128
+    assert lib.kda_chunk_forward_workspace_size(1, 8192, 32, 128, 128, 1, 0, 64) == two_pass_ws(128 + 1, 32, REC128)
 
 
 def prefill_ex(lib, algo, ws, wsb):
@@ -128,7 +133,7 @@ def prefill_ex(lib, algo, ws, wsb):
 
 
 def test_prefill_ex_rejects(lib):
-    need = (2 + 1) * 2 * REC128
+    need = two_pass_ws(2 + 1, 2, REC128)
     assert prefill_ex(lib, 7, A[8], need) == INVALID            # unknown algo
     assert prefill_ex(lib, 2, A[8], need - 1) == WORKSPACE      # workspace too small
     assert prefill_ex(lib, 2, None, 0) == WORKSPACE             # workspace missing
