@@ -7,7 +7,10 @@ fp32 initial state, 64-token chunks.  The decode workload (N=256 sequences,
 H=32, one token per step through kda_recurrent_step, fresh inputs per step) is
 timed in the same run and reported under "decode"; the backward of the
 prefill_8k workload (kda_chunk_backward) under "backward_8k"; the same prefill on raw
-inputs through the fused prologue under "prefill_prologue_8k".
+inputs through the fused prologue under "prefill_prologue_8k"; the 128k-token prefill
+(T=131072) under "prefill_128k"; the 1,048,576-token packed prefill under
+"prefill_varlen_1m" and the 256 decode steps of its 22 sequences under
+"decode_varlen_22".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -31,7 +34,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PREFILL = dict(B=1, T=8192, H=32, dk=128, dv=128)
+PREFILL_LONG = dict(B=1, T=131072, H=32, dk=128, dv=128)
 DECODE = dict(N=256, H=32, dk=128, dv=128, steps=1024)
+DECODE_VARLEN = dict(N=22, H=32, dk=128, dv=128, steps=256)
 CHUNK = 64
 # Algorithmic bytes per token-head: q, k, v (bf16) + log_alpha (fp32) + beta + o (bf16).
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 4 * 128 + 4 + 2 * 128          # 1540
@@ -52,7 +57,7 @@ PROLOGUE_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 2 * 128 + 4 + 2 * 128             
 # dram__bytes_write.sum) of the current kernels on these workloads; keyed by the kernels
 # one step runs.  A kernel set without a capture on its workload reports null.
 NCU_TRAFFIC = {
-    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.8e6 + 181.5e6 + 308.3e6 + 50.5e6,
+    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.8e6 + 181.3e6 + 308.3e6 + 50.5e6,
     # chunk_tc_kernel (--algo fused): captured before its timeout-path change, so reported null
     ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.2e6,
     # backward: all four kernels of one call; T=2048 captured, T=8192 scaled by the chunk slots (129 / 33)
@@ -79,7 +84,7 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.00025):
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
@@ -96,14 +101,27 @@ class ClockSampler:
         except Exception as e:  # noqa: BLE001
             self.error = str(e)
 
-    def _run(self):
+    def _sample(self):
         nv = self._nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
-            except Exception:  # noqa: BLE001
-                pass
+            self._sample()
+            time.sleep(self._period)
+
+    def poll(self, event):
+        """Sample from the calling thread until `event` (recorded after the timed
+        launches) has completed: a short region whose launches were enqueued while
+        the sampler thread waited for the interpreter still gets its samples."""
+        if self._h is None:
+            return
+        while not event.query():
+            self._sample()
             time.sleep(self._period)
 
     def __enter__(self):
@@ -197,6 +215,7 @@ def run_prefill(args, world, rank, dev):
             step()
             ends[i].record(stream)
         t_all1.record(stream)
+        clk.poll(t_all1)
         torch.cuda.synchronize(dev)
     _barrier(world)
     total_ms = t_all0.elapsed_time(t_all1)
@@ -253,7 +272,7 @@ def run_prefill_gdn(args, world, rank, dev):
         step()
     torch.cuda.synchronize(dev)
     stream = torch.cuda.current_stream(dev)
-    reps = max(5, min(args.steps, 50))
+    reps = 300
     _barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -289,7 +308,7 @@ def run_prefill_prologue(args, world, rank, dev):
         step()
     torch.cuda.synchronize(dev)
     stream = torch.cuda.current_stream(dev)
-    reps = max(5, min(args.steps, 50))
+    reps = 300
     _barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -363,7 +382,7 @@ def run_prefill_varlen(args, world, rank, dev):
         step()
     torch.cuda.synchronize(dev)
     stream = torch.cuda.current_stream(dev)
-    reps = 3
+    reps = 4
     _barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -378,6 +397,95 @@ def run_prefill_varlen(args, world, rank, dev):
     del d, o, fs
     return dict(ms=ms, tokens=shape.T, alg_bytes=alg_bytes, alg_flops=token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD,
                 seqs=shape.num_seqs, launches=reps * len(kernels), kernels=kernels)
+
+
+def run_prefill_long(args, world, rank, dev):
+    """The 128k-token prefill (B=1, T=131072, H=32, d=128), kda_chunk_forward (AUTO)."""
+    import torch
+
+    import gated_delta_rule_85_b200 as kda
+    from gated_delta_rule_85_b200.workloads import PrefillShape, prefill_inputs
+
+    shape = PrefillShape(**PREFILL_LONG, dtype=torch.bfloat16)
+    d = prefill_inputs(shape, seed=rank, device=dev)
+    o = torch.empty((1, shape.T, shape.H, shape.dv), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, shape.H, shape.dk, shape.dv), dtype=torch.float32, device=dev)
+    ws_n = kda.workspace_size(1, shape.T, shape.H, shape.dk, shape.dv, 1)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev) if ws_n else None
+    kernels = ["chunk_intra_kernel", "chunk_inter_kernel"] if ws_n else ["chunk_tc_kernel"]
+
+    def step():
+        kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], o=o, final_state=fs,
+                          workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    reps = 16
+    _barrier(world)
+    with ClockSampler(dev.index) as clk:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    token_heads = shape.T * shape.H
+    alg_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * shape.H * STATE_BYTES
+    del d, o, fs, ws
+    return dict(ms=ms, tokens=shape.T, alg_bytes=alg_bytes, alg_flops=token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD,
+                launches=reps * len(kernels), kernels=kernels, clocks=clk.summary(), reps=reps)
+
+
+def run_decode_varlen(args, world, rank, dev):
+    """256 decode steps of the 22 packed sequences of the 1M-token workload, one CUDA
+    graph per 256 steps (states ~93 MB: L2-resident, launch-bound)."""
+    import torch
+
+    import gated_delta_rule_85_b200 as kda
+    from gated_delta_rule_85_b200.workloads import DecodeShape, decode_all_steps
+
+    shape = DecodeShape(**DECODE_VARLEN, dtype=torch.bfloat16)
+    d = decode_all_steps(shape, seed=rank, device=dev)
+    state = d["state"]
+    o = torch.empty((shape.N, shape.H, shape.dv), dtype=torch.bfloat16, device=dev)
+
+    def run_all():
+        for s in range(shape.steps):
+            kda.recurrent_step(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["beta"][s], state, o=o)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        run_all()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_all()
+    torch.cuda.synchronize(dev)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    reps = 40
+    stream = torch.cuda.current_stream(dev)
+    _barrier(world)
+    with ClockSampler(dev.index) as clk:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if not torch.isfinite(state).all():
+        raise RuntimeError("non-finite decode state")
+    del g, d, state
+    return dict(ms=ms, launches=reps * shape.steps, clocks=clk.summary())
 
 
 def run_decode(args, world, rank, dev, pool_slots=0):
@@ -540,6 +648,8 @@ def main(argv=None):
     ap.add_argument("--no-gdn", action="store_true", help="skip the Gated DeltaNet (scalar gate) prefill line")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward (gradients) line")
     ap.add_argument("--no-prologue", action="store_true", help="skip the fused-prologue (raw inputs) prefill line")
+    ap.add_argument("--no-long", action="store_true", help="skip the 128k-token prefill line")
+    ap.add_argument("--no-varlen-decode", action="store_true", help="skip the 22-sequence decode line")
     ap.add_argument("--only-backward", action="store_true",
                     help="time only the backward and print its line (profiling a smaller --backward-T)")
     ap.add_argument("--backward-T", type=int, default=PREFILL["T"], help="tokens of the backward workload")
@@ -582,6 +692,8 @@ def main(argv=None):
     gd = None if args.no_gdn else run_prefill_gdn(args, world, rank, dev)
     bw = None if args.no_backward else run_backward(args, world, rank, dev)
     pr = None if args.no_prologue else run_prefill_prologue(args, world, rank, dev)
+    lg = None if args.no_long else run_prefill_long(args, world, rank, dev)
+    dv22 = None if args.no_varlen_decode else run_decode_varlen(args, world, rank, dev)
 
     hbm_gbs, bf16_tflops, peak_src = _peaks()
     ms_step = pre["total_ms"] / args.steps
@@ -595,7 +707,10 @@ def main(argv=None):
     tflops = alg_flops / (launch_ms * 1e-3) / 1e12
     line = {
         "metric": "KDA chunked prefill tokens/s (B=1, T=8192, H=32, d=128)",
-        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "value": value, "unit": "tokens/s",
+        # the decode half of the metric up front (its full block is "decode" below)
+        "decode_tokens_per_s": None, "decode_ms_per_step": None, "decode_hbm_frac": None,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic", "config": config_block(args.algo),
         "roofline": {"kernel": " + ".join(pre["kernels"]), "bound": "hbm", "achieved": gbs, "peak": hbm_gbs,
@@ -626,6 +741,9 @@ def main(argv=None):
             "clocks": dec["clocks"],
         }
         line["gpu_launches"] += dec["launches"]
+        line["decode_tokens_per_s"] = line["decode"]["value"]
+        line["decode_ms_per_step"] = step_ms
+        line["decode_hbm_frac"] = dgbs / hbm_gbs
     if gd is not None:
         gbytes = token_heads * (PREFILL_BYTES_PER_TOKEN_HEAD - 4 * 128 + 4) + 2 * PREFILL["H"] * STATE_BYTES
         ggbs = gbytes / (gd["ms"] * 1e-3) / 1e9
@@ -682,6 +800,34 @@ def main(argv=None):
                          "tensor": {"achieved_tflops": vtf, "peak_tflops": bf16_tflops, "frac": vtf / bf16_tflops}},
         }
         line["gpu_launches"] += vl["launches"]
+    if lg is not None:
+        lgbs = lg["alg_bytes"] / (lg["ms"] * 1e-3) / 1e9
+        ltf = lg["alg_flops"] / (lg["ms"] * 1e-3) / 1e12
+        line["prefill_128k"] = {
+            "metric": "KDA chunked prefill tokens/s (B=1, T=131072, H=32, d=128)",
+            "value": world * lg["tokens"] / (lg["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": lg["ms"],
+            "steps": lg["reps"],
+            "roofline": {"kernel": " + ".join(lg["kernels"]), "bound": "hbm", "achieved": lgbs, "peak": hbm_gbs,
+                         "unit": "GB/s", "frac": lgbs / hbm_gbs, "traffic": None, "algorithmic_bytes": lg["alg_bytes"],
+                         "tensor": {"achieved_tflops": ltf, "peak_tflops": bf16_tflops, "frac": ltf / bf16_tflops}},
+            "clocks": lg["clocks"],
+        }
+        line["gpu_launches"] += lg["launches"]
+    if dv22 is not None:
+        step_ms = dv22["ms"] / dv22["launches"]
+        n22 = DECODE_VARLEN["N"] * DECODE_VARLEN["H"]
+        vbytes = n22 * DECODE_BYTES_PER_PAIR
+        line["decode_varlen_22"] = {
+            "metric": "KDA decode tokens/s after the 1M-token packed prefill (22 sequences, H=32, d=128, "
+                      "256 steps per CUDA graph)",
+            "value": world * DECODE_VARLEN["N"] / (step_ms * 1e-3), "unit": "tokens/s", "ms_per_step": step_ms,
+            "steps": dv22["launches"], "graph": "256 steps per CUDA graph replay",
+            "roofline": None,
+            "note": f"launch-bound: {vbytes / 1e6:.0f} MB of state per step stays in the 126 MB L2; "
+                    f"{vbytes / (step_ms * 1e-3) / 1e9:.0f} GB/s of state traffic, no roofline claim",
+            "clocks": dv22["clocks"],
+        }
+        line["gpu_launches"] += dv22["launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(heads=32)
     if rank == 0:

@@ -40,17 +40,11 @@ struct Rec {
 
 inline long long chunk_slots(long long tokens, int num_seqs) { return (tokens + C - 1) / C + num_seqs; }
 
-// Workspace: the records [slot][H] of the first pass, then one byte per (slot, head)
-// marking the chunks left to the tier-B kernel.
-inline size_t two_pass_records_bytes(long long tokens, int H, int dk, int num_seqs) {
+// Workspace: the records [slot][H] of the first pass.
+inline size_t two_pass_workspace_bytes(long long tokens, int H, int dk, int num_seqs) {
     if (tokens <= 0) return 0;
     const size_t rec = dk == 64 ? (size_t)Rec<64>::BYTES : (size_t)Rec<128>::BYTES;
     return (size_t)chunk_slots(tokens, num_seqs) * (size_t)H * rec;
-}
-inline size_t two_pass_workspace_bytes(long long tokens, int H, int dk, int num_seqs) {
-    if (tokens <= 0) return 0;
-    const size_t marks = ((size_t)chunk_slots(tokens, num_seqs) * (size_t)H + 255) / 256 * 256;
-    return two_pass_records_bytes(tokens, H, dk, num_seqs) + marks;
 }
 
 // First token of sequence n (clamped like seq_span).
@@ -168,17 +162,15 @@ __device__ __noinline__ void intra_fixup(uint32_t tl, int quad, int warp, int r,
 // log_alpha points to the bf16 gate pre-activation x [tokens, H, DK],
 // log_alpha = -softplus(x).
 // One (chunk slot, head) of the first pass.  TB = false: tier A only -- a chunk
-// that needs tier B is only marked in `flags` (1; 0 for every other slot) and left
-// to chunk_intra_strong_kernel.  TB = true: tier B.  All threads of the CTA call
-// it; ph_mma carries the MMA mbarrier phase across calls.  Returns false when a
-// bounded wait ran out.
+// that needs tier B is left at once (returns 1) for intra_chunk_strong.  TB = true:
+// tier B.  All threads of the CTA call it; ph_mma carries the MMA mbarrier phase.
+// Returns 0 when done (or the slot has no chunk) and -1 when a bounded wait ran out.
 template <int DK, bool GS, bool PRO, bool TB>
-__device__ __forceinline__ bool intra_chunk(int slot, int h, const __nv_bfloat16 *__restrict__ q,
-                                            const __nv_bfloat16 *__restrict__ k,
-                                            const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                                            const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
-                                            uint8_t *__restrict__ ws, uint8_t *__restrict__ flags, uint8_t *sm,
-                                            uint32_t tmem, uint32_t &ph_mma) {
+__device__ __forceinline__ int intra_chunk(int slot, int h, const __nv_bfloat16 *__restrict__ q,
+                                           const __nv_bfloat16 *__restrict__ k,
+                                           const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                                           const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
+                                           uint8_t *__restrict__ ws, uint8_t *sm, uint32_t tmem, uint32_t &ph_mma) {
     using L = IntraLayout<DK>;
     using R = Rec<DK>;
     constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG, SPB = 16 / SEGLEN, NW = DK / 32;
@@ -196,10 +188,7 @@ __device__ __forceinline__ bool intra_chunk(int slot, int h, const __nv_bfloat16
     long long t0, t1;
     seq_span(cu_seqlens, T, lo, t0, t1);
     const long long cs = t0 + (long long)(slot - (lo + t0 / C)) * C;
-    if (cs < t0 || cs >= t1) {   // slot without a chunk
-        if (!TB && tid == 0) flags[(size_t)slot * H + h] = 0;
-        return true;
-    }
+    if (cs < t0 || cs >= t1) return 0;   // slot without a chunk
     const int Lc = (int)min((long long)C, t1 - cs);
     const uint32_t sb = ptx::smem_u32(sm);
     float *fA = reinterpret_cast<float *>(sm + L::FA);
@@ -314,12 +303,8 @@ __device__ __forceinline__ bool intra_chunk(int slot, int h, const __nv_bfloat16
         if (maybe_strong) {
             const bool strong =
                 tot[0] < -DECAY_LIM || tot[1] < -DECAY_LIM || tot[2] < -DECAY_LIM || tot[3] < -DECAY_LIM;
-            if (__syncthreads_or(strong)) {   // uniform over the CTA: leave this chunk to tier B
-                if (tid == 0) flags[(size_t)slot * H + h] = 1;
-                return true;
-            }
+            if (__syncthreads_or(strong)) return 1;   // uniform over the CTA: tier B
         }
-        if (tid == 0) flags[(size_t)slot * H + h] = 0;
     }
     const float sgv[4] = {sg.x, sg.y, sg.z, sg.w};
     if (seg == 0) {
@@ -543,16 +528,30 @@ __device__ __forceinline__ bool intra_chunk(int slot, int h, const __nv_bfloat16
         if (!ok) ptx::mbar_wait_bounded(bar_mma, ph_mma ^ 1u, WAIT_LIMIT_CYCLES);   // MMAs still in flight
         ptx::bulk_wait_all();
     }
-    return ok;
+    return ok ? 0 : -1;
 }
 
-// First pass, tier A: one CTA per (chunk slot, head).
+// Tier B of one chunk, kept out of line so that its code does not weigh on the
+// register allocation of the common (tier-A) path.
+template <int DK, bool GS, bool PRO>
+__device__ __noinline__ int intra_chunk_strong(int slot, int h, const __nv_bfloat16 *__restrict__ q,
+                                               const __nv_bfloat16 *__restrict__ k,
+                                               const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                                               const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
+                                               uint8_t *__restrict__ ws, uint8_t *sm, uint32_t tmem, uint32_t *ph_mma) {
+    uint32_t ph = *ph_mma;
+    const int r = intra_chunk<DK, GS, PRO, true>(slot, h, q, k, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws, sm,
+                                                 tmem, ph);
+    *ph_mma = ph;
+    return r;
+}
+
+// First pass: one CTA per (chunk slot, head); tier A inline, tier B out of line.
 template <int DK, bool GS, bool PRO>
 __global__ void __launch_bounds__(NT, 2)
 chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                   const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, uint8_t *__restrict__ ws,
-                   uint8_t *__restrict__ flags) {
+                   const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, uint8_t *__restrict__ ws) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t bar_mma = ptx::smem_u32(sm) + IntraLayout<DK>::MISC;
@@ -570,54 +569,12 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     uint32_t ph_mma = 0;
-    intra_chunk<DK, GS, PRO, false>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta, cu_seqlens, T, H,
-                                    num_seqs, ws, flags, sm, tmem, ph_mma);
-    ptx::tc_fence_before();
-    __syncthreads();
-    if ((threadIdx.x >> 5) == 0) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, INTRA_TMEM_COLS);
-    }
-}
-
-// First pass, tier B: the chunks chunk_intra_kernel marked, one CTA per SM walking
-// the (slot, head) marks; nothing to do (and quick) when no chunk decays that fast.
-template <int DK, bool GS, bool PRO>
-__global__ void __launch_bounds__(NT, 1)
-chunk_intra_strong_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                          const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                          const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
-                          uint8_t *__restrict__ ws, uint8_t *__restrict__ flags, long long items) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const uint32_t bar_mma = ptx::smem_u32(sm) + IntraLayout<DK>::MISC;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + IntraLayout<DK>::MISC + 8);
-    __shared__ int s_any;
-    if (threadIdx.x == 0) s_any = 0;
-    __syncthreads();
-    for (long long it = blockIdx.x + (long long)threadIdx.x * gridDim.x; it < items; it += (long long)blockDim.x * gridDim.x)
-        if (flags[it]) s_any = 1;
-    __syncthreads();
-    if (!s_any) return;   // no marked chunk for this CTA
-    if ((threadIdx.x >> 5) == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTRA_TMEM_COLS);
-        ptx::tmem_relinquish();
-    }
-    if (threadIdx.x == 0) {
-        ptx::mbar_init(bar_mma, 1);
-        ptx::fence_mbar_init();
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    uint32_t ph_mma = 0;
-    for (long long it = blockIdx.x; it < items; it += gridDim.x) {
-        if (!flags[it]) continue;   // uniform: every thread reads the same mark
-        __syncthreads();            // the previous chunk's last shared-memory reads are done
-        if (!intra_chunk<DK, GS, PRO, true>((int)(it / H), (int)(it % H), q, k, log_alpha, beta, cu_seqlens, T, H,
-                                            num_seqs, ws, flags, sm, tmem, ph_mma))
-            break;
+    const int r = intra_chunk<DK, GS, PRO, false>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta,
+                                                  cu_seqlens, T, H, num_seqs, ws, sm, tmem, ph_mma);
+    if (r == 1) {   // the chunk decays faster than tier A covers (uniform over the CTA)
+        __syncthreads();
+        intra_chunk_strong<DK, GS, PRO>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta, cu_seqlens, T, H,
+                                        num_seqs, ws, sm, tmem, &ph_mma);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -849,18 +806,6 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
 
 // ------------------------------------------------------------------ host side
 
-// Multiprocessor count of the current device (148 on B200), looked up once per device.
-inline int sm_count() {
-    static int cached[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cached[dev]) {
-        int n = 0;
-        cached[dev] = (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) ? n : 148;
-    }
-    return cached[dev];
-}
-
 template <int DK, int DVT, bool GS, bool PRO>
 int launch_two_pass_t(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                       const float *init_state, void *o, float *final_state, const int32_t *cu_seqlens,
@@ -877,7 +822,6 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         return KDA_ERR_UNSUPPORTED;
     }
     constexpr int smem1 = IntraLayout<DK>::ALLOC;
-    uint8_t *marks = (uint8_t *)workspace + two_pass_records_bytes(tokens, H, DK, num_seqs);
     auto k1 = chunk_intra_kernel<DK, GS, PRO>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
     if (e != cudaSuccess) {
@@ -885,25 +829,10 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         return KDA_ERR_CUDA;
     }
     k1<<<dim3((unsigned)rec_slots, H), NT, smem1, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
-                                                     beta, cu_seqlens, T, H, num_seqs, (uint8_t *)workspace, marks);
+                                                     beta, cu_seqlens, T, H, num_seqs, (uint8_t *)workspace);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "chunk_intra launch: %s", cudaGetErrorString(e));
-        return KDA_ERR_CUDA;
-    }
-    auto k1b = chunk_intra_strong_kernel<DK, GS, PRO>;
-    e = cudaFuncSetAttribute(k1b, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
-    if (e != cudaSuccess) {
-        snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_intra_strong): %s", cudaGetErrorString(e));
-        return KDA_ERR_CUDA;
-    }
-    const long long items = rec_slots * H;
-    const int ctas = (int)std::min<long long>(items, (long long)sm_count());
-    k1b<<<ctas, NT, smem1, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha, beta, cu_seqlens, T, H,
-                                 num_seqs, (uint8_t *)workspace, marks, items);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) {
-        snprintf(msg, msg_len, "chunk_intra_strong launch: %s", cudaGetErrorString(e));
         return KDA_ERR_CUDA;
     }
     constexpr int NBUF = inter_nbuf<DK, DVT>();

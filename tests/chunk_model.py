@@ -78,3 +78,73 @@ def chunked_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, 
                 o[c0:c1, h] = O
             fs[n, h] = S
     return o.reshape(B, T, H, dv), fs
+
+
+# ---------------------------------------------------------------------------
+# The tensor-core kernels' split of the Gram's pairwise decay into two operand
+# factors (bf16 operands, fp32 exponents), in the two tiers they choose per chunk.
+
+DECAY_LIM = 80.0
+
+
+def bf16_round(x):
+    """Round to bfloat16 (nearest even) and widen back to float64."""
+    x = np.asarray(x, np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def exact_gram(q, k, g):
+    """[Akk; Aqk] rows (k rows then q rows) x 64 columns: sum_c x_ic k_jc e^{G_ic - G_jc} for j <= i."""
+    C = k.shape[0]
+    G = np.cumsum(np.asarray(g, np.float64), 0)
+    out = np.zeros((2 * C, C))
+    x = np.concatenate([k, q], 0)
+    for r in range(2 * C):
+        i = r % C
+        for j in range(i + 1):
+            out[r, j] = np.sum(x[r] * k[j] * np.exp(G[i] - G[j]))
+    return out
+
+
+def tiered_gram(q, k, g):
+    """The same Gram as the kernels compute it.  Tier A (every channel's chunk
+    decay >= -DECAY_LIM): e^{G_i} x_i against e^{-G_j} k_j.  Tier B: per 16-token
+    block b, rows scaled from the block start against e^{G_s(b) - G_j} k_j for
+    j < 16 (b + 1); channels whose in-block decay passes -DECAY_LIM are left out of
+    the block's own columns and their diagonal terms added in fp32 from running
+    products of alpha.  Returns (gram, tier)."""
+    C, D = k.shape
+    g = np.asarray(g, np.float32)
+    G = np.cumsum(g, 0, dtype=np.float32)
+    x = np.concatenate([k, q], 0)
+    Gx = np.concatenate([G, G], 0)
+    if np.all(G[-1] >= -DECAY_LIM):
+        A = bf16_round(np.exp(Gx) * x)
+        B = bf16_round(np.exp(-G) * k)
+        return A @ B.T, "A"
+    Gs = np.zeros((5, D), np.float32)
+    for b in range(1, 5):
+        Gs[b] = G[16 * b - 1]
+    Gs[4] = G[-1]
+    bad = (Gs[1:] - Gs[:4]) < -DECAY_LIM                     # [block, channel]
+    blk = (np.arange(2 * C) % C) // 16
+    A = bf16_round(np.exp(Gx - Gs[blk]) * x)
+    gram = np.zeros((2 * C, C))
+    for b in range(4):
+        n = 16 * (b + 1)
+        Bb = np.exp(np.minimum(Gs[b][None, :] - G[:n], DECAY_LIM)) * k[:n]
+        Bb[16 * b:n][:, bad[b]] = 0.0
+        Db = A @ bf16_round(Bb).T
+        gram[blk == b, :n] = Db[blk == b]
+    alpha = np.exp(g).astype(np.float32)
+    for r in range(2 * C):
+        i = r % C
+        b = i // 16
+        for c in np.nonzero(bad[b])[0]:
+            P = np.float32(1.0)
+            for j in range(i, 16 * b - 1, -1):
+                gram[r, j] += np.float32(x[r, c]) * np.float32(k[j, c]) * P
+                P = np.float32(P * alpha[j, c])
+    return gram, "B"

@@ -108,8 +108,8 @@ REC128, REC64 = 58368, 33792   # two-pass workspace bytes per (chunk slot, head)
 
 
 def two_pass_ws(slots, H, rec):
-    """Records of every (chunk slot, head), then one mark byte each (rounded up to 256 bytes)."""
-    return slots * H * rec + (slots * H + 255) // 256 * 256
+    """One record per (chunk slot, head)."""
+    return slots * H * rec
 
 
 def test_workspace_sizes(lib):
