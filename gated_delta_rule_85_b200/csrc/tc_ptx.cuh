@@ -210,6 +210,19 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint3
     return d;
 }
 
+// Descriptor of an MN-major bf16 operand whose rows (one K index each) are 64 bytes
+// (32 MN elements) in the 64-byte swizzle: 8 K rows form a 512-byte swizzle atom,
+// K atoms are `sbo` bytes apart, 32-element MN blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw64(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;                       // layout: 64-byte swizzle
+    return d;
+}
+
 // Instruction descriptor: kind::f16 with bf16 A and B, fp32 D; A and B K-major
 // unless a_mn / b_mn select MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false, bool b_mn = false) {
