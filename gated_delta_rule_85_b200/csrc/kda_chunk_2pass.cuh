@@ -621,20 +621,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
     constexpr int CPT = DVT / 2;
     constexpr uint32_t TX = (uint32_t)(R::BYTES + C * DVT * 2);
-    // MN-major operand rows: 64 bytes (32 columns, 64-byte swizzle) at DVT = 32,
-    // else 128 bytes (64 columns, 128-byte swizzle) per column block
-    constexpr int RB = DVT >= 64 ? 128 : 64, NB = RB / 2;
-    // byte offset of the 16-byte group holding columns n .. n+7 of operand row k (rows per column block `krows`)
-    auto mn_off = [](int k, int n, int krows) -> uint32_t {
-        const int blk = n / NB, g = (n % NB) / 8;
-        const int sg = RB == 128 ? (g ^ (k & 7)) : (g ^ ((k >> 1) & 3));
-        return (uint32_t)(blk * krows * RB + k * RB + sg * 16);
-    };
-    // descriptor of K step s (16 rows) of an MN-major operand with `krows` rows per column block
-    auto mn_desc = [](uint32_t addr, int s, int krows) -> uint64_t {
-        return RB == 128 ? ptx::desc_mnmajor_sw128(addr + s * 16 * RB, krows * RB, 8 * RB)
-                         : ptx::desc_mnmajor_sw64(addr + s * 16 * RB, krows * RB, 8 * RB);
-    };
+    using MN = MnOp<DVT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = ptx::smem_u32(sm);
@@ -709,7 +696,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
         if (has_row) {
 #pragma unroll
             for (int g = 0; g < CPT / 8; ++g)
-                *reinterpret_cast<uint4 *>(sm + L::SP + mn_off(srow, scol + 8 * g, DK)) =
+                *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) =
                     make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
                                pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
         }
@@ -723,7 +710,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
             constexpr uint32_t ix = ptx::idesc_bf16_f32(128, DVT, false, true);
 #pragma unroll
             for (int s = 0; s < DK / 16; ++s)
-                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KQ, s, 128), mn_desc(sb + L::SP, s, DK), ix, s > 0);
+                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KQ, s, 128), MN::desc(sb + L::SP, s, DK), ix, s > 0);
             ptx::mma_commit(bar_mma);
             ++n_commit;
         }
@@ -747,7 +734,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int g = 0; g < 2; ++g)
-                    *reinterpret_cast<uint4 *>(sm + L::ZT + mn_off(j, scol + cc * 16 + 8 * g, C)) = make_uint4(
+                    *reinterpret_cast<uint4 *>(sm + L::ZT + MN::off(j, scol + cc * 16 + 8 * g, C)) = make_uint4(
                         pack_bf16(v16[8 * g] - x16[8 * g], v16[8 * g + 1] - x16[8 * g + 1]),
                         pack_bf16(v16[8 * g + 2] - x16[8 * g + 2], v16[8 * g + 3] - x16[8 * g + 3]),
                         pack_bf16(v16[8 * g + 4] - x16[8 * g + 4], v16[8 * g + 5] - x16[8 * g + 5]),
@@ -764,10 +751,10 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
             constexpr uint32_t iz = ptx::idesc_bf16_f32(128, DVT, false, true);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + XCOL_DS, kdesc(rb + R::KP, s, DK + 64), mn_desc(sb + L::ZT, s, C), iz, s > 0);
+                ptx::mma_bf16(tmem + XCOL_DS, kdesc(rb + R::KP, s, DK + 64), MN::desc(sb + L::ZT, s, C), iz, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KP, s, DK + 64, DK - 64), mn_desc(sb + L::ZT, s, C), iz, 1);
+                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C), iz, 1);
             ptx::mma_commit(bar_mma);
             ++n_commit;
         }

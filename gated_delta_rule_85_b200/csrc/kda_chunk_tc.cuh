@@ -66,13 +66,12 @@ struct Layout {
     // bf16 MMA operands, 128-byte swizzled, 1024-byte aligned
     static constexpr int KQ = 0;                             // [KA][128][128 B] e^G K (0-63), e^G Q (64-127);
                                                              //   tier B: the block-relative rows first
-    static constexpr int KSR = 64 + DVT;                     // rows of the combined B operand
-    static constexpr int KS = KQ + KA * 128 * 128;           // [KA][64+DVT][128 B] rows 0-63: tier A e^{-G} K,
-                                                             //   tier B Kbar (tokens); rows 64..: S^T (value columns)
-    static constexpr int RX = KS + KA * KSR * 128;           // Kt/Pt, Tb^T, Z^T; tier B: block operands B_0..B_3
+    static constexpr int KB = KQ + KA * 128 * 128;           // [KA][64][128 B] tier A e^{-G} K, tier B Kbar (tokens)
+    static constexpr int SB = KB + KA * 64 * 128;            // bf16 S, MN-major (key rows = K, value columns = N)
+    static constexpr int RX = SB + DK * DVT * 2;             // Kt/Pt, Tb^T, Z; tier B: block operands B_0..B_3
     static constexpr int KP = RX;                            //   [DK+64][128 B] Kt (0..DK-1), Aqk -> Pt (DK..)
     static constexpr int TB = KP + (DK + 64) * 128;          //   [64][128 B]    Tb^T
-    static constexpr int ZT = TB + 64 * 128;                 //   [DVT][128 B]   Z^T
+    static constexpr int ZT = TB + 64 * 128;                 //   bf16 Z, MN-major (tokens = K, value columns = N)
     static constexpr int RX_USE = ZT + DVT * 128 - RX;
     static constexpr int BT_BYTES = KA * BT_ROWS * 128;
     static constexpr int RX_BYTES = ((RX_USE > BT_BYTES ? RX_USE : BT_BYTES) + 1023) / 1024 * 1024;
@@ -94,7 +93,8 @@ struct Layout {
     static constexpr int MISC = BAD + 4 * (DK / 32) * 4;     // mbarriers, TMEM base, flags
     static constexpr int BYTES = MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;               // room to align the base to 1024 B
-    static_assert(KQ % 1024 == 0 && KS % 1024 == 0 && KP % 1024 == 0 && TB % 1024 == 0 && ZT % 1024 == 0 &&
+    static_assert(KQ % 1024 == 0 && KB % 1024 == 0 && SB % 1024 == 0 && KP % 1024 == 0 && TB % 1024 == 0 &&
+                      ZT % 1024 == 0 &&
                       QIN % 1024 == 0 && VIN % 128 == 0,
                   "tile alignment");
     static_assert(ALLOC <= 232448, "shared memory budget");
@@ -110,6 +110,26 @@ __device__ __forceinline__ uint32_t sw128(int row, int k, int rows) {
 __device__ __forceinline__ uint32_t sw128_chunk(int row, int g) {
     return (uint32_t)(row * 128 + ((g ^ (row & 7)) << 4));
 }
+
+// bf16 MN-major operand of DVT columns (N) by `krows` rows (K): rows of 64 bytes
+// (32 columns, 64-byte swizzle) at DVT = 32, else 128 bytes (64 columns, 128-byte
+// swizzle) per column block; a thread that holds consecutive columns of one row
+// writes them as 16-byte groups.
+template <int DVT>
+struct MnOp {
+    static constexpr int RB = DVT >= 64 ? 128 : 64, NB = RB / 2;
+    // byte offset of the 16-byte group holding columns n .. n+7 of row k
+    static __device__ __forceinline__ uint32_t off(int k, int n, int krows) {
+        const int blk = n / NB, g = (n % NB) / 8;
+        const int sg = RB == 128 ? (g ^ (k & 7)) : (g ^ ((k >> 1) & 3));
+        return (uint32_t)(blk * krows * RB + k * RB + sg * 16);
+    }
+    // descriptor of K step s (16 rows)
+    static __device__ __forceinline__ uint64_t desc(uint32_t addr, int s, int krows) {
+        return RB == 128 ? ptx::desc_mnmajor_sw128(addr + s * 16 * RB, krows * RB, 8 * RB)
+                         : ptx::desc_mnmajor_sw64(addr + s * 16 * RB, krows * RB, 8 * RB);
+    }
+};
 
 __device__ __forceinline__ void st_bf16(uint8_t *base, uint32_t off, float x) {
     *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
@@ -623,7 +643,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float eb[4];   // tier A: e^{-G_j} (<= e^{DECAY_LIM}); tier B: Kbar, e^{G_last - G_j} (<= 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) eb[e] = exp2_fast(((tier_b ? tot[e] : 0.f) - pre[e] - sgv[e]) * LOG2E);
-                store_cols(L::KS, L::KSR, eb);
+                store_cols(L::KB, 64, eb);
             }
             if (tier_b) {
 #pragma unroll 1
@@ -642,20 +662,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (has_row) {
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) st_bf16(sm, L::KS + sw128(64 + scol + j, srow, L::KSR), S[j]);
+            for (int g = 0; g < CPT / 8; ++g)
+                *reinterpret_cast<uint4 *>(sm + L::SB + MnOp<DVT>::off(srow, scol + 8 * g, DK)) =
+                    make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
+                               pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
 
         if (!tier_b) {
-            // ---- 2. [Gram | X; Y] = [e^G K; e^G Q] [e^{-G} K; S^T]^T in one N = 64 + DVT MMA chain
+            // ---- 2. Gram = [e^G K; e^G Q] (e^{-G} K)^T and [X; Y] = [e^G K; e^G Q] S (S MN-major)
             if (tid == 0) {
                 ptx::tc_fence_after();
-                constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64 + DVT);
+                constexpr uint32_t ig = ptx::idesc_bf16_f32(128, 64);
+                constexpr uint32_t ixy = ptx::idesc_bf16_f32(128, DVT, false, true);
 #pragma unroll
                 for (int s = 0; s < DK / 16; ++s)
-                    ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KS, s, L::KSR), ig, s > 0);
+                    ptx::mma_bf16(tmem + COL_GRAM, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KB, s, 64), ig, s > 0);
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)
+                    ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KQ, s, 128), MnOp<DVT>::desc(sb + L::SB, s, DK), ixy,
+                                  s > 0);
                 ptx::mma_commit(bar_mma);
                 ++n_commit;
             }
@@ -718,10 +746,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             __syncthreads();
             if (tid == 0) {
                 ptx::tc_fence_after();
-                constexpr uint32_t ixy = ptx::idesc_bf16_f32(128, DVT);
+                constexpr uint32_t ixy = ptx::idesc_bf16_f32(128, DVT, false, true);
 #pragma unroll
                 for (int s = 0; s < DK / 16; ++s)
-                    ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KQ, s, 128), kdesc(sb + L::KS, s, L::KSR, 64), ixy,
+                    ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KQ, s, 128), MnOp<DVT>::desc(sb + L::SB, s, DK), ixy,
                                   s > 0);
                 ptx::mma_commit(bar_mma);
                 ++n_commit;
@@ -824,7 +852,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < 16; ++u) st_bf16(sm, L::ZT + sw128(cc * 16 + u, j, DVT), v16[u] - x16[u]);
+                for (int g = 0; g < 2; ++g)
+                    *reinterpret_cast<uint4 *>(sm + L::ZT + MnOp<DVT>::off(j, cc * 16 + 8 * g, C)) = make_uint4(
+                        pack_bf16(v16[8 * g] - x16[8 * g], v16[8 * g + 1] - x16[8 * g + 1]),
+                        pack_bf16(v16[8 * g + 2] - x16[8 * g + 2], v16[8 * g + 3] - x16[8 * g + 3]),
+                        pack_bf16(v16[8 * g + 4] - x16[8 * g + 4], v16[8 * g + 5] - x16[8 * g + 5]),
+                        pack_bf16(v16[8 * g + 6] - x16[8 * g + 6], v16[8 * g + 7] - x16[8 * g + 7]));
             }
         } else {
             // blocks (0,1) and (2,3) of T are read by the merge products as zeros;
@@ -861,7 +894,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t ipt = ptx::idesc_bf16_f32(128, 64);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + COL_KT, ptx::desc_mnmajor_sw128(sb + L::KS + s * 2048, L::KSR * 128, 1024),
+                ptx::mma_bf16(tmem + COL_KT, ptx::desc_mnmajor_sw128(sb + L::KB + s * 2048, 64 * 128, 1024),
                               kdesc(sb + L::TB, s, 64), ikt, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
@@ -903,13 +936,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ---- 6. dS = Kt Z ; O = Y + Pt Z (accumulated onto the Y rows of [X; Y])
         if (tid == 0) {
             ptx::tc_fence_after();
-            constexpr uint32_t iz = ptx::idesc_bf16_f32(128, DVT);
+            constexpr uint32_t iz = ptx::idesc_bf16_f32(128, DVT, false, true);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + COL_DS, kdesc(sb + L::KP, s, DK + 64), kdesc(sb + L::ZT, s, DVT), iz, s > 0);
+                ptx::mma_bf16(tmem + COL_DS, kdesc(sb + L::KP, s, DK + 64), MnOp<DVT>::desc(sb + L::ZT, s, C), iz, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KP, s, DK + 64, DK - 64), kdesc(sb + L::ZT, s, DVT), iz, 1);
+                ptx::mma_bf16(tmem + COL_XY, kdesc(sb + L::KP, s, DK + 64, DK - 64), MnOp<DVT>::desc(sb + L::ZT, s, C), iz,
+                              1);
             ptx::mma_commit(bar_mma);
             ++n_commit;
         }
