@@ -98,6 +98,10 @@ def load_library():
     lib.kda_gdn_chunk_backward.restype = ci
     lib.kda_chunk_backward_workspace_size.argtypes = [ci] * 6
     lib.kda_chunk_backward_workspace_size.restype = sz
+    lib.kda_chunk_backward_workspace_size_ex.argtypes = [ci] * 8
+    lib.kda_chunk_backward_workspace_size_ex.restype = sz
+    lib.kda_chunk_backward_ex.argtypes = lib.kda_chunk_backward.argtypes + [ci]
+    lib.kda_chunk_backward_ex.restype = ci
     lib.kda_last_error.argtypes = []
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci, vp]
@@ -278,8 +282,17 @@ def recurrent_step_prologue(q_raw, k_raw, v, gate_x, beta, state, o=None):
     return o
 
 
-def backward_workspace_size(B, T, H, dk, dv, num_seqs) -> int:
-    return int(load_library().kda_chunk_backward_workspace_size(B, T, H, dk, dv, num_seqs))
+BACKWARD_ALGOS = {"auto": 0, "tensor": 1, "simt": 2}   # KDA_BWD_AUTO, KDA_BWD_TENSOR, KDA_BWD_SIMT
+
+
+def backward_workspace_size(B, T, H, dk, dv, num_seqs, dtype=None, algo="auto") -> int:
+    """Workspace bytes of kda_chunk_backward: enough for any schedule when dtype is
+    None, else what the schedule `algo` takes for that dtype (torch dtype)."""
+    lib = load_library()
+    if dtype is None:
+        return int(lib.kda_chunk_backward_workspace_size(B, T, H, dk, dv, num_seqs))
+    code = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}[dtype]
+    return int(lib.kda_chunk_backward_workspace_size_ex(B, T, H, dk, dv, num_seqs, code, BACKWARD_ALGOS[algo]))
 
 
 def gdn_chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=None, cu_seqlens=None, *,
@@ -293,7 +306,7 @@ def gdn_chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_st
 
 
 def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=None, cu_seqlens=None, *,
-                   dinit_state=True, workspace=None, out=None, _gate_scalar=False):
+                   dinit_state=True, workspace=None, out=None, algo="auto", _gate_scalar=False):
     """Gradients of sum <d_o, o> + <dfinal_state, final_state> through the chunked
     prefill (kda_chunk_backward): a dict with dq, dk, dv (in q's dtype),
     dlog_alpha, dbeta and dinit_state (float32; None when dinit_state=False).
@@ -301,7 +314,9 @@ def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=
     Inputs are the forward call's, in the include/kda.h layouts; d_o has o's
     shape and dtype, dfinal_state is float32 [N, H, dk, dv] or None (zero).
     The workspace (uint8, CUDA) and the outputs (`out`, a dict with any of the
-    keys above) are allocated here unless given.  Device tensors only.
+    keys above) are allocated here unless given.  algo: "auto", "tensor" or
+    "simt" (kda_chunk_backward_ex; the Gated DeltaNet backward takes "auto").
+    Device tensors only.
     """
     gate = SimpleNamespace(shape=q.shape, dtype=log_alpha.dtype) if _gate_scalar else log_alpha
     B, T, H, dk, dv, N = _prefill_args(q, k, v, gate, beta, init_state, cu_seqlens)
@@ -323,14 +338,22 @@ def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=
     else:
         g["dinit_state"] = None
     _need_cuda(*g.values())
-    need = int(lib.kda_chunk_backward_workspace_size(B, T, H, dk, dv, N))
+    if algo not in BACKWARD_ALGOS or (_gate_scalar and algo != "auto"):
+        raise ValueError(f"unknown backward algo {algo!r}")
+    if _gate_scalar:
+        need = int(lib.kda_chunk_backward_workspace_size(B, T, H, dk, dv, N))
+    else:
+        need = int(lib.kda_chunk_backward_workspace_size_ex(B, T, H, dk, dv, N, _dtype_code(q), BACKWARD_ALGOS[algo]))
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    entry = lib.kda_gdn_chunk_backward if _gate_scalar else lib.kda_chunk_backward
-    rc = entry(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(d_o), _p(dfinal_state), _p(g["dq"]),
-               _p(g["dk"]), _p(g["dv"]), _p(g["dlog_alpha"]), _p(g["dbeta"]), _p(g["dinit_state"]), _p(cu_seqlens),
-               B, T, H, dk, dv, N, _dtype_code(q), CHUNK, _p(workspace), ws_bytes, _stream(dev))
+    args = (_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(d_o), _p(dfinal_state), _p(g["dq"]),
+            _p(g["dk"]), _p(g["dv"]), _p(g["dlog_alpha"]), _p(g["dbeta"]), _p(g["dinit_state"]), _p(cu_seqlens),
+            B, T, H, dk, dv, N, _dtype_code(q), CHUNK, _p(workspace), ws_bytes, _stream(dev))
+    if _gate_scalar:
+        rc = lib.kda_gdn_chunk_backward(*args)
+    else:
+        rc = lib.kda_chunk_backward_ex(*args, BACKWARD_ALGOS[algo])
     _check(rc)
     return g
 

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libkda.so")
 SOURCES = ["kda_lib.cu"]
 DEPS = ["kda_common.cuh", "kda_decode.cuh", "kda_chunk_simt.cuh", "kda_chunk_tc.cuh", "kda_chunk_2pass.cuh",
-        "kda_bwd_simt.cuh", "tc_ptx.cuh"]
+        "kda_bwd_simt.cuh", "kda_bwd_tc.cuh", "tc_ptx.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

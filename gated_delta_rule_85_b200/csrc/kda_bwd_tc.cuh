@@ -1,0 +1,947 @@
+// KDA backward on the tensor cores (tcgen05, bf16 operands, fp32 accumulators in
+// TMEM) for bf16 inputs with dk = dv = 128.
+//
+// The chunk form of the forward ("Kimi Linear、独自の土俵でFull Attentionを上回る"
+// (remio.ai), § "Kimi Linearがより賢いRecurrent Memoryを使う方法": chunkwise
+// training on the diagonal-plus-low-rank transition), with per chunk (C = 64
+// tokens) G the running sum of log_alpha, Khat = e^G K, Qhat = e^G Q,
+// Kbar = e^{G_last - G} K, D = e^{G_last}, Akk (j < i), Aqk (j <= i),
+// T = (I + Diag(beta) Akk)^{-1}, Tb = T Diag(beta), Kt = Kbar^T Tb, Pt = Aqk Tb:
+//   W = V - Khat S,  U = Tb W,  S' = Diag(D) S + Kbar^T U,  O = Qhat S + Aqk U.
+// Differentiated, with dO and dS' (the adjoint of the state after the chunk):
+//   dU = Aqk^T dO + Kbar dS',  lam = T^T dU,  mu = Diag(beta) lam = Pt^T dO + Kt^T dS',
+//   dV = mu,  dbeta_i = <lam_i, W_i - (Akk U)_i>,
+//   dAqk = dO U^T (j <= i),  dAkk = -Diag(beta) lam U^T (j < i),
+//   dQhat = dO S^T,  dKhat = -mu S^T,  dKbar = U dS'^T,
+//   dS = Diag(D) dS' + Qhat^T dO - Khat^T mu,
+// then the chain rule through the decay factors and a reverse running sum for
+// dlog_alpha.  Five launches:
+//   1. chunk_intra_kernel<BX>: the forward's first pass, plus Akk, Aqk and T;
+//   2. chunk_inter_kernel<CK>: the forward's state sweep, storing each chunk's
+//      starting state (bf16) instead of the output;
+//   3. chunk_adj_kernel: the adjoint sweep, chunks in reverse, storing each
+//      chunk's ending adjoint (bf16) and dS_0;
+//   4. bwd_grad_kernel (per chunk, head): every product above that needs S or
+//      dS', in a transposed form whose 128 rows are value or key channels
+//      (W^T, U^T, dU^T, lam^T: M = dv; the sums over the value columns: M = dk);
+//   5. bwd_chain_kernel (per chunk, head): the pair terms of dAqk and dAkk through
+//      e^{G_i - G_j} and the chain rule -> dq, dk, dlog_alpha.
+#pragma once
+
+#include <cstring>
+
+#include "kda_chunk_2pass.cuh"
+
+namespace kda {
+namespace tc {
+
+// ------------------------------------------------------------------ adjoint sweep
+
+template <int DK, int DVT, int NBUF>
+struct AdjLayout {
+    static constexpr int KA = DK / 64;
+    static constexpr int REC = Rec<DK>::BYTES;
+    static constexpr int SP = NBUF * REC;                 // bf16 dS, MN-major (K = key rows, N = value columns)
+    static constexpr int MU = SP + KA * DVT * 128;        // bf16 -mu, MN-major (K = tokens, N = value columns)
+    static constexpr int DOT = MU + DVT * 128;            // bf16 [NBUF] dO tiles [64][DVT], MN-major (TMA swizzle)
+    static constexpr int MISC = DOT + NBUF * C * DVT * 2; // mbarriers, TMEM base
+    static constexpr int BYTES = MISC + 64;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(REC % 1024 == 0 && SP % 1024 == 0 && MU % 1024 == 0 && DOT % 1024 == 0, "tile alignment");
+};
+
+constexpr uint32_t ACOL_MU = 0;     // [128 x DVT] mu (lanes 0-63; lanes 64-127 unused)
+constexpr uint32_t ACOL_DS = 128;   // [128 x DVT] Qhat^T dO - Khat^T mu
+
+// One CTA per (value tile, head, sequence), chunks from the last to the first.
+// Per chunk: mu = Pt^T dO + Kt^T dS' (M = 128 over a 64-row operand: the A
+// descriptor's second 64-row half reads neighbouring bytes, whose rows are
+// ignored), then dS = Diag(D) dS' + [Khat^T Qhat^T] [-mu; dO] (M = dk).
+// dS' of each chunk (its end) goes to the unit's DSC tile; dS_0 to dinit_state.
+template <int DK, int DVT, int NBUF>
+__global__ void __launch_bounds__(NT, 1)
+chunk_adj_kernel(const __grid_constant__ CUtensorMap tm_do, uint8_t *__restrict__ ws,
+                 const float *__restrict__ dfinal, float *__restrict__ dinit_state,
+                 const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
+    using L = AdjLayout<DK, DVT, NBUF>;
+    using R = Rec<DK>;
+    using U = BwdUnit<DK>;
+    static_assert(DK == 128 && (DVT == 32 || DVT == 64), "tile shape");
+    constexpr int CPT = DVT / 2;
+    constexpr uint32_t TX = (uint32_t)(R::BYTES + C * DVT * 2);
+    using MN = MnOp<DVT>;
+    using M64 = MnOp<64>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = ptx::smem_u32(sm);
+    const uint32_t bar_rec = sb + L::MISC, bar_mma = sb + L::MISC + 32;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 40);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int col_base = blockIdx.x * DVT, h = blockIdx.y;
+    const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
+    long long t0, t1;
+    seq_span(cu_seqlens, T, n, t0, t1);
+    const int nck = (int)((t1 - t0 + C - 1) / C);
+    const long long first = n + t0 / C;
+
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTER_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int b = 0; b < NBUF; ++b) ptx::mbar_init(bar_rec + 8 * b, 1);
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+        if (nck > 0) ptx::prefetch_tmap(&tm_do);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t ph_mma = 0, ph_rec = 0;
+    int n_issued = 0, n_commit = 0;
+
+    auto issue = [&](int t) {   // thread 0: record and dO tile of step t (chunk nck - 1 - t) into buffer t % NBUF
+        const int b = t % NBUF, ci = nck - 1 - t;
+        n_issued = t + 1;
+        const uint32_t bar = bar_rec + 8 * b;
+        ptx::mbar_arrive_expect_tx(bar, TX);
+        ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * U::BYTES, (uint32_t)R::BYTES, bar);
+        ptx::tma_load_3d(sb + L::DOT + b * C * DVT * 2, &tm_do, bar, col_base, h, (int)(t0 + (long long)ci * C));
+    };
+
+    const int srow = quad * 32 + lane;
+    const int scol = half * CPT;
+    const long long st_off = ((long long)n * H + h) * DK * DV + col_base + scol;
+    float S[CPT];   // dS' (fp32), this thread's row and columns
+#pragma unroll
+    for (int j = 0; j < CPT; j += 4) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (dfinal) x = load4(dfinal + st_off + (long long)srow * DV + j);
+        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+    }
+    if (tid == 0)
+        for (int t = 0; t < NBUF && t < nck; ++t) issue(t);
+
+    bool ok = true;
+    for (int t = 0; t < nck; ++t) {
+        const int ci = nck - 1 - t, b = t % NBUF;
+        const uint32_t rb = sb + b * R::BYTES, dob = sb + L::DOT + b * C * DVT * 2;
+        uint32_t ph = (ph_rec >> b) & 1u;
+        ok = wait_all(bar_rec + 8 * b, ph);
+        ph_rec ^= 1u << b;
+        if (!ok) break;
+
+        // ---- 1. dS' -> bf16 B operand and the unit's checkpoint
+        const float dch = reinterpret_cast<const float *>(sm + b * R::BYTES + R::DCH)[srow];
+        {
+            uint8_t *ck = ws + ((size_t)(first + ci) * H + h) * U::BYTES + U::DSC;
+#pragma unroll
+            for (int g = 0; g < CPT / 8; ++g) {
+                const uint4 w = make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
+                                           pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
+                *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) = w;
+                *reinterpret_cast<uint4 *>(ck + sw128(srow, col_base + scol + 8 * g, DK)) = w;
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- 2. mu = Pt^T dO + Kt^T dS'  (A: MN-major views of the record's [Kt; Pt] rows)
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t im = ptx::idesc_bf16_f32(128, DVT, true, true);
+            const uint32_t kp = rb + R::KP;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + ACOL_MU, ptx::desc_mnmajor_sw128(kp + (DK + 16 * s) * 128, 2048, 1024),
+                              MN::desc(dob, s, C), im, s > 0);
+#pragma unroll
+            for (int s = 0; s < DK / 16; ++s)
+                ptx::mma_bf16(tmem + ACOL_MU, ptx::desc_mnmajor_sw128(kp + s * 2048, 2048, 1024),
+                              MN::desc(sb + L::SP, s, DK), im, 1);
+            ptx::mma_commit(bar_mma);
+            ++n_commit;
+        }
+        if (!(ok = wait_all(bar_mma, ph_mma))) break;
+
+        // ---- 3. -mu (TMEM lanes 0-63) -> bf16 B operand rows
+        if (quad < 2) {
+            const int j = quad * 32 + lane;
+#pragma unroll 1
+            for (int cc = 0; cc < CPT / 16; ++cc) {
+                float x16[16];
+                ptx::tmem_ld16(tl + ACOL_MU + scol + cc * 16, x16);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int g = 0; g < 2; ++g)
+                    *reinterpret_cast<uint4 *>(sm + L::MU + MN::off(j, scol + cc * 16 + 8 * g, C)) =
+                        make_uint4(pack_bf16(-x16[8 * g], -x16[8 * g + 1]), pack_bf16(-x16[8 * g + 2], -x16[8 * g + 3]),
+                                   pack_bf16(-x16[8 * g + 4], -x16[8 * g + 5]),
+                                   pack_bf16(-x16[8 * g + 6], -x16[8 * g + 7]));
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- 4. Khat^T (-mu) + Qhat^T dO  (A: MN-major view of the record's [Khat; Qhat] rows)
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t id = ptx::idesc_bf16_f32(128, DVT, true, true);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + ACOL_DS, M64::desc(rb + R::KQ, s, 128), MN::desc(sb + L::MU, s, C), id, s > 0);
+#pragma unroll
+            for (int s = 4; s < 8; ++s)
+                ptx::mma_bf16(tmem + ACOL_DS, M64::desc(rb + R::KQ, s, 128), MN::desc(dob, s - 4, C), id, 1);
+            ptx::mma_commit(bar_mma);
+            ++n_commit;
+        }
+        if (!(ok = wait_all(bar_mma, ph_mma))) break;
+        if (tid == 0 && t + NBUF < nck) issue(t + NBUF);   // buffer b fully consumed
+
+        // ---- 5. dS <- Diag(D) dS' + (4)
+#pragma unroll
+        for (int cc = 0; cc < CPT / 16; ++cc) {
+            float d16[16];
+            ptx::tmem_ld16(tl + ACOL_DS + scol + cc * 16, d16);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
+        }
+        ptx::tc_fence_before();
+    }
+
+    if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded), then leave
+        for (int b = 0; b < NBUF; ++b) {
+            const int arms = n_issued > b ? (n_issued - 1 - b) / NBUF + 1 : 0;
+            if (arms > 0) ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((arms - 1) & 1), WAIT_LIMIT_CYCLES);
+        }
+        if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
+    }
+    __syncthreads();
+    if (ok && dinit_state) {
+#pragma unroll
+        for (int j = 0; j < CPT; j += 4)
+            store4(dinit_state + st_off + (long long)srow * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, INTER_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ per-chunk sums
+
+// Chunk of `slot`: the last sequence n whose first slot n + floor(t0_n / 64) is
+// <= slot owns it.  False for a slot without a chunk (uniform over the CTA).
+__device__ __forceinline__ bool slot_chunk(const int32_t *cu_seqlens, int T, int num_seqs, int slot, long long &cs,
+                                           int &Lc) {
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (mid + seq_begin(cu_seqlens, T, mid) / C <= slot) lo = mid;
+        else hi = mid - 1;
+    }
+    long long t0, t1;
+    seq_span(cu_seqlens, T, lo, t0, t1);
+    cs = t0 + (long long)(slot - (lo + t0 / C)) * C;
+    if (cs < t0 || cs >= t1) return false;
+    Lc = (int)min((long long)C, t1 - cs);
+    return true;
+}
+
+// Running sum G of log_alpha over one chunk, per (token, channel), for the 8 tokens x
+// 4 channels of this thread (tokens 8 seg.., channels 4 cg..; 256 threads): rows
+// past Lc count as log_alpha = 0 and k = q = 0.  fSeg: [8][128] fp32 scratch.
+// Returns the thread's G values, k (and q) rows as bf16 pairs, and G_last.
+template <bool WITH_Q>
+__device__ __forceinline__ void chunk_decay(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                                            const float *__restrict__ log_alpha, long long cs, int Lc, int H, int h,
+                                            float *fSeg, float (&G)[8][4], uint2 (&kv)[8], uint2 (&qv)[8],
+                                            float (&tot)[4]) {
+    constexpr int DK = 128;
+    const int tid = threadIdx.x, cg = tid & 31, seg = tid >> 5, c0 = 4 * cg, i0 = 8 * seg;
+    float4 gv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const long long off = ((cs + min(i0 + u, Lc - 1)) * H + h) * DK + c0;
+        gv[u] = __ldg(reinterpret_cast<const float4 *>(log_alpha + off));
+        kv[u] = __ldg(reinterpret_cast<const uint2 *>(k + off));
+        if constexpr (WITH_Q) qv[u] = __ldg(reinterpret_cast<const uint2 *>(q + off));
+    }
+    float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const bool in = i0 + u < Lc;
+        const float g4[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            run[e] += in ? g4[e] : 0.f;
+            G[u][e] = run[e];
+        }
+        if (!in) {
+            kv[u] = make_uint2(0u, 0u);
+            qv[u] = make_uint2(0u, 0u);
+        }
+    }
+    *reinterpret_cast<float4 *>(fSeg + seg * DK + c0) = make_float4(run[0], run[1], run[2], run[3]);
+    __syncthreads();
+    float pre[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) tot[e] = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < 8; ++s2) {
+        const float4 x = *reinterpret_cast<const float4 *>(fSeg + s2 * DK + c0);
+        const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (s2 < seg) pre[e] += xv[e];
+            tot[e] += xv[e];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) G[u][e] += pre[e];
+}
+
+// Sum over the 32 lanes of a warp of x[j] for each j: lane l ends with the sum of
+// element l (a butterfly that halves the vector at each step, 31 shuffles).
+__device__ __forceinline__ float warp_transpose_sum32(float (&x)[32]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const bool up = (lane & w) != 0;
+#pragma unroll
+        for (int u = 0; u < w; ++u) {
+            const float send = up ? x[u] : x[u + w];
+            const float keep = up ? x[u + w] : x[u];
+            x[u] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+    }
+    return x[0];
+}
+
+struct GradLayout {   // dk = dv = 128; bf16 tiles with a 128-byte swizzle unless noted
+    static constexpr int KH = 0;                // [2][64][128 B]   Khat rows (K-major B, N = tokens)
+    static constexpr int EX = 16384;            // BwdX             Akk | Aqk | T
+    static constexpr int SS = 40960;            // [2][128][128 B]  S at the chunk's start
+    static constexpr int DS = 73728;            // [2][128][128 B]  dS' at its end
+    static constexpr int DOL = 106496;          // [2][128][128 B]  dO rows 0-63 (TMA), lam rows 64-127
+    static constexpr int KBR = 139264;          // [2][64][128 B]   Kbar rows (K-major B, N = tokens)
+    static constexpr int VV = 155648;           // [64][128]        V, no swizzle
+    static constexpr int AW = 172032;           // [128][128 B]     (Diag(beta) W)^T, then U^T
+    static constexpr int ADU = 188416;          // [128][128 B]     dU^T, then -mu rows [2][64][128 B]
+    static constexpr int FB = 204800;           // fp32 [64]        beta
+    static constexpr int FD = FB + 256;         // fp32 [128]       e^{G_last}
+    static constexpr int FSEG = FD + 512;       // fp32 [8][128]    segment sums
+    static constexpr int FDB = FSEG + 4096;     // fp32 [4][64]     <lam, W> per lane quadrant
+    static constexpr int FDB2 = FDB + 1024;     // fp32 [2][64]     sum_j Akk L per column half
+    static constexpr int FGC = FDB2 + 512;      // fp32 [2][128]    sum_v S dS' per column half
+    static constexpr int MISC = FGC + 1024;     // mbarriers, TMEM base
+    static constexpr int BYTES = MISC + 64;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(ALLOC <= 232448, "shared memory budget");
+};
+
+constexpr uint32_t GRAD_TMEM_COLS = 256;
+// TMEM columns, 64 each: phase 1 W-part and dU^T; phase 2 U^T, lam^T; phase 3
+// [dAqk; L], S dO^T, -S mu^T, dS' U^T
+constexpr uint32_t GC_0 = 0, GC_1 = 64, GC_2 = 128, GC_3 = 192;
+
+// One CTA per (chunk slot, head), 256 threads.  Warps w and w + 4 share TMEM lane
+// quadrant w & 3 (value channel or key channel 32 (w & 3) + lane) and split the 64
+// token columns in halves.  Writes dV and dbeta, and over the chunk's own unit the
+// sums XQ, XK, XB, the masked dAkk/dAqk tile and DGC for bwd_chain_kernel.
+__global__ void __launch_bounds__(NT, 1)
+bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_v,
+                const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
+                const float *__restrict__ beta, __nv_bfloat16 *__restrict__ dv_out, float *__restrict__ dbeta,
+                const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, uint8_t *__restrict__ ws) {
+    using L = GradLayout;
+    using R = Rec<128>;
+    using U = BwdUnit<128>;
+    constexpr int DK = 128, DV = 128;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = ptx::smem_u32(sm);
+    const uint32_t bar_ld = sb + L::MISC, bar_mma = sb + L::MISC + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 16);
+    float *fB = reinterpret_cast<float *>(sm + L::FB), *fD = reinterpret_cast<float *>(sm + L::FD);
+    float *fSeg = reinterpret_cast<float *>(sm + L::FSEG), *fDB = reinterpret_cast<float *>(sm + L::FDB);
+    float *fDB2 = reinterpret_cast<float *>(sm + L::FDB2), *fGC = reinterpret_cast<float *>(sm + L::FGC);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, half = warp >> 2;
+    const int slot = blockIdx.x, h = blockIdx.y;
+    long long cs;
+    int Lc;
+    if (!slot_chunk(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
+    uint8_t *unit = ws + ((size_t)slot * H + h) * U::BYTES;
+
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), GRAD_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (tid == 0) {
+        ptx::mbar_init(bar_ld, 1);
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+        ptx::mbar_arrive_expect_tx(bar_ld, 16384u + (uint32_t)BwdX::BYTES + 2u * 32768u + 16384u + 16384u);
+        ptx::bulk_load(sb + L::KH, unit + R::KQ, 8192u, bar_ld);                 // Khat rows of atom 0
+        ptx::bulk_load(sb + L::KH + 8192, unit + R::KQ + 16384, 8192u, bar_ld);  // and of atom 1
+        ptx::bulk_load(sb + L::EX, unit + U::BXO, (uint32_t)BwdX::BYTES, bar_ld);
+        ptx::bulk_load(sb + L::SS, unit + U::SC, 32768u, bar_ld);
+        ptx::bulk_load(sb + L::DS, unit + U::DSC, 32768u, bar_ld);
+        ptx::tma_load_3d(sb + L::DOL, &tm_do, bar_ld, 0, h, (int)cs);
+        ptx::tma_load_3d(sb + L::DOL + 16384, &tm_do, bar_ld, 64, h, (int)cs);
+        ptx::tma_load_3d(sb + L::VV, &tm_v, bar_ld, 0, h, (int)cs);
+    }
+    if (tid < C) fB[tid] = tid < Lc ? beta[(cs + tid) * H + h] : 0.f;
+    {   // Kbar = e^{G_last - G} K (factors <= 1) and e^{G_last}, while the copies fly
+        float G[8][4], tot[4];
+        uint2 kv[8], qv[8];
+        chunk_decay<false>(nullptr, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
+        const int c0 = 4 * (tid & 31), i0 = 8 * (tid >> 5);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float4 k4 = bf16x4_to_float4(kv[u]);
+            st_bf16x4(sm, L::KBR + sw128(i0 + u, c0, 64), k4.x * __expf(tot[0] - G[u][0]),
+                      k4.y * __expf(tot[1] - G[u][1]), k4.z * __expf(tot[2] - G[u][2]), k4.w * __expf(tot[3] - G[u][3]));
+        }
+        if (tid < 32) *reinterpret_cast<float4 *>(fD + c0) = make_float4(__expf(tot[0]), __expf(tot[1]),
+                                                                         __expf(tot[2]), __expf(tot[3]));
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t ph_ld = 0, ph_mma = 0;
+    int n_commit = 0;
+    bool ok = wait_all(bar_ld, ph_ld);
+    if (ok && Lc < C) {   // rows past the chunk's end: zero dO and V (the copies read the next tokens)
+        for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
+            const int i = Lc + idx / 16, g = idx % 16;
+            *reinterpret_cast<uint4 *>(sm + L::DOL + (g >> 3) * 16384 + i * 128 + (g & 7) * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sm + L::VV + i * 256 + g * 16) = make_uint4(0, 0, 0, 0);
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    // ---- phase 1: S^T Khat^T (-> W^T = V^T - that) ; dU^T = dO^T Aqk + dS'^T Kbar^T
+    if (ok && tid == 0) {
+        ptx::tc_fence_after();
+        constexpr uint32_t i_mk = ptx::idesc_bf16_f32(128, 64, true, false);
+        constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            ptx::mma_bf16(tmem + GC_0, ptx::desc_mnmajor_sw128(sb + L::SS + s * 2048, 16384, 1024),
+                          kdesc(sb + L::KH, s, 64), i_mk, s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(sb + L::DOL + s * 2048, 16384, 1024),
+                          ptx::desc_mnmajor_sw128(sb + L::EX + BwdX::AQK + s * 2048, 8192, 1024), i_mm, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(sb + L::DS + s * 2048, 16384, 1024),
+                          kdesc(sb + L::KBR, s, 64), i_mk, 1);
+        ptx::mma_commit(bar_mma);
+        ++n_commit;
+    }
+    if (ok) ok = wait_all(bar_mma, ph_mma);
+    const int vr = quad * 32 + lane;   // this lane's TMEM row: value channel (phases 1-2) or key channel
+    if (ok) {   // W^T (scaled by beta_i) and dU^T -> bf16 K-major A operands, rows = value channels
+        float x[32], y[32];
+        ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
+        ptx::tmem_ld32(tl + GC_1 + 32 * half, y);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int i = 32 * half + u;
+            const float vi = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + L::VV + (i * DV + vr) * 2));
+            x[u] = fB[i] * (vi - x[u]);
+        }
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+            st_bf16x8(sm, L::AW + sw128_chunk(vr, 4 * half + gq), x + 8 * gq);
+            st_bf16x8(sm, L::ADU + sw128_chunk(vr, 4 * half + gq), y + 8 * gq);
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    // ---- phase 2: U^T = (beta W)^T T^T ; lam^T = dU^T T
+    if (ok && tid == 0) {
+        ptx::tc_fence_after();
+        constexpr uint32_t i_kk = ptx::idesc_bf16_f32(128, 64);
+        constexpr uint32_t i_km = ptx::idesc_bf16_f32(128, 64, false, true);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            ptx::mma_bf16(tmem + GC_2, kdesc(sb + L::AW, s, 128), kdesc(sb + L::EX + BwdX::TI, s, 64), i_kk, s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            ptx::mma_bf16(tmem + GC_3, kdesc(sb + L::ADU, s, 128),
+                          ptx::desc_mnmajor_sw128(sb + L::EX + BwdX::TI + s * 2048, 8192, 1024), i_km, s > 0);
+        ptx::mma_commit(bar_mma);
+        ++n_commit;
+    }
+    if (ok) ok = wait_all(bar_mma, ph_mma);
+    if (ok) {
+        float x[32];
+        // U^T -> bf16 (rows = value channels): the MN-major B of [dO; lam] U^T and dS' U^T
+        ptx::tmem_ld32(tl + GC_2 + 32 * half, x);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::AW + sw128_chunk(vr, 4 * half + gq), x + 8 * gq);
+        // <lam_j, W_j> summed over this warp's 32 value channels
+        float lam[32], p[32];
+        ptx::tmem_ld32(tl + GC_3 + 32 * half, lam);
+        ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int j = 32 * half + u;
+            const float vj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + L::VV + (j * DV + vr) * 2));
+            p[u] = lam[u] * (vj - x[u]);
+        }
+        fDB[quad * 64 + 32 * half + lane] = warp_transpose_sum32(p);
+        // mu = beta lam: dV; lam rows under dO in DOL; -mu rows in ADU (K-major B, N = tokens)
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int j = 32 * half + u;
+            const float mu = fB[j] * lam[u];
+            if (j < Lc) dv_out[((cs + j) * H + h) * DV + vr] = __float2bfloat16_rn(mu);
+            st_bf16(sm, L::DOL + sw128(64 + j, vr, 128), lam[u]);
+            st_bf16(sm, L::ADU + sw128(j, vr, 64), -mu);
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    // ---- phase 3: [dAqk; L] = [dO; lam] U^T ; S dO^T ; S (-mu)^T ; dS' U^T
+    if (ok && tid == 0) {
+        ptx::tc_fence_after();
+        constexpr uint32_t i_kk = ptx::idesc_bf16_f32(128, 64);
+        constexpr uint32_t i_km = ptx::idesc_bf16_f32(128, 64, false, true);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            ptx::mma_bf16(tmem + GC_0, kdesc(sb + L::DOL, s, 128),
+                          ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_km, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            ptx::mma_bf16(tmem + GC_1, kdesc(sb + L::SS, s, 128), kdesc(sb + L::DOL, s, 128), i_kk, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            ptx::mma_bf16(tmem + GC_2, kdesc(sb + L::SS, s, 128), kdesc(sb + L::ADU, s, 64), i_kk, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            ptx::mma_bf16(tmem + GC_3, kdesc(sb + L::DS, s, 128),
+                          ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_km, s > 0);
+        ptx::mma_commit(bar_mma);
+        ++n_commit;
+    }
+    if (ok) {   // meanwhile: sum_v S dS' for this lane's key channel over the half's 64 value columns
+        float acc = 0.f;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            float a8[8], b8[8];
+            unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::SS + half * 16384 + sw128_chunk(vr, g)), a8);
+            unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::DS + half * 16384 + sw128_chunk(vr, g)), b8);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc = fmaf(a8[u], b8[u], acc);
+        }
+        fGC[half * 128 + vr] = acc;
+    }
+    if (ok) ok = wait_all(bar_mma, ph_mma);
+    if (ok) {
+        // the chunk's unit is no longer read by anyone: the sums go over it
+        float x[32];
+        ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
+        ptx::tmem_wait_ld();
+        if (quad < 2) {   // rows 0-63: dAqk (j <= i) -> unit rows 64-127 of DA
+            const int i = vr;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) x[u] = (32 * half + u <= i) ? x[u] : 0.f;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq)
+                st_global_bf16x8(unit + U::DA + sw128_chunk(64 + i, 4 * half + gq), x + 8 * gq);
+        } else {          // rows 64-127: L = lam U^T -> dAkk = -beta_i L (j < i), and sum_j Akk L
+            const int i = vr - 64;
+            const float bi = fB[i];
+            float dot = 0.f, a8[8];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::EX + BwdX::AKK + sw128_chunk(i, 4 * half + gq)),
+                              a8);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) dot = fmaf(a8[u], x[8 * gq + u], dot);
+            }
+            fDB2[half * 64 + i] = dot;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) x[u] = (32 * half + u < i) ? -bi * x[u] : 0.f;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq)
+                st_global_bf16x8(unit + U::DA + sw128_chunk(i, 4 * half + gq), x + 8 * gq);
+        }
+        // XQ, XK, XB: row = key channel vr, columns 32 half .. (fp32, 128 contiguous bytes per thread)
+#pragma unroll 1
+        for (int m = 0; m < 3; ++m) {
+            ptx::tmem_ld32(tl + GC_1 + 64 * m + 32 * half, x);
+            ptx::tmem_wait_ld();
+            float *dst = reinterpret_cast<float *>(unit + U::XQ + m * (DK * C * 4)) + vr * C + 32 * half;
+#pragma unroll
+            for (int u = 0; u < 32; u += 4)
+                *reinterpret_cast<float4 *>(dst + u) = make_float4(x[u], x[u + 1], x[u + 2], x[u + 3]);
+        }
+    }
+    __syncthreads();
+    if (ok) {
+        if (tid < C && tid < Lc) {
+            const float db = fDB[tid] + fDB[64 + tid] + fDB[128 + tid] + fDB[192 + tid] - fDB2[tid] - fDB2[64 + tid];
+            dbeta[(cs + tid) * H + h] = db;
+        }
+        if (tid < DK)
+            reinterpret_cast<float *>(unit + U::DGC)[tid] = fD[tid] * (fGC[tid] + fGC[128 + tid]);
+    }
+    if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded)
+        ptx::mbar_wait_bounded(bar_ld, 0u, WAIT_LIMIT_CYCLES);
+        if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, GRAD_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ chain rule
+
+struct ChainLayout {   // dk = 128
+    static constexpr int DA = 0;                // bf16 [128][128 B]  dAkk rows 0-63, dAqk rows 64-127
+    static constexpr int KE = 16384;            // tier A: bf16 [2][64][128 B] e^{-G} K (MN-major A, M = key channels)
+    static constexpr int KQE = 32768;           // tier A: bf16 [2][128][128 B] e^{G - G_last} [K; Q];
+                                                //   tier B: q then k, bf16 [64][128] each, no swizzle
+    static constexpr int FG = 65536;            // fp32 [64][128] G
+    static constexpr int FSEG = FG + 32768;     // fp32 [8][128]  segment sums
+    static constexpr int FX = FSEG + 4096;      // fp32 [2][2][128] per column half: sum_i k_i b_i, sum_i dG_i
+    static constexpr int MISC = FX + 2048;      // mbarriers, TMEM base
+    static constexpr int BYTES = MISC + 64;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(2 * (ALLOC + 1024) <= 233472, "two CTAs per SM");
+};
+
+constexpr uint32_t CHAIN_TMEM_COLS = 256;
+constexpr uint32_t HC_RQ = 0, HC_RK = 64, HC_CT = 128;
+
+// bf16 element (r, j) of a one-atom (64-column) tile with a 128-byte swizzle.
+__device__ __forceinline__ float ld_sw128(const uint8_t *tile, int r, int j) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + r * 128 + ((((j >> 3) ^ (r & 7))) << 4) +
+                                                                      ((j & 7) << 1)));
+}
+
+// One CTA per (chunk slot, head), 256 threads; thread (key channel c = 32 (w & 3) +
+// lane, token half w >> 2).  With dA = (dAkk, dAqk) from bwd_grad_kernel, the pair
+// terms of channel c are
+//   row terms  RQ_i = sum_{j<=i} dAqk[i][j] e^{G_i-G_j} k_j,  RK_i = sum_{j<i} dAkk[i][j] e^{G_i-G_j} k_j,
+//   col terms  CT_j = sum_{i>=j} (dAqk[i][j] q_i + dAkk[i][j] k_i) e^{G_i-G_j}.
+// Tier A (every channel's chunk decay >= -DECAY_LIM): RQ = e^{G_i} [(e^{-G} K)^T dAqk^T]_i,
+// RK likewise, CT = e^{G_last - G_j} [(e^{G - G_last} [K; Q])^T [dAkk; dAqk]]_j on the
+// tensor cores: every operand factor is >= 1 and <= e^DECAY_LIM and the products are
+// scaled down afterwards, so no gradient underflows on the way.  Tier B: the exact
+// sums on the CUDA cores.  Then, with a = e^G dKhat + RK, b = e^{G_last - G} dKbar:
+//   dq = e^G dQhat + RQ,  dk = a + b + CT,  dG = q dq + k (a - b - CT),
+//   dlog_alpha_t = e^{G_last} sum_v S dS' + sum_i k_i b_i + sum_{i>=t} dG_i.
+__global__ void __launch_bounds__(NT, 2)
+bwd_chain_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                 const float *__restrict__ log_alpha, const int32_t *__restrict__ cu_seqlens, int T, int H,
+                 int num_seqs, const uint8_t *__restrict__ ws, __nv_bfloat16 *__restrict__ dq,
+                 __nv_bfloat16 *__restrict__ dk_out, float *__restrict__ dlog_alpha) {
+    using L = ChainLayout;
+    using U = BwdUnit<128>;
+    constexpr int DK = 128;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = ptx::smem_u32(sm);
+    const uint32_t bar_ld = sb + L::MISC, bar_mma = sb + L::MISC + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 16);
+    float *fG = reinterpret_cast<float *>(sm + L::FG), *fSeg = reinterpret_cast<float *>(sm + L::FSEG);
+    float *fX = reinterpret_cast<float *>(sm + L::FX);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, half = warp >> 2;
+    const int slot = blockIdx.x, h = blockIdx.y;
+    long long cs;
+    int Lc;
+    if (!slot_chunk(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
+    const uint8_t *unit = ws + ((size_t)slot * H + h) * U::BYTES;
+
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), CHAIN_TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (tid == 0) {
+        ptx::mbar_init(bar_ld, 1);
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+        ptx::mbar_arrive_expect_tx(bar_ld, 16384u);
+        ptx::bulk_load(sb + L::DA, unit + U::DA, 16384u, bar_ld);
+    }
+    bool strong;
+    {
+        float G[8][4], tot[4];
+        uint2 kv[8], qv[8];
+        chunk_decay<true>(q, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
+        const int c0 = 4 * (tid & 31), i0 = 8 * (tid >> 5);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4 *>(fG + (i0 + u) * DK + c0) = make_float4(G[u][0], G[u][1], G[u][2], G[u][3]);
+        strong = __syncthreads_or(tot[0] < -DECAY_LIM || tot[1] < -DECAY_LIM || tot[2] < -DECAY_LIM ||
+                                  tot[3] < -DECAY_LIM) != 0;
+        if (!strong) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u;
+                const float4 k4 = bf16x4_to_float4(kv[u]), q4 = bf16x4_to_float4(qv[u]);
+                float en[4], er[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    en[e] = __expf(-G[u][e]);             // <= e^DECAY_LIM
+                    er[e] = __expf(G[u][e] - tot[e]);     // <= e^DECAY_LIM
+                }
+                st_bf16x4(sm, L::KE + sw128(i, c0, 64), k4.x * en[0], k4.y * en[1], k4.z * en[2], k4.w * en[3]);
+                st_bf16x4(sm, L::KQE + sw128(i, c0, 128), k4.x * er[0], k4.y * er[1], k4.z * er[2], k4.w * er[3]);
+                st_bf16x4(sm, L::KQE + sw128(64 + i, c0, 128), q4.x * er[0], q4.y * er[1], q4.z * er[2],
+                          q4.w * er[3]);
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                *reinterpret_cast<uint2 *>(sm + L::KQE + ((i0 + u) * DK + c0) * 2) = qv[u];
+                *reinterpret_cast<uint2 *>(sm + L::KQE + 16384 + ((i0 + u) * DK + c0) * 2) = kv[u];
+            }
+        }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t ph_ld = 0, ph_mma = 0;
+    bool ok = wait_all(bar_ld, ph_ld);
+    bool mma_pending = false;
+    if (ok && !strong) {
+        if (tid == 0) {
+            constexpr uint32_t i_mk = ptx::idesc_bf16_f32(128, 64, true, false);
+            constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + HC_RQ, ptx::desc_mnmajor_sw128(sb + L::KE + s * 2048, 8192, 1024),
+                              kdesc(sb + L::DA + 8192, s, 64), i_mk, s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + HC_RK, ptx::desc_mnmajor_sw128(sb + L::KE + s * 2048, 8192, 1024),
+                              kdesc(sb + L::DA, s, 64), i_mk, s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                ptx::mma_bf16(tmem + HC_CT, ptx::desc_mnmajor_sw128(sb + L::KQE + s * 2048, 16384, 1024),
+                              ptx::desc_mnmajor_sw128(sb + L::DA + s * 2048, 8192, 1024), i_mm, s > 0);
+            ptx::mma_commit(bar_mma);
+        }
+        mma_pending = true;
+        ok = wait_all(bar_mma, ph_mma);
+        mma_pending = !ok;
+    }
+
+    const int c = quad * 32 + lane;
+    const float gl = fG[(C - 1) * DK + c];   // G_last (rows past Lc add nothing)
+    const float *xq = reinterpret_cast<const float *>(unit + U::XQ) + c * C + 32 * half;
+    const float *xk = reinterpret_cast<const float *>(unit + U::XK) + c * C + 32 * half;
+    const float *xb = reinterpret_cast<const float *>(unit + U::XB) + c * C + 32 * half;
+    const uint8_t *da = sm + L::DA;
+    const __nv_bfloat16 *sq = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KQE);
+    const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KQE + 16384);
+    float dG[32], kb = 0.f, sdg = 0.f;
+    if (ok) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            float rq[16], rk[16], ct[16];
+            if (!strong) {
+                ptx::tmem_ld16(tl + HC_RQ + 32 * half + 16 * cc, rq);
+                ptx::tmem_ld16(tl + HC_RK + 32 * half + 16 * cc, rk);
+                ptx::tmem_ld16(tl + HC_CT + 32 * half + 16 * cc, ct);
+                ptx::tmem_wait_ld();
+            }
+#pragma unroll
+            for (int u4 = 0; u4 < 16; u4 += 4) {
+                const float4 xq4 = *reinterpret_cast<const float4 *>(xq + 16 * cc + u4);
+                const float4 xk4 = *reinterpret_cast<const float4 *>(xk + 16 * cc + u4);
+                const float4 xb4 = *reinterpret_cast<const float4 *>(xb + 16 * cc + u4);
+                const float vq[4] = {xq4.x, xq4.y, xq4.z, xq4.w};
+                const float vk[4] = {xk4.x, xk4.y, xk4.z, xk4.w};
+                const float vb[4] = {xb4.x, xb4.y, xb4.z, xb4.w};
+                float qi[4], ki[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const int i = 32 * half + 16 * cc + u4 + w;
+                    const long long off = ((cs + min(i, Lc - 1)) * H + h) * DK + c;
+                    qi[w] = i < Lc ? __bfloat162float(q[off]) : 0.f;
+                    ki[w] = i < Lc ? __bfloat162float(k[off]) : 0.f;
+                }
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const int u = u4 + w, i = 32 * half + 16 * cc + u;
+                    const float Gi = fG[i * DK + c];
+                    const float eg = __expf(Gi), eb = __expf(gl - Gi);
+                    float RQ, RK, CT;
+                    if (!strong) {
+                        RQ = eg * rq[u];
+                        RK = eg * rk[u];
+                        CT = eb * ct[u];
+                    } else {   // exact pair terms of this (token, channel)
+                        RQ = 0.f; RK = 0.f; CT = 0.f;
+                        for (int j = 0; j <= i; ++j) {
+                            const float f = __expf(Gi - fG[j * DK + c]) * __bfloat162float(sk[j * DK + c]);
+                            RQ = fmaf(ld_sw128(da, 64 + i, j), f, RQ);
+                            RK = fmaf(ld_sw128(da, i, j), f, RK);
+                        }
+                        for (int m = i; m < C; ++m) {
+                            const float f = __expf(fG[m * DK + c] - Gi);
+                            const float x = ld_sw128(da, 64 + m, i) * __bfloat162float(sq[m * DK + c]) +
+                                            ld_sw128(da, m, i) * __bfloat162float(sk[m * DK + c]);
+                            CT = fmaf(x, f, CT);
+                        }
+                    }
+                    const float dqi = fmaf(eg, vq[w], RQ);
+                    const float a = fmaf(eg, vk[w], RK), b = eb * vb[w];
+                    const float dki = a + b + CT;
+                    const float g = qi[w] * dqi + ki[w] * (a - b - CT);
+                    dG[16 * cc + u] = g;
+                    sdg += g;
+                    kb = fmaf(ki[w], b, kb);
+                    if (i < Lc) {
+                        const long long o = ((cs + i) * H + h) * DK + c;
+                        dq[o] = __float2bfloat16_rn(dqi);
+                        dk_out[o] = __float2bfloat16_rn(dki);
+                    }
+                }
+            }
+        }
+        fX[half * DK + c] = kb;
+        fX[2 * DK + half * DK + c] = sdg;
+    }
+    __syncthreads();
+    if (ok) {
+        float run = reinterpret_cast<const float *>(unit + U::DGC)[c] + fX[c] + fX[DK + c];
+        if (half == 0) run += fX[2 * DK + DK + c];   // all of the later half's dG
+#pragma unroll
+        for (int u = 31; u >= 0; --u) {
+            const int i = 32 * half + u;
+            run += dG[u];
+            if (i < Lc) dlog_alpha[((cs + i) * H + h) * DK + c] = run;
+        }
+    }
+    if (!ok && tid == 0) {   // a wait timed out: let the copy and MMAs in flight land (bounded)
+        ptx::mbar_wait_bounded(bar_ld, 0u, WAIT_LIMIT_CYCLES);
+        if (mma_pending) ptx::mbar_wait_bounded(bar_mma, 0u, WAIT_LIMIT_CYCLES);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, CHAIN_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+// Workspace of the tensor-core backward: one BwdUnit per (chunk slot, head).
+inline size_t backward_tc_workspace_bytes(long long tokens, int H, int num_seqs) {
+    if (tokens <= 0) return 0;
+    return (size_t)chunk_slots(tokens, num_seqs) * (size_t)H * (size_t)BwdUnit<128>::BYTES;
+}
+
+template <typename K>
+inline int set_smem_tc(K kern, int bytes, const char *what, char *msg, size_t msg_len) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) return KDA_OK;
+    snprintf(msg, msg_len, "cudaFuncSetAttribute(%s): %s", what, cudaGetErrorString(e));
+    return KDA_ERR_CUDA;
+}
+
+inline int launch_ok(const char *what, char *msg, size_t msg_len) {
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return KDA_OK;
+    snprintf(msg, msg_len, "%s launch: %s", what, cudaGetErrorString(e));
+    return KDA_ERR_CUDA;
+}
+
+// The five launches for bf16 inputs, dk = dv = 128 (per-channel decay).
+inline int launch_backward_tc(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                              const float *init_state, const void *d_o, const float *dfinal, void *dq, void *dk_out,
+                              void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state,
+                              const int32_t *cu_seqlens, long long tokens, int T, int H, int num_seqs,
+                              void *workspace, cudaStream_t st, char *msg, size_t msg_len) {
+    constexpr int DK = 128, DV = 128, DVT = 32, NBUF = 2;
+    const long long slots = tokens > 0 ? chunk_slots(tokens, num_seqs) : 0;
+    if (slots > 0x7fffffffLL) {
+        snprintf(msg, msg_len, "%lld chunk slots exceed the grid limit", slots);
+        return KDA_ERR_UNSUPPORTED;
+    }
+    uint8_t *ws = (uint8_t *)workspace;
+    const auto *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k;
+    CUtensorMap t_v32, t_do32, t_do64, t_v128;
+    memset(&t_do32, 0, sizeof(t_do32));   // no tokens: the adjoint sweep only copies dfinal, never loading
+    if (slots > 0 && (!make_tmap(&t_v32, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, DVT) ||
+        !make_tmap(&t_do32, d_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, DVT,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_tmap(&t_do64, d_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&t_v128, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 128))) {
+        snprintf(msg, msg_len, "building TMA descriptors failed (driver entry point cuTensorMapEncodeTiled)");
+        return KDA_ERR_CUDA;
+    }
+    int rc;
+    auto k1 = chunk_intra_kernel<DK, false, false, true>;
+    auto k2 = chunk_inter_kernel<DK, DVT, NBUF, true>;
+    auto k3 = chunk_adj_kernel<DK, DVT, NBUF>;
+    auto k4 = bwd_grad_kernel;
+    auto k5 = bwd_chain_kernel;
+    constexpr int s1 = IntraLayout<DK>::ALLOC, s2 = InterLayout<DK, DVT, NBUF>::ALLOC;
+    constexpr int s3 = AdjLayout<DK, DVT, NBUF>::ALLOC, s4 = GradLayout::ALLOC, s5 = ChainLayout::ALLOC;
+    if ((rc = set_smem_tc(k1, s1, "chunk_intra", msg, msg_len)) || (rc = set_smem_tc(k2, s2, "chunk_inter", msg, msg_len)) ||
+        (rc = set_smem_tc(k3, s3, "chunk_adj", msg, msg_len)) || (rc = set_smem_tc(k4, s4, "bwd_grad", msg, msg_len)) ||
+        (rc = set_smem_tc(k5, s5, "bwd_chain", msg, msg_len)))
+        return rc;
+    const dim3 per_chunk((unsigned)slots, H), per_chain(DV / DVT, H, num_seqs);
+    if (slots > 0) {
+        k1<<<per_chunk, NT, s1, st>>>(qb, kb, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws);
+        if ((rc = launch_ok("chunk_intra", msg, msg_len))) return rc;
+        k2<<<per_chain, NT, s2, st>>>(t_v32, ws, init_state, nullptr, nullptr, cu_seqlens, T, H, DV, nullptr, 0, ws);
+        if ((rc = launch_ok("chunk_inter", msg, msg_len))) return rc;
+    }
+    k3<<<per_chain, NT, s3, st>>>(t_do32, ws, dfinal, dinit_state, cu_seqlens, T, H, DV);
+    if ((rc = launch_ok("chunk_adj", msg, msg_len))) return rc;
+    if (slots > 0) {
+        k4<<<per_chunk, NT, s4, st>>>(t_do64, t_v128, kb, log_alpha, beta, (__nv_bfloat16 *)dv_out, dbeta, cu_seqlens,
+                                      T, H, num_seqs, ws);
+        if ((rc = launch_ok("bwd_grad", msg, msg_len))) return rc;
+        k5<<<per_chunk, NT, s5, st>>>(qb, kb, log_alpha, cu_seqlens, T, H, num_seqs, ws, (__nv_bfloat16 *)dq,
+                                      (__nv_bfloat16 *)dk_out, dlog_alpha);
+        if ((rc = launch_ok("bwd_chain", msg, msg_len))) return rc;
+    }
+    return KDA_OK;
+}
+
+}  // namespace tc
+}  // namespace kda

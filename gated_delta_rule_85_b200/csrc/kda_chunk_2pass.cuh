@@ -38,6 +38,39 @@ struct Rec {
     static constexpr int BYTES = (DCH + DK * 4 + 1023) / 1024 * 1024;
 };
 
+// What the backward needs of a chunk beyond the record (first pass with BX): bf16
+// 64 x 64 tiles, row i of 128 bytes with a 128-byte swizzle, fp32 values rounded once.
+struct BwdX {
+    static constexpr int AKK = 0;        // Akk[i][j], j < i (zero elsewhere), without beta
+    static constexpr int AQK = 8192;     // Aqk[i][j], j <= i (zero above)
+    static constexpr int TI = 16384;     // T = (I + Diag(beta) Akk)^{-1}, unit lower (zero above)
+    static constexpr int BYTES = 24576;
+};
+
+// Backward workspace unit of one (chunk slot, head), dk = dv = 128 (kda_bwd_tc.cuh):
+// the record and the extras from the first pass, the state at the chunk's start
+// (forward sweep) and its adjoint at the chunk's end (adjoint sweep), both bf16
+// [DV/64][DK][128 B] with a 128-byte swizzle.  The per-chunk gradient kernel then
+// writes its sums over the first bytes of the same unit (fields XQ..DGC).
+template <int DK>
+struct BwdUnit {
+    static constexpr int DV = 128;
+    static constexpr int REC = 0;
+    static constexpr int BXO = Rec<DK>::BYTES;
+    static constexpr int SC = BXO + BwdX::BYTES;
+    static constexpr int DSC = SC + DK * DV * 2;
+    static constexpr int BYTES = DSC + DK * DV * 2;
+    static constexpr int XQ = 0;                       // fp32 [DK][64]  S dO^T                (dQhat^T)
+    static constexpr int XK = XQ + DK * C * 4;         // fp32 [DK][64]  -S mu^T               (dKhat^T)
+    static constexpr int XB = XK + DK * C * 4;         // fp32 [DK][64]  dS U^T                (dKbar^T)
+    static constexpr int DA = XB + DK * C * 4;         // bf16 [128][128 B]: dAkk rows 0-63, dAqk rows 64-127
+    static constexpr int DGC = DA + 128 * 128;         // fp32 [DK]      e^{G_last} sum_v S dS
+    static constexpr int GRAD_END = DGC + DK * 4;
+    static_assert(GRAD_END <= BYTES, "the sums fit over the unit");
+    static_assert(BXO % 1024 == 0 && SC % 1024 == 0 && DSC % 1024 == 0 && BYTES % 1024 == 0 && DA % 1024 == 0,
+                  "tile alignment");
+};
+
 inline long long chunk_slots(long long tokens, int num_seqs) { return (tokens + C - 1) / C + num_seqs; }
 
 // Workspace: the records [slot][H] of the first pass.
@@ -165,12 +198,13 @@ __device__ __noinline__ void intra_fixup(uint32_t tl, int quad, int warp, int r,
 // that needs tier B is left at once (returns 1) for intra_chunk_strong.  TB = true:
 // tier B.  All threads of the CTA call it; ph_mma carries the MMA mbarrier phase.
 // Returns 0 when done (or the slot has no chunk) and -1 when a bounded wait ran out.
-template <int DK, bool GS, bool PRO, bool TB>
+template <int DK, bool GS, bool PRO, bool TB, bool BX>
 __device__ __forceinline__ int intra_chunk(int slot, int h, const __nv_bfloat16 *__restrict__ q,
                                            const __nv_bfloat16 *__restrict__ k,
                                            const float *__restrict__ log_alpha, const float *__restrict__ beta,
                                            const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
-                                           uint8_t *__restrict__ ws, uint8_t *sm, uint32_t tmem, uint32_t &ph_mma) {
+                                           uint8_t *__restrict__ ws, uint8_t *sm, uint32_t tmem,
+                                           uint32_t &ph_mma) {
     using L = IntraLayout<DK>;
     using R = Rec<DK>;
     constexpr int NCG = DK / 4, NSEG = L::NSEG, SEGLEN = C / NSEG, SPB = 16 / SEGLEN, NW = DK / 32;
@@ -200,7 +234,9 @@ __device__ __forceinline__ int intra_chunk(int slot, int h, const __nv_bfloat16 
     float *fSeg = reinterpret_cast<float *>(sm + L::FSEG);
     uint32_t *bad = reinterpret_cast<uint32_t *>(sm + L::BAD);
     const uint32_t bar_mma = sb + L::MISC;
-    uint8_t *rec = ws + ((size_t)slot * H + h) * R::BYTES;
+    // BX: ws holds backward units (record, then the extras)
+    uint8_t *rec = ws + ((size_t)slot * H + h) * (size_t)(BX ? BwdUnit<DK>::BYTES : R::BYTES);
+    uint8_t *xr = rec + BwdUnit<DK>::BXO;
 
     if (tid < C) fB[tid] = tid < Lc ? beta[(cs + tid) * H + h] : 0.f;
     if (tid < 4 * NW) bad[tid] = 0u;
@@ -446,12 +482,24 @@ __device__ __forceinline__ int intra_chunk(int slot, int h, const __nv_bfloat16 
                         a.w = (j + 3 < i) ? bi * g32[u + 3] : 0.f;
                         *reinterpret_cast<float4 *>(fA + i * AS + j) = a;
                     }
+                    if constexpr (BX) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) g32[u] = (hh * 32 + u < i) ? g32[u] : 0.f;
+#pragma unroll
+                        for (int gq = 0; gq < 4; ++gq)
+                            st_global_bf16x8(xr + BwdX::AKK + sw128_chunk(i, hh * 4 + gq), g32 + gq * 8);
+                    }
                 } else {
                     const int i = r;
 #pragma unroll
                     for (int u = 0; u < 32; ++u) g32[u] = (hh * 32 + u <= i) ? g32[u] : 0.f;
 #pragma unroll
                     for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::AQ + sw128_chunk(i, hh * 4 + gq), g32 + gq * 8);
+                    if constexpr (BX) {
+#pragma unroll
+                        for (int gq = 0; gq < 4; ++gq)
+                            st_global_bf16x8(xr + BwdX::AQK + sw128_chunk(i, hh * 4 + gq), g32 + gq * 8);
+                    }
                 }
             }
             if (warp < 2) {
@@ -476,7 +524,7 @@ __device__ __forceinline__ int intra_chunk(int slot, int h, const __nv_bfloat16 
             }
         }
         __syncthreads();
-        invert_merge_blocks(fA, fT, fM, sm + L::TB, fB, warp, lane);
+        invert_merge_blocks<BX>(fA, fT, fM, sm + L::TB, fB, warp, lane);
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncthreads();
@@ -494,6 +542,17 @@ __device__ __forceinline__ int intra_chunk(int slot, int h, const __nv_bfloat16 
             for (int s = 0; s < 4; ++s)
                 ptx::mma_bf16(tmem + ICOL_PT, kdesc(sb + L::TB, s, 128), kdesc(sb + L::TB, s, 64), ipt, s > 0);
             ptx::mma_commit(bar_mma);
+        }
+        if constexpr (BX) {   // T rows while the products run: 16 columns per thread
+            const int row = tid >> 2;
+#pragma unroll
+            for (int gg = 0; gg < 2; ++gg) {
+                const int g8 = (tid & 3) * 2 + gg;
+                float t8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) t8[u] = (8 * g8 + u <= row) ? fT[row * AS + 8 * g8 + u] : 0.f;
+                st_global_bf16x8(xr + BwdX::TI + sw128_chunk(row, g8), t8);
+            }
         }
         ok = wait_all(bar_mma, ph_mma);
     }
@@ -533,21 +592,23 @@ __device__ __forceinline__ int intra_chunk(int slot, int h, const __nv_bfloat16 
 
 // Tier B of one chunk, kept out of line so that its code does not weigh on the
 // register allocation of the common (tier-A) path.
-template <int DK, bool GS, bool PRO>
+template <int DK, bool GS, bool PRO, bool BX>
 __device__ __noinline__ int intra_chunk_strong(int slot, int h, const __nv_bfloat16 *__restrict__ q,
                                                const __nv_bfloat16 *__restrict__ k,
                                                const float *__restrict__ log_alpha, const float *__restrict__ beta,
                                                const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
-                                               uint8_t *__restrict__ ws, uint8_t *sm, uint32_t tmem, uint32_t *ph_mma) {
+                                               uint8_t *__restrict__ ws, uint8_t *sm, uint32_t tmem,
+                                               uint32_t *ph_mma) {
     uint32_t ph = *ph_mma;
-    const int r = intra_chunk<DK, GS, PRO, true>(slot, h, q, k, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws, sm,
-                                                 tmem, ph);
+    const int r = intra_chunk<DK, GS, PRO, true, BX>(slot, h, q, k, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws,
+                                                     sm, tmem, ph);
     *ph_mma = ph;
     return r;
 }
 
 // First pass: one CTA per (chunk slot, head); tier A inline, tier B out of line.
-template <int DK, bool GS, bool PRO>
+// BX (the backward): ws holds [slot][H] BwdUnit; the extras go beside each record.
+template <int DK, bool GS, bool PRO, bool BX = false>
 __global__ void __launch_bounds__(NT, 2)
 chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -569,12 +630,12 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     uint32_t ph_mma = 0;
-    const int r = intra_chunk<DK, GS, PRO, false>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta,
-                                                  cu_seqlens, T, H, num_seqs, ws, sm, tmem, ph_mma);
+    const int r = intra_chunk<DK, GS, PRO, false, BX>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta,
+                                                      cu_seqlens, T, H, num_seqs, ws, sm, tmem, ph_mma);
     if (r == 1) {   // the chunk decays faster than tier A covers (uniform over the CTA)
         __syncthreads();
-        intra_chunk_strong<DK, GS, PRO>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta, cu_seqlens, T, H,
-                                        num_seqs, ws, sm, tmem, &ph_mma);
+        intra_chunk_strong<DK, GS, PRO, BX>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta, cu_seqlens, T,
+                                            H, num_seqs, ws, sm, tmem, &ph_mma);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -610,17 +671,21 @@ constexpr uint32_t INTER_TMEM_COLS = 256;
 constexpr uint32_t XCOL_XY = 0;       // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O
 constexpr uint32_t XCOL_DS = 128;     // [128 x DVT] Kt Z (lanes 0..dk-1)
 
-template <int DK, int DVT, int NBUF>
+// CK (the backward's state sweep, dv = 128): ws (and ckpt, the same bytes, writable)
+// hold [slot][H] BwdUnit; no output; instead the state at each chunk's start, bf16,
+// into the unit's SC tile (a K-major operand S with K = value columns, MN-major for S^T).
+template <int DK, int DVT, int NBUF, bool CK = false>
 __global__ void __launch_bounds__(NT, 1)
 chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__restrict__ ws,
                    const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
                    float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV,
-                   const int32_t *__restrict__ slots, int num_slots) {
+                   const int32_t *__restrict__ slots, int num_slots, uint8_t *__restrict__ ckpt) {
     using L = InterLayout<DK, DVT, NBUF>;
     using R = Rec<DK>;
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
     constexpr int CPT = DVT / 2;
     constexpr uint32_t TX = (uint32_t)(R::BYTES + C * DVT * 2);
+    constexpr size_t USTRIDE = CK ? (size_t)BwdUnit<DK>::BYTES : (size_t)R::BYTES;   // bytes per (slot, head)
     using MN = MnOp<DVT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -661,7 +726,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
         n_issued = ci + 1;
         const uint32_t bar = bar_rec + 8 * b;
         ptx::mbar_arrive_expect_tx(bar, TX);
-        ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * R::BYTES, (uint32_t)R::BYTES, bar);
+        ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * USTRIDE, (uint32_t)R::BYTES, bar);
         ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, &tm_v, bar, col_base, h, (int)(t0 + (long long)ci * C));
     };
 
@@ -694,11 +759,14 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
         // ---- 1. S^T -> bf16 B operand
         const float dch = has_row ? reinterpret_cast<const float *>(sm + b * R::BYTES + R::DCH)[srow] : 0.f;
         if (has_row) {
+            uint8_t *ck = CK ? ckpt + ((size_t)(first + ci) * H + h) * USTRIDE + BwdUnit<DK>::SC : nullptr;
 #pragma unroll
-            for (int g = 0; g < CPT / 8; ++g)
-                *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) =
-                    make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
-                               pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
+            for (int g = 0; g < CPT / 8; ++g) {
+                const uint4 w = make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
+                                           pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
+                *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) = w;
+                if constexpr (CK) *reinterpret_cast<uint4 *>(ck + sw128(srow, col_base + scol + 8 * g, DK)) = w;
+            }
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
@@ -752,9 +820,12 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
 #pragma unroll
             for (int s = 0; s < 4; ++s)
                 ptx::mma_bf16(tmem + XCOL_DS, kdesc(rb + R::KP, s, DK + 64), MN::desc(sb + L::ZT, s, C), iz, s > 0);
+            if constexpr (!CK) {
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C), iz, 1);
+                for (int s = 0; s < 4; ++s)
+                    ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C),
+                                  iz, 1);
+            }
             ptx::mma_commit(bar_mma);
             ++n_commit;
         }
@@ -772,7 +843,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
                 for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
             }
         }
-        if (quad >= 2) {
+        if (!CK && quad >= 2) {
             const int i = (quad - 2) * 32 + lane;
 #pragma unroll 1
             for (int cc = 0; cc < CPT / 16; ++cc) {
@@ -855,7 +926,7 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
     }
     k2<<<dim3(dv / DVT, H, num_seqs), NT, smem2, st>>>(tv, (const uint8_t *)workspace, init_state,
                                                         (__nv_bfloat16 *)o, final_state, cu_seqlens, T, H, dv,
-                                                        slots, num_slots);
+                                                        slots, num_slots, nullptr);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "chunk_inter launch: %s", cudaGetErrorString(e));

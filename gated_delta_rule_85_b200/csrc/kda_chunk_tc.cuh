@@ -253,6 +253,7 @@ __device__ __forceinline__ void invert_diag_blocks(const float *A, float *Tm, ui
 // [L11^-1 0; -L22^-1 L21 L11^-1  L22^-1] at 32 (two pairs of 16-blocks) and at 64,
 // each block product one 16 x 8 tile per warp on the tensor cores (tf32 inputs,
 // fp32 accumulation).  All 256 threads take part.
+template <bool KEEP_T = false>
 __device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, float *M, uint8_t *tb,
                                                     const float *beta, int warp, int lane) {
     if (warp < 4) {   // M_p = A[2p+1][2p] T[2p][2p]
@@ -281,6 +282,8 @@ __device__ __forceinline__ void invert_merge_blocks(const float *A, float *Tm, f
         float d[4] = {0.f, 0.f, 0.f, 0.f};
         warp_mm16x8_tf32<4>(d, Tm + (32 + 16 * mt) * AS + 32, AS, M + 8 * nt, 36, lane);
         warp_store16x8_tbt(tb, 32 + 16 * mt, 8 * nt, d, -1.f, beta, lane);
+        // KEEP_T: T[hi][lo] into Tm too (this step reads only columns 32.. of Tm)
+        if constexpr (KEEP_T) warp_store16x8(Tm + (32 + 16 * mt) * AS + 8 * nt, AS, d, -1.f, lane);
     }
 }
 
@@ -1020,7 +1023,8 @@ inline EncodeTiledFn encode_fn() {
 
 // [tokens, H, inner] row-major tensor -> box (box_inner, 1, 64 tokens).
 inline bool make_tmap(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, long long tokens,
-                      int H, int inner, int box_inner) {
+                      int H, int inner, int box_inner,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)tokens};
@@ -1028,7 +1032,7 @@ inline bool make_tmap(CUtensorMap *m, const void *base, CUtensorMapDataType dt, 
     cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)C};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

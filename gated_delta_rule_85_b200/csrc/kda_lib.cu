@@ -11,6 +11,7 @@
 #include "kda_chunk_tc.cuh"
 #include "kda_chunk_2pass.cuh"
 #include "kda_bwd_simt.cuh"
+#include "kda_bwd_tc.cuh"
 
 namespace {
 
@@ -334,12 +335,27 @@ int launch_backward(const void *q, const void *k, const void *v, const float *lo
     return KDA_OK;
 }
 
-// Both backward entry points after the shared checks; gate_scalar: Gated DeltaNet.
+// The tensor-core backward covers bf16 inputs, per-channel decay, dk = dv = 128.
+bool backward_tc_eligible(int dtype, int dk, int dv, bool gate_scalar) {
+    return dtype == KDA_BF16 && dk == 128 && dv == 128 && !gate_scalar;
+}
+
+// Workspace bytes of the backward path that `algo` selects (0 for an unusable choice).
+size_t backward_ws(long long tokens, int H, int dk, int dv, int num_seqs, int dtype, bool gate_scalar, int algo) {
+    const bool tc = backward_tc_eligible(dtype, dk, dv, gate_scalar);
+    if (algo == KDA_BWD_TENSOR && !tc) return 0;
+    if (tc && algo != KDA_BWD_SIMT) return kda::tc::backward_tc_workspace_bytes(tokens, H, num_seqs);
+    return kda::bwd::backward_workspace_bytes(tokens, H, dk, dv, num_seqs);
+}
+
+// Every backward entry point after the shared checks; gate_scalar: Gated DeltaNet.
 int backward_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                   const float *init_state, const void *d_o, const float *dfinal_state, void *dq, void *dk_out,
                   void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state, const int32_t *cu_seqlens,
                   int B, int T, int H, int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace,
-                  size_t ws_bytes, void *stream, bool gate_scalar) {
+                  size_t ws_bytes, void *stream, bool gate_scalar, int algo = KDA_BWD_AUTO) {
+    if (algo != KDA_BWD_AUTO && algo != KDA_BWD_TENSOR && algo != KDA_BWD_SIMT)
+        return fail(KDA_ERR_INVALID_ARG, "unknown backward algo %d", algo);
     // The forward checks cover the inputs (o stands in for d_o).
     int rc = check_prefill(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, cu_seqlens, B, T, H, dk, dv,
                            num_seqs, dtype, chunk, gate_scalar);
@@ -354,7 +370,10 @@ int backward_impl(const void *q, const void *k, const void *v, const float *log_
     if (gate_scalar && dlog_alpha && !aligned(dlog_alpha, 4))
         return fail(KDA_ERR_MISALIGNED, "dlog_alpha is not 4-byte aligned");
     const long long tokens = (long long)B * T;
-    const size_t need = kda::bwd::backward_workspace_bytes(tokens, H, dk, dv, num_seqs);
+    const bool use_tc = backward_tc_eligible(dtype, dk, dv, gate_scalar) && algo != KDA_BWD_SIMT;
+    if (algo == KDA_BWD_TENSOR && !use_tc)
+        return fail(KDA_ERR_UNSUPPORTED, "the tensor-core backward takes bf16, per-channel decay, dk = dv = 128");
+    const size_t need = backward_ws(tokens, H, dk, dv, num_seqs, dtype, gate_scalar, algo);
     if (need > 0 && (!workspace || ws_bytes < need))
         return fail(KDA_ERR_WORKSPACE, "backward workspace of %zu bytes needed, %zu given%s", need, ws_bytes,
                     workspace ? "" : " (NULL)");
@@ -363,6 +382,13 @@ int backward_impl(const void *q, const void *k, const void *v, const float *log_
         return fail(KDA_ERR_UNSUPPORTED, "too many chunk slots for one grid");
     if (num_seqs == 0) return KDA_OK;
     cudaStream_t st = (cudaStream_t)stream;
+    if (use_tc) {
+        char msg[256] = "";
+        const int rc2 = kda::tc::launch_backward_tc(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq,
+                                                    dk_out, dv_out, dlog_alpha, dbeta, dinit_state, cu_seqlens,
+                                                    tokens, T, H, num_seqs, workspace, st, msg, sizeof(msg));
+        return rc2 ? fail(rc2, "%s", msg) : KDA_OK;
+    }
 #define KDA_BWD_ARGS                                                                                      \
     (q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, dlog_alpha, dbeta, dinit_state, \
      cu_seqlens, tokens, T, H, dv, num_seqs, workspace, st)
@@ -588,6 +614,22 @@ int kda_recurrent_step_prologue(const void *q_raw, const void *k_raw, const void
 size_t kda_chunk_backward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs) {
     if (B < 1 || T < 0 || H < 1 || num_seqs < 0 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
     return kda::bwd::backward_workspace_bytes((long long)B * T, H, dk, dv, num_seqs);
+}
+
+size_t kda_chunk_backward_workspace_size_ex(int B, int T, int H, int dk, int dv, int num_seqs, int dtype, int algo) {
+    if (B < 1 || T < 0 || H < 1 || num_seqs < 0 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return 0;
+    return backward_ws((long long)B * T, H, dk, dv, num_seqs, dtype, false, algo);
+}
+
+int kda_chunk_backward_ex(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                          const float *init_state, const void *d_o, const float *dfinal_state, void *dq, void *dk_out,
+                          void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state,
+                          const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv, int num_seqs, int dtype,
+                          int chunk, void *workspace, size_t ws_bytes, void *stream, int algo) {
+    return backward_impl(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, dlog_alpha,
+                         dbeta, dinit_state, cu_seqlens, B, T, H, dk, dv, num_seqs, dtype, chunk, workspace, ws_bytes,
+                         stream, false, algo);
 }
 
 int kda_chunk_backward(const void *q, const void *k, const void *v, const float *log_alpha,

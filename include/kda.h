@@ -326,16 +326,17 @@ int kda_recurrent_step_prologue(const void *q_raw, const void *k_raw, const void
  *                 the gradient at the given initial state (at zero when
  *                 init_state is NULL).
  *   workspace     device memory of at least kda_chunk_backward_workspace_size()
- *                 bytes for the same sizes, 16-byte aligned; no contents are
- *                 required.  Per (64-token chunk slot, head) it holds the fp32
- *                 state at the chunk's start (4 dk dv bytes) and the partial
- *                 sums of every 32-column value tile (about 132 KB per tile at
- *                 dk = 128).  Calls that can overlap in time need separate
- *                 workspaces.  About 570 KB per (chunk, head) at dk = dv = 128
- *                 (2 GB for 8192 tokens x 32 heads): a long input is taken in
- *                 pieces from its end, each piece's dinit_state passed as the
- *                 previous piece's dfinal_state and its init_state the forward
- *                 state at the piece's start -- exact by the chain rule.
+ *                 bytes for the same sizes (enough for either schedule; the
+ *                 schedule this call takes needs kda_chunk_backward_workspace_size_ex
+ *                 with KDA_BWD_AUTO), 16-byte aligned; no contents are required.
+ *                 It holds per (64-token chunk slot, head) what the schedules
+ *                 below keep between their launches: about 145 KB for the
+ *                 tensor-core schedule, 570 KB for the SIMT one (dk = dv = 128).
+ *                 Calls that can overlap in time need separate workspaces.  A
+ *                 long input can be taken in pieces from its end, each piece's
+ *                 dinit_state passed as the previous piece's dfinal_state and its
+ *                 init_state the forward state at the piece's start -- exact by
+ *                 the chain rule.
  * The caller owns every buffer; all pointers except cu_seqlens and beta are
  * 16-byte aligned.  Every gradient is overwritten, not accumulated; tokens
  * outside every sequence (packed input with cu_seqlens[N] < T) are not written.
@@ -350,6 +351,41 @@ int kda_chunk_backward(const void *q, const void *k, const void *v, const float 
                        float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
                        int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
                        void *stream);
+
+/*
+ * Backward schedules (kda_chunk_backward_ex):
+ *   KDA_BWD_TENSOR  bf16 inputs, per-channel decay, dk = dv = 128: five launches
+ *                   on the tensor cores (tcgen05): the forward's first pass with
+ *                   the chunk's Akk, Aqk and T kept, the state sweep storing each
+ *                   chunk's starting state (bf16), the adjoint sweep storing each
+ *                   chunk's ending adjoint (bf16), the per-chunk products that
+ *                   need them, and the chain rule through the decay factors.
+ *                   Workspace: one 145 KB unit per (64-token chunk slot, head)
+ *                   (0.61 GB for 8192 tokens x 32 heads).  Operands are bf16
+ *                   with fp32 accumulation, like the forward's tensor-core path.
+ *   KDA_BWD_SIMT    the fp32-record schedule on warp-level MMAs (any supported
+ *                   dtype and size; the workspace described above).
+ *   KDA_BWD_AUTO    TENSOR where it applies, else SIMT (what kda_chunk_backward does).
+ */
+#define KDA_BWD_AUTO 0
+#define KDA_BWD_TENSOR 1
+#define KDA_BWD_SIMT 2
+
+/* Workspace bytes kda_chunk_backward_ex needs with this dtype and algo (0 when the
+ * sizes are unsupported or KDA_BWD_TENSOR does not apply).  Never more than
+ * kda_chunk_backward_workspace_size for the same sizes. */
+size_t kda_chunk_backward_workspace_size_ex(int B, int T, int H, int dk, int dv, int num_seqs, int dtype,
+                                            int algo);
+
+/* kda_chunk_backward with an explicit schedule (KDA_BWD_*).  KDA_ERR_UNSUPPORTED
+ * when KDA_BWD_TENSOR is asked for inputs it does not cover; KDA_ERR_INVALID_ARG
+ * for an unknown algo; otherwise as kda_chunk_backward. */
+int kda_chunk_backward_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *init_state, const void *d_o,
+                          const float *dfinal_state, void *dq, void *dk_out, void *dv_out, float *dlog_alpha,
+                          float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
+                          int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
+                          void *stream, int algo);
 
 /*
  * Backward of the Gated DeltaNet prefill (kda_gdn_chunk_forward): the same

@@ -65,21 +65,35 @@ def run(d, c, **kw):
                               c.get("dfinal_state"), d.get("cu_seqlens"), **kw)
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, BF16])
+# (dtype, schedule): the tensor-core schedule covers bf16 with dk = dv = 128;
+# the SIMT schedule takes everything (AUTO picks it for the other sizes).
+SCHEDULES = [(torch.float32, "auto"), (BF16, "simt"), (BF16, "auto")]
+
+
+@pytest.mark.parametrize("dtype,algo", SCHEDULES)
 @pytest.mark.parametrize("B,T,H,dk,dv", [(2, 200, 2, 128, 128), (2, 130, 3, 64, 64), (1, 64, 2, 128, 64),
-                                         (3, 1, 2, 64, 128), (1, 333, 1, 128, 128)])
-def test_backward_matches_oracle(dtype, B, T, H, dk, dv):
+                                         (3, 1, 2, 64, 128), (1, 333, 1, 128, 128), (2, 64, 2, 128, 128),
+                                         (1, 129, 2, 128, 128)])
+def test_backward_matches_oracle(dtype, algo, B, T, H, dk, dv):
     shape = PrefillShape(B=B, T=T, H=H, dk=dk, dv=dv, dtype=dtype)
     d = prefill_inputs(shape, 100 + T + dk, DEV)
     c = backward_cotangents(shape, 200 + T, DEV)
-    got = run(d, c)
+    got = run(d, c, algo=algo)
     torch.cuda.synchronize()
-    check(got, oracle_grads(d, c), dtype, what=f"B{B} T{T} dk{dk} dv{dv}")
+    check(got, oracle_grads(d, c), dtype, what=f"{algo} B{B} T{T} dk{dk} dv{dv}")
     assert kda.device_status() == 0
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, BF16])
-def test_backward_packed_sequences(dtype):
+def test_backward_tensor_schedule_refuses_other_sizes():
+    shape = PrefillShape(B=1, T=64, H=1, dk=64, dv=64, dtype=BF16)
+    d = prefill_inputs(shape, 3, DEV)
+    c = backward_cotangents(shape, 4, DEV)
+    with pytest.raises(kda.KDAError):
+        run(d, c, algo="tensor")
+
+
+@pytest.mark.parametrize("dtype,algo", SCHEDULES)
+def test_backward_packed_sequences(dtype, algo):
     """Packed input with empty, single-token, exact-chunk and ragged sequences;
     equal bit for bit to running each sequence alone."""
     lens = [0, 1, 63, 64, 65, 130, 7, 0]
@@ -87,33 +101,34 @@ def test_backward_packed_sequences(dtype):
     shape = PrefillShape(B=1, T=sum(lens), H=3, dk=128, dv=128, dtype=dtype, cu_seqlens=cu)
     d = prefill_inputs(shape, 7, DEV)
     c = backward_cotangents(shape, 8, DEV)
-    got = run(d, c)
+    got = run(d, c, algo=algo)
     torch.cuda.synchronize()
-    check(got, oracle_grads(d, c), dtype, what="packed")
+    check(got, oracle_grads(d, c), dtype, what=f"packed {algo}")
     for n, L in enumerate(lens):
         a = cu[n]
         one = {x: d[x][:, a:a + L] for x in ("q", "k", "v", "log_alpha", "beta")}
         one["init_state"] = d["init_state"][n:n + 1]
         co = {"d_o": c["d_o"][:, a:a + L], "dfinal_state": c["dfinal_state"][n:n + 1]}
-        g1 = run(one, co)
+        g1 = run(one, co, algo=algo)
         for name in GRADS:
             whole = got[name][n:n + 1] if name == "dinit_state" else got[name][:, a:a + L]
             assert torch.equal(whole, g1[name]), (n, name)
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, BF16])
-def test_backward_strong_decay_blocks(dtype):
+@pytest.mark.parametrize("dtype,algo", SCHEDULES)
+def test_backward_strong_decay_blocks(dtype, algo):
     """Sequence 0 decays by ~3.5 per token (more than the in-block range the
-    diagonal blocks may take through a block boundary), sequence 1 as usual: both
-    the exact diagonal path and the tensor-core one run, and both match."""
+    diagonal blocks may take through a block boundary, and far past the chunk
+    range of the tensor-core chain rule), sequence 1 as usual: both the exact
+    path and the tensor-core one run, and both match."""
     shape = PrefillShape(B=2, T=160, H=2, dk=128, dv=128, dtype=dtype)
     d = prefill_inputs(shape, 77, DEV)
     gen = torch.Generator(device=DEV).manual_seed(79)
     d["log_alpha"][0] = -3.5 + 0.2 * torch.rand(d["log_alpha"][0].shape, generator=gen, device=DEV)
     c = backward_cotangents(shape, 78, DEV)
-    got = run(d, c)
+    got = run(d, c, algo=algo)
     torch.cuda.synchronize()
-    check(got, oracle_grads(d, c), dtype, what="strong decay")
+    check(got, oracle_grads(d, c), dtype, what=f"strong decay {algo}")
 
 
 def test_backward_without_states():
@@ -129,9 +144,10 @@ def test_backward_without_states():
     assert got["dinit_state"].abs().max().item() > 0
 
 
-def test_backward_no_tokens():
+@pytest.mark.parametrize("dv", [64, 128])
+def test_backward_no_tokens(dv):
     """T = 0: nothing to differentiate through; dinit_state = dfinal_state exactly."""
-    shape = PrefillShape(B=3, T=0, H=2, dk=128, dv=64, dtype=BF16)
+    shape = PrefillShape(B=3, T=0, H=2, dk=128, dv=dv, dtype=BF16)
     d = prefill_inputs(shape, 5, DEV)
     c = backward_cotangents(shape, 6, DEV)
     got = run(d, c)
@@ -143,12 +159,13 @@ def test_backward_no_tokens():
     assert torch.count_nonzero(got["dinit_state"]).item() == 0
 
 
-def test_backward_is_deterministic():
+@pytest.mark.parametrize("algo", ["simt", "tensor"])
+def test_backward_is_deterministic(algo):
     shape = PrefillShape(B=1, T=300, H=4, dk=128, dv=128, dtype=BF16)
     d = prefill_inputs(shape, 9, DEV)
     c = backward_cotangents(shape, 10, DEV)
-    a = run(d, c)
-    b = run(d, c)
+    a = run(d, c, algo=algo)
+    b = run(d, c, algo=algo)
     for name in GRADS:
         assert torch.equal(a[name], b[name]), name
 
@@ -165,13 +182,14 @@ def test_backward_skips_dinit_state():
 
 
 @pytest.mark.slow
-def test_backward_prefill_8k_sampled_heads():
+@pytest.mark.parametrize("algo", ["simt", "tensor"])
+def test_backward_prefill_8k_sampled_heads(algo):
     """Full-size prefill_8k (B=1, T=8192, H=32, d=128, bf16) in one call; the oracle
     runs on three of the 32 heads (heads are independent)."""
     shape = PrefillShape(B=1, T=8192, H=32, dk=128, dv=128, dtype=BF16)
     d = prefill_inputs(shape, 0, DEV)
     c = backward_cotangents(shape, 0, DEV)
-    got = run(d, c)
+    got = run(d, c, algo=algo)
     torch.cuda.synchronize()
     assert kda.device_status() == 0
     heads = [0, 17, 31]
@@ -202,7 +220,7 @@ def test_gdn_backward_matches_oracle(dtype, packed):
     want["dlog_alpha"] = want["dlog_alpha"].sum(axis=-1)
     check(got, want, dtype, what="gdn")
     # the same kernels with the rate broadcast and the channel gradients summed
-    full = run(d_b, c)
+    full = run(d_b, c, algo="simt")
     torch.testing.assert_close(got["dlog_alpha"], full["dlog_alpha"].sum(-1), rtol=1e-4, atol=1e-4)
     for name in ("dq", "dk", "dv", "dbeta", "dinit_state"):
         assert torch.equal(got[name], full[name]), name
