@@ -15,17 +15,17 @@
 //   dQhat = dO S^T,  dKhat = -mu S^T,  dKbar = U dS'^T,
 //   dS = Diag(D) dS' + Qhat^T dO - Khat^T mu,
 // then the chain rule through the decay factors and a reverse running sum for
-// dlog_alpha.  Five launches:
+// dlog_alpha.  Three launches:
 //   1. chunk_intra_kernel<BX>: the forward's first pass, plus Akk, Aqk and T;
-//   2. chunk_inter_kernel<CK>: the forward's state sweep, storing each chunk's
-//      starting state (bf16) instead of the output;
-//   3. chunk_adj_kernel: the adjoint sweep, chunks in reverse, storing each
-//      chunk's ending adjoint (bf16) and dS_0;
-//   4. bwd_grad_kernel (per chunk, head): every product above that needs S or
+//   2. bwd_sweeps_kernel: the two serial sweeps side by side -- the forward's state
+//      sweep storing each chunk's starting state (bf16) instead of the output
+//      (inter_body<CK>), and the adjoint sweep, chunks in reverse, storing each
+//      chunk's ending adjoint (bf16) and dS_0 (adj_body);
+//   3. bwd_grad_kernel (per chunk, head): every product above that needs S or
 //      dS', in a transposed form whose 128 rows are value or key channels
-//      (W^T, U^T, dU^T, lam^T: M = dv; the sums over the value columns: M = dk);
-//   5. bwd_chain_kernel (per chunk, head): the pair terms of dAqk and dAkk through
-//      e^{G_i - G_j} and the chain rule -> dq, dk, dlog_alpha.
+//      (W^T, U^T, dU^T, lam^T: M = dv; the sums over the value columns: M = dk),
+//      then the pair terms of dAqk and dAkk through e^{G_i - G_j} and the chain
+//      rule -> dq, dk, dv, dlog_alpha, dbeta.
 #pragma once
 
 #include <cstring>
@@ -59,10 +59,9 @@ constexpr uint32_t ACOL_DS = 128;   // [128 x DVT] Qhat^T dO - Khat^T mu
 // ignored), then dS = Diag(D) dS' + [Khat^T Qhat^T] [-mu; dO] (M = dk).
 // dS' of each chunk (its end) goes to the unit's DSC tile; dS_0 to dinit_state.
 template <int DK, int DVT, int NBUF>
-__global__ void __launch_bounds__(NT, 1)
-chunk_adj_kernel(const __grid_constant__ CUtensorMap tm_do, uint8_t *__restrict__ ws,
-                 const float *__restrict__ dfinal, float *__restrict__ dinit_state,
-                 const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
+__device__ __forceinline__ void adj_body(int tile, const CUtensorMap *tm_do, uint8_t *__restrict__ ws,
+                                         const float *__restrict__ dfinal, float *__restrict__ dinit_state,
+                                         const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
     using L = AdjLayout<DK, DVT, NBUF>;
     using R = Rec<DK>;
     using U = BwdUnit<DK>;
@@ -79,7 +78,7 @@ chunk_adj_kernel(const __grid_constant__ CUtensorMap tm_do, uint8_t *__restrict_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
-    const int col_base = blockIdx.x * DVT, h = blockIdx.y;
+    const int col_base = tile * DVT, h = blockIdx.y;
     const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
     long long t0, t1;
     seq_span(cu_seqlens, T, n, t0, t1);
@@ -94,7 +93,7 @@ chunk_adj_kernel(const __grid_constant__ CUtensorMap tm_do, uint8_t *__restrict_
         for (int b = 0; b < NBUF; ++b) ptx::mbar_init(bar_rec + 8 * b, 1);
         ptx::mbar_init(bar_mma, 1);
         ptx::fence_mbar_init();
-        if (nck > 0) ptx::prefetch_tmap(&tm_do);
+        if (nck > 0) ptx::prefetch_tmap(tm_do);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -110,7 +109,7 @@ chunk_adj_kernel(const __grid_constant__ CUtensorMap tm_do, uint8_t *__restrict_
         const uint32_t bar = bar_rec + 8 * b;
         ptx::mbar_arrive_expect_tx(bar, TX);
         ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * U::BYTES, (uint32_t)R::BYTES, bar);
-        ptx::tma_load_3d(sb + L::DOT + b * C * DVT * 2, &tm_do, bar, col_base, h, (int)(t0 + (long long)ci * C));
+        ptx::tma_load_3d(sb + L::DOT + b * C * DVT * 2, tm_do, bar, col_base, h, (int)(t0 + (long long)ci * C));
     };
 
     const int srow = quad * 32 + lane;
@@ -238,6 +237,28 @@ chunk_adj_kernel(const __grid_constant__ CUtensorMap tm_do, uint8_t *__restrict_
     }
 }
 
+// Both state sweeps in one launch (they are independent): CTAs with
+// blockIdx.x < DV / DVT run the forward sweep (chunk-start states), the others the
+// adjoint sweep, one per (value tile, head, sequence) each.
+template <int DK, int DVT, int NBUF>
+__global__ void __launch_bounds__(NT, 1)
+bwd_sweeps_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  uint8_t *__restrict__ ws, const float *__restrict__ init_state, const float *__restrict__ dfinal,
+                  float *__restrict__ dinit_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
+    const int nt = DV / DVT;
+    if ((int)blockIdx.x < nt)
+        inter_body<DK, DVT, NBUF, true>((int)blockIdx.x, &tm_v, ws, init_state, nullptr, nullptr, cu_seqlens, T, H,
+                                        DV, nullptr, 0, ws);
+    else
+        adj_body<DK, DVT, NBUF>((int)blockIdx.x - nt, &tm_do, ws, dfinal, dinit_state, cu_seqlens, T, H, DV);
+}
+
+template <int DK, int DVT, int NBUF>
+constexpr int sweeps_smem() {
+    return InterLayout<DK, DVT, NBUF>::ALLOC > AdjLayout<DK, DVT, NBUF>::ALLOC ? InterLayout<DK, DVT, NBUF>::ALLOC
+                                                                               : AdjLayout<DK, DVT, NBUF>::ALLOC;
+}
+
 // ------------------------------------------------------------------ per-chunk sums
 
 // Chunk of `slot`: the last sequence n whose first slot n + floor(t0_n / 64) is
@@ -331,6 +352,7 @@ __device__ __forceinline__ float warp_transpose_sum32(float (&x)[32]) {
 }
 
 struct GradLayout {   // dk = dv = 128; bf16 tiles with a 128-byte swizzle unless noted
+    // phases 1-3
     static constexpr int KH = 0;                // [2][64][128 B]   Khat rows (K-major B, N = tokens)
     static constexpr int EX = 16384;            // BwdX             Akk | Aqk | T
     static constexpr int SS = 40960;            // [2][128][128 B]  S at the chunk's start
@@ -340,32 +362,111 @@ struct GradLayout {   // dk = dv = 128; bf16 tiles with a 128-byte swizzle unles
     static constexpr int VV = 155648;           // [64][128]        V, no swizzle
     static constexpr int AW = 172032;           // [128][128 B]     (Diag(beta) W)^T, then U^T
     static constexpr int ADU = 188416;          // [128][128 B]     dU^T, then -mu rows [2][64][128 B]
-    static constexpr int FB = 204800;           // fp32 [64]        beta
-    static constexpr int FD = FB + 256;         // fp32 [128]       e^{G_last}
-    static constexpr int FSEG = FD + 512;       // fp32 [8][128]    segment sums
-    static constexpr int FDB = FSEG + 4096;     // fp32 [4][64]     <lam, W> per lane quadrant
-    static constexpr int FDB2 = FDB + 1024;     // fp32 [2][64]     sum_j Akk L per column half
-    static constexpr int FGC = FDB2 + 512;      // fp32 [2][128]    sum_v S dS' per column half
-    static constexpr int MISC = FGC + 1024;     // mbarriers, TMEM base
+    // the chain rule, over tiles that phase 3 has finished with
+    static constexpr int DA = KH;               // [128][128 B]     dAkk rows 0-63, dAqk rows 64-127
+    static constexpr int KE = SS;               // [2 parts][2][64][128 B]  e^{-G} K: bf16 high part, low part
+    static constexpr int KQE = DS;              // [2 parts][2][128][128 B] e^{G - G_last} [K; Q], high, low
+    static constexpr int FG = KBR;              // fp32 [64][128]   G
+    static constexpr int QR = AW;               // bf16 [64][128]   q, no swizzle
+    static constexpr int KR = ADU;              // bf16 [64][128]   k, no swizzle
+    // fp32 scratch
+    static constexpr int FB = 204800;           // [64]        beta
+    static constexpr int FD = FB + 256;         // [128]       e^{G_last}
+    static constexpr int FSEG = FD + 512;       // [8][128]    segment sums
+    static constexpr int FDB = FSEG + 4096;     // [4][64]     <lam, W> per lane quadrant
+    static constexpr int FDB2 = FDB + 1024;     // [2][64]     sum_j Akk L per column half
+    static constexpr int FGC = FDB2 + 512;      // [2][128]    sum_v S dS' per column half
+    static constexpr int FX = FGC + 1024;       // [2][2][128] per token half: sum_i k_i b_i, sum_i dG_i
+    static constexpr int MISC = FX + 2048;      // mbarriers, TMEM base
     static constexpr int BYTES = MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;
+    static_assert(KE + 2 * 16384 <= KQE && KQE + 2 * 32768 <= FG && FG + 32768 <= QR && QR + 16384 <= KR &&
+                      KR + 16384 <= FB,
+                  "chain-rule tiles over the dead phase 1-3 tiles");
     static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
 constexpr uint32_t GRAD_TMEM_COLS = 256;
-// TMEM columns, 64 each: phase 1 W-part and dU^T; phase 2 U^T, lam^T; phase 3
-// [dAqk; L], S dO^T, -S mu^T, dS' U^T
+// TMEM columns, 64 each.  Phase 1: S^T Khat^T, dU^T.  Phase 2: U^T, lam^T.  Phase 3:
+// [dAqk; L], S dO^T, -S mu^T, dS' U^T.  Phase 4 (tier A) adds the row terms onto
+// S dO^T and -S mu^T (the same factor e^G scales both) and puts the column terms
+// over [dAqk; L], which has been read out.
 constexpr uint32_t GC_0 = 0, GC_1 = 64, GC_2 = 128, GC_3 = 192;
+
+// bf16 element (r, j) of a one-atom (64-column) tile with a 128-byte swizzle.
+__device__ __forceinline__ float ld_sw128(const uint8_t *tile, int r, int j) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + r * 128 + ((((j >> 3) ^ (r & 7))) << 4) +
+                                                                      ((j & 7) << 1)));
+}
+
+// Four values as a bf16 high part and the bf16 rounding of the remainder.
+__device__ __forceinline__ void st_split_bf16x4(uint8_t *sm, uint32_t hi, uint32_t lo, const float (&x)[4]) {
+    float h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        h[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+        l[e] = x[e] - h[e];
+    }
+    st_bf16x4(sm, hi, h[0], h[1], h[2], h[3]);
+    st_bf16x4(sm, lo, l[0], l[1], l[2], l[3]);
+}
+
+// Tier B of the chain rule (a chunk decaying faster than the tensor-core factors
+// cover): the exact pair terms RQ, RK, CT of key channel c for tokens i0 .. i0+31,
+// into fp32 [3][64][128] at out.  Kept out of line and not unrolled: it runs only
+// for such chunks.
+__device__ __noinline__ void chain_pairs_exact(const uint8_t *da, const float *fG, const __nv_bfloat16 *sq,
+                                               const __nv_bfloat16 *sk, int c, int i0, float *out) {
+    constexpr int DK = 128;
+#pragma unroll 1
+    for (int i = i0; i < i0 + 32; ++i) {
+        const float Gi = fG[i * DK + c];
+        float RQ = 0.f, RK = 0.f, CT = 0.f;
+#pragma unroll 1
+        for (int j = 0; j <= i; ++j) {
+            const float f = __expf(Gi - fG[j * DK + c]) * __bfloat162float(sk[j * DK + c]);
+            RQ = fmaf(ld_sw128(da, 64 + i, j), f, RQ);
+            RK = fmaf(ld_sw128(da, i, j), f, RK);
+        }
+#pragma unroll 1
+        for (int m = i; m < C; ++m) {
+            const float f = __expf(fG[m * DK + c] - Gi);
+            const float x = ld_sw128(da, 64 + m, i) * __bfloat162float(sq[m * DK + c]) +
+                            ld_sw128(da, m, i) * __bfloat162float(sk[m * DK + c]);
+            CT = fmaf(x, f, CT);
+        }
+        out[i * DK + c] = RQ;
+        out[C * DK + i * DK + c] = RK;
+        out[2 * C * DK + i * DK + c] = CT;
+    }
+}
 
 // One CTA per (chunk slot, head), 256 threads.  Warps w and w + 4 share TMEM lane
 // quadrant w & 3 (value channel or key channel 32 (w & 3) + lane) and split the 64
-// token columns in halves.  Writes dV and dbeta, and over the chunk's own unit the
-// sums XQ, XK, XB, the masked dAkk/dAqk tile and DGC for bwd_chain_kernel.
+// token columns in halves.
+//   Phases 1-3: every product that needs S or dS' -> dV, dbeta, dAqk/dAkk and
+//   dQhat^T, dKhat^T, dKbar^T (M = key channels), kept in TMEM.
+//   Phase 4, the chain rule through the decay factors, with the pair terms of
+//   channel c
+//     RQ_i = sum_{j<=i} dAqk[i][j] e^{G_i-G_j} k_j,  RK_i = sum_{j<i} dAkk[i][j] e^{G_i-G_j} k_j,
+//     CT_j = sum_{i>=j} (dAqk[i][j] q_i + dAkk[i][j] k_i) e^{G_i-G_j}.
+//   Tier A (every channel's chunk decay >= -DECAY_LIM): RQ = e^{G_i} [(e^{-G} K)^T dAqk^T]_i,
+//   RK likewise, CT = e^{G_last - G_j} [(e^{G - G_last} [K; Q])^T [dAkk; dAqk]]_j on the
+//   tensor cores: every operand factor is >= 1 and <= e^DECAY_LIM and the products are
+//   scaled down afterwards, so no gradient underflows on the way; the decay-scaled
+//   operands are split into a bf16 high and low part (two products), because each
+//   pair term enters dG_i and dG_j with opposite signs and cancels in the running
+//   sum of dlog_alpha only as far as its two roundings agree.  Tier B: the exact
+//   sums on the CUDA cores.  Then, with a = e^G dKhat + RK, b = e^{G_last - G} dKbar:
+//     dq = e^G dQhat + RQ,  dk = a + b + CT,  dG = q dq + k (a - b - CT),
+//     dlog_alpha_t = e^{G_last} sum_v S dS' + sum_i k_i b_i + sum_{i>=t} dG_i.
 __global__ void __launch_bounds__(NT, 1)
 bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_v,
-                const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
-                const float *__restrict__ beta, __nv_bfloat16 *__restrict__ dv_out, float *__restrict__ dbeta,
-                const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, uint8_t *__restrict__ ws) {
+                const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, const uint8_t *__restrict__ ws,
+                __nv_bfloat16 *__restrict__ dq, __nv_bfloat16 *__restrict__ dk_out, __nv_bfloat16 *__restrict__ dv_out,
+                float *__restrict__ dlog_alpha, float *__restrict__ dbeta) {
     using L = GradLayout;
     using R = Rec<128>;
     using U = BwdUnit<128>;
@@ -378,12 +479,13 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
     float *fB = reinterpret_cast<float *>(sm + L::FB), *fD = reinterpret_cast<float *>(sm + L::FD);
     float *fSeg = reinterpret_cast<float *>(sm + L::FSEG), *fDB = reinterpret_cast<float *>(sm + L::FDB);
     float *fDB2 = reinterpret_cast<float *>(sm + L::FDB2), *fGC = reinterpret_cast<float *>(sm + L::FGC);
+    float *fX = reinterpret_cast<float *>(sm + L::FX), *fG = reinterpret_cast<float *>(sm + L::FG);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, half = warp >> 2;
     const int slot = blockIdx.x, h = blockIdx.y;
     long long cs;
     int Lc;
     if (!slot_chunk(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
-    uint8_t *unit = ws + ((size_t)slot * H + h) * U::BYTES;
+    const uint8_t *unit = ws + ((size_t)slot * H + h) * U::BYTES;
 
     if (warp == 0) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), GRAD_TMEM_COLS);
@@ -404,11 +506,12 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
         ptx::tma_load_3d(sb + L::VV, &tm_v, bar_ld, 0, h, (int)cs);
     }
     if (tid < C) fB[tid] = tid < Lc ? beta[(cs + tid) * H + h] : 0.f;
+    // G, k and q of this thread's 8 tokens x 4 channels, kept for phase 4
+    float G[8][4], tot[4];
+    uint2 kv[8], qv[8];
+    chunk_decay<true>(q, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
+    const int c0 = 4 * (tid & 31), i0 = 8 * (tid >> 5);
     {   // Kbar = e^{G_last - G} K (factors <= 1) and e^{G_last}, while the copies fly
-        float G[8][4], tot[4];
-        uint2 kv[8], qv[8];
-        chunk_decay<false>(nullptr, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
-        const int c0 = 4 * (tid & 31), i0 = 8 * (tid >> 5);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const float4 k4 = bf16x4_to_float4(kv[u]);
@@ -419,7 +522,8 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
                                                                          __expf(tot[2]), __expf(tot[3]));
     }
     ptx::tc_fence_before();
-    __syncthreads();
+    const bool strong = __syncthreads_or(tot[0] < -DECAY_LIM || tot[1] < -DECAY_LIM || tot[2] < -DECAY_LIM ||
+                                         tot[3] < -DECAY_LIM) != 0;   // uniform: tier B
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
@@ -563,20 +667,19 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
         }
         fGC[half * 128 + vr] = acc;
     }
-    if (ok) ok = wait_all(bar_mma, ph_mma);
+    if (ok) ok = wait_all(bar_mma, ph_mma);   // phase 1-3 tiles are free from here on
     if (ok) {
-        // the chunk's unit is no longer read by anyone: the sums go over it
+        // dA -> the bf16 tile (masked): rows 0-63 of TMEM hold dAqk, rows 64-127 L = lam U^T
         float x[32];
         ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
         ptx::tmem_wait_ld();
-        if (quad < 2) {   // rows 0-63: dAqk (j <= i) -> unit rows 64-127 of DA
+        if (quad < 2) {   // dAqk (j <= i) -> rows 64-127 of DA
             const int i = vr;
 #pragma unroll
             for (int u = 0; u < 32; ++u) x[u] = (32 * half + u <= i) ? x[u] : 0.f;
 #pragma unroll
-            for (int gq = 0; gq < 4; ++gq)
-                st_global_bf16x8(unit + U::DA + sw128_chunk(64 + i, 4 * half + gq), x + 8 * gq);
-        } else {          // rows 64-127: L = lam U^T -> dAkk = -beta_i L (j < i), and sum_j Akk L
+            for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::DA + sw128_chunk(64 + i, 4 * half + gq), x + 8 * gq);
+        } else {          // dAkk = -beta_i L (j < i) -> rows 0-63 of DA; and sum_j Akk L for dbeta
             const int i = vr - 64;
             const float bi = fB[i];
             float dot = 0.f, a8[8];
@@ -591,28 +694,130 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
 #pragma unroll
             for (int u = 0; u < 32; ++u) x[u] = (32 * half + u < i) ? -bi * x[u] : 0.f;
 #pragma unroll
-            for (int gq = 0; gq < 4; ++gq)
-                st_global_bf16x8(unit + U::DA + sw128_chunk(i, 4 * half + gq), x + 8 * gq);
+            for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::DA + sw128_chunk(i, 4 * half + gq), x + 8 * gq);
         }
-        // XQ, XK, XB: row = key channel vr, columns 32 half .. (fp32, 128 contiguous bytes per thread)
-#pragma unroll 1
-        for (int m = 0; m < 3; ++m) {
-            ptx::tmem_ld32(tl + GC_1 + 64 * m + 32 * half, x);
-            ptx::tmem_wait_ld();
-            float *dst = reinterpret_cast<float *>(unit + U::XQ + m * (DK * C * 4)) + vr * C + 32 * half;
+        // G, raw q and k (row-major), and in tier A the split decay-scaled operands
 #pragma unroll
-            for (int u = 0; u < 32; u += 4)
-                *reinterpret_cast<float4 *>(dst + u) = make_float4(x[u], x[u + 1], x[u + 2], x[u + 3]);
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u;
+            *reinterpret_cast<float4 *>(fG + i * DK + c0) = make_float4(G[u][0], G[u][1], G[u][2], G[u][3]);
+            *reinterpret_cast<uint2 *>(sm + L::QR + (i * DK + c0) * 2) = qv[u];
+            *reinterpret_cast<uint2 *>(sm + L::KR + (i * DK + c0) * 2) = kv[u];
+            if (!strong) {
+                const float4 k4 = bf16x4_to_float4(kv[u]), q4 = bf16x4_to_float4(qv[u]);
+                const float kq[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
+                float xe[4], xk[4], xq[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float en = __expf(-G[u][e]), er = __expf(G[u][e] - tot[e]);   // <= e^DECAY_LIM
+                    xe[e] = kq[e] * en;
+                    xk[e] = kq[e] * er;
+                    xq[e] = qq[e] * er;
+                }
+                st_split_bf16x4(sm, L::KE + sw128(i, c0, 64), L::KE + 16384 + sw128(i, c0, 64), xe);
+                st_split_bf16x4(sm, L::KQE + sw128(i, c0, 128), L::KQE + 32768 + sw128(i, c0, 128), xk);
+                st_split_bf16x4(sm, L::KQE + sw128(64 + i, c0, 128), L::KQE + 32768 + sw128(64 + i, c0, 128), xq);
+            }
         }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    // ---- phase 4 (tier A): row terms onto S dO^T and -S mu^T; column terms over dA
+    if (ok && !strong) {
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t i_mk = ptx::idesc_bf16_f32(128, 64, true, false);
+            constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t ke = sb + L::KE + part * 16384, kqe = sb + L::KQE + part * 32768;
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(ke + s * 2048, 8192, 1024),
+                                  kdesc(sb + L::DA + 8192, s, 64), i_mk, 1);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    ptx::mma_bf16(tmem + GC_2, ptx::desc_mnmajor_sw128(ke + s * 2048, 8192, 1024),
+                                  kdesc(sb + L::DA, s, 64), i_mk, 1);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    ptx::mma_bf16(tmem + GC_0, ptx::desc_mnmajor_sw128(kqe + s * 2048, 16384, 1024),
+                                  ptx::desc_mnmajor_sw128(sb + L::DA + s * 2048, 8192, 1024), i_mm, part > 0 || s > 0);
+            }
+            ptx::mma_commit(bar_mma);
+            ++n_commit;
+        }
+        ok = wait_all(bar_mma, ph_mma);
+    }
+
+    // ---- readout: thread (key channel c, token half)
+    const int c = vr;
+    const float gl = fG[(C - 1) * DK + c];   // G_last (rows past Lc add nothing)
+    const float *fP = reinterpret_cast<const float *>(sm + L::KE);   // tier B: exact RQ, RK, CT
+    if (ok && strong)
+        chain_pairs_exact(sm + L::DA, fG, reinterpret_cast<const __nv_bfloat16 *>(sm + L::QR),
+                          reinterpret_cast<const __nv_bfloat16 *>(sm + L::KR), c, 32 * half,
+                          reinterpret_cast<float *>(sm + L::KE));
+    const __nv_bfloat16 *sq = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QR);
+    const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KR);
+    float dG[32], kb = 0.f, sdg = 0.f;
+    if (ok) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            float t1[16], t2[16], t3[16], t0[16];
+            const uint32_t col = 32 * half + 16 * cc;
+            ptx::tmem_ld16(tl + GC_1 + col, t1);
+            ptx::tmem_ld16(tl + GC_2 + col, t2);
+            ptx::tmem_ld16(tl + GC_3 + col, t3);
+            if (!strong) ptx::tmem_ld16(tl + GC_0 + col, t0);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int i = col + u;
+                const float Gi = fG[i * DK + c];
+                const float qi = __bfloat162float(sq[i * DK + c]), ki = __bfloat162float(sk[i * DK + c]);
+                const float eg = __expf(Gi), eb = __expf(gl - Gi);
+                float RQ = 0.f, RK = 0.f, CT;
+                if (!strong) {
+                    CT = eb * t0[u];
+                } else {
+                    RQ = fP[i * DK + c];
+                    RK = fP[C * DK + i * DK + c];
+                    CT = fP[2 * C * DK + i * DK + c];
+                }
+                const float dqi = fmaf(eg, t1[u], RQ);
+                const float a = fmaf(eg, t2[u], RK), b = eb * t3[u];
+                const float dki = a + b + CT;
+                const float g = qi * dqi + ki * (a - b - CT);
+                dG[16 * cc + u] = g;
+                sdg += g;
+                kb = fmaf(ki, b, kb);
+                if (i < Lc) {
+                    const long long o = ((cs + i) * H + h) * DK + c;
+                    dq[o] = __float2bfloat16_rn(dqi);
+                    dk_out[o] = __float2bfloat16_rn(dki);
+                }
+            }
+        }
+        fX[half * DK + c] = kb;
+        fX[2 * DK + half * DK + c] = sdg;
     }
     __syncthreads();
     if (ok) {
+        float run = fD[c] * (fGC[c] + fGC[128 + c]) + fX[c] + fX[DK + c];
+        if (half == 0) run += fX[2 * DK + DK + c];   // all of the later half's dG
+#pragma unroll
+        for (int u = 31; u >= 0; --u) {
+            const int i = 32 * half + u;
+            run += dG[u];
+            if (i < Lc) dlog_alpha[((cs + i) * H + h) * DK + c] = run;
+        }
         if (tid < C && tid < Lc) {
             const float db = fDB[tid] + fDB[64 + tid] + fDB[128 + tid] + fDB[192 + tid] - fDB2[tid] - fDB2[64 + tid];
             dbeta[(cs + tid) * H + h] = db;
         }
-        if (tid < DK)
-            reinterpret_cast<float *>(unit + U::DGC)[tid] = fD[tid] * (fGC[tid] + fGC[128 + tid]);
     }
     if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded)
         ptx::mbar_wait_bounded(bar_ld, 0u, WAIT_LIMIT_CYCLES);
@@ -623,243 +828,6 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
     if (warp == 0) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, GRAD_TMEM_COLS);
-    }
-}
-
-// ------------------------------------------------------------------ chain rule
-
-struct ChainLayout {   // dk = 128
-    static constexpr int DA = 0;                // bf16 [128][128 B]  dAkk rows 0-63, dAqk rows 64-127
-    static constexpr int KE = 16384;            // tier A: bf16 [2][64][128 B] e^{-G} K (MN-major A, M = key channels)
-    static constexpr int KQE = 32768;           // tier A: bf16 [2][128][128 B] e^{G - G_last} [K; Q];
-                                                //   tier B: q then k, bf16 [64][128] each, no swizzle
-    static constexpr int FG = 65536;            // fp32 [64][128] G
-    static constexpr int FSEG = FG + 32768;     // fp32 [8][128]  segment sums
-    static constexpr int FX = FSEG + 4096;      // fp32 [2][2][128] per column half: sum_i k_i b_i, sum_i dG_i
-    static constexpr int MISC = FX + 2048;      // mbarriers, TMEM base
-    static constexpr int BYTES = MISC + 64;
-    static constexpr int ALLOC = BYTES + 1024;
-    static_assert(2 * (ALLOC + 1024) <= 233472, "two CTAs per SM");
-};
-
-constexpr uint32_t CHAIN_TMEM_COLS = 256;
-constexpr uint32_t HC_RQ = 0, HC_RK = 64, HC_CT = 128;
-
-// bf16 element (r, j) of a one-atom (64-column) tile with a 128-byte swizzle.
-__device__ __forceinline__ float ld_sw128(const uint8_t *tile, int r, int j) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + r * 128 + ((((j >> 3) ^ (r & 7))) << 4) +
-                                                                      ((j & 7) << 1)));
-}
-
-// One CTA per (chunk slot, head), 256 threads; thread (key channel c = 32 (w & 3) +
-// lane, token half w >> 2).  With dA = (dAkk, dAqk) from bwd_grad_kernel, the pair
-// terms of channel c are
-//   row terms  RQ_i = sum_{j<=i} dAqk[i][j] e^{G_i-G_j} k_j,  RK_i = sum_{j<i} dAkk[i][j] e^{G_i-G_j} k_j,
-//   col terms  CT_j = sum_{i>=j} (dAqk[i][j] q_i + dAkk[i][j] k_i) e^{G_i-G_j}.
-// Tier A (every channel's chunk decay >= -DECAY_LIM): RQ = e^{G_i} [(e^{-G} K)^T dAqk^T]_i,
-// RK likewise, CT = e^{G_last - G_j} [(e^{G - G_last} [K; Q])^T [dAkk; dAqk]]_j on the
-// tensor cores: every operand factor is >= 1 and <= e^DECAY_LIM and the products are
-// scaled down afterwards, so no gradient underflows on the way.  Tier B: the exact
-// sums on the CUDA cores.  Then, with a = e^G dKhat + RK, b = e^{G_last - G} dKbar:
-//   dq = e^G dQhat + RQ,  dk = a + b + CT,  dG = q dq + k (a - b - CT),
-//   dlog_alpha_t = e^{G_last} sum_v S dS' + sum_i k_i b_i + sum_{i>=t} dG_i.
-__global__ void __launch_bounds__(NT, 2)
-bwd_chain_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                 const float *__restrict__ log_alpha, const int32_t *__restrict__ cu_seqlens, int T, int H,
-                 int num_seqs, const uint8_t *__restrict__ ws, __nv_bfloat16 *__restrict__ dq,
-                 __nv_bfloat16 *__restrict__ dk_out, float *__restrict__ dlog_alpha) {
-    using L = ChainLayout;
-    using U = BwdUnit<128>;
-    constexpr int DK = 128;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const uint32_t sb = ptx::smem_u32(sm);
-    const uint32_t bar_ld = sb + L::MISC, bar_mma = sb + L::MISC + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 16);
-    float *fG = reinterpret_cast<float *>(sm + L::FG), *fSeg = reinterpret_cast<float *>(sm + L::FSEG);
-    float *fX = reinterpret_cast<float *>(sm + L::FX);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, half = warp >> 2;
-    const int slot = blockIdx.x, h = blockIdx.y;
-    long long cs;
-    int Lc;
-    if (!slot_chunk(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
-    const uint8_t *unit = ws + ((size_t)slot * H + h) * U::BYTES;
-
-    if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), CHAIN_TMEM_COLS);
-        ptx::tmem_relinquish();
-    }
-    if (tid == 0) {
-        ptx::mbar_init(bar_ld, 1);
-        ptx::mbar_init(bar_mma, 1);
-        ptx::fence_mbar_init();
-        ptx::mbar_arrive_expect_tx(bar_ld, 16384u);
-        ptx::bulk_load(sb + L::DA, unit + U::DA, 16384u, bar_ld);
-    }
-    bool strong;
-    {
-        float G[8][4], tot[4];
-        uint2 kv[8], qv[8];
-        chunk_decay<true>(q, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
-        const int c0 = 4 * (tid & 31), i0 = 8 * (tid >> 5);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<float4 *>(fG + (i0 + u) * DK + c0) = make_float4(G[u][0], G[u][1], G[u][2], G[u][3]);
-        strong = __syncthreads_or(tot[0] < -DECAY_LIM || tot[1] < -DECAY_LIM || tot[2] < -DECAY_LIM ||
-                                  tot[3] < -DECAY_LIM) != 0;
-        if (!strong) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u;
-                const float4 k4 = bf16x4_to_float4(kv[u]), q4 = bf16x4_to_float4(qv[u]);
-                float en[4], er[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    en[e] = __expf(-G[u][e]);             // <= e^DECAY_LIM
-                    er[e] = __expf(G[u][e] - tot[e]);     // <= e^DECAY_LIM
-                }
-                st_bf16x4(sm, L::KE + sw128(i, c0, 64), k4.x * en[0], k4.y * en[1], k4.z * en[2], k4.w * en[3]);
-                st_bf16x4(sm, L::KQE + sw128(i, c0, 128), k4.x * er[0], k4.y * er[1], k4.z * er[2], k4.w * er[3]);
-                st_bf16x4(sm, L::KQE + sw128(64 + i, c0, 128), q4.x * er[0], q4.y * er[1], q4.z * er[2],
-                          q4.w * er[3]);
-            }
-        } else {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                *reinterpret_cast<uint2 *>(sm + L::KQE + ((i0 + u) * DK + c0) * 2) = qv[u];
-                *reinterpret_cast<uint2 *>(sm + L::KQE + 16384 + ((i0 + u) * DK + c0) * 2) = kv[u];
-            }
-        }
-    }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t ph_ld = 0, ph_mma = 0;
-    bool ok = wait_all(bar_ld, ph_ld);
-    bool mma_pending = false;
-    if (ok && !strong) {
-        if (tid == 0) {
-            constexpr uint32_t i_mk = ptx::idesc_bf16_f32(128, 64, true, false);
-            constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + HC_RQ, ptx::desc_mnmajor_sw128(sb + L::KE + s * 2048, 8192, 1024),
-                              kdesc(sb + L::DA + 8192, s, 64), i_mk, s > 0);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + HC_RK, ptx::desc_mnmajor_sw128(sb + L::KE + s * 2048, 8192, 1024),
-                              kdesc(sb + L::DA, s, 64), i_mk, s > 0);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                ptx::mma_bf16(tmem + HC_CT, ptx::desc_mnmajor_sw128(sb + L::KQE + s * 2048, 16384, 1024),
-                              ptx::desc_mnmajor_sw128(sb + L::DA + s * 2048, 8192, 1024), i_mm, s > 0);
-            ptx::mma_commit(bar_mma);
-        }
-        mma_pending = true;
-        ok = wait_all(bar_mma, ph_mma);
-        mma_pending = !ok;
-    }
-
-    const int c = quad * 32 + lane;
-    const float gl = fG[(C - 1) * DK + c];   // G_last (rows past Lc add nothing)
-    const float *xq = reinterpret_cast<const float *>(unit + U::XQ) + c * C + 32 * half;
-    const float *xk = reinterpret_cast<const float *>(unit + U::XK) + c * C + 32 * half;
-    const float *xb = reinterpret_cast<const float *>(unit + U::XB) + c * C + 32 * half;
-    const uint8_t *da = sm + L::DA;
-    const __nv_bfloat16 *sq = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KQE);
-    const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KQE + 16384);
-    float dG[32], kb = 0.f, sdg = 0.f;
-    if (ok) {
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            float rq[16], rk[16], ct[16];
-            if (!strong) {
-                ptx::tmem_ld16(tl + HC_RQ + 32 * half + 16 * cc, rq);
-                ptx::tmem_ld16(tl + HC_RK + 32 * half + 16 * cc, rk);
-                ptx::tmem_ld16(tl + HC_CT + 32 * half + 16 * cc, ct);
-                ptx::tmem_wait_ld();
-            }
-#pragma unroll
-            for (int u4 = 0; u4 < 16; u4 += 4) {
-                const float4 xq4 = *reinterpret_cast<const float4 *>(xq + 16 * cc + u4);
-                const float4 xk4 = *reinterpret_cast<const float4 *>(xk + 16 * cc + u4);
-                const float4 xb4 = *reinterpret_cast<const float4 *>(xb + 16 * cc + u4);
-                const float vq[4] = {xq4.x, xq4.y, xq4.z, xq4.w};
-                const float vk[4] = {xk4.x, xk4.y, xk4.z, xk4.w};
-                const float vb[4] = {xb4.x, xb4.y, xb4.z, xb4.w};
-                float qi[4], ki[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const int i = 32 * half + 16 * cc + u4 + w;
-                    const long long off = ((cs + min(i, Lc - 1)) * H + h) * DK + c;
-                    qi[w] = i < Lc ? __bfloat162float(q[off]) : 0.f;
-                    ki[w] = i < Lc ? __bfloat162float(k[off]) : 0.f;
-                }
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const int u = u4 + w, i = 32 * half + 16 * cc + u;
-                    const float Gi = fG[i * DK + c];
-                    const float eg = __expf(Gi), eb = __expf(gl - Gi);
-                    float RQ, RK, CT;
-                    if (!strong) {
-                        RQ = eg * rq[u];
-                        RK = eg * rk[u];
-                        CT = eb * ct[u];
-                    } else {   // exact pair terms of this (token, channel)
-                        RQ = 0.f; RK = 0.f; CT = 0.f;
-                        for (int j = 0; j <= i; ++j) {
-                            const float f = __expf(Gi - fG[j * DK + c]) * __bfloat162float(sk[j * DK + c]);
-                            RQ = fmaf(ld_sw128(da, 64 + i, j), f, RQ);
-                            RK = fmaf(ld_sw128(da, i, j), f, RK);
-                        }
-                        for (int m = i; m < C; ++m) {
-                            const float f = __expf(fG[m * DK + c] - Gi);
-                            const float x = ld_sw128(da, 64 + m, i) * __bfloat162float(sq[m * DK + c]) +
-                                            ld_sw128(da, m, i) * __bfloat162float(sk[m * DK + c]);
-                            CT = fmaf(x, f, CT);
-                        }
-                    }
-                    const float dqi = fmaf(eg, vq[w], RQ);
-                    const float a = fmaf(eg, vk[w], RK), b = eb * vb[w];
-                    const float dki = a + b + CT;
-                    const float g = qi[w] * dqi + ki[w] * (a - b - CT);
-                    dG[16 * cc + u] = g;
-                    sdg += g;
-                    kb = fmaf(ki[w], b, kb);
-                    if (i < Lc) {
-                        const long long o = ((cs + i) * H + h) * DK + c;
-                        dq[o] = __float2bfloat16_rn(dqi);
-                        dk_out[o] = __float2bfloat16_rn(dki);
-                    }
-                }
-            }
-        }
-        fX[half * DK + c] = kb;
-        fX[2 * DK + half * DK + c] = sdg;
-    }
-    __syncthreads();
-    if (ok) {
-        float run = reinterpret_cast<const float *>(unit + U::DGC)[c] + fX[c] + fX[DK + c];
-        if (half == 0) run += fX[2 * DK + DK + c];   // all of the later half's dG
-#pragma unroll
-        for (int u = 31; u >= 0; --u) {
-            const int i = 32 * half + u;
-            run += dG[u];
-            if (i < Lc) dlog_alpha[((cs + i) * H + h) * DK + c] = run;
-        }
-    }
-    if (!ok && tid == 0) {   // a wait timed out: let the copy and MMAs in flight land (bounded)
-        ptx::mbar_wait_bounded(bar_ld, 0u, WAIT_LIMIT_CYCLES);
-        if (mma_pending) ptx::mbar_wait_bounded(bar_mma, 0u, WAIT_LIMIT_CYCLES);
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, CHAIN_TMEM_COLS);
     }
 }
 
@@ -886,13 +854,13 @@ inline int launch_ok(const char *what, char *msg, size_t msg_len) {
     return KDA_ERR_CUDA;
 }
 
-// The five launches for bf16 inputs, dk = dv = 128 (per-channel decay).
+// The three launches for bf16 inputs, dk = dv = 128 (per-channel decay).
 inline int launch_backward_tc(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                               const float *init_state, const void *d_o, const float *dfinal, void *dq, void *dk_out,
                               void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state,
                               const int32_t *cu_seqlens, long long tokens, int T, int H, int num_seqs,
                               void *workspace, cudaStream_t st, char *msg, size_t msg_len) {
-    constexpr int DK = 128, DV = 128, DVT = 32, NBUF = 2;
+    constexpr int DK = 128, DV = 128, DVT = 64, NBUF = 2;   // one wave of sweeps at 32 heads
     const long long slots = tokens > 0 ? chunk_slots(tokens, num_seqs) : 0;
     if (slots > 0x7fffffffLL) {
         snprintf(msg, msg_len, "%lld chunk slots exceed the grid limit", slots);
@@ -900,11 +868,11 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
     }
     uint8_t *ws = (uint8_t *)workspace;
     const auto *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k;
-    CUtensorMap t_v32, t_do32, t_do64, t_v128;
-    memset(&t_do32, 0, sizeof(t_do32));   // no tokens: the adjoint sweep only copies dfinal, never loading
-    if (slots > 0 && (!make_tmap(&t_v32, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, DVT) ||
-        !make_tmap(&t_do32, d_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, DVT,
-                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+    static_assert(DVT == 64, "the sweeps' dO tile is the 128-byte-swizzled 64-column box");
+    CUtensorMap t_v64, t_do64, t_v128;
+    memset(&t_v64, 0, sizeof(t_v64));   // no tokens: the sweeps load nothing (the adjoint one copies dfinal)
+    memset(&t_do64, 0, sizeof(t_do64));
+    if (slots > 0 && (!make_tmap(&t_v64, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, DVT) ||
         !make_tmap(&t_do64, d_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap(&t_v128, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 128))) {
@@ -913,32 +881,26 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
     }
     int rc;
     auto k1 = chunk_intra_kernel<DK, false, false, true>;
-    auto k2 = chunk_inter_kernel<DK, DVT, NBUF, true>;
-    auto k3 = chunk_adj_kernel<DK, DVT, NBUF>;
+    auto k2 = bwd_sweeps_kernel<DK, DVT, NBUF>;
     auto k4 = bwd_grad_kernel;
-    auto k5 = bwd_chain_kernel;
-    constexpr int s1 = IntraLayout<DK>::ALLOC, s2 = InterLayout<DK, DVT, NBUF>::ALLOC;
-    constexpr int s3 = AdjLayout<DK, DVT, NBUF>::ALLOC, s4 = GradLayout::ALLOC, s5 = ChainLayout::ALLOC;
-    if ((rc = set_smem_tc(k1, s1, "chunk_intra", msg, msg_len)) || (rc = set_smem_tc(k2, s2, "chunk_inter", msg, msg_len)) ||
-        (rc = set_smem_tc(k3, s3, "chunk_adj", msg, msg_len)) || (rc = set_smem_tc(k4, s4, "bwd_grad", msg, msg_len)) ||
-        (rc = set_smem_tc(k5, s5, "bwd_chain", msg, msg_len)))
+    constexpr int s1 = IntraLayout<DK>::ALLOC, s2 = sweeps_smem<DK, DVT, NBUF>(), s4 = GradLayout::ALLOC;
+    if ((rc = set_smem_tc(k1, s1, "chunk_intra", msg, msg_len)) || (rc = set_smem_tc(k2, s2, "bwd_sweeps", msg, msg_len)) ||
+        (rc = set_smem_tc(k4, s4, "bwd_grad", msg, msg_len)))
         return rc;
-    const dim3 per_chunk((unsigned)slots, H), per_chain(DV / DVT, H, num_seqs);
+    const dim3 per_chunk((unsigned)slots, H);
     if (slots > 0) {
         k1<<<per_chunk, NT, s1, st>>>(qb, kb, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws);
         if ((rc = launch_ok("chunk_intra", msg, msg_len))) return rc;
-        k2<<<per_chain, NT, s2, st>>>(t_v32, ws, init_state, nullptr, nullptr, cu_seqlens, T, H, DV, nullptr, 0, ws);
-        if ((rc = launch_ok("chunk_inter", msg, msg_len))) return rc;
     }
-    k3<<<per_chain, NT, s3, st>>>(t_do32, ws, dfinal, dinit_state, cu_seqlens, T, H, DV);
-    if ((rc = launch_ok("chunk_adj", msg, msg_len))) return rc;
+    // both sweeps; with no tokens only the adjoint half has work (dinit_state = dfinal)
+    k2<<<dim3(2 * (DV / DVT), H, num_seqs), NT, s2, st>>>(t_v64, t_do64, ws, init_state, dfinal, dinit_state,
+                                                          cu_seqlens, T, H, DV);
+    if ((rc = launch_ok("bwd_sweeps", msg, msg_len))) return rc;
     if (slots > 0) {
-        k4<<<per_chunk, NT, s4, st>>>(t_do64, t_v128, kb, log_alpha, beta, (__nv_bfloat16 *)dv_out, dbeta, cu_seqlens,
-                                      T, H, num_seqs, ws);
+        k4<<<per_chunk, NT, s4, st>>>(t_do64, t_v128, qb, kb, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws,
+                                      (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk_out, (__nv_bfloat16 *)dv_out,
+                                      dlog_alpha, dbeta);
         if ((rc = launch_ok("bwd_grad", msg, msg_len))) return rc;
-        k5<<<per_chunk, NT, s5, st>>>(qb, kb, log_alpha, cu_seqlens, T, H, num_seqs, ws, (__nv_bfloat16 *)dq,
-                                      (__nv_bfloat16 *)dk_out, dlog_alpha);
-        if ((rc = launch_ok("bwd_chain", msg, msg_len))) return rc;
     }
     return KDA_OK;
 }

@@ -50,8 +50,7 @@ struct BwdX {
 // Backward workspace unit of one (chunk slot, head), dk = dv = 128 (kda_bwd_tc.cuh):
 // the record and the extras from the first pass, the state at the chunk's start
 // (forward sweep) and its adjoint at the chunk's end (adjoint sweep), both bf16
-// [DV/64][DK][128 B] with a 128-byte swizzle.  The per-chunk gradient kernel then
-// writes its sums over the first bytes of the same unit (fields XQ..DGC).
+// [DV/64][DK][128 B] with a 128-byte swizzle.
 template <int DK>
 struct BwdUnit {
     static constexpr int DV = 128;
@@ -60,15 +59,7 @@ struct BwdUnit {
     static constexpr int SC = BXO + BwdX::BYTES;
     static constexpr int DSC = SC + DK * DV * 2;
     static constexpr int BYTES = DSC + DK * DV * 2;
-    static constexpr int XQ = 0;                       // fp32 [DK][64]  S dO^T                (dQhat^T)
-    static constexpr int XK = XQ + DK * C * 4;         // fp32 [DK][64]  -S mu^T               (dKhat^T)
-    static constexpr int XB = XK + DK * C * 4;         // fp32 [DK][64]  dS U^T                (dKbar^T)
-    static constexpr int DA = XB + DK * C * 4;         // bf16 [128][128 B]: dAkk rows 0-63, dAqk rows 64-127
-    static constexpr int DGC = DA + 128 * 128;         // fp32 [DK]      e^{G_last} sum_v S dS
-    static constexpr int GRAD_END = DGC + DK * 4;
-    static_assert(GRAD_END <= BYTES, "the sums fit over the unit");
-    static_assert(BXO % 1024 == 0 && SC % 1024 == 0 && DSC % 1024 == 0 && BYTES % 1024 == 0 && DA % 1024 == 0,
-                  "tile alignment");
+    static_assert(BXO % 1024 == 0 && SC % 1024 == 0 && DSC % 1024 == 0 && BYTES % 1024 == 0, "tile alignment");
 };
 
 inline long long chunk_slots(long long tokens, int num_seqs) { return (tokens + C - 1) / C + num_seqs; }
@@ -675,11 +666,11 @@ constexpr uint32_t XCOL_DS = 128;     // [128 x DVT] Kt Z (lanes 0..dk-1)
 // hold [slot][H] BwdUnit; no output; instead the state at each chunk's start, bf16,
 // into the unit's SC tile (a K-major operand S with K = value columns, MN-major for S^T).
 template <int DK, int DVT, int NBUF, bool CK = false>
-__global__ void __launch_bounds__(NT, 1)
-chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__restrict__ ws,
-                   const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
-                   float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV,
-                   const int32_t *__restrict__ slots, int num_slots, uint8_t *__restrict__ ckpt) {
+__device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, const uint8_t *__restrict__ ws,
+                                           const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
+                                           float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens,
+                                           int T, int H, int DV, const int32_t *__restrict__ slots, int num_slots,
+                                           uint8_t *__restrict__ ckpt) {
     using L = InterLayout<DK, DVT, NBUF>;
     using R = Rec<DK>;
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
@@ -695,7 +686,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
-    const int col_base = blockIdx.x * DVT, h = blockIdx.y;
+    const int col_base = tile * DVT, h = blockIdx.y;
     const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
 
     long long t0, t1;
@@ -711,7 +702,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
         for (int b = 0; b < NBUF; ++b) ptx::mbar_init(bar_rec + 8 * b, 1);
         ptx::mbar_init(bar_mma, 1);
         ptx::fence_mbar_init();
-        ptx::prefetch_tmap(&tm_v);
+        if (nck > 0) ptx::prefetch_tmap(tm_v);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -727,7 +718,7 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
         const uint32_t bar = bar_rec + 8 * b;
         ptx::mbar_arrive_expect_tx(bar, TX);
         ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * USTRIDE, (uint32_t)R::BYTES, bar);
-        ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, &tm_v, bar, col_base, h, (int)(t0 + (long long)ci * C));
+        ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, tm_v, bar, col_base, h, (int)(t0 + (long long)ci * C));
     };
 
     const int srow = quad * 32 + lane;
@@ -882,6 +873,16 @@ chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__re
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, INTER_TMEM_COLS);
     }
+}
+
+template <int DK, int DVT, int NBUF, bool CK = false>
+__global__ void __launch_bounds__(NT, 1)
+chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__restrict__ ws,
+                   const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
+                   float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV,
+                   const int32_t *__restrict__ slots, int num_slots, uint8_t *__restrict__ ckpt) {
+    inter_body<DK, DVT, NBUF, CK>((int)blockIdx.x, &tm_v, ws, init_state, o, final_state, cu_seqlens, T, H, DV, slots,
+                                  num_slots, ckpt);
 }
 
 // ------------------------------------------------------------------ host side
