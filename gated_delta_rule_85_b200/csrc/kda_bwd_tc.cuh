@@ -357,11 +357,11 @@ struct GradLayout {   // dk = dv = 128; bf16 tiles with a 128-byte swizzle unles
     static constexpr int EX = 16384;            // BwdX             Akk | Aqk | T
     static constexpr int SS = 40960;            // [2][128][128 B]  S at the chunk's start
     static constexpr int DS = 73728;            // [2][128][128 B]  dS' at its end
-    static constexpr int DOL = 106496;          // [2][128][128 B]  dO rows 0-63 (TMA), lam rows 64-127
-    static constexpr int KBR = 139264;          // [2][64][128 B]   Kbar rows (K-major B, N = tokens)
+    static constexpr int DOL = 106496;          // [2][128][128 B]  dO rows 0-63 (TMA); rows 64-127 unused
+    static constexpr int KBR = 139264;          // [2][64][128 B]   Kbar rows (K-major B, N = tokens), then lam^T
     static constexpr int VV = 155648;           // [64][128]        V, no swizzle
     static constexpr int AW = 172032;           // [128][128 B]     (Diag(beta) W)^T, then U^T
-    static constexpr int ADU = 188416;          // [128][128 B]     dU^T, then -mu rows [2][64][128 B]
+    static constexpr int ADU = 188416;          // [128][128 B]     dU^T, then -mu^T
     // the chain rule, over tiles that phase 3 has finished with
     static constexpr int DA = KH;               // [128][128 B]     dAkk rows 0-63, dAqk rows 64-127
     static constexpr int KE = SS;               // [2 parts][2][64][128 B]  e^{-G} K: bf16 high part, low part
@@ -386,12 +386,12 @@ struct GradLayout {   // dk = dv = 128; bf16 tiles with a 128-byte swizzle unles
     static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
-constexpr uint32_t GRAD_TMEM_COLS = 256;
+constexpr uint32_t GRAD_TMEM_COLS = 512;
 // TMEM columns, 64 each.  Phase 1: S^T Khat^T, dU^T.  Phase 2: U^T, lam^T.  Phase 3:
-// [dAqk; L], S dO^T, -S mu^T, dS' U^T.  Phase 4 (tier A) adds the row terms onto
-// S dO^T and -S mu^T (the same factor e^G scales both) and puts the column terms
-// over [dAqk; L], which has been read out.
-constexpr uint32_t GC_0 = 0, GC_1 = 64, GC_2 = 128, GC_3 = 192;
+// dAqk, S dO^T, -S mu^T, dS' U^T, L = lam U^T (dAqk and L in lanes 0-63).  Phase 4
+// (tier A) adds the row terms onto S dO^T and -S mu^T (the same factor e^G scales
+// both) and puts the column terms over dAqk, which has been read out.
+constexpr uint32_t GC_0 = 0, GC_1 = 64, GC_2 = 128, GC_3 = 192, GC_4 = 256;
 
 // bf16 element (r, j) of a one-atom (64-column) tile with a 128-byte swizzle.
 __device__ __forceinline__ float ld_sw128(const uint8_t *tile, int r, int j) {
@@ -619,35 +619,47 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
             p[u] = lam[u] * (vj - x[u]);
         }
         fDB[quad * 64 + 32 * half + lane] = warp_transpose_sum32(p);
-        // mu = beta lam: dV; lam rows under dO in DOL; -mu rows in ADU (K-major B, N = tokens)
+        // mu = beta lam: dV; lam^T and -mu^T (rows = value channels) for phase 3
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
             const int j = 32 * half + u;
             const float mu = fB[j] * lam[u];
             if (j < Lc) dv_out[((cs + j) * H + h) * DV + vr] = __float2bfloat16_rn(mu);
-            st_bf16(sm, L::DOL + sw128(64 + j, vr, 128), lam[u]);
-            st_bf16(sm, L::ADU + sw128(j, vr, 64), -mu);
+            p[u] = -mu;
+        }
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+            st_bf16x8(sm, L::KBR + sw128_chunk(vr, 4 * half + gq), lam + 8 * gq);
+            st_bf16x8(sm, L::ADU + sw128_chunk(vr, 4 * half + gq), p + 8 * gq);
         }
     }
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
 
-    // ---- phase 3: [dAqk; L] = [dO; lam] U^T ; S dO^T ; S (-mu)^T ; dS' U^T
+    // ---- phase 3: dAqk = dO U^T ; S dO^T ; S (-mu)^T ; dS' U^T ; L = lam U^T
+    // (dAqk and L: M = 128 over 64-row operands, whose second halves read neighbouring
+    // bytes; those rows are ignored)
     if (ok && tid == 0) {
         ptx::tc_fence_after();
         constexpr uint32_t i_kk = ptx::idesc_bf16_f32(128, 64);
         constexpr uint32_t i_km = ptx::idesc_bf16_f32(128, 64, false, true);
+        constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
 #pragma unroll
         for (int s = 0; s < 8; ++s)
             ptx::mma_bf16(tmem + GC_0, kdesc(sb + L::DOL, s, 128),
                           ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_km, s > 0);
 #pragma unroll
         for (int s = 0; s < 8; ++s)
+            ptx::mma_bf16(tmem + GC_4, ptx::desc_mnmajor_sw128(sb + L::KBR + s * 2048, 8192, 1024),
+                          ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_mm, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
             ptx::mma_bf16(tmem + GC_1, kdesc(sb + L::SS, s, 128), kdesc(sb + L::DOL, s, 128), i_kk, s > 0);
 #pragma unroll
         for (int s = 0; s < 8; ++s)
-            ptx::mma_bf16(tmem + GC_2, kdesc(sb + L::SS, s, 128), kdesc(sb + L::ADU, s, 64), i_kk, s > 0);
+            ptx::mma_bf16(tmem + GC_2, kdesc(sb + L::SS, s, 128),
+                          ptx::desc_mnmajor_sw128(sb + L::ADU + s * 2048, 8192, 1024), i_km, s > 0);
 #pragma unroll
         for (int s = 0; s < 8; ++s)
             ptx::mma_bf16(tmem + GC_3, kdesc(sb + L::DS, s, 128),
@@ -669,18 +681,19 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
     }
     if (ok) ok = wait_all(bar_mma, ph_mma);   // phase 1-3 tiles are free from here on
     if (ok) {
-        // dA -> the bf16 tile (masked): rows 0-63 of TMEM hold dAqk, rows 64-127 L = lam U^T
-        float x[32];
-        ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
-        ptx::tmem_wait_ld();
-        if (quad < 2) {   // dAqk (j <= i) -> rows 64-127 of DA
+        // dA -> the bf16 tile (masked), TMEM lanes 0-63: dAqk (j <= i) -> rows 64-127;
+        // L = lam U^T -> dAkk = -beta_i L (j < i) -> rows 0-63, and sum_j Akk L for dbeta
+        if (quad < 2) {
             const int i = vr;
+            float x[32];
+            ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
+            ptx::tmem_wait_ld();
 #pragma unroll
             for (int u = 0; u < 32; ++u) x[u] = (32 * half + u <= i) ? x[u] : 0.f;
 #pragma unroll
             for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::DA + sw128_chunk(64 + i, 4 * half + gq), x + 8 * gq);
-        } else {          // dAkk = -beta_i L (j < i) -> rows 0-63 of DA; and sum_j Akk L for dbeta
-            const int i = vr - 64;
+            ptx::tmem_ld32(tl + GC_4 + 32 * half, x);
+            ptx::tmem_wait_ld();
             const float bi = fB[i];
             float dot = 0.f, a8[8];
 #pragma unroll
