@@ -369,6 +369,11 @@ struct GradLayout {   // dk = dv = 128; bf16 tiles with a 128-byte swizzle unles
     static constexpr int FG = KBR;              // fp32 [64][128]   G
     static constexpr int QR = AW;               // bf16 [64][128]   q, no swizzle
     static constexpr int KR = ADU;              // bf16 [64][128]   k, no swizzle
+    // output rows staged for 16-byte stores
+    static constexpr int OV = KH;               // bf16 [64][128]   dv (readout 2, stored during phase 3)
+    static constexpr int OQ = 0;                // bf16 [64][128]   dq  } over DA and EX, after phase 4
+    static constexpr int OK = 16384;            // bf16 [64][128]   dk  }
+    static constexpr int OG = FG;               // fp32 [64][128]   dlog_alpha, over G after the readout
     // fp32 scratch
     static constexpr int FB = 204800;           // [64]        beta
     static constexpr int FD = FB + 256;         // [128]       e^{G_last}
@@ -624,7 +629,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
         for (int u = 0; u < 32; ++u) {
             const int j = 32 * half + u;
             const float mu = fB[j] * lam[u];
-            if (j < Lc) dv_out[((cs + j) * H + h) * DV + vr] = __float2bfloat16_rn(mu);
+            reinterpret_cast<__nv_bfloat16 *>(sm + L::OV)[j * DV + vr] = __float2bfloat16_rn(mu);
             p[u] = -mu;
         }
 #pragma unroll
@@ -667,7 +672,12 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
         ptx::mma_commit(bar_mma);
         ++n_commit;
     }
-    if (ok) {   // meanwhile: sum_v S dS' for this lane's key channel over the half's 64 value columns
+    if (ok) {   // meanwhile: the dv rows, and sum_v S dS' for this lane's key channel over the half's 64 value columns
+        for (int idx = tid; idx < Lc * (DV / 8); idx += NT) {
+            const int j = idx / (DV / 8), g = idx % (DV / 8);
+            *reinterpret_cast<uint4 *>(dv_out + ((cs + j) * H + h) * DV + 8 * g) =
+                *reinterpret_cast<const uint4 *>(sm + L::OV + (j * DV + 8 * g) * 2);
+        }
         float acc = 0.f;
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
@@ -773,6 +783,9 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
         chain_pairs_exact(sm + L::DA, fG, reinterpret_cast<const __nv_bfloat16 *>(sm + L::QR),
                           reinterpret_cast<const __nv_bfloat16 *>(sm + L::KR), c, 32 * half,
                           reinterpret_cast<float *>(sm + L::KE));
+    if (strong) __syncthreads();   // every thread is done with DA before dq and dk go over it
+    __nv_bfloat16 *oq = reinterpret_cast<__nv_bfloat16 *>(sm + L::OQ);
+    __nv_bfloat16 *okk = reinterpret_cast<__nv_bfloat16 *>(sm + L::OK);
     const __nv_bfloat16 *sq = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QR);
     const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KR);
     float dG[32], kb = 0.f, sdg = 0.f;
@@ -807,29 +820,40 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
                 dG[16 * cc + u] = g;
                 sdg += g;
                 kb = fmaf(ki, b, kb);
-                if (i < Lc) {
-                    const long long o = ((cs + i) * H + h) * DK + c;
-                    dq[o] = __float2bfloat16_rn(dqi);
-                    dk_out[o] = __float2bfloat16_rn(dki);
-                }
+                oq[i * DK + c] = __float2bfloat16_rn(dqi);
+                okk[i * DK + c] = __float2bfloat16_rn(dki);
             }
         }
         fX[half * DK + c] = kb;
         fX[2 * DK + half * DK + c] = sdg;
     }
     __syncthreads();
+    float *og = reinterpret_cast<float *>(sm + L::OG);   // over G, which nobody reads any more
     if (ok) {
         float run = fD[c] * (fGC[c] + fGC[128 + c]) + fX[c] + fX[DK + c];
         if (half == 0) run += fX[2 * DK + DK + c];   // all of the later half's dG
 #pragma unroll
         for (int u = 31; u >= 0; --u) {
-            const int i = 32 * half + u;
             run += dG[u];
-            if (i < Lc) dlog_alpha[((cs + i) * H + h) * DK + c] = run;
+            og[(32 * half + u) * DK + c] = run;
         }
         if (tid < C && tid < Lc) {
             const float db = fDB[tid] + fDB[64 + tid] + fDB[128 + tid] + fDB[192 + tid] - fDB2[tid] - fDB2[64 + tid];
             dbeta[(cs + tid) * H + h] = db;
+        }
+    }
+    __syncthreads();
+    if (ok) {   // dq, dk, dlog_alpha rows as 16-byte stores
+        for (int idx = tid; idx < Lc * (DK / 8); idx += NT) {
+            const int i = idx / (DK / 8), g = idx % (DK / 8);
+            const long long o = ((cs + i) * H + h) * DK + 8 * g;
+            *reinterpret_cast<uint4 *>(dq + o) = *reinterpret_cast<const uint4 *>(oq + i * DK + 8 * g);
+            *reinterpret_cast<uint4 *>(dk_out + o) = *reinterpret_cast<const uint4 *>(okk + i * DK + 8 * g);
+        }
+        for (int idx = tid; idx < Lc * (DK / 4); idx += NT) {
+            const int i = idx / (DK / 4), g = idx % (DK / 4);
+            *reinterpret_cast<float4 *>(dlog_alpha + ((cs + i) * H + h) * DK + 4 * g) =
+                *reinterpret_cast<const float4 *>(og + i * DK + 4 * g);
         }
     }
     if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded)
