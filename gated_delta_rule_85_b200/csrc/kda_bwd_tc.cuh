@@ -140,8 +140,9 @@ __device__ __forceinline__ void adj_body(int tile, const CUtensorMap *tm_do, uin
             uint8_t *ck = ws + ((size_t)(first + ci) * H + h) * U::BYTES + U::DSC;
 #pragma unroll
             for (int g = 0; g < CPT / 8; ++g) {
-                const uint4 w = make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
-                                           pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
+                const uint4 w =
+                    make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
+                               pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
                 *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) = w;
                 *reinterpret_cast<uint4 *>(ck + sw128(srow, col_base + scol + 8 * g, DK)) = w;
             }
@@ -446,7 +447,8 @@ __device__ __noinline__ void chain_pairs_exact(const uint8_t *da, const float *f
     }
 }
 
-// One CTA per (chunk slot, head), 256 threads.  Warps w and w + 4 share TMEM lane
+// Persistent: each CTA (256 threads, one per SM) takes (chunk slot, head) items in
+// turn, prefetching the next one's inputs into L2.  Warps w and w + 4 share TMEM lane
 // quadrant w & 3 (value channel or key channel 32 (w & 3) + lane) and split the 64
 // token columns in halves.
 //   Phases 1-3: every product that needs S or dS' -> dV, dbeta, dAqk/dAkk and
@@ -467,9 +469,11 @@ __device__ __noinline__ void chain_pairs_exact(const uint8_t *da, const float *f
 //     dlog_alpha_t = e^{G_last} sum_v S dS' + sum_i k_i b_i + sum_{i>=t} dG_i.
 __global__ void __launch_bounds__(NT, 1)
 bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_v,
-                const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, const uint8_t *__restrict__ ws,
+                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16 *__restrict__ q,
+                const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
+                const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
+                int nslots, const uint8_t *__restrict__ ws,
                 __nv_bfloat16 *__restrict__ dq, __nv_bfloat16 *__restrict__ dk_out, __nv_bfloat16 *__restrict__ dv_out,
                 float *__restrict__ dlog_alpha, float *__restrict__ dbeta) {
     using L = GradLayout;
@@ -486,12 +490,6 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
     float *fDB2 = reinterpret_cast<float *>(sm + L::FDB2), *fGC = reinterpret_cast<float *>(sm + L::FGC);
     float *fX = reinterpret_cast<float *>(sm + L::FX), *fG = reinterpret_cast<float *>(sm + L::FG);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3, half = warp >> 2;
-    const int slot = blockIdx.x, h = blockIdx.y;
-    long long cs;
-    int Lc;
-    if (!slot_chunk(cu_seqlens, T, num_seqs, slot, cs, Lc)) return;
-    const uint8_t *unit = ws + ((size_t)slot * H + h) * U::BYTES;
-
     if (warp == 0) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), GRAD_TMEM_COLS);
         ptx::tmem_relinquish();
@@ -500,364 +498,407 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
         ptx::mbar_init(bar_ld, 1);
         ptx::mbar_init(bar_mma, 1);
         ptx::fence_mbar_init();
-        ptx::mbar_arrive_expect_tx(bar_ld, 16384u + (uint32_t)BwdX::BYTES + 2u * 32768u + 16384u + 16384u);
-        ptx::bulk_load(sb + L::KH, unit + R::KQ, 8192u, bar_ld);                 // Khat rows of atom 0
-        ptx::bulk_load(sb + L::KH + 8192, unit + R::KQ + 16384, 8192u, bar_ld);  // and of atom 1
-        ptx::bulk_load(sb + L::EX, unit + U::BXO, (uint32_t)BwdX::BYTES, bar_ld);
-        ptx::bulk_load(sb + L::SS, unit + U::SC, 32768u, bar_ld);
-        ptx::bulk_load(sb + L::DS, unit + U::DSC, 32768u, bar_ld);
-        ptx::tma_load_3d(sb + L::DOL, &tm_do, bar_ld, 0, h, (int)cs);
-        ptx::tma_load_3d(sb + L::DOL + 16384, &tm_do, bar_ld, 64, h, (int)cs);
-        ptx::tma_load_3d(sb + L::VV, &tm_v, bar_ld, 0, h, (int)cs);
-    }
-    if (tid < C) fB[tid] = tid < Lc ? beta[(cs + tid) * H + h] : 0.f;
-    // G, k and q of this thread's 8 tokens x 4 channels, kept for phase 4
-    float G[8][4], tot[4];
-    uint2 kv[8], qv[8];
-    chunk_decay<true>(q, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
-    const int c0 = 4 * (tid & 31), i0 = 8 * (tid >> 5);
-    {   // Kbar = e^{G_last - G} K (factors <= 1) and e^{G_last}, while the copies fly
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const float4 k4 = bf16x4_to_float4(kv[u]);
-            st_bf16x4(sm, L::KBR + sw128(i0 + u, c0, 64), k4.x * __expf(tot[0] - G[u][0]),
-                      k4.y * __expf(tot[1] - G[u][1]), k4.z * __expf(tot[2] - G[u][2]), k4.w * __expf(tot[3] - G[u][3]));
-        }
-        if (tid < 32) *reinterpret_cast<float4 *>(fD + c0) = make_float4(__expf(tot[0]), __expf(tot[1]),
-                                                                         __expf(tot[2]), __expf(tot[3]));
     }
     ptx::tc_fence_before();
-    const bool strong = __syncthreads_or(tot[0] < -DECAY_LIM || tot[1] < -DECAY_LIM || tot[2] < -DECAY_LIM ||
-                                         tot[3] < -DECAY_LIM) != 0;   // uniform: tier B
+    __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     uint32_t ph_ld = 0, ph_mma = 0;
-    int n_commit = 0;
-    bool ok = wait_all(bar_ld, ph_ld);
-    if (ok && Lc < C) {   // rows past the chunk's end: zero dO and V (the copies read the next tokens)
-        for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
-            const int i = Lc + idx / 16, g = idx % 16;
-            *reinterpret_cast<uint4 *>(sm + L::DOL + (g >> 3) * 16384 + i * 128 + (g & 7) * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(sm + L::VV + i * 256 + g * 16) = make_uint4(0, 0, 0, 0);
-        }
-    }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-
-    // ---- phase 1: S^T Khat^T (-> W^T = V^T - that) ; dU^T = dO^T Aqk + dS'^T Kbar^T
-    if (ok && tid == 0) {
-        ptx::tc_fence_after();
-        constexpr uint32_t i_mk = ptx::idesc_bf16_f32(128, 64, true, false);
-        constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-            ptx::mma_bf16(tmem + GC_0, ptx::desc_mnmajor_sw128(sb + L::SS + s * 2048, 16384, 1024),
-                          kdesc(sb + L::KH, s, 64), i_mk, s > 0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-            ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(sb + L::DOL + s * 2048, 16384, 1024),
-                          ptx::desc_mnmajor_sw128(sb + L::EX + BwdX::AQK + s * 2048, 8192, 1024), i_mm, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-            ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(sb + L::DS + s * 2048, 16384, 1024),
-                          kdesc(sb + L::KBR, s, 64), i_mk, 1);
-        ptx::mma_commit(bar_mma);
-        ++n_commit;
-    }
-    if (ok) ok = wait_all(bar_mma, ph_mma);
-    const int vr = quad * 32 + lane;   // this lane's TMEM row: value channel (phases 1-2) or key channel
-    if (ok) {   // W^T (scaled by beta_i) and dU^T -> bf16 K-major A operands, rows = value channels
-        float x[32], y[32];
-        ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
-        ptx::tmem_ld32(tl + GC_1 + 32 * half, y);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            const int i = 32 * half + u;
-            const float vi = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + L::VV + (i * DV + vr) * 2));
-            x[u] = fB[i] * (vi - x[u]);
-        }
-#pragma unroll
-        for (int gq = 0; gq < 4; ++gq) {
-            st_bf16x8(sm, L::AW + sw128_chunk(vr, 4 * half + gq), x + 8 * gq);
-            st_bf16x8(sm, L::ADU + sw128_chunk(vr, 4 * half + gq), y + 8 * gq);
-        }
-    }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-
-    // ---- phase 2: U^T = (beta W)^T T^T ; lam^T = dU^T T
-    if (ok && tid == 0) {
-        ptx::tc_fence_after();
-        constexpr uint32_t i_kk = ptx::idesc_bf16_f32(128, 64);
-        constexpr uint32_t i_km = ptx::idesc_bf16_f32(128, 64, false, true);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-            ptx::mma_bf16(tmem + GC_2, kdesc(sb + L::AW, s, 128), kdesc(sb + L::EX + BwdX::TI, s, 64), i_kk, s > 0);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-            ptx::mma_bf16(tmem + GC_3, kdesc(sb + L::ADU, s, 128),
-                          ptx::desc_mnmajor_sw128(sb + L::EX + BwdX::TI + s * 2048, 8192, 1024), i_km, s > 0);
-        ptx::mma_commit(bar_mma);
-        ++n_commit;
-    }
-    if (ok) ok = wait_all(bar_mma, ph_mma);
-    if (ok) {
-        float x[32];
-        // U^T -> bf16 (rows = value channels): the MN-major B of [dO; lam] U^T and dS' U^T
-        ptx::tmem_ld32(tl + GC_2 + 32 * half, x);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::AW + sw128_chunk(vr, 4 * half + gq), x + 8 * gq);
-        // <lam_j, W_j> summed over this warp's 32 value channels
-        float lam[32], p[32];
-        ptx::tmem_ld32(tl + GC_3 + 32 * half, lam);
-        ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            const int j = 32 * half + u;
-            const float vj = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + L::VV + (j * DV + vr) * 2));
-            p[u] = lam[u] * (vj - x[u]);
-        }
-        fDB[quad * 64 + 32 * half + lane] = warp_transpose_sum32(p);
-        // mu = beta lam: dV; lam^T and -mu^T (rows = value channels) for phase 3
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            const int j = 32 * half + u;
-            const float mu = fB[j] * lam[u];
-            reinterpret_cast<__nv_bfloat16 *>(sm + L::OV)[j * DV + vr] = __float2bfloat16_rn(mu);
-            p[u] = -mu;
-        }
-#pragma unroll
-        for (int gq = 0; gq < 4; ++gq) {
-            st_bf16x8(sm, L::KBR + sw128_chunk(vr, 4 * half + gq), lam + 8 * gq);
-            st_bf16x8(sm, L::ADU + sw128_chunk(vr, 4 * half + gq), p + 8 * gq);
-        }
-    }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-
-    // ---- phase 3: dAqk = dO U^T ; S dO^T ; S (-mu)^T ; dS' U^T ; L = lam U^T
-    // (dAqk and L: M = 128 over 64-row operands, whose second halves read neighbouring
-    // bytes; those rows are ignored)
-    if (ok && tid == 0) {
-        ptx::tc_fence_after();
-        constexpr uint32_t i_kk = ptx::idesc_bf16_f32(128, 64);
-        constexpr uint32_t i_km = ptx::idesc_bf16_f32(128, 64, false, true);
-        constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-            ptx::mma_bf16(tmem + GC_0, kdesc(sb + L::DOL, s, 128),
-                          ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_km, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-            ptx::mma_bf16(tmem + GC_4, ptx::desc_mnmajor_sw128(sb + L::KBR + s * 2048, 8192, 1024),
-                          ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_mm, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-            ptx::mma_bf16(tmem + GC_1, kdesc(sb + L::SS, s, 128), kdesc(sb + L::DOL, s, 128), i_kk, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-            ptx::mma_bf16(tmem + GC_2, kdesc(sb + L::SS, s, 128),
-                          ptx::desc_mnmajor_sw128(sb + L::ADU + s * 2048, 8192, 1024), i_km, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-            ptx::mma_bf16(tmem + GC_3, kdesc(sb + L::DS, s, 128),
-                          ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_km, s > 0);
-        ptx::mma_commit(bar_mma);
-        ++n_commit;
-    }
-    if (ok) {   // meanwhile: the dv rows, and sum_v S dS' for this lane's key channel over the half's 64 value columns
-        for (int idx = tid; idx < Lc * (DV / 8); idx += NT) {
-            const int j = idx / (DV / 8), g = idx % (DV / 8);
-            *reinterpret_cast<uint4 *>(dv_out + ((cs + j) * H + h) * DV + 8 * g) =
-                *reinterpret_cast<const uint4 *>(sm + L::OV + (j * DV + 8 * g) * 2);
-        }
-        float acc = 0.f;
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            float a8[8], b8[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::SS + half * 16384 + sw128_chunk(vr, g)), a8);
-            unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::DS + half * 16384 + sw128_chunk(vr, g)), b8);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) acc = fmaf(a8[u], b8[u], acc);
-        }
-        fGC[half * 128 + vr] = acc;
-    }
-    if (ok) ok = wait_all(bar_mma, ph_mma);   // phase 1-3 tiles are free from here on
-    if (ok) {
-        // dA -> the bf16 tile (masked), TMEM lanes 0-63: dAqk (j <= i) -> rows 64-127;
-        // L = lam U^T -> dAkk = -beta_i L (j < i) -> rows 0-63, and sum_j Akk L for dbeta
-        if (quad < 2) {
-            const int i = vr;
-            float x[32];
-            ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int u = 0; u < 32; ++u) x[u] = (32 * half + u <= i) ? x[u] : 0.f;
-#pragma unroll
-            for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::DA + sw128_chunk(64 + i, 4 * half + gq), x + 8 * gq);
-            ptx::tmem_ld32(tl + GC_4 + 32 * half, x);
-            ptx::tmem_wait_ld();
-            const float bi = fB[i];
-            float dot = 0.f, a8[8];
-#pragma unroll
-            for (int gq = 0; gq < 4; ++gq) {
-                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::EX + BwdX::AKK + sw128_chunk(i, 4 * half + gq)),
-                              a8);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) dot = fmaf(a8[u], x[8 * gq + u], dot);
-            }
-            fDB2[half * 64 + i] = dot;
-#pragma unroll
-            for (int u = 0; u < 32; ++u) x[u] = (32 * half + u < i) ? -bi * x[u] : 0.f;
-#pragma unroll
-            for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::DA + sw128_chunk(i, 4 * half + gq), x + 8 * gq);
-        }
-        // G, raw q and k (row-major), and in tier A the split decay-scaled operands
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u;
-            *reinterpret_cast<float4 *>(fG + i * DK + c0) = make_float4(G[u][0], G[u][1], G[u][2], G[u][3]);
-            *reinterpret_cast<uint2 *>(sm + L::QR + (i * DK + c0) * 2) = qv[u];
-            *reinterpret_cast<uint2 *>(sm + L::KR + (i * DK + c0) * 2) = kv[u];
-            if (!strong) {
-                const float4 k4 = bf16x4_to_float4(kv[u]), q4 = bf16x4_to_float4(qv[u]);
-                const float kq[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
-                float xe[4], xk[4], xq[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float en = __expf(-G[u][e]), er = __expf(G[u][e] - tot[e]);   // <= e^DECAY_LIM
-                    xe[e] = kq[e] * en;
-                    xk[e] = kq[e] * er;
-                    xq[e] = qq[e] * er;
-                }
-                st_split_bf16x4(sm, L::KE + sw128(i, c0, 64), L::KE + 16384 + sw128(i, c0, 64), xe);
-                st_split_bf16x4(sm, L::KQE + sw128(i, c0, 128), L::KQE + 32768 + sw128(i, c0, 128), xk);
-                st_split_bf16x4(sm, L::KQE + sw128(64 + i, c0, 128), L::KQE + 32768 + sw128(64 + i, c0, 128), xq);
-            }
-        }
-    }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-
-    // ---- phase 4 (tier A): row terms onto S dO^T and -S mu^T; column terms over dA
-    if (ok && !strong) {
+    int n_commit = 0, n_ld = 0;
+    bool ok = true;
+    const int n_items = nslots * H;
+    // thread 0: an item's inputs into L2 (nothing waits on it; the item's own copies find them there)
+    auto prefetch = [&](int it) {
+        const int ps = it % nslots, hp = it / nslots;
+        long long pcs;
+        int pLc;
+        if (!slot_chunk(cu_seqlens, T, num_seqs, ps, pcs, pLc)) return;
+        const uint8_t *pu = ws + ((size_t)ps * H + hp) * U::BYTES;
+        ptx::bulk_prefetch_l2(pu + R::KQ, 8192u);
+        ptx::bulk_prefetch_l2(pu + R::KQ + 16384, 8192u);
+        ptx::bulk_prefetch_l2(pu + U::BXO, (uint32_t)(U::BYTES - U::BXO));
+        ptx::tma_prefetch_l2_3d(&tm_do, 0, hp, (int)pcs);
+        ptx::tma_prefetch_l2_3d(&tm_do, 64, hp, (int)pcs);
+        ptx::tma_prefetch_l2_3d(&tm_v, 0, hp, (int)pcs);
+        ptx::tma_prefetch_l2_3d(&tm_q, 0, hp, (int)pcs);
+        ptx::tma_prefetch_l2_3d(&tm_k, 0, hp, (int)pcs);
+        ptx::tma_prefetch_l2_3d(&tm_g, 0, hp, (int)pcs);
+    };
+    // persistent: items (slot, head), slot fastest, strided by the grid
+    for (int it = (int)blockIdx.x; ok && it < n_items; it += (int)gridDim.x) {
+        const int slot = it % nslots, h = it / nslots;
+        long long cs;
+        int Lc;
+        if (!slot_chunk(cu_seqlens, T, num_seqs, slot, cs, Lc)) continue;   // uniform: a slot without a chunk
+        const uint8_t *unit = ws + ((size_t)slot * H + h) * U::BYTES;
         if (tid == 0) {
+            ptx::mbar_arrive_expect_tx(bar_ld, 16384u + (uint32_t)BwdX::BYTES + 2u * 32768u + 16384u + 16384u);
+            ptx::bulk_load(sb + L::KH, unit + R::KQ, 8192u, bar_ld);                 // Khat rows of atom 0
+            ptx::bulk_load(sb + L::KH + 8192, unit + R::KQ + 16384, 8192u, bar_ld);  // and of atom 1
+            ptx::bulk_load(sb + L::EX, unit + U::BXO, (uint32_t)BwdX::BYTES, bar_ld);
+            ptx::bulk_load(sb + L::SS, unit + U::SC, 32768u, bar_ld);
+            ptx::bulk_load(sb + L::DS, unit + U::DSC, 32768u, bar_ld);
+            ptx::tma_load_3d(sb + L::DOL, &tm_do, bar_ld, 0, h, (int)cs);
+            ptx::tma_load_3d(sb + L::DOL + 16384, &tm_do, bar_ld, 64, h, (int)cs);
+            ptx::tma_load_3d(sb + L::VV, &tm_v, bar_ld, 0, h, (int)cs);
+            ++n_ld;
+            if (it + (int)gridDim.x < n_items) prefetch(it + (int)gridDim.x);
+        }
+        if (tid < C) fB[tid] = tid < Lc ? beta[(cs + tid) * H + h] : 0.f;
+        // G, k and q of this thread's 8 tokens x 4 channels, kept for phase 4
+        float G[8][4], tot[4];
+        uint2 kv[8], qv[8];
+        chunk_decay<true>(q, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
+        const int c0 = 4 * (tid & 31), i0 = 8 * (tid >> 5);
+        {   // Kbar = e^{G_last - G} K (factors <= 1) and e^{G_last}, while the copies fly
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float4 k4 = bf16x4_to_float4(kv[u]);
+                st_bf16x4(sm, L::KBR + sw128(i0 + u, c0, 64), k4.x * __expf(tot[0] - G[u][0]),
+                          k4.y * __expf(tot[1] - G[u][1]), k4.z * __expf(tot[2] - G[u][2]),
+                          k4.w * __expf(tot[3] - G[u][3]));
+            }
+            if (tid < 32) *reinterpret_cast<float4 *>(fD + c0) = make_float4(__expf(tot[0]), __expf(tot[1]),
+                                                                             __expf(tot[2]), __expf(tot[3]));
+        }
+        ptx::tc_fence_before();
+        const bool strong = __syncthreads_or(tot[0] < -DECAY_LIM || tot[1] < -DECAY_LIM || tot[2] < -DECAY_LIM ||
+                                             tot[3] < -DECAY_LIM) != 0;   // uniform: tier B
+        ptx::tc_fence_after();
+        ok = wait_all(bar_ld, ph_ld);
+        if (ok && Lc < C) {   // rows past the chunk's end: zero dO and V (the copies read the next tokens)
+            for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
+                const int i = Lc + idx / 16, g = idx % 16;
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(sm + L::DOL + (g >> 3) * 16384 + i * 128 + (g & 7) * 16) = z;
+                *reinterpret_cast<uint4 *>(sm + L::VV + i * 256 + g * 16) = z;
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- phase 1: S^T Khat^T (-> W^T = V^T - that) ; dU^T = dO^T Aqk + dS'^T Kbar^T
+        if (ok && tid == 0) {
             ptx::tc_fence_after();
             constexpr uint32_t i_mk = ptx::idesc_bf16_f32(128, 64, true, false);
             constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t ke = sb + L::KE + part * 16384, kqe = sb + L::KQE + part * 32768;
+            for (int s = 0; s < 8; ++s)
+                ptx::mma_bf16(tmem + GC_0, ptx::desc_mnmajor_sw128(sb + L::SS + s * 2048, 16384, 1024),
+                              kdesc(sb + L::KH, s, 64), i_mk, s > 0);
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(ke + s * 2048, 8192, 1024),
-                                  kdesc(sb + L::DA + 8192, s, 64), i_mk, 1);
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(sb + L::DOL + s * 2048, 16384, 1024),
+                              ptx::desc_mnmajor_sw128(sb + L::EX + BwdX::AQK + s * 2048, 8192, 1024), i_mm, s > 0);
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    ptx::mma_bf16(tmem + GC_2, ptx::desc_mnmajor_sw128(ke + s * 2048, 8192, 1024),
-                                  kdesc(sb + L::DA, s, 64), i_mk, 1);
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    ptx::mma_bf16(tmem + GC_0, ptx::desc_mnmajor_sw128(kqe + s * 2048, 16384, 1024),
-                                  ptx::desc_mnmajor_sw128(sb + L::DA + s * 2048, 8192, 1024), i_mm, part > 0 || s > 0);
-            }
+            for (int s = 0; s < 8; ++s)
+                ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(sb + L::DS + s * 2048, 16384, 1024),
+                              kdesc(sb + L::KBR, s, 64), i_mk, 1);
             ptx::mma_commit(bar_mma);
             ++n_commit;
         }
-        ok = wait_all(bar_mma, ph_mma);
-    }
-
-    // ---- readout: thread (key channel c, token half)
-    const int c = vr;
-    const float gl = fG[(C - 1) * DK + c];   // G_last (rows past Lc add nothing)
-    const float *fP = reinterpret_cast<const float *>(sm + L::KE);   // tier B: exact RQ, RK, CT
-    if (ok && strong)
-        chain_pairs_exact(sm + L::DA, fG, reinterpret_cast<const __nv_bfloat16 *>(sm + L::QR),
-                          reinterpret_cast<const __nv_bfloat16 *>(sm + L::KR), c, 32 * half,
-                          reinterpret_cast<float *>(sm + L::KE));
-    if (strong) __syncthreads();   // every thread is done with DA before dq and dk go over it
-    __nv_bfloat16 *oq = reinterpret_cast<__nv_bfloat16 *>(sm + L::OQ);
-    __nv_bfloat16 *okk = reinterpret_cast<__nv_bfloat16 *>(sm + L::OK);
-    const __nv_bfloat16 *sq = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QR);
-    const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KR);
-    float dG[32], kb = 0.f, sdg = 0.f;
-    if (ok) {
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            float t1[16], t2[16], t3[16], t0[16];
-            const uint32_t col = 32 * half + 16 * cc;
-            ptx::tmem_ld16(tl + GC_1 + col, t1);
-            ptx::tmem_ld16(tl + GC_2 + col, t2);
-            ptx::tmem_ld16(tl + GC_3 + col, t3);
-            if (!strong) ptx::tmem_ld16(tl + GC_0 + col, t0);
+        if (ok) ok = wait_all(bar_mma, ph_mma);
+        const int vr = quad * 32 + lane;   // this lane's TMEM row: value channel (phases 1-2) or key channel
+        if (ok) {   // W^T (scaled by beta_i) and dU^T -> bf16 K-major A operands, rows = value channels
+            float x[32], y[32];
+            ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
+            ptx::tmem_ld32(tl + GC_1 + 32 * half, y);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int i = col + u;
-                const float Gi = fG[i * DK + c];
-                const float qi = __bfloat162float(sq[i * DK + c]), ki = __bfloat162float(sk[i * DK + c]);
-                const float eg = __expf(Gi), eb = __expf(gl - Gi);
-                float RQ = 0.f, RK = 0.f, CT;
-                if (!strong) {
-                    CT = eb * t0[u];
-                } else {
-                    RQ = fP[i * DK + c];
-                    RK = fP[C * DK + i * DK + c];
-                    CT = fP[2 * C * DK + i * DK + c];
-                }
-                const float dqi = fmaf(eg, t1[u], RQ);
-                const float a = fmaf(eg, t2[u], RK), b = eb * t3[u];
-                const float dki = a + b + CT;
-                const float g = qi * dqi + ki * (a - b - CT);
-                dG[16 * cc + u] = g;
-                sdg += g;
-                kb = fmaf(ki, b, kb);
-                oq[i * DK + c] = __float2bfloat16_rn(dqi);
-                okk[i * DK + c] = __float2bfloat16_rn(dki);
+            for (int u = 0; u < 32; ++u) {
+                const int i = 32 * half + u;
+                const float vi = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sm + L::VV)[i * DV + vr]);
+                x[u] = fB[i] * (vi - x[u]);
+            }
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                st_bf16x8(sm, L::AW + sw128_chunk(vr, 4 * half + gq), x + 8 * gq);
+                st_bf16x8(sm, L::ADU + sw128_chunk(vr, 4 * half + gq), y + 8 * gq);
             }
         }
-        fX[half * DK + c] = kb;
-        fX[2 * DK + half * DK + c] = sdg;
-    }
-    __syncthreads();
-    float *og = reinterpret_cast<float *>(sm + L::OG);   // over G, which nobody reads any more
-    if (ok) {
-        float run = fD[c] * (fGC[c] + fGC[128 + c]) + fX[c] + fX[DK + c];
-        if (half == 0) run += fX[2 * DK + DK + c];   // all of the later half's dG
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- phase 2: U^T = (beta W)^T T^T ; lam^T = dU^T T
+        if (ok && tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t i_kk = ptx::idesc_bf16_f32(128, 64);
+            constexpr uint32_t i_km = ptx::idesc_bf16_f32(128, 64, false, true);
 #pragma unroll
-        for (int u = 31; u >= 0; --u) {
-            run += dG[u];
-            og[(32 * half + u) * DK + c] = run;
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + GC_2, kdesc(sb + L::AW, s, 128), kdesc(sb + L::EX + BwdX::TI, s, 64), i_kk, s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                ptx::mma_bf16(tmem + GC_3, kdesc(sb + L::ADU, s, 128),
+                              ptx::desc_mnmajor_sw128(sb + L::EX + BwdX::TI + s * 2048, 8192, 1024), i_km, s > 0);
+            ptx::mma_commit(bar_mma);
+            ++n_commit;
         }
-        if (tid < C && tid < Lc) {
-            const float db = fDB[tid] + fDB[64 + tid] + fDB[128 + tid] + fDB[192 + tid] - fDB2[tid] - fDB2[64 + tid];
-            dbeta[(cs + tid) * H + h] = db;
+        if (ok) ok = wait_all(bar_mma, ph_mma);
+        if (ok) {
+            float x[32];
+            // U^T -> bf16 (rows = value channels): the MN-major B of [dO; lam] U^T and dS' U^T
+            ptx::tmem_ld32(tl + GC_2 + 32 * half, x);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::AW + sw128_chunk(vr, 4 * half + gq), x + 8 * gq);
+            // <lam_j, W_j> summed over this warp's 32 value channels
+            float lam[32], p[32];
+            ptx::tmem_ld32(tl + GC_3 + 32 * half, lam);
+            ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const int j = 32 * half + u;
+                const float vj = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sm + L::VV)[j * DV + vr]);
+                p[u] = lam[u] * (vj - x[u]);
+            }
+            fDB[quad * 64 + 32 * half + lane] = warp_transpose_sum32(p);
+            // mu = beta lam: dV; lam^T and -mu^T (rows = value channels) for phase 3
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const int j = 32 * half + u;
+                const float mu = fB[j] * lam[u];
+                reinterpret_cast<__nv_bfloat16 *>(sm + L::OV)[j * DV + vr] = __float2bfloat16_rn(mu);
+                p[u] = -mu;
+            }
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                st_bf16x8(sm, L::KBR + sw128_chunk(vr, 4 * half + gq), lam + 8 * gq);
+                st_bf16x8(sm, L::ADU + sw128_chunk(vr, 4 * half + gq), p + 8 * gq);
+            }
         }
-    }
-    __syncthreads();
-    if (ok) {   // dq, dk, dlog_alpha rows as 16-byte stores
-        for (int idx = tid; idx < Lc * (DK / 8); idx += NT) {
-            const int i = idx / (DK / 8), g = idx % (DK / 8);
-            const long long o = ((cs + i) * H + h) * DK + 8 * g;
-            *reinterpret_cast<uint4 *>(dq + o) = *reinterpret_cast<const uint4 *>(oq + i * DK + 8 * g);
-            *reinterpret_cast<uint4 *>(dk_out + o) = *reinterpret_cast<const uint4 *>(okk + i * DK + 8 * g);
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- phase 3: dAqk = dO U^T ; S dO^T ; S (-mu)^T ; dS' U^T ; L = lam U^T
+        // (dAqk and L: M = 128 over 64-row operands, whose second halves read neighbouring
+        // bytes; those rows are ignored)
+        if (ok && tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t i_kk = ptx::idesc_bf16_f32(128, 64);
+            constexpr uint32_t i_km = ptx::idesc_bf16_f32(128, 64, false, true);
+            constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                ptx::mma_bf16(tmem + GC_0, kdesc(sb + L::DOL, s, 128),
+                              ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_km, s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                ptx::mma_bf16(tmem + GC_4, ptx::desc_mnmajor_sw128(sb + L::KBR + s * 2048, 8192, 1024),
+                              ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_mm, s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                ptx::mma_bf16(tmem + GC_1, kdesc(sb + L::SS, s, 128), kdesc(sb + L::DOL, s, 128), i_kk, s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                ptx::mma_bf16(tmem + GC_2, kdesc(sb + L::SS, s, 128),
+                              ptx::desc_mnmajor_sw128(sb + L::ADU + s * 2048, 8192, 1024), i_km, s > 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                ptx::mma_bf16(tmem + GC_3, kdesc(sb + L::DS, s, 128),
+                              ptx::desc_mnmajor_sw128(sb + L::AW + s * 2048, 8192, 1024), i_km, s > 0);
+            ptx::mma_commit(bar_mma);
+            ++n_commit;
         }
-        for (int idx = tid; idx < Lc * (DK / 4); idx += NT) {
-            const int i = idx / (DK / 4), g = idx % (DK / 4);
-            *reinterpret_cast<float4 *>(dlog_alpha + ((cs + i) * H + h) * DK + 4 * g) =
-                *reinterpret_cast<const float4 *>(og + i * DK + 4 * g);
+        if (ok) {   // meanwhile: the dv rows, and sum_v S dS' (this lane's key channel, the half's 64 columns)
+            for (int idx = tid; idx < Lc * (DV / 8); idx += NT) {
+                const int j = idx / (DV / 8), g = idx % (DV / 8);
+                *reinterpret_cast<uint4 *>(dv_out + ((cs + j) * H + h) * DV + 8 * g) =
+                    *reinterpret_cast<const uint4 *>(sm + L::OV + (j * DV + 8 * g) * 2);
+            }
+            float acc = 0.f;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                float a8[8], b8[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::SS + half * 16384 + sw128_chunk(vr, g)), a8);
+                unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + L::DS + half * 16384 + sw128_chunk(vr, g)), b8);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc = fmaf(a8[u], b8[u], acc);
+            }
+            fGC[half * 128 + vr] = acc;
         }
+        if (ok) ok = wait_all(bar_mma, ph_mma);   // phase 1-3 tiles are free from here on
+        if (ok) {
+            // dA -> the bf16 tile (masked), TMEM lanes 0-63: dAqk (j <= i) -> rows 64-127;
+            // L = lam U^T -> dAkk = -beta_i L (j < i) -> rows 0-63, and sum_j Akk L for dbeta
+            if (quad < 2) {
+                const int i = vr;
+                float x[32];
+                ptx::tmem_ld32(tl + GC_0 + 32 * half, x);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 32; ++u) x[u] = (32 * half + u <= i) ? x[u] : 0.f;
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::DA + sw128_chunk(64 + i, 4 * half + gq), x + 8 * gq);
+                ptx::tmem_ld32(tl + GC_4 + 32 * half, x);
+                ptx::tmem_wait_ld();
+                const float bi = fB[i];
+                float dot = 0.f, a8[8];
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    const uint32_t ao = L::EX + BwdX::AKK + sw128_chunk(i, 4 * half + gq);
+                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(sm + ao), a8);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) dot = fmaf(a8[u], x[8 * gq + u], dot);
+                }
+                fDB2[half * 64 + i] = dot;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) x[u] = (32 * half + u < i) ? -bi * x[u] : 0.f;
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) st_bf16x8(sm, L::DA + sw128_chunk(i, 4 * half + gq), x + 8 * gq);
+            }
+            // G, raw q and k (row-major), and in tier A the split decay-scaled operands
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u;
+                *reinterpret_cast<float4 *>(fG + i * DK + c0) = make_float4(G[u][0], G[u][1], G[u][2], G[u][3]);
+                *reinterpret_cast<uint2 *>(sm + L::QR + (i * DK + c0) * 2) = qv[u];
+                *reinterpret_cast<uint2 *>(sm + L::KR + (i * DK + c0) * 2) = kv[u];
+                if (!strong) {
+                    const float4 k4 = bf16x4_to_float4(kv[u]), q4 = bf16x4_to_float4(qv[u]);
+                    const float kq[4] = {k4.x, k4.y, k4.z, k4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
+                    float xe[4], xk[4], xq[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float en = __expf(-G[u][e]), er = __expf(G[u][e] - tot[e]);   // <= e^DECAY_LIM
+                        xe[e] = kq[e] * en;
+                        xk[e] = kq[e] * er;
+                        xq[e] = qq[e] * er;
+                    }
+                    st_split_bf16x4(sm, L::KE + sw128(i, c0, 64), L::KE + 16384 + sw128(i, c0, 64), xe);
+                    st_split_bf16x4(sm, L::KQE + sw128(i, c0, 128), L::KQE + 32768 + sw128(i, c0, 128), xk);
+                    st_split_bf16x4(sm, L::KQE + sw128(64 + i, c0, 128), L::KQE + 32768 + sw128(64 + i, c0, 128), xq);
+                }
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+
+        // ---- phase 4 (tier A): row terms onto S dO^T and -S mu^T; column terms over dA
+        if (ok && !strong) {
+            if (tid == 0) {
+                ptx::tc_fence_after();
+                constexpr uint32_t i_mk = ptx::idesc_bf16_f32(128, 64, true, false);
+                constexpr uint32_t i_mm = ptx::idesc_bf16_f32(128, 64, true, true);
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t ke = sb + L::KE + part * 16384, kqe = sb + L::KQE + part * 32768;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        ptx::mma_bf16(tmem + GC_1, ptx::desc_mnmajor_sw128(ke + s * 2048, 8192, 1024),
+                                      kdesc(sb + L::DA + 8192, s, 64), i_mk, 1);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        ptx::mma_bf16(tmem + GC_2, ptx::desc_mnmajor_sw128(ke + s * 2048, 8192, 1024),
+                                      kdesc(sb + L::DA, s, 64), i_mk, 1);
+#pragma unroll
+                    for (int s = 0; s < 8; ++s)
+                        ptx::mma_bf16(tmem + GC_0, ptx::desc_mnmajor_sw128(kqe + s * 2048, 16384, 1024),
+                                      ptx::desc_mnmajor_sw128(sb + L::DA + s * 2048, 8192, 1024), i_mm,
+                                      part > 0 || s > 0);
+                }
+                ptx::mma_commit(bar_mma);
+                ++n_commit;
+            }
+            ok = wait_all(bar_mma, ph_mma);
+        }
+
+        // ---- readout: thread (key channel c, token half)
+        const int c = vr;
+        const float gl = fG[(C - 1) * DK + c];   // G_last (rows past Lc add nothing)
+        const float *fP = reinterpret_cast<const float *>(sm + L::KE);   // tier B: exact RQ, RK, CT
+        if (ok && strong)
+            chain_pairs_exact(sm + L::DA, fG, reinterpret_cast<const __nv_bfloat16 *>(sm + L::QR),
+                              reinterpret_cast<const __nv_bfloat16 *>(sm + L::KR), c, 32 * half,
+                              reinterpret_cast<float *>(sm + L::KE));
+        if (strong) __syncthreads();   // every thread is done with DA before dq and dk go over it
+        __nv_bfloat16 *oq = reinterpret_cast<__nv_bfloat16 *>(sm + L::OQ);
+        __nv_bfloat16 *okk = reinterpret_cast<__nv_bfloat16 *>(sm + L::OK);
+        const __nv_bfloat16 *sq = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QR);
+        const __nv_bfloat16 *sk = reinterpret_cast<const __nv_bfloat16 *>(sm + L::KR);
+        float dG[32], kb = 0.f, sdg = 0.f;
+        if (ok) {
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                float t1[16], t2[16], t3[16], t0[16];
+                const uint32_t col = 32 * half + 16 * cc;
+                ptx::tmem_ld16(tl + GC_1 + col, t1);
+                ptx::tmem_ld16(tl + GC_2 + col, t2);
+                ptx::tmem_ld16(tl + GC_3 + col, t3);
+                if (!strong) ptx::tmem_ld16(tl + GC_0 + col, t0);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int i = col + u;
+                    const float Gi = fG[i * DK + c];
+                    const float qi = __bfloat162float(sq[i * DK + c]), ki = __bfloat162float(sk[i * DK + c]);
+                    const float eg = __expf(Gi), eb = __expf(gl - Gi);
+                    float RQ = 0.f, RK = 0.f, CT;
+                    if (!strong) {
+                        CT = eb * t0[u];
+                    } else {
+                        RQ = fP[i * DK + c];
+                        RK = fP[C * DK + i * DK + c];
+                        CT = fP[2 * C * DK + i * DK + c];
+                    }
+                    const float dqi = fmaf(eg, t1[u], RQ);
+                    const float a = fmaf(eg, t2[u], RK), b = eb * t3[u];
+                    const float dki = a + b + CT;
+                    const float g = qi * dqi + ki * (a - b - CT);
+                    dG[16 * cc + u] = g;
+                    sdg += g;
+                    kb = fmaf(ki, b, kb);
+                    oq[i * DK + c] = __float2bfloat16_rn(dqi);
+                    okk[i * DK + c] = __float2bfloat16_rn(dki);
+                }
+            }
+            fX[half * DK + c] = kb;
+            fX[2 * DK + half * DK + c] = sdg;
+        }
+        __syncthreads();
+        float *og = reinterpret_cast<float *>(sm + L::OG);   // over G, which nobody reads any more
+        if (ok) {
+            float run = fD[c] * (fGC[c] + fGC[128 + c]) + fX[c] + fX[DK + c];
+            if (half == 0) run += fX[2 * DK + DK + c];   // all of the later half's dG
+#pragma unroll
+            for (int u = 31; u >= 0; --u) {
+                run += dG[u];
+                og[(32 * half + u) * DK + c] = run;
+            }
+            if (tid < C && tid < Lc) {
+                const float db =
+                    fDB[tid] + fDB[64 + tid] + fDB[128 + tid] + fDB[192 + tid] - fDB2[tid] - fDB2[64 + tid];
+                dbeta[(cs + tid) * H + h] = db;
+            }
+        }
+        __syncthreads();
+        if (ok) {   // dq, dk, dlog_alpha rows as 16-byte stores
+            for (int idx = tid; idx < Lc * (DK / 8); idx += NT) {
+                const int i = idx / (DK / 8), g = idx % (DK / 8);
+                const long long o = ((cs + i) * H + h) * DK + 8 * g;
+                *reinterpret_cast<uint4 *>(dq + o) = *reinterpret_cast<const uint4 *>(oq + i * DK + 8 * g);
+                *reinterpret_cast<uint4 *>(dk_out + o) = *reinterpret_cast<const uint4 *>(okk + i * DK + 8 * g);
+            }
+            for (int idx = tid; idx < Lc * (DK / 4); idx += NT) {
+                const int i = idx / (DK / 4), g = idx % (DK / 4);
+                *reinterpret_cast<float4 *>(dlog_alpha + ((cs + i) * H + h) * DK + 4 * g) =
+                    *reinterpret_cast<const float4 *>(og + i * DK + 4 * g);
+            }
+        }
+        // this item's shared-memory reads complete before the next item's copies land
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
     }
     if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded)
-        ptx::mbar_wait_bounded(bar_ld, 0u, WAIT_LIMIT_CYCLES);
+        if (n_ld > 0) ptx::mbar_wait_bounded(bar_ld, (uint32_t)((n_ld - 1) & 1), WAIT_LIMIT_CYCLES);
         if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
     }
     ptx::tc_fence_before();
@@ -906,13 +947,16 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
     uint8_t *ws = (uint8_t *)workspace;
     const auto *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k;
     static_assert(DVT == 64, "the sweeps' dO tile is the 128-byte-swizzled 64-column box");
-    CUtensorMap t_v64, t_do64, t_v128;
+    CUtensorMap t_v64, t_do64, t_v128, t_q, t_k, t_g;
     memset(&t_v64, 0, sizeof(t_v64));   // no tokens: the sweeps load nothing (the adjoint one copies dfinal)
     memset(&t_do64, 0, sizeof(t_do64));
     if (slots > 0 && (!make_tmap(&t_v64, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, DVT) ||
         !make_tmap(&t_do64, d_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap(&t_v128, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 128))) {
+        !make_tmap(&t_v128, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 128) ||
+        !make_tmap(&t_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DK, DK) ||
+        !make_tmap(&t_k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DK, DK) ||
+        !make_tmap(&t_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, DK, DK))) {
         snprintf(msg, msg_len, "building TMA descriptors failed (driver entry point cuTensorMapEncodeTiled)");
         return KDA_ERR_CUDA;
     }
@@ -921,8 +965,8 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
     auto k2 = bwd_sweeps_kernel<DK, DVT, NBUF>;
     auto k4 = bwd_grad_kernel;
     constexpr int s1 = IntraLayout<DK>::ALLOC, s2 = sweeps_smem<DK, DVT, NBUF>(), s4 = GradLayout::ALLOC;
-    if ((rc = set_smem_tc(k1, s1, "chunk_intra", msg, msg_len)) || (rc = set_smem_tc(k2, s2, "bwd_sweeps", msg, msg_len)) ||
-        (rc = set_smem_tc(k4, s4, "bwd_grad", msg, msg_len)))
+    if ((rc = set_smem_tc(k1, s1, "chunk_intra", msg, msg_len)) ||
+        (rc = set_smem_tc(k2, s2, "bwd_sweeps", msg, msg_len)) || (rc = set_smem_tc(k4, s4, "bwd_grad", msg, msg_len)))
         return rc;
     const dim3 per_chunk((unsigned)slots, H);
     if (slots > 0) {
@@ -934,9 +978,15 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
                                                           cu_seqlens, T, H, DV);
     if ((rc = launch_ok("bwd_sweeps", msg, msg_len))) return rc;
     if (slots > 0) {
-        k4<<<per_chunk, NT, s4, st>>>(t_do64, t_v128, qb, kb, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws,
-                                      (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk_out, (__nv_bfloat16 *)dv_out,
-                                      dlog_alpha, dbeta);
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                      cudaSuccess)
+            sms = 148;
+        const long long items = slots * H;
+        const unsigned grid = (unsigned)(items < sms ? items : sms);
+        k4<<<grid, NT, s4, st>>>(t_do64, t_v128, t_q, t_k, t_g, qb, kb, log_alpha, beta, cu_seqlens, T, H, num_seqs,
+                                 (int)slots, ws, (__nv_bfloat16 *)dq, (__nv_bfloat16 *)dk_out, (__nv_bfloat16 *)dv_out,
+                                 dlog_alpha, dbeta);
         if ((rc = launch_ok("bwd_grad", msg, msg_len))) return rc;
     }
     return KDA_OK;
