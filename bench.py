@@ -51,18 +51,20 @@ DECODE_BYTES_PER_PAIR = 2 * STATE_BYTES + PREFILL_BYTES_PER_TOKEN_HEAD        # 
 # product is two products of the same size (recomputation is not credited).
 BACKWARD_BYTES_PER_TOKEN_HEAD = 4 * 2 * 128 + 4 * 128 + 4 + 3 * 2 * 128 + 4 * 128 + 4   # 2824
 BACKWARD_FLOPS_PER_TOKEN_HEAD = 2 * PREFILL_FLOPS_PER_TOKEN_HEAD                      # 360448
+# The tensor-core backward of bf16 inputs with dk = dv = 128: three launches per call.
+BACKWARD_KERNELS = "chunk_intra_kernel (with the backward extras) + bwd_sweeps_kernel + bwd_grad_kernel"
+BACKWARD_LAUNCHES = 3
 # Fused prologue, per token-head: raw q, k, v and the gate pre-activation (bf16), beta, o.
 PROLOGUE_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 2 * 128 + 4 + 2 * 128                    # 1284
 # DRAM bytes (read + write) per launch, taken from ncu captures (dram__bytes_read.sum +
 # dram__bytes_write.sum) of the current kernels on these workloads; keyed by the kernels
 # one step runs.  A kernel set without a capture on its workload reports null.
 NCU_TRAFFIC = {
-    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.8e6 + 181.3e6 + 308.3e6 + 50.5e6,
+    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.9e6 + 181.3e6 + 308.3e6 + 51.3e6,
     # chunk_tc_kernel (--algo fused): captured before its timeout-path change, so reported null
     ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.2e6,
-    # backward: all four kernels of one call; T=2048 captured, T=8192 scaled by the chunk slots (129 / 33)
-    ("backward_T2048", "bwd"): 795.0e6 + 428.8e6,
-    ("backward_T8192", "bwd"): (795.0e6 + 428.8e6) * 129 / 33,
+    # backward: the three kernels of one call (read + write of each)
+    ("backward_T8192", "bwd"): 270.0e6 + 282.4e6 + 492.3e6 + 233.7e6 + 915.8e6 + 311.0e6,
 }
 
 
@@ -333,7 +335,7 @@ def run_backward(args, world, rank, dev):
     shape = PrefillShape(**cfg, dtype=torch.bfloat16)
     d = prefill_inputs(shape, seed=rank, device=dev)
     c = backward_cotangents(shape, seed=rank, device=dev)
-    ws = torch.empty(kda.backward_workspace_size(1, cfg["T"], cfg["H"], 128, 128, 1), dtype=torch.uint8,
+    ws = torch.empty(kda.backward_workspace_size(1, cfg["T"], cfg["H"], 128, 128, 1, torch.bfloat16), dtype=torch.uint8,
                      device=dev)
     out = {}
 
@@ -356,7 +358,7 @@ def run_backward(args, world, rank, dev):
     torch.cuda.synchronize(dev)
     ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
     del d, c, ws, out
-    return dict(ms=ms, launches=reps * 4)
+    return dict(ms=ms, launches=reps * BACKWARD_LAUNCHES)
 
 
 def run_prefill_varlen(args, world, rank, dev):
@@ -613,7 +615,7 @@ def backward_block(args, world, bw, hbm_gbs, bf16_tflops):
     return {
         "metric": f"KDA chunked backward tokens/s (gradients of the prefill: B=1, T={T}, H={H}, d=128)",
         "value": world * T / (bw["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": bw["ms"],
-        "roofline": {"kernel": "bwd_prep_kernel + bwd_state_kernel + bwd_part_kernel + bwd_chunk_kernel",
+        "roofline": {"kernel": BACKWARD_KERNELS,
                      "bound": "hbm", "achieved": bgbs, "peak": hbm_gbs, "unit": "GB/s", "frac": bgbs / hbm_gbs,
                      "traffic": NCU_TRAFFIC.get((f"backward_T{T}", "bwd")), "algorithmic_bytes": bbytes,
                      "tensor": {"achieved_tflops": btf, "peak_tflops": bf16_tflops, "frac": btf / bf16_tflops,

@@ -675,7 +675,10 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
     using R = Rec<DK>;
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
     constexpr int CPT = DVT / 2;
-    constexpr uint32_t TX = (uint32_t)(R::BYTES + C * DVT * 2);
+    // CK loads only what the state update reads: the Khat rows of [Khat; Qhat], the Kt rows of
+    // [Kt; Pt] and e^{G_last} (the Qhat rows then hold stale bytes, whose products are never read)
+    constexpr uint32_t REC_TX = CK ? (uint32_t)(DK / 64 * 64 * 128 + DK * 128 + DK * 4) : (uint32_t)R::BYTES;
+    constexpr uint32_t TX = REC_TX + (uint32_t)(C * DVT * 2);
     constexpr size_t USTRIDE = CK ? (size_t)BwdUnit<DK>::BYTES : (size_t)R::BYTES;   // bytes per (slot, head)
     using MN = MnOp<DVT>;
     extern __shared__ uint8_t smem_raw[];
@@ -717,7 +720,16 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
         n_issued = ci + 1;
         const uint32_t bar = bar_rec + 8 * b;
         ptx::mbar_arrive_expect_tx(bar, TX);
-        ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * USTRIDE, (uint32_t)R::BYTES, bar);
+        const uint8_t *src = ws + ((size_t)(first + ci) * H + h) * USTRIDE;
+        if constexpr (CK) {
+#pragma unroll
+            for (int a = 0; a < DK / 64; ++a)
+                ptx::bulk_load(sb + b * R::BYTES + R::KQ + a * 16384, src + R::KQ + a * 16384, 64 * 128, bar);
+            ptx::bulk_load(sb + b * R::BYTES + R::KP, src + R::KP, DK * 128, bar);
+            ptx::bulk_load(sb + b * R::BYTES + R::DCH, src + R::DCH, DK * 4, bar);
+        } else {
+            ptx::bulk_load(sb + b * R::BYTES, src, (uint32_t)R::BYTES, bar);
+        }
         ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, tm_v, bar, col_base, h, (int)(t0 + (long long)ci * C));
     };
 
