@@ -15,7 +15,8 @@ import torch
 
 import gated_delta_rule_85_b200 as kda
 import oracle
-from gated_delta_rule_85_b200.workloads import PrefillShape, backward_cotangents, prefill_inputs, to_f64
+from gated_delta_rule_85_b200.workloads import (PrefillShape, STRONG_KINDS, backward_cotangents, prefill_inputs,
+                                                strong_decay, to_f64)
 from kda_testutil import max_abs, rel_l2
 
 pytestmark = pytest.mark.gpu
@@ -142,6 +143,30 @@ def test_backward_without_states():
     torch.cuda.synchronize()
     check(got, oracle_grads(d, c), torch.float32, what="no states")
     assert got["dinit_state"].abs().max().item() > 0
+
+
+@pytest.mark.parametrize("kind", STRONG_KINDS)
+@pytest.mark.parametrize("algo", ["simt", "tensor"])
+@pytest.mark.parametrize("packed", [False, True])
+def test_backward_strong_decay_kinds(kind, algo, packed):
+    """The forward's strong-decay patterns -- single-token hard resets (-100), whole
+    chunks at -2, strong and weak channels mixed in one head -- through both bf16
+    schedules; the tensor-core one takes its exact tier for these chunks, dense and
+    packed (empty and one-token sequences included)."""
+    if packed:
+        lens = [70, 0, 129, 1, 256]
+        cu = tuple(np.cumsum([0] + lens).tolist())
+        shape = PrefillShape(B=1, T=cu[-1], H=2, dk=128, dv=128, dtype=BF16, cu_seqlens=cu)
+    else:
+        shape = PrefillShape(B=2, T=300, H=2, dk=128, dv=128, dtype=BF16)
+    d = prefill_inputs(shape, 600 + len(kind), DEV)
+    strong_decay(d["log_alpha"], kind, 21)
+    c = backward_cotangents(shape, 601, DEV)
+    kda.device_status(clear=True)
+    got = run(d, c, algo=algo)
+    torch.cuda.synchronize()
+    assert kda.device_status(clear=True) == 0
+    check(got, oracle_grads(d, c), BF16, what=f"{kind} {algo}")
 
 
 @pytest.mark.parametrize("dv", [64, 128])
