@@ -102,6 +102,8 @@ def load_library():
     lib.kda_chunk_backward_workspace_size_ex.restype = sz
     lib.kda_chunk_backward_ex.argtypes = lib.kda_chunk_backward.argtypes + [ci]
     lib.kda_chunk_backward_ex.restype = ci
+    lib.kda_gdn_chunk_backward_ex.argtypes = lib.kda_chunk_backward_ex.argtypes
+    lib.kda_gdn_chunk_backward_ex.restype = ci
     lib.kda_last_error.argtypes = []
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ci, vp]
@@ -296,13 +298,13 @@ def backward_workspace_size(B, T, H, dk, dv, num_seqs, dtype=None, algo="auto") 
 
 
 def gdn_chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=None, cu_seqlens=None, *,
-                       dinit_state=True, workspace=None, out=None):
-    """Gradients through the Gated DeltaNet prefill (kda_gdn_chunk_backward):
+                       dinit_state=True, workspace=None, out=None, algo="auto"):
+    """Gradients through the Gated DeltaNet prefill (kda_gdn_chunk_backward_ex):
     log_alpha and the returned dlog_alpha are [B, T, H]; otherwise as chunk_backward."""
     if log_alpha.shape != q.shape[:3]:
         raise ValueError("log_alpha must be [B, T, H] (one rate per token-head)")
     return chunk_backward(q, k, v, log_alpha, beta, d_o, init_state, dfinal_state, cu_seqlens,
-                          dinit_state=dinit_state, workspace=workspace, out=out, _gate_scalar=True)
+                          dinit_state=dinit_state, workspace=workspace, out=out, algo=algo, _gate_scalar=True)
 
 
 def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=None, cu_seqlens=None, *,
@@ -315,7 +317,7 @@ def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=
     shape and dtype, dfinal_state is float32 [N, H, dk, dv] or None (zero).
     The workspace (uint8, CUDA) and the outputs (`out`, a dict with any of the
     keys above) are allocated here unless given.  algo: "auto", "tensor" or
-    "simt" (kda_chunk_backward_ex; the Gated DeltaNet backward takes "auto").
+    "simt" (kda_chunk_backward_ex).
     Device tensors only.
     """
     gate = SimpleNamespace(shape=q.shape, dtype=log_alpha.dtype) if _gate_scalar else log_alpha
@@ -338,22 +340,17 @@ def chunk_backward(q, k, v, log_alpha, beta, d_o, init_state=None, dfinal_state=
     else:
         g["dinit_state"] = None
     _need_cuda(*g.values())
-    if algo not in BACKWARD_ALGOS or (_gate_scalar and algo != "auto"):
+    if algo not in BACKWARD_ALGOS:
         raise ValueError(f"unknown backward algo {algo!r}")
-    if _gate_scalar:
-        need = int(lib.kda_chunk_backward_workspace_size(B, T, H, dk, dv, N))
-    else:
-        need = int(lib.kda_chunk_backward_workspace_size_ex(B, T, H, dk, dv, N, _dtype_code(q), BACKWARD_ALGOS[algo]))
+    need = int(lib.kda_chunk_backward_workspace_size_ex(B, T, H, dk, dv, N, _dtype_code(q), BACKWARD_ALGOS[algo]))
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = (_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(init_state), _p(d_o), _p(dfinal_state), _p(g["dq"]),
             _p(g["dk"]), _p(g["dv"]), _p(g["dlog_alpha"]), _p(g["dbeta"]), _p(g["dinit_state"]), _p(cu_seqlens),
             B, T, H, dk, dv, N, _dtype_code(q), CHUNK, _p(workspace), ws_bytes, _stream(dev))
-    if _gate_scalar:
-        rc = lib.kda_gdn_chunk_backward(*args)
-    else:
-        rc = lib.kda_chunk_backward_ex(*args, BACKWARD_ALGOS[algo])
+    entry = lib.kda_gdn_chunk_backward_ex if _gate_scalar else lib.kda_chunk_backward_ex
+    rc = entry(*args, BACKWARD_ALGOS[algo])
     _check(rc)
     return g
 

@@ -283,8 +283,9 @@ __device__ __forceinline__ bool slot_chunk(const int32_t *cu_seqlens, int T, int
 // Running sum G of log_alpha over one chunk, per (token, channel), for the 8 tokens x
 // 4 channels of this thread (tokens 8 seg.., channels 4 cg..; 256 threads): rows
 // past Lc count as log_alpha = 0 and k = q = 0.  fSeg: [8][128] fp32 scratch.
-// Returns the thread's G values, k (and q) rows as bf16 pairs, and G_last.
-template <bool WITH_Q>
+// Returns the thread's G values, k (and q) rows as bf16 pairs, and G_last.  GS: one
+// rate per (token, head) ([tokens, H]), the same for every channel.
+template <bool WITH_Q, bool GS = false>
 __device__ __forceinline__ void chunk_decay(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                                             const float *__restrict__ log_alpha, long long cs, int Lc, int H, int h,
                                             float *fSeg, float (&G)[8][4], uint2 (&kv)[8], uint2 (&qv)[8],
@@ -294,8 +295,13 @@ __device__ __forceinline__ void chunk_decay(const __nv_bfloat16 *__restrict__ q,
     float4 gv[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-        const long long off = ((cs + min(i0 + u, Lc - 1)) * H + h) * DK + c0;
-        gv[u] = __ldg(reinterpret_cast<const float4 *>(log_alpha + off));
+        const long long row = cs + min(i0 + u, Lc - 1), off = (row * H + h) * DK + c0;
+        if constexpr (GS) {
+            const float gs = __ldg(log_alpha + row * H + h);
+            gv[u] = make_float4(gs, gs, gs, gs);
+        } else {
+            gv[u] = __ldg(reinterpret_cast<const float4 *>(log_alpha + off));
+        }
         kv[u] = __ldg(reinterpret_cast<const uint2 *>(k + off));
         if constexpr (WITH_Q) qv[u] = __ldg(reinterpret_cast<const uint2 *>(q + off));
     }
@@ -467,6 +473,7 @@ __device__ __noinline__ void chain_pairs_exact(const uint8_t *da, const float *f
 //   sums on the CUDA cores.  Then, with a = e^G dKhat + RK, b = e^{G_last - G} dKbar:
 //     dq = e^G dQhat + RQ,  dk = a + b + CT,  dG = q dq + k (a - b - CT),
 //     dlog_alpha_t = e^{G_last} sum_v S dS' + sum_i k_i b_i + sum_{i>=t} dG_i.
+template <bool GS>
 __global__ void __launch_bounds__(NT, 1)
 bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -523,7 +530,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
         ptx::tma_prefetch_l2_3d(&tm_v, 0, hp, (int)pcs);
         ptx::tma_prefetch_l2_3d(&tm_q, 0, hp, (int)pcs);
         ptx::tma_prefetch_l2_3d(&tm_k, 0, hp, (int)pcs);
-        ptx::tma_prefetch_l2_3d(&tm_g, 0, hp, (int)pcs);
+        if constexpr (!GS) ptx::tma_prefetch_l2_3d(&tm_g, 0, hp, (int)pcs);
     };
     // persistent: items (slot, head), slot fastest, strided by the grid
     for (int it = (int)blockIdx.x; ok && it < n_items; it += (int)gridDim.x) {
@@ -549,7 +556,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
         // G, k and q of this thread's 8 tokens x 4 channels, kept for phase 4
         float G[8][4], tot[4];
         uint2 kv[8], qv[8];
-        chunk_decay<true>(q, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
+        chunk_decay<true, GS>(q, k, log_alpha, cs, Lc, H, h, fSeg, G, kv, qv, tot);
         const int c0 = 4 * (tid & 31), i0 = 8 * (tid >> 5);
         {   // Kbar = e^{G_last - G} K (factors <= 1) and e^{G_last}, while the copies fly
 #pragma unroll
@@ -885,10 +892,20 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant
                 *reinterpret_cast<uint4 *>(dq + o) = *reinterpret_cast<const uint4 *>(oq + i * DK + 8 * g);
                 *reinterpret_cast<uint4 *>(dk_out + o) = *reinterpret_cast<const uint4 *>(okk + i * DK + 8 * g);
             }
-            for (int idx = tid; idx < Lc * (DK / 4); idx += NT) {
-                const int i = idx / (DK / 4), g = idx % (DK / 4);
-                *reinterpret_cast<float4 *>(dlog_alpha + ((cs + i) * H + h) * DK + 4 * g) =
-                    *reinterpret_cast<const float4 *>(og + i * DK + 4 * g);
+            if constexpr (GS) {   // the shared rate's gradient: the sum over the channels, one warp per row
+                for (int i = warp; i < Lc; i += NT / 32) {
+                    const float4 x = *reinterpret_cast<const float4 *>(og + i * DK + 4 * lane);
+                    float t = (x.x + x.y) + (x.z + x.w);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+                    if (lane == 0) dlog_alpha[(cs + i) * H + h] = t;
+                }
+            } else {
+                for (int idx = tid; idx < Lc * (DK / 4); idx += NT) {
+                    const int i = idx / (DK / 4), g = idx % (DK / 4);
+                    *reinterpret_cast<float4 *>(dlog_alpha + ((cs + i) * H + h) * DK + 4 * g) =
+                        *reinterpret_cast<const float4 *>(og + i * DK + 4 * g);
+                }
             }
         }
         // this item's shared-memory reads complete before the next item's copies land
@@ -932,7 +949,9 @@ inline int launch_ok(const char *what, char *msg, size_t msg_len) {
     return KDA_ERR_CUDA;
 }
 
-// The three launches for bf16 inputs, dk = dv = 128 (per-channel decay).
+// The three launches for bf16 inputs, dk = dv = 128; GS: one decay rate per
+// (token, head) (Gated DeltaNet), log_alpha and dlog_alpha [tokens, H].
+template <bool GS>
 inline int launch_backward_tc(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                               const float *init_state, const void *d_o, const float *dfinal, void *dq, void *dk_out,
                               void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state,
@@ -950,20 +969,21 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
     CUtensorMap t_v64, t_do64, t_v128, t_q, t_k, t_g;
     memset(&t_v64, 0, sizeof(t_v64));   // no tokens: the sweeps load nothing (the adjoint one copies dfinal)
     memset(&t_do64, 0, sizeof(t_do64));
+    memset(&t_g, 0, sizeof(t_g));       // GS: log_alpha is not prefetched by tensor map
     if (slots > 0 && (!make_tmap(&t_v64, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, DVT) ||
         !make_tmap(&t_do64, d_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap(&t_v128, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DV, 128) ||
         !make_tmap(&t_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DK, DK) ||
         !make_tmap(&t_k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, DK, DK) ||
-        !make_tmap(&t_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, DK, DK))) {
+        (!GS && !make_tmap(&t_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, DK, DK)))) {
         snprintf(msg, msg_len, "building TMA descriptors failed (driver entry point cuTensorMapEncodeTiled)");
         return KDA_ERR_CUDA;
     }
     int rc;
-    auto k1 = chunk_intra_kernel<DK, false, false, true>;
+    auto k1 = chunk_intra_kernel<DK, GS, false, true>;
     auto k2 = bwd_sweeps_kernel<DK, DVT, NBUF>;
-    auto k4 = bwd_grad_kernel;
+    auto k4 = bwd_grad_kernel<GS>;
     constexpr int s1 = IntraLayout<DK>::ALLOC, s2 = sweeps_smem<DK, DVT, NBUF>(), s4 = GradLayout::ALLOC;
     if ((rc = set_smem_tc(k1, s1, "chunk_intra", msg, msg_len)) ||
         (rc = set_smem_tc(k2, s2, "bwd_sweeps", msg, msg_len)) || (rc = set_smem_tc(k4, s4, "bwd_grad", msg, msg_len)))

@@ -335,9 +335,10 @@ int launch_backward(const void *q, const void *k, const void *v, const float *lo
     return KDA_OK;
 }
 
-// The tensor-core backward covers bf16 inputs, per-channel decay, dk = dv = 128.
+// The tensor-core backward covers bf16 inputs with dk = dv = 128 (either gate).
 bool backward_tc_eligible(int dtype, int dk, int dv, bool gate_scalar) {
-    return dtype == KDA_BF16 && dk == 128 && dv == 128 && !gate_scalar;
+    (void)gate_scalar;
+    return dtype == KDA_BF16 && dk == 128 && dv == 128;
 }
 
 // Workspace bytes of the backward path that `algo` selects (0 for an unusable choice).
@@ -372,7 +373,7 @@ int backward_impl(const void *q, const void *k, const void *v, const float *log_
     const long long tokens = (long long)B * T;
     const bool use_tc = backward_tc_eligible(dtype, dk, dv, gate_scalar) && algo != KDA_BWD_SIMT;
     if (algo == KDA_BWD_TENSOR && !use_tc)
-        return fail(KDA_ERR_UNSUPPORTED, "the tensor-core backward takes bf16, per-channel decay, dk = dv = 128");
+        return fail(KDA_ERR_UNSUPPORTED, "the tensor-core backward takes bf16 inputs with dk = dv = 128");
     const size_t need = backward_ws(tokens, H, dk, dv, num_seqs, dtype, gate_scalar, algo);
     if (need > 0 && (!workspace || ws_bytes < need))
         return fail(KDA_ERR_WORKSPACE, "backward workspace of %zu bytes needed, %zu given%s", need, ws_bytes,
@@ -384,9 +385,14 @@ int backward_impl(const void *q, const void *k, const void *v, const float *log_
     cudaStream_t st = (cudaStream_t)stream;
     if (use_tc) {
         char msg[256] = "";
-        const int rc2 = kda::tc::launch_backward_tc(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq,
-                                                    dk_out, dv_out, dlog_alpha, dbeta, dinit_state, cu_seqlens,
-                                                    tokens, T, H, num_seqs, workspace, st, msg, sizeof(msg));
+        const int rc2 =
+            gate_scalar
+                ? kda::tc::launch_backward_tc<true>(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out,
+                                                    dv_out, dlog_alpha, dbeta, dinit_state, cu_seqlens, tokens, T, H,
+                                                    num_seqs, workspace, st, msg, sizeof(msg))
+                : kda::tc::launch_backward_tc<false>(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq,
+                                                     dk_out, dv_out, dlog_alpha, dbeta, dinit_state, cu_seqlens,
+                                                     tokens, T, H, num_seqs, workspace, st, msg, sizeof(msg));
         return rc2 ? fail(rc2, "%s", msg) : KDA_OK;
     }
 #define KDA_BWD_ARGS                                                                                      \
@@ -641,6 +647,17 @@ int kda_chunk_backward(const void *q, const void *k, const void *v, const float 
     return backward_impl(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, dlog_alpha,
                          dbeta, dinit_state, cu_seqlens, B, T, H, dk, dv, num_seqs, dtype, chunk, workspace, ws_bytes,
                          stream, false);
+}
+
+int kda_gdn_chunk_backward_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                              const float *beta, const float *init_state, const void *d_o, const float *dfinal_state,
+                              void *dq, void *dk_out, void *dv_out, float *dlog_alpha, float *dbeta,
+                              float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H, int dk, int dv,
+                              int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes, void *stream,
+                              int algo) {
+    return backward_impl(q, k, v, log_alpha, beta, init_state, d_o, dfinal_state, dq, dk_out, dv_out, dlog_alpha,
+                         dbeta, dinit_state, cu_seqlens, B, T, H, dk, dv, num_seqs, dtype, chunk, workspace, ws_bytes,
+                         stream, true, algo);
 }
 
 int kda_gdn_chunk_backward(const void *q, const void *k, const void *v, const float *log_alpha,

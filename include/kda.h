@@ -354,12 +354,14 @@ int kda_chunk_backward(const void *q, const void *k, const void *v, const float 
 
 /*
  * Backward schedules (kda_chunk_backward_ex):
- *   KDA_BWD_TENSOR  bf16 inputs, per-channel decay, dk = dv = 128: five launches
- *                   on the tensor cores (tcgen05): the forward's first pass with
- *                   the chunk's Akk, Aqk and T kept, the state sweep storing each
- *                   chunk's starting state (bf16), the adjoint sweep storing each
- *                   chunk's ending adjoint (bf16), the per-chunk products that
- *                   need them, and the chain rule through the decay factors.
+ *   KDA_BWD_TENSOR  bf16 inputs with dk = dv = 128 (per-channel decay, or one rate
+ *                   per token-head through kda_gdn_chunk_backward_ex): three
+ *                   launches on the tensor cores (tcgen05) -- the forward's first
+ *                   pass keeping the chunk's Akk, Aqk and T; the state sweep
+ *                   storing each chunk's starting state and the adjoint sweep
+ *                   storing each chunk's ending adjoint (bf16), side by side; and
+ *                   per (chunk, head) the products that need them and the chain
+ *                   rule through the decay factors.
  *                   Workspace: one 145 KB unit per (64-token chunk slot, head)
  *                   (0.61 GB for 8192 tokens x 32 heads).  Operands are bf16
  *                   with fp32 accumulation, like the forward's tensor-core path.
@@ -379,7 +381,8 @@ size_t kda_chunk_backward_workspace_size_ex(int B, int T, int H, int dk, int dv,
 
 /* kda_chunk_backward with an explicit schedule (KDA_BWD_*).  KDA_ERR_UNSUPPORTED
  * when KDA_BWD_TENSOR is asked for inputs it does not cover; KDA_ERR_INVALID_ARG
- * for an unknown algo; otherwise as kda_chunk_backward. */
+ * for an unknown algo; otherwise as kda_chunk_backward.  The workspace is
+ * kda_chunk_backward_workspace_size_ex's for the same sizes, dtype and algo. */
 int kda_chunk_backward_ex(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, const float *init_state, const void *d_o,
                           const float *dfinal_state, void *dq, void *dk_out, void *dv_out, float *dlog_alpha,
@@ -402,6 +405,15 @@ int kda_gdn_chunk_backward(const void *q, const void *k, const void *v, const fl
                            float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
                            int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
                            void *stream);
+
+/* kda_gdn_chunk_backward with an explicit schedule (KDA_BWD_*), as
+ * kda_chunk_backward_ex (the same workspace sizes). */
+int kda_gdn_chunk_backward_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                              const float *beta, const float *init_state, const void *d_o,
+                              const float *dfinal_state, void *dq, void *dk_out, void *dv_out, float *dlog_alpha,
+                              float *dbeta, float *dinit_state, const int32_t *cu_seqlens, int B, int T, int H,
+                              int dk, int dv, int num_seqs, int dtype, int chunk, void *workspace, size_t ws_bytes,
+                              void *stream, int algo);
 
 /* Message for the calling thread's last non-OK return ("" if none). */
 const char *kda_last_error(void);

@@ -221,31 +221,34 @@ def test_backward_prefill_8k_sampled_heads(algo):
     check(got, oracle_grads(d, c, heads), BF16, heads=heads, what="prefill_8k")
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, BF16])
+@pytest.mark.parametrize("dtype,algo", SCHEDULES)
 @pytest.mark.parametrize("packed", [False, True])
-def test_gdn_backward_matches_oracle(dtype, packed):
+@pytest.mark.parametrize("d128", [False, True])
+def test_gdn_backward_matches_oracle(dtype, algo, packed, d128):
     """Gated DeltaNet (one decay rate per token-head): the oracle's gradients with
     the rate broadcast over the key channels, dlog_alpha summed over them (the
-    gradient of a broadcast value)."""
+    gradient of a broadcast value).  d128: dk = dv = 128, which the tensor-core
+    schedule takes."""
     if packed:
         lens = [70, 0, 129, 1]
-        shape = PrefillShape(B=1, T=sum(lens), H=2, dk=128, dv=64, dtype=dtype, gate="scalar",
+        shape = PrefillShape(B=1, T=sum(lens), H=2, dk=128, dv=128 if d128 else 64, dtype=dtype, gate="scalar",
                              cu_seqlens=tuple(np.cumsum([0] + lens).tolist()))
     else:
-        shape = PrefillShape(B=2, T=150, H=2, dk=64, dv=128, dtype=dtype, gate="scalar")
+        shape = PrefillShape(B=2, T=150, H=2, dk=128 if d128 else 64, dv=128, dtype=dtype, gate="scalar")
     d = prefill_inputs(shape, 91, DEV)
     assert d["log_alpha"].shape == d["beta"].shape
     c = backward_cotangents(shape, 92, DEV)
     got = kda.gdn_chunk_backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], c["d_o"], d["init_state"],
-                                 c["dfinal_state"], d["cu_seqlens"])
+                                 c["dfinal_state"], d["cu_seqlens"], algo=algo)
     torch.cuda.synchronize()
+    assert kda.device_status() == 0
     dk = shape.dk
     d_b = dict(d, log_alpha=d["log_alpha"][..., None].expand(*d["log_alpha"].shape, dk).contiguous())
     want = oracle_grads(d_b, c)
     want["dlog_alpha"] = want["dlog_alpha"].sum(axis=-1)
-    check(got, want, dtype, what="gdn")
-    # the same kernels with the rate broadcast and the channel gradients summed
-    full = run(d_b, c, algo="simt")
+    check(got, want, dtype, what=f"gdn {algo}")
+    # the same schedule with the rate broadcast and the channel gradients summed
+    full = run(d_b, c, algo=algo)
     torch.testing.assert_close(got["dlog_alpha"], full["dlog_alpha"].sum(-1), rtol=1e-4, atol=1e-4)
     for name in ("dq", "dk", "dv", "dbeta", "dinit_state"):
         assert torch.equal(got[name], full[name]), name
