@@ -54,6 +54,7 @@ BACKWARD_FLOPS_PER_TOKEN_HEAD = 2 * PREFILL_FLOPS_PER_TOKEN_HEAD                
 # The tensor-core backward of bf16 inputs with dk = dv = 128: three launches per call.
 BACKWARD_KERNELS = "chunk_intra_kernel (with the backward extras) + bwd_sweeps_kernel + bwd_grad_kernel"
 BACKWARD_LAUNCHES = 3
+BACKWARD_REPS = 100   # ~0.1 s of backward_8k calls in the timed region
 # Fused prologue, per token-head: raw q, k, v and the gate pre-activation (bf16), beta, o.
 PROLOGUE_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 2 * 128 + 4 + 2 * 128                    # 1284
 # DRAM bytes (read + write) per launch, taken from ncu captures (dram__bytes_read.sum +
@@ -124,7 +125,6 @@ class ClockSampler:
             return
         while not event.query():
             self._sample()
-            time.sleep(self._period)
 
     def __enter__(self):
         if self._h is not None:
@@ -168,6 +168,23 @@ def _barrier(world):
         import torch.distributed as dist
 
         dist.barrier()
+
+
+def _time_reps(dev, stream, reps, step):
+    """CUDA-event time (ms) of `reps` calls of step() on `stream`, and the NVML clocks
+    sampled while they run (from this thread too once the launches are queued)."""
+    import torch
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        e0.record(stream)
+        for _ in range(reps):
+            step()
+        e1.record(stream)
+        clk.poll(e1)
+        torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1), clk.summary()
 
 
 def _job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
@@ -276,16 +293,10 @@ def run_prefill_gdn(args, world, rank, dev):
     stream = torch.cuda.current_stream(dev)
     reps = 300
     _barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    total, clocks = _time_reps(dev, stream, reps, step)
+    ms = _max_over_ranks(total / reps, world, dev)
     del d
-    return dict(ms=ms, launches=reps * (2 if ws_n else 1))
+    return dict(ms=ms, launches=reps * (2 if ws_n else 1), clocks=clocks)
 
 
 def run_prefill_prologue(args, world, rank, dev):
@@ -312,16 +323,10 @@ def run_prefill_prologue(args, world, rank, dev):
     stream = torch.cuda.current_stream(dev)
     reps = 300
     _barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    total, clocks = _time_reps(dev, stream, reps, step)
+    ms = _max_over_ranks(total / reps, world, dev)
     del d
-    return dict(ms=ms, launches=reps * 2)
+    return dict(ms=ms, launches=reps * 2, clocks=clocks)
 
 
 def run_backward(args, world, rank, dev):
@@ -347,18 +352,12 @@ def run_backward(args, world, rank, dev):
         step()
     torch.cuda.synchronize(dev)
     stream = torch.cuda.current_stream(dev)
-    reps = max(5, min(args.steps, 30))
+    reps = BACKWARD_REPS
     _barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    total, clocks = _time_reps(dev, stream, reps, step)
+    ms = _max_over_ranks(total / reps, world, dev)
     del d, c, ws, out
-    return dict(ms=ms, launches=reps * BACKWARD_LAUNCHES)
+    return dict(ms=ms, launches=reps * BACKWARD_LAUNCHES, clocks=clocks, reps=reps)
 
 
 def run_prefill_varlen(args, world, rank, dev):
@@ -386,19 +385,13 @@ def run_prefill_varlen(args, world, rank, dev):
     stream = torch.cuda.current_stream(dev)
     reps = 4
     _barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = _max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+    total, clocks = _time_reps(dev, stream, reps, step)
+    ms = _max_over_ranks(total / reps, world, dev)
     token_heads = shape.T * shape.H
     alg_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * shape.num_seqs * shape.H * STATE_BYTES
     del d, o, fs
     return dict(ms=ms, tokens=shape.T, alg_bytes=alg_bytes, alg_flops=token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD,
-                seqs=shape.num_seqs, launches=reps * len(kernels), kernels=kernels)
+                seqs=shape.num_seqs, launches=reps * len(kernels), kernels=kernels, clocks=clocks)
 
 
 def run_prefill_long(args, world, rank, dev):
@@ -620,6 +613,7 @@ def backward_block(args, world, bw, hbm_gbs, bf16_tflops):
                      "traffic": NCU_TRAFFIC.get((f"backward_T{T}", "bwd")), "algorithmic_bytes": bbytes,
                      "tensor": {"achieved_tflops": btf, "peak_tflops": bf16_tflops, "frac": btf / bf16_tflops,
                                 "algorithmic_flops": bflops}},
+        "calls": bw["reps"], "clocks": bw["clocks"],
     }
 
 
@@ -627,7 +621,7 @@ def main_backward_only(args, world, rank, dev):
     bw = run_backward(args, world, rank, dev)
     hbm_gbs, bf16_tflops, _ = _peaks()
     line = backward_block(args, world, bw, hbm_gbs, bf16_tflops)
-    line.update({"n_gpus": world, "steps": max(5, min(args.steps, 30)), "warmup": args.warmup,
+    line.update({"n_gpus": world, "steps": bw["reps"], "warmup": args.warmup,
                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                  "data": "synthetic", "config": {"workload": f"backward T={args.backward_T} H=32 d=128 bf16"},
                  "gpu_launches": bw["launches"]})
@@ -757,6 +751,7 @@ def main(argv=None):
                          "achieved": ggbs, "peak": hbm_gbs, "unit": "GB/s", "frac": ggbs / hbm_gbs, "traffic": None,
                          "algorithmic_bytes": gbytes,
                          "tensor": {"achieved_tflops": gtf, "peak_tflops": bf16_tflops, "frac": gtf / bf16_tflops}},
+            "clocks": gd["clocks"],
         }
         line["gpu_launches"] += gd["launches"]
     if pr is not None:
@@ -771,6 +766,7 @@ def main(argv=None):
                          "achieved": pgbs, "peak": hbm_gbs, "unit": "GB/s", "frac": pgbs / hbm_gbs, "traffic": None,
                          "algorithmic_bytes": pbytes,
                          "tensor": {"achieved_tflops": ptf, "peak_tflops": bf16_tflops, "frac": ptf / bf16_tflops}},
+            "clocks": pr["clocks"],
         }
         line["gpu_launches"] += pr["launches"]
     if bw is not None:
@@ -800,6 +796,7 @@ def main(argv=None):
                          "unit": "GB/s", "frac": vgbs / hbm_gbs, "traffic": None,
                          "algorithmic_bytes": vl["alg_bytes"],
                          "tensor": {"achieved_tflops": vtf, "peak_tflops": bf16_tflops, "frac": vtf / bf16_tflops}},
+            "clocks": vl["clocks"],
         }
         line["gpu_launches"] += vl["launches"]
     if lg is not None:
