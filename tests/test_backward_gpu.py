@@ -132,16 +132,17 @@ def test_backward_strong_decay_blocks(dtype, algo):
     check(got, oracle_grads(d, c), dtype, what=f"strong decay {algo}")
 
 
-def test_backward_without_states():
+@pytest.mark.parametrize("dtype,dk,algo", [(torch.float32, 64, "auto"), (BF16, 128, "tensor")])
+def test_backward_without_states(dtype, dk, algo):
     """init_state NULL (zeros) and dfinal_state NULL (zero cotangent): dinit_state is
     the gradient at the zero state."""
-    shape = PrefillShape(B=2, T=150, H=2, dk=64, dv=128, dtype=torch.float32, init_state="none")
+    shape = PrefillShape(B=2, T=150, H=2, dk=dk, dv=128, dtype=dtype, init_state="none")
     d = prefill_inputs(shape, 31, DEV)
     assert d["init_state"] is None
     c = backward_cotangents(shape, 32, DEV, dfinal=False)
-    got = run(d, c)
+    got = run(d, c, algo=algo)
     torch.cuda.synchronize()
-    check(got, oracle_grads(d, c), torch.float32, what="no states")
+    check(got, oracle_grads(d, c), dtype, what=f"no states {algo}")
     assert got["dinit_state"].abs().max().item() > 0
 
 
@@ -195,12 +196,13 @@ def test_backward_is_deterministic(algo):
         assert torch.equal(a[name], b[name]), name
 
 
-def test_backward_skips_dinit_state():
-    shape = PrefillShape(B=1, T=100, H=2, dk=64, dv=64, dtype=BF16)
+@pytest.mark.parametrize("dk,dv,algo", [(64, 64, "auto"), (128, 128, "tensor")])
+def test_backward_skips_dinit_state(dk, dv, algo):
+    shape = PrefillShape(B=1, T=100, H=2, dk=dk, dv=dv, dtype=BF16)
     d = prefill_inputs(shape, 11, DEV)
     c = backward_cotangents(shape, 12, DEV)
-    full = run(d, c)
-    part = run(d, c, dinit_state=False)
+    full = run(d, c, algo=algo)
+    part = run(d, c, dinit_state=False, algo=algo)
     assert part["dinit_state"] is None
     for name in GRADS[:-1]:
         assert torch.equal(full[name], part[name]), name
@@ -278,3 +280,33 @@ def test_backward_split_resume_chain_rule(split):
         both = torch.cat([g1[name], g2[name]], dim=1)
         torch.testing.assert_close(both, whole[name], rtol=1e-4, atol=1e-5, msg=name)
     torch.testing.assert_close(g1["dinit_state"], whole["dinit_state"], rtol=1e-4, atol=1e-5)
+
+
+def test_backward_split_resume_tensor_schedule():
+    """The split/resume chain rule on the tensor-core schedule (bf16, dk = dv = 128),
+    split at a chunk boundary: the two parts joined by the state and its adjoint
+    match one call to bf16 accuracy, and each part matches the oracle."""
+    shape = PrefillShape(B=1, T=300, H=2, dk=128, dv=128, dtype=BF16)
+    d = prefill_inputs(shape, 57, DEV)
+    c = backward_cotangents(shape, 58, DEV)
+    whole = run(d, c, algo="tensor")
+    split = 128
+    cut = lambda x, a, b: x[:, a:b].contiguous()
+    first = {x: cut(d[x], 0, split) for x in ("q", "k", "v", "log_alpha", "beta")}
+    first["init_state"] = d["init_state"]
+    second = {x: cut(d[x], split, 300) for x in ("q", "k", "v", "log_alpha", "beta")}
+    _, S_mid = kda.chunk_forward(*(first[x] for x in ("q", "k", "v", "log_alpha", "beta")), first["init_state"],
+                                 simt=True)
+    second["init_state"] = S_mid
+    c2 = {"d_o": cut(c["d_o"], split, 300), "dfinal_state": c["dfinal_state"]}
+    g2 = run(second, c2, algo="tensor")
+    c1 = {"d_o": cut(c["d_o"], 0, split), "dfinal_state": g2["dinit_state"]}
+    g1 = run(first, c1, algo="tensor")
+    torch.cuda.synchronize()
+    check(g2, oracle_grads(second, c2), BF16, what="second part")
+    check(g1, oracle_grads(first, c1), BF16, what="first part")
+    for name in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+        both = to_f64(torch.cat([g1[name], g2[name]], dim=1))
+        assert rel_l2(both, to_f64(whole[name])) <= 1e-2, name
+    assert rel_l2(to_f64(g1["dinit_state"]), to_f64(whole["dinit_state"])) <= 1e-2
+
