@@ -189,7 +189,11 @@ def chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *,
     (allocate and return), False (skip) or a preallocated float32 tensor.
     `algo` picks the tensor-core schedule ("auto", "fused", "two_pass"); the
     workspace it needs is allocated here unless `workspace` (uint8, CUDA) is
-    given.  With `simt=True` the fp32 CUDA-core path (kda_chunk_forward_simt)
+    given.  "auto" takes the two-pass schedule for few (sequence, head) chains
+    while its workspace is at most 4 GiB (58 KB per 64-token chunk and head: 3.8 GB
+    at 131072 tokens x 32 heads); pass a reusable `workspace`
+    (workspace_size(..., algo=...)) to keep it across calls, or algo="fused" to
+    need none.  With `simt=True` the fp32 CUDA-core path (kda_chunk_forward_simt)
     runs instead.  Host (CPU) inputs are copied to the current CUDA device and
     the results copied back, all inside this call.
     Returns (o, final_state or None).
