@@ -183,6 +183,38 @@ def test_backward_workspace_sizes(lib):
     assert f(1, 100, 2, 96, 128, 1) == 0         # unsupported dk
 
 
+UNIT128 = 148480   # tensor-core backward bytes per (chunk slot, head) at dk = dv = 128
+BWD_AUTO, BWD_TENSOR, BWD_SIMT = 0, 1, 2
+
+
+def test_backward_workspace_sizes_by_schedule(lib):
+    f = lib.kda_chunk_backward_workspace_size_ex
+    assert f(1, 8192, 32, 128, 128, 1, 0, BWD_AUTO) == 129 * 32 * UNIT128     # bf16, dk = dv = 128: tensor cores
+    assert f(1, 8192, 32, 128, 128, 1, 0, BWD_TENSOR) == 129 * 32 * UNIT128
+    assert f(1, 8192, 32, 128, 128, 1, 0, BWD_SIMT) == bwd_ws(129, 32, 128, 128)
+    assert f(1, 8192, 32, 128, 128, 1, 1, BWD_AUTO) == bwd_ws(129, 32, 128, 128)   # fp32: SIMT
+    assert f(1, 8192, 32, 128, 128, 1, 1, BWD_TENSOR) == 0                          # not covered
+    assert f(1, 100, 2, 128, 64, 1, 0, BWD_AUTO) == bwd_ws(2 + 1, 2, 128, 64)      # dv = 64: SIMT
+    assert f(1, 100, 2, 128, 64, 1, 0, BWD_TENSOR) == 0
+    assert f(2, 0, 2, 128, 128, 2, 0, BWD_AUTO) == 0                                # no tokens
+    # the dtype-free query covers either schedule
+    for args in [(1, 8192, 32, 128, 128, 1), (3, 100, 2, 64, 64, 3), (1, 100, 2, 128, 64, 1)]:
+        for dtype in (0, 1):
+            assert lib.kda_chunk_backward_workspace_size(*args) >= f(*args, dtype, BWD_AUTO)
+
+
+def test_backward_ex_rejects(lib):
+    def call(entry, algo, dtype=0, dk=128, dv=128, wsb=1 << 30):
+        return entry(A[0], A[1], A[2], A[3], A[4], A[5], A[6], A[7], A[8], A[9], A[10], A[11], A[11] + 0x8000,
+                     A[11] + 0x4000, None, 1, 128, 2, dk, dv, 1, dtype, 64, A[0] + 0x8000, wsb, None, algo)
+    for entry in (lib.kda_chunk_backward_ex, lib.kda_gdn_chunk_backward_ex):
+        assert call(entry, 7) == INVALID                           # no such schedule
+        assert call(entry, BWD_TENSOR, dtype=1) == UNSUPPORTED      # fp32 inputs: SIMT only
+        assert call(entry, BWD_TENSOR, dk=64, dv=64) == UNSUPPORTED
+        assert call(entry, BWD_TENSOR, wsb=2 * 3 * UNIT128 - 16) == WORKSPACE   # one byte row short
+        assert lib.kda_last_error().decode() != ""
+
+
 def backward(lib, **over):
     a = dict(q=A[0], k=A[1], v=A[2], g=A[3], b=A[4], s0=A[5], do=A[6], dF=A[7], dq=A[8], dk_=A[9], dv_=A[10],
              dg=A[11], db=A[11] + 0x8000, ds0=A[11] + 0x4000, cu=None, B=1, T=128, H=2, dk=128, dv=128, N=1,
