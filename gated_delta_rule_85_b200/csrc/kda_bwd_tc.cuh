@@ -262,24 +262,6 @@ constexpr int sweeps_smem() {
 
 // ------------------------------------------------------------------ per-chunk sums
 
-// Chunk of `slot`: the last sequence n whose first slot n + floor(t0_n / 64) is
-// <= slot owns it.  False for a slot without a chunk (uniform over the CTA).
-__device__ __forceinline__ bool slot_chunk(const int32_t *cu_seqlens, int T, int num_seqs, int slot, long long &cs,
-                                           int &Lc) {
-    int lo = 0, hi = num_seqs - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (mid + seq_begin(cu_seqlens, T, mid) / C <= slot) lo = mid;
-        else hi = mid - 1;
-    }
-    long long t0, t1;
-    seq_span(cu_seqlens, T, lo, t0, t1);
-    cs = t0 + (long long)(slot - (lo + t0 / C)) * C;
-    if (cs < t0 || cs >= t1) return false;
-    Lc = (int)min((long long)C, t1 - cs);
-    return true;
-}
-
 // Running sum G of log_alpha over one chunk, per (token, channel), for the 8 tokens x
 // 4 channels of this thread (tokens 8 seg.., channels 4 cg..; 256 threads): rows
 // past Lc count as log_alpha = 0 and k = q = 0.  fSeg: [8][128] fp32 scratch.
@@ -988,9 +970,14 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
     if ((rc = set_smem_tc(k1, s1, "chunk_intra", msg, msg_len)) ||
         (rc = set_smem_tc(k2, s2, "bwd_sweeps", msg, msg_len)) || (rc = set_smem_tc(k4, s4, "bwd_grad", msg, msg_len)))
         return rc;
-    const dim3 per_chunk((unsigned)slots, H);
     if (slots > 0) {
-        k1<<<per_chunk, NT, s1, st>>>(qb, kb, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws);
+        CUtensorMap iq, ik, ig;
+        if (!intra_tmaps(&iq, &ik, &ig, q, k, log_alpha, GS, false, tokens, H, DK)) {
+            snprintf(msg, msg_len, "building TMA descriptors failed (driver entry point cuTensorMapEncodeTiled)");
+            return KDA_ERR_CUDA;
+        }
+        k1<<<intra_grid(slots * H), NT, s1, st>>>(iq, ik, ig, qb, kb, log_alpha, beta, cu_seqlens, T, H, num_seqs,
+                                                  (int)slots, ws);
         if ((rc = launch_ok("chunk_intra", msg, msg_len))) return rc;
     }
     // both sweeps; with no tokens only the adjoint half has work (dinit_state = dfinal)

@@ -23,6 +23,8 @@
 // token ranges; a dense batch uses t0 = n T.
 #pragma once
 
+#include <cstring>
+
 #include "kda_chunk_tc.cuh"
 
 namespace kda {
@@ -77,6 +79,25 @@ __device__ __forceinline__ long long seq_begin(const int32_t *cu_seqlens, int T,
 }
 
 // ------------------------------------------------------------------ pass 1
+
+// Chunk of `slot`: the last sequence n whose first slot n + floor(t0_n / 64) is
+// <= slot owns it.  False for a slot without a chunk (uniform over the CTA).
+__device__ __forceinline__ bool slot_chunk(const int32_t *cu_seqlens, int T, int num_seqs, int slot, long long &cs,
+                                           int &Lc) {
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (mid + seq_begin(cu_seqlens, T, mid) / C <= slot) lo = mid;
+        else hi = mid - 1;
+    }
+    long long t0, t1;
+    seq_span(cu_seqlens, T, lo, t0, t1);
+    cs = t0 + (long long)(slot - (lo + t0 / C)) * C;
+    if (cs < t0 || cs >= t1) return false;
+    Lc = (int)min((long long)C, t1 - cs);
+    return true;
+}
+
 
 template <int DK>
 struct IntraLayout {
@@ -597,13 +618,20 @@ __device__ __noinline__ int intra_chunk_strong(int slot, int h, const __nv_bfloa
     return r;
 }
 
-// First pass: one CTA per (chunk slot, head); tier A inline, tier B out of line.
+// First pass: persistent, two CTAs per SM taking (chunk slot, head) items in turn
+// (slot fastest); tier A inline, tier B out of line.  While an item runs, thread 0
+// prefetches the next item's q, k and gate rows into L2 (tensor-map prefetches; no
+// completion is awaited), so its loads find them there.  tm_g covers the
+// per-channel gate (fp32 log_alpha, or the bf16 pre-activation with PRO); the
+// scalar gate of GS is not prefetched.
 // BX (the backward): ws holds [slot][H] BwdUnit; the extras go beside each record.
 template <int DK, bool GS, bool PRO, bool BX = false>
 __global__ void __launch_bounds__(NT, 2)
-chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                   const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs, uint8_t *__restrict__ ws) {
+chunk_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16 *__restrict__ q,
+                   const __nv_bfloat16 *__restrict__ k, const float *__restrict__ log_alpha,
+                   const float *__restrict__ beta, const int32_t *__restrict__ cu_seqlens, int T, int H, int num_seqs,
+                   int nslots, uint8_t *__restrict__ ws) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t bar_mma = ptx::smem_u32(sm) + IntraLayout<DK>::MISC;
@@ -621,12 +649,31 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     uint32_t ph_mma = 0;
-    const int r = intra_chunk<DK, GS, PRO, false, BX>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta,
-                                                      cu_seqlens, T, H, num_seqs, ws, sm, tmem, ph_mma);
-    if (r == 1) {   // the chunk decays faster than tier A covers (uniform over the CTA)
+    const int n_items = nslots * H;
+    for (int it = (int)blockIdx.x; it < n_items; it += (int)gridDim.x) {
+        if (threadIdx.x == 0 && it + (int)gridDim.x < n_items) {
+            const int nx = it + (int)gridDim.x, ns = nx % nslots, nh = nx / nslots;
+            long long ncs;
+            int nLc;
+            if (slot_chunk(cu_seqlens, T, num_seqs, ns, ncs, nLc)) {
+                ptx::tma_prefetch_l2_3d(&tm_q, 0, nh, (int)ncs);
+                ptx::tma_prefetch_l2_3d(&tm_k, 0, nh, (int)ncs);
+                if constexpr (!GS) ptx::tma_prefetch_l2_3d(&tm_g, 0, nh, (int)ncs);
+            }
+        }
+        const int slot = it % nslots, h = it / nslots;
+        const int r = intra_chunk<DK, GS, PRO, false, BX>(slot, h, q, k, log_alpha, beta, cu_seqlens, T, H,
+                                                          num_seqs, ws, sm, tmem, ph_mma);
+        if (r == 1) {   // the chunk decays faster than tier A covers (uniform over the CTA)
+            __syncthreads();
+            intra_chunk_strong<DK, GS, PRO, BX>(slot, h, q, k, log_alpha, beta, cu_seqlens, T, H, num_seqs, ws, sm,
+                                                tmem, &ph_mma);
+        }
+        if (r < 0) break;   // a wait timed out (flagged; uniform)
+        // this item's shared memory and TMEM are free before the next item starts
+        ptx::tc_fence_before();
         __syncthreads();
-        intra_chunk_strong<DK, GS, PRO, BX>((int)blockIdx.x, (int)blockIdx.y, q, k, log_alpha, beta, cu_seqlens, T,
-                                            H, num_seqs, ws, sm, tmem, &ph_mma);
+        ptx::tc_fence_after();
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -634,6 +681,27 @@ chunk_intra_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, INTRA_TMEM_COLS);
     }
+}
+
+// Grid of the persistent first pass: two CTAs per SM, at most one per item.
+inline unsigned intra_grid(long long items) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess)
+        sms = 148;
+    return (unsigned)(items < 2LL * sms ? items : 2LL * sms);
+}
+
+// Tensor maps the first pass prefetches with (q, k and the per-channel gate rows).
+inline bool intra_tmaps(CUtensorMap *tq, CUtensorMap *tk, CUtensorMap *tg, const void *q, const void *k,
+                        const void *gate, bool gate_scalar, bool gate_bf16, long long tokens, int H, int dk) {
+    memset(tg, 0, sizeof(*tg));
+    if (!make_tmap(tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, dk, dk) ||
+        !make_tmap(tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, dk, dk))
+        return false;
+    if (gate_scalar) return true;
+    return gate_bf16 ? make_tmap(tg, gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, dk, dk)
+                     : make_tmap(tg, gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, dk, dk);
 }
 
 // ------------------------------------------------------------------ pass 2
@@ -921,8 +989,14 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_intra): %s", cudaGetErrorString(e));
         return KDA_ERR_CUDA;
     }
-    k1<<<dim3((unsigned)rec_slots, H), NT, smem1, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
-                                                     beta, cu_seqlens, T, H, num_seqs, (uint8_t *)workspace);
+    CUtensorMap tq, tk, tg;
+    if (!intra_tmaps(&tq, &tk, &tg, q, k, log_alpha, GS, PRO, tokens, H, DK)) {
+        snprintf(msg, msg_len, "building TMA descriptors failed (driver entry point cuTensorMapEncodeTiled)");
+        return KDA_ERR_CUDA;
+    }
+    k1<<<intra_grid(rec_slots * H), NT, smem1, st>>>(tq, tk, tg, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                                  log_alpha, beta, cu_seqlens, T, H, num_seqs, (int)rec_slots,
+                                                  (uint8_t *)workspace);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "chunk_intra launch: %s", cudaGetErrorString(e));
