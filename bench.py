@@ -61,11 +61,11 @@ PROLOGUE_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 2 * 128 + 4 + 2 * 128             
 # dram__bytes_write.sum) of the current kernels on these workloads; keyed by the kernels
 # one step runs.  A kernel set without a capture on its workload reports null.
 NCU_TRAFFIC = {
-    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 269.9e6 + 181.3e6 + 308.3e6 + 51.3e6,
+    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 272.1e6 + 184.8e6 + 308.4e6 + 50.7e6,
     # chunk_tc_kernel (--algo fused): captured before its timeout-path change, so reported null
     ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.2e6,
     # backward: the three kernels of one call (read + write of each)
-    ("backward_T8192", "bwd"): 270.0e6 + 282.4e6 + 492.3e6 + 233.7e6 + 915.8e6 + 311.0e6,
+    ("backward_T8192", "bwd"): 274.1e6 + 285.5e6 + 492.0e6 + 233.2e6 + 911.2e6 + 311.1e6,
 }
 
 
@@ -116,6 +116,11 @@ class ClockSampler:
         while not self._stop.is_set():
             self._sample()
             time.sleep(self._period)
+
+    def sample_now(self):
+        """One sample from the calling thread (between the launches of a timed region)."""
+        if self._h is not None:
+            self._sample()
 
     def poll(self, event):
         """Sample from the calling thread until `event` (recorded after the timed
@@ -233,6 +238,7 @@ def run_prefill(args, world, rank, dev):
             starts[i].record(stream)
             step()
             ends[i].record(stream)
+            clk.sample_now()   # the queued calls keep the GPU busy meanwhile
         t_all1.record(stream)
         clk.poll(t_all1)
         torch.cuda.synchronize(dev)
