@@ -117,11 +117,6 @@ class ClockSampler:
             self._sample()
             time.sleep(self._period)
 
-    def sample_now(self):
-        """One sample from the calling thread (between the launches of a timed region)."""
-        if self._h is not None:
-            self._sample()
-
     def poll(self, event):
         """Sample from the calling thread until `event` (recorded after the timed
         launches) has completed: a short region whose launches were enqueued while
@@ -238,7 +233,6 @@ def run_prefill(args, world, rank, dev):
             starts[i].record(stream)
             step()
             ends[i].record(stream)
-            clk.sample_now()   # the queued calls keep the GPU busy meanwhile
         t_all1.record(stream)
         clk.poll(t_all1)
         torch.cuda.synchronize(dev)
