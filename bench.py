@@ -27,7 +27,6 @@ import json
 import os
 import statistics
 import sys
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -78,8 +77,39 @@ def _peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+_SAMPLER_CHILD = r"""
+import select, sys, time
+import pynvml
+pynvml.nvmlInit()
+uuid, index, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
+h = None
+if uuid:
+    try:
+        h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+    except Exception:
+        h = None
+if h is None:
+    h = pynvml.nvmlDeviceGetHandleByIndex(index)
+print("ready", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+out = []
+while not select.select([sys.stdin], [], [], period)[0]:
+    t = time.monotonic()
+    try:
+        out.append((t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                    int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+    except Exception:
+        pass
+sys.stdout.write("".join(f"{t!r} {c} {r}\n" for t, c, r in out))
+"""
+
+
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML while running."""
+    """Samples SM clock and clock-event reasons through NVML while a timed region runs.
+
+    The reads happen in a child process (an NVML read can take ~0.2 ms, and a
+    sampler thread in this process would compete with the launch loop for the
+    interpreter); samples whose CLOCK_MONOTONIC time falls between entering and
+    leaving the `with` block are kept."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -87,55 +117,63 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.00025):
+    def __init__(self, device_index: int, period_s: float = 0.0005):
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
-        self._stop = threading.Event()
+        self.error = None
+        self._index = device_index
         self._period = period_s
-        self._h = None
-        try:
-            import pynvml
+        self._proc = None
+        self._t0 = self._t1 = None
 
-            pynvml.nvmlInit()
-            self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-        except Exception as e:  # noqa: BLE001
-            self.error = str(e)
-
-    def _sample(self):
-        nv = self._nv
+    def _uuid(self) -> str:
         try:
-            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-            self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            import torch
+
+            u = str(torch.cuda.get_device_properties(self._index).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
         except Exception:  # noqa: BLE001
-            pass
-
-    def _run(self):
-        while not self._stop.is_set():
-            self._sample()
-            time.sleep(self._period)
+            return ""
 
     def poll(self, event):
-        """Sample from the calling thread until `event` (recorded after the timed
-        launches) has completed: a short region whose launches were enqueued while
-        the sampler thread waited for the interpreter still gets its samples."""
-        if self._h is None:
-            return
-        while not event.query():
-            self._sample()
+        """Kept for the call sites: the child process samples on its own."""
 
     def __enter__(self):
-        if self._h is not None:
-            self._t = threading.Thread(target=self._run, daemon=True)
-            self._t.start()
+        import subprocess
+
+        try:
+            self._proc = subprocess.Popen(
+                [sys.executable, "-c", _SAMPLER_CHILD, self._uuid(), str(self._index), str(self._period)],
+                stdin=subprocess.PIPE, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            line = self._proc.stdout.readline().split()
+            if not line or line[0] != "ready":
+                raise RuntimeError("NVML sampler did not start")
+            self.max_mhz = int(line[1])
+        except Exception as e:  # noqa: BLE001
+            self.error = str(e)
+            self._stop_child()
+        self._t0 = time.monotonic()
         return self
 
+    def _stop_child(self):
+        if self._proc is None:
+            return ""
+        try:
+            out, _ = self._proc.communicate(input="stop\n", timeout=30)
+        except Exception:  # noqa: BLE001
+            self._proc.kill()
+            out = ""
+        self._proc = None
+        return out
+
     def __exit__(self, *exc):
-        if self._h is not None:
-            self._stop.set()
-            self._t.join()
+        self._t1 = time.monotonic()
+        for row in self._stop_child().splitlines():
+            t, c, r = row.split()
+            if self._t0 <= float(t) <= self._t1:
+                self.samples.append(int(c))
+                self.reasons |= int(r)
 
     def summary(self):
         if not self.samples:
@@ -229,11 +267,13 @@ def run_prefill(args, world, rank, dev):
         t_all0 = torch.cuda.Event(enable_timing=True)
         t_all1 = torch.cuda.Event(enable_timing=True)
         t_all0.record(stream)
+        h0 = time.perf_counter()
         for i in range(args.steps):
             starts[i].record(stream)
             step()
             ends[i].record(stream)
         t_all1.record(stream)
+        host_ms = (time.perf_counter() - h0) * 1e3 / args.steps   # host time to enqueue one step
         clk.poll(t_all1)
         torch.cuda.synchronize(dev)
     _barrier(world)
@@ -243,7 +283,7 @@ def run_prefill(args, world, rank, dev):
 
     if args.no_e2e:
         return dict(total_ms=total_ms, per_launch_ms=per_launch_ms, clocks=clk.summary(), e2e_ms=float("nan"),
-                    h2d=0, d2h=0, e2e_steps=0, kernels=kernels)
+                    h2d=0, d2h=0, e2e_steps=0, kernels=kernels, host_ms=host_ms)
     # End to end through the public API with host buffers: H2D of every input,
     # the kernel, D2H of o and the final state, every step.
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in d.items()}
@@ -266,7 +306,7 @@ def run_prefill(args, world, rank, dev):
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     del d
     return dict(total_ms=total_ms, per_launch_ms=per_launch_ms, clocks=clk.summary(), e2e_ms=e2e_ms,
-                h2d=h2d, d2h=d2h, e2e_steps=e2e_steps, kernels=kernels)
+                h2d=h2d, d2h=d2h, e2e_steps=e2e_steps, kernels=kernels, host_ms=host_ms)
 
 
 def run_prefill_gdn(args, world, rank, dev):
@@ -408,6 +448,14 @@ def run_prefill_long(args, world, rank, dev):
     ws_n = kda.workspace_size(1, shape.T, shape.H, shape.dk, shape.dv, 1)
     ws = torch.empty(ws_n, dtype=torch.uint8, device=dev) if ws_n else None
     kernels = ["chunk_intra_kernel", "chunk_inter_kernel"] if ws_n else ["chunk_tc_kernel"]
+    # AUTO runs one sequence beyond its workspace budget in windows of launch pairs
+    windows = 1
+    full = kda.workspace_size(1, shape.T, shape.H, shape.dk, shape.dv, 1, algo="two_pass")
+    if ws_n and ws_n < full:
+        per_chunk = full // (-(-shape.T // 64) + 1)
+        carry = -(-2 * shape.H * shape.dk * shape.dv * 4 // 1024) * 1024
+        window = ((ws_n - carry) // per_chunk - 1) * 64
+        windows = -(-shape.T // window)
 
     def step():
         kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], o=o, final_state=fs,
@@ -432,7 +480,8 @@ def run_prefill_long(args, world, rank, dev):
     alg_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * shape.H * STATE_BYTES
     del d, o, fs, ws
     return dict(ms=ms, tokens=shape.T, alg_bytes=alg_bytes, alg_flops=token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD,
-                launches=reps * len(kernels), kernels=kernels, clocks=clk.summary(), reps=reps)
+                launches=reps * len(kernels) * windows, kernels=kernels, clocks=clk.summary(), reps=reps,
+                workspace_bytes=ws_n, windows=windows)
 
 
 def run_decode_varlen(args, world, rank, dev):
@@ -721,6 +770,8 @@ def main(argv=None):
                 "api": "gated_delta_rule_85_b200.chunk_forward with pinned host tensors"},
         "gpu_launches": args.steps * len(pre["kernels"]),
         "clocks": pre["clocks"],
+        # host time to enqueue one step (events + the API call); below ms_per_step the GPU never waits
+        "host_enqueue_ms_per_step": pre["host_ms"],
     }
     if dec is not None:
         step_ms = dec["ms"] / dec["launches"]
@@ -805,7 +856,8 @@ def main(argv=None):
         line["prefill_128k"] = {
             "metric": "KDA chunked prefill tokens/s (B=1, T=131072, H=32, d=128)",
             "value": world * lg["tokens"] / (lg["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": lg["ms"],
-            "steps": lg["reps"],
+            "steps": lg["reps"], "gpu_launches": lg["launches"], "workspace_bytes": lg["workspace_bytes"],
+            "windows": lg["windows"],
             "roofline": {"kernel": " + ".join(lg["kernels"]), "bound": "hbm", "achieved": lgbs, "peak": hbm_gbs,
                          "unit": "GB/s", "frac": lgbs / hbm_gbs, "traffic": None, "algorithmic_bytes": lg["alg_bytes"],
                          "tensor": {"achieved_tflops": ltf, "peak_tflops": bf16_tflops, "frac": ltf / bf16_tflops}},

@@ -24,7 +24,8 @@ import torch
 __all__ = [
     "chunk_forward", "chunk_backward", "gdn_chunk_backward", "backward_workspace_size", "chunk_forward_prologue",
     "recurrent_step_prologue", "chunk_forward_simt", "chunk_forward_static_ws", "chunk_forward_slots", "recurrent_step",
-    "recurrent_step_slots", "gdn_chunk_forward", "gdn_recurrent_step", "workspace_size", "device_status",
+    "recurrent_step_slots", "gdn_chunk_forward", "gdn_recurrent_step", "workspace_size", "set_auto_workspace_limit",
+    "device_status",
     "debug_wait_timeout", "last_error", "library_path", "load_library", "KDAError", "KDA_BF16", "KDA_F32", "CHUNK",
     "DEV_WAIT_TIMEOUT", "DEV_DECAY_RANGE", "DEV_BAD_SLOT", "ALGOS",
 ]
@@ -112,6 +113,8 @@ def load_library():
     lib.kda_debug_wait_timeout.restype = ci
     lib.kda_api_version.argtypes = []
     lib.kda_api_version.restype = ci
+    lib.kda_set_auto_workspace_limit.argtypes = [sz]
+    lib.kda_set_auto_workspace_limit.restype = sz
     _lib = lib
     return lib
 
@@ -155,6 +158,12 @@ def _algo_code(algo: str) -> int:
     return ALGOS[algo]
 
 
+def set_auto_workspace_limit(nbytes: int) -> int:
+    """AUTO's workspace budget in bytes (kda_set_auto_workspace_limit; 0 restores the
+    1 GiB default).  Returns the previous budget."""
+    return int(load_library().kda_set_auto_workspace_limit(int(nbytes)))
+
+
 def workspace_size(B, T, H, dk, dv, num_seqs, dtype=KDA_BF16, algo="auto") -> int:
     return int(load_library().kda_chunk_forward_workspace_size_ex(B, T, H, dk, dv, num_seqs, dtype, CHUNK,
                                                                   _algo_code(algo)))
@@ -190,10 +199,11 @@ def chunk_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *,
     `algo` picks the tensor-core schedule ("auto", "fused", "two_pass"); the
     workspace it needs is allocated here unless `workspace` (uint8, CUDA) is
     given.  "auto" takes the two-pass schedule for few (sequence, head) chains
-    while its workspace is at most 4 GiB (58 KB per 64-token chunk and head: 3.8 GB
-    at 131072 tokens x 32 heads); pass a reusable `workspace`
-    (workspace_size(..., algo=...)) to keep it across calls, or algo="fused" to
-    need none.  With `simt=True` the fp32 CUDA-core path (kda_chunk_forward_simt)
+    within AUTO's workspace budget (1 GiB, set_auto_workspace_limit), running a
+    single long sequence in windows that fit it (the two-pass records are 58 KB per
+    64-token chunk and head, 3.8 GB unwindowed at 131072 tokens x 32 heads); pass a
+    reusable `workspace` (workspace_size(..., algo=...)) to keep it across calls,
+    or algo="fused" to need none.  With `simt=True` the fp32 CUDA-core path (kda_chunk_forward_simt)
     runs instead.  Host (CPU) inputs are copied to the current CUDA device and
     the results copied back, all inside this call.
     Returns (o, final_state or None).

@@ -1,5 +1,7 @@
 // libkda: the C ABI declared in include/kda.h.  One translation unit holds every
 // kernel so the device status word is a single symbol per device.
+#include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -64,21 +66,80 @@ int check_prefill(const void *q, const void *k, const void *v, const float *log_
     return KDA_OK;
 }
 
-// Which tensor-core schedule runs, and the workspace it needs.
+// Which tensor-core schedule runs, the workspace it needs, and (two-pass on one
+// sequence longer than the budget allows) the window of tokens per launch pair.
 struct Plan {
     int algo;
     size_t ws;
+    long long window;   // 0: the whole input in one launch pair
 };
 
-constexpr size_t kAutoTwoPassLimit = (size_t)4 << 30;   // AUTO takes TWO_PASS only up to this workspace
-constexpr long long kAutoChainLimit = 2 * 148;          // ... and below this many (sequence, head) chains
+constexpr size_t kAutoTwoPassDefault = (size_t)1 << 30;  // AUTO's workspace budget unless set
+constexpr long long kAutoChainLimit = 2 * 148;           // AUTO takes TWO_PASS below this many chains
+static std::atomic<size_t> g_auto_ws_limit{kAutoTwoPassDefault};
 
-Plan plan_prefill(long long tokens, int H, int dk, int num_seqs, int algo) {
+// The state carried between windows: two fp32 [H][dk][dv] buffers at the
+// workspace's start (window w reads one and writes the other).
+size_t window_carry_bytes(int H, int dk, int dv) {
+    return ((size_t)2 * H * dk * dv * sizeof(float) + 1023) / 1024 * 1024;
+}
+
+// Longest window (a multiple of the chunk) whose records and carry fit in `limit`; 0 if none.
+long long window_tokens(int H, int dk, int dv, size_t limit) {
+    const size_t carry = window_carry_bytes(H, dk, dv);
+    const size_t per_chunk = kda::tc::two_pass_workspace_bytes(1, H, dk, 0);   // records of one chunk slot
+    if (limit <= carry + per_chunk) return 0;
+    const long long chunks = (long long)((limit - carry) / per_chunk) - 1;     // one slot of slack per sequence
+    return chunks > 0 ? chunks * kda::tc::C : 0;
+}
+
+Plan plan_prefill(int B, long long tokens, int H, int dk, int dv, int num_seqs, int algo) {
     const size_t ws2 = kda::tc::two_pass_workspace_bytes(tokens, H, dk, num_seqs);
-    if (algo == KDA_ALGO_AUTO)
-        algo = ((long long)num_seqs * H < kAutoChainLimit && ws2 <= kAutoTwoPassLimit) ? KDA_ALGO_TWO_PASS
-                                                                                       : KDA_ALGO_FUSED;
-    return Plan{algo, algo == KDA_ALGO_TWO_PASS ? ws2 : 0};
+    if (algo == KDA_ALGO_AUTO) {
+        const size_t limit = g_auto_ws_limit.load(std::memory_order_relaxed);
+        algo = KDA_ALGO_FUSED;
+        if ((long long)num_seqs * H < kAutoChainLimit) {
+            if (ws2 <= limit) {
+                algo = KDA_ALGO_TWO_PASS;
+            } else if (B == 1 && num_seqs == 1) {
+                const long long w = window_tokens(H, dk, dv, limit);
+                if (w > 0)
+                    return Plan{KDA_ALGO_TWO_PASS,
+                                window_carry_bytes(H, dk, dv) + kda::tc::two_pass_workspace_bytes(w, H, dk, 1), w};
+            }
+        }
+    }
+    return Plan{algo, algo == KDA_ALGO_TWO_PASS ? ws2 : 0, 0};
+}
+
+// One sequence (B = 1, no cu_seqlens) through the two-pass schedule in windows of
+// `window` tokens: each window is a first-pass/second-pass launch pair on its own
+// slice of the inputs and outputs, reusing the records' space; the state passes
+// from one window to the next in fp32 through the carry buffers, so the result is
+// the one-pair result.
+int two_pass_windows(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                     const float *init_state, void *o, float *final_state, int T, int H, int dk, int dv,
+                     long long window, bool gate_scalar, void *workspace, cudaStream_t st, char *msg,
+                     size_t msg_len) {
+    float *carry = (float *)workspace;
+    const size_t state_elems = (size_t)H * dk * dv;
+    void *rec = (uint8_t *)workspace + window_carry_bytes(H, dk, dv);
+    const size_t gate_elems = gate_scalar ? 1 : (size_t)dk;   // log_alpha values per (token, head)
+    int w = 0;
+    for (long long t0 = 0; t0 < T; t0 += window, ++w) {
+        const int tw = (int)std::min(window, (long long)T - t0);
+        const bool last = t0 + tw >= T;
+        const size_t th = (size_t)t0 * H;
+        const float *s_in = w == 0 ? init_state : carry + (size_t)((w - 1) & 1) * state_elems;
+        float *s_out = last ? final_state : carry + (size_t)(w & 1) * state_elems;
+        const int rc = kda::tc::launch_two_pass(
+            (const __nv_bfloat16 *)q + th * dk, (const __nv_bfloat16 *)k + th * dk,
+            (const __nv_bfloat16 *)v + th * dv, log_alpha + th * gate_elems, beta + th, s_in,
+            (__nv_bfloat16 *)o + th * dv, s_out, nullptr, tw, tw, H, dk, dv, 1, nullptr, 0, gate_scalar, rec, st,
+            msg, msg_len);
+        if (rc) return rc;
+    }
+    return KDA_OK;
 }
 
 // Scratch of kda_chunk_forward_static_ws: file scope, reserved on each device
@@ -216,7 +277,9 @@ int prefill_impl(const void *q, const void *k, const void *v, const float *log_a
                  int H, int dk, int dv, int num_seqs, int algo, const int32_t *slots, int num_slots,
                  bool gate_scalar, void *workspace, size_t ws_bytes, cudaStream_t st) {
     const long long tokens = (long long)B * T;
-    const Plan plan = plan_prefill(tokens, H, dk, num_seqs, algo);
+    Plan plan = plan_prefill(B, tokens, H, dk, dv, num_seqs, algo);
+    // windows slice one plain sequence; with cu_seqlens or state slots AUTO takes the fused schedule
+    if (plan.window && (cu_seqlens || slots)) plan = Plan{KDA_ALGO_FUSED, 0, 0};
     if (plan.ws && (!workspace || ws_bytes < plan.ws))
         return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", plan.ws, ws_bytes);
     if (workspace && !aligned(workspace, 256)) return fail(KDA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
@@ -228,6 +291,9 @@ int prefill_impl(const void *q, const void *k, const void *v, const float *log_a
     if (tokens == 0)
         rc = slots ? KDA_OK   // states stay in their slots
                    : kda::tc::state_passthrough(init_state, final_state, num_seqs, H, dk, dv, st, msg, sizeof(msg));
+    else if (plan.window)
+        rc = two_pass_windows(q, k, v, log_alpha, beta, init_state, o, final_state, T, H, dk, dv, plan.window,
+                              gate_scalar, workspace, st, msg, sizeof(msg));
     else if (plan.algo == KDA_ALGO_TWO_PASS)
         rc = kda::tc::launch_two_pass(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, tokens, T,
                                       H, dk, dv, num_seqs, slots, num_slots, gate_scalar, workspace, st, msg,
@@ -438,7 +504,11 @@ size_t kda_chunk_forward_workspace_size_ex(int B, int T, int H, int dk, int dv, 
                                            int chunk, int algo) {
     (void)dv; (void)chunk;
     if (dtype != KDA_BF16 || B < 1 || T < 0 || H < 1 || num_seqs < 0 || (dk != 64 && dk != 128)) return 0;
-    return plan_prefill((long long)B * T, H, dk, num_seqs, algo).ws;
+    return plan_prefill(B, (long long)B * T, H, dk, dv, num_seqs, algo).ws;
+}
+
+size_t kda_set_auto_workspace_limit(size_t bytes) {
+    return g_auto_ws_limit.exchange(bytes ? bytes : kAutoTwoPassDefault);
 }
 
 size_t kda_chunk_forward_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype,
@@ -512,7 +582,7 @@ int kda_chunk_forward_static_ws(const void *q, const void *k, const void *v, con
     if (dtype == KDA_F32)
         return kda_chunk_forward_simt(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B,
                                       T, H, dk, dv, num_seqs, dtype, chunk, stream);
-    const size_t need = plan_prefill((long long)B * T, H, dk, num_seqs, KDA_ALGO_TWO_PASS).ws;
+    const size_t need = plan_prefill(B, (long long)B * T, H, dk, dv, num_seqs, KDA_ALGO_TWO_PASS).ws;
     // Too large for the built-in scratch: the fused schedule, which needs no scratch at all.
     if (need > KDA_STATIC_WS_BYTES)
         return kda_chunk_forward_ex(q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, B, T, H, dk,

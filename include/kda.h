@@ -135,12 +135,28 @@ int kda_chunk_forward(const void *q, const void *k, const void *v, const float *
  *                      dk = 128, 33 KB at dk = 64); a second kernel walks the
  *                      chunks with only the state-dependent products left.
  *                      Best when there are few chains.
- *   KDA_ALGO_AUTO      TWO_PASS when num_seqs * H < 296 and its workspace is at
- *                      most 4 GiB, else FUSED.  kda_chunk_forward uses AUTO.
+ *   KDA_ALGO_AUTO      TWO_PASS when num_seqs * H < 296 and its workspace fits
+ *                      AUTO's budget (1 GiB unless kda_set_auto_workspace_limit
+ *                      says otherwise).  A single sequence (B = 1, num_seqs = 1)
+ *                      whose workspace would not fit runs TWO_PASS in windows:
+ *                      consecutive slices of the tokens, each one launch pair
+ *                      on the same records, the state handed from one window to
+ *                      the next in fp32 (the result is the one-pair result), so
+ *                      its workspace stays within the budget at any length.
+ *                      Everything else runs FUSED.  A windowed plan called with
+ *                      cu_seqlens or state slots runs FUSED instead.
+ *                      kda_chunk_forward uses AUTO.
  */
 #define KDA_ALGO_AUTO 0
 #define KDA_ALGO_FUSED 1
 #define KDA_ALGO_TWO_PASS 2
+
+/* Sets AUTO's workspace budget in bytes (0 restores the default of 1 GiB) and
+ * returns the previous one.  Process-wide; the workspace size a call needs is the
+ * one kda_chunk_forward_workspace_size_ex reports under the budget in force at
+ * that call, so change it between calls, not between a size query and its call
+ * (a smaller workspace than the plan needs is KDA_ERR_WORKSPACE). */
+size_t kda_set_auto_workspace_limit(size_t bytes);
 
 /* Workspace bytes kda_chunk_forward_ex needs for these sizes and `algo` (0 when none). */
 size_t kda_chunk_forward_workspace_size_ex(int B, int T, int H, int dk, int dv, int num_seqs,

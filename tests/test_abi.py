@@ -120,11 +120,48 @@ def test_workspace_sizes(lib):
     assert f(1, 8192, 32, 128, 128, 1, 0, 64, FUSED) == 0
     assert f(1, 8192, 32, 128, 128, 1, 0, 64, AUTO) == two_pass_ws(128 + 1, 32, REC128)     # 32 chains: two-pass
     assert f(1, 1 << 20, 32, 128, 128, 22, 0, 64, AUTO) == 0                         # 704 chains: fused
-    assert f(1, 1 << 20, 8, 128, 128, 1, 0, 64, AUTO) == 0                           # > 4 GiB: fused
+    assert f(2, 1 << 19, 8, 128, 128, 2, 0, 64, AUTO) == 0      # two sequences over AUTO's 1 GiB: fused
     assert f(3, 100, 2, 64, 64, 3, 0, 64, TWO_PASS) == two_pass_ws(5 + 3, 2, REC64)
     assert f(1, 100, 2, 64, 64, 1, 1, 64, TWO_PASS) == 0                             # fp32 path
     assert f(2, 0, 2, 128, 128, 2, 0, 64, TWO_PASS) == 0                             # no tokens
     assert lib.kda_chunk_forward_workspace_size(1, 8192, 32, 128, 128, 1, 0, 64) == two_pass_ws(128 + 1, 32, REC128)
+
+
+def windowed_ws(H, dk, dv, rec, limit):
+    """AUTO's windowed two-pass workspace: two fp32 [H][dk][dv] carry states (rounded
+    up to 1 KiB) and the records of the longest window that fits `limit`, plus the
+    one slack slot a sequence has."""
+    carry = -(-2 * H * dk * dv * 4 // 1024) * 1024
+    chunks = (limit - carry) // (H * rec) - 1
+    return carry + (chunks + 1) * H * rec
+
+
+def test_auto_workspace_budget(lib):
+    f = lib.kda_chunk_forward_workspace_size_ex
+    TWO_PASS, AUTO = 2, 0
+    GiB = 1 << 30
+    assert lib.kda_set_auto_workspace_limit(0) == GiB        # the default, left in place
+    # prefill_128k: 2049 slots x 32 heads x 58368 B = 3.8 GB unwindowed, <= 1 GiB windowed
+    assert f(1, 131072, 32, 128, 128, 1, 0, 64, TWO_PASS) == two_pass_ws(2048 + 1, 32, REC128)
+    w = f(1, 131072, 32, 128, 128, 1, 0, 64, AUTO)
+    assert w == windowed_ws(32, 128, 128, REC128, GiB)
+    assert GiB - 32 * REC128 < w <= GiB
+    assert f(1, 1 << 20, 8, 128, 128, 1, 0, 64, AUTO) == windowed_ws(8, 128, 128, REC128, GiB)
+    # a smaller budget: small inputs go windowed too; multi-sequence inputs go fused
+    limit = 2 << 20   # windows of 320 tokens at H=4, dk=dv=128; 832 at dk=dv=64
+    try:
+        assert lib.kda_set_auto_workspace_limit(limit) == GiB
+        assert f(1, 1000, 4, 128, 128, 1, 0, 64, AUTO) == windowed_ws(4, 128, 128, REC128, limit)
+        assert f(1, 1000, 4, 64, 64, 1, 0, 64, AUTO) == windowed_ws(4, 64, 64, REC64, limit)
+        assert f(1, 100, 4, 128, 128, 1, 0, 64, AUTO) == two_pass_ws(2 + 1, 4, REC128)   # fits: one pair
+        assert f(2, 1000, 4, 128, 128, 2, 0, 64, AUTO) == 0
+        assert f(1, 1000, 4, 128, 128, 1, 0, 64, TWO_PASS) == two_pass_ws(16 + 1, 4, REC128)
+        # a budget below one window's carry and record: fused
+        lib.kda_set_auto_workspace_limit(4096)
+        assert f(1, 1000, 4, 128, 128, 1, 0, 64, AUTO) == 0
+    finally:
+        lib.kda_set_auto_workspace_limit(0)
+    assert lib.kda_set_auto_workspace_limit(0) == GiB
 
 
 def prefill_ex(lib, algo, ws, wsb):

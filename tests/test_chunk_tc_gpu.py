@@ -120,3 +120,65 @@ def test_scalar_gate_gated_deltanet_regime(algo):
     o_ref, S_ref = oracle_prefill(d)
     assert_close(to_f64(o), o_ref, BF16, "o")
     assert_close(to_f64(S), S_ref, BF16, "final state")
+
+
+@pytest.fixture
+def small_auto_budget():
+    """AUTO's workspace budget at 2 MiB: one sequence at H=4 runs the two-pass
+    schedule in windows of 320 tokens (dk=dv=128) or 832 tokens (dk=dv=64)."""
+    prev = kda.set_auto_workspace_limit(2 << 20)
+    yield
+    kda.set_auto_workspace_limit(prev)
+
+
+@pytest.mark.parametrize("T,dk,dv", [(1000, 128, 128), (640, 128, 128), (1000, 64, 64), (2000, 64, 128)])
+def test_auto_windows_match_oracle_and_one_launch_pair(T, dk, dv, small_auto_budget):
+    """Windows of the two-pass schedule (ragged last window, exact multiple, two
+    head sizes): the state handed on in fp32 between windows gives the oracle's
+    result and the one-pair result."""
+    H = 4
+    assert kda.workspace_size(1, T, H, dk, dv, 1, algo="auto") < kda.workspace_size(1, T, H, dk, dv, 1,
+                                                                                      algo="two_pass")
+    shape = PrefillShape(B=1, T=T, H=H, dk=dk, dv=dv, dtype=BF16)
+    d, o, S = _run(shape, seed=31 + T + dk, algo="auto")
+    o_ref, S_ref = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+    assert_close(to_f64(S), S_ref, BF16, "final state")
+    o2, S2 = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"],
+                               algo="two_pass")
+    torch.cuda.synchronize()
+    assert rel_l2(to_f64(o), to_f64(o2)) < 1e-3
+    assert rel_l2(to_f64(S), to_f64(S2)) < 1e-3
+
+
+def test_auto_windows_zero_start_no_final_state(small_auto_budget):
+    shape = PrefillShape(B=1, T=777, H=4, dk=128, dv=128, dtype=BF16, init_state="none")
+    d, o, S = _run(shape, seed=41, final_state=False)
+    assert S is None
+    o_ref, _ = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+
+
+def test_auto_windows_scalar_gate(small_auto_budget):
+    """kda_gdn_chunk_forward through the windows: the [T, H] gate is sliced per window."""
+    shape = PrefillShape(B=1, T=900, H=4, dk=128, dv=128, dtype=BF16, gate="scalar")
+    d = prefill_inputs(shape, 43, torch.device("cuda"))
+    o, S = kda.gdn_chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"])
+    torch.cuda.synchronize()
+    assert kda.device_status() == 0
+    full = dict(d, log_alpha=d["log_alpha"].unsqueeze(-1).expand(*d["q"].shape).contiguous())
+    o_ref, S_ref = oracle_prefill(full)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+    assert_close(to_f64(S), S_ref, BF16, "final state")
+
+
+def test_auto_windowed_plan_with_cu_seqlens_runs_fused(small_auto_budget):
+    """A single packed sequence (cu_seqlens) cannot be sliced on the host: the
+    windowed plan runs the fused schedule, with no workspace."""
+    shape = PrefillShape(B=1, T=1000, H=4, dk=128, dv=128, dtype=BF16, cu_seqlens=(0, 1000))
+    d = prefill_inputs(shape, 44, torch.device("cuda"))
+    o, S = kda.chunk_forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["init_state"], d["cu_seqlens"])
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle_prefill(d)
+    assert_close(to_f64(o), o_ref, BF16, "o")
+    assert_close(to_f64(S), S_ref, BF16, "final state")
