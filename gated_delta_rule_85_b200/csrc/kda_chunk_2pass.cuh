@@ -729,15 +729,6 @@ constexpr int inter_nbuf() {
 constexpr uint32_t INTER_TMEM_COLS = 256;
 constexpr uint32_t XCOL_XY = 0;       // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O
 constexpr uint32_t XCOL_DS = 128;     // [128 x DVT] Kt Z (lanes 0..dk-1)
-// With output, [X; Y] alternates by chunk parity between two buffers XY_STRIDE apart and
-// Kt Z follows them: 256 columns up to 64-column value tiles (two CTAs of a small layout
-// can share an SM's 512), 512 for 128-column tiles (one CTA per SM by shared memory).
-template <int DVT, bool CK>
-struct InterCols {
-    static constexpr uint32_t XY_STRIDE = CK ? 0u : (DVT <= 64 ? 64u : 128u);
-    static constexpr uint32_t DS = CK ? XCOL_DS : 2 * XY_STRIDE;
-    static constexpr uint32_t ALLOC = (CK || DVT <= 64) ? INTER_TMEM_COLS : 512u;
-};
 
 // CK (the backward's state sweep, dv = 128): ws (and ckpt, the same bytes, writable)
 // hold [slot][H] BwdUnit; no output; instead the state at each chunk's start, bf16,
@@ -757,20 +748,11 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
     constexpr uint32_t REC_TX = CK ? (uint32_t)(DK / 64 * 64 * 128 + DK * 128 + DK * 4) : (uint32_t)R::BYTES;
     constexpr uint32_t TX = REC_TX + (uint32_t)(C * DVT * 2);
     constexpr size_t USTRIDE = CK ? (size_t)BwdUnit<DK>::BYTES : (size_t)R::BYTES;   // bytes per (slot, head)
-    // With output, the Pt Z product (rows DK-64 .. DK+63 of [Kt; Pt]) and the readout of O
-    // run off the serial path: O of chunk c leaves TMEM while chunk c+1's first product
-    // runs, so [X; Y] alternates between two TMEM buffers and the record bytes that
-    // product reads (LATE) are reloaded only once it has completed (bar_o).
-    using TC = InterCols<DVT, CK>;
-    constexpr uint32_t TCOLS = TC::ALLOC, COL_DS = TC::DS;
-    static_assert(TC::DS + DVT <= TC::ALLOC, "TMEM columns");
-    constexpr uint32_t LATE = (uint32_t)(R::KP + (DK - 64) * 128), LATE_BYTES = 128 * 128;
-    static_assert(LATE % 16 == 0 && LATE + LATE_BYTES == (uint32_t)R::DCH, "record layout");
     using MN = MnOp<DVT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = ptx::smem_u32(sm);
-    const uint32_t bar_rec = sb + L::MISC, bar_mma = sb + L::MISC + 32, bar_o = sb + L::MISC + 48;
+    const uint32_t bar_rec = sb + L::MISC, bar_mma = sb + L::MISC + 32;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 40);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -784,13 +766,12 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
     const long long first = n + t0 / C;   // slot of chunk 0
 
     if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TCOLS);
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTER_TMEM_COLS);
         ptx::tmem_relinquish();
     }
     if (tid == 0) {
         for (int b = 0; b < NBUF; ++b) ptx::mbar_init(bar_rec + 8 * b, 1);
         ptx::mbar_init(bar_mma, 1);
-        ptx::mbar_init(bar_o, 1);
         ptx::fence_mbar_init();
         if (nck > 0) ptx::prefetch_tmap(tm_v);
     }
@@ -801,11 +782,8 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     uint32_t ph_mma = 0, ph_rec = 0;   // ph_rec: one parity bit per buffer
     int n_issued = 0, n_commit = 0;    // thread 0: chunks whose copies were issued, MMA commits
-    int n_late = 0, n_commit_o = 0;    // thread 0: chunks whose LATE bytes were issued, bar_o commits
 
-    // thread 0: record and V tile of chunk ci into buffer ci % NBUF (with output, all but the
-    // LATE bytes unless `late`; the barrier expects them all, so its phase waits for issue_late)
-    auto issue = [&](int ci, bool late) {
+    auto issue = [&](int ci) {   // thread 0: record and V tile of chunk ci into buffer ci % NBUF
         const int b = ci % NBUF;
         n_issued = ci + 1;
         const uint32_t bar = bar_rec + 8 * b;
@@ -818,47 +796,14 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
             ptx::bulk_load(sb + b * R::BYTES + R::KP, src + R::KP, DK * 128, bar);
             ptx::bulk_load(sb + b * R::BYTES + R::DCH, src + R::DCH, DK * 4, bar);
         } else {
-            ptx::bulk_load(sb + b * R::BYTES, src, LATE, bar);
-            ptx::bulk_load(sb + b * R::BYTES + R::DCH, src + R::DCH, (uint32_t)(R::BYTES - R::DCH), bar);
+            ptx::bulk_load(sb + b * R::BYTES, src, (uint32_t)R::BYTES, bar);
         }
         ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, tm_v, bar, col_base, h, (int)(t0 + (long long)ci * C));
-        if (!CK && late) {
-            ptx::bulk_load(sb + b * R::BYTES + LATE, src + LATE, LATE_BYTES, bar);
-            n_late = ci + 1;
-        }
-    };
-    auto issue_late = [&](int ci) {   // thread 0, after the Pt Z product of chunk ci - NBUF completed
-        const uint8_t *src = ws + ((size_t)(first + ci) * H + h) * USTRIDE;
-        ptx::bulk_load(sb + (ci % NBUF) * R::BYTES + LATE, src + LATE, LATE_BYTES, bar_rec + 8 * (ci % NBUF));
-        n_late = ci + 1;
     };
 
     const int srow = quad * 32 + lane;
     const bool has_row = srow < DK;
     const int scol = half * CPT;
-    // quads 2-3 (TMEM lanes 64-127): O rows of chunk c -> o, once its Pt Z product has landed
-    auto store_o = [&](int c) -> bool {
-        const bool got = ptx::mbar_wait_bounded(bar_o, (uint32_t)(c & 1), WAIT_LIMIT_CYCLES);
-        ptx::tc_fence_after();
-        const long long cs = t0 + (long long)c * C;
-        const int Lc = (int)min((long long)C, t1 - cs);
-        const int i = (quad - 2) * 32 + lane;
-#pragma unroll 1
-        for (int cc = 0; cc < CPT / 16; ++cc) {
-            float o16[16];
-            ptx::tmem_ld16(tl + XCOL_XY + (uint32_t)(c & 1) * TC::XY_STRIDE + scol + cc * 16, o16);
-            ptx::tmem_wait_ld();
-            if (got && i < Lc) {
-                __nv_bfloat16 *dst = o + ((cs + i) * H + h) * DV + col_base + scol + cc * 16;
-                reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pack_bf16(o16[0], o16[1]), pack_bf16(o16[2], o16[3]),
-                                                               pack_bf16(o16[4], o16[5]), pack_bf16(o16[6], o16[7]));
-                reinterpret_cast<uint4 *>(dst)[1] =
-                    make_uint4(pack_bf16(o16[8], o16[9]), pack_bf16(o16[10], o16[11]), pack_bf16(o16[12], o16[13]),
-                               pack_bf16(o16[14], o16[15]));
-            }
-        }
-        return got;
-    };
     const int row = state_row(slots, num_slots, n);
     const long long st_off = ((long long)(row < 0 ? 0 : row) * H + h) * DK * DV + col_base + scol;
     float S[CPT];
@@ -869,7 +814,7 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
         S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
     }
     if (tid == 0)
-        for (int ci = 0; ci < NBUF && ci < nck; ++ci) issue(ci, true);
+        for (int ci = 0; ci < NBUF && ci < nck; ++ci) issue(ci);
 
     bool ok = true;
     for (int ci = 0; ci < nck; ++ci) {
@@ -898,28 +843,17 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 2. [X; Y] = [e^G K; e^G Q] S ; meanwhile O of the previous chunk -> o
-        const uint32_t xy = XCOL_XY + (uint32_t)(ci & 1) * TC::XY_STRIDE;
+        // ---- 2. [X; Y] = [e^G K; e^G Q] S
         if (tid == 0) {
             ptx::tc_fence_after();
             constexpr uint32_t ix = ptx::idesc_bf16_f32(128, DVT, false, true);
 #pragma unroll
             for (int s = 0; s < DK / 16; ++s)
-                ptx::mma_bf16(tmem + xy, kdesc(rb + R::KQ, s, 128), MN::desc(sb + L::SP, s, DK), ix, s > 0);
+                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KQ, s, 128), MN::desc(sb + L::SP, s, DK), ix, s > 0);
             ptx::mma_commit(bar_mma);
             ++n_commit;
         }
-        int o_fail = 0;
-        if constexpr (!CK) {
-            if (ci > 0) {
-                if (quad >= 2) o_fail = !store_o(ci - 1);
-                if (tid == 0 && ci - 1 + NBUF < nck) {   // the Pt Z product of chunk ci-1 read its LATE bytes
-                    o_fail |= !ptx::mbar_wait_bounded(bar_o, (uint32_t)((ci - 1) & 1), WAIT_LIMIT_CYCLES);
-                    if (!o_fail) issue_late(ci - 1 + NBUF);
-                }
-            }
-        }
-        if (!(ok = wait_all(bar_mma, ph_mma, o_fail))) break;
+        if (!(ok = wait_all(bar_mma, ph_mma))) break;
 
         // ---- 3. Z = V - X (X in TMEM lanes 0-63) -> Z^T
         if (quad < 2) {
@@ -928,7 +862,7 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
 #pragma unroll 1
             for (int cc = 0; cc < CPT / 16; ++cc) {
                 float x16[16], v16[16];
-                ptx::tmem_ld16(tl + xy + scol + cc * 16, x16);
+                ptx::tmem_ld16(tl + XCOL_XY + scol + cc * 16, x16);
                 if (j < Lc) {
                     unpack_bf16x8(*reinterpret_cast<const uint4 *>(vin + (j * DVT + scol + cc * 16) * 2), v16);
                     unpack_bf16x8(*reinterpret_cast<const uint4 *>(vin + (j * DVT + scol + cc * 16 + 8) * 2), v16 + 8);
@@ -950,60 +884,62 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
         ptx::tc_fence_before();
         __syncthreads();
 
-        // ---- 4. dS = Kt Z (bar_mma) ; O = Y + Pt Z onto the Y rows of [X; Y] (bar_o)
+        // ---- 4. dS = Kt Z ; O = Y + Pt Z (onto the Y rows of [X; Y])
         if (tid == 0) {
             ptx::tc_fence_after();
             constexpr uint32_t iz = ptx::idesc_bf16_f32(128, DVT, false, true);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + COL_DS, kdesc(rb + R::KP, s, DK + 64), MN::desc(sb + L::ZT, s, C), iz, s > 0);
-            ptx::mma_commit(bar_mma);
-            ++n_commit;
+                ptx::mma_bf16(tmem + XCOL_DS, kdesc(rb + R::KP, s, DK + 64), MN::desc(sb + L::ZT, s, C), iz, s > 0);
             if constexpr (!CK) {
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    ptx::mma_bf16(tmem + xy, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C), iz, 1);
-                ptx::mma_commit(bar_o);
-                ++n_commit_o;
+                    ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C),
+                                  iz, 1);
             }
+            ptx::mma_commit(bar_mma);
+            ++n_commit;
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
-        // buffer b: consumed but for the LATE bytes the Pt Z product still reads
-        if (tid == 0 && ci + NBUF < nck) issue(ci + NBUF, CK);
+        if (tid == 0 && ci + NBUF < nck) issue(ci + NBUF);   // buffer b fully consumed
 
         // ---- 5. S <- Diag(e^{G_last}) S + dS ; O rows (TMEM lanes 64-127) -> o
         if (has_row) {
 #pragma unroll
             for (int cc = 0; cc < CPT / 16; ++cc) {
                 float d16[16];
-                ptx::tmem_ld16(tl + COL_DS + scol + cc * 16, d16);
+                ptx::tmem_ld16(tl + XCOL_DS + scol + cc * 16, d16);
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
             }
         }
-        ptx::tc_fence_before();
-    }
-    if constexpr (!CK) {   // O of the last chunk
-        int o_fail = 0;
-        if (ok && nck > 0 && quad >= 2) o_fail = !store_o(nck - 1);
-        if (__syncthreads_or(o_fail)) {
-            if (tid == 0) flag_status(KDA_DEV_WAIT_TIMEOUT);
-            ok = false;
+        if (!CK && quad >= 2) {
+            const int i = (quad - 2) * 32 + lane;
+#pragma unroll 1
+            for (int cc = 0; cc < CPT / 16; ++cc) {
+                float o16[16];
+                ptx::tmem_ld16(tl + XCOL_XY + scol + cc * 16, o16);
+                ptx::tmem_wait_ld();
+                if (i < Lc) {
+                    __nv_bfloat16 *dst = o + ((cs + i) * H + h) * DV + col_base + scol + cc * 16;
+                    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pack_bf16(o16[0], o16[1]), pack_bf16(o16[2], o16[3]),
+                                                                   pack_bf16(o16[4], o16[5]), pack_bf16(o16[6], o16[7]));
+                    reinterpret_cast<uint4 *>(dst)[1] =
+                        make_uint4(pack_bf16(o16[8], o16[9]), pack_bf16(o16[10], o16[11]),
+                                   pack_bf16(o16[12], o16[13]), pack_bf16(o16[14], o16[15]));
+                }
+            }
         }
+        ptx::tc_fence_before();
     }
 
     if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded), then leave
-        if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
-        if (n_commit_o > 0) ptx::mbar_wait_bounded(bar_o, (uint32_t)((n_commit_o - 1) & 1), WAIT_LIMIT_CYCLES);
-        // a chunk whose LATE bytes were held back: no product reads its buffer any more, so
-        // issue them, letting that buffer's barrier phase complete
-        if constexpr (!CK)
-            for (int c = n_late; c < n_issued; ++c) issue_late(c);
         for (int b = 0; b < NBUF; ++b) {
             const int arms = n_issued > b ? (n_issued - 1 - b) / NBUF + 1 : 0;   // loads into buffer b
             if (arms > 0) ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((arms - 1) & 1), WAIT_LIMIT_CYCLES);
         }
+        if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
     }
     __syncthreads();
     if (ok && final_state && has_row && row >= 0) {
@@ -1015,7 +951,7 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
     __syncthreads();
     if (warp == 0) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, TCOLS);
+        ptx::tmem_dealloc(tmem, INTER_TMEM_COLS);
     }
 }
 
