@@ -719,13 +719,6 @@ struct InterLayout {
     static_assert(REC % 1024 == 0 && SP % 1024 == 0 && ZT % 1024 == 0 && VIN % 128 == 0, "tile alignment");
 };
 
-// Two record buffers: one chunk of lead hides the record load, and the smaller
-// footprint measured faster than three buffers (0.210 vs 0.220 ms at prefill_8k).
-template <int DK, int DVT>
-constexpr int inter_nbuf() {
-    return 2;
-}
-
 constexpr uint32_t INTER_TMEM_COLS = 256;
 constexpr uint32_t XCOL_XY = 0;       // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O
 constexpr uint32_t XCOL_DS = 128;     // [128 x DVT] Kt Z (lanes 0..dk-1)
@@ -955,14 +948,316 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
     }
 }
 
-template <int DK, int DVT, int NBUF, bool CK = false>
-__global__ void __launch_bounds__(NT, 1)
+// ---- pass 2 with output: warp-specialised
+//
+// Eight compute warps and one issue warp.  Lane 0 of the issue warp loads the
+// records and V tiles and issues every tcgen05.mma (each issue holds its thread
+// for tens of cycles); the compute warps never wait on an issuing thread, only on
+// the products they consume.  Per chunk c (buffer b = c % NBUF):
+//
+//   compute (all)      wait record b; e^{G_last} -> register; quads 2-3 then release b
+//   issue              wait record b and S_c in bf16 (bar_s) -> [X; Y] = [K^; Q^] S_c
+//                      into XY[c & 1], commit bar_x
+//   compute (quads 0-1) wait bar_x -> Z = V - X in bf16 -> bar_z, release b
+//   compute (quads 2-3) wait bar_o[(c-1) & 1] -> O of chunk c-1 -> o
+//   issue              wait bar_z -> dS = Kt Z (commit bar_ds), O = Y + Pt Z onto
+//                      XY[c & 1] (commit bar_o[c & 1]); then, once chunk c-1's
+//                      buffer is released and its products are done, load chunk
+//                      c-1+NBUF into it
+//   compute (all)      wait bar_ds -> S <- Diag(e^{G_last}) S + dS -> S_{c+1} in bf16 -> bar_s
+//
+// so the serial path per chunk is the two dependent products and the two
+// elementwise steps between them; the output product, the readout of O and the
+// record loads overlap it.  Every wait is bounded: a thread whose wait runs out
+// flags the device status and leaves its loop; the others then run out in turn.
+
+constexpr int NT_WS = NT + 32;   // 8 compute warps + the issue warp
+
+template <int DK, int DVT, int NBUF>
+struct InterWsLayout {
+    using B = InterLayout<DK, DVT, NBUF>;
+    static constexpr int SP = B::SP, ZT = B::ZT, VIN = B::VIN, MISC = B::MISC;
+    // MISC: bar_rec[NBUF], bar_free[NBUF], bar_s, bar_x, bar_z, bar_ds, bar_o[2], TMEM base
+    static constexpr int BAR_REC = MISC, BAR_FREE = MISC + 32, BAR_S = MISC + 64, BAR_X = MISC + 72,
+                         BAR_Z = MISC + 80, BAR_DS = MISC + 88, BAR_O = MISC + 96, TSLOT = MISC + 112;
+    static constexpr int BYTES = MISC + 128;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(NBUF <= 4, "barrier slots");
+};
+
+// Three record buffers (two chunks of lead for each load) where they fit.
+template <int DK, int DVT>
+constexpr int inter_ws_nbuf() {
+    return InterWsLayout<DK, DVT, 3>::ALLOC <= 232448 ? 3 : 2;
+}
+
+// TMEM: [X; Y] alternates by chunk parity between two buffers XY_STRIDE apart; Kt Z
+// follows them.  256 columns up to 64-column value tiles, 512 for 128-column tiles.
+template <int DVT>
+struct InterWsCols {
+    static constexpr uint32_t XY_STRIDE = DVT <= 64 ? 64u : 128u;
+    static constexpr uint32_t DS = 2 * XY_STRIDE;
+    static constexpr uint32_t ALLOC = DVT <= 64 ? 256u : 512u;
+    static_assert(DS + DVT <= ALLOC, "TMEM columns");
+};
+
+template <int DK, int DVT, int NBUF>
+__device__ __forceinline__ void inter_ws_body(int tile, const CUtensorMap *tm_v, const uint8_t *__restrict__ ws,
+                                              const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
+                                              float *__restrict__ final_state,
+                                              const int32_t *__restrict__ cu_seqlens, int T, int H, int DV,
+                                              const int32_t *__restrict__ slots, int num_slots) {
+    using L = InterWsLayout<DK, DVT, NBUF>;
+    using R = Rec<DK>;
+    using TC = InterWsCols<DVT>;
+    using MN = MnOp<DVT>;
+    static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
+    constexpr int CPT = DVT / 2;
+    constexpr uint32_t TX = (uint32_t)R::BYTES + (uint32_t)(C * DVT * 2);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = ptx::smem_u32(sm);
+    const uint32_t bar_rec = sb + L::BAR_REC, bar_free = sb + L::BAR_FREE, bar_s = sb + L::BAR_S,
+                   bar_x = sb + L::BAR_X, bar_z = sb + L::BAR_Z, bar_ds = sb + L::BAR_DS, bar_o = sb + L::BAR_O;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::TSLOT);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = (warp >> 2) & 1;
+    const int col_base = tile * DVT, h = blockIdx.y;
+    const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
+
+    long long t0, t1;
+    seq_span(cu_seqlens, T, n, t0, t1);
+    const int nck = (int)((t1 - t0 + C - 1) / C);
+    const long long first = n + t0 / C;   // slot of chunk 0
+
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TC::ALLOC);
+        ptx::tmem_relinquish();
+    }
+    if (tid == NT) {
+        for (int b = 0; b < NBUF; ++b) {
+            ptx::mbar_init(bar_rec + 8 * b, 1);
+            ptx::mbar_init(bar_free + 8 * b, NT / 32);   // one arrival per compute warp
+        }
+        ptx::mbar_init(bar_s, NT / 32);
+        ptx::mbar_init(bar_x, 1);
+        ptx::mbar_init(bar_z, 4);                         // the four warps of quads 0-1
+        ptx::mbar_init(bar_ds, 1);
+        ptx::mbar_init(bar_o, 1);
+        ptx::mbar_init(bar_o + 8, 1);
+        ptx::fence_mbar_init();
+        if (nck > 0) ptx::prefetch_tmap(tm_v);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+
+    if (warp == NT / 32) {
+        // ---------------- issue warp (lane 0)
+        if (lane == 0) {
+            int n_issued = 0, n_mma = 0;   // chunks whose loads were issued; chunks with all products issued
+            auto issue = [&](int ci) {     // record and V tile of chunk ci into buffer ci % NBUF
+                const int b = ci % NBUF;
+                const uint32_t bar = bar_rec + 8 * b;
+                ptx::mbar_arrive_expect_tx(bar, TX);
+                ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * R::BYTES, (uint32_t)R::BYTES,
+                               bar);
+                ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, tm_v, bar, col_base, h,
+                                 (int)(t0 + (long long)ci * C));
+                n_issued = ci + 1;
+            };
+            for (int ci = 0; ci < NBUF && ci < nck; ++ci) issue(ci);
+            constexpr uint32_t idx = ptx::idesc_bf16_f32(128, DVT, false, true);
+            for (int ci = 0; ci < nck && ok; ++ci) {
+                const int b = ci % NBUF;
+                const uint32_t rb = sb + b * R::BYTES;
+                const uint32_t xy = XCOL_XY + (uint32_t)(ci & 1) * TC::XY_STRIDE;
+                ok = ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((ci / NBUF) & 1), WAIT_LIMIT_CYCLES) &&
+                     ptx::mbar_wait_bounded(bar_s, (uint32_t)(ci & 1), WAIT_LIMIT_CYCLES);
+                if (!ok) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)
+                    ptx::mma_bf16(tmem + xy, kdesc(rb + R::KQ, s, 128), MN::desc(sb + L::SP, s, DK), idx, s > 0);
+                ptx::mma_commit(bar_x);
+                // chunk ci-1's buffer: released by the compute warps, its products done
+                if (ci >= 1 && ci - 1 + NBUF < nck) {
+                    const int cp = ci - 1;
+                    ok = ptx::mbar_wait_bounded(bar_free + 8 * (cp % NBUF), (uint32_t)((cp / NBUF) & 1),
+                                                WAIT_LIMIT_CYCLES) &&
+                         ptx::mbar_wait_bounded(bar_o + 8 * (cp & 1), (uint32_t)((cp >> 1) & 1), WAIT_LIMIT_CYCLES);
+                    if (!ok) break;
+                    issue(cp + NBUF);
+                }
+                ok = ptx::mbar_wait_bounded(bar_z, (uint32_t)(ci & 1), WAIT_LIMIT_CYCLES);
+                if (!ok) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    ptx::mma_bf16(tmem + TC::DS, kdesc(rb + R::KP, s, DK + 64), MN::desc(sb + L::ZT, s, C), idx,
+                                  s > 0);
+                ptx::mma_commit(bar_ds);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    ptx::mma_bf16(tmem + xy, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C), idx,
+                                  1);
+                ptx::mma_commit(bar_o + 8 * (ci & 1));
+                n_mma = ci + 1;
+            }
+            if (!ok) {
+                flag_status(KDA_DEV_WAIT_TIMEOUT);
+                // let the products and copies in flight land (bounded) before the CTA leaves
+                if (n_mma > 0) {
+                    const int cl = n_mma - 1;
+                    ptx::mbar_wait_bounded(bar_o + 8 * (cl & 1), (uint32_t)((cl >> 1) & 1), WAIT_LIMIT_CYCLES);
+                }
+                for (int c = max(0, n_issued - NBUF); c < n_issued; ++c)
+                    ptx::mbar_wait_bounded(bar_rec + 8 * (c % NBUF), (uint32_t)((c / NBUF) & 1), WAIT_LIMIT_CYCLES);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- compute warps: thread <-> key row srow, value columns scol..scol+CPT-1
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const int srow = quad * 32 + lane;
+        const bool has_row = srow < DK;
+        const int scol = half * CPT;
+        const int row = state_row(slots, num_slots, n);
+        const long long st_off = ((long long)(row < 0 ? 0 : row) * H + h) * DK * DV + col_base + scol;
+        float S[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; j += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (has_row && init_state && row >= 0) x = load4(init_state + st_off + (long long)srow * DV + j);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+        auto put_state = [&]() {   // S -> bf16 B operand of the next [X; Y] product, then bar_s
+            if (has_row) {
+#pragma unroll
+                for (int g = 0; g < CPT / 8; ++g)
+                    *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) =
+                        make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
+                                   pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
+                ptx::fence_proxy_async_smem();
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_s);
+        };
+        // quads 2-3 (TMEM lanes 64-127): O rows of chunk c -> o
+        auto store_o = [&](int c) -> bool {
+            if (!ptx::mbar_wait_bounded(bar_o + 8 * (c & 1), (uint32_t)((c >> 1) & 1), WAIT_LIMIT_CYCLES)) return false;
+            ptx::tc_fence_after();
+            const long long cs = t0 + (long long)c * C;
+            const int Lc = (int)min((long long)C, t1 - cs);
+            const int i = (quad - 2) * 32 + lane;
+#pragma unroll 1
+            for (int cc = 0; cc < CPT / 16; ++cc) {
+                float o16[16];
+                ptx::tmem_ld16(tl + XCOL_XY + (uint32_t)(c & 1) * TC::XY_STRIDE + scol + cc * 16, o16);
+                ptx::tmem_wait_ld();
+                if (i < Lc) {
+                    __nv_bfloat16 *dst = o + ((cs + i) * H + h) * DV + col_base + scol + cc * 16;
+                    reinterpret_cast<uint4 *>(dst)[0] =
+                        make_uint4(pack_bf16(o16[0], o16[1]), pack_bf16(o16[2], o16[3]), pack_bf16(o16[4], o16[5]),
+                                   pack_bf16(o16[6], o16[7]));
+                    reinterpret_cast<uint4 *>(dst)[1] =
+                        make_uint4(pack_bf16(o16[8], o16[9]), pack_bf16(o16[10], o16[11]),
+                                   pack_bf16(o16[12], o16[13]), pack_bf16(o16[14], o16[15]));
+                }
+            }
+            return true;
+        };
+        if (nck > 0) put_state();
+        for (int ci = 0; ci < nck; ++ci) {
+            const long long cs = t0 + (long long)ci * C;
+            const int Lc = (int)min((long long)C, t1 - cs);
+            const int b = ci % NBUF;
+            const uint32_t xy = XCOL_XY + (uint32_t)(ci & 1) * TC::XY_STRIDE;
+            if (!(ok = ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((ci / NBUF) & 1), WAIT_LIMIT_CYCLES))) break;
+            const float dch = has_row ? reinterpret_cast<const float *>(sm + b * R::BYTES + R::DCH)[srow] : 0.f;
+            if (quad < 2) {
+                // ---- Z = V - X (X in TMEM lanes 0-63) -> Z^T, bf16
+                if (!(ok = ptx::mbar_wait_bounded(bar_x, (uint32_t)(ci & 1), WAIT_LIMIT_CYCLES))) break;
+                ptx::tc_fence_after();
+                const int j = quad * 32 + lane;
+                const uint8_t *vin = sm + L::VIN + b * C * DVT * 2;
+#pragma unroll 1
+                for (int cc = 0; cc < CPT / 16; ++cc) {
+                    float x16[16], v16[16];
+                    ptx::tmem_ld16(tl + xy + scol + cc * 16, x16);
+                    if (j < Lc) {
+                        unpack_bf16x8(*reinterpret_cast<const uint4 *>(vin + (j * DVT + scol + cc * 16) * 2), v16);
+                        unpack_bf16x8(*reinterpret_cast<const uint4 *>(vin + (j * DVT + scol + cc * 16 + 8) * 2),
+                                      v16 + 8);
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) v16[u] = 0.f;
+                    }
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int g = 0; g < 2; ++g)
+                        *reinterpret_cast<uint4 *>(sm + L::ZT + MN::off(j, scol + cc * 16 + 8 * g, C)) = make_uint4(
+                            pack_bf16(v16[8 * g] - x16[8 * g], v16[8 * g + 1] - x16[8 * g + 1]),
+                            pack_bf16(v16[8 * g + 2] - x16[8 * g + 2], v16[8 * g + 3] - x16[8 * g + 3]),
+                            pack_bf16(v16[8 * g + 4] - x16[8 * g + 4], v16[8 * g + 5] - x16[8 * g + 5]),
+                            pack_bf16(v16[8 * g + 6] - x16[8 * g + 6], v16[8 * g + 7] - x16[8 * g + 7]));
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(bar_z);
+                    ptx::mbar_arrive(bar_free + 8 * b);   // V and e^{G_last} of buffer b read
+                }
+            } else {
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar_free + 8 * b);   // e^{G_last} read
+                if (ci > 0 && !(ok = store_o(ci - 1))) break;
+            }
+            // ---- S <- Diag(e^{G_last}) S + Kt Z
+            if (!(ok = ptx::mbar_wait_bounded(bar_ds, (uint32_t)(ci & 1), WAIT_LIMIT_CYCLES))) break;
+            ptx::tc_fence_after();
+            if (has_row) {
+#pragma unroll
+                for (int cc = 0; cc < CPT / 16; ++cc) {
+                    float d16[16];
+                    ptx::tmem_ld16(tl + TC::DS + scol + cc * 16, d16);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
+                }
+            }
+            if (ci + 1 < nck) put_state();
+        }
+        if (ok && nck > 0 && quad >= 2) ok = store_o(nck - 1);   // O of the last chunk
+        if (!ok) flag_status(KDA_DEV_WAIT_TIMEOUT);
+        if (ok && final_state && has_row && row >= 0) {
+#pragma unroll
+            for (int j = 0; j < CPT; j += 4)
+                store4(final_state + st_off + (long long)srow * DV + j,
+                       make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, TC::ALLOC);
+    }
+}
+
+template <int DK, int DVT, int NBUF>
+__global__ void __launch_bounds__(NT_WS, 1)
 chunk_inter_kernel(const __grid_constant__ CUtensorMap tm_v, const uint8_t *__restrict__ ws,
                    const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
                    float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV,
-                   const int32_t *__restrict__ slots, int num_slots, uint8_t *__restrict__ ckpt) {
-    inter_body<DK, DVT, NBUF, CK>((int)blockIdx.x, &tm_v, ws, init_state, o, final_state, cu_seqlens, T, H, DV, slots,
-                                  num_slots, ckpt);
+                   const int32_t *__restrict__ slots, int num_slots) {
+    inter_ws_body<DK, DVT, NBUF>((int)blockIdx.x, &tm_v, ws, init_state, o, final_state, cu_seqlens, T, H, DV, slots,
+                                 num_slots);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1002,8 +1297,8 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         snprintf(msg, msg_len, "chunk_intra launch: %s", cudaGetErrorString(e));
         return KDA_ERR_CUDA;
     }
-    constexpr int NBUF = inter_nbuf<DK, DVT>();
-    constexpr int smem2 = InterLayout<DK, DVT, NBUF>::ALLOC;
+    constexpr int NBUF = inter_ws_nbuf<DK, DVT>();
+    constexpr int smem2 = InterWsLayout<DK, DVT, NBUF>::ALLOC;
     static_assert(smem2 <= 232448, "shared memory budget");
     auto k2 = chunk_inter_kernel<DK, DVT, NBUF>;
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
@@ -1011,9 +1306,9 @@ int launch_two_pass_t(const void *q, const void *k, const void *v, const float *
         snprintf(msg, msg_len, "cudaFuncSetAttribute(chunk_inter): %s", cudaGetErrorString(e));
         return KDA_ERR_CUDA;
     }
-    k2<<<dim3(dv / DVT, H, num_seqs), NT, smem2, st>>>(tv, (const uint8_t *)workspace, init_state,
-                                                        (__nv_bfloat16 *)o, final_state, cu_seqlens, T, H, dv,
-                                                        slots, num_slots, nullptr);
+    k2<<<dim3(dv / DVT, H, num_seqs), NT_WS, smem2, st>>>(tv, (const uint8_t *)workspace, init_state,
+                                                           (__nv_bfloat16 *)o, final_state, cu_seqlens, T, H, dv,
+                                                           slots, num_slots);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(msg, msg_len, "chunk_inter launch: %s", cudaGetErrorString(e));

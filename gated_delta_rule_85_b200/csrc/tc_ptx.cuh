@@ -52,6 +52,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity
     }
 }
 
+// One arrival (release at CTA scope: this thread's prior writes are visible to the waiter).
+__device__ __forceinline__ void mbar_arrive(uint32_t addr) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
 }
