@@ -60,7 +60,7 @@ PROLOGUE_BYTES_PER_TOKEN_HEAD = 3 * 2 * 128 + 2 * 128 + 4 + 2 * 128             
 # dram__bytes_write.sum) of the current kernels on these workloads; keyed by the kernels
 # one step runs.  A kernel set without a capture on its workload reports null.
 NCU_TRAFFIC = {
-    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 272.1e6 + 184.8e6 + 308.4e6 + 50.7e6,
+    ("prefill_8k", "chunk_intra_kernel + chunk_inter_kernel"): 272.3e6 + 185.0e6 + 308.4e6 + 50.4e6,
     # chunk_tc_kernel (--algo fused): captured before its timeout-path change, so reported null
     ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.2e6,
     # backward: the three kernels of one call (read + write of each)
