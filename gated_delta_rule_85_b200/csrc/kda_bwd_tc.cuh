@@ -17,10 +17,11 @@
 // then the chain rule through the decay factors and a reverse running sum for
 // dlog_alpha.  Three launches:
 //   1. chunk_intra_kernel<BX>: the forward's first pass, plus Akk, Aqk and T;
-//   2. bwd_sweeps_kernel: the two serial sweeps side by side -- the forward's state
-//      sweep storing each chunk's starting state (bf16) instead of the output
-//      (inter_body<CK>), and the adjoint sweep, chunks in reverse, storing each
-//      chunk's ending adjoint (bf16) and dS_0 (adj_body);
+//   2. bwd_sweeps_kernel: the two serial sweeps side by side, each warp-specialised
+//      like the forward's second pass -- the forward's state sweep storing each
+//      chunk's starting state (bf16) instead of the output (inter_ws_body<CK>), and
+//      the adjoint sweep, chunks in reverse, storing each chunk's ending adjoint
+//      (bf16) and dS_0 (adj_ws_body);
 //   3. bwd_grad_kernel (per chunk, head): every product above that needs S or
 //      dS', in a transposed form whose 128 rows are value or key channels
 //      (W^T, U^T, dU^T, lam^T: M = dv; the sums over the value columns: M = dk),
@@ -50,19 +51,45 @@ struct AdjLayout {
     static_assert(REC % 1024 == 0 && SP % 1024 == 0 && MU % 1024 == 0 && DOT % 1024 == 0, "tile alignment");
 };
 
-constexpr uint32_t ACOL_MU = 0;     // [128 x DVT] mu (lanes 0-63; lanes 64-127 unused)
-constexpr uint32_t ACOL_DS = 128;   // [128 x DVT] Qhat^T dO - Khat^T mu
-
-// One CTA per (value tile, head, sequence), chunks from the last to the first.
-// Per chunk: mu = Pt^T dO + Kt^T dS' (M = 128 over a 64-row operand: the A
-// descriptor's second 64-row half reads neighbouring bytes, whose rows are
-// ignored), then dS = Diag(D) dS' + [Khat^T Qhat^T] [-mu; dO] (M = dk).
-// dS' of each chunk (its end) goes to the unit's DSC tile; dS_0 to dinit_state.
+// Adjoint sweep: one CTA per (value tile, head, sequence), chunks from the last to
+// the first, warp-specialised like the forward's second pass (8 compute warps + 1
+// issue warp).  Per step t (chunk c = nck-1-t, buffer b = t % NBUF):
+//
+//   issue              wait record b -> the state-independent products first:
+//                      MU = Pt^T dO (M = 128 over a 64-row operand: the A
+//                      descriptor's second 64-row half reads neighbouring bytes,
+//                      whose rows are ignored) and DS[t & 1] = Qhat^T dO; then wait
+//                      dS' in bf16 (bar_s) -> MU += Kt^T dS', commit bar_mu
+//   compute (quads 0-1) wait bar_mu -> -mu in bf16 -> bar_z
+//   issue              wait bar_z -> DS[t & 1] += Khat^T (-mu) (M = dk), commit bar_ds;
+//                      meanwhile, once step t-1's buffer is released and its
+//                      products are done (bar_mu of step t), load step t-1+NBUF into it
+//   compute (all)      wait bar_ds -> dS <- Diag(D) dS' + DS -> dS' of the next step in
+//                      bf16 (and the unit's DSC checkpoint) -> bar_s
+//
+// so only Kt^T dS' (8 MMAs), the -mu conversion, Khat^T (-mu) (4 MMAs) and the update
+// are on the serial path.  dS_0 goes to dinit_state.  Bounded waits as in the forward.
 template <int DK, int DVT, int NBUF>
-__device__ __forceinline__ void adj_body(int tile, const CUtensorMap *tm_do, uint8_t *__restrict__ ws,
-                                         const float *__restrict__ dfinal, float *__restrict__ dinit_state,
-                                         const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
-    using L = AdjLayout<DK, DVT, NBUF>;
+struct AdjWsLayout {
+    using B = AdjLayout<DK, DVT, NBUF>;
+    static constexpr int SP = B::SP, MU = B::MU, DOT = B::DOT, MISC = B::MISC;
+    // MISC: bar_rec[NBUF], bar_free[NBUF], bar_s, bar_mu, bar_z, bar_ds, TMEM base
+    static constexpr int BAR_REC = MISC, BAR_FREE = MISC + 32, BAR_S = MISC + 64, BAR_MU = MISC + 72,
+                         BAR_Z = MISC + 80, BAR_DS = MISC + 88, TSLOT = MISC + 112;
+    static constexpr int BYTES = MISC + 128;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(NBUF <= 4, "barrier slots");
+};
+
+constexpr uint32_t ACOL_MU = 0;     // [128 x DVT] mu (lanes 0-63; lanes 64-127 unused)
+constexpr uint32_t ACOL_DS = 64;    // [128 x DVT] x 2 by step parity: Qhat^T dO - Khat^T mu
+static_assert(ACOL_DS + 2 * 64 <= INTER_TMEM_COLS, "TMEM columns");
+
+template <int DK, int DVT, int NBUF>
+__device__ __forceinline__ void adj_ws_body(int tile, const CUtensorMap *tm_do, uint8_t *__restrict__ ws,
+                                            const float *__restrict__ dfinal, float *__restrict__ dinit_state,
+                                            const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
+    using L = AdjWsLayout<DK, DVT, NBUF>;
     using R = Rec<DK>;
     using U = BwdUnit<DK>;
     static_assert(DK == 128 && (DVT == 32 || DVT == 64), "tile shape");
@@ -73,11 +100,12 @@ __device__ __forceinline__ void adj_body(int tile, const CUtensorMap *tm_do, uin
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = ptx::smem_u32(sm);
-    const uint32_t bar_rec = sb + L::MISC, bar_mma = sb + L::MISC + 32;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 40);
+    const uint32_t bar_rec = sb + L::BAR_REC, bar_free = sb + L::BAR_FREE, bar_s = sb + L::BAR_S,
+                   bar_mu = sb + L::BAR_MU, bar_z = sb + L::BAR_Z, bar_ds = sb + L::BAR_DS;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::TSLOT);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, half = (warp >> 2) & 1;
     const int col_base = tile * DVT, h = blockIdx.y;
     const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
     long long t0, t1;
@@ -89,9 +117,15 @@ __device__ __forceinline__ void adj_body(int tile, const CUtensorMap *tm_do, uin
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTER_TMEM_COLS);
         ptx::tmem_relinquish();
     }
-    if (tid == 0) {
-        for (int b = 0; b < NBUF; ++b) ptx::mbar_init(bar_rec + 8 * b, 1);
-        ptx::mbar_init(bar_mma, 1);
+    if (tid == NT) {
+        for (int b = 0; b < NBUF; ++b) {
+            ptx::mbar_init(bar_rec + 8 * b, 1);
+            ptx::mbar_init(bar_free + 8 * b, NT / 32);
+        }
+        ptx::mbar_init(bar_s, NT / 32);
+        ptx::mbar_init(bar_mu, 1);
+        ptx::mbar_init(bar_z, 4);
+        ptx::mbar_init(bar_ds, 1);
         ptx::fence_mbar_init();
         if (nck > 0) ptx::prefetch_tmap(tm_do);
     }
@@ -99,136 +133,147 @@ __device__ __forceinline__ void adj_body(int tile, const CUtensorMap *tm_do, uin
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t ph_mma = 0, ph_rec = 0;
-    int n_issued = 0, n_commit = 0;
-
-    auto issue = [&](int t) {   // thread 0: record and dO tile of step t (chunk nck - 1 - t) into buffer t % NBUF
-        const int b = t % NBUF, ci = nck - 1 - t;
-        n_issued = t + 1;
-        const uint32_t bar = bar_rec + 8 * b;
-        ptx::mbar_arrive_expect_tx(bar, TX);
-        ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * U::BYTES, (uint32_t)R::BYTES, bar);
-        ptx::tma_load_3d(sb + L::DOT + b * C * DVT * 2, tm_do, bar, col_base, h, (int)(t0 + (long long)ci * C));
-    };
-
-    const int srow = quad * 32 + lane;
-    const int scol = half * CPT;
-    const long long st_off = ((long long)n * H + h) * DK * DV + col_base + scol;
-    float S[CPT];   // dS' (fp32), this thread's row and columns
-#pragma unroll
-    for (int j = 0; j < CPT; j += 4) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (dfinal) x = load4(dfinal + st_off + (long long)srow * DV + j);
-        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-    }
-    if (tid == 0)
-        for (int t = 0; t < NBUF && t < nck; ++t) issue(t);
-
     bool ok = true;
-    for (int t = 0; t < nck; ++t) {
-        const int ci = nck - 1 - t, b = t % NBUF;
-        const uint32_t rb = sb + b * R::BYTES, dob = sb + L::DOT + b * C * DVT * 2;
-        uint32_t ph = (ph_rec >> b) & 1u;
-        ok = wait_all(bar_rec + 8 * b, ph);
-        ph_rec ^= 1u << b;
-        if (!ok) break;
 
-        // ---- 1. dS' -> bf16 B operand and the unit's checkpoint
-        const float dch = reinterpret_cast<const float *>(sm + b * R::BYTES + R::DCH)[srow];
-        {
-            uint8_t *ck = ws + ((size_t)(first + ci) * H + h) * U::BYTES + U::DSC;
+    if (warp == NT / 32) {
+        // ---------------- issue warp (lane 0)
+        if (lane == 0) {
+            int n_issued = 0, n_done = 0;   // steps whose loads were issued; steps with all products issued
+            auto issue = [&](int t) {      // record and dO tile of step t (chunk nck-1-t) into buffer t % NBUF
+                const int b = t % NBUF, ci = nck - 1 - t;
+                const uint32_t bar = bar_rec + 8 * b;
+                ptx::mbar_arrive_expect_tx(bar, TX);
+                ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * U::BYTES, (uint32_t)R::BYTES,
+                               bar);
+                ptx::tma_load_3d(sb + L::DOT + b * C * DVT * 2, tm_do, bar, col_base, h,
+                                 (int)(t0 + (long long)ci * C));
+                n_issued = t + 1;
+            };
+            for (int t = 0; t < NBUF && t < nck; ++t) issue(t);
+            constexpr uint32_t im = ptx::idesc_bf16_f32(128, DVT, true, true);
+            for (int t = 0; t < nck && ok; ++t) {
+                const int b = t % NBUF;
+                const uint32_t rb = sb + b * R::BYTES, dob = sb + L::DOT + b * C * DVT * 2, kp = rb + R::KP;
+                const uint32_t ds = ACOL_DS + (uint32_t)(t & 1) * 64;
+                if (!(ok = ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((t / NBUF) & 1), WAIT_LIMIT_CYCLES)))
+                    break;
+                ptx::tc_fence_after();
+                // state-independent: MU = Pt^T dO, DS = Qhat^T dO (MU was read before the last bar_z;
+                // DS[t & 1] before the bar_s of step t-1)
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    ptx::mma_bf16(tmem + ACOL_MU, ptx::desc_mnmajor_sw128(kp + (DK + 16 * s) * 128, 2048, 1024),
+                                  MN::desc(dob, s, C), im, s > 0);
+#pragma unroll
+                for (int s = 4; s < 8; ++s)
+                    ptx::mma_bf16(tmem + ds, M64::desc(rb + R::KQ, s, 128), MN::desc(dob, s - 4, C), im, s > 4);
+                if (!(ok = ptx::mbar_wait_bounded(bar_s, (uint32_t)(t & 1), WAIT_LIMIT_CYCLES))) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)
+                    ptx::mma_bf16(tmem + ACOL_MU, ptx::desc_mnmajor_sw128(kp + s * 2048, 2048, 1024),
+                                  MN::desc(sb + L::SP, s, DK), im, 1);
+                ptx::mma_commit(bar_mu);
+                // step t-1's buffer: released by the compute warps, its products done (bar_mu of step t)
+                if (t >= 1 && t - 1 + NBUF < nck) {
+                    ok = ptx::mbar_wait_bounded(bar_free + 8 * ((t - 1) % NBUF), (uint32_t)(((t - 1) / NBUF) & 1),
+                                                WAIT_LIMIT_CYCLES) &&
+                         ptx::mbar_wait_bounded(bar_mu, (uint32_t)(t & 1), WAIT_LIMIT_CYCLES);
+                    if (!ok) break;
+                    issue(t - 1 + NBUF);
+                }
+                if (!(ok = ptx::mbar_wait_bounded(bar_z, (uint32_t)(t & 1), WAIT_LIMIT_CYCLES))) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    ptx::mma_bf16(tmem + ds, M64::desc(rb + R::KQ, s, 128), MN::desc(sb + L::MU, s, C), im, 1);
+                ptx::mma_commit(bar_ds);
+                n_done = t + 1;
+            }
+            if (!ok) {
+                flag_status(KDA_DEV_WAIT_TIMEOUT);
+                // let the products and copies in flight land (bounded) before the CTA leaves
+                if (n_done > 0) ptx::mbar_wait_bounded(bar_ds, (uint32_t)((n_done - 1) & 1), WAIT_LIMIT_CYCLES);
+                for (int t = max(0, n_issued - NBUF); t < n_issued; ++t)
+                    ptx::mbar_wait_bounded(bar_rec + 8 * (t % NBUF), (uint32_t)((t / NBUF) & 1), WAIT_LIMIT_CYCLES);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- compute warps: thread <-> key row srow, value columns scol..scol+CPT-1
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const int srow = quad * 32 + lane;
+        const int scol = half * CPT;
+        const long long st_off = ((long long)n * H + h) * DK * DV + col_base + scol;
+        float S[CPT];   // dS' (fp32), this thread's row and columns
+#pragma unroll
+        for (int j = 0; j < CPT; j += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (dfinal) x = load4(dfinal + st_off + (long long)srow * DV + j);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+        // dS' of step t (the end of chunk nck-1-t) -> bf16 B operand and the unit's checkpoint, then bar_s
+        auto put_adj = [&](int t) {
+            uint8_t *ck = ws + ((size_t)(first + nck - 1 - t) * H + h) * U::BYTES + U::DSC;
 #pragma unroll
             for (int g = 0; g < CPT / 8; ++g) {
-                const uint4 w =
-                    make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
-                               pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
+                const uint4 w = make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
+                                           pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
                 *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) = w;
                 *reinterpret_cast<uint4 *>(ck + sw128(srow, col_base + scol + 8 * g, DK)) = w;
             }
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncthreads();
-
-        // ---- 2. mu = Pt^T dO + Kt^T dS'  (A: MN-major views of the record's [Kt; Pt] rows)
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            constexpr uint32_t im = ptx::idesc_bf16_f32(128, DVT, true, true);
-            const uint32_t kp = rb + R::KP;
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + ACOL_MU, ptx::desc_mnmajor_sw128(kp + (DK + 16 * s) * 128, 2048, 1024),
-                              MN::desc(dob, s, C), im, s > 0);
-#pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                ptx::mma_bf16(tmem + ACOL_MU, ptx::desc_mnmajor_sw128(kp + s * 2048, 2048, 1024),
-                              MN::desc(sb + L::SP, s, DK), im, 1);
-            ptx::mma_commit(bar_mma);
-            ++n_commit;
-        }
-        if (!(ok = wait_all(bar_mma, ph_mma))) break;
-
-        // ---- 3. -mu (TMEM lanes 0-63) -> bf16 B operand rows
-        if (quad < 2) {
-            const int j = quad * 32 + lane;
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_s);
+        };
+        if (nck > 0) put_adj(0);
+        for (int t = 0; t < nck; ++t) {
+            const int b = t % NBUF;
+            if (!(ok = ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((t / NBUF) & 1), WAIT_LIMIT_CYCLES))) break;
+            const float dch = reinterpret_cast<const float *>(sm + b * R::BYTES + R::DCH)[srow];
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_free + 8 * b);   // e^{G_last} read; the rest only feeds MMAs
+            if (quad < 2) {
+                // ---- -mu (TMEM lanes 0-63) -> bf16 B operand rows
+                if (!(ok = ptx::mbar_wait_bounded(bar_mu, (uint32_t)(t & 1), WAIT_LIMIT_CYCLES))) break;
+                ptx::tc_fence_after();
+                const int j = quad * 32 + lane;
 #pragma unroll 1
+                for (int cc = 0; cc < CPT / 16; ++cc) {
+                    float x16[16];
+                    ptx::tmem_ld16(tl + ACOL_MU + scol + cc * 16, x16);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int g = 0; g < 2; ++g)
+                        *reinterpret_cast<uint4 *>(sm + L::MU + MN::off(j, scol + cc * 16 + 8 * g, C)) = make_uint4(
+                            pack_bf16(-x16[8 * g], -x16[8 * g + 1]), pack_bf16(-x16[8 * g + 2], -x16[8 * g + 3]),
+                            pack_bf16(-x16[8 * g + 4], -x16[8 * g + 5]), pack_bf16(-x16[8 * g + 6], -x16[8 * g + 7]));
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar_z);
+            }
+            // ---- dS <- Diag(D) dS' + Qhat^T dO - Khat^T mu
+            if (!(ok = ptx::mbar_wait_bounded(bar_ds, (uint32_t)(t & 1), WAIT_LIMIT_CYCLES))) break;
+            ptx::tc_fence_after();
+#pragma unroll
             for (int cc = 0; cc < CPT / 16; ++cc) {
-                float x16[16];
-                ptx::tmem_ld16(tl + ACOL_MU + scol + cc * 16, x16);
+                float d16[16];
+                ptx::tmem_ld16(tl + ACOL_DS + (uint32_t)(t & 1) * 64 + scol + cc * 16, d16);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int g = 0; g < 2; ++g)
-                    *reinterpret_cast<uint4 *>(sm + L::MU + MN::off(j, scol + cc * 16 + 8 * g, C)) =
-                        make_uint4(pack_bf16(-x16[8 * g], -x16[8 * g + 1]), pack_bf16(-x16[8 * g + 2], -x16[8 * g + 3]),
-                                   pack_bf16(-x16[8 * g + 4], -x16[8 * g + 5]),
-                                   pack_bf16(-x16[8 * g + 6], -x16[8 * g + 7]));
+                for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
             }
+            if (t + 1 < nck) put_adj(t + 1);
         }
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncthreads();
-
-        // ---- 4. Khat^T (-mu) + Qhat^T dO  (A: MN-major view of the record's [Khat; Qhat] rows)
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            constexpr uint32_t id = ptx::idesc_bf16_f32(128, DVT, true, true);
+        if (!ok) flag_status(KDA_DEV_WAIT_TIMEOUT);
+        if (ok && dinit_state) {
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + ACOL_DS, M64::desc(rb + R::KQ, s, 128), MN::desc(sb + L::MU, s, C), id, s > 0);
-#pragma unroll
-            for (int s = 4; s < 8; ++s)
-                ptx::mma_bf16(tmem + ACOL_DS, M64::desc(rb + R::KQ, s, 128), MN::desc(dob, s - 4, C), id, 1);
-            ptx::mma_commit(bar_mma);
-            ++n_commit;
+            for (int j = 0; j < CPT; j += 4)
+                store4(dinit_state + st_off + (long long)srow * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
         }
-        if (!(ok = wait_all(bar_mma, ph_mma))) break;
-        if (tid == 0 && t + NBUF < nck) issue(t + NBUF);   // buffer b fully consumed
-
-        // ---- 5. dS <- Diag(D) dS' + (4)
-#pragma unroll
-        for (int cc = 0; cc < CPT / 16; ++cc) {
-            float d16[16];
-            ptx::tmem_ld16(tl + ACOL_DS + scol + cc * 16, d16);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
-        }
-        ptx::tc_fence_before();
-    }
-
-    if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded), then leave
-        for (int b = 0; b < NBUF; ++b) {
-            const int arms = n_issued > b ? (n_issued - 1 - b) / NBUF + 1 : 0;
-            if (arms > 0) ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((arms - 1) & 1), WAIT_LIMIT_CYCLES);
-        }
-        if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
-    }
-    __syncthreads();
-    if (ok && dinit_state) {
-#pragma unroll
-        for (int j = 0; j < CPT; j += 4)
-            store4(dinit_state + st_off + (long long)srow * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -240,24 +285,25 @@ __device__ __forceinline__ void adj_body(int tile, const CUtensorMap *tm_do, uin
 
 // Both state sweeps in one launch (they are independent): CTAs with
 // blockIdx.x < DV / DVT run the forward sweep (chunk-start states), the others the
-// adjoint sweep, one per (value tile, head, sequence) each.
+// adjoint sweep, one per (value tile, head, sequence) each; 8 compute warps and
+// one issue warp in either role.
 template <int DK, int DVT, int NBUF>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT_WS, 1)
 bwd_sweeps_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   uint8_t *__restrict__ ws, const float *__restrict__ init_state, const float *__restrict__ dfinal,
                   float *__restrict__ dinit_state, const int32_t *__restrict__ cu_seqlens, int T, int H, int DV) {
     const int nt = DV / DVT;
     if ((int)blockIdx.x < nt)
-        inter_body<DK, DVT, NBUF, true>((int)blockIdx.x, &tm_v, ws, init_state, nullptr, nullptr, cu_seqlens, T, H,
-                                        DV, nullptr, 0, ws);
+        inter_ws_body<DK, DVT, NBUF, true>((int)blockIdx.x, &tm_v, ws, init_state, nullptr, nullptr, cu_seqlens, T,
+                                           H, DV, nullptr, 0, ws);
     else
-        adj_body<DK, DVT, NBUF>((int)blockIdx.x - nt, &tm_do, ws, dfinal, dinit_state, cu_seqlens, T, H, DV);
+        adj_ws_body<DK, DVT, NBUF>((int)blockIdx.x - nt, &tm_do, ws, dfinal, dinit_state, cu_seqlens, T, H, DV);
 }
 
 template <int DK, int DVT, int NBUF>
 constexpr int sweeps_smem() {
-    return InterLayout<DK, DVT, NBUF>::ALLOC > AdjLayout<DK, DVT, NBUF>::ALLOC ? InterLayout<DK, DVT, NBUF>::ALLOC
-                                                                               : AdjLayout<DK, DVT, NBUF>::ALLOC;
+    return InterWsLayout<DK, DVT, NBUF>::ALLOC > AdjWsLayout<DK, DVT, NBUF>::ALLOC ? InterWsLayout<DK, DVT, NBUF>::ALLOC
+                                                                                   : AdjWsLayout<DK, DVT, NBUF>::ALLOC;
 }
 
 // ------------------------------------------------------------------ per-chunk sums
@@ -939,7 +985,7 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
                               void *dv_out, float *dlog_alpha, float *dbeta, float *dinit_state,
                               const int32_t *cu_seqlens, long long tokens, int T, int H, int num_seqs,
                               void *workspace, cudaStream_t st, char *msg, size_t msg_len) {
-    constexpr int DK = 128, DV = 128, DVT = 64, NBUF = 2;   // one wave of sweeps at 32 heads
+    constexpr int DK = 128, DV = 128, DVT = 64, NBUF = 3;   // one wave of sweeps at 32 heads
     const long long slots = tokens > 0 ? chunk_slots(tokens, num_seqs) : 0;
     if (slots > 0x7fffffffLL) {
         snprintf(msg, msg_len, "%lld chunk slots exceed the grid limit", slots);
@@ -981,8 +1027,8 @@ inline int launch_backward_tc(const void *q, const void *k, const void *v, const
         if ((rc = launch_ok("chunk_intra", msg, msg_len))) return rc;
     }
     // both sweeps; with no tokens only the adjoint half has work (dinit_state = dfinal)
-    k2<<<dim3(2 * (DV / DVT), H, num_seqs), NT, s2, st>>>(t_v64, t_do64, ws, init_state, dfinal, dinit_state,
-                                                          cu_seqlens, T, H, DV);
+    k2<<<dim3(2 * (DV / DVT), H, num_seqs), NT_WS, s2, st>>>(t_v64, t_do64, ws, init_state, dfinal, dinit_state,
+                                                             cu_seqlens, T, H, DV);
     if ((rc = launch_ok("bwd_sweeps", msg, msg_len))) return rc;
     if (slots > 0) {
         int dev = 0, sms = 148;

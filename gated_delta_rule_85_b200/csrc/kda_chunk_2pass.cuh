@@ -721,234 +721,8 @@ struct InterLayout {
 
 constexpr uint32_t INTER_TMEM_COLS = 256;
 constexpr uint32_t XCOL_XY = 0;       // [128 x DVT] rows 0-63 X, rows 64-127 Y, then O
-constexpr uint32_t XCOL_DS = 128;     // [128 x DVT] Kt Z (lanes 0..dk-1)
 
-// CK (the backward's state sweep, dv = 128): ws (and ckpt, the same bytes, writable)
-// hold [slot][H] BwdUnit; no output; instead the state at each chunk's start, bf16,
-// into the unit's SC tile (a K-major operand S with K = value columns, MN-major for S^T).
-template <int DK, int DVT, int NBUF, bool CK = false>
-__device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, const uint8_t *__restrict__ ws,
-                                           const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
-                                           float *__restrict__ final_state, const int32_t *__restrict__ cu_seqlens,
-                                           int T, int H, int DV, const int32_t *__restrict__ slots, int num_slots,
-                                           uint8_t *__restrict__ ckpt) {
-    using L = InterLayout<DK, DVT, NBUF>;
-    using R = Rec<DK>;
-    static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
-    constexpr int CPT = DVT / 2;
-    // CK loads only what the state update reads: the Khat rows of [Khat; Qhat], the Kt rows of
-    // [Kt; Pt] and e^{G_last} (the Qhat rows then hold stale bytes, whose products are never read)
-    constexpr uint32_t REC_TX = CK ? (uint32_t)(DK / 64 * 64 * 128 + DK * 128 + DK * 4) : (uint32_t)R::BYTES;
-    constexpr uint32_t TX = REC_TX + (uint32_t)(C * DVT * 2);
-    constexpr size_t USTRIDE = CK ? (size_t)BwdUnit<DK>::BYTES : (size_t)R::BYTES;   // bytes per (slot, head)
-    using MN = MnOp<DVT>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const uint32_t sb = ptx::smem_u32(sm);
-    const uint32_t bar_rec = sb + L::MISC, bar_mma = sb + L::MISC + 32;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC + 40);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
-    const int col_base = tile * DVT, h = blockIdx.y;
-    const int n = seq_for_cta(cu_seqlens, T, (int)gridDim.z);
-
-    long long t0, t1;
-    seq_span(cu_seqlens, T, n, t0, t1);
-    const int nck = (int)((t1 - t0 + C - 1) / C);
-    const long long first = n + t0 / C;   // slot of chunk 0
-
-    if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), INTER_TMEM_COLS);
-        ptx::tmem_relinquish();
-    }
-    if (tid == 0) {
-        for (int b = 0; b < NBUF; ++b) ptx::mbar_init(bar_rec + 8 * b, 1);
-        ptx::mbar_init(bar_mma, 1);
-        ptx::fence_mbar_init();
-        if (nck > 0) ptx::prefetch_tmap(tm_v);
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t ph_mma = 0, ph_rec = 0;   // ph_rec: one parity bit per buffer
-    int n_issued = 0, n_commit = 0;    // thread 0: chunks whose copies were issued, MMA commits
-
-    auto issue = [&](int ci) {   // thread 0: record and V tile of chunk ci into buffer ci % NBUF
-        const int b = ci % NBUF;
-        n_issued = ci + 1;
-        const uint32_t bar = bar_rec + 8 * b;
-        ptx::mbar_arrive_expect_tx(bar, TX);
-        const uint8_t *src = ws + ((size_t)(first + ci) * H + h) * USTRIDE;
-        if constexpr (CK) {
-#pragma unroll
-            for (int a = 0; a < DK / 64; ++a)
-                ptx::bulk_load(sb + b * R::BYTES + R::KQ + a * 16384, src + R::KQ + a * 16384, 64 * 128, bar);
-            ptx::bulk_load(sb + b * R::BYTES + R::KP, src + R::KP, DK * 128, bar);
-            ptx::bulk_load(sb + b * R::BYTES + R::DCH, src + R::DCH, DK * 4, bar);
-        } else {
-            ptx::bulk_load(sb + b * R::BYTES, src, (uint32_t)R::BYTES, bar);
-        }
-        ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, tm_v, bar, col_base, h, (int)(t0 + (long long)ci * C));
-    };
-
-    const int srow = quad * 32 + lane;
-    const bool has_row = srow < DK;
-    const int scol = half * CPT;
-    const int row = state_row(slots, num_slots, n);
-    const long long st_off = ((long long)(row < 0 ? 0 : row) * H + h) * DK * DV + col_base + scol;
-    float S[CPT];
-#pragma unroll
-    for (int j = 0; j < CPT; j += 4) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (has_row && init_state && row >= 0) x = load4(init_state + st_off + (long long)srow * DV + j);
-        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-    }
-    if (tid == 0)
-        for (int ci = 0; ci < NBUF && ci < nck; ++ci) issue(ci);
-
-    bool ok = true;
-    for (int ci = 0; ci < nck; ++ci) {
-        const long long cs = t0 + (long long)ci * C;
-        const int Lc = (int)min((long long)C, t1 - cs);
-        const int b = ci % NBUF;
-        const uint32_t rb = sb + b * R::BYTES;
-        uint32_t ph = (ph_rec >> b) & 1u;
-        ok = wait_all(bar_rec + 8 * b, ph);
-        ph_rec ^= 1u << b;
-        if (!ok) break;
-
-        // ---- 1. S^T -> bf16 B operand
-        const float dch = has_row ? reinterpret_cast<const float *>(sm + b * R::BYTES + R::DCH)[srow] : 0.f;
-        if (has_row) {
-            uint8_t *ck = CK ? ckpt + ((size_t)(first + ci) * H + h) * USTRIDE + BwdUnit<DK>::SC : nullptr;
-#pragma unroll
-            for (int g = 0; g < CPT / 8; ++g) {
-                const uint4 w = make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
-                                           pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
-                *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) = w;
-                if constexpr (CK) *reinterpret_cast<uint4 *>(ck + sw128(srow, col_base + scol + 8 * g, DK)) = w;
-            }
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncthreads();
-
-        // ---- 2. [X; Y] = [e^G K; e^G Q] S
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            constexpr uint32_t ix = ptx::idesc_bf16_f32(128, DVT, false, true);
-#pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KQ, s, 128), MN::desc(sb + L::SP, s, DK), ix, s > 0);
-            ptx::mma_commit(bar_mma);
-            ++n_commit;
-        }
-        if (!(ok = wait_all(bar_mma, ph_mma))) break;
-
-        // ---- 3. Z = V - X (X in TMEM lanes 0-63) -> Z^T
-        if (quad < 2) {
-            const int j = quad * 32 + lane;
-            const uint8_t *vin = sm + L::VIN + b * C * DVT * 2;
-#pragma unroll 1
-            for (int cc = 0; cc < CPT / 16; ++cc) {
-                float x16[16], v16[16];
-                ptx::tmem_ld16(tl + XCOL_XY + scol + cc * 16, x16);
-                if (j < Lc) {
-                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(vin + (j * DVT + scol + cc * 16) * 2), v16);
-                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(vin + (j * DVT + scol + cc * 16 + 8) * 2), v16 + 8);
-                } else {
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) v16[u] = 0.f;
-                }
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int g = 0; g < 2; ++g)
-                    *reinterpret_cast<uint4 *>(sm + L::ZT + MN::off(j, scol + cc * 16 + 8 * g, C)) = make_uint4(
-                        pack_bf16(v16[8 * g] - x16[8 * g], v16[8 * g + 1] - x16[8 * g + 1]),
-                        pack_bf16(v16[8 * g + 2] - x16[8 * g + 2], v16[8 * g + 3] - x16[8 * g + 3]),
-                        pack_bf16(v16[8 * g + 4] - x16[8 * g + 4], v16[8 * g + 5] - x16[8 * g + 5]),
-                        pack_bf16(v16[8 * g + 6] - x16[8 * g + 6], v16[8 * g + 7] - x16[8 * g + 7]));
-            }
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncthreads();
-
-        // ---- 4. dS = Kt Z ; O = Y + Pt Z (onto the Y rows of [X; Y])
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            constexpr uint32_t iz = ptx::idesc_bf16_f32(128, DVT, false, true);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                ptx::mma_bf16(tmem + XCOL_DS, kdesc(rb + R::KP, s, DK + 64), MN::desc(sb + L::ZT, s, C), iz, s > 0);
-            if constexpr (!CK) {
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    ptx::mma_bf16(tmem + XCOL_XY, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C),
-                                  iz, 1);
-            }
-            ptx::mma_commit(bar_mma);
-            ++n_commit;
-        }
-        if (!(ok = wait_all(bar_mma, ph_mma))) break;
-        if (tid == 0 && ci + NBUF < nck) issue(ci + NBUF);   // buffer b fully consumed
-
-        // ---- 5. S <- Diag(e^{G_last}) S + dS ; O rows (TMEM lanes 64-127) -> o
-        if (has_row) {
-#pragma unroll
-            for (int cc = 0; cc < CPT / 16; ++cc) {
-                float d16[16];
-                ptx::tmem_ld16(tl + XCOL_DS + scol + cc * 16, d16);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
-            }
-        }
-        if (!CK && quad >= 2) {
-            const int i = (quad - 2) * 32 + lane;
-#pragma unroll 1
-            for (int cc = 0; cc < CPT / 16; ++cc) {
-                float o16[16];
-                ptx::tmem_ld16(tl + XCOL_XY + scol + cc * 16, o16);
-                ptx::tmem_wait_ld();
-                if (i < Lc) {
-                    __nv_bfloat16 *dst = o + ((cs + i) * H + h) * DV + col_base + scol + cc * 16;
-                    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pack_bf16(o16[0], o16[1]), pack_bf16(o16[2], o16[3]),
-                                                                   pack_bf16(o16[4], o16[5]), pack_bf16(o16[6], o16[7]));
-                    reinterpret_cast<uint4 *>(dst)[1] =
-                        make_uint4(pack_bf16(o16[8], o16[9]), pack_bf16(o16[10], o16[11]),
-                                   pack_bf16(o16[12], o16[13]), pack_bf16(o16[14], o16[15]));
-                }
-            }
-        }
-        ptx::tc_fence_before();
-    }
-
-    if (!ok && tid == 0) {   // a wait timed out: let the copies and MMAs in flight land (bounded), then leave
-        for (int b = 0; b < NBUF; ++b) {
-            const int arms = n_issued > b ? (n_issued - 1 - b) / NBUF + 1 : 0;   // loads into buffer b
-            if (arms > 0) ptx::mbar_wait_bounded(bar_rec + 8 * b, (uint32_t)((arms - 1) & 1), WAIT_LIMIT_CYCLES);
-        }
-        if (n_commit > 0) ptx::mbar_wait_bounded(bar_mma, (uint32_t)((n_commit - 1) & 1), WAIT_LIMIT_CYCLES);
-    }
-    __syncthreads();
-    if (ok && final_state && has_row && row >= 0) {
-#pragma unroll
-        for (int j = 0; j < CPT; j += 4)
-            store4(final_state + st_off + (long long)srow * DV + j, make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, INTER_TMEM_COLS);
-    }
-}
-
-// ---- pass 2 with output: warp-specialised
+// ---- pass 2: warp-specialised
 //
 // Eight compute warps and one issue warp.  Lane 0 of the issue warp loads the
 // records and V tiles and issues every tcgen05.mma (each issue holds its thread
@@ -970,6 +744,12 @@ __device__ __forceinline__ void inter_body(int tile, const CUtensorMap *tm_v, co
 // elementwise steps between them; the output product, the readout of O and the
 // record loads overlap it.  Every wait is bounded: a thread whose wait runs out
 // flags the device status and leaves its loop; the others then run out in turn.
+//
+// CK (the backward's forward state sweep, dv = 128): ws (and ckpt, the same bytes,
+// writable) hold [slot][H] BwdUnit; only the Khat rows, the Kt rows and e^{G_last}
+// of each record are loaded (the Qhat rows hold stale bytes whose products are
+// never read); no output; instead the state at each chunk's start, bf16, goes to
+// the unit's SC tile (a K-major operand S with K = value columns, MN-major for S^T).
 
 constexpr int NT_WS = NT + 32;   // 8 compute warps + the issue warp
 
@@ -1001,19 +781,22 @@ struct InterWsCols {
     static_assert(DS + DVT <= ALLOC, "TMEM columns");
 };
 
-template <int DK, int DVT, int NBUF>
+template <int DK, int DVT, int NBUF, bool CK = false>
 __device__ __forceinline__ void inter_ws_body(int tile, const CUtensorMap *tm_v, const uint8_t *__restrict__ ws,
                                               const float *__restrict__ init_state, __nv_bfloat16 *__restrict__ o,
                                               float *__restrict__ final_state,
                                               const int32_t *__restrict__ cu_seqlens, int T, int H, int DV,
-                                              const int32_t *__restrict__ slots, int num_slots) {
+                                              const int32_t *__restrict__ slots, int num_slots,
+                                              uint8_t *__restrict__ ckpt = nullptr) {
     using L = InterWsLayout<DK, DVT, NBUF>;
     using R = Rec<DK>;
     using TC = InterWsCols<DVT>;
     using MN = MnOp<DVT>;
     static_assert(DVT % 32 == 0 && DVT >= 32 && DVT <= 128, "value tile");
     constexpr int CPT = DVT / 2;
-    constexpr uint32_t TX = (uint32_t)R::BYTES + (uint32_t)(C * DVT * 2);
+    constexpr uint32_t REC_TX = CK ? (uint32_t)(DK / 64 * 64 * 128 + DK * 128 + DK * 4) : (uint32_t)R::BYTES;
+    constexpr uint32_t TX = REC_TX + (uint32_t)(C * DVT * 2);
+    constexpr size_t USTRIDE = CK ? (size_t)BwdUnit<DK>::BYTES : (size_t)R::BYTES;   // bytes per (slot, head)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = ptx::smem_u32(sm);
@@ -1063,8 +846,16 @@ __device__ __forceinline__ void inter_ws_body(int tile, const CUtensorMap *tm_v,
                 const int b = ci % NBUF;
                 const uint32_t bar = bar_rec + 8 * b;
                 ptx::mbar_arrive_expect_tx(bar, TX);
-                ptx::bulk_load(sb + b * R::BYTES, ws + ((size_t)(first + ci) * H + h) * R::BYTES, (uint32_t)R::BYTES,
-                               bar);
+                const uint8_t *src = ws + ((size_t)(first + ci) * H + h) * USTRIDE;
+                if constexpr (CK) {
+#pragma unroll
+                    for (int a = 0; a < DK / 64; ++a)
+                        ptx::bulk_load(sb + b * R::BYTES + R::KQ + a * 16384, src + R::KQ + a * 16384, 64 * 128, bar);
+                    ptx::bulk_load(sb + b * R::BYTES + R::KP, src + R::KP, DK * 128, bar);
+                    ptx::bulk_load(sb + b * R::BYTES + R::DCH, src + R::DCH, DK * 4, bar);
+                } else {
+                    ptx::bulk_load(sb + b * R::BYTES, src, (uint32_t)R::BYTES, bar);
+                }
                 ptx::tma_load_3d(sb + L::VIN + b * C * DVT * 2, tm_v, bar, col_base, h,
                                  (int)(t0 + (long long)ci * C));
                 n_issued = ci + 1;
@@ -1100,11 +891,13 @@ __device__ __forceinline__ void inter_ws_body(int tile, const CUtensorMap *tm_v,
                     ptx::mma_bf16(tmem + TC::DS, kdesc(rb + R::KP, s, DK + 64), MN::desc(sb + L::ZT, s, C), idx,
                                   s > 0);
                 ptx::mma_commit(bar_ds);
+                if constexpr (!CK) {
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    ptx::mma_bf16(tmem + xy, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C), idx,
-                                  1);
-                ptx::mma_commit(bar_o + 8 * (ci & 1));
+                    for (int s = 0; s < 4; ++s)
+                        ptx::mma_bf16(tmem + xy, kdesc(rb + R::KP, s, DK + 64, DK - 64), MN::desc(sb + L::ZT, s, C),
+                                      idx, 1);
+                }
+                ptx::mma_commit(bar_o + 8 * (ci & 1));   // CK: marks chunk ci's products done, for the reload
                 n_mma = ci + 1;
             }
             if (!ok) {
@@ -1134,13 +927,19 @@ __device__ __forceinline__ void inter_ws_body(int tile, const CUtensorMap *tm_v,
             if (has_row && init_state && row >= 0) x = load4(init_state + st_off + (long long)srow * DV + j);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
-        auto put_state = [&]() {   // S -> bf16 B operand of the next [X; Y] product, then bar_s
+        // S (the state at chunk c's start) -> bf16 B operand of chunk c's [X; Y] product
+        // (CK: and the unit's checkpoint), then bar_s
+        auto put_state = [&](int c) {
             if (has_row) {
+                uint8_t *ck = CK ? ckpt + ((size_t)(first + c) * H + h) * USTRIDE + BwdUnit<DK>::SC : nullptr;
 #pragma unroll
-                for (int g = 0; g < CPT / 8; ++g)
-                    *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) =
+                for (int g = 0; g < CPT / 8; ++g) {
+                    const uint4 w =
                         make_uint4(pack_bf16(S[8 * g], S[8 * g + 1]), pack_bf16(S[8 * g + 2], S[8 * g + 3]),
                                    pack_bf16(S[8 * g + 4], S[8 * g + 5]), pack_bf16(S[8 * g + 6], S[8 * g + 7]));
+                    *reinterpret_cast<uint4 *>(sm + L::SP + MN::off(srow, scol + 8 * g, DK)) = w;
+                    if constexpr (CK) *reinterpret_cast<uint4 *>(ck + sw128(srow, col_base + scol + 8 * g, DK)) = w;
+                }
                 ptx::fence_proxy_async_smem();
             }
             ptx::tc_fence_before();
@@ -1171,7 +970,7 @@ __device__ __forceinline__ void inter_ws_body(int tile, const CUtensorMap *tm_v,
             }
             return true;
         };
-        if (nck > 0) put_state();
+        if (nck > 0) put_state(0);
         for (int ci = 0; ci < nck; ++ci) {
             const long long cs = t0 + (long long)ci * C;
             const int Lc = (int)min((long long)C, t1 - cs);
@@ -1216,7 +1015,7 @@ __device__ __forceinline__ void inter_ws_body(int tile, const CUtensorMap *tm_v,
             } else {
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar_free + 8 * b);   // e^{G_last} read
-                if (ci > 0 && !(ok = store_o(ci - 1))) break;
+                if (!CK && ci > 0 && !(ok = store_o(ci - 1))) break;
             }
             // ---- S <- Diag(e^{G_last}) S + Kt Z
             if (!(ok = ptx::mbar_wait_bounded(bar_ds, (uint32_t)(ci & 1), WAIT_LIMIT_CYCLES))) break;
@@ -1231,9 +1030,9 @@ __device__ __forceinline__ void inter_ws_body(int tile, const CUtensorMap *tm_v,
                     for (int u = 0; u < 16; ++u) S[cc * 16 + u] = fmaf(dch, S[cc * 16 + u], d16[u]);
                 }
             }
-            if (ci + 1 < nck) put_state();
+            if (ci + 1 < nck) put_state(ci + 1);
         }
-        if (ok && nck > 0 && quad >= 2) ok = store_o(nck - 1);   // O of the last chunk
+        if (!CK && ok && nck > 0 && quad >= 2) ok = store_o(nck - 1);   // O of the last chunk
         if (!ok) flag_status(KDA_DEV_WAIT_TIMEOUT);
         if (ok && final_state && has_row && row >= 0) {
 #pragma unroll
