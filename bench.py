@@ -64,7 +64,7 @@ NCU_TRAFFIC = {
     # chunk_tc_kernel (--algo fused): captured before its timeout-path change, so reported null
     ("decode_b256", "decode_step_kernel"): 547.4e6 + 481.2e6,
     # backward: the three kernels of one call (read + write of each)
-    ("backward_T8192", "bwd"): 274.1e6 + 285.5e6 + 492.0e6 + 233.2e6 + 911.2e6 + 311.1e6,
+    ("backward_T8192", "bwd"): 274.2e6 + 287.8e6 + 492.7e6 + 232.3e6 + 912.7e6 + 311.0e6,
 }
 
 
